@@ -1,0 +1,208 @@
+"""Seeded synthetic inputs for the selective state update (decode, prefill, replay).
+
+This module only draws random numbers and lays them out in the shapes the
+Selective State Update page (TensorRT-Edge-LLM C++ API, ``invokeSelectiveStateUpdate``,
+``invokeSelectiveStateUpdatePrefill`` and ``MambaReplayLayerInfo``) gives for each
+argument. It holds no part of the recurrence: both the CUDA path and the CPU oracle
+receive the same tensors from here and do all of the arithmetic themselves.
+
+Value laws (one set for every workload):
+  x, z, B, C, pool state ~ N(0, 1); dt ~ N(0, 1); dt_bias ~ N(0, 0.1);
+  A = -exp(U(0, 2)); D ~ N(0, 1).
+  The "slow decay" variant draws A = -exp(U(-2, 0)) and sets dt_bias = -4, so that the
+  state remembers many tokens.
+Every tensor is drawn in fp32 from one ``torch.Generator`` in a fixed order
+(pool, x, B, C, dt, z, A, dt_bias, D, stateIndices, padding positions, lengths) and then
+cast to its storage dtype, so both sides see the same (already rounded) values.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional, Sequence
+
+import torch
+
+F32, F16, BF16 = torch.float32, torch.float16, torch.bfloat16
+
+
+@dataclasses.dataclass
+class SSUCase:
+    """One seeded workload: shapes, flags and CPU tensors.
+
+    Shapes (batch-major, contiguous):
+      decode:  x, z [batch, H, Dm]; B, C [batch, G, N]; dt [batch, H]
+      prefill / replay inputs: x, z [batch, T, H, Dm]; B, C [batch, T, G, N]; dt [batch, T, H]
+      pool [P, H, Dm, N] (slot stride H*Dm*N elements unless ``slot_stride`` says more)
+      A, dt_bias, D [H] fp32; state_indices [batch] int32 (None = row b uses slot b)
+      context_lengths / accepted_lengths [batch] int32 (None = all T tokens)
+    """
+
+    name: str
+    batch: int
+    P: int
+    H: int
+    G: int
+    Dm: int
+    N: int
+    T: Optional[int]          # None for the single-token decode form
+    active: int
+    slot_stride: int
+    x: torch.Tensor
+    B: torch.Tensor
+    C: torch.Tensor
+    dt: torch.Tensor
+    A: torch.Tensor
+    pool: torch.Tensor        # flat storage of P * slot_stride elements
+    z: Optional[torch.Tensor] = None
+    dt_bias: Optional[torch.Tensor] = None
+    D: Optional[torch.Tensor] = None
+    state_indices: Optional[torch.Tensor] = None
+    context_lengths: Optional[torch.Tensor] = None
+    accepted_lengths: Optional[torch.Tensor] = None
+    dt_softplus: bool = True
+
+    @property
+    def x_dtype(self):
+        return self.x.dtype
+
+    @property
+    def bc_dtype(self):
+        return self.B.dtype
+
+    @property
+    def state_dtype(self):
+        return self.pool.dtype
+
+    def to(self, device) -> "SSUCase":
+        """Copy of the case with every tensor moved to ``device``."""
+        fields = {}
+        for f in dataclasses.fields(self):
+            v = getattr(self, f.name)
+            fields[f.name] = v.to(device) if isinstance(v, torch.Tensor) else v
+        return SSUCase(**fields)
+
+
+def make_case(
+    name: str = "case",
+    *,
+    seed: int,
+    batch: int,
+    P: Optional[int] = None,
+    H: int,
+    G: int,
+    Dm: int,
+    N: int,
+    T: Optional[int] = None,
+    active: Optional[int] = None,
+    x_dtype=F32,
+    bc_dtype=F32,
+    state_dtype=F32,
+    z: bool = False,
+    dt_bias: bool = True,
+    D: bool = True,
+    dt_softplus: bool = True,
+    indices: str | Sequence[int] = "perm",
+    n_pad: int = 0,
+    lengths: Optional[str] = None,
+    slot_pad: int = 0,
+    slow_decay: bool = False,
+) -> SSUCase:
+    """Draw one workload.
+
+    indices: "perm" (distinct slots from a random permutation of [0, P)), "none"
+      (no stateIndices: row b is slot b) or an explicit list.
+    n_pad: how many of the first ``active`` rows get stateIndices = -1 (random rows).
+    lengths: None, "context" (contextLengths ~ U{1..T}) or "accepted"
+      (acceptedLengths ~ U{0..T}).
+    slot_pad: extra elements per pool slot beyond H*Dm*N (a padded slot stride).
+    """
+    if P is None:
+        P = batch
+    if active is None:
+        active = batch
+    g = torch.Generator().manual_seed(seed)
+    slot = H * Dm * N
+    stride = slot + slot_pad
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, dtype=F32)
+
+    pool = randn(P * stride).to(state_dtype)
+    lead = (batch,) if T is None else (batch, T)
+    x = randn(*lead, H, Dm).to(x_dtype)
+    B = randn(*lead, G, N).to(bc_dtype)
+    C = randn(*lead, G, N).to(bc_dtype)
+    dt = randn(*lead, H)
+    zt = randn(*lead, H, Dm).to(x_dtype) if z else None
+    if slow_decay:
+        A = -torch.exp(torch.rand(H, generator=g, dtype=F32) * 2.0 - 2.0)
+    else:
+        A = -torch.exp(torch.rand(H, generator=g, dtype=F32) * 2.0)
+    if slow_decay:
+        bias = torch.full((H,), -4.0, dtype=F32)
+    else:
+        bias = randn(H) * 0.1 if dt_bias else None
+    Dv = randn(H) if D else None
+
+    if isinstance(indices, str):
+        if indices == "perm":
+            si = torch.randperm(P, generator=g)[:batch].to(torch.int32)
+        elif indices == "none":
+            si = None
+        else:
+            raise ValueError(f"unknown indices mode {indices!r}")
+    else:
+        si = torch.tensor(list(indices), dtype=torch.int32)
+    if n_pad:
+        if si is None:
+            raise ValueError("padding rows need stateIndices")
+        rows = torch.randperm(active, generator=g)[:n_pad]
+        si = si.clone()
+        si[rows] = -1
+
+    ctx = acc = None
+    if lengths == "context":
+        ctx = torch.randint(1, T + 1, (batch,), generator=g, dtype=torch.int32)
+    elif lengths == "accepted":
+        acc = torch.randint(0, T + 1, (batch,), generator=g, dtype=torch.int32)
+    elif lengths is not None:
+        raise ValueError(f"unknown lengths mode {lengths!r}")
+
+    return SSUCase(
+        name=name, batch=batch, P=P, H=H, G=G, Dm=Dm, N=N, T=T, active=active,
+        slot_stride=stride, x=x, B=B, C=C, dt=dt, A=A, pool=pool, z=zt,
+        dt_bias=bias, D=Dv, state_indices=si, context_lengths=ctx,
+        accepted_lengths=acc, dt_softplus=dt_softplus,
+    )
+
+
+# The five named workloads. Seeds: 0 for the tiny decode, then 1..4 in order.
+CONFIGS = {
+    # batch 2, pool of 4 slots, H 4, Dm 16, N 16, fp32 everything, stateIndices [2, 0]
+    "tiny_decode": dict(seed=0, batch=2, P=4, H=4, G=1, Dm=16, N=16,
+                        x_dtype=F32, bc_dtype=F32, state_dtype=F32, z=False,
+                        indices=[2, 0]),
+    # Mamba2-2.7B-like decode: batch 256 over a 512-slot pool, H 80, Dm 64, N 128
+    "mamba2_decode_b256": dict(seed=1, batch=256, P=512, H=80, G=1, Dm=64, N=128,
+                               x_dtype=BF16, bc_dtype=BF16, state_dtype=F32, z=True),
+    # CUDA-graph decode captured at batch 128 with 96 live rows, 24 of them padding
+    "padded_graph_decode": dict(seed=2, batch=128, active=96, n_pad=24, P=256, H=64,
+                                G=8, Dm=64, N=128, x_dtype=F16, bc_dtype=F16,
+                                state_dtype=F16, z=True),
+    # multi-token prefill, contextLengths ~ U{1..512}, pool of 32 slots
+    "prefill_b16_t512": dict(seed=3, batch=16, P=32, T=512, H=80, G=1, Dm=64, N=128,
+                             x_dtype=BF16, bc_dtype=BF16, state_dtype=F32, z=True,
+                             lengths="context"),
+    # speculative replay of up to 5 drafted tokens, acceptedLengths ~ U{0..5}
+    "spec_replay_b64_t5": dict(seed=4, batch=64, P=128, T=5, H=80, G=1, Dm=64, N=128,
+                               x_dtype=BF16, bc_dtype=BF16, state_dtype=F32, z=True,
+                               lengths="accepted"),
+}
+
+
+def make_config(name: str, **overrides) -> SSUCase:
+    """Draw one of the named workloads (``CONFIGS``), optionally with overrides."""
+    kw = dict(CONFIGS[name])
+    kw.update(overrides)
+    return make_case(name, **kw)

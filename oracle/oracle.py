@@ -1,0 +1,185 @@
+"""Python access to the float64 CPU oracle (``ssu_oracle.c``).
+
+TEST INFRASTRUCTURE. Only the test suite, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg import this module. It never touches the CUDA library.
+
+The functions take CPU torch tensors (used here only as typed host buffers) and return
+float64 outputs. The pool is updated in place in its own storage type, exactly as the
+Selective State Update page (TensorRT-Edge-LLM C++ API) describes for
+``invokeSelectiveStateUpdate``, ``invokeSelectiveStateUpdatePrefill`` and the replay.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "ssu_oracle.c")
+LIB = os.path.join(HERE, "libssu_oracle.so")
+
+_CODES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2, torch.float64: 3}
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc into ``oracle/libssu_oracle.so``."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = LIB + ".tmp"
+        subprocess.run(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-Wall", "-Wextra",
+             "-fno-fast-math", "-ffp-contract=off", "-o", tmp, SRC, "-lm"],
+            check=True,
+        )
+        os.replace(tmp, LIB)
+    return LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(LIB)
+        vp, i32, i64, i = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int
+        L.oracle_decode.argtypes = [vp, i, vp, vp, vp, i, vp, vp, vp, vp, vp, i, i64, i32,
+                                    vp, vp, i32, i32, i32, i32, i32, i32, i, vp]
+        L.oracle_prefill.argtypes = [vp, i, vp, vp, vp, i, vp, vp, vp, vp, vp, i, i64, i32,
+                                     vp, vp, vp, vp, vp, vp, vp,
+                                     i32, i32, i32, i32, i32, i32, i32, i, vp]
+        L.oracle_replay.argtypes = [vp, i, i64, i32, vp, vp, vp, vp, vp, vp,
+                                    i32, i32, i32, i32, i32, i32, i32, vp]
+        L.oracle_clear_slot.argtypes = [vp, i64, i32, i32]
+        L.oracle_copy_slot.argtypes = [vp, i32, i32, vp, i32, i32, i64]
+        L.oracle_f16_to_double.argtypes = [ctypes.c_uint16]
+        L.oracle_f16_to_double.restype = ctypes.c_double
+        L.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        L.oracle_bf16_to_double.restype = ctypes.c_double
+        L.oracle_double_to_f16.argtypes = [ctypes.c_double]
+        L.oracle_double_to_f16.restype = ctypes.c_uint16
+        L.oracle_double_to_bf16.argtypes = [ctypes.c_double]
+        L.oracle_double_to_bf16.restype = ctypes.c_uint16
+        for f in ("oracle_decode", "oracle_prefill", "oracle_replay",
+                  "oracle_clear_slot", "oracle_copy_slot"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    assert t.device.type == "cpu" and t.is_contiguous(), "oracle takes contiguous CPU tensors"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"{what}: oracle rejected the arguments (code {rc})")
+
+
+def decode(x, A, B, C, dt, pool, *, dt_bias=None, D=None, z=None, state_indices=None,
+           batch, active=None, H, G, Dm, N, slot_stride=None, P=None, dt_softplus=True,
+           out=None):
+    """One decode token; ``pool`` (flat, storage dtype) is updated in place.
+
+    Returns (out float64 [batch,H,Dm], err_flags). Rows not visited keep ``out``'s
+    initial contents (NaN unless ``out`` is given).
+    """
+    active = batch if active is None else active
+    slot_stride = H * Dm * N if slot_stride is None else slot_stride
+    P = pool.numel() // slot_stride if P is None else P
+    if out is None:
+        out = torch.full((batch, H, Dm), float("nan"), dtype=torch.float64)
+    err = ctypes.c_int32(0)
+    rc = lib().oracle_decode(
+        _p(x), _CODES[x.dtype], _p(A), _p(B), _p(C), _CODES[B.dtype], _p(dt), _p(dt_bias),
+        _p(D), _p(z), _p(pool), _CODES[pool.dtype], slot_stride, P, _p(out),
+        _p(state_indices), batch, active, H, G, Dm, N, int(dt_softplus),
+        ctypes.byref(err))
+    _check(rc, "oracle_decode")
+    return out, err.value
+
+
+def prefill(x, A, B, C, dt, pool, *, dt_bias=None, D=None, z=None, state_indices=None,
+            context_lengths=None, stash=None, batch, active=None, T, H, G, Dm, N,
+            slot_stride=None, P=None, dt_softplus=True, out=None):
+    """All T tokens in one call. ``stash`` is None or a tuple (DA, U, Bst, DT) of fp32
+    CPU tensors written in place. Returns (out float64 [batch,T,H,Dm], err_flags)."""
+    active = batch if active is None else active
+    slot_stride = H * Dm * N if slot_stride is None else slot_stride
+    P = pool.numel() // slot_stride if P is None else P
+    if out is None:
+        out = torch.full((batch, T, H, Dm), float("nan"), dtype=torch.float64)
+    DA, U, Bst, DT = stash if stash is not None else (None, None, None, None)
+    err = ctypes.c_int32(0)
+    rc = lib().oracle_prefill(
+        _p(x), _CODES[x.dtype], _p(A), _p(B), _p(C), _CODES[B.dtype], _p(dt), _p(dt_bias),
+        _p(D), _p(z), _p(pool), _CODES[pool.dtype], slot_stride, P, _p(out),
+        _p(state_indices), _p(context_lengths), _p(DA), _p(U), _p(Bst), _p(DT),
+        batch, active, T, H, G, Dm, N, int(dt_softplus), ctypes.byref(err))
+    _check(rc, "oracle_prefill")
+    return out, err.value
+
+
+def new_stash(batch, T, H, G, Dm, N, fill=float("nan")):
+    """Fresh fp32 stash buffers (DA, U, Bst, DT) filled with ``fill``."""
+    return (torch.full((batch, T, H), fill, dtype=torch.float32),
+            torch.full((batch, T, H, Dm), fill, dtype=torch.float32),
+            torch.full((batch, T, G, N), fill, dtype=torch.float32),
+            torch.full((batch, T, H), fill, dtype=torch.float32))
+
+
+def replay(pool, stash, accepted_lengths, *, state_indices=None, batch, active=None, T,
+           H, G, Dm, N, slot_stride=None, P=None):
+    """Re-apply the first acceptedLengths[b] stashed tokens in place. Returns err_flags."""
+    active = batch if active is None else active
+    slot_stride = H * Dm * N if slot_stride is None else slot_stride
+    P = pool.numel() // slot_stride if P is None else P
+    DA, U, Bst, DT = stash
+    err = ctypes.c_int32(0)
+    rc = lib().oracle_replay(
+        _p(pool), _CODES[pool.dtype], slot_stride, P, _p(DA), _p(U), _p(Bst), _p(DT),
+        _p(accepted_lengths), _p(state_indices), batch, active, T, H, G, Dm, N,
+        ctypes.byref(err))
+    _check(rc, "oracle_replay")
+    return err.value
+
+
+def clear_slot(pool, slot_bytes, P, slot):
+    _check(lib().oracle_clear_slot(_p(pool), slot_bytes, P, slot), "oracle_clear_slot")
+
+
+def copy_slot(dst_pool, dst_P, dst_slot, src_pool, src_P, src_slot, slot_bytes):
+    _check(lib().oracle_copy_slot(_p(dst_pool), dst_P, dst_slot, _p(src_pool), src_P,
+                                  src_slot, slot_bytes), "oracle_copy_slot")
+
+
+# --- convenience wrappers over a workloads.SSUCase (inputs only; no arithmetic) ---
+
+def decode_case(case, pool=None):
+    """Run the oracle decode on a case; returns (out, pool_after, err)."""
+    pool = case.pool.clone() if pool is None else pool
+    out, err = decode(case.x, case.A, case.B, case.C, case.dt, pool, dt_bias=case.dt_bias,
+                      D=case.D, z=case.z, state_indices=case.state_indices,
+                      batch=case.batch, active=case.active, H=case.H, G=case.G,
+                      Dm=case.Dm, N=case.N, slot_stride=case.slot_stride, P=case.P,
+                      dt_softplus=case.dt_softplus)
+    return out, pool, err
+
+
+def prefill_case(case, pool=None, stash=False):
+    """Run the oracle prefill on a case; returns (out, pool_after, stash or None, err)."""
+    pool = case.pool.clone() if pool is None else pool
+    st = new_stash(case.batch, case.T, case.H, case.G, case.Dm, case.N) if stash else None
+    out, err = prefill(case.x, case.A, case.B, case.C, case.dt, pool, dt_bias=case.dt_bias,
+                       D=case.D, z=case.z, state_indices=case.state_indices,
+                       context_lengths=case.context_lengths, stash=st, batch=case.batch,
+                       active=case.active, T=case.T, H=case.H, G=case.G, Dm=case.Dm,
+                       N=case.N, slot_stride=case.slot_stride, P=case.P,
+                       dt_softplus=case.dt_softplus)
+    return out, pool, st, err

@@ -1,0 +1,429 @@
+/*
+ * ssu_oracle.c -- plain, slow float64 CPU oracle for the Mamba selective state update.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg call this code; the product path never does. It shares no code,
+ * header or constant with the CUDA library.
+ *
+ * Source of the method: "Selective State Update" page of the TensorRT-Edge-LLM C++ API
+ * (mamba_ssm::invokeSelectiveStateUpdate, invokeSelectiveStateUpdatePrefill,
+ * struct MambaReplayLayerInfo, invokeMambaStateClear), the padding contract of the
+ * FlashInfer page "flashinfer.gdn_fused_decode_step" (parameter state_indices), and the
+ * "Recurrent State Manager" page (clearSlot, copySlotFrom).
+ *
+ * Per active row b and head h, one token does
+ *     dt_eff    = softplus(dt + dt_bias)  (or dt + dt_bias when softplus is off)
+ *     new_state = state * exp(A * dt_eff) + B * dt_eff * x
+ *     out       = sum_n new_state[n] * C[n] + D * x,   then out *= silu(z) if z is given
+ * Everything is computed in double. Inputs are decoded exactly from their storage type;
+ * the pool is read in its storage type and the final state is rounded once (to nearest,
+ * ties to even) when it is stored back. Outputs are returned unrounded, in double.
+ *
+ * Readings taken where the pages leave a point open:
+ *   - head h uses group g = h / (H / G) (contiguous blocks of heads per group);
+ *   - dt_bias is added whenever it is given, with or without softplus;
+ *   - the replay stash holds DA = exp(A * dt_eff) (the decay factor), DT = dt_eff,
+ *     U = x and B, all fp32, because the replay call receives no A, dt_bias or softplus;
+ *   - positions t >= contextLengths[b] are neither read nor written; a row whose length
+ *     is 0 is left untouched;
+ *   - a padding row (stateIndices[b] < 0) reads and writes no state; its outputs are 0
+ *     (all T positions in prefill); the replay writes nothing for it;
+ *   - an index >= P, a length > T or a negative length is undefined on the pages; here
+ *     the row is skipped (index) or the length clamped, and a bit is set in err_flags:
+ *     1 = index >= P, 2 = acceptedLengths > T, 4 = contextLengths > T, 8 = negative length.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* storage types understood by the oracle */
+enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2, OR_F64 = 3 };
+
+/* ---------------- exact decoding of the storage formats ---------------- */
+
+/* IEEE binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits. */
+double oracle_f16_to_double(uint16_t h)
+{
+    int sign = h >> 15, e = (h >> 10) & 31, m = h & 1023;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);              /* zero or subnormal */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(m + 1024), e - 25);  /* (1 + m/1024) * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/* bfloat16 is the upper half of an IEEE binary32. */
+double oracle_bf16_to_double(uint16_t h)
+{
+    uint32_t bits = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* ---------------- rounding to nearest, ties to even ---------------- */
+
+/* Round v to a binary format with p significand bits (implicit bit included),
+ * minimum normal exponent emin and maximum exponent emax. */
+static double round_to_format(double v, int p, int emin, int emax)
+{
+    if (isnan(v) || isinf(v) || v == 0.0)
+        return v;
+    double a = fabs(v);
+    int E;
+    frexp(a, &E);           /* a = f * 2^E, f in [0.5, 1) */
+    int e = E - 1;          /* a in [2^e, 2^(e+1)) */
+    if (e < emin)
+        e = emin;           /* subnormal range: fixed quantum */
+    double q = ldexp(1.0, e - (p - 1));
+    double r = nearbyint(a / q) * q;   /* default mode: to nearest, ties to even */
+    double maxfin = ldexp(2.0 - ldexp(1.0, -(p - 1)), emax);
+    if (r > maxfin)
+        r = INFINITY;
+    return copysign(r, v);
+}
+
+uint16_t oracle_double_to_f16(double v)
+{
+    if (isnan(v))
+        return 0x7e00;
+    double r = round_to_format(v, 11, -14, 15);
+    uint16_t sign = signbit(r) ? 0x8000 : 0;
+    double a = fabs(r);
+    if (isinf(a))
+        return sign | 0x7c00;
+    if (a < ldexp(1.0, -14))                 /* subnormal: a = m * 2^-24 exactly */
+        return sign | (uint16_t)(a / ldexp(1.0, -24));
+    int E;
+    double f = frexp(a, &E);                 /* a = (2f) * 2^(E-1), 2f in [1, 2) */
+    uint16_t frac = (uint16_t)((2.0 * f - 1.0) * 1024.0);
+    return sign | (uint16_t)((E - 1 + 15) << 10) | frac;
+}
+
+uint16_t oracle_double_to_bf16(double v)
+{
+    if (isnan(v))
+        return 0x7fc0;
+    /* every bfloat16 value is exactly a binary32, whose upper half is the encoding */
+    float f = (float)round_to_format(v, 8, -126, 127);
+    uint32_t bits;
+    memcpy(&bits, &f, sizeof bits);
+    return (uint16_t)(bits >> 16);
+}
+
+/* ---------------- typed element access ---------------- */
+
+static double load(const void *p, int dt, int64_t i)
+{
+    switch (dt) {
+    case OR_F32: return (double)((const float *)p)[i];
+    case OR_F16: return oracle_f16_to_double(((const uint16_t *)p)[i]);
+    case OR_BF16: return oracle_bf16_to_double(((const uint16_t *)p)[i]);
+    default: return ((const double *)p)[i];
+    }
+}
+
+static void store(void *p, int dt, int64_t i, double v)
+{
+    switch (dt) {
+    case OR_F32: ((float *)p)[i] = (float)v; break;   /* C conversion: to nearest even */
+    case OR_F16: ((uint16_t *)p)[i] = oracle_double_to_f16(v); break;
+    case OR_BF16: ((uint16_t *)p)[i] = oracle_double_to_bf16(v); break;
+    default: ((double *)p)[i] = v; break;
+    }
+}
+
+static int valid_dtype(int dt) { return dt >= OR_F32 && dt <= OR_F64; }
+
+/* ---------------- scalar helpers ---------------- */
+
+/* softplus(v) = log(1 + e^v), written so that neither branch overflows */
+static double softplus(double v)
+{
+    return v > 0.0 ? v + log1p(exp(-v)) : log1p(exp(v));
+}
+
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* dt after the optional bias and the optional softplus */
+static double effective_dt(double dt, const float *dt_bias, int h, int dt_softplus)
+{
+    double v = dt + (dt_bias ? (double)dt_bias[h] : 0.0);
+    return dt_softplus ? softplus(v) : v;
+}
+
+/* Resolve row b to a pool slot. Returns the slot, -1 for a padding row, or -2 when
+ * the index is out of range (flag bit 1 set). */
+static int64_t resolve_slot(const int32_t *state_indices, int32_t b, int32_t P,
+                            int32_t *err)
+{
+    int64_t s = state_indices ? state_indices[b] : b;
+    if (s < 0)
+        return -1;
+    if (s >= P) {
+        *err |= 1;
+        return -2;
+    }
+    return s;
+}
+
+static int check_common(int32_t batch, int32_t active, int32_t H, int32_t G,
+                        int32_t Dm, int32_t N, int64_t slot_stride)
+{
+    if (batch < 0 || active < 0 || active > batch)
+        return 2;
+    if (H <= 0 || G <= 0 || Dm <= 0 || N <= 0 || H % G != 0)
+        return 2;
+    if (slot_stride < (int64_t)H * Dm * N)
+        return 2;
+    return 0;
+}
+
+/* ---------------- decode (seq_len == 1) ----------------
+ * Selective State Update page, mamba_ssm::invokeSelectiveStateUpdate:
+ * x [batch,H,Dm], A [H], B/C [batch,G,N], dt [batch,H], dt_bias/D [H], z like x,
+ * state pool [P,H,Dm,N] updated in place through stateIndices, output [batch,H,Dm]. */
+int oracle_decode(const void *x, int x_dt, const float *A,
+                  const void *B, const void *C, int bc_dt,
+                  const float *dt, const float *dt_bias, const float *D, const void *z,
+                  void *pool, int state_dt, int64_t slot_stride, int32_t P,
+                  double *out, const int32_t *state_indices,
+                  int32_t batch, int32_t active, int32_t H, int32_t G, int32_t Dm,
+                  int32_t N, int dt_softplus, int32_t *err_flags)
+{
+    if (!x || !A || !B || !C || !dt || !pool || !out)
+        return 1;
+    if (!valid_dtype(x_dt) || !valid_dtype(bc_dt) || !valid_dtype(state_dt))
+        return 3;
+    if (check_common(batch, active, H, G, Dm, N, slot_stride))
+        return 2;
+    int32_t err = 0;
+    int heads_per_group = H / G;
+    double *snew = malloc(sizeof(double) * (size_t)N);
+    for (int32_t b = 0; b < active; ++b) {
+        int64_t s = resolve_slot(state_indices, b, P, &err);
+        if (s == -1) {                       /* padding row: output zero, no state */
+            for (int64_t i = 0; i < (int64_t)H * Dm; ++i)
+                out[(int64_t)b * H * Dm + i] = 0.0;
+            continue;
+        }
+        if (s < 0)
+            continue;
+        for (int h = 0; h < H; ++h) {
+            int g = h / heads_per_group;
+            double dte = effective_dt(dt[(int64_t)b * H + h], dt_bias, h, dt_softplus);
+            double decay = exp((double)A[h] * dte);
+            for (int d = 0; d < Dm; ++d) {
+                int64_t xi = ((int64_t)b * H + h) * Dm + d;
+                double xv = load(x, x_dt, xi);
+                double y = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    int64_t si = s * slot_stride + ((int64_t)h * Dm + d) * N + n;
+                    int64_t bi = ((int64_t)b * G + g) * N + n;
+                    snew[n] = load(pool, state_dt, si) * decay
+                              + load(B, bc_dt, bi) * dte * xv;
+                    y += snew[n] * load(C, bc_dt, bi);
+                }
+                for (int n = 0; n < N; ++n)
+                    store(pool, state_dt, s * slot_stride + ((int64_t)h * Dm + d) * N + n,
+                          snew[n]);
+                if (D)
+                    y += (double)D[h] * xv;
+                if (z)
+                    y *= silu(load(z, x_dt, xi));
+                out[xi] = y;
+            }
+        }
+    }
+    free(snew);
+    if (err_flags)
+        *err_flags |= err;
+    return 0;
+}
+
+/* ---------------- prefill (seq_len > 1) ----------------
+ * Selective State Update page, mamba_ssm::invokeSelectiveStateUpdatePrefill:
+ * x, z, out [batch,T,H,Dm]; B, C [batch,T,G,N]; dt [batch,T,H]; all T tokens in one
+ * call, with optional contextLengths. With the replay stash (DA, U, Bst, DT, all fp32:
+ * [batch,T,H], [batch,T,H,Dm], [batch,T,G,N], [batch,T,H]) the committed state is
+ * read only and the per-token replay inputs are written instead. Without the stash
+ * the state after L_b tokens is stored back once. The state stays in double across
+ * the tokens (no rounding between tokens). */
+int oracle_prefill(const void *x, int x_dt, const float *A,
+                   const void *B, const void *C, int bc_dt,
+                   const float *dt, const float *dt_bias, const float *D, const void *z,
+                   void *pool, int state_dt, int64_t slot_stride, int32_t P,
+                   double *out, const int32_t *state_indices,
+                   const int32_t *context_lengths,
+                   float *st_DA, float *st_U, float *st_B, float *st_DT,
+                   int32_t batch, int32_t active, int32_t T, int32_t H, int32_t G,
+                   int32_t Dm, int32_t N, int dt_softplus, int32_t *err_flags)
+{
+    if (!x || !A || !B || !C || !dt || !pool || !out)
+        return 1;
+    if (!valid_dtype(x_dt) || !valid_dtype(bc_dt) || !valid_dtype(state_dt))
+        return 3;
+    if (check_common(batch, active, H, G, Dm, N, slot_stride) || T < 0)
+        return 2;
+    int given = (st_DA != 0) + (st_U != 0) + (st_B != 0) + (st_DT != 0);
+    if (given != 0 && given != 4)
+        return 1;
+    int stash = given == 4;
+    int32_t err = 0;
+    int heads_per_group = H / G;
+    double *S = malloc(sizeof(double) * (size_t)Dm * N);
+    for (int32_t b = 0; b < active; ++b) {
+        int64_t s = resolve_slot(state_indices, b, P, &err);
+        if (s == -1) {                       /* padding row: every position outputs 0 */
+            for (int64_t i = 0; i < (int64_t)T * H * Dm; ++i)
+                out[(int64_t)b * T * H * Dm + i] = 0.0;
+            continue;
+        }
+        if (s < 0)
+            continue;
+        int32_t L = context_lengths ? context_lengths[b] : T;
+        if (L > T) {
+            err |= 4;
+            L = T;
+        }
+        if (L < 0) {
+            err |= 8;
+            L = 0;
+        }
+        if (L == 0)
+            continue;
+        for (int h = 0; h < H; ++h) {
+            int g = h / heads_per_group;
+            for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
+                S[i] = load(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i);
+            for (int32_t t = 0; t < L; ++t) {
+                int64_t bt = (int64_t)b * T + t;
+                double dte = effective_dt(dt[bt * H + h], dt_bias, h, dt_softplus);
+                double decay = exp((double)A[h] * dte);
+                if (stash) {
+                    st_DA[bt * H + h] = (float)decay;
+                    st_DT[bt * H + h] = (float)dte;
+                    for (int n = 0; n < N; ++n)
+                        st_B[(bt * G + g) * N + n] = (float)load(B, bc_dt, (bt * G + g) * N + n);
+                }
+                for (int d = 0; d < Dm; ++d) {
+                    int64_t xi = (bt * H + h) * Dm + d;
+                    double xv = load(x, x_dt, xi);
+                    if (stash)
+                        st_U[xi] = (float)xv;
+                    double y = 0.0;
+                    for (int n = 0; n < N; ++n) {
+                        int64_t bi = (bt * G + g) * N + n;
+                        double *sp = &S[(int64_t)d * N + n];
+                        *sp = *sp * decay + load(B, bc_dt, bi) * dte * xv;
+                        y += *sp * load(C, bc_dt, bi);
+                    }
+                    if (D)
+                        y += (double)D[h] * xv;
+                    if (z)
+                        y *= silu(load(z, x_dt, xi));
+                    out[xi] = y;
+                }
+            }
+            if (!stash)
+                for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
+                    store(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i, S[i]);
+        }
+    }
+    free(S);
+    if (err_flags)
+        *err_flags |= err;
+    return 0;
+}
+
+/* ---------------- replay of accepted tokens ----------------
+ * Selective State Update page, struct MambaReplayLayerInfo and
+ * invokeMambaReplayReconstructBatched: re-run the recurrence over the first
+ * acceptedLengths[b] stashed tokens, in place on the committed state; a count of 0
+ * leaves the row untouched; rows b >= activeBatchSize are not visited. */
+int oracle_replay(void *pool, int state_dt, int64_t slot_stride, int32_t P,
+                  const float *st_DA, const float *st_U, const float *st_B,
+                  const float *st_DT, const int32_t *accepted_lengths,
+                  const int32_t *state_indices, int32_t batch, int32_t active, int32_t T,
+                  int32_t H, int32_t G, int32_t Dm, int32_t N, int32_t *err_flags)
+{
+    if (!pool || !st_DA || !st_U || !st_B || !st_DT || !accepted_lengths)
+        return 1;
+    if (!valid_dtype(state_dt))
+        return 3;
+    if (check_common(batch, active, H, G, Dm, N, slot_stride) || T < 0)
+        return 2;
+    int32_t err = 0;
+    int heads_per_group = H / G;
+    double *S = malloc(sizeof(double) * (size_t)Dm * N);
+    for (int32_t b = 0; b < active; ++b) {
+        int64_t s = resolve_slot(state_indices, b, P, &err);
+        if (s < 0)
+            continue;                        /* padding row or bad index: no state */
+        int32_t k = accepted_lengths[b];
+        if (k > T) {
+            err |= 2;
+            k = T;
+        }
+        if (k < 0) {
+            err |= 8;
+            k = 0;
+        }
+        if (k == 0)
+            continue;
+        for (int h = 0; h < H; ++h) {
+            int g = h / heads_per_group;
+            for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
+                S[i] = load(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i);
+            for (int32_t t = 0; t < k; ++t) {
+                int64_t bt = (int64_t)b * T + t;
+                double decay = st_DA[bt * H + h];
+                double dte = st_DT[bt * H + h];
+                for (int d = 0; d < Dm; ++d) {
+                    double u = st_U[(bt * H + h) * Dm + d];
+                    for (int n = 0; n < N; ++n) {
+                        double *sp = &S[(int64_t)d * N + n];
+                        *sp = *sp * decay + (double)st_B[(bt * G + g) * N + n] * dte * u;
+                    }
+                }
+            }
+            for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
+                store(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i, S[i]);
+        }
+    }
+    free(S);
+    if (err_flags)
+        *err_flags |= err;
+    return 0;
+}
+
+/* ---------------- slot maintenance ----------------
+ * Selective State Update page, invokeMambaStateClear (one slot, or all when slot is -1)
+ * and Recurrent State Manager page, clearSlot / copySlotFrom. */
+int oracle_clear_slot(void *pool, int64_t slot_bytes, int32_t P, int32_t slot)
+{
+    if (!pool || slot_bytes < 0 || P < 0 || slot < -1 || slot >= P)
+        return 2;
+    if (slot == -1)
+        memset(pool, 0, (size_t)slot_bytes * (size_t)P);
+    else
+        memset((char *)pool + (int64_t)slot * slot_bytes, 0, (size_t)slot_bytes);
+    return 0;
+}
+
+int oracle_copy_slot(void *dst_pool, int32_t dst_P, int32_t dst_slot,
+                     const void *src_pool, int32_t src_P, int32_t src_slot,
+                     int64_t slot_bytes)
+{
+    if (!dst_pool || !src_pool || slot_bytes < 0)
+        return 2;
+    if (dst_slot < 0 || dst_slot >= dst_P || src_slot < 0 || src_slot >= src_P)
+        return 2;
+    memmove((char *)dst_pool + (int64_t)dst_slot * slot_bytes,
+            (const char *)src_pool + (int64_t)src_slot * slot_bytes, (size_t)slot_bytes);
+    return 0;
+}

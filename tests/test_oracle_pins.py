@@ -1,0 +1,441 @@
+"""Pins for the float64 CPU oracle, against things other than itself.
+
+Each test ties the oracle to a fact the pages or the mathematics fix: the decode
+formula of the Selective State Update page (TensorRT-Edge-LLM C++ API,
+invokeSelectiveStateUpdate), the prefill/stash and replay contracts on the same page,
+the padding contract of flashinfer.gdn_fused_decode_step (state_indices), closed forms,
+an independent vectorised formulation and the IEEE storage formats.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from einsum_ref import decode_dense, f64, prefill_dense
+from linear_attention_recurrent_selective_b200.workloads import make_case, make_config
+
+F64 = torch.float64
+
+
+def dense_state(case, pool=None):
+    pool = case.pool if pool is None else pool
+    P = case.P
+    full = pool.view(P, case.slot_stride)[:, : case.H * case.Dm * case.N]
+    return full.reshape(P, case.H, case.Dm, case.N)
+
+
+def same_bits(a, b):
+    """Byte identity (NaN-aware) of two tensors of one dtype."""
+    return a.dtype == b.dtype and a.shape == b.shape and torch.equal(
+        a.contiguous().view(torch.uint8), b.contiguous().view(torch.uint8))
+
+
+def softplus(v):
+    return v + math.log1p(math.exp(-v)) if v > 0 else math.log1p(math.exp(v))
+
+
+# ---------------------------------------------------------------- storage formats
+
+def test_f16_decode_all_bit_patterns(orc):
+    L = orc.lib()
+    bits = np.arange(65536, dtype=np.uint16)
+    want = bits.view(np.float16).astype(np.float64)
+    got = np.array([L.oracle_f16_to_double(int(b)) for b in bits])
+    same = (got == want) | (np.isnan(got) & np.isnan(want))
+    assert same.all()
+
+
+def test_bf16_decode_all_bit_patterns(orc):
+    L = orc.lib()
+    bits = torch.arange(65536, dtype=torch.int32).to(torch.int16)
+    want = bits.view(torch.bfloat16).double().numpy()
+    got = np.array([L.oracle_bf16_to_double(int(b) & 0xFFFF) for b in bits])
+    same = (got == want) | (np.isnan(got) & np.isnan(want))
+    assert same.all()
+
+
+def test_f16_encode_round_to_nearest_even(orc):
+    L = orc.lib()
+    rng = np.random.default_rng(0)
+    vals = np.concatenate([
+        rng.standard_normal(4000) * 10.0 ** rng.uniform(-9, 5, 4000),
+        [0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e6, -1e6, 2.0 ** -24, 2.0 ** -25,
+         3 * 2.0 ** -26, 2.0 ** -14, 1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11,
+         2.0 ** -14 - 2.0 ** -25],
+    ])
+    with np.errstate(over="ignore"):
+        want = vals.astype(np.float16).view(np.uint16)   # numpy rounds from double directly
+    got = np.array([L.oracle_double_to_f16(float(v)) for v in vals], dtype=np.uint16)
+    assert (got == want).all()
+    # ties go to the even neighbour
+    assert L.oracle_double_to_f16(1 + 2.0 ** -11) == 0x3C00
+    assert L.oracle_double_to_f16(1 + 3 * 2.0 ** -11) == 0x3C02
+
+
+def test_bf16_encode_round_to_nearest_even(orc):
+    L = orc.lib()
+    g = torch.Generator().manual_seed(1)
+    v = torch.randn(4000, generator=g) * torch.exp(torch.rand(4000, generator=g) * 60 - 30)
+    v = torch.cat([v, torch.tensor([0.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 3e38, 1e-40])])
+    want = v.to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    got = np.array([L.oracle_double_to_bf16(float(x)) for x in v.double()], dtype=np.uint16)
+    assert (got == want).all()
+
+
+# ---------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("shape", [
+    dict(batch=2, P=4, H=4, G=1, Dm=16, N=16),
+    dict(batch=3, P=7, H=6, G=3, Dm=5, N=8),
+    dict(batch=4, P=4, H=2, G=2, Dm=3, N=7),
+])
+@pytest.mark.parametrize("z", [False, True])
+@pytest.mark.parametrize("softplus", [False, True])
+def test_decode_matches_einsum(orc, shape, z, softplus):
+    case = make_case(seed=11, state_dtype=F64, z=z, dt_softplus=softplus, **shape)
+    idx = case.state_indices.long()
+    s0 = dense_state(case)[idx].double().numpy()
+    new, y = decode_dense(s0, f64(case.x), f64(case.A), f64(case.B), f64(case.C),
+                          f64(case.dt), f64(case.dt_bias), f64(case.D), f64(case.z),
+                          case.G, softplus)
+    out, pool, err = orc.decode_case(case)
+    assert err == 0
+    np.testing.assert_allclose(out.numpy(), y, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dense_state(case, pool)[idx].numpy(), new, rtol=1e-12,
+                               atol=1e-12)
+
+
+def test_tiny_decode_config_matches_einsum(orc):
+    case = make_config("tiny_decode")
+    idx = case.state_indices.long()
+    s0 = dense_state(case)[idx].double().numpy()
+    new, y = decode_dense(s0, f64(case.x), f64(case.A), f64(case.B), f64(case.C),
+                          f64(case.dt), f64(case.dt_bias), f64(case.D), None, case.G, True)
+    out, pool, err = orc.decode_case(case)
+    np.testing.assert_allclose(out.numpy(), y, rtol=1e-12, atol=1e-12)
+    # fp32 pool: the stored state is the float64 result rounded once to fp32
+    got = dense_state(case, pool)[idx]
+    assert torch.equal(got, torch.from_numpy(new).float())
+    # slots 1 and 3 are not indexed: byte-identical
+    for s in (1, 3):
+        assert torch.equal(dense_state(case, pool)[s], dense_state(case)[s])
+
+
+def test_zero_dt_leaves_state_bit_identical(orc):
+    # softplus off, no bias, dt = 0: decay exp(0) = 1 and the input term vanishes
+    case = make_case(seed=3, batch=3, P=5, H=4, G=2, Dm=8, N=16, dt_bias=False,
+                     dt_softplus=False, z=False)
+    case.dt.zero_()
+    out, pool, _ = orc.decode_case(case)
+    assert torch.equal(pool, case.pool)
+    idx = case.state_indices.long()
+    S = dense_state(case)[idx].double()
+    grp = torch.arange(case.H) // (case.H // case.G)
+    y = torch.einsum("bhdn,bhn->bhd", S, case.C.double()[:, grp])
+    y += case.D.double()[None, :, None] * case.x.double()
+    np.testing.assert_allclose(out.numpy(), y.numpy(), rtol=1e-13, atol=1e-13)
+
+
+def test_scalar_worked_example(orc):
+    # H = Dm = N = G = 1, softplus off: dt = 0.5, A = -2 -> decay e^-1;
+    # state 2, B 3, x 4, C 0.5, D 0.25, z 1:
+    #   new state = 2 e^-1 + 3 * 0.5 * 4 = 6 + 2/e
+    #   out = ((6 + 2/e) * 0.5 + 0.25 * 4) * silu(1),  silu(1) = 1 / (1 + e^-1)
+    f = lambda v: torch.tensor(v, dtype=torch.float32)
+    pool = torch.tensor([2.0], dtype=F64)
+    out, err = orc.decode(f([[[4.0]]]), f([-2.0]), f([[[3.0]]]), f([[[0.5]]]), f([[0.5]]),
+                          pool, D=f([0.25]), z=f([[[1.0]]]), batch=1, H=1, G=1, Dm=1, N=1,
+                          dt_softplus=False)
+    e = math.e
+    assert pool.item() == pytest.approx(6 + 2 / e, rel=1e-15)
+    assert out.item() == pytest.approx((3 + 1 / e + 1) / (1 + 1 / e), rel=1e-15)
+
+
+def test_group_map_contiguous_blocks(orc):
+    # H = 4, G = 2: heads 0,1 read group 0 and heads 2,3 read group 1. With B of group 1
+    # zero, heads 2,3 see pure decay while heads 0,1 still get input.
+    case = make_case(seed=5, batch=2, P=2, H=4, G=2, Dm=3, N=4, indices="none",
+                     state_dtype=F64)
+    case.B[:, 1].zero_()
+    out, pool, _ = orc.decode_case(case)
+    S0, S1 = dense_state(case), dense_state(case, pool)
+    v = case.dt.double() + case.dt_bias.double()
+    dte = torch.nn.functional.softplus(v)
+    decay = torch.exp(case.A.double()[None] * dte)
+    for h in (2, 3):
+        np.testing.assert_allclose(S1[:, h], S0[:, h] * decay[:, h, None, None], rtol=1e-14)
+    for h in (0, 1):
+        assert not torch.allclose(S1[:, h], S0[:, h] * decay[:, h, None, None])
+
+
+def test_padding_rows_and_inactive_rows(orc):
+    # 10 rows captured, 7 active, 2 of the active rows are padding (index -1)
+    case = make_case(seed=7, batch=10, P=16, H=4, G=2, Dm=8, N=16, active=7, n_pad=2,
+                     z=True, x_dtype=torch.float16, bc_dtype=torch.float16,
+                     state_dtype=torch.float16)
+    out, pool, err = orc.decode_case(case)
+    assert err == 0
+    si = case.state_indices
+    pad = [b for b in range(7) if si[b] < 0]
+    assert len(pad) == 2
+    for b in pad:
+        assert torch.all(out[b] == 0)
+    assert torch.isnan(out[7:]).all()               # rows >= active not written
+    live = {int(si[b]) for b in range(7) if si[b] >= 0}
+    for s in range(case.P):
+        same = torch.equal(dense_state(case, pool)[s], dense_state(case)[s])
+        assert same == (s not in live), s            # exactly the live slots change
+
+
+def test_index_out_of_range_sets_flag_and_skips(orc):
+    case = make_case(seed=8, batch=3, P=4, H=2, G=1, Dm=4, N=8, indices=[1, 4, 7])
+    out, pool, err = orc.decode_case(case)
+    assert err == 1
+    assert torch.isnan(out[1:]).all()
+    changed = [s for s in range(4)
+               if not torch.equal(dense_state(case, pool)[s], dense_state(case)[s])]
+    assert changed == [1]
+
+
+def test_padded_slot_stride_untouched(orc):
+    case = make_case(seed=9, batch=2, P=3, H=2, G=1, Dm=4, N=8, slot_pad=5)
+    _, pool, _ = orc.decode_case(case)
+    tail = lambda p: p.view(case.P, case.slot_stride)[:, case.H * case.Dm * case.N:]
+    assert torch.equal(tail(pool), tail(case.pool))
+
+
+def test_linearity_without_gate(orc):
+    # with z absent, (state, x) -> (state', y) is linear for fixed A, B, C, dt, D
+    c1 = make_case(seed=10, batch=2, H=3, G=1, Dm=4, N=6, indices="none", state_dtype=F64,
+                   x_dtype=F64)
+    c2 = make_case(seed=20, batch=2, H=3, G=1, Dm=4, N=6, indices="none", state_dtype=F64,
+                   x_dtype=F64)
+    al, be = 0.7, -1.3
+
+    def run(pool, x):
+        pool = pool.clone()
+        out, _ = orc.decode(x, c1.A, c1.B, c1.C, c1.dt, pool, dt_bias=c1.dt_bias, D=c1.D,
+                            batch=2, H=3, G=1, Dm=4, N=6)
+        return pool, out
+
+    p1, y1 = run(c1.pool, c1.x)
+    p2, y2 = run(c2.pool, c2.x)
+    p3, y3 = run(al * c1.pool + be * c2.pool, al * c1.x + be * c2.x)
+    np.testing.assert_allclose(p3, al * p1 + be * p2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(y3, al * y1 + be * y2, rtol=1e-12, atol=1e-12)
+
+
+def test_indices_equal_gather_run_scatter(orc):
+    # Selective State Update page, invokeMambaStateGather / Scatter: running through
+    # stateIndices equals gathering the rows to a dense batch, running with identity
+    # indices and scattering back.
+    case = make_case(seed=12, batch=5, P=9, H=4, G=2, Dm=4, N=8, z=True)
+    out_idx, pool_idx, _ = orc.decode_case(case)
+    idx = case.state_indices.long()
+    slot = case.slot_stride
+    dense = case.pool.view(case.P, slot)[idx].clone().reshape(-1)
+    out_dense, _ = orc.decode(case.x, case.A, case.B, case.C, case.dt, dense,
+                              dt_bias=case.dt_bias, D=case.D, z=case.z, batch=5, H=4, G=2,
+                              Dm=4, N=8)
+    scattered = case.pool.clone().view(case.P, slot)
+    scattered[idx] = dense.view(5, slot)
+    assert torch.equal(out_idx, out_dense)
+    assert torch.equal(scattered.reshape(-1), pool_idx)
+
+
+def test_16bit_pool_store_is_round_of_exact(orc):
+    for sdt in (torch.float16, torch.bfloat16):
+        case = make_case(seed=13, batch=3, P=3, H=2, G=1, Dm=8, N=16, state_dtype=sdt,
+                         indices="none")
+        _, pool16, _ = orc.decode_case(case)
+        exact = case.pool.double()
+        _, pool64 = orc.decode_case(case, pool=exact)[:2]
+        assert torch.equal(pool16, pool64.to(sdt))
+
+
+# ---------------------------------------------------------------- prefill
+
+def test_prefill_matches_einsum_with_lengths(orc):
+    case = make_case(seed=14, batch=4, P=6, T=7, H=4, G=2, Dm=3, N=8, z=True,
+                     state_dtype=F64, lengths="context")
+    case.context_lengths[0] = 7
+    idx = case.state_indices.long()
+    s0 = dense_state(case)[idx].numpy().copy()
+    L = case.context_lengths.numpy()
+    sT, y = prefill_dense(s0, f64(case.x), f64(case.A), f64(case.B), f64(case.C),
+                          f64(case.dt), f64(case.dt_bias), f64(case.D), f64(case.z),
+                          case.G, True, lengths=L)
+    out, pool, _, err = orc.prefill_case(case)
+    assert err == 0
+    np.testing.assert_allclose(out.numpy(), y, rtol=1e-12, atol=1e-12)   # NaN where t >= L
+    np.testing.assert_allclose(dense_state(case, pool)[idx].numpy(), sT, rtol=1e-12,
+                               atol=1e-12)
+
+
+def test_T_decodes_equal_one_prefill(orc):
+    case = make_case(seed=15, batch=3, P=5, T=6, H=4, G=1, Dm=4, N=8, z=True,
+                     state_dtype=F64, slow_decay=True)
+    out_p, pool_p, _, _ = orc.prefill_case(case)
+    pool_d = case.pool.clone()
+    for t in range(case.T):
+        out_t, _ = orc.decode(case.x[:, t].contiguous(), case.A, case.B[:, t].contiguous(),
+                              case.C[:, t].contiguous(), case.dt[:, t].contiguous(), pool_d,
+                              dt_bias=case.dt_bias, D=case.D, z=case.z[:, t].contiguous(),
+                              state_indices=case.state_indices, batch=3, H=4, G=1, Dm=4,
+                              N=8)
+        assert same_bits(out_t, out_p[:, t].contiguous())
+    assert torch.equal(pool_d, pool_p)
+
+
+def test_pure_decay_closed_form(orc):
+    # B = 0: S_T = S_0 * exp(A * sum_t dt_eff_t)
+    case = make_case(seed=16, batch=2, P=2, T=9, H=3, G=1, Dm=2, N=4, indices="none",
+                     state_dtype=F64, slow_decay=True)
+    case.B.zero_()
+    _, pool, _, _ = orc.prefill_case(case)
+    for b in range(2):
+        for h in range(3):
+            tot = sum(softplus(float(case.dt[b, t, h]) + float(case.dt_bias[h]))
+                      for t in range(case.T))
+            want = dense_state(case)[b, h] * math.exp(float(case.A[h]) * tot)
+            np.testing.assert_allclose(dense_state(case, pool)[b, h], want, rtol=1e-12)
+
+
+def test_pure_accumulation_closed_form(orc):
+    # A = 0: S_T = S_0 + sum_t B_t * dt_eff_t * x_t
+    case = make_case(seed=17, batch=2, P=2, T=5, H=2, G=1, Dm=3, N=4, indices="none",
+                     state_dtype=F64)
+    case.A.zero_()
+    _, pool, _, _ = orc.prefill_case(case)
+    S0, S1 = dense_state(case), dense_state(case, pool)
+    for b in range(2):
+        for h in range(2):
+            acc = S0[b, h].clone()
+            for t in range(case.T):
+                dte = softplus(float(case.dt[b, t, h]) + float(case.dt_bias[h]))
+                acc += dte * torch.outer(case.x[b, t, h].double(), case.B[b, t, 0].double())
+            np.testing.assert_allclose(S1[b, h], acc, rtol=1e-12, atol=1e-12)
+
+
+def test_scalar_recurrence_closed_form(orc):
+    # H = Dm = N = G = 1: s_t = a_t s_{t-1} + b_t, so
+    # s_T = (prod_t a_t) s_0 + sum_t b_t prod_{u>t} a_u, and y_t = s_t C_t + D x_t, gated.
+    case = make_case(seed=18, batch=1, P=1, T=8, H=1, G=1, Dm=1, N=1, indices="none",
+                     state_dtype=F64, z=True, slow_decay=True)
+    out, pool, _, _ = orc.prefill_case(case)
+    A, bias, D = float(case.A[0]), float(case.dt_bias[0]), float(case.D[0])
+    a, bb = [], []
+    for t in range(case.T):
+        dte = softplus(float(case.dt[0, t, 0]) + bias)
+        a.append(math.exp(A * dte))
+        bb.append(float(case.B[0, t, 0, 0]) * dte * float(case.x[0, t, 0, 0]))
+    s0 = float(case.pool[0])
+    sT = math.prod(a) * s0 + sum(bb[t] * math.prod(a[t + 1:]) for t in range(case.T))
+    assert float(pool[0]) == pytest.approx(sT, rel=1e-13, abs=1e-14)
+    s = s0
+    for t in range(case.T):
+        s = a[t] * s + bb[t]
+        zt = float(case.z[0, t, 0, 0])
+        y = (s * float(case.C[0, t, 0, 0]) + D * float(case.x[0, t, 0, 0])) * zt / (1 + math.exp(-zt))
+        assert float(out[0, t, 0, 0]) == pytest.approx(y, rel=1e-13, abs=1e-14)
+
+
+def test_prefill_stash_leaves_pool_and_matches_no_stash(orc):
+    case = make_case(seed=19, batch=4, P=8, T=5, H=4, G=2, Dm=4, N=8, z=True,
+                     x_dtype=torch.bfloat16, bc_dtype=torch.bfloat16, lengths="context")
+    out_s, pool_s, st, _ = orc.prefill_case(case, stash=True)
+    out_n, _, _, _ = orc.prefill_case(case)
+    assert torch.equal(pool_s, case.pool)             # committed state read only
+    assert same_bits(out_s, out_n)
+    DA, U, Bst, DT = st
+    for b in range(case.batch):
+        L = int(case.context_lengths[b])
+        # U and B are the inputs widened exactly; positions >= L are untouched
+        assert torch.equal(U[b, :L], case.x[b, :L].float())
+        assert torch.equal(Bst[b, :L], case.B[b, :L].float())
+        assert torch.isnan(U[b, L:]).all() and torch.isnan(DA[b, L:]).all()
+        dte = torch.nn.functional.softplus(case.dt[b, :L].double() + case.dt_bias.double())
+        np.testing.assert_allclose(DT[b, :L], dte, rtol=1e-7)
+        np.testing.assert_allclose(DA[b, :L], torch.exp(case.A.double() * dte), rtol=1e-7)
+
+
+@pytest.mark.parametrize("k", [0, 1, 3, 5])
+def test_replay_k_equals_k_decodes(orc, k):
+    case = make_case(seed=21, batch=3, P=6, T=5, H=4, G=2, Dm=4, N=8, z=True,
+                     state_dtype=F64)
+    _, _, st, _ = orc.prefill_case(case, stash=True)
+    acc = torch.full((3,), k, dtype=torch.int32)
+    pool_r = case.pool.clone()
+    assert orc.replay(pool_r, st, acc, state_indices=case.state_indices, batch=3, T=5, H=4,
+                      G=2, Dm=4, N=8) == 0
+    pool_d = case.pool.clone()
+    for t in range(k):
+        orc.decode(case.x[:, t].contiguous(), case.A, case.B[:, t].contiguous(),
+                   case.C[:, t].contiguous(), case.dt[:, t].contiguous(), pool_d,
+                   dt_bias=case.dt_bias, D=case.D, state_indices=case.state_indices,
+                   batch=3, H=4, G=2, Dm=4, N=8)
+    if k == 0:
+        assert torch.equal(pool_r, case.pool)
+    # the stash carries fp32 decay/dt: agreement to fp32 rounding of those factors
+    np.testing.assert_allclose(pool_r, pool_d, rtol=1e-6, atol=1e-6)
+
+
+def test_replay_rows_and_flags(orc):
+    case = make_case(seed=22, batch=6, P=10, T=4, H=2, G=1, Dm=4, N=8, active=5, n_pad=1,
+                     lengths="accepted")
+    _, _, st, _ = orc.prefill_case(case, stash=True)
+    acc = torch.tensor([4, 2, 0, 9, -1, 3], dtype=torch.int32)
+    pool = case.pool.clone()
+    err = orc.replay(pool, st, acc, state_indices=case.state_indices, batch=6, active=5,
+                     T=4, H=2, G=1, Dm=4, N=8)
+    assert err == 2 | 8
+    si = case.state_indices
+    touched = {int(si[b]) for b in range(5) if si[b] >= 0 and int(acc[b]) > 0}
+    for s in range(case.P):
+        same = torch.equal(dense_state(case, pool)[s], dense_state(case)[s])
+        assert same == (s not in touched)
+
+
+def test_prefill_length_flags(orc):
+    case = make_case(seed=23, batch=3, P=3, T=4, H=2, G=1, Dm=2, N=4, indices="none")
+    case.context_lengths = torch.tensor([9, -2, 0], dtype=torch.int32)
+    out, pool, _, err = orc.prefill_case(case)
+    assert err == 4 | 8
+    assert not torch.isnan(out[0]).any()           # clamped to T
+    assert torch.isnan(out[1:]).all()              # length <= 0: row untouched
+    assert torch.equal(dense_state(case, pool)[1:], dense_state(case)[1:])
+
+
+def test_clear_and_copy_slot(orc):
+    pool = torch.arange(1, 4 * 6 + 1, dtype=torch.float32)
+    orc.clear_slot(pool, 6 * 4, 4, 2)
+    assert (pool.view(4, 6)[2] == 0).all() and (pool.view(4, 6)[[0, 1, 3]] != 0).all()
+    orc.clear_slot(pool, 6 * 4, 4, -1)
+    assert (pool == 0).all()
+    src = torch.arange(3 * 6, dtype=torch.float32)
+    dst = torch.zeros(5 * 6)
+    orc.copy_slot(dst, 5, 4, src, 3, 1, 6 * 4)
+    assert torch.equal(dst.view(5, 6)[4], src.view(3, 6)[1])
+    assert (dst.view(5, 6)[:4] == 0).all()
+
+
+def test_golden_tiny_decode_snapshot(orc):
+    # Snapshot written by tests/golden/make_golden.py; changing the oracle's arithmetic
+    # must regenerate it on purpose.
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "tiny_decode.txt")
+    sec, vals = None, {"out": [], "state": []}
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        if line in vals:
+            sec = line
+            continue
+        vals[sec].append(float(line))
+    case = make_config("tiny_decode")
+    out, pool, _ = orc.decode_case(case)
+    assert out.reshape(-1).tolist() == vals["out"]
+    assert pool.view(4, -1)[[2, 0]].reshape(-1).tolist() == vals["state"]
