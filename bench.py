@@ -1,0 +1,468 @@
+#!/usr/bin/env python3
+"""Benchmark of the selective state update over a paged state pool (one JSON line).
+
+Headline step: one ssu_decode launch over the Mamba2-2.7B-like decode workload
+(batch 256 over a 512-slot pool, 80 heads, dim 64, dstate 128, one group, bf16
+x/B/C/z/out, fp32 dt/A/D/dt_bias and fp32 state, softplus with dt_bias, z gate,
+stateIndices a random subset of the pool). Each step reads and writes 20,480 head
+states of 32 KiB: 671 MB of state per step, far above the 126 MB L2, so consecutive
+steps do not hit in L2 and no flush is needed (checked at run time).
+
+  value      seq-head updates/s over all ranks (K steps x batch x heads / max time)
+  roofline   the decode kernel's algorithmic bytes / its mean launch time (CUDA events
+             on the launching stream) against the measured HBM copy bandwidth
+  e2e        the same metric through the public binding with the step's inputs copied
+             from pinned host memory and the output copied back inside the timed region
+  forms      (one GPU only) the prefill scan and the speculative replay on their own
+             workloads, same timing method
+  cpu_baseline  the float64 CPU oracle on a bounded sample, rank 0, one GPU only
+
+Multi-GPU (torchrun): replicas only -- every rank runs its own pool and batch, no data
+collective; the barrier and the max-over-ranks reduction are measurement plumbing.
+`--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "decode state-update HBM GB/s (% of B200 peak); seq-head updates/s at batch 256"
+UNIT = "seq-head updates/s"
+WORKLOAD = "mamba2_decode_b256"
+FALLBACK_HBM_GBS = 6650.0
+
+REASON_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_bytes(batch, H, G, Dm, N, state_bytes, io_bytes):
+    """Algorithmic bytes of one decode launch: every state element read and written once,
+    x/z/out once per (row, head, dim), B/C once per (row, group), dt once per (row, head),
+    A/D/dt_bias once per head, one index per row."""
+    units = batch * H
+    state = units * Dm * N * state_bytes * 2
+    io = units * Dm * io_bytes * 3 + units * 4 + batch * G * N * io_bytes * 2
+    return state, state + io + H * 12 + batch * 4
+
+
+def world():
+    return int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank float over the process group (identity without one)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step: int, steps: int, n_ranks: int, seconds: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return units_per_rank_step * steps * n_ranks / seconds
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons via NVML while the timed region runs."""
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples = []      # (t, sm_mhz, reasons_mask)
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self._handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self._nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report the absence instead of clocks
+            self.error = repr(e)
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = n.nvmlDeviceGetClockInfo(self._handle, n.NVML_CLOCK_SM)
+                reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+                self.samples.append((time.perf_counter(), mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def start(self):
+        if self._handle is not None:
+            self._thread.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._thread.is_alive():
+            self._thread.join()
+
+    def summary(self, t0: float, t1: float):
+        if self._handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": "NVML unavailable: " + getattr(self, "error", "")}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "samples inside the timed region"
+        if not win:   # timed region shorter than the poll period: nearest samples
+            win = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+            note = "timed region shorter than the poll period: nearest samples"
+        mask = 0
+        for s in win:
+            mask |= s[2]
+        return {"sm_mhz": statistics.median(s[1] for s in win) if win else None,
+                "sm_max_mhz": self.max_mhz,
+                "reasons": [v for k, v in REASON_BITS.items() if mask & k and k != 0x1],
+                "samples": len(win), "note": note}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_decode(args, device):
+    from linear_attention_recurrent_selective_b200 import ssu
+    from linear_attention_recurrent_selective_b200.workloads import make_config
+
+    overrides = {}
+    if args.batch:
+        overrides = dict(batch=args.batch, P=2 * args.batch)
+    case = make_config(WORKLOAD, **overrides)
+    d = case.to(device)
+    pool = d.pool
+    out = torch.empty_like(d.x)
+    units = case.batch * case.H
+    state_b, alg_b = decode_bytes(case.batch, case.H, case.G, case.Dm, case.N,
+                                  pool.element_size(), d.x.element_size())
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = state_b < 2 * l2
+    flush_buf = torch.empty(4 * l2 // 4, dtype=torch.float32, device=device) if flush else None
+
+    def step():
+        ssu.ssu_decode(d.x, d.A, d.B, d.C, d.dt, pool, out, dt_bias=d.dt_bias, D=d.D, z=d.z,
+                       state_indices=d.state_indices, active_batch=case.active,
+                       slot_stride=case.slot_stride, P=case.P)
+
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        if flush:
+            flush_buf.zero_()
+        step()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_all0, t_all1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(device.index).start()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    wall0 = time.perf_counter()
+    t_all0.record(stream)
+    for k in range(args.steps):
+        if flush:
+            flush_buf.zero_()
+        starts[k].record(stream)
+        step()
+        ends[k].record(stream)
+    t_all1.record(stream)
+    torch.cuda.synchronize(device)
+    wall1 = time.perf_counter()
+    barrier(device)
+    torch.cuda.synchronize(device)
+    clocks.stop()
+    total_ms = t_all0.elapsed_time(t_all1)
+    kern_ms = statistics.fmean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    res = dict(case=case, units=units, total_ms=total_ms, kern_ms=kern_ms, state_b=state_b,
+               alg_b=alg_b, clocks=clocks.summary(wall0, wall1), flush=flush, l2=l2)
+
+    # ---- end to end through the binding: pinned host inputs in, output back out
+    host = {k: getattr(case, k).pin_memory() for k in ("x", "z", "B", "C", "dt",
+                                                       "state_indices")}
+    dev_in = {k: torch.empty_like(v, device=device) for k, v in host.items()}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        for k in host:
+            dev_in[k].copy_(host[k], non_blocking=True)
+        ssu.ssu_decode(dev_in["x"], d.A, dev_in["B"], dev_in["C"], dev_in["dt"], pool, out,
+                       dt_bias=d.dt_bias, D=d.D, z=dev_in["z"],
+                       state_indices=dev_in["state_indices"], active_batch=case.active,
+                       slot_stride=case.slot_stride, P=case.P)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    res["e2e_ms"] = e0.elapsed_time(e1)
+    res["h2d"] = sum(v.numel() * v.element_size() for v in host.values())
+    res["d2h"] = out_h.numel() * out_h.element_size()
+    return res
+
+
+def time_launches(fn, steps, warmup, device):
+    stream = torch.cuda.current_stream(device)
+    for _ in range(warmup):
+        fn()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    torch.cuda.synchronize(device)
+    for k in range(steps):
+        starts[k].record(stream)
+        fn()
+        ends[k].record(stream)
+    torch.cuda.synchronize(device)
+    return statistics.fmean(s.elapsed_time(e) for s, e in zip(starts, ends))
+
+
+def run_forms(args, device, hbm_peak):
+    """Prefill (batch 16, T 512, contextLengths ~ U{1..512}) and speculative replay
+    (batch 64, 5 drafted tokens, acceptedLengths ~ U{0..5}) on one GPU."""
+    from linear_attention_recurrent_selective_b200 import ssu
+    from linear_attention_recurrent_selective_b200.workloads import make_config
+
+    forms = {}
+    steps, warm = max(3, min(args.steps, 50)), max(3, min(args.warmup, 5))
+
+    case = make_config("prefill_b16_t512")
+    d = case.to(device)
+    pool = d.pool.clone()
+    out = torch.empty_like(d.x)
+    f = dict(dtype=torch.float32, device=device)
+    b, T, H, G, Dm, N = case.batch, case.T, case.H, case.G, case.Dm, case.N
+    stash = (torch.empty(b, T, H, **f), torch.empty(b, T, H, Dm, **f),
+             torch.empty(b, T, G, N, **f), torch.empty(b, T, H, **f))
+    tokens = int(case.context_lengths.sum())
+
+    def prefill(st):
+        ssu.ssu_prefill(d.x, d.A, d.B, d.C, d.dt, pool, out, dt_bias=d.dt_bias, D=d.D, z=d.z,
+                        state_indices=d.state_indices, context_lengths=d.context_lengths,
+                        stash=st, slot_stride=case.slot_stride, P=case.P)
+
+    flop = tokens * H * Dm * N * 5       # per state element: mul + FMA update, FMA output
+    sm = torch.cuda.get_device_properties(device).multi_processor_count
+    alu_peak = sm * 128 * 2 * 1.965e9 / 1e12   # fp32 FMA lanes x 2 FLOP x max SM clock
+    for name, st in (("prefill", None), ("prefill_stash", stash)):
+        ms = time_launches(lambda: prefill(st), steps, warm, device)
+        forms[name] = {
+            "workload": "prefill_b16_t512", "tokens": tokens, "ms_per_launch": ms,
+            "tokens_per_s": tokens / (ms / 1e3),
+            "roofline": {"bound": "alu", "achieved": flop / (ms / 1e3) / 1e12,
+                         "peak": alu_peak, "unit": "TFLOP/s",
+                         "frac": flop / (ms / 1e3) / 1e12 / alu_peak, "traffic": None}}
+
+    rcase = make_config("spec_replay_b64_t5")
+    rd = rcase.to(device)
+    rpool = rd.pool.clone()
+    b, T, H, G, Dm, N = rcase.batch, rcase.T, rcase.H, rcase.G, rcase.Dm, rcase.N
+    rst = (torch.empty(b, T, H, **f), torch.empty(b, T, H, Dm, **f),
+           torch.empty(b, T, G, N, **f), torch.empty(b, T, H, **f))
+    rout = torch.empty_like(rd.x)
+    # the stash comes from this library's prefill in stash mode (the pool stays as is)
+    ssu.ssu_prefill(rd.x, rd.A, rd.B, rd.C, rd.dt, rpool, rout, dt_bias=rd.dt_bias, D=rd.D,
+                    z=rd.z, state_indices=rd.state_indices, stash=rst,
+                    slot_stride=rcase.slot_stride, P=rcase.P)
+    acc = rd.accepted_lengths
+    ms = time_launches(lambda: ssu.ssu_replay(rpool, rst, acc, state_indices=rd.state_indices,
+                                              slot_stride=rcase.slot_stride, P=rcase.P),
+                       steps, warm, device)
+    acc_h = rcase.accepted_lengths
+    rows = int((acc_h > 0).sum())
+    nacc = int(acc_h.sum())
+    rbytes = rows * H * Dm * N * 4 * 2 + nacc * (H * (4 + 4 + Dm * 4) + G * N * 4) + b * 4
+    forms["replay"] = {
+        "workload": "spec_replay_b64_t5", "accepted_tokens": nacc, "ms_per_launch": ms,
+        "accepted_tokens_per_s": nacc / (ms / 1e3),
+        "roofline": {"bound": "hbm", "achieved": rbytes / (ms / 1e3) / 1e9,
+                     "peak": hbm_peak, "unit": "GB/s",
+                     "frac": rbytes / (ms / 1e3) / 1e9 / hbm_peak, "traffic": None}}
+    return forms
+
+
+def cpu_baseline_decode(case, max_seconds=20.0):
+    """The float64 oracle on whole decode steps of the same workload, timed on this host."""
+    from oracle import oracle
+    oracle.build()
+    units = case.batch * case.H
+    runs, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode_case(case)
+        runs += 1
+        el = time.perf_counter() - t0
+        if el > max_seconds / 2 or runs >= 2:
+            break
+    return {"value": units * runs / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{runs} full decode step(s) of the batch-{case.batch} workload "
+                      f"({units} seq-head updates each), single thread, {el:.1f} s"}
+
+
+def config_block(case, res=None):
+    c = {"workload": WORKLOAD, "batch": case.batch, "pool_slots": case.P, "nheads": case.H,
+         "dim": case.Dm, "dstate": case.N, "ngroups": case.G, "state_dtype": "f32",
+         "io_dtype": str(case.x.dtype).replace("torch.", ""), "z_gate": case.z is not None,
+         "dt_softplus": case.dt_softplus, "parallelism": "replicas"}
+    if res is not None:
+        c["l2"] = (f"state per step {res['state_b'] / 1e6:.0f} MB vs L2 {res['l2'] / 1e6:.0f} MB: "
+                   + ("L2 flushed between steps" if res["flush"] else "inputs larger than L2, no flush"))
+    return c
+
+
+def main_ours(args):
+    n_world, rank, local = world()
+    if n_world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local if n_world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(device)
+    hbm_peak, peak_src = measured_peaks()
+
+    res = run_decode(args, device)
+    case = res["case"]
+    t_max = max_over_ranks(res["total_ms"], device)
+    e2e_max = max_over_ranks(res["e2e_ms"], device)
+    value = job_throughput(res["units"], args.steps, n_world, t_max / 1e3)
+    e2e_value = job_throughput(res["units"], args.steps, n_world, e2e_max / 1e3)
+    achieved = res["alg_b"] / (res["kern_ms"] / 1e3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n_world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": config_block(case, res),
+        "state_hbm_gbs": res["state_b"] / (res["kern_ms"] / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": args.traffic,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_src == "measured" else "fallback 6.65 TB/s",
+                     "kernel": "ssu_decode_kernel", "kernel_ms": res["kern_ms"],
+                     "algorithmic_bytes": res["alg_b"]},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": res["h2d"],
+                "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": args.steps,
+        "clocks": res["clocks"],
+    }
+    if n_world == 1 and not args.no_forms:
+        line["forms"] = run_forms(args, device, hbm_peak)
+    if n_world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_decode(case)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if n_world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def main_reference(args):
+    """The float64 CPU oracle as the reference arm: rank 0 only, bounded per-step samples."""
+    n_world, rank, _ = world()
+    if rank != 0:
+        return
+    from linear_attention_recurrent_selective_b200.workloads import make_config
+    from oracle import oracle
+    oracle.build()
+    case = make_config(WORKLOAD)
+    # one head-row of work is ~20 ms in the oracle: keep the whole run near a minute
+    rows = max(1, min(case.batch, int(60.0 / max(1, args.steps + args.warmup) / 0.02)))
+    sub = case
+    import dataclasses
+    pick = {f: getattr(case, f)[:rows].contiguous()
+            for f in ("x", "z", "B", "C", "dt", "state_indices")}
+    sub = dataclasses.replace(case, batch=rows, active=rows, **pick)
+    for _ in range(args.warmup):
+        oracle.decode_case(sub)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.decode_case(sub)
+    el = time.perf_counter() - t0
+    units = rows * case.H * args.steps
+    value = units / el
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n_world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_block(case), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} of {case.batch} rows x {case.H} heads per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the batch (pool = 2 x batch), e.g. for a small profile")
+    ap.add_argument("--no-forms", action="store_true", help="skip the prefill/replay forms")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu DRAM bytes per decode launch for this build (else null)")
+    a = ap.parse_args(argv)
+    if a.warmup < 3 and a.impl == "ours":
+        ap.error("--warmup must be at least 3")
+    return a
+
+
+if __name__ == "__main__":
+    args = parse()
+    if args.impl == "reference":
+        main_reference(args)
+    else:
+        main_ours(args)

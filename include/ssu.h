@@ -1,0 +1,175 @@
+/*
+ * ssu.h -- C ABI of the B200 selective-state-update library (libssu.so).
+ *
+ * The Mamba selective state update over a paged recurrent-state pool, in its three
+ * forms (single-token decode, multi-token prefill with an optional replay stash, and
+ * the replay of accepted speculative tokens), plus slot clear and slot copy.
+ *
+ * Sources: the "Selective State Update" page of the TensorRT-Edge-LLM C++ API
+ * (mamba_ssm::invokeSelectiveStateUpdate, invokeSelectiveStateUpdatePrefill,
+ * struct MambaReplayLayerInfo, invokeMambaReplayReconstructBatched,
+ * invokeMambaStateClear), the padding contract of the FlashInfer page
+ * "flashinfer.gdn_fused_decode_step" (parameters state_indices and ssm_state), and the
+ * "Recurrent State Manager" page (clearSlot, clear, copySlotFrom).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Device pointers unless stated otherwise. The caller owns every buffer; the library
+ *    allocates nothing, keeps no state between calls and never synchronises the host.
+ *    All work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
+ *    stream), so every entry point may be recorded into a CUDA graph.
+ *  - Optional inputs are NULL when absent.
+ *  - Layouts are dense, row-major and batch-major as written beside each argument.
+ *    Names: batch rows b, tokens t, heads h < nheads (H), groups g < ngroups (G),
+ *    dim index d < dim (Dm), state index n < dstate (N). Head h reads group
+ *    g = h / (H / G); H must be a multiple of G.
+ *  - The state pool is [P, H, Dm, N] with dstate innermost. Slot s starts at element
+ *    s * slot_stride; slot_stride >= H*Dm*N allows padded slots (the padding is never
+ *    touched). The pool pointer must be 16-byte aligned and slot_stride * element size
+ *    a multiple of 16 bytes.
+ *  - state_indices [batch] int32 maps row b to its pool slot (NULL: row b uses slot b).
+ *    A negative index marks a padding row: its state is neither read nor written and
+ *    its output rows are written as zero. Indices of the active rows that are >= 0 must
+ *    be distinct (two rows updating one slot would race).
+ *  - Only rows b < active_batch are visited; rows beyond it are left untouched, so a
+ *    graph captured at the maximum batch can run a smaller live batch.
+ *  - An index >= P, or a length outside [0, T], is a caller bug that the pages leave
+ *    undefined. Here it never causes an out-of-bounds access: the row is skipped (index)
+ *    or the length clamped, and a bit is OR-ed into the optional device int32 err_flags:
+ *    SSU_FLAG_INDEX_RANGE, SSU_FLAG_ACCEPTED_RANGE, SSU_FLAG_CONTEXT_RANGE,
+ *    SSU_FLAG_NEGATIVE_LENGTH.
+ *  - Return value: SSU_OK, or an ssu_status error, in which case nothing was launched
+ *    (SSU_ERR_CUDA: the launch itself failed). Sizes and dtype codes are checked first;
+ *    a call with nothing to do (active_batch == 0, or T == 0) then returns SSU_OK without
+ *    looking at any pointer, since empty tensors may carry NULL data pointers.
+ *  - Arithmetic is fp32; fp16/bf16 values are widened exactly and results are rounded
+ *    to nearest-even once when stored.
+ */
+#ifndef SSU_H
+#define SSU_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t, declared here so the header needs no CUDA include. */
+typedef struct CUstream_st *ssu_stream_t;
+
+typedef enum { SSU_F32 = 0, SSU_F16 = 1, SSU_BF16 = 2 } ssu_dtype;
+
+typedef enum {
+    SSU_OK = 0,
+    SSU_ERR_NULL = 1,         /* a required pointer is NULL, or the stash is partial */
+    SSU_ERR_SHAPE = 2,        /* sizes inconsistent (H % G, active > batch, stride, ...) */
+    SSU_ERR_DTYPE = 3,        /* dtype code not one of ssu_dtype */
+    SSU_ERR_UNSUPPORTED = 4,  /* dstate not in {8,16,32,64,128,256} */
+    SSU_ERR_CUDA = 5,         /* the kernel launch failed */
+    SSU_ERR_ALIGN = 6         /* pool pointer or slot stride not 16-byte aligned */
+} ssu_status;
+
+enum {
+    SSU_FLAG_INDEX_RANGE = 1,     /* state_indices[b] >= P: row skipped */
+    SSU_FLAG_ACCEPTED_RANGE = 2,  /* accepted_lengths[b] > T: clamped to T */
+    SSU_FLAG_CONTEXT_RANGE = 4,   /* context_lengths[b] > T: clamped to T */
+    SSU_FLAG_NEGATIVE_LENGTH = 8  /* a negative length: treated as 0 */
+};
+
+/*
+ * ssu_decode -- one token (seq_len == 1) for every active row.
+ * Selective State Update page, mamba_ssm::invokeSelectiveStateUpdate:
+ *     dt_eff    = softplus(dt + dt_bias) if dt_softplus, else dt + dt_bias
+ *     new_state = state * exp(A * dt_eff) + B * dt_eff * x        (in place, in the pool)
+ *     out       = sum_n new_state[n] * C[n] + D * x,  times silu(z) if z is given
+ *
+ *   x        [batch, H, Dm]  x_dtype          A        [H] fp32
+ *   B, C     [batch, G, N]   bc_dtype         dt       [batch, H] fp32
+ *   dt_bias  [H] fp32 (optional)              D        [H] fp32 (optional)
+ *   z        [batch, H, Dm]  x_dtype (optional gate)
+ *   state    pool [P, H, Dm, N] state_dtype, slot stride slot_stride elements; in place
+ *   out      [batch, H, Dm]  x_dtype; rows b >= active_batch are not written
+ *   state_indices [batch] int32 (optional); err_flags int32 (optional)
+ * The output is reduced from the fp32 new state before it is rounded to state_dtype.
+ */
+int ssu_decode(const void *x, int x_dtype, const float *A,
+               const void *B, const void *C, int bc_dtype,
+               const float *dt, const float *dt_bias, const float *D, const void *z,
+               void *state, int state_dtype, int64_t slot_stride, int32_t P,
+               void *out, const int32_t *state_indices,
+               int32_t batch, int32_t active_batch, int32_t nheads, int32_t ngroups,
+               int32_t dim, int32_t dstate, int dt_softplus, int32_t *err_flags,
+               ssu_stream_t stream);
+
+/*
+ * ssu_prefill -- all T tokens (seq_len > 1) in one launch.
+ * Selective State Update page, mamba_ssm::invokeSelectiveStateUpdatePrefill:
+ * the decode recurrence run over t < L_b = context_lengths[b] (all T when NULL), with
+ * the state held on chip across the tokens.
+ *
+ *   x, z, out [batch, T, H, Dm] x_dtype;  B, C [batch, T, G, N] bc_dtype;
+ *   dt [batch, T, H] fp32; other arguments as in ssu_decode.
+ *   Without the stash: the state after L_b tokens is stored back once (not when L_b=0).
+ *   With the replay stash (all four or none; fp32, written for t < L_b only):
+ *     st_dA [batch, T, H]      = exp(A * dt_eff)   (the decay factor)
+ *     st_U  [batch, T, H, Dm]  = x (unscaled, widened)
+ *     st_B  [batch, T, G, N]   = B (widened)
+ *     st_dt [batch, T, H]      = dt_eff
+ *   and the committed state is only read, never written.
+ *   Positions t >= L_b of out and of the stash are not written. A padding row writes
+ *   zeros to out at every t < T and touches nothing else.
+ */
+int ssu_prefill(const void *x, int x_dtype, const float *A,
+                const void *B, const void *C, int bc_dtype,
+                const float *dt, const float *dt_bias, const float *D, const void *z,
+                void *state, int state_dtype, int64_t slot_stride, int32_t P,
+                void *out, const int32_t *state_indices, const int32_t *context_lengths,
+                float *st_dA, float *st_U, float *st_B, float *st_dt,
+                int32_t batch, int32_t active_batch, int32_t T, int32_t nheads,
+                int32_t ngroups, int32_t dim, int32_t dstate, int dt_softplus,
+                int32_t *err_flags, ssu_stream_t stream);
+
+/*
+ * ssu_replay -- re-apply accepted speculative tokens to the committed state.
+ * Selective State Update page, struct MambaReplayLayerInfo and
+ * invokeMambaReplayReconstructBatched: for t < k_b = accepted_lengths[b],
+ *     state = state * st_dA[b,t,h] + st_B[b,t,g,n] * st_dt[b,t,h] * st_U[b,t,h,d]
+ * in place; the state is written once, and not at all when k_b == 0.
+ *   stash buffers as written by ssu_prefill, with T their token extent;
+ *   accepted_lengths [batch] int32 (required); no output.
+ */
+int ssu_replay(void *state, int state_dtype, int64_t slot_stride, int32_t P,
+               const float *st_dA, const float *st_U, const float *st_B,
+               const float *st_dt, const int32_t *accepted_lengths,
+               const int32_t *state_indices, int32_t batch, int32_t active_batch,
+               int32_t T, int32_t nheads, int32_t ngroups, int32_t dim, int32_t dstate,
+               int32_t *err_flags, ssu_stream_t stream);
+
+/*
+ * pool_clear_slot -- zero one slot, or every slot when slot == -1.
+ * Selective State Update page, invokeMambaStateClear; Recurrent State Manager page,
+ * clearSlot / clear. slot_bytes is the slot stride in bytes; other slots are untouched.
+ * Returns SSU_ERR_SHAPE for slot < -1 or slot >= P.
+ */
+int pool_clear_slot(void *pool, int64_t slot_bytes, int32_t P, int32_t slot,
+                    ssu_stream_t stream);
+
+/*
+ * pool_copy_slot -- copy one slot between two pools with the same per-slot geometry
+ * (slot_bytes), which may hold different slot counts.
+ * Recurrent State Manager page, copySlotFrom. The two slot ranges must not overlap
+ * partially (the same slot of the same pool is a no-op copy).
+ * Returns SSU_ERR_SHAPE for a slot outside its pool.
+ */
+int pool_copy_slot(void *dst_pool, int32_t dst_P, int32_t dst_slot,
+                   const void *src_pool, int32_t src_P, int32_t src_slot,
+                   int64_t slot_bytes, ssu_stream_t stream);
+
+/* A constant string naming an ssu_status value. */
+const char *ssu_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSU_H */

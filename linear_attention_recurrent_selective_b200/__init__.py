@@ -1,0 +1,18 @@
+"""B200-native selective state update over a paged recurrent-state pool.
+
+The compute lives in libssu.so (hand-written sm_100a CUDA kernels behind a C ABI,
+include/ssu.h); this package is its thin Python binding plus the seeded synthetic
+workload generator.
+"""
+
+from .ssu import (  # noqa: F401
+    ENTRY_POINTS,
+    SSUError,
+    SSULibraryMissing,
+    lib,
+    pool_clear_slot,
+    pool_copy_slot,
+    ssu_decode,
+    ssu_prefill,
+    ssu_replay,
+)

@@ -1,0 +1,238 @@
+// ssu_api.cu -- the extern "C" boundary of libssu: argument checks, then one launch.
+//
+// Every entry point validates its arguments on the host without touching device memory
+// (so it stays legal under CUDA-graph capture), returns an ssu_status error without
+// launching anything when a check fails, and otherwise enqueues exactly one kernel on
+// the caller's stream. Values that live on the device (stateIndices, contextLengths,
+// acceptedLengths) are checked in-kernel, as the padding contract of the FlashInfer page
+// flashinfer.gdn_fused_decode_step requires for graph replay.
+#include "ssu_common.cuh"
+
+namespace {
+
+bool valid_dtype(int d) { return d == SSU_F32 || d == SSU_F16 || d == SSU_BF16; }
+
+int elem_bytes(int d) { return d == SSU_F32 ? 4 : 2; }
+
+bool supported_dstate(int n)
+{
+    return n == 8 || n == 16 || n == 32 || n == 64 || n == 128 || n == 256;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Sizes and dtypes only (no pointer is looked at), so that an empty batch, whose tensors
+// may carry NULL data pointers, can be accepted before the pointer checks.
+int check_sizes(int state_dtype, int64_t slot_stride, int32_t P, const int32_t *idx,
+                int32_t batch, int32_t active, int32_t H, int32_t G, int32_t Dm, int32_t N)
+{
+    if (!valid_dtype(state_dtype))
+        return SSU_ERR_DTYPE;
+    if (batch < 0 || active < 0 || active > batch || P < 0)
+        return SSU_ERR_SHAPE;
+    if (H <= 0 || G <= 0 || Dm <= 0 || N <= 0 || H % G != 0)
+        return SSU_ERR_SHAPE;
+    if (slot_stride < (int64_t)H * Dm * N)
+        return SSU_ERR_SHAPE;
+    if (!idx && active > P)               // row b is slot b: every active row needs one
+        return SSU_ERR_SHAPE;
+    if (!supported_dstate(N))
+        return SSU_ERR_UNSUPPORTED;
+    return SSU_OK;
+}
+
+int check_pool_alignment(const void *state, int state_dtype, int64_t slot_stride)
+{
+    if (!aligned16(state) || (slot_stride * elem_bytes(state_dtype)) % 16 != 0)
+        return SSU_ERR_ALIGN;
+    return SSU_OK;
+}
+
+int finish(int rc)
+{
+    if (rc != SSU_OK)
+        return rc;
+    return cudaGetLastError() == cudaSuccess ? SSU_OK : SSU_ERR_CUDA;
+}
+
+ssu::DecodeArgs pack_decode(const void *x, int x_dtype, const float *A, const void *B,
+                            const void *C, int bc_dtype, const float *dt,
+                            const float *dt_bias, const float *D, const void *z,
+                            void *state, int64_t slot_stride, int32_t P, void *out,
+                            const int32_t *idx, int32_t batch, int32_t active, int32_t H,
+                            int32_t G, int32_t Dm, int32_t N, int softplus, int32_t *err)
+{
+    ssu::DecodeArgs a;
+    a.x = x;
+    a.A = A;
+    a.B = B;
+    a.C = C;
+    a.dt = dt;
+    a.dt_bias = dt_bias;
+    a.D = D;
+    a.z = z;
+    a.state = state;
+    a.out = out;
+    a.idx = idx;
+    a.err = err;
+    a.slot_stride = slot_stride;
+    a.P = P;
+    a.batch = batch;
+    a.active = active;
+    a.H = H;
+    a.G = G;
+    a.Dm = Dm;
+    a.N = N;
+    a.x_dtype = x_dtype;
+    a.bc_dtype = bc_dtype;
+    a.softplus = softplus ? 1 : 0;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssu_decode(const void *x, int x_dtype, const float *A, const void *B, const void *C,
+               int bc_dtype, const float *dt, const float *dt_bias, const float *D,
+               const void *z, void *state, int state_dtype, int64_t slot_stride, int32_t P,
+               void *out, const int32_t *state_indices, int32_t batch,
+               int32_t active_batch, int32_t nheads, int32_t ngroups, int32_t dim,
+               int32_t dstate, int dt_softplus, int32_t *err_flags, ssu_stream_t stream)
+{
+    if (!valid_dtype(x_dtype) || !valid_dtype(bc_dtype))
+        return SSU_ERR_DTYPE;
+    int rc = check_sizes(state_dtype, slot_stride, P, state_indices, batch, active_batch,
+                         nheads, ngroups, dim, dstate);
+    if (rc != SSU_OK || active_batch == 0)
+        return rc;
+    if (!x || !A || !B || !C || !dt || !state || !out)
+        return SSU_ERR_NULL;
+    if ((rc = check_pool_alignment(state, state_dtype, slot_stride)) != SSU_OK)
+        return rc;
+    ssu::DecodeArgs a = pack_decode(x, x_dtype, A, B, C, bc_dtype, dt, dt_bias, D, z, state,
+                                    slot_stride, P, out, state_indices, batch, active_batch,
+                                    nheads, ngroups, dim, dstate, dt_softplus, err_flags);
+    return finish(ssu::launch_decode(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int ssu_prefill(const void *x, int x_dtype, const float *A, const void *B, const void *C,
+                int bc_dtype, const float *dt, const float *dt_bias, const float *D,
+                const void *z, void *state, int state_dtype, int64_t slot_stride, int32_t P,
+                void *out, const int32_t *state_indices, const int32_t *context_lengths,
+                float *st_dA, float *st_U, float *st_B, float *st_dt, int32_t batch,
+                int32_t active_batch, int32_t T, int32_t nheads, int32_t ngroups,
+                int32_t dim, int32_t dstate, int dt_softplus, int32_t *err_flags,
+                ssu_stream_t stream)
+{
+    if (!valid_dtype(x_dtype) || !valid_dtype(bc_dtype))
+        return SSU_ERR_DTYPE;
+    if (T < 0)
+        return SSU_ERR_SHAPE;
+    int rc = check_sizes(state_dtype, slot_stride, P, state_indices, batch, active_batch,
+                         nheads, ngroups, dim, dstate);
+    if (rc != SSU_OK || active_batch == 0 || T == 0)
+        return rc;
+    if (!x || !A || !B || !C || !dt || !state || !out)
+        return SSU_ERR_NULL;
+    const int given = (st_dA != nullptr) + (st_U != nullptr) + (st_B != nullptr) +
+                      (st_dt != nullptr);
+    if (given != 0 && given != 4)
+        return SSU_ERR_NULL;
+    if ((rc = check_pool_alignment(state, state_dtype, slot_stride)) != SSU_OK)
+        return rc;
+    ssu::PrefillArgs a;
+    a.d = pack_decode(x, x_dtype, A, B, C, bc_dtype, dt, dt_bias, D, z, state, slot_stride,
+                      P, out, state_indices, batch, active_batch, nheads, ngroups, dim,
+                      dstate, dt_softplus, err_flags);
+    a.ctx = context_lengths;
+    a.st_dA = st_dA;
+    a.st_U = st_U;
+    a.st_B = st_B;
+    a.st_dt = st_dt;
+    a.T = T;
+    return finish(ssu::launch_prefill(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int ssu_replay(void *state, int state_dtype, int64_t slot_stride, int32_t P,
+               const float *st_dA, const float *st_U, const float *st_B, const float *st_dt,
+               const int32_t *accepted_lengths, const int32_t *state_indices,
+               int32_t batch, int32_t active_batch, int32_t T, int32_t nheads,
+               int32_t ngroups, int32_t dim, int32_t dstate, int32_t *err_flags,
+               ssu_stream_t stream)
+{
+    if (T < 0)
+        return SSU_ERR_SHAPE;
+    int rc = check_sizes(state_dtype, slot_stride, P, state_indices, batch, active_batch,
+                         nheads, ngroups, dim, dstate);
+    if (rc != SSU_OK || active_batch == 0 || T == 0)
+        return rc;
+    if (!state || !st_dA || !st_U || !st_B || !st_dt || !accepted_lengths)
+        return SSU_ERR_NULL;
+    if ((rc = check_pool_alignment(state, state_dtype, slot_stride)) != SSU_OK)
+        return rc;
+    if (!aligned16(st_B))
+        return SSU_ERR_ALIGN;
+    ssu::ReplayArgs a;
+    a.state = state;
+    a.st_dA = st_dA;
+    a.st_U = st_U;
+    a.st_B = st_B;
+    a.st_dt = st_dt;
+    a.acc = accepted_lengths;
+    a.idx = state_indices;
+    a.err = err_flags;
+    a.slot_stride = slot_stride;
+    a.P = P;
+    a.batch = batch;
+    a.active = active_batch;
+    a.T = T;
+    a.H = nheads;
+    a.G = ngroups;
+    a.Dm = dim;
+    a.N = dstate;
+    return finish(ssu::launch_replay(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int pool_clear_slot(void *pool, int64_t slot_bytes, int32_t P, int32_t slot,
+                    ssu_stream_t stream)
+{
+    if (!pool)
+        return SSU_ERR_NULL;
+    if (slot_bytes < 0 || P < 0 || slot < -1 || slot >= P)
+        return SSU_ERR_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (slot == -1)
+        return finish(ssu::launch_clear(pool, slot_bytes * P, s));
+    return finish(ssu::launch_clear(static_cast<uint8_t *>(pool) + slot * slot_bytes,
+                                    slot_bytes, s));
+}
+
+int pool_copy_slot(void *dst_pool, int32_t dst_P, int32_t dst_slot, const void *src_pool,
+                   int32_t src_P, int32_t src_slot, int64_t slot_bytes, ssu_stream_t stream)
+{
+    if (!dst_pool || !src_pool)
+        return SSU_ERR_NULL;
+    if (slot_bytes < 0 || dst_slot < 0 || dst_slot >= dst_P || src_slot < 0 ||
+        src_slot >= src_P)
+        return SSU_ERR_SHAPE;
+    return finish(ssu::launch_copy(static_cast<uint8_t *>(dst_pool) + dst_slot * slot_bytes,
+                                   static_cast<const uint8_t *>(src_pool) + src_slot * slot_bytes,
+                                   slot_bytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+const char *ssu_status_string(int status)
+{
+    switch (status) {
+    case SSU_OK: return "SSU_OK";
+    case SSU_ERR_NULL: return "SSU_ERR_NULL: a required pointer is NULL or the stash is partial";
+    case SSU_ERR_SHAPE: return "SSU_ERR_SHAPE: inconsistent sizes";
+    case SSU_ERR_DTYPE: return "SSU_ERR_DTYPE: unknown dtype code";
+    case SSU_ERR_UNSUPPORTED: return "SSU_ERR_UNSUPPORTED: dstate not in {8,16,32,64,128,256}";
+    case SSU_ERR_CUDA: return "SSU_ERR_CUDA: kernel launch failed";
+    case SSU_ERR_ALIGN: return "SSU_ERR_ALIGN: pool or slot stride not 16-byte aligned";
+    default: return "unknown ssu_status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,199 @@
+// ssu_common.cuh -- shared device helpers and launch descriptors for libssu (sm_100a).
+//
+// Storage types follow the Selective State Update page of the TensorRT-Edge-LLM C++ API:
+// the state pool is half or float, A/dt/D/dt_bias are fp32, and x/B/C/z/out may be fp32,
+// fp16 or bf16. Every value is widened to fp32 for arithmetic and rounded to nearest
+// even once when stored.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssu.h"
+
+namespace ssu {
+
+// ---------------------------------------------------------------- launch descriptors
+
+struct DecodeArgs {
+    const void *x;
+    const float *A;
+    const void *B;
+    const void *C;
+    const float *dt;
+    const float *dt_bias;
+    const float *D;
+    const void *z;
+    void *state;
+    void *out;
+    const int32_t *idx;
+    int32_t *err;
+    int64_t slot_stride;
+    int32_t P, batch, active, H, G, Dm, N;
+    int x_dtype, bc_dtype, softplus;
+};
+
+struct PrefillArgs {
+    DecodeArgs d;             // x/B/C/dt/z/out carry a token axis [batch, T, ...]
+    const int32_t *ctx;       // contextLengths [batch] or NULL
+    float *st_dA, *st_U, *st_B, *st_dt;  // replay stash, all or none
+    int32_t T;
+};
+
+struct ReplayArgs {
+    void *state;
+    const float *st_dA, *st_U, *st_B, *st_dt;
+    const int32_t *acc;
+    const int32_t *idx;
+    int32_t *err;
+    int64_t slot_stride;
+    int32_t P, batch, active, T, H, G, Dm, N;
+};
+
+// Host launchers, one per kernel family; each returns SSU_OK or SSU_ERR_UNSUPPORTED.
+int launch_decode(const DecodeArgs &a, int state_dtype, cudaStream_t s);
+int launch_prefill(const PrefillArgs &a, int state_dtype, cudaStream_t s);
+int launch_replay(const ReplayArgs &a, int state_dtype, cudaStream_t s);
+int launch_clear(void *pool, int64_t bytes, cudaStream_t s);
+int launch_copy(void *dst, const void *src, int64_t bytes, cudaStream_t s);
+
+// ---------------------------------------------------------------- scalar access
+
+__device__ __forceinline__ float ld_f32(const void *p, int dtype, int64_t i)
+{
+    if (dtype == SSU_BF16)
+        return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+    if (dtype == SSU_F16)
+        return __half2float(static_cast<const __half *>(p)[i]);
+    return static_cast<const float *>(p)[i];
+}
+
+__device__ __forceinline__ void st_f32(void *p, int dtype, int64_t i, float v)
+{
+    if (dtype == SSU_BF16)
+        static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(v);
+    else if (dtype == SSU_F16)
+        static_cast<__half *>(p)[i] = __float2half_rn(v);
+    else
+        static_cast<float *>(p)[i] = v;
+}
+
+// softplus(v) = log(1 + e^v); above 20 the correction log1p(e^-v) < 2.1e-9 is dropped.
+__device__ __forceinline__ float softplus_f(float v)
+{
+    return v > 20.f ? v : log1pf(expf(v));
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.f + expf(-z)); }
+
+// dt after the optional bias and the optional softplus (one value per row, token, head)
+__device__ __forceinline__ float effective_dt(float dt, const float *bias, int h, int sp)
+{
+    float v = dt + (bias ? bias[h] : 0.f);
+    return sp ? softplus_f(v) : v;
+}
+
+// ---------------------------------------------------------------- 16-byte state vectors
+
+template <typename S> struct Vec16;
+
+template <> struct Vec16<float> {
+    static constexpr int kElems = 4;
+    static __device__ __forceinline__ void unpack(const uint4 &v, float *f)
+    {
+        f[0] = __uint_as_float(v.x);
+        f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z);
+        f[3] = __uint_as_float(v.w);
+    }
+    static __device__ __forceinline__ uint4 pack(const float *f)
+    {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]),
+                          __float_as_uint(f[2]), __float_as_uint(f[3]));
+    }
+};
+
+template <typename H2, typename Cvt> struct Vec16Half {
+    static constexpr int kElems = 8;
+    static __device__ __forceinline__ void unpack(const uint4 &v, float *f)
+    {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            H2 h;
+            memcpy(&h, &w[i], 4);
+            float2 p = Cvt::to_f2(h);
+            f[2 * i] = p.x;
+            f[2 * i + 1] = p.y;
+        }
+    }
+    static __device__ __forceinline__ uint4 pack(const float *f)
+    {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            H2 h = Cvt::from_f2(f[2 * i], f[2 * i + 1]);
+            memcpy(&w[i], &h, 4);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+struct CvtHalf {
+    static __device__ __forceinline__ float2 to_f2(__half2 h) { return __half22float2(h); }
+    static __device__ __forceinline__ __half2 from_f2(float a, float b)
+    {
+        return __floats2half2_rn(a, b);
+    }
+};
+struct CvtBf16 {
+    static __device__ __forceinline__ float2 to_f2(__nv_bfloat162 h)
+    {
+        return __bfloat1622float2(h);
+    }
+    static __device__ __forceinline__ __nv_bfloat162 from_f2(float a, float b)
+    {
+        return __floats2bfloat162_rn(a, b);
+    }
+};
+
+template <> struct Vec16<__half> : Vec16Half<__half2, CvtHalf> {};
+template <> struct Vec16<__nv_bfloat16> : Vec16Half<__nv_bfloat162, CvtBf16> {};
+
+// Four consecutive state elements as floats (8- or 16-byte access).
+template <typename S> struct Quad;
+template <> struct Quad<float> {
+    static __device__ __forceinline__ float4 load(const float *p)
+    {
+        return *reinterpret_cast<const float4 *>(p);
+    }
+    static __device__ __forceinline__ void store(float *p, float4 v)
+    {
+        *reinterpret_cast<float4 *>(p) = v;
+    }
+};
+template <typename S, typename H2, typename Cvt> struct QuadHalf {
+    static __device__ __forceinline__ float4 load(const S *p)
+    {
+        uint2 w = *reinterpret_cast<const uint2 *>(p);
+        H2 a, b;
+        memcpy(&a, &w.x, 4);
+        memcpy(&b, &w.y, 4);
+        float2 fa = Cvt::to_f2(a), fb = Cvt::to_f2(b);
+        return make_float4(fa.x, fa.y, fb.x, fb.y);
+    }
+    static __device__ __forceinline__ void store(S *p, float4 v)
+    {
+        H2 a = Cvt::from_f2(v.x, v.y), b = Cvt::from_f2(v.z, v.w);
+        uint2 w;
+        memcpy(&w.x, &a, 4);
+        memcpy(&w.y, &b, 4);
+        *reinterpret_cast<uint2 *>(p) = w;
+    }
+};
+template <> struct Quad<__half> : QuadHalf<__half, __half2, CvtHalf> {};
+template <> struct Quad<__nv_bfloat16> : QuadHalf<__nv_bfloat16, __nv_bfloat162, CvtBf16> {};
+
+}  // namespace ssu

@@ -1,0 +1,60 @@
+"""Run a workloads.SSUCase through the CUDA library (via the C-ABI binding) and return
+host copies of what it wrote. Outputs and stash buffers start as NaN so that positions
+the kernels must not write stay recognisable."""
+
+import torch
+
+from linear_attention_recurrent_selective_b200 import ssu
+
+NAN = float("nan")
+
+
+def dev(case):
+    return case.to("cuda")
+
+
+def decode(case, pool=None, err=True, out=None, stream=None):
+    d = dev(case)
+    pool = d.pool.clone() if pool is None else pool
+    out = torch.full_like(d.x, NAN) if out is None else out
+    e = torch.zeros(1, dtype=torch.int32, device="cuda") if err else None
+    ssu.ssu_decode(d.x, d.A, d.B, d.C, d.dt, pool, out, dt_bias=d.dt_bias, D=d.D, z=d.z,
+                   state_indices=d.state_indices, active_batch=case.active,
+                   dt_softplus=case.dt_softplus, err_flags=e, slot_stride=case.slot_stride,
+                   P=case.P, stream=stream)
+    torch.cuda.synchronize()
+    return out.cpu(), pool.cpu(), (int(e.item()) if err else None)
+
+
+def new_stash(case, fill=NAN):
+    b, T, H, G, Dm, N = case.batch, case.T, case.H, case.G, case.Dm, case.N
+    f = dict(dtype=torch.float32, device="cuda")
+    return (torch.full((b, T, H), fill, **f), torch.full((b, T, H, Dm), fill, **f),
+            torch.full((b, T, G, N), fill, **f), torch.full((b, T, H), fill, **f))
+
+
+def prefill(case, pool=None, stash=False, err=True):
+    d = dev(case)
+    pool = d.pool.clone() if pool is None else pool
+    out = torch.full_like(d.x, NAN)
+    st = new_stash(case) if stash else None
+    e = torch.zeros(1, dtype=torch.int32, device="cuda") if err else None
+    ssu.ssu_prefill(d.x, d.A, d.B, d.C, d.dt, pool, out, dt_bias=d.dt_bias, D=d.D, z=d.z,
+                    state_indices=d.state_indices, context_lengths=d.context_lengths,
+                    stash=st, active_batch=case.active, dt_softplus=case.dt_softplus,
+                    err_flags=e, slot_stride=case.slot_stride, P=case.P)
+    torch.cuda.synchronize()
+    st_cpu = tuple(t.cpu() for t in st) if st is not None else None
+    return out.cpu(), pool.cpu(), st_cpu, (int(e.item()) if err else None)
+
+
+def replay(case, stash, accepted, pool=None, err=True):
+    d = dev(case)
+    pool = d.pool.clone() if pool is None else pool
+    st = tuple(t.cuda() for t in stash)
+    e = torch.zeros(1, dtype=torch.int32, device="cuda") if err else None
+    ssu.ssu_replay(pool, st, accepted.cuda(), state_indices=d.state_indices,
+                   active_batch=case.active, err_flags=e, slot_stride=case.slot_stride,
+                   P=case.P)
+    torch.cuda.synchronize()
+    return pool.cpu(), (int(e.item()) if err else None)

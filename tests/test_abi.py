@@ -1,0 +1,94 @@
+"""CPU checks of the C-ABI library: it loads, exports every declared entry point, and
+rejects bad arguments on the host before any CUDA call (no GPU needed for those)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_recurrent_selective_b200 import ssu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssu.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
+
+
+@pytest.fixture(scope="module")
+def L():
+    from linear_attention_recurrent_selective_b200 import build
+    build.build()
+    return ssu.lib()
+
+
+def test_header_declares_the_entry_points():
+    assert declared_functions() == list(ssu.ENTRY_POINTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code in range(7):
+        assert L.ssu_status_string(code).startswith(b"SSU_")
+
+
+# Pointers below are never dereferenced: each call fails validation on the host first.
+P16 = ctypes.c_void_p(256)
+
+
+def decode_args(**kw):
+    a = dict(x=P16, x_dt=2, A=P16, B=P16, C=P16, bc_dt=2, dt=P16, dt_bias=None, D=None,
+             z=None, state=P16, state_dt=0, stride=80 * 64 * 128, P=512, out=P16, idx=P16,
+             batch=256, active=256, H=80, G=1, Dm=64, N=128, sp=1, err=None, stream=None)
+    a.update(kw)
+    return list(a.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), 1), (dict(state=None), 1), (dict(out=None), 1),
+    (dict(x_dt=7), 3), (dict(state_dt=-1), 3),
+    (dict(active=300), 2), (dict(active=-1), 2), (dict(G=3), 2),
+    (dict(stride=100), 2), (dict(idx=None, P=16), 2),
+    (dict(N=48, stride=80 * 64 * 48), 4),
+    (dict(state=ctypes.c_void_p(264)), 6),
+    (dict(stride=80 * 64 * 128 + 1), 6),
+])
+def test_decode_rejects_bad_arguments(L, kw, status):
+    assert L.ssu_decode(*decode_args(**kw)) == status
+
+
+def test_prefill_rejects_partial_stash(L):
+    args = [P16, 2, P16, P16, P16, 2, P16, None, None, None, P16, 0, 80 * 64 * 128, 32, P16,
+            None, None, P16, None, P16, P16, 16, 16, 512, 80, 1, 64, 128, 1, None, None]
+    assert L.ssu_prefill(*args) == 1
+    args[16] = None
+    args[17:21] = [None] * 4
+    args[22] = -1      # T < 0
+    assert L.ssu_prefill(*args) == 2
+
+
+def test_replay_and_pool_reject_bad_arguments(L):
+    assert L.ssu_replay(P16, 0, 8192, 8, P16, P16, P16, P16, None, None, 4, 4, 5, 1, 1, 64,
+                        128, None, None) == 1
+    assert L.ssu_replay(P16, 0, 8192, 8, P16, P16, ctypes.c_void_p(260), P16, P16, None, 4,
+                        4, 5, 1, 1, 64, 128, None, None) == 6
+    assert L.pool_clear_slot(P16, 1024, 4, 4, None) == 2
+    assert L.pool_clear_slot(P16, 1024, 4, -2, None) == 2
+    assert L.pool_clear_slot(None, 1024, 4, 0, None) == 1
+    assert L.pool_copy_slot(P16, 4, 4, P16, 8, 0, 1024, None) == 2
+    assert L.pool_copy_slot(P16, 4, 0, P16, 8, -1, 1024, None) == 2
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(ssu, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(ssu, "_lib", None)
+    with pytest.raises(ssu.SSULibraryMissing):
+        ssu.lib()

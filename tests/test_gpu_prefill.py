@@ -1,0 +1,123 @@
+"""GPU parity of ssu_prefill (multi-token scan, optional replay stash) against the oracle.
+
+Selective State Update page (TensorRT-Edge-LLM C++ API),
+invokeSelectiveStateUpdatePrefill."""
+
+import dataclasses
+
+import pytest
+import torch
+
+import gpu_run
+from linear_attention_recurrent_selective_b200 import ssu
+from linear_attention_recurrent_selective_b200.workloads import make_case, make_config
+from parity import changed_slots, check_fp32, check_out, check_state, same_bits
+
+pytestmark = pytest.mark.gpu
+
+F32, F16, BF16 = torch.float32, torch.float16, torch.bfloat16
+
+
+def compare_prefill(orc, case, stash):
+    out_o, pool_o, st_o, err_o = orc.prefill_case(case, stash=stash)
+    out_g, pool_g, st_g, err_g = gpu_run.prefill(case, stash=stash)
+    assert err_g == err_o
+    check_out(out_g, out_o, case.x_dtype)
+    check_state(pool_g, pool_o, case.state_dtype)
+    assert changed_slots(case.pool, pool_g, case) == changed_slots(case.pool, pool_o, case)
+    if stash:
+        assert same_bits(pool_g, case.pool)          # committed state read only
+        dA_g, U_g, B_g, dt_g = st_g
+        dA_o, U_o, B_o, dt_o = st_o
+        assert same_bits(U_g, U_o) and same_bits(B_g, B_o)   # exact widening, same spots
+        check_fp32(dA_g, dA_o)
+        check_fp32(dt_g, dt_o)
+    return out_g, pool_g, st_g
+
+
+SHAPES = [
+    # (N, state dtype, Dm, H, G, T, x dtype)
+    (8, F32, 9, 4, 2, 20, F32),
+    (16, F16, 16, 2, 1, 17, F16),
+    (32, BF16, 33, 4, 4, 5, BF16),
+    (64, F32, 70, 3, 1, 40, BF16),
+    (128, F32, 64, 4, 1, 33, BF16),
+    (128, F16, 40, 4, 2, 16, F16),
+    (256, F32, 36, 2, 1, 18, F32),
+]
+
+
+@pytest.mark.parametrize("N,sdt,Dm,H,G,T,xdt", SHAPES)
+@pytest.mark.parametrize("stash", [False, True])
+def test_prefill_shapes(orc, N, sdt, Dm, H, G, T, xdt, stash):
+    case = make_case(seed=200 + N + T, batch=5, P=9, T=T, H=H, G=G, Dm=Dm, N=N, x_dtype=xdt,
+                     bc_dtype=xdt, state_dtype=sdt, z=True, active=4, n_pad=1,
+                     lengths="context", slot_pad=4 if sdt == F32 else 8)
+    case.context_lengths[0] = T
+    compare_prefill(orc, case, stash)
+
+
+def test_prefill_without_lengths_or_options(orc):
+    case = make_case(seed=210, batch=3, P=3, T=24, H=4, G=2, Dm=20, N=64, indices="none",
+                     z=False, dt_bias=False, D=False, dt_softplus=False)
+    case.dt = case.dt.abs()          # without softplus the caller passes a positive step
+    compare_prefill(orc, case, stash=False)
+
+
+def test_prefill_length_edge_cases(orc):
+    case = make_case(seed=211, batch=5, P=8, T=6, H=2, G=1, Dm=16, N=32, z=True,
+                     lengths="context")
+    case.context_lengths = torch.tensor([0, 6, 9, -3, 1], dtype=torch.int32)
+    out_o, pool_o, _, err_o = orc.prefill_case(case)
+    out_g, pool_g, _, err_g = gpu_run.prefill(case)
+    assert err_g == err_o == ssu.FLAG_CONTEXT_RANGE | ssu.FLAG_NEGATIVE_LENGTH
+    check_out(out_g, out_o, case.x_dtype)
+    check_state(pool_g, pool_o, case.state_dtype)
+    assert torch.isnan(out_g[0].float()).all() and torch.isnan(out_g[3].float()).all()
+
+
+def test_prefill_b16_t512_sampled_rows(orc):
+    """Full-size multi-token prefill on the GPU (the benchmarked launch); the oracle
+    recomputes three rows (the longest, the shortest and one more) one by one."""
+    case = make_config("prefill_b16_t512")
+    out_g, pool_g, st_g, _ = gpu_run.prefill(case, stash=True)
+    out_n, pool_n, _, _ = gpu_run.prefill(case, stash=False)
+    assert same_bits(out_g, out_n)                  # stash changes nothing in the outputs
+    assert same_bits(pool_g, case.pool)
+    L = case.context_lengths
+    rows = sorted({int(L.argmax()), int(L.argmin()), 5})
+    for b in rows:
+        rows_of = {f: getattr(case, f)[b: b + 1].contiguous()
+                   for f in ("x", "B", "C", "dt", "z", "state_indices", "context_lengths")}
+        sub = dataclasses.replace(case, batch=1, active=1, **rows_of)
+        out_o, pool_o, st_o, _ = orc.prefill_case(sub, stash=True)
+        check_out(out_g[b: b + 1], out_o, case.x_dtype)
+        assert same_bits(st_g[1][b: b + 1], st_o[1]) and same_bits(st_g[2][b: b + 1], st_o[2])
+        check_fp32(st_g[0][b: b + 1], st_o[0])
+        _, pool_o, _, _ = orc.prefill_case(sub, stash=False)
+        s = int(case.state_indices[b])
+        sl = slice(s * case.slot_stride, (s + 1) * case.slot_stride)
+        check_state(pool_n[sl], pool_o[sl], case.state_dtype)
+    touched = {int(case.state_indices[b]) for b in range(case.batch)}
+    assert changed_slots(case.pool, pool_n, case) == touched
+
+
+def test_T_decodes_equal_one_prefill_on_gpu():
+    """GPU against GPU: T decode steps leave the same fp32 state as one T-token prefill
+    (bit for bit: same per-element arithmetic), and the same outputs up to the order of
+    the dstate reduction."""
+    case = make_case(seed=212, batch=4, P=8, T=7, H=4, G=2, Dm=64, N=128, x_dtype=BF16,
+                     bc_dtype=BF16, z=True, slow_decay=True)
+    out_p, pool_p, _, _ = gpu_run.prefill(case)
+    d = case.to("cuda")
+    pool = d.pool.clone()
+    for t in range(case.T):
+        out = torch.empty(d.x[:, t].shape, dtype=d.x.dtype, device="cuda")
+        ssu.ssu_decode(d.x[:, t].contiguous(), d.A, d.B[:, t].contiguous(),
+                       d.C[:, t].contiguous(), d.dt[:, t].contiguous(), pool, out,
+                       dt_bias=d.dt_bias, D=d.D, z=d.z[:, t].contiguous(),
+                       state_indices=d.state_indices, slot_stride=case.slot_stride, P=case.P)
+        o = out_p[:, t].double()
+        assert ((out.cpu().double() - o).abs() <= (2.0 ** -7) * o.abs() + 1e-5).all()
+    torch.cuda.synchronize()
+    assert same_bits(pool.cpu(), pool_p)
