@@ -37,7 +37,8 @@
  *    undefined. Here it never causes an out-of-bounds access: the row is skipped (index)
  *    or the length clamped, and a bit is OR-ed into the optional device int32 err_flags:
  *    SSU_FLAG_INDEX_RANGE, SSU_FLAG_ACCEPTED_RANGE, SSU_FLAG_CONTEXT_RANGE,
- *    SSU_FLAG_NEGATIVE_LENGTH.
+ *    SSU_FLAG_NEGATIVE_LENGTH. Kernels that wait on their own asynchronous copies bound
+ *    every wait and report SSU_FLAG_TIMEOUT instead of hanging.
  *  - Return value: SSU_OK, or an ssu_status error, in which case nothing was launched
  *    (SSU_ERR_CUDA: the launch itself failed). Sizes and dtype codes are checked first;
  *    a call with nothing to do (active_batch == 0, or T == 0) then returns SSU_OK without
@@ -66,14 +67,18 @@ typedef enum {
     SSU_ERR_DTYPE = 3,        /* dtype code not one of ssu_dtype */
     SSU_ERR_UNSUPPORTED = 4,  /* dstate not in {8,16,32,64,128,256} */
     SSU_ERR_CUDA = 5,         /* the kernel launch failed */
-    SSU_ERR_ALIGN = 6         /* pool pointer or slot stride not 16-byte aligned */
+    SSU_ERR_ALIGN = 6         /* pool pointer or slot stride not 16-byte aligned, or (in
+                                 ssu_prefill / ssu_replay) B, C or the stash B not 16-byte
+                                 aligned */
 } ssu_status;
 
 enum {
     SSU_FLAG_INDEX_RANGE = 1,     /* state_indices[b] >= P: row skipped */
     SSU_FLAG_ACCEPTED_RANGE = 2,  /* accepted_lengths[b] > T: clamped to T */
     SSU_FLAG_CONTEXT_RANGE = 4,   /* context_lengths[b] > T: clamped to T */
-    SSU_FLAG_NEGATIVE_LENGTH = 8  /* a negative length: treated as 0 */
+    SSU_FLAG_NEGATIVE_LENGTH = 8, /* a negative length: treated as 0 */
+    SSU_FLAG_TIMEOUT = 16         /* an internal wait gave up after 2 s (never expected);
+                                     the outputs of that launch are incomplete */
 };
 
 /*

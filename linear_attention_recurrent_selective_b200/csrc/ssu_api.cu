@@ -141,6 +141,8 @@ int ssu_prefill(const void *x, int x_dtype, const float *A, const void *B, const
         return SSU_ERR_NULL;
     if ((rc = check_pool_alignment(state, state_dtype, slot_stride)) != SSU_OK)
         return rc;
+    if (!aligned16(B) || !aligned16(C) || (st_B && !aligned16(st_B)))
+        return SSU_ERR_ALIGN;
     ssu::PrefillArgs a;
     a.d = pack_decode(x, x_dtype, A, B, C, bc_dtype, dt, dt_bias, D, z, state, slot_stride,
                       P, out, state_indices, batch, active_batch, nheads, ngroups, dim,

@@ -10,169 +10,184 @@
 // CUDA-graph replay.
 //
 // The step is a pure stream over the state pool: every state element is read once and
-// written once (8 FLOP per 4 bytes of fp32 state), so the kernel is HBM-bound. Design:
-//   * one CTA (8 warps) per (row b, head h, dim tile); consecutive CTAs walk the heads of
-//     one slot, i.e. contiguous memory;
-//   * a row of N state elements is covered by LPR lanes with 16-byte accesses, so each
-//     warp instruction moves 512 contiguous bytes; each thread keeps RPT rows in flight
-//     (all loads are issued before any arithmetic) to hold enough bytes in flight per SM;
-//   * B and C for the lane's state columns and the per-(b,h) decay live in registers;
-//     the input term is formed as B * (dt * x), the association the prefill and replay
-//     kernels use too, so fp32 states agree bit for bit across the three forms;
-//   * the dstate reduction is a butterfly of warp shuffles inside each lane group;
-//   * the new state is stored back to the same addresses with 16-byte stores.
-#include "ssu_common.cuh"
+// written once (5 FLOP per 8 bytes of fp32 traffic), so the kernel is bound by HBM. It
+// runs on the per-warp bulk-copy pipeline of ssu_stream.cuh and keeps every dependent
+// load off the per-tile path:
+//   * the per-unit scalars (dt_eff, exp(A dt_eff), D), the lane's B and C columns and the
+//     unit's x and z are loaded once per unit, at addresses that do not depend on the
+//     slot index, before the unit's first tile is waited for;
+//   * a tile is read with conflict-free 16-byte shared loads, updated in registers and
+//     written straight back to the pool with coalesced 16-byte global stores (each warp
+//     instruction covers 512 contiguous bytes); the input term is formed as B * (dt * x),
+//     the association the prefill and replay kernels use too, so fp32 states agree bit
+//     for bit across the three forms;
+//   * the dstate reduction is a butterfly of warp shuffles inside each lane group; the
+//     per-row sums are collected in shared memory and the unit's outputs (skip term and
+//     gate applied) are written with one coalesced store per 32 rows.
+#include "ssu_stream.cuh"
 
 namespace ssu {
 namespace {
 
-constexpr int kDecodeWarps = 8;
+using namespace stream;
 
-template <typename S, int N, int RPT>
-__global__ void __launch_bounds__(kDecodeWarps * 32)
-ssu_decode_kernel(const DecodeArgs a)
-{
-    using V = Vec16<S>;
-    constexpr int VEC = V::kElems;                       // state elements per 16 bytes
-    constexpr int LPR = (N / VEC) < 32 ? (N / VEC) : 32;  // lanes per state row
-    constexpr int E = N / LPR;                           // elements per lane and row
-    constexpr int NV = E / VEC;                          // 16-byte vectors per lane and row
-    constexpr int RPW = 32 / LPR;                        // rows per warp instruction
-    constexpr int RPP = kDecodeWarps * RPW;              // rows per CTA pass
-    constexpr int RT = RPP * RPT;                        // rows per CTA (dim tile)
-
-    const int H = a.H, Dm = a.Dm;
-    const int dtiles = (Dm + RT - 1) / RT;
-    int unit = blockIdx.x;
-    const int dtile = unit % dtiles;
-    unit /= dtiles;
-    const int h = unit % H;
-    const int b = unit / H;
-
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int ln = lane % LPR;
-    const int rbase = dtile * RT + warp * RPW + lane / LPR;
-    const int64_t xrow = ((int64_t)b * H + h) * Dm;
-
-    const int slot = a.idx ? a.idx[b] : b;
-    if (slot < 0) {                       // padding row: output zero, state untouched
-        if (ln == 0) {
-#pragma unroll
-            for (int i = 0; i < RPT; ++i) {
-                const int r = rbase + i * RPP;
-                if (r < Dm)
-                    st_f32(a.out, a.x_dtype, xrow + r, 0.f);
-            }
-        }
-        return;
+struct DecodeRows {
+    const int32_t *idx;
+    int32_t P;
+    __device__ __forceinline__ int2 resolve(int b) const
+    {
+        return make_int2(idx ? idx[b] : b, 0);
     }
-    if (slot >= a.P) {                    // caller bug: skip the row and report it
-        if (threadIdx.x == 0 && dtile == 0 && h == 0 && a.err)
-            atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
-        return;
-    }
+    __device__ __forceinline__ bool moves(int2 r) const { return r.x >= 0 && r.x < P; }
+};
 
-    // ---- issue every state load of this thread first
-    S *base = static_cast<S *>(a.state) + (int64_t)slot * a.slot_stride + (int64_t)h * Dm * N;
-    uint4 raw[RPT][NV];
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int r = rbase + i * RPP;
-        const uint4 *rp = reinterpret_cast<const uint4 *>(base + (int64_t)r * N);
-#pragma unroll
-        for (int v = 0; v < NV; ++v)
-            raw[i][v] = r < Dm ? rp[v * LPR + ln] : make_uint4(0, 0, 0, 0);
-    }
-
-    // ---- per-(b, h) scalars and the lane's columns of B and C
-    const int g = h / (H / a.G);
-    const float dte = effective_dt(a.dt[(int64_t)b * H + h], a.dt_bias, h, a.softplus);
-    const float dA = expf(a.A[h] * dte);
-    const float Dh = a.D ? a.D[h] : 0.f;
-    const int64_t bc = ((int64_t)b * a.G + g) * N;
-    float Bn[E], Cn[E];
-#pragma unroll
-    for (int v = 0; v < NV; ++v)
-#pragma unroll
-        for (int k = 0; k < VEC; ++k) {
-            const int n = (v * LPR + ln) * VEC + k;
-            Bn[v * VEC + k] = ld_f32(a.B, a.bc_dtype, bc + n);
-            Cn[v * VEC + k] = ld_f32(a.C, a.bc_dtype, bc + n);
-        }
-    float xv[RPT];
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int r = rbase + i * RPP;
-        xv[i] = r < Dm ? ld_f32(a.x, a.x_dtype, xrow + r) : 0.f;
-    }
-
-    // ---- update, reduce, store
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int r = rbase + i * RPP;
-        const float dtx = dte * xv[i];
-        float acc = 0.f;
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            float f[VEC];
-            V::unpack(raw[i][v], f);
-#pragma unroll
-            for (int k = 0; k < VEC; ++k) {
-                const float s = fmaf(f[k], dA, Bn[v * VEC + k] * dtx);
-                f[k] = s;
-                acc = fmaf(s, Cn[v * VEC + k], acc);
-            }
-            raw[i][v] = V::pack(f);
-        }
-#pragma unroll
-        for (int off = LPR / 2; off > 0; off >>= 1)
-            acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (r < Dm) {
-            uint4 *rp = reinterpret_cast<uint4 *>(base + (int64_t)r * N);
-#pragma unroll
-            for (int v = 0; v < NV; ++v)
-                rp[v * LPR + ln] = raw[i][v];
-            if (ln == 0) {
-                float y = acc + Dh * xv[i];
-                if (a.z)
-                    y *= silu_f(ld_f32(a.z, a.x_dtype, xrow + r));
-                st_f32(a.out, a.x_dtype, xrow + r, y);
-            }
-        }
-    }
-}
-
-template <typename S, int N, int RPT>
-int launch_rpt(const DecodeArgs &a, cudaStream_t s)
-{
-    constexpr int VEC = Vec16<S>::kElems;
-    constexpr int LPR = (N / VEC) < 32 ? (N / VEC) : 32;
-    constexpr int RT = kDecodeWarps * (32 / LPR) * RPT;
-    const int64_t dtiles = (a.Dm + RT - 1) / RT;
-    const int64_t grid = (int64_t)a.active * a.H * dtiles;
-    if (grid == 0)
-        return SSU_OK;
-    if (grid > 0x7fffffffLL)
-        return SSU_ERR_SHAPE;
-    ssu_decode_kernel<S, N, RPT><<<(unsigned)grid, kDecodeWarps * 32, 0, s>>>(a);
-    return SSU_OK;
-}
-
-// Rows per thread: as many as the dim extent fills (up to 8), so that small dims do not
-// leave most of the CTA idle and large dims keep 128 bytes in flight per thread.
 template <typename S, int N>
-int launch_n(const DecodeArgs &a, cudaStream_t s)
+__global__ void __launch_bounds__(kWarps * 32)
+ssu_decode_kernel(const DecodeArgs a, const int cph, const int nunits)
 {
-    constexpr int VEC = Vec16<S>::kElems;
-    constexpr int LPR = (N / VEC) < 32 ? (N / VEC) : 32;
-    constexpr int RPP = kDecodeWarps * (32 / LPR);
-    if (a.Dm >= 8 * RPP)
-        return launch_rpt<S, N, 8>(a, s);
-    if (a.Dm >= 4 * RPP)
-        return launch_rpt<S, N, 4>(a, s);
-    if (a.Dm >= 2 * RPP)
-        return launch_rpt<S, N, 2>(a, s);
-    return launch_rpt<S, N, 1>(a, s);
+    using G = Geo<S, N>;
+    using V = Vec16<S>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const WarpViews w = warp_views(smem, warp);
+    float *xs = w.f0;                           // unit x, [CR]
+    float *ys = w.f1;                           // unit row sums, [CR]
+    init_ring(w, lane);
+
+    const int H = a.H, Dm = a.Dm, hpg = H / a.G;
+    const int gw = blockIdx.x * kWarps + warp;
+    const int nw = gridDim.x * kWarps;
+    const DecodeRows rows{a.idx, a.P};
+    Producer<S, N, DecodeRows> prod;
+    if (lane == 0) {
+        prod.start(rows, gw, nw, cph, nunits, H, Dm);
+#pragma unroll
+        for (int s = 0; s < kStages; ++s)
+            prod.issue(rows, a.state, a.slot_stride, gw, nw, cph, nunits, H, Dm, w, s);
+    }
+
+    const int ln = lane % G::LPR, sub = lane / G::LPR;
+    int c = 0;                                  // tiles consumed by this warp
+    for (int u = gw; u < nunits; u += nw) {
+        const Unit un = unit_at(u, cph, G::CR, H, Dm);
+        const int tiles = (un.rows + G::RT - 1) / G::RT;
+        const int64_t xrow = ((int64_t)un.b * H + un.h) * Dm + un.row0;
+
+        // ---- per-unit inputs: addresses independent of the slot index
+        const float dte = effective_dt(a.dt[(int64_t)un.b * H + un.h], a.dt_bias, un.h,
+                                       a.softplus);
+        const float dA = expf(a.A[un.h] * dte);
+        const float Dh = a.D ? a.D[un.h] : 0.f;
+        float Bn[G::E], Cn[G::E], xo[G::XR], zo[G::XR];
+        {
+            const int64_t bc = ((int64_t)un.b * a.G + un.h / hpg) * N;
+#pragma unroll
+            for (int v = 0; v < G::NV; ++v)
+#pragma unroll
+                for (int e = 0; e < G::VEC; ++e) {
+                    Bn[v * G::VEC + e] = ld_f32(a.B, a.bc_dtype, bc + G::col(v, ln, e));
+                    Cn[v * G::VEC + e] = ld_f32(a.C, a.bc_dtype, bc + G::col(v, ln, e));
+                }
+        }
+#pragma unroll
+        for (int m = 0; m < G::XR; ++m) {
+            const int r = lane + 32 * m;
+            const bool in = r < un.rows;
+            xo[m] = in ? ld_f32(a.x, a.x_dtype, xrow + r) : 0.f;
+            zo[m] = (in && a.z) ? ld_f32(a.z, a.x_dtype, xrow + r) : 0.f;
+            if (r < G::CR)
+                xs[r] = xo[m];
+        }
+        __syncwarp();
+
+        int slot = -1;
+        for (int j = 0; j < tiles; ++j, ++c) {
+            if (!wait_tile(w, c, lane == 0 ? prod.issued : 0, lane, a.err))
+                return;
+            const int s = c % kStages;
+            slot = w.ctl->slot[s];
+            if (rows.moves(make_int2(slot, 0))) {
+                const int rt = min(G::RT, un.rows - j * G::RT);
+                const uint8_t *buf = w.ring + s * kTileBytes;
+                S *dst = static_cast<S *>(a.state) + (int64_t)slot * a.slot_stride +
+                         ((int64_t)un.h * Dm + un.row0 + j * G::RT) * N;
+                uint4 raw[G::RPT][G::NV];
+#pragma unroll
+                for (int i = 0; i < G::RPT; ++i) {
+                    const int r = i * G::RPW + sub;
+#pragma unroll
+                    for (int v = 0; v < G::NV; ++v)
+                        raw[i][v] = r < rt ? *reinterpret_cast<const uint4 *>(
+                                                 buf + r * G::ROW_BYTES + (v * G::LPR + ln) * 16)
+                                           : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int i = 0; i < G::RPT; ++i) {
+                    const int r = i * G::RPW + sub;
+                    const float dtx = r < rt ? dte * xs[j * G::RT + r] : 0.f;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int v = 0; v < G::NV; ++v) {
+                        float f[G::VEC];
+                        V::unpack(raw[i][v], f);
+#pragma unroll
+                        for (int e = 0; e < G::VEC; ++e) {
+                            const float sn = fmaf(f[e], dA, Bn[v * G::VEC + e] * dtx);
+                            f[e] = sn;
+                            acc = fmaf(sn, Cn[v * G::VEC + e], acc);
+                        }
+                        if (r < rt)
+                            *reinterpret_cast<uint4 *>(dst + (int64_t)r * N + G::col(v, ln, 0)) =
+                                V::pack(f);
+                    }
+#pragma unroll
+                    for (int off = G::LPR / 2; off > 0; off >>= 1)
+                        acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                    if (ln == 0 && r < rt)
+                        ys[j * G::RT + r] = acc;
+                }
+            }
+            __syncwarp();                        // every lane is done with buffer s
+            if (lane == 0)
+                prod.issue(rows, a.state, a.slot_stride, gw, nw, cph, nunits, H, Dm, w, s);
+        }
+
+        // ---- the unit's outputs, one coalesced store per 32 rows
+        if (slot >= a.P) {                       // caller bug: skip the row and report it
+            if (lane == 0 && un.h == 0 && un.row0 == 0 && a.err)
+                atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
+        } else {
+#pragma unroll
+            for (int m = 0; m < G::XR; ++m) {
+                const int r = lane + 32 * m;
+                if (r < un.rows) {
+                    float y = 0.f;               // padding row: zero
+                    if (slot >= 0) {
+                        y = ys[r] + Dh * xo[m];
+                        if (a.z)
+                            y *= silu_f(zo[m]);
+                    }
+                    st_f32(a.out, a.x_dtype, xrow + r, y);
+                }
+            }
+        }
+        __syncwarp();                            // xs / ys are reused by the next unit
+    }
+}
+
+template <typename S, int N>
+int launch_n(const DecodeArgs &a, cudaStream_t stream)
+{
+    using G = Geo<S, N>;
+    const int64_t cph = (a.Dm + G::CR - 1) / G::CR;
+    const int64_t nunits = (int64_t)a.active * a.H * cph;
+    if (nunits == 0)
+        return SSU_OK;
+    if (nunits > 0x7fffffffLL)
+        return SSU_ERR_SHAPE;
+    const int grid = persistent_grid<ssu_decode_kernel<S, N>>(nunits);
+    ssu_decode_kernel<S, N><<<grid, kWarps * 32, kSmemBytes, stream>>>(a, (int)cph, (int)nunits);
+    return SSU_OK;
 }
 
 template <typename S>

@@ -4,152 +4,204 @@
 // and invokeMambaReplayReconstructBatched: re-run the recurrence over the first
 // acceptedLengths[b] tokens of the replay stash written by the prefill, in place on the
 // committed state; a row whose accepted count is 0 is left untouched, and the loop is
-// bounded by activeBatchSize.
+// bounded by activeBatchSize. The stash carries the finished factors of each token:
+//     state = state * dA[t] + B[t][n] * (dt[t] * U[t][d])
+// (dA = exp(A * dt_eff), dt = dt_eff, U = x), the same association the decode and
+// prefill kernels use, so fp32 results agree bit for bit with the decode steps.
 //
-// With at most a handful of tokens per row the work is dominated by one read and one
-// write of each touched state row, so the kernel has the decode kernel's streaming
-// layout (16-byte accesses, several rows in flight per thread, loads issued first) and
-// keeps the state in registers while the stashed tokens are applied.
-#include "ssu_common.cuh"
+// With a handful of tokens per row the work is one read and one write of every touched
+// state row, so the kernel runs on the per-warp bulk-copy pipeline of ssu_stream.cuh;
+// rows with nothing accepted are never copied. The stash values are read through L1
+// (B and dA/dt are shared by all tiles of a unit).
+#include "ssu_stream.cuh"
 
 namespace ssu {
 namespace {
 
-constexpr int kReplayWarps = 8;
+using namespace stream;
 
-template <typename S, int N, int RPT>
-__global__ void __launch_bounds__(kReplayWarps * 32)
-ssu_replay_kernel(const ReplayArgs a)
+constexpr int kPre = 4;   // stashed tokens per unit held in registers
+
+// The lane's E columns of an fp32 [N] row, as 16-byte loads.
+template <typename G>
+__device__ __forceinline__ void load_cols(const float *row, int ln, float *dst)
 {
-    using V = Vec16<S>;
-    constexpr int VEC = V::kElems;
-    constexpr int LPR = (N / VEC) < 32 ? (N / VEC) : 32;
-    constexpr int E = N / LPR;
-    constexpr int NV = E / VEC;
-    constexpr int RPW = 32 / LPR;
-    constexpr int RPP = kReplayWarps * RPW;
-    constexpr int RT = RPP * RPT;
-
-    const int H = a.H, Dm = a.Dm, T = a.T;
-    const int dtiles = (Dm + RT - 1) / RT;
-    int unit = blockIdx.x;
-    const int dtile = unit % dtiles;
-    unit /= dtiles;
-    const int h = unit % H;
-    const int b = unit / H;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int ln = lane % LPR;
-    const int rbase = dtile * RT + warp * RPW + lane / LPR;
-    const bool reporter = threadIdx.x == 0 && dtile == 0 && h == 0;
-
-    const int slot = a.idx ? a.idx[b] : b;
-    if (slot < 0)
-        return;                           // padding row: nothing to commit
-    if (slot >= a.P) {
-        if (reporter && a.err)
-            atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
-        return;
-    }
-    int k = a.acc[b];
-    if (k > T) {
-        if (reporter && a.err)
-            atomicOr(a.err, SSU_FLAG_ACCEPTED_RANGE);
-        k = T;
-    }
-    if (k < 0) {
-        if (reporter && a.err)
-            atomicOr(a.err, SSU_FLAG_NEGATIVE_LENGTH);
-        k = 0;
-    }
-    if (k == 0)
-        return;                           // nothing accepted: row untouched
-
-    S *base = static_cast<S *>(a.state) + (int64_t)slot * a.slot_stride + (int64_t)h * Dm * N;
-    uint4 raw[RPT][NV];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int r = rbase + i * RPP;
-        const uint4 *rp = reinterpret_cast<const uint4 *>(base + (int64_t)r * N);
+    for (int v = 0; v < G::NV; ++v)
 #pragma unroll
-        for (int v = 0; v < NV; ++v)
-            raw[i][v] = r < Dm ? rp[v * LPR + ln] : make_uint4(0, 0, 0, 0);
-    }
-    float s[RPT][E];
-#pragma unroll
-    for (int i = 0; i < RPT; ++i)
-#pragma unroll
-        for (int v = 0; v < NV; ++v)
-            V::unpack(raw[i][v], &s[i][v * VEC]);
-
-    const int g = h / (H / a.G);
-    for (int t = 0; t < k; ++t) {
-        const int64_t bt = (int64_t)b * T + t;
-        const float dA = a.st_dA[bt * H + h];
-        const float dte = a.st_dt[bt * H + h];
-        const float *Bt = a.st_B + (bt * a.G + g) * N;
-        float Bn[E];
-#pragma unroll
-        for (int v = 0; v < NV; ++v)
-#pragma unroll
-            for (int k4 = 0; k4 < VEC; k4 += 4) {
-                const float4 q = *reinterpret_cast<const float4 *>(Bt + (v * LPR + ln) * VEC + k4);
-                Bn[v * VEC + k4] = q.x;
-                Bn[v * VEC + k4 + 1] = q.y;
-                Bn[v * VEC + k4 + 2] = q.z;
-                Bn[v * VEC + k4 + 3] = q.w;
-            }
-        const float *Ut = a.st_U + (bt * H + h) * Dm;
-#pragma unroll
-        for (int i = 0; i < RPT; ++i) {
-            const int r = rbase + i * RPP;
-            const float dtu = r < Dm ? dte * Ut[r] : 0.f;
-#pragma unroll
-            for (int j = 0; j < E; ++j)
-                s[i][j] = fmaf(s[i][j], dA, Bn[j] * dtu);
+        for (int e4 = 0; e4 < G::VEC; e4 += 4) {
+            const float4 q = *reinterpret_cast<const float4 *>(row + G::col(v, ln, e4));
+            dst[v * G::VEC + e4] = q.x;
+            dst[v * G::VEC + e4 + 1] = q.y;
+            dst[v * G::VEC + e4 + 2] = q.z;
+            dst[v * G::VEC + e4 + 3] = q.w;
         }
-    }
-
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int r = rbase + i * RPP;
-        if (r < Dm) {
-            uint4 *rp = reinterpret_cast<uint4 *>(base + (int64_t)r * N);
-#pragma unroll
-            for (int v = 0; v < NV; ++v)
-                rp[v * LPR + ln] = V::pack(&s[i][v * VEC]);
-        }
-    }
 }
 
-template <typename S, int N, int RPT>
-int launch_rpt(const ReplayArgs &a, cudaStream_t s)
+struct ReplayRows {
+    const int32_t *idx;
+    const int32_t *acc;
+    int32_t P, T;
+    __device__ __forceinline__ int2 resolve(int b) const
+    {
+        return make_int2(idx ? idx[b] : b, acc[b]);
+    }
+    __device__ __forceinline__ bool moves(int2 r) const
+    {
+        return r.x >= 0 && r.x < P && min(r.y, T) > 0;
+    }
+};
+
+template <typename S, int N>
+__global__ void __launch_bounds__(kWarps * 32)
+ssu_replay_kernel(const ReplayArgs a, const int cph, const int nunits)
 {
-    constexpr int VEC = Vec16<S>::kElems;
-    constexpr int LPR = (N / VEC) < 32 ? (N / VEC) : 32;
-    constexpr int RT = kReplayWarps * (32 / LPR) * RPT;
-    const int64_t dtiles = (a.Dm + RT - 1) / RT;
-    const int64_t grid = (int64_t)a.active * a.H * dtiles;
-    if (grid == 0 || a.T == 0)
-        return SSU_OK;
-    if (grid > 0x7fffffffLL)
-        return SSU_ERR_SHAPE;
-    ssu_replay_kernel<S, N, RPT><<<(unsigned)grid, kReplayWarps * 32, 0, s>>>(a);
-    return SSU_OK;
+    using G = Geo<S, N>;
+    using V = Vec16<S>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const WarpViews w = warp_views(smem, warp);
+    init_ring(w, lane);
+
+    const int H = a.H, Dm = a.Dm, T = a.T, hpg = H / a.G;
+    const int gw = blockIdx.x * kWarps + warp;
+    const int nw = gridDim.x * kWarps;
+    const ReplayRows rows{a.idx, a.acc, a.P, T};
+    Producer<S, N, ReplayRows> prod;
+    if (lane == 0) {
+        prod.start(rows, gw, nw, cph, nunits, H, Dm);
+#pragma unroll
+        for (int s = 0; s < kStages; ++s)
+            prod.issue(rows, a.state, a.slot_stride, gw, nw, cph, nunits, H, Dm, w, s);
+    }
+
+    const int ln = lane % G::LPR, sub = lane / G::LPR;
+    int c = 0;
+    for (int u = gw; u < nunits; u += nw) {
+        const Unit un = unit_at(u, cph, G::CR, H, Dm);
+        const int tiles = (un.rows + G::RT - 1) / G::RT;
+        const int g = un.h / hpg;
+
+        // ---- the unit's first kPre stashed tokens, loaded before its first tile is
+        // waited for (addresses stay inside the stash whatever the accepted count is)
+        float pdA[kPre], pdt[kPre], pB[kPre][G::E], pU[kPre][G::XR];
+#pragma unroll
+        for (int t = 0; t < kPre; ++t) {
+            if (t < T) {
+                const int64_t bt = (int64_t)un.b * T + t;
+                pdA[t] = a.st_dA[bt * H + un.h];
+                pdt[t] = a.st_dt[bt * H + un.h];
+                load_cols<G>(a.st_B + (bt * a.G + g) * N, ln, pB[t]);
+                const float *Ut = a.st_U + (bt * H + un.h) * Dm + un.row0;
+#pragma unroll
+                for (int m = 0; m < G::XR; ++m)
+                    pU[t][m] = lane + 32 * m < un.rows ? Ut[lane + 32 * m] : 0.f;
+            }
+        }
+
+        int2 r2 = make_int2(-1, 0);
+        for (int j = 0; j < tiles; ++j, ++c) {
+            if (!wait_tile(w, c, lane == 0 ? prod.issued : 0, lane, a.err))
+                return;
+            const int s = c % kStages;
+            r2 = make_int2(w.ctl->slot[s], w.ctl->extra[s]);
+            if (rows.moves(r2)) {
+                const int k = min(r2.y, T);
+                const int rt = min(G::RT, un.rows - j * G::RT);
+                const int r0 = un.row0 + j * G::RT;
+                const uint8_t *buf = w.ring + s * kTileBytes;
+                float st[G::RPT][G::E];
+#pragma unroll
+                for (int i = 0; i < G::RPT; ++i) {
+                    const int r = i * G::RPW + sub;
+#pragma unroll
+                    for (int v = 0; v < G::NV; ++v) {
+                        const uint4 q = r < rt ? *reinterpret_cast<const uint4 *>(
+                                                     buf + r * G::ROW_BYTES + (v * G::LPR + ln) * 16)
+                                               : make_uint4(0, 0, 0, 0);
+                        V::unpack(q, &st[i][v * G::VEC]);
+                    }
+                }
+                // tokens held in registers; U of unit row q lives in lane q % 32, slot
+                // q / 32, and the rows of one warp access never straddle 32, so the slot
+                // index is warp-uniform
+#pragma unroll
+                for (int t = 0; t < kPre; ++t) {
+                    if (t < k) {
+#pragma unroll
+                        for (int i = 0; i < G::RPT; ++i) {
+                            const int q = j * G::RT + i * G::RPW + sub;
+                            float um = pU[t][0];
+#pragma unroll
+                            for (int m = 1; m < G::XR; ++m)
+                                um = (q >> 5) == m ? pU[t][m] : um;
+                            const float uq = __shfl_sync(0xffffffffu, um, q & 31);
+                            const float dtu = pdt[t] * uq;
+#pragma unroll
+                            for (int e = 0; e < G::E; ++e)
+                                st[i][e] = fmaf(st[i][e], pdA[t], pB[t][e] * dtu);
+                        }
+                    }
+                }
+                // longer acceptances: the remaining tokens straight from the stash
+                for (int t = kPre; t < k; ++t) {
+                    const int64_t bt = (int64_t)un.b * T + t;
+                    const float dA = a.st_dA[bt * H + un.h];
+                    const float dte = a.st_dt[bt * H + un.h];
+                    const float *Ut = a.st_U + (bt * H + un.h) * Dm + r0;
+                    float Bn[G::E];
+                    load_cols<G>(a.st_B + (bt * a.G + g) * N, ln, Bn);
+#pragma unroll
+                    for (int i = 0; i < G::RPT; ++i) {
+                        const int r = i * G::RPW + sub;
+                        const float dtu = r < rt ? dte * Ut[r] : 0.f;
+#pragma unroll
+                        for (int e = 0; e < G::E; ++e)
+                            st[i][e] = fmaf(st[i][e], dA, Bn[e] * dtu);
+                    }
+                }
+                S *dst = static_cast<S *>(a.state) + (int64_t)r2.x * a.slot_stride +
+                         ((int64_t)un.h * Dm + r0) * N;
+#pragma unroll
+                for (int i = 0; i < G::RPT; ++i) {
+                    const int r = i * G::RPW + sub;
+                    if (r < rt) {
+#pragma unroll
+                        for (int v = 0; v < G::NV; ++v)
+                            *reinterpret_cast<uint4 *>(dst + (int64_t)r * N + G::col(v, ln, 0)) =
+                                V::pack(&st[i][v * G::VEC]);
+                    }
+                }
+            }
+            __syncwarp();                        // every lane is done with buffer s
+            if (lane == 0)
+                prod.issue(rows, a.state, a.slot_stride, gw, nw, cph, nunits, H, Dm, w, s);
+        }
+        // ---- caller bugs, reported once per row (the row is clamped or skipped)
+        if (lane == 0 && un.h == 0 && un.row0 == 0 && a.err) {
+            if (r2.x >= a.P)
+                atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
+            else if (r2.x >= 0 && r2.y > T)
+                atomicOr(a.err, SSU_FLAG_ACCEPTED_RANGE);
+            else if (r2.x >= 0 && r2.y < 0)
+                atomicOr(a.err, SSU_FLAG_NEGATIVE_LENGTH);
+        }
+    }
 }
 
 template <typename S, int N>
-int launch_n(const ReplayArgs &a, cudaStream_t s)
+int launch_n(const ReplayArgs &a, cudaStream_t stream)
 {
-    constexpr int VEC = Vec16<S>::kElems;
-    constexpr int LPR = (N / VEC) < 32 ? (N / VEC) : 32;
-    constexpr int RPP = kReplayWarps * (32 / LPR);
-    if (a.Dm >= 8 * RPP)
-        return launch_rpt<S, N, 8>(a, s);
-    if (a.Dm >= 4 * RPP)
-        return launch_rpt<S, N, 4>(a, s);
-    if (a.Dm >= 2 * RPP)
-        return launch_rpt<S, N, 2>(a, s);
-    return launch_rpt<S, N, 1>(a, s);
+    using G = Geo<S, N>;
+    const int64_t cph = (a.Dm + G::CR - 1) / G::CR;
+    const int64_t nunits = (int64_t)a.active * a.H * cph;
+    if (nunits == 0 || a.T == 0)
+        return SSU_OK;
+    if (nunits > 0x7fffffffLL)
+        return SSU_ERR_SHAPE;
+    const int grid = persistent_grid<ssu_replay_kernel<S, N>>(nunits);
+    ssu_replay_kernel<S, N><<<grid, kWarps * 32, kSmemBytes, stream>>>(a, (int)cph, (int)nunits);
+    return SSU_OK;
 }
 
 template <typename S>

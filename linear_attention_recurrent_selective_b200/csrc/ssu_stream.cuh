@@ -1,0 +1,215 @@
+// ssu_stream.cuh -- the per-warp streaming pipeline shared by the HBM-bound kernels
+// (decode and replay), which read every touched state row once and write it once.
+//
+// Work is cut into "units": up to kUnitRows rows (at most 32 KB) of one head of one
+// batch row's slot. Persistent CTAs of kWarps warps each run an independent pipeline:
+// warp w of the grid takes units w, w + W, w + 2W, ... (W = warps in the grid), so all
+// warps sweep the pool together in address order. A unit is cut into tiles of up to
+// kTileBytes of contiguous state; every warp owns a ring of kStages shared-memory tile
+// buffers that the bulk-copy engine fills (cp.async.bulk, completion counted on a
+// per-buffer mbarrier), so kStages-1 tiles are in flight while the warp computes on one.
+// Lane 0 is the producer: it resolves the slot (and any per-row extra, such as an
+// accepted length) of the unit after the one it is copying one unit early, so the
+// index loads never stall the ring. Rows that touch no state (padding, out-of-range
+// index, nothing accepted) complete their buffer's barrier without a copy, which keeps
+// the consumer's phase bookkeeping uniform.
+#pragma once
+
+#include "ssu_async.cuh"
+#include "ssu_common.cuh"
+
+namespace ssu {
+namespace stream {
+
+// Pipeline shape; the defaults are the measured best on B200 for the batch-256 decode
+// and can be overridden at build time for tuning sweeps.
+#ifndef SSU_STREAM_WARPS
+#define SSU_STREAM_WARPS 8
+#endif
+#ifndef SSU_STREAM_STAGES
+#define SSU_STREAM_STAGES 3
+#endif
+constexpr int kWarps = SSU_STREAM_WARPS;    // warps per CTA, each an independent pipeline
+constexpr int kStages = SSU_STREAM_STAGES;  // tile buffers per warp
+constexpr int kTileBytes = 4096;            // one tile: 8 warp-wide 512-byte accesses
+constexpr int kUnitRows = 128;              // at most this many rows per unit
+constexpr int kUnitTiles = 8;               // and at most 32 KB of state
+
+template <typename S, int N> struct Geo {
+    static constexpr int VEC = Vec16<S>::kElems;                 // elements per 16 bytes
+    static constexpr int LPR = (N / VEC) < 32 ? (N / VEC) : 32;  // lanes per state row
+    static constexpr int E = N / LPR;                           // elements per lane and row
+    static constexpr int NV = E / VEC;                          // 16-byte vectors per lane/row
+    static constexpr int RPW = 32 / LPR;                        // rows per warp access
+    static constexpr int ROW_BYTES = N * (int)sizeof(S);
+    static constexpr int RT = kTileBytes / ROW_BYTES;           // rows per full tile
+    static constexpr int RPT = RT / RPW;                        // row accesses per lane/tile
+    static constexpr int CR = (kUnitTiles * RT) < kUnitRows ? (kUnitTiles * RT) : kUnitRows;
+    static constexpr int XR = (CR + 31) / 32;                   // unit rows per lane
+    static_assert(RT >= 1 && RPT >= 1 && RPT * RPW == RT, "tile geometry");
+    // state column n of vector v, element e for lane-in-row ln
+    static __device__ __forceinline__ int col(int v, int ln, int e) { return (v * LPR + ln) * VEC + e; }
+};
+
+struct Ring {
+    uint64_t full[kStages];
+    int slot[kStages];    // slot of the unit whose tile sits in each buffer
+    int extra[kStages];   // per-row extra of that unit (e.g. the accepted length)
+};
+static_assert(sizeof(Ring) <= 128, "per-warp control block");
+
+constexpr int kRingBytes = kStages * kTileBytes;
+constexpr int kStageBytes = 2 * kUnitRows * 4;           // two per-unit float rows
+constexpr int kPerWarpBytes = kRingBytes + kStageBytes + 128;   // a multiple of 128
+constexpr int kSmemBytes = kWarps * kPerWarpBytes;
+
+struct Unit {
+    int b, h, row0, rows;
+};
+
+__device__ __forceinline__ Unit unit_at(int u, int cph, int CR, int H, int Dm)
+{
+    Unit un;
+    const int c = u % cph;
+    const int v = u / cph;
+    un.h = v % H;
+    un.b = v / H;
+    un.row0 = c * CR;
+    un.rows = min(CR, Dm - un.row0);
+    return un;
+}
+
+// Per-warp views of the dynamic shared memory.
+struct WarpViews {
+    uint8_t *ring;     // kStages tile buffers
+    float *f0, *f1;    // two [kUnitRows] float rows for per-unit staging
+    Ring *ctl;
+};
+
+__device__ __forceinline__ WarpViews warp_views(uint8_t *smem, int warp)
+{
+    WarpViews w;
+    w.ring = smem + warp * kPerWarpBytes;
+    w.f0 = reinterpret_cast<float *>(w.ring + kRingBytes);
+    w.f1 = w.f0 + kUnitRows;
+    w.ctl = reinterpret_cast<Ring *>(w.f1 + kUnitRows);
+    return w;
+}
+
+// Lane 0's side of a warp's pipeline. `Rows` maps a batch row to {slot, extra} and says
+// whether a unit of that row moves state:
+//   int2 resolve(int b) const;  bool moves(int2 r) const;
+template <typename S, int N, typename Rows> struct Producer {
+    using G = Geo<S, N>;
+    int k;        // position in this warp's unit sequence
+    int j;        // next tile within the unit
+    int tiles;    // tiles of the current unit
+    int2 cur;     // {slot, extra} of the current unit
+    int2 nxt;     // the same for the next unit (loaded one unit early)
+    int issued;   // tiles issued so far
+
+    __device__ void start(const Rows &rows, int gw, int nw, int cph, int nunits, int H, int Dm)
+    {
+        k = 0;
+        j = 0;
+        issued = 0;
+        tiles = 0;
+        cur = make_int2(-1, 0);
+        nxt = make_int2(-1, 0);
+        if (gw < nunits) {
+            const Unit un = unit_at(gw, cph, G::CR, H, Dm);
+            cur = rows.resolve(un.b);
+            tiles = (un.rows + G::RT - 1) / G::RT;
+            if (gw + nw < nunits)
+                nxt = rows.resolve(unit_at(gw + nw, cph, G::CR, H, Dm).b);
+        }
+    }
+
+    __device__ void issue(const Rows &rows, const void *state, int64_t slot_stride, int gw,
+                          int nw, int cph, int nunits, int H, int Dm, const WarpViews &w, int s)
+    {
+        const int u = gw + k * nw;
+        if (u >= nunits)
+            return;
+        const Unit un = unit_at(u, cph, G::CR, H, Dm);
+        w.ctl->slot[s] = cur.x;
+        w.ctl->extra[s] = cur.y;
+        if (rows.moves(cur)) {
+            const int nr = min(G::RT, un.rows - j * G::RT);
+            const uint32_t bytes = (uint32_t)(nr * G::ROW_BYTES);
+            const S *src = static_cast<const S *>(state) + (int64_t)cur.x * slot_stride +
+                           ((int64_t)un.h * Dm + un.row0 + j * G::RT) * N;
+            mbar_arrive_expect_tx(&w.ctl->full[s], bytes);
+            bulk_load(w.ring + s * kTileBytes, src, bytes, &w.ctl->full[s]);
+        } else {
+            mbar_arrive(&w.ctl->full[s]);
+        }
+        ++issued;
+        if (++j == tiles) {                  // move to this warp's next unit
+            j = 0;
+            ++k;
+            const int u2 = gw + k * nw;
+            if (u2 < nunits) {
+                cur = nxt;
+                tiles = (unit_at(u2, cph, G::CR, H, Dm).rows + G::RT - 1) / G::RT;
+                if (u2 + nw < nunits)
+                    nxt = rows.resolve(unit_at(u2 + nw, cph, G::CR, H, Dm).b);
+            }
+        }
+    }
+};
+
+// Initialise the warp's ring barriers (lane 0) and make them visible to the copy engine.
+__device__ __forceinline__ void init_ring(const WarpViews &w, int lane)
+{
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < kStages; ++s)
+            mbar_init(&w.ctl->full[s], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+}
+
+// Wait for consumed-tile number c; on a (never expected) timeout, report it, let the
+// copies this warp started land and return false. The verdict is warp-uniform.
+__device__ __forceinline__ bool wait_tile(const WarpViews &w, int c, int issued_lane0,
+                                          int lane, int32_t *err)
+{
+    const int s = c % kStages;
+    if (__all_sync(0xffffffffu, mbar_wait(&w.ctl->full[s], (uint32_t)(c / kStages) & 1u)))
+        return true;
+    if (lane == 0 && err)
+        atomicOr(err, SSU_FLAG_TIMEOUT);
+    const int issued = __shfl_sync(0xffffffffu, issued_lane0, 0);
+    for (int cc = c; cc < issued; ++cc)
+        if (!mbar_wait(&w.ctl->full[cc % kStages], (uint32_t)(cc / kStages) & 1u))
+            break;
+    return false;
+}
+
+// Grid size for a persistent launch: as many CTAs as fit, no more than the work needs.
+// One instantiation (and one cache of the occupancy query) per kernel.
+template <auto kernel>
+int persistent_grid(int64_t nunits)
+{
+    static int blocks_per_sm[64];
+    static int sms[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        dev = 0;
+    if (blocks_per_sm[dev] == 0) {
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        int occ = 0, n = 0;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kWarps * 32, kSmemBytes);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        sms[dev] = n > 0 ? n : 148;
+        blocks_per_sm[dev] = occ > 0 ? occ : 1;
+    }
+    const int64_t want = (nunits + kWarps - 1) / kWarps;
+    const int64_t cap = (int64_t)sms[dev] * blocks_per_sm[dev];
+    return (int)(want < cap ? want : cap);
+}
+
+}  // namespace stream
+}  // namespace ssu

@@ -33,6 +33,7 @@ FLAG_INDEX_RANGE = 1
 FLAG_ACCEPTED_RANGE = 2
 FLAG_CONTEXT_RANGE = 4
 FLAG_NEGATIVE_LENGTH = 8
+FLAG_TIMEOUT = 16
 
 # Every C entry point declared in include/ssu.h, in declaration order.
 ENTRY_POINTS = ("ssu_decode", "ssu_prefill", "ssu_replay", "pool_clear_slot",
