@@ -64,6 +64,43 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+DECODE_SOURCES = ("ssu_decode.cu", "ssu_stream.cuh", "ssu_async.cuh", "ssu_common.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ssu_decode_kernel.md")
+
+
+def decode_source_hash() -> str:
+    """sha256 over the decode kernel's sources, to tie an ncu traffic figure to them."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "linear_attention_recurrent_selective_b200", "csrc", name),
+                  "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(batch: int):
+    """DRAM bytes per decode launch recorded from ncu in the decode profile summary, or
+    None when the summary is missing, is for another batch, or was taken on sources
+    other than the ones built now."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+    except OSError:
+        return None
+    rec = {}
+    for line in text.splitlines():
+        if line.startswith("traffic_record:"):
+            for kv in line.split(":", 1)[1].split():
+                k, _, v = kv.partition("=")
+                rec[k] = v
+    if rec.get("source_sha256") != decode_source_hash() or rec.get("batch") != str(batch):
+        return None
+    try:
+        return int(rec["bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def decode_bytes(batch, H, G, Dm, N, state_bytes, io_bytes):
     """Algorithmic bytes of one decode launch: every state element read and written once,
     x/z/out once per (row, head, dim), B/C once per (row, group), dt once per (row, head),
@@ -266,16 +303,14 @@ def time_launches(fn, steps, warmup, device):
     return statistics.fmean(s.elapsed_time(e) for s, e in zip(starts, ends))
 
 
-def run_forms(args, device, hbm_peak):
-    """Prefill (batch 16, T 512, contextLengths ~ U{1..512}) and speculative replay
-    (batch 64, 5 drafted tokens, acceptedLengths ~ U{0..5}) on one GPU."""
+def form_prefill(args, device, batch=0):
+    """Multi-token prefill (batch 16, T 512, contextLengths ~ U{1..512}), without and with
+    the replay stash; FP32-issue bound, reported against the FP32 FMA peak."""
     from linear_attention_recurrent_selective_b200 import ssu
     from linear_attention_recurrent_selective_b200.workloads import make_config
 
-    forms = {}
     steps, warm = max(3, min(args.steps, 50)), max(3, min(args.warmup, 5))
-
-    case = make_config("prefill_b16_t512")
+    case = make_config("prefill_b16_t512", **(dict(batch=batch, P=2 * batch) if batch else {}))
     d = case.to(device)
     pool = d.pool.clone()
     out = torch.empty_like(d.x)
@@ -293,23 +328,34 @@ def run_forms(args, device, hbm_peak):
     flop = tokens * H * Dm * N * 5       # per state element: mul + FMA update, FMA output
     sm = torch.cuda.get_device_properties(device).multi_processor_count
     alu_peak = sm * 128 * 2 * 1.965e9 / 1e12   # fp32 FMA lanes x 2 FLOP x max SM clock
+    forms = {}
     for name, st in (("prefill", None), ("prefill_stash", stash)):
         ms = time_launches(lambda: prefill(st), steps, warm, device)
         forms[name] = {
-            "workload": "prefill_b16_t512", "tokens": tokens, "ms_per_launch": ms,
+            "workload": "prefill_b16_t512", "batch": b, "tokens": tokens, "ms_per_launch": ms,
             "tokens_per_s": tokens / (ms / 1e3),
             "roofline": {"bound": "alu", "achieved": flop / (ms / 1e3) / 1e12,
                          "peak": alu_peak, "unit": "TFLOP/s",
-                         "frac": flop / (ms / 1e3) / 1e12 / alu_peak, "traffic": None}}
+                         "frac": flop / (ms / 1e3) / 1e12 / alu_peak, "traffic": None,
+                         "peak_source": "derived: SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz"}}
+    return forms
 
-    rcase = make_config("spec_replay_b64_t5")
+
+def form_replay(args, device, hbm_peak, batch=0):
+    """Speculative replay (batch 64, 5 drafted tokens, acceptedLengths ~ U{0..5}); the stash
+    comes from this library's prefill in stash mode. HBM bound."""
+    from linear_attention_recurrent_selective_b200 import ssu
+    from linear_attention_recurrent_selective_b200.workloads import make_config
+
+    steps, warm = max(3, min(args.steps, 50)), max(3, min(args.warmup, 5))
+    f = dict(dtype=torch.float32, device=device)
+    rcase = make_config("spec_replay_b64_t5", **(dict(batch=batch, P=2 * batch) if batch else {}))
     rd = rcase.to(device)
     rpool = rd.pool.clone()
     b, T, H, G, Dm, N = rcase.batch, rcase.T, rcase.H, rcase.G, rcase.Dm, rcase.N
     rst = (torch.empty(b, T, H, **f), torch.empty(b, T, H, Dm, **f),
            torch.empty(b, T, G, N, **f), torch.empty(b, T, H, **f))
     rout = torch.empty_like(rd.x)
-    # the stash comes from this library's prefill in stash mode (the pool stays as is)
     ssu.ssu_prefill(rd.x, rd.A, rd.B, rd.C, rd.dt, rpool, rout, dt_bias=rd.dt_bias, D=rd.D,
                     z=rd.z, state_indices=rd.state_indices, stash=rst,
                     slot_stride=rcase.slot_stride, P=rcase.P)
@@ -321,13 +367,13 @@ def run_forms(args, device, hbm_peak):
     rows = int((acc_h > 0).sum())
     nacc = int(acc_h.sum())
     rbytes = rows * H * Dm * N * 4 * 2 + nacc * (H * (4 + 4 + Dm * 4) + G * N * 4) + b * 4
-    forms["replay"] = {
-        "workload": "spec_replay_b64_t5", "accepted_tokens": nacc, "ms_per_launch": ms,
-        "accepted_tokens_per_s": nacc / (ms / 1e3),
+    return {"replay": {
+        "workload": "spec_replay_b64_t5", "batch": b, "accepted_tokens": nacc,
+        "ms_per_launch": ms, "accepted_tokens_per_s": nacc / (ms / 1e3),
+        "algorithmic_bytes": rbytes,
         "roofline": {"bound": "hbm", "achieved": rbytes / (ms / 1e3) / 1e9,
                      "peak": hbm_peak, "unit": "GB/s",
-                     "frac": rbytes / (ms / 1e3) / 1e9 / hbm_peak, "traffic": None}}
-    return forms
+                     "frac": rbytes / (ms / 1e3) / 1e9 / hbm_peak, "traffic": None}}}
 
 
 def cpu_baseline_decode(case, max_seconds=20.0):
@@ -367,6 +413,12 @@ def main_ours(args):
     device = torch.device("cuda", local if n_world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(device)
     hbm_peak, peak_src = measured_peaks()
+    if args.form in ("prefill", "replay"):       # one kernel alone, e.g. under a profiler
+        forms = (form_prefill(args, device, args.batch) if args.form == "prefill"
+                 else form_replay(args, device, hbm_peak, args.batch))
+        if rank == 0:
+            print(json.dumps({"form": args.form, "forms": forms}), flush=True)
+        return
 
     res = run_decode(args, device)
     case = res["case"]
@@ -383,7 +435,7 @@ def main_ours(args):
         "data": "synthetic", "config": config_block(case, res),
         "state_hbm_gbs": res["state_b"] / (res["kern_ms"] / 1e3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": args.traffic,
+                     "frac": achieved / hbm_peak, "traffic": recorded_traffic(case.batch),
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_src == "measured" else "fallback 6.65 TB/s",
                      "kernel": "ssu_decode_kernel", "kernel_ms": res["kern_ms"],
@@ -393,9 +445,9 @@ def main_ours(args):
         "gpu_launches": args.steps,
         "clocks": res["clocks"],
     }
-    if n_world == 1 and not args.no_forms:
-        line["forms"] = run_forms(args, device, hbm_peak)
-    if n_world == 1 and rank == 0 and not args.no_cpu_baseline:
+    if n_world == 1 and not args.no_forms and args.form == "all":
+        line["forms"] = {**form_prefill(args, device), **form_replay(args, device, hbm_peak)}
+    if n_world == 1 and rank == 0 and not args.no_cpu_baseline and args.form == "all":
         line["cpu_baseline"] = cpu_baseline_decode(case)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -451,9 +503,9 @@ def parse(argv=None):
     ap.add_argument("--batch", type=int, default=0,
                     help="override the batch (pool = 2 x batch), e.g. for a small profile")
     ap.add_argument("--no-forms", action="store_true", help="skip the prefill/replay forms")
+    ap.add_argument("--form", choices=("all", "decode", "prefill", "replay"), default="all",
+                    help="run one kernel only (for profiling); its line carries that form")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu DRAM bytes per decode launch for this build (else null)")
     a = ap.parse_args(argv)
     if a.warmup < 3 and a.impl == "ours":
         ap.error("--warmup must be at least 3")

@@ -80,6 +80,24 @@ __device__ __forceinline__ void st_f32(void *p, int dtype, int64_t i, float v)
         static_cast<float *>(p)[i] = v;
 }
 
+// Raw bits of element i (16-bit types zero-extended), for prefetches whose widening is
+// deferred until the value is used, so that no instruction waits on the load early.
+__device__ __forceinline__ uint32_t ld_bits(const void *p, int dtype, int64_t i)
+{
+    if (dtype == SSU_F32)
+        return static_cast<const uint32_t *>(p)[i];
+    return static_cast<const uint16_t *>(p)[i];
+}
+
+__device__ __forceinline__ float bits_f32(uint32_t v, int dtype)
+{
+    if (dtype == SSU_F32)
+        return __uint_as_float(v);
+    if (dtype == SSU_BF16)
+        return __uint_as_float(v << 16);
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(v)));
+}
+
 // softplus(v) = log(1 + e^v); above 20 the correction log1p(e^-v) < 2.1e-9 is dropped.
 __device__ __forceinline__ float softplus_f(float v)
 {

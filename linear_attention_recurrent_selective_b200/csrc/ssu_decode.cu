@@ -31,6 +31,10 @@ namespace {
 
 using namespace stream;
 
+// Units of up to 8 tiles (32 KB): one unit is a whole head of the batch-256 workload,
+// so its metadata is loaded once per 64 KB of traffic.
+constexpr int kUT = 8;
+
 struct DecodeRows {
     const int32_t *idx;
     int32_t P;
@@ -45,7 +49,7 @@ template <typename S, int N>
 __global__ void __launch_bounds__(kWarps * 32)
 ssu_decode_kernel(const DecodeArgs a, const int cph, const int nunits)
 {
-    using G = Geo<S, N>;
+    using G = Geo<S, N, kUT>;
     using V = Vec16<S>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -58,7 +62,7 @@ ssu_decode_kernel(const DecodeArgs a, const int cph, const int nunits)
     const int gw = blockIdx.x * kWarps + warp;
     const int nw = gridDim.x * kWarps;
     const DecodeRows rows{a.idx, a.P};
-    Producer<S, N, DecodeRows> prod;
+    Producer<G, N, DecodeRows> prod;
     if (lane == 0) {
         prod.start(rows, gw, nw, cph, nunits, H, Dm);
 #pragma unroll
@@ -178,7 +182,7 @@ ssu_decode_kernel(const DecodeArgs a, const int cph, const int nunits)
 template <typename S, int N>
 int launch_n(const DecodeArgs &a, cudaStream_t stream)
 {
-    using G = Geo<S, N>;
+    using G = Geo<S, N, kUT>;
     const int64_t cph = (a.Dm + G::CR - 1) / G::CR;
     const int64_t nunits = (int64_t)a.active * a.H * cph;
     if (nunits == 0)

@@ -11,18 +11,21 @@
 // costs a multiply and two FMAs, and each output row a reduction over dstate. The kernel
 // is bound by FP32 issue, so the design minimises everything that is not an FMA:
 //   * one CTA per (batch row, head, tile of up to 128 dim rows); a lane owns R rows x K
-//     consecutive state columns (32 fp32 registers), so one 16-byte shared load of B or
-//     C serves R rows and the x values of its R rows come in R/4 shared loads;
+//     state columns (32 fp32 registers; 2 x 16 for dstate 128) in groups of 4 that
+//     interleave with those of the other lanes of its row group, so a 16-byte shared load
+//     of B or C serves R rows, covers consecutive addresses within the row group, and is
+//     a broadcast across row groups (one wavefront per load);
 //   * the update and the output partial sums use the packed two-wide FP32 instructions
 //     of sm_100 (__fmul2_rn / __ffma2_rn, element-wise round-to-nearest, so each element
 //     is computed exactly as by fmaf and the state matches the decode kernel bit for bit);
 //   * the R partial sums of a lane are reduced across the LPR lanes sharing its rows by
-//     a transposed butterfly: each step halves the values a lane holds, so 8 rows over
-//     32 lanes take 9 shuffles instead of 40;
+//     a transposed butterfly: each step halves the values a lane holds (2 rows over 8
+//     lanes take 3 shuffles);
 //   * inputs are staged per chunk of TC tokens into double-buffered shared memory
 //     (B and C widened to fp32, x and z, dt_eff and exp(A dt_eff)); the next chunk's raw
-//     inputs are loaded into registers before the current chunk is computed, so their
-//     latency hides behind TC tokens of arithmetic;
+//     inputs are loaded into registers (as raw bits: nothing widens them before the
+//     chunk ends) before the current chunk is computed, so their latency hides behind
+//     TC tokens of arithmetic;
 //   * per-token row sums go to shared memory, and the chunk's outputs (D skip term and
 //     silu(z) gate applied) are written with coalesced stores;
 //   * the replay stash is written from the staging registers (B by one CTA per group,
@@ -38,8 +41,22 @@ namespace {
 
 constexpr int kRankMax = 32;    // batches up to this size are scheduled longest-first
 
+// Columns of state per lane (at least N/32) and tokens per unrolled step of the scan;
+// the defaults are the measured best on B200, overridable at build time for sweeps.
+#ifndef SSU_PREFILL_K
+#define SSU_PREFILL_K 16
+#endif
+#ifndef SSU_PREFILL_UNROLL
+#define SSU_PREFILL_UNROLL 1
+#endif
+#ifndef SSU_PREFILL_PACKED
+#define SSU_PREFILL_PACKED 1
+#endif
+constexpr int kUnroll = SSU_PREFILL_UNROLL;
+
 template <typename S, int N> struct PGeo {
-    static constexpr int K = (N / 32) > 4 ? (N / 32) : 4;    // state columns per lane
+    static constexpr int KW = (N / 32) > SSU_PREFILL_K ? (N / 32) : SSU_PREFILL_K;
+    static constexpr int K = KW < N ? KW : N;                // state columns per lane
     static constexpr int LPR = N / K;                        // lanes sharing a row
     static constexpr int RGW = 32 / LPR;                     // row groups per warp
     static constexpr int R = 32 / K;                         // rows per lane
@@ -63,7 +80,11 @@ template <typename S, int N> struct PGeo {
     static constexpr bool XREG = XPT <= 8;                   // else staged synchronously
     static constexpr int NVF = R >= LPR ? R / LPR : 1;       // row sums a lane ends with
     static constexpr int DUP = R >= LPR ? 1 : LPR / R;       // lanes holding the same sum
-    static_assert(K % 4 == 0 && R % 4 == 0 && RTC % 4 == 0 && W >= 1, "prefill geometry");
+    static constexpr int XV = R % 4 == 0 ? 4 : (R % 2 == 0 ? 2 : 1);   // x floats per load
+    // first column of the lane's q-th group of 4: the groups of the lanes of a row group
+    // interleave, so each 16-byte shared load of B or C covers consecutive addresses
+    static __device__ __forceinline__ int col(int ln, int q) { return 4 * (ln + LPR * q); }
+    static_assert(K % 4 == 0 && R * K == 32 && RTC % 4 == 0 && W >= 1, "prefill geometry");
 };
 
 // Transposed butterfly over the lanes of a row group: on entry v[0..NV) are this lane's
@@ -124,6 +145,7 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
     using P = PGeo<S, N>;
     extern __shared__ __align__(16) float sm[];
     __shared__ int s_row;
+    __shared__ int s_len[kRankMax];
 
     const DecodeArgs &a = pa.d;
     const int H = a.H, Dm = a.Dm, T = pa.T, G = a.G;
@@ -136,13 +158,14 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
     const int h = rem / dtiles, dtile = rem % dtiles;
     int b = rank;
     if (a.active <= kRankMax) {
+        if (tid < a.active)
+            s_len[tid] = sched_len(pa, tid);
+        __syncthreads();
         if (tid < a.active) {
-            const int mine = sched_len(pa, tid);
+            const int mine = s_len[tid];
             int r = 0;
-            for (int o = 0; o < a.active; ++o) {
-                const int lo = sched_len(pa, o);
-                r += (lo > mine) || (lo == mine && o < tid);
-            }
+            for (int o = 0; o < a.active; ++o)
+                r += (s_len[o] > mine) || (s_len[o] == mine && o < tid);
             if (r == rank)
                 s_row = tid;
         }
@@ -190,7 +213,6 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
     // ---- this lane's rows and columns
     const int rg = lane / P::LPR, ln = lane % P::LPR;
     const int lrow = warp * P::RPWARP + rg * P::R;      // first local row of the lane
-    const int col0 = ln * P::K;
     S *base = static_cast<S *>(a.state) + (int64_t)slot * a.slot_stride + (int64_t)h * Dm * N;
 
     float2 st[P::R][P::K / 2];
@@ -201,7 +223,7 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
         for (int q = 0; q < P::K / 4; ++q) {
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             if (row < Dm)
-                v = Quad<S>::load(base + (int64_t)row * N + col0 + 4 * q);
+                v = Quad<S>::load(base + (int64_t)row * N + P::col(ln, q));
             st[i][2 * q] = make_float2(v.x, v.y);
             st[i][2 * q + 1] = make_float2(v.z, v.w);
         }
@@ -209,7 +231,7 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
 
     // ---- staging of one chunk: raw loads into registers, then widen into a buffer
     uint4 rb[P::VBMAX], rc[P::VBMAX];
-    float rx[P::XREG ? P::XPT : 1], rz[P::XREG ? P::XPT : 1];
+    uint32_t rx[P::XREG ? P::XPT : 1], rz[P::XREG ? P::XPT : 1];   // raw bits of x and z
     float rdt = 0.f;
     const int vb = 16 / (a.bc_dtype == SSU_F32 ? 4 : 2);   // B/C elements per 16 bytes
     const int nvec = P::TC * N / vb;
@@ -231,13 +253,13 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
             for (int k = 0; k < P::XPT; ++k) {
                 const int e = tid + k * P::THREADS;
                 const int t = e / P::RTC, row = row0 + e % P::RTC;
-                rx[k] = 0.f;
-                rz[k] = 0.f;
+                rx[k] = 0u;                         // zero bits are 0.0 in every format
+                rz[k] = 0u;
                 if (e < P::TC * P::RTC && t0 + t < L && row < Dm) {
                     const int64_t xi = (((int64_t)b * T + t0 + t) * H + h) * Dm + row;
-                    rx[k] = ld_f32(a.x, a.x_dtype, xi);
+                    rx[k] = ld_bits(a.x, a.x_dtype, xi);
                     if (a.z)
-                        rz[k] = ld_f32(a.z, a.x_dtype, xi);
+                        rz[k] = ld_bits(a.z, a.x_dtype, xi);
                 }
             }
         }
@@ -274,8 +296,8 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
             const bool in = t0 + t < L && row < Dm;
             const int64_t xi = (((int64_t)b * T + t0 + t) * H + h) * Dm + row;
             if constexpr (P::XREG) {
-                xv = rx[k];
-                zv = rz[k];
+                xv = bits_f32(rx[k], a.x_dtype);
+                zv = bits_f32(rz[k], a.x_dtype);
             } else if (in) {
                 xv = ld_f32(a.x, a.x_dtype, xi);
                 if (a.z)
@@ -312,30 +334,38 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
             load_chunk(t0 + P::TC);            // in flight during this chunk's arithmetic
 
         // ---- the recurrence, token by token, state in registers
-        for (int t = 0; t < nt; ++t) {
+        auto token = [&](const int t) {
             const float dA = cur[P::OFF_DA + t];
             const float dte = cur[P::OFF_DT + t];
             const float2 dA2 = make_float2(dA, dA);
             float2 B2[P::K / 2], C2[P::K / 2];
 #pragma unroll
             for (int q = 0; q < P::K / 4; ++q) {
-                const float4 b4 = *reinterpret_cast<const float4 *>(cur + t * N + col0 + 4 * q);
+                const float4 b4 = *reinterpret_cast<const float4 *>(cur + t * N + P::col(ln, q));
                 const float4 c4 =
-                    *reinterpret_cast<const float4 *>(cur + P::OFF_C + t * N + col0 + 4 * q);
+                    *reinterpret_cast<const float4 *>(cur + P::OFF_C + t * N + P::col(ln, q));
                 B2[2 * q] = make_float2(b4.x, b4.y);
                 B2[2 * q + 1] = make_float2(b4.z, b4.w);
                 C2[2 * q] = make_float2(c4.x, c4.y);
                 C2[2 * q + 1] = make_float2(c4.z, c4.w);
             }
             float xv[P::R];
+            const float *xt = cur + P::OFF_X + t * P::RTC + lrow;
 #pragma unroll
-            for (int q = 0; q < P::R / 4; ++q) {
-                const float4 x4 =
-                    *reinterpret_cast<const float4 *>(cur + P::OFF_X + t * P::RTC + lrow + 4 * q);
-                xv[4 * q] = x4.x;
-                xv[4 * q + 1] = x4.y;
-                xv[4 * q + 2] = x4.z;
-                xv[4 * q + 3] = x4.w;
+            for (int q = 0; q < P::R; q += P::XV) {
+                if constexpr (P::XV == 4) {
+                    const float4 x4 = *reinterpret_cast<const float4 *>(xt + q);
+                    xv[q] = x4.x;
+                    xv[q + 1] = x4.y;
+                    xv[q + 2] = x4.z;
+                    xv[q + 3] = x4.w;
+                } else if constexpr (P::XV == 2) {
+                    const float2 x2 = *reinterpret_cast<const float2 *>(xt + q);
+                    xv[q] = x2.x;
+                    xv[q + 1] = x2.y;
+                } else {
+                    xv[q] = xt[q];
+                }
             }
             float part[P::R];
 #pragma unroll
@@ -345,8 +375,15 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
                 float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int k = 0; k < P::K / 2; ++k) {
+#if SSU_PREFILL_PACKED
                     st[i][k] = __ffma2_rn(st[i][k], dA2, __fmul2_rn(B2[k], d2));
                     acc = __ffma2_rn(st[i][k], C2[k], acc);
+#else
+                    st[i][k].x = fmaf(st[i][k].x, dA, B2[k].x * dtx);
+                    st[i][k].y = fmaf(st[i][k].y, dA, B2[k].y * dtx);
+                    acc.x = fmaf(st[i][k].x, C2[k].x, acc.x);
+                    acc.y = fmaf(st[i][k].y, C2[k].y, acc.y);
+#endif
                 }
                 part[i] = acc.x + acc.y;
             }
@@ -357,7 +394,15 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
                 for (int i = 0; i < P::NVF; ++i)
                     cur[P::OFF_Y + t * P::RTC + lrow + first + i] = part[i];
             }
+        };
+        int t = 0;
+        for (; t + kUnroll <= nt; t += kUnroll) {
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u)
+                token(t + u);
         }
+        for (; t < nt; ++t)
+            token(t);
         __syncthreads();                         // row sums of this chunk complete
 
         // ---- outputs of the chunk: skip term and gate, coalesced along dim
@@ -383,7 +428,7 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
             if (row < Dm) {
 #pragma unroll
                 for (int q = 0; q < P::K / 4; ++q)
-                    Quad<S>::store(base + (int64_t)row * N + col0 + 4 * q,
+                    Quad<S>::store(base + (int64_t)row * N + P::col(ln, q),
                                    make_float4(st[i][2 * q].x, st[i][2 * q].y,
                                                st[i][2 * q + 1].x, st[i][2 * q + 1].y));
             }

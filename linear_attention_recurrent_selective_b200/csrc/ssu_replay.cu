@@ -20,6 +20,10 @@ namespace {
 
 using namespace stream;
 
+// Units of up to 2 tiles (8 KB): a replay touches few rows, and small units spread
+// them evenly over the warps of the grid.
+constexpr int kUT = 2;
+
 constexpr int kPre = 4;   // stashed tokens per unit held in registers
 
 // The lane's E columns of an fp32 [N] row, as 16-byte loads.
@@ -56,7 +60,7 @@ template <typename S, int N>
 __global__ void __launch_bounds__(kWarps * 32)
 ssu_replay_kernel(const ReplayArgs a, const int cph, const int nunits)
 {
-    using G = Geo<S, N>;
+    using G = Geo<S, N, kUT>;
     using V = Vec16<S>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -67,7 +71,7 @@ ssu_replay_kernel(const ReplayArgs a, const int cph, const int nunits)
     const int gw = blockIdx.x * kWarps + warp;
     const int nw = gridDim.x * kWarps;
     const ReplayRows rows{a.idx, a.acc, a.P, T};
-    Producer<S, N, ReplayRows> prod;
+    Producer<G, N, ReplayRows> prod;
     if (lane == 0) {
         prod.start(rows, gw, nw, cph, nunits, H, Dm);
 #pragma unroll
@@ -192,7 +196,7 @@ ssu_replay_kernel(const ReplayArgs a, const int cph, const int nunits)
 template <typename S, int N>
 int launch_n(const ReplayArgs &a, cudaStream_t stream)
 {
-    using G = Geo<S, N>;
+    using G = Geo<S, N, kUT>;
     const int64_t cph = (a.Dm + G::CR - 1) / G::CR;
     const int64_t nunits = (int64_t)a.active * a.H * cph;
     if (nunits == 0 || a.T == 0)

@@ -1,8 +1,8 @@
 // ssu_stream.cuh -- the per-warp streaming pipeline shared by the HBM-bound kernels
 // (decode and replay), which read every touched state row once and write it once.
 //
-// Work is cut into "units": up to kUnitRows rows (at most 32 KB) of one head of one
-// batch row's slot. Persistent CTAs of kWarps warps each run an independent pipeline:
+// Work is cut into "units": up to kUnitRows rows (and at most UT tiles) of one head of
+// one batch row's slot. Persistent CTAs of kWarps warps each run an independent pipeline:
 // warp w of the grid takes units w, w + W, w + 2W, ... (W = warps in the grid), so all
 // warps sweep the pool together in address order. A unit is cut into tiles of up to
 // kTileBytes of contiguous state; every warp owns a ring of kStages shared-memory tile
@@ -33,18 +33,19 @@ constexpr int kWarps = SSU_STREAM_WARPS;    // warps per CTA, each an independen
 constexpr int kStages = SSU_STREAM_STAGES;  // tile buffers per warp
 constexpr int kTileBytes = 4096;            // one tile: 8 warp-wide 512-byte accesses
 constexpr int kUnitRows = 128;              // at most this many rows per unit
-constexpr int kUnitTiles = 8;               // and at most 32 KB of state
 
-template <typename S, int N> struct Geo {
+// Geometry of a unit of at most UT tiles (UT * 4 KB of state) for state type S, dstate N.
+template <typename S, int N, int UT> struct Geo {
     static constexpr int VEC = Vec16<S>::kElems;                 // elements per 16 bytes
     static constexpr int LPR = (N / VEC) < 32 ? (N / VEC) : 32;  // lanes per state row
     static constexpr int E = N / LPR;                           // elements per lane and row
     static constexpr int NV = E / VEC;                          // 16-byte vectors per lane/row
     static constexpr int RPW = 32 / LPR;                        // rows per warp access
-    static constexpr int ROW_BYTES = N * (int)sizeof(S);
+    static constexpr int ELEM = (int)sizeof(S);
+    static constexpr int ROW_BYTES = N * ELEM;
     static constexpr int RT = kTileBytes / ROW_BYTES;           // rows per full tile
     static constexpr int RPT = RT / RPW;                        // row accesses per lane/tile
-    static constexpr int CR = (kUnitTiles * RT) < kUnitRows ? (kUnitTiles * RT) : kUnitRows;
+    static constexpr int CR = (UT * RT) < kUnitRows ? (UT * RT) : kUnitRows;
     static constexpr int XR = (CR + 31) / 32;                   // unit rows per lane
     static_assert(RT >= 1 && RPT >= 1 && RPT * RPW == RT, "tile geometry");
     // state column n of vector v, element e for lane-in-row ln
@@ -99,8 +100,7 @@ __device__ __forceinline__ WarpViews warp_views(uint8_t *smem, int warp)
 // Lane 0's side of a warp's pipeline. `Rows` maps a batch row to {slot, extra} and says
 // whether a unit of that row moves state:
 //   int2 resolve(int b) const;  bool moves(int2 r) const;
-template <typename S, int N, typename Rows> struct Producer {
-    using G = Geo<S, N>;
+template <typename G, int N, typename Rows> struct Producer {
     int k;        // position in this warp's unit sequence
     int j;        // next tile within the unit
     int tiles;    // tiles of the current unit
@@ -137,8 +137,9 @@ template <typename S, int N, typename Rows> struct Producer {
         if (rows.moves(cur)) {
             const int nr = min(G::RT, un.rows - j * G::RT);
             const uint32_t bytes = (uint32_t)(nr * G::ROW_BYTES);
-            const S *src = static_cast<const S *>(state) + (int64_t)cur.x * slot_stride +
-                           ((int64_t)un.h * Dm + un.row0 + j * G::RT) * N;
+            const char *src = static_cast<const char *>(state) +
+                              ((int64_t)cur.x * slot_stride +
+                               ((int64_t)un.h * Dm + un.row0 + j * G::RT) * N) * G::ELEM;
             mbar_arrive_expect_tx(&w.ctl->full[s], bytes);
             bulk_load(w.ring + s * kTileBytes, src, bytes, &w.ctl->full[s]);
         } else {
