@@ -8,32 +8,30 @@
 //
 // The state of one (row, head) stays in registers for the whole token loop, so the pool
 // is read once and (without the stash) written once; per token every state element
-// costs a multiply and two FMAs, and each output row a reduction over dstate. The kernel
-// is bound by FP32 issue, so the design minimises everything that is not an FMA:
-//   * one CTA per (batch row, head, tile of up to 128 dim rows); a lane owns R rows x K
-//     state columns (32 fp32 registers; 2 x 16 for dstate 128) in groups of 4 that
-//     interleave with those of the other lanes of its row group, so a 16-byte shared load
-//     of B or C serves R rows, covers consecutive addresses within the row group, and is
-//     a broadcast across row groups (one wavefront per load);
-//   * the update and the output partial sums use the packed two-wide FP32 instructions
-//     of sm_100 (__fmul2_rn / __ffma2_rn, element-wise round-to-nearest, so each element
-//     is computed exactly as by fmaf and the state matches the decode kernel bit for bit);
-//   * the R partial sums of a lane are reduced across the LPR lanes sharing its rows by
-//     a transposed butterfly: each step halves the values a lane holds (2 rows over 8
-//     lanes take 3 shuffles);
-//   * inputs are staged per chunk of TC tokens into double-buffered shared memory
-//     (B and C widened to fp32, x and z, dt_eff and exp(A dt_eff)); the next chunk's raw
-//     inputs are loaded into registers (as raw bits: nothing widens them before the
-//     chunk ends) before the current chunk is computed, so their latency hides behind
-//     TC tokens of arithmetic;
-//   * per-token row sums go to shared memory, and the chunk's outputs (D skip term and
-//     silu(z) gate applied) are written with coalesced stores;
-//   * the replay stash is written from the staging registers (B by one CTA per group,
-//     dA/dt by one CTA per head, U by every CTA for its rows);
+// costs a multiply and two FMAs. The kernel is bound by FP32 issue, so the design spends
+// as few instructions as possible on anything else:
+//   * a lane owns whole state rows (all N columns of R rows, 128 fp32 registers at
+//     dstate 128; above 128 columns two lanes share a row). The dstate reduction of an
+//     output row then completes inside the lane -- no shuffles -- and every lane of a
+//     warp reads the same B and C values, so each 16-byte shared load is a broadcast
+//     (one wavefront);
+//   * the update and the output sums use the packed two-wide FP32 instructions of sm_100
+//     (__fmul2_rn / __ffma2_rn, element-wise round-to-nearest, so every element is
+//     computed exactly as fmaf(s, dA, B * (dt * x)) and the state matches the decode
+//     kernel bit for bit), with two partial sums per row to shorten dependency chains;
+//   * inputs arrive per chunk of kTC tokens: B, C, x and z are fetched by the bulk-copy
+//     engine (cp.async.bulk, completion on an mbarrier, bounded waits) into a
+//     double-buffered raw stage one chunk ahead; B and C are widened to fp32 once per
+//     chunk; x and z are widened where they are used; shapes whose rows are not 16-byte
+//     aligned take a plain-load path instead;
+//   * outputs (D skip term and silu(z) gate applied) and the U stash are written by the
+//     lane that owns the row, 32 consecutive rows per warp store;
+//   * CTAs of two warps with a register budget that keeps several CTAs per SM resident,
+//     so each scheduler has more than one warp of FMAs to interleave;
 //   * CTAs take (row, head) work in order of decreasing context length (ranked in-kernel
-//     from the device lengths for batches of up to kRankMax rows, one comparison per row
-//     and thread), so the longest scans start first and the tail of the launch stays
-//     short; larger batches keep the natural order.
+//     from the device lengths for batches of up to kRankMax rows), so the longest scans
+//     start first.
+#include "ssu_async.cuh"
 #include "ssu_common.cuh"
 
 namespace ssu {
@@ -41,92 +39,58 @@ namespace {
 
 constexpr int kRankMax = 32;    // batches up to this size are scheduled longest-first
 
-// Columns of state per lane (at least N/32) and tokens per unrolled step of the scan;
-// the defaults are the measured best on B200, overridable at build time for sweeps.
-#ifndef SSU_PREFILL_K
-#define SSU_PREFILL_K 16
+// Tokens per staged chunk and the register budget (CTAs of kWarpsPerCta warps that must
+// fit kMinCtas per SM); the defaults are the measured best on B200, overridable at build
+// time for tuning sweeps.
+#ifndef SSU_PREFILL_TC
+#define SSU_PREFILL_TC 16
 #endif
-#ifndef SSU_PREFILL_UNROLL
-#define SSU_PREFILL_UNROLL 1
+#ifndef SSU_PREFILL_MIN_CTAS
+#define SSU_PREFILL_MIN_CTAS 4
 #endif
-#ifndef SSU_PREFILL_PACKED
-#define SSU_PREFILL_PACKED 1
+#ifndef SSU_PREFILL_NA
+#define SSU_PREFILL_NA 2
 #endif
-constexpr int kUnroll = SSU_PREFILL_UNROLL;
+#ifndef SSU_PREFILL_UNROLL_T
+#define SSU_PREFILL_UNROLL_T 1
+#endif
+#define SSU_STRINGIFY(x) #x
+#define SSU_PRAGMA_UNROLL(n) _Pragma(SSU_STRINGIFY(unroll n))
+constexpr int kTC = SSU_PREFILL_TC;
+constexpr int kWarpsPerCta = 2;
+constexpr int kMinCtas = SSU_PREFILL_MIN_CTAS;
 
-template <typename S, int N> struct PGeo {
-    static constexpr int KW = (N / 32) > SSU_PREFILL_K ? (N / 32) : SSU_PREFILL_K;
-    static constexpr int K = KW < N ? KW : N;                // state columns per lane
-    static constexpr int LPR = N / K;                        // lanes sharing a row
-    static constexpr int RGW = 32 / LPR;                     // row groups per warp
-    static constexpr int R = 32 / K;                         // rows per lane
-    static constexpr int RPWARP = RGW * R;                   // rows per warp
-    static constexpr int W = (128 / RPWARP) < 8 ? (128 / RPWARP) : 8;   // warps per CTA
-    static constexpr int RTC = W * RPWARP;                   // dim rows per CTA
-    static constexpr int THREADS = W * 32;
-    static constexpr int TC = N > 128 ? 8 : 16;              // tokens per staged chunk
-    // one staging buffer, in floats: B, C [TC][N]; x, z, row sums [TC][RTC]; dA, dt [TC]
-    static constexpr int OFF_C = TC * N;
-    static constexpr int OFF_X = 2 * TC * N;
-    static constexpr int OFF_Z = OFF_X + TC * RTC;
-    static constexpr int OFF_Y = OFF_Z + TC * RTC;
-    static constexpr int OFF_DA = OFF_Y + TC * RTC;
-    static constexpr int OFF_DT = OFF_DA + TC;
-    static constexpr int BUF = OFF_DT + TC;
-    static constexpr int SMEM = 2 * BUF * 4;
-    // raw staging registers per thread: 16-byte vectors of B/C, elements of x/z
-    static constexpr int VBMAX = (TC * N / 4 + THREADS - 1) / THREADS;
-    static constexpr int XPT = (TC * RTC + THREADS - 1) / THREADS;
-    static constexpr bool XREG = XPT <= 8;                   // else staged synchronously
-    static constexpr int NVF = R >= LPR ? R / LPR : 1;       // row sums a lane ends with
-    static constexpr int DUP = R >= LPR ? 1 : LPR / R;       // lanes holding the same sum
-    static constexpr int XV = R % 4 == 0 ? 4 : (R % 2 == 0 ? 2 : 1);   // x floats per load
-    // first column of the lane's q-th group of 4: the groups of the lanes of a row group
-    // interleave, so each 16-byte shared load of B or C covers consecutive addresses
-    static __device__ __forceinline__ int col(int ln, int q) { return 4 * (ln + LPR * q); }
-    static_assert(K % 4 == 0 && R * K == 32 && RTC % 4 == 0 && W >= 1, "prefill geometry");
+template <int N> struct PGeo {
+    static constexpr int LPR = N > 128 ? N / 128 : 1;        // lanes sharing a row
+    static constexpr int K = N / LPR;                        // state columns per lane
+    static constexpr int R = N >= 128 ? 1 : ((128 / N) < 4 ? (128 / N) : 4);   // rows/lane
+    static constexpr int RSTEP = 32 / LPR;                   // row stride inside a warp
+    static constexpr int RW = RSTEP * R;                     // rows per warp
+    static constexpr int NA = SSU_PREFILL_NA;                // partial sums per row
+    static_assert(K % 4 == 0 && (K / 4) % NA == 0, "prefill geometry");
 };
 
-// Transposed butterfly over the lanes of a row group: on entry v[0..NV) are this lane's
-// partial sums of NV consecutive rows; on exit v[0..) holds complete sums of the rows
-// first, first+1, ... (how many: PGeo::NVF).
-template <int NV, int OFF> struct Fold {
-    static __device__ __forceinline__ void run(float *v, int ln, int &first)
+// Shared-memory layout of one CTA, all offsets 16-byte aligned: two raw stages (B, C, x,
+// z in their storage types), B and C widened to fp32, dA and dt_eff per token, barriers.
+struct PLayout {
+    int raw_b, raw_c, raw_x, raw_z, raw_bytes;
+    int f_b, f_c, f_da, f_dt, bars, total;
+    __host__ __device__ static int up16(int v) { return (v + 15) & ~15; }
+    __host__ __device__ PLayout(int N, int rtc, int es_bc, int es_x)
     {
-        if constexpr (OFF > 0) {
-            if constexpr (NV > 1) {
-                constexpr int HALF = NV / 2;
-                const bool upper = (ln & OFF) != 0;
-#pragma unroll
-                for (int i = 0; i < HALF; ++i) {
-                    const float send = upper ? v[i] : v[i + HALF];
-                    const float keep = upper ? v[i + HALF] : v[i];
-                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
-                }
-                if (upper)
-                    first += HALF;
-                Fold<HALF, OFF / 2>::run(v, ln, first);
-            } else {
-                v[0] += __shfl_xor_sync(0xffffffffu, v[0], OFF);
-                Fold<1, OFF / 2>::run(v, ln, first);
-            }
-        }
+        raw_b = 0;
+        raw_c = up16(kTC * N * es_bc);
+        raw_x = raw_c + up16(kTC * N * es_bc);
+        raw_z = raw_x + up16(kTC * rtc * es_x);
+        raw_bytes = raw_z + up16(kTC * rtc * es_x);
+        f_b = 2 * raw_bytes;
+        f_c = f_b + kTC * N * 4;
+        f_da = f_c + kTC * N * 4;
+        f_dt = f_da + kTC * 4;
+        bars = up16(f_dt + kTC * 4);
+        total = bars + 16;
     }
 };
-
-__device__ __forceinline__ void widen16(const uint4 &q, int dtype, float *f)
-{
-    if (dtype == SSU_F32) {
-        f[0] = __uint_as_float(q.x);
-        f[1] = __uint_as_float(q.y);
-        f[2] = __uint_as_float(q.z);
-        f[3] = __uint_as_float(q.w);
-    } else if (dtype == SSU_BF16) {
-        Vec16<__nv_bfloat16>::unpack(q, f);
-    } else {
-        Vec16<__half>::unpack(q, f);
-    }
-}
 
 // Length used for scheduling: padding and out-of-range rows do (almost) no work.
 __device__ __forceinline__ int sched_len(const PrefillArgs &pa, int b)
@@ -139,17 +103,26 @@ __device__ __forceinline__ int sched_len(const PrefillArgs &pa, int b)
 }
 
 template <typename S, int N>
-__global__ void __launch_bounds__(PGeo<S, N>::THREADS)
-ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
+__global__ void __launch_bounds__(kWarpsPerCta * 32, kMinCtas)
+ssu_prefill_kernel(const PrefillArgs pa, const int dtiles, const int rtc, const int bulk)
 {
-    using P = PGeo<S, N>;
-    extern __shared__ __align__(16) float sm[];
+    using P = PGeo<N>;
+    extern __shared__ __align__(16) uint8_t sm[];
     __shared__ int s_row;
     __shared__ int s_len[kRankMax];
 
     const DecodeArgs &a = pa.d;
     const int H = a.H, Dm = a.Dm, T = pa.T, G = a.G;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nthreads = blockDim.x;
+    const int es_bc = a.bc_dtype == SSU_F32 ? 4 : 2;
+    const int es_x = a.x_dtype == SSU_F32 ? 4 : 2;
+    const PLayout lay(N, rtc, es_bc, es_x);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + lay.bars);
+    float *fB = reinterpret_cast<float *>(sm + lay.f_b);
+    float *fC = reinterpret_cast<float *>(sm + lay.f_c);
+    float *sdA = reinterpret_cast<float *>(sm + lay.f_da);
+    float *sdt = reinterpret_cast<float *>(sm + lay.f_dt);
 
     // ---- which (row, head, dim tile): rows ranked by decreasing length
     const int per_row = H * dtiles;
@@ -173,14 +146,14 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
         b = s_row;
     }
 
-    const int row0 = dtile * P::RTC;
+    const int row0 = dtile * rtc;
+    const int rows_c = min(rtc, Dm - row0);
     const bool reporter = tid == 0 && dtile == 0 && h == 0;
     const int slot = a.idx ? a.idx[b] : b;
     if (slot < 0) {                    // padding row: zero outputs at every position
-        for (int i = tid; i < T * P::RTC; i += P::THREADS) {
-            const int t = i / P::RTC, row = row0 + i % P::RTC;
-            if (row < Dm)
-                st_f32(a.out, a.x_dtype, (((int64_t)b * T + t) * H + h) * Dm + row, 0.f);
+        for (int i = tid; i < T * rows_c; i += nthreads) {
+            const int t = i / rows_c, row = row0 + i % rows_c;
+            st_f32(a.out, a.x_dtype, (((int64_t)b * T + t) * H + h) * Dm + row, 0.f);
         }
         return;
     }
@@ -209,226 +182,222 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
     const bool write_head = stash && dtile == 0;
     const float Ah = a.A[h];
     const float Dh = a.D ? a.D[h] : 0.f;
+    const char *Bg = static_cast<const char *>(a.B);
+    const char *Cg = static_cast<const char *>(a.C);
+    const char *Xg = static_cast<const char *>(a.x);
+    const char *Zg = static_cast<const char *>(a.z);
 
-    // ---- this lane's rows and columns
-    const int rg = lane / P::LPR, ln = lane % P::LPR;
-    const int lrow = warp * P::RPWARP + rg * P::R;      // first local row of the lane
+    // ---- fetch chunk c (tokens c*kTC ..) into raw stage c & 1
+    auto fetch = [&](int c) {
+        uint8_t *raw = sm + (c & 1) * lay.raw_bytes;
+        const int t0 = c * kTC, nt = min(kTC, L - t0);
+        const int64_t bt0 = (int64_t)b * T + t0;
+        if (bulk) {                    // one thread drives the copy engine
+            if (tid == 0) {
+                uint64_t *bar = &full[c & 1];
+                const uint32_t nb = (uint32_t)(N * es_bc), nx = (uint32_t)(rows_c * es_x);
+                mbar_arrive_expect_tx(bar, 2u * nt * nb + (a.z ? 2u : 1u) * nt * nx);
+                if (G == 1) {
+                    bulk_load(raw + lay.raw_b, Bg + bt0 * nb, nt * nb, bar);
+                    bulk_load(raw + lay.raw_c, Cg + bt0 * nb, nt * nb, bar);
+                } else {
+                    for (int t = 0; t < nt; ++t) {
+                        const int64_t off = ((bt0 + t) * G + g) * nb;
+                        bulk_load(raw + lay.raw_b + t * nb, Bg + off, nb, bar);
+                        bulk_load(raw + lay.raw_c + t * nb, Cg + off, nb, bar);
+                    }
+                }
+                for (int t = 0; t < nt; ++t) {
+                    const int64_t off = (((bt0 + t) * H + h) * Dm + row0) * es_x;
+                    bulk_load(raw + lay.raw_x + t * rtc * es_x, Xg + off, nx, bar);
+                    if (a.z)
+                        bulk_load(raw + lay.raw_z + t * rtc * es_x, Zg + off, nx, bar);
+                }
+            }
+        } else {                       // rows not 16-byte aligned: plain loads, synchronous
+            for (int i = tid; i < nt * N; i += nthreads) {
+                const int t = i / N, n = i % N;
+                const int64_t off = ((bt0 + t) * G + g) * N + n;
+                memcpy(raw + lay.raw_b + (t * N + n) * es_bc, Bg + off * es_bc, es_bc);
+                memcpy(raw + lay.raw_c + (t * N + n) * es_bc, Cg + off * es_bc, es_bc);
+            }
+            for (int i = tid; i < nt * rows_c; i += nthreads) {
+                const int t = i / rows_c, r = i % rows_c;
+                const int64_t off = ((bt0 + t) * H + h) * Dm + row0 + r;
+                memcpy(raw + lay.raw_x + (t * rtc + r) * es_x, Xg + off * es_x, es_x);
+                if (a.z)
+                    memcpy(raw + lay.raw_z + (t * rtc + r) * es_x, Zg + off * es_x, es_x);
+            }
+        }
+    };
+
+    if (tid == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // ---- this lane's rows and columns: rows rbase + i*RSTEP, float4 groups q*LPR + ln
+    const int ln = lane % P::LPR;
+    const int rbase = warp * P::RW + lane / P::LPR;
     S *base = static_cast<S *>(a.state) + (int64_t)slot * a.slot_stride + (int64_t)h * Dm * N;
-
     float2 st[P::R][P::K / 2];
 #pragma unroll
     for (int i = 0; i < P::R; ++i) {
-        const int row = row0 + lrow + i;
+        const int r = rbase + i * P::RSTEP;
+        const bool in = r < rows_c;
 #pragma unroll
         for (int q = 0; q < P::K / 4; ++q) {
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (row < Dm)
-                v = Quad<S>::load(base + (int64_t)row * N + P::col(ln, q));
+            if (in)
+                v = Quad<S>::load(base + (int64_t)(row0 + r) * N + 4 * (q * P::LPR + ln));
             st[i][2 * q] = make_float2(v.x, v.y);
             st[i][2 * q + 1] = make_float2(v.z, v.w);
         }
     }
 
-    // ---- staging of one chunk: raw loads into registers, then widen into a buffer
-    uint4 rb[P::VBMAX], rc[P::VBMAX];
-    uint32_t rx[P::XREG ? P::XPT : 1], rz[P::XREG ? P::XPT : 1];   // raw bits of x and z
-    float rdt = 0.f;
-    const int vb = 16 / (a.bc_dtype == SSU_F32 ? 4 : 2);   // B/C elements per 16 bytes
-    const int nvec = P::TC * N / vb;
+    const int nchunks = (L + kTC - 1) / kTC;
+    fetch(0);
+    if (nchunks > 1)
+        fetch(1);
+    float rdt = 0.f;                                     // dt of the coming chunk (tid < kTC)
+    if (tid < kTC && tid < L)
+        rdt = a.dt[((int64_t)b * T + tid) * H + h];
+    const int ve = 16 / es_bc;                           // B/C elements per 16 bytes
 
-    auto load_chunk = [&](int t0) {
-#pragma unroll
-        for (int k = 0; k < P::VBMAX; ++k) {
-            const int q = tid + k * P::THREADS;
-            const int e = q * vb, t = e / N, n = e % N;
-            if (q < nvec && t0 + t < L) {
-                const int64_t off = (((int64_t)b * T + t0 + t) * G + g) * N + n;
-                const int es = a.bc_dtype == SSU_F32 ? 4 : 2;
-                rb[k] = *reinterpret_cast<const uint4 *>(static_cast<const char *>(a.B) + off * es);
-                rc[k] = *reinterpret_cast<const uint4 *>(static_cast<const char *>(a.C) + off * es);
-            }
-        }
-        if constexpr (P::XREG) {
-#pragma unroll
-            for (int k = 0; k < P::XPT; ++k) {
-                const int e = tid + k * P::THREADS;
-                const int t = e / P::RTC, row = row0 + e % P::RTC;
-                rx[k] = 0u;                         // zero bits are 0.0 in every format
-                rz[k] = 0u;
-                if (e < P::TC * P::RTC && t0 + t < L && row < Dm) {
-                    const int64_t xi = (((int64_t)b * T + t0 + t) * H + h) * Dm + row;
-                    rx[k] = ld_bits(a.x, a.x_dtype, xi);
-                    if (a.z)
-                        rz[k] = ld_bits(a.z, a.x_dtype, xi);
+    for (int c = 0; c < nchunks; ++c) {
+        const int t0 = c * kTC, nt = min(kTC, L - t0);
+        const uint8_t *raw = sm + (c & 1) * lay.raw_bytes;
+        if (bulk) {
+            if (!__syncthreads_and(mbar_wait(&full[c & 1], (uint32_t)(c >> 1) & 1u))) {
+                // Never expected: report, let the copies already started land, stop.
+                if (tid == 0) {
+                    if (a.err)
+                        atomicOr(a.err, SSU_FLAG_TIMEOUT);
+                    for (int cc = c; cc < min(c + 2, nchunks); ++cc)
+                        if (!mbar_wait(&full[cc & 1], (uint32_t)(cc >> 1) & 1u))
+                            break;
                 }
+                return;
+            }
+        } else {
+            __syncthreads();
+        }
+        // ---- widen B and C (16 bytes at a time), finish dt and dA, write the token stash
+        for (int i = tid * ve; i < nt * N; i += nthreads * ve) {
+            float fb[8], fc[8];
+            const uint4 qb = *reinterpret_cast<const uint4 *>(raw + lay.raw_b + i * es_bc);
+            const uint4 qc = *reinterpret_cast<const uint4 *>(raw + lay.raw_c + i * es_bc);
+            if (a.bc_dtype == SSU_F32) {
+                Vec16<float>::unpack(qb, fb);
+                Vec16<float>::unpack(qc, fc);
+            } else if (a.bc_dtype == SSU_BF16) {
+                Vec16<__nv_bfloat16>::unpack(qb, fb);
+                Vec16<__nv_bfloat16>::unpack(qc, fc);
+            } else {
+                Vec16<__half>::unpack(qb, fb);
+                Vec16<__half>::unpack(qc, fc);
+            }
+            for (int e = 0; e < ve; e += 4) {
+                const float4 b4 = make_float4(fb[e], fb[e + 1], fb[e + 2], fb[e + 3]);
+                *reinterpret_cast<float4 *>(fB + i + e) = b4;
+                *reinterpret_cast<float4 *>(fC + i + e) =
+                    make_float4(fc[e], fc[e + 1], fc[e + 2], fc[e + 3]);
+                if (write_group)
+                    *reinterpret_cast<float4 *>(
+                        pa.st_B + (((int64_t)b * T + t0 + (i + e) / N) * G + g) * N +
+                        (i + e) % N) = b4;
             }
         }
-        if (tid < P::TC && t0 + tid < L)
-            rdt = a.dt[((int64_t)b * T + t0 + tid) * H + h];
-    };
-
-    auto store_chunk = [&](int t0, float *buf) {
-#pragma unroll
-        for (int k = 0; k < P::VBMAX; ++k) {
-            const int q = tid + k * P::THREADS;
-            const int e = q * vb, t = e / N, n = e % N;
-            if (q < nvec && t0 + t < L) {
-                float fb[8], fc[8];
-                widen16(rb[k], a.bc_dtype, fb);
-                widen16(rc[k], a.bc_dtype, fc);
-                for (int i = 0; i < vb; i += 4) {
-                    const float4 b4 = make_float4(fb[i], fb[i + 1], fb[i + 2], fb[i + 3]);
-                    *reinterpret_cast<float4 *>(buf + t * N + n + i) = b4;
-                    *reinterpret_cast<float4 *>(buf + P::OFF_C + t * N + n + i) =
-                        make_float4(fc[i], fc[i + 1], fc[i + 2], fc[i + 3]);
-                    if (write_group)
-                        *reinterpret_cast<float4 *>(
-                            pa.st_B + (((int64_t)b * T + t0 + t) * G + g) * N + n + i) = b4;
-                }
-            }
-        }
-        for (int k = 0; k < P::XPT; ++k) {
-            const int e = tid + k * P::THREADS;
-            if (e >= P::TC * P::RTC)
-                break;
-            const int t = e / P::RTC, r = e % P::RTC, row = row0 + r;
-            float xv = 0.f, zv = 0.f;
-            const bool in = t0 + t < L && row < Dm;
-            const int64_t xi = (((int64_t)b * T + t0 + t) * H + h) * Dm + row;
-            if constexpr (P::XREG) {
-                xv = bits_f32(rx[k], a.x_dtype);
-                zv = bits_f32(rz[k], a.x_dtype);
-            } else if (in) {
-                xv = ld_f32(a.x, a.x_dtype, xi);
-                if (a.z)
-                    zv = ld_f32(a.z, a.x_dtype, xi);
-            }
-            buf[P::OFF_X + t * P::RTC + r] = xv;
-            buf[P::OFF_Z + t * P::RTC + r] = zv;
-            if (stash && in)
-                pa.st_U[xi] = xv;
-        }
-        if (tid < P::TC && t0 + tid < L) {
+        if (tid < nt) {
             const int64_t bth = ((int64_t)b * T + t0 + tid) * H + h;
             const float dte = effective_dt(rdt, a.dt_bias, h, a.softplus);
             const float dA = expf(Ah * dte);
-            buf[P::OFF_DT + tid] = dte;
-            buf[P::OFF_DA + tid] = dA;
+            sdt[tid] = dte;
+            sdA[tid] = dA;
             if (write_head) {
                 pa.st_dA[bth] = dA;
                 pa.st_dt[bth] = dte;
             }
+            if (t0 + kTC + tid < L)                      // prefetch the next chunk's dt
+                rdt = a.dt[((int64_t)b * T + t0 + kTC + tid) * H + h];
         }
-    };
-
-    load_chunk(0);
-    store_chunk(0, sm);
-    __syncthreads();
-
-    for (int c = 0, t0 = 0; t0 < L; ++c, t0 += P::TC) {
-        float *cur = sm + (c & 1) * P::BUF;
-        float *nxt = sm + ((c & 1) ^ 1) * P::BUF;
-        const int nt = min(P::TC, L - t0);
-        const bool more = t0 + P::TC < L;
-        if (more)
-            load_chunk(t0 + P::TC);            // in flight during this chunk's arithmetic
+        __syncthreads();
 
         // ---- the recurrence, token by token, state in registers
-        auto token = [&](const int t) {
-            const float dA = cur[P::OFF_DA + t];
-            const float dte = cur[P::OFF_DT + t];
+        SSU_PRAGMA_UNROLL(SSU_PREFILL_UNROLL_T)
+        for (int t = 0; t < nt; ++t) {
+            const float dA = sdA[t];
+            const float dte = sdt[t];
             const float2 dA2 = make_float2(dA, dA);
-            float2 B2[P::K / 2], C2[P::K / 2];
-#pragma unroll
-            for (int q = 0; q < P::K / 4; ++q) {
-                const float4 b4 = *reinterpret_cast<const float4 *>(cur + t * N + P::col(ln, q));
-                const float4 c4 =
-                    *reinterpret_cast<const float4 *>(cur + P::OFF_C + t * N + P::col(ln, q));
-                B2[2 * q] = make_float2(b4.x, b4.y);
-                B2[2 * q + 1] = make_float2(b4.z, b4.w);
-                C2[2 * q] = make_float2(c4.x, c4.y);
-                C2[2 * q + 1] = make_float2(c4.z, c4.w);
-            }
             float xv[P::R];
-            const float *xt = cur + P::OFF_X + t * P::RTC + lrow;
-#pragma unroll
-            for (int q = 0; q < P::R; q += P::XV) {
-                if constexpr (P::XV == 4) {
-                    const float4 x4 = *reinterpret_cast<const float4 *>(xt + q);
-                    xv[q] = x4.x;
-                    xv[q + 1] = x4.y;
-                    xv[q + 2] = x4.z;
-                    xv[q + 3] = x4.w;
-                } else if constexpr (P::XV == 2) {
-                    const float2 x2 = *reinterpret_cast<const float2 *>(xt + q);
-                    xv[q] = x2.x;
-                    xv[q + 1] = x2.y;
-                } else {
-                    xv[q] = xt[q];
-                }
-            }
-            float part[P::R];
+            float2 d2[P::R];
+            float2 acc[P::R][P::NA];
 #pragma unroll
             for (int i = 0; i < P::R; ++i) {
+                const int r = rbase + i * P::RSTEP;
+                xv[i] = r < rows_c ? ld_f32(raw + lay.raw_x, a.x_dtype, t * rtc + r) : 0.f;
                 const float dtx = dte * xv[i];
-                const float2 d2 = make_float2(dtx, dtx);
-                float2 acc = make_float2(0.f, 0.f);
+                d2[i] = make_float2(dtx, dtx);
 #pragma unroll
-                for (int k = 0; k < P::K / 2; ++k) {
-#if SSU_PREFILL_PACKED
-                    st[i][k] = __ffma2_rn(st[i][k], dA2, __fmul2_rn(B2[k], d2));
-                    acc = __ffma2_rn(st[i][k], C2[k], acc);
-#else
-                    st[i][k].x = fmaf(st[i][k].x, dA, B2[k].x * dtx);
-                    st[i][k].y = fmaf(st[i][k].y, dA, B2[k].y * dtx);
-                    acc.x = fmaf(st[i][k].x, C2[k].x, acc.x);
-                    acc.y = fmaf(st[i][k].y, C2[k].y, acc.y);
-#endif
+                for (int j = 0; j < P::NA; ++j)
+                    acc[i][j] = make_float2(0.f, 0.f);
+            }
+            const float *Bt = fB + t * N;
+            const float *Ct = fC + t * N;
+#pragma unroll
+            for (int q = 0; q < P::K / 4; ++q) {
+                const float4 b4 = *reinterpret_cast<const float4 *>(Bt + 4 * (q * P::LPR + ln));
+                const float4 c4 = *reinterpret_cast<const float4 *>(Ct + 4 * (q * P::LPR + ln));
+                const float2 b01 = make_float2(b4.x, b4.y), b23 = make_float2(b4.z, b4.w);
+                const float2 c01 = make_float2(c4.x, c4.y), c23 = make_float2(c4.z, c4.w);
+#pragma unroll
+                for (int i = 0; i < P::R; ++i) {
+                    st[i][2 * q] = __ffma2_rn(st[i][2 * q], dA2, __fmul2_rn(b01, d2[i]));
+                    st[i][2 * q + 1] = __ffma2_rn(st[i][2 * q + 1], dA2, __fmul2_rn(b23, d2[i]));
+                    acc[i][q % P::NA] = __ffma2_rn(st[i][2 * q], c01, acc[i][q % P::NA]);
+                    acc[i][q % P::NA] = __ffma2_rn(st[i][2 * q + 1], c23, acc[i][q % P::NA]);
                 }
-                part[i] = acc.x + acc.y;
             }
-            int first = 0;
-            Fold<P::R, P::LPR / 2>::run(part, ln, first);
-            if (ln % P::DUP == 0) {
 #pragma unroll
-                for (int i = 0; i < P::NVF; ++i)
-                    cur[P::OFF_Y + t * P::RTC + lrow + first + i] = part[i];
-            }
-        };
-        int t = 0;
-        for (; t + kUnroll <= nt; t += kUnroll) {
+            for (int i = 0; i < P::R; ++i) {
+                float y = 0.f;
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u)
-                token(t + u);
-        }
-        for (; t < nt; ++t)
-            token(t);
-        __syncthreads();                         // row sums of this chunk complete
-
-        // ---- outputs of the chunk: skip term and gate, coalesced along dim
-        for (int i = tid; i < nt * P::RTC; i += P::THREADS) {
-            const int t = i / P::RTC, r = i % P::RTC, row = row0 + r;
-            if (row < Dm) {
-                float y = cur[P::OFF_Y + t * P::RTC + r] + Dh * cur[P::OFF_X + t * P::RTC + r];
-                if (a.z)
-                    y *= silu_f(cur[P::OFF_Z + t * P::RTC + r]);
-                st_f32(a.out, a.x_dtype, (((int64_t)b * T + t0 + t) * H + h) * Dm + row, y);
+                for (int j = 0; j < P::NA; ++j)
+                    y += acc[i][j].x + acc[i][j].y;
+                if constexpr (P::LPR > 1)
+                    y += __shfl_xor_sync(0xffffffffu, y, 1);
+                const int r = rbase + i * P::RSTEP;
+                if (ln == 0 && r < rows_c) {
+                    const int64_t xi = (((int64_t)b * T + t0 + t) * H + h) * Dm + row0 + r;
+                    y += Dh * xv[i];
+                    if (a.z) {
+                        // silu(z) = z * sigmoid(z), with the fast exponential and division
+                        // (relative error ~1e-7, far inside the output tolerance)
+                        const float zv = ld_f32(raw + lay.raw_z, a.x_dtype, t * rtc + r);
+                        y *= __fdividef(zv, 1.f + __expf(-zv));
+                    }
+                    st_f32(a.out, a.x_dtype, xi, y);
+                    if (stash)
+                        pa.st_U[xi] = xv[i];
+                }
             }
         }
-        if (more)
-            store_chunk(t0 + P::TC, nxt);
-        __syncthreads();                         // next chunk staged; this one consumed
+        __syncthreads();                                 // raw stage c & 1 and fB/fC free
+        if (c + 2 < nchunks)
+            fetch(c + 2);
     }
 
     // ---- final state, once (the stash mode leaves the committed state read-only)
     if (!stash) {
 #pragma unroll
         for (int i = 0; i < P::R; ++i) {
-            const int row = row0 + lrow + i;
-            if (row < Dm) {
+            const int r = rbase + i * P::RSTEP;
+            if (r < rows_c) {
 #pragma unroll
                 for (int q = 0; q < P::K / 4; ++q)
-                    Quad<S>::store(base + (int64_t)row * N + P::col(ln, q),
+                    Quad<S>::store(base + (int64_t)(row0 + r) * N + 4 * (q * P::LPR + ln),
                                    make_float4(st[i][2 * q].x, st[i][2 * q].y,
                                                st[i][2 * q + 1].x, st[i][2 * q + 1].y));
             }
@@ -436,26 +405,40 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles)
     }
 }
 
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 template <typename S, int N>
 int launch_n(const PrefillArgs &a, cudaStream_t s)
 {
-    using P = PGeo<S, N>;
-    const int64_t dtiles = (a.d.Dm + P::RTC - 1) / P::RTC;
+    using P = PGeo<N>;
+    const int Dm = a.d.Dm;
+    const int warps = kWarpsPerCta;
+    const int rtc = warps * P::RW;
+    const int64_t dtiles = (Dm + rtc - 1) / rtc;
     const int64_t grid = (int64_t)a.d.active * a.d.H * dtiles;
     if (grid == 0 || a.T == 0)
         return SSU_OK;
     if (grid > 0x7fffffffLL)
         return SSU_ERR_SHAPE;
-    static bool configured[64];
+    const int es_bc = a.d.bc_dtype == SSU_F32 ? 4 : 2;
+    const int es_x = a.d.x_dtype == SSU_F32 ? 4 : 2;
+    // Bulk copies need 16-byte aligned rows: B/C rows always are (N >= 8 elements of at
+    // least 2 bytes, 16-byte aligned base checked by the caller); x/z rows are when Dm
+    // and the dim tile are multiples of 16 bytes.
+    const int bulk = aligned16(a.d.x) && (!a.d.z || aligned16(a.d.z)) &&
+                     (Dm * es_x) % 16 == 0 && (rtc * es_x) % 16 == 0;
+    const PLayout lay(N, rtc, es_bc, es_x);
+    static int configured[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         dev = 0;
-    if (!configured[dev]) {
+    if (configured[dev] < lay.total) {
         cudaFuncSetAttribute(ssu_prefill_kernel<S, N>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
-        configured[dev] = true;
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+        configured[dev] = lay.total;
     }
-    ssu_prefill_kernel<S, N><<<(unsigned)grid, P::THREADS, P::SMEM, s>>>(a, (int)dtiles);
+    ssu_prefill_kernel<S, N><<<(unsigned)grid, warps * 32, lay.total, s>>>(a, (int)dtiles, rtc,
+                                                                          bulk);
     return SSU_OK;
 }
 
