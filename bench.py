@@ -376,6 +376,81 @@ def form_replay(args, device, hbm_peak, batch=0):
                      "frac": rbytes / (ms / 1e3) / 1e9 / hbm_peak, "traffic": None}}}
 
 
+def form_layers(args, device, hbm_peak):
+    """Multi-layer launches and row movement on one GPU: the speculative replay over 8
+    layers in one launch, the gather of the batch-256 decode rows into a dense batch, and
+    the clear of one slot across 64 layers. All HBM bound."""
+    from linear_attention_recurrent_selective_b200 import ssu
+    from linear_attention_recurrent_selective_b200.workloads import make_config
+
+    steps, warm = max(3, min(args.steps, 50)), max(3, min(args.warmup, 5))
+    forms = {}
+    f = dict(dtype=torch.float32, device=device)
+
+    # replay over 8 layers: each layer has its own pool and stash (stash from this
+    # library's prefill in stash mode, one per layer)
+    layers = 8
+    rcase = make_config("spec_replay_b64_t5")
+    rd = rcase.to(device)
+    b, T, H, G, Dm, N = rcase.batch, rcase.T, rcase.H, rcase.G, rcase.Dm, rcase.N
+    pools, stashes = [], []
+    for _ in range(layers):
+        pool = rd.pool.clone()
+        st = (torch.empty(b, T, H, **f), torch.empty(b, T, H, Dm, **f),
+              torch.empty(b, T, G, N, **f), torch.empty(b, T, H, **f))
+        ssu.ssu_prefill(rd.x, rd.A, rd.B, rd.C, rd.dt, pool, torch.empty_like(rd.x),
+                        dt_bias=rd.dt_bias, D=rd.D, z=rd.z, state_indices=rd.state_indices,
+                        stash=st, slot_stride=rcase.slot_stride, P=rcase.P)
+        pools.append(pool)
+        stashes.append(st)
+    table = ssu.replay_layer_table(list(zip(pools, stashes)))
+    acc = rd.accepted_lengths
+    ms = time_launches(lambda: ssu.ssu_replay_layers(table, layers, pools[0], stashes[0], acc,
+                                                     state_indices=rd.state_indices,
+                                                     slot_stride=rcase.slot_stride, P=rcase.P),
+                       steps, warm, device)
+    acc_h = rcase.accepted_lengths
+    rows, nacc = int((acc_h > 0).sum()), int(acc_h.sum())
+    per_layer = rows * H * Dm * N * 4 * 2 + nacc * (H * (4 + 4 + Dm * 4) + G * N * 4) + b * 4
+    forms["replay_layers"] = {
+        "workload": "spec_replay_b64_t5 x 8 layers", "ms_per_launch": ms,
+        "accepted_tokens_per_s": layers * nacc / (ms / 1e3),
+        "roofline": {"bound": "hbm", "achieved": layers * per_layer / (ms / 1e3) / 1e9,
+                     "peak": hbm_peak, "unit": "GB/s",
+                     "frac": layers * per_layer / (ms / 1e3) / 1e9 / hbm_peak, "traffic": None}}
+    del pools, stashes, table
+
+    # gather of the 256 active rows of the batch-256 decode pool (2.6 MB slots)
+    dcase = make_config(WORKLOAD)
+    dpool = dcase.pool.to(device).view(dcase.P, dcase.slot_stride)
+    dense = torch.empty(dcase.batch, dcase.slot_stride, **f)
+    idx = dcase.state_indices.to(device)
+    ms = time_launches(lambda: ssu.pool_gather(dpool, dense, state_indices=idx), steps, warm,
+                       device)
+    gbytes = 2 * dense.numel() * 4
+    forms["gather"] = {
+        "workload": "mamba2_decode_b256 rows -> dense batch", "ms_per_launch": ms,
+        "roofline": {"bound": "hbm", "achieved": gbytes / (ms / 1e3) / 1e9, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": gbytes / (ms / 1e3) / 1e9 / hbm_peak,
+                     "traffic": None}}
+    del dpool, dense
+
+    # clear one slot (2.6 MB of state, 40 KB of conv state) across 64 layers
+    nl, P, slot_elems, conv_elems = 64, 4, 80 * 64 * 128, 10240
+    recs = [torch.ones(P, slot_elems, **f) for _ in range(nl)]
+    convs = [torch.ones(P, conv_elems, dtype=torch.bfloat16, device=device) for _ in range(nl)]
+    ltab = ssu.layer_states_table(list(zip(recs, convs)))
+    ms = time_launches(lambda: ssu.pool_clear_slot_layers(ltab, nl, P, 1, slot_elems * 4,
+                                                          conv_elems * 2), steps, warm, device)
+    cbytes = nl * (slot_elems * 4 + conv_elems * 2)
+    forms["clear_layers"] = {
+        "workload": "one slot x 64 layers (fp32 state + bf16 conv)", "ms_per_launch": ms,
+        "roofline": {"bound": "hbm", "achieved": cbytes / (ms / 1e3) / 1e9, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": cbytes / (ms / 1e3) / 1e9 / hbm_peak,
+                     "traffic": None}}
+    return forms
+
+
 def cpu_baseline_decode(case, max_seconds=20.0):
     """The float64 oracle on whole decode steps of the same workload, timed on this host."""
     from oracle import oracle
@@ -413,9 +488,13 @@ def main_ours(args):
     device = torch.device("cuda", local if n_world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(device)
     hbm_peak, peak_src = measured_peaks()
-    if args.form in ("prefill", "replay"):       # one kernel alone, e.g. under a profiler
-        forms = (form_prefill(args, device, args.batch) if args.form == "prefill"
-                 else form_replay(args, device, hbm_peak, args.batch))
+    if args.form in ("prefill", "replay", "layers"):   # one form alone, e.g. under ncu
+        if args.form == "prefill":
+            forms = form_prefill(args, device, args.batch)
+        elif args.form == "replay":
+            forms = form_replay(args, device, hbm_peak, args.batch)
+        else:
+            forms = form_layers(args, device, hbm_peak)
         if rank == 0:
             print(json.dumps({"form": args.form, "forms": forms}), flush=True)
         return
@@ -446,7 +525,8 @@ def main_ours(args):
         "clocks": res["clocks"],
     }
     if n_world == 1 and not args.no_forms and args.form == "all":
-        line["forms"] = {**form_prefill(args, device), **form_replay(args, device, hbm_peak)}
+        line["forms"] = {**form_prefill(args, device), **form_replay(args, device, hbm_peak),
+                         **form_layers(args, device, hbm_peak)}
     if n_world == 1 and rank == 0 and not args.no_cpu_baseline and args.form == "all":
         line["cpu_baseline"] = cpu_baseline_decode(case)
     if rank == 0:
@@ -503,7 +583,8 @@ def parse(argv=None):
     ap.add_argument("--batch", type=int, default=0,
                     help="override the batch (pool = 2 x batch), e.g. for a small profile")
     ap.add_argument("--no-forms", action="store_true", help="skip the prefill/replay forms")
-    ap.add_argument("--form", choices=("all", "decode", "prefill", "replay"), default="all",
+    ap.add_argument("--form", choices=("all", "decode", "prefill", "replay", "layers"),
+                    default="all",
                     help="run one kernel only (for profiling); its line carries that form")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args(argv)

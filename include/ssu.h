@@ -77,9 +77,29 @@ enum {
     SSU_FLAG_ACCEPTED_RANGE = 2,  /* accepted_lengths[b] > T: clamped to T */
     SSU_FLAG_CONTEXT_RANGE = 4,   /* context_lengths[b] > T: clamped to T */
     SSU_FLAG_NEGATIVE_LENGTH = 8, /* a negative length: treated as 0 */
-    SSU_FLAG_TIMEOUT = 16         /* an internal wait gave up after 2 s (never expected);
+    SSU_FLAG_TIMEOUT = 16,        /* an internal wait gave up after 2 s (never expected);
                                      the outputs of that launch are incomplete */
+    SSU_FLAG_LAYER = 32           /* a per-layer pointer was NULL or not 16-byte aligned:
+                                     that layer was skipped */
 };
+
+/* Per-layer device pointers of a multi-layer replay: one entry per layer, in a device
+ * array (Selective State Update page, struct MambaReplayLayerInfo). All layers share the
+ * geometry, slot stride and pool size given to the call. */
+typedef struct {
+    void *state;          /* the layer's pool [P, H, Dm, N], 16-byte aligned */
+    const float *st_dA;   /* the layer's replay stash, as written by ssu_prefill */
+    const float *st_U;
+    const float *st_B;    /* 16-byte aligned */
+    const float *st_dt;
+} ssu_replay_layer;
+
+/* Per-layer device pointers of the recurrent and convolution states (Selective State
+ * Update page, struct MambaStateLayerInfo), for the multi-layer slot clear. */
+typedef struct {
+    void *recurrent_state;
+    void *conv_state;     /* may be NULL: the layer has no convolution state */
+} ssu_layer_states;
 
 /*
  * ssu_decode -- one token (seq_len == 1) for every active row.
@@ -151,6 +171,21 @@ int ssu_replay(void *state, int state_dtype, int64_t slot_stride, int32_t P,
                int32_t *err_flags, ssu_stream_t stream);
 
 /*
+ * ssu_replay_layers -- ssu_replay over num_layers layers in one launch.
+ * Selective State Update page, invokeMambaReplayReconstructBatched with a device array of
+ * MambaReplayLayerInfo: every layer re-applies the first accepted_lengths[b] tokens of its
+ * own stash to its own pool; accepted_lengths and state_indices are shared by the layers.
+ *   layers      device array [num_layers] of ssu_replay_layer
+ *   other arguments as in ssu_replay (their geometry applies to every layer)
+ * A layer whose pointers are NULL or misaligned is skipped and flagged SSU_FLAG_LAYER.
+ */
+int ssu_replay_layers(const ssu_replay_layer *layers, int32_t num_layers, int state_dtype,
+                      int64_t slot_stride, int32_t P, const int32_t *accepted_lengths,
+                      const int32_t *state_indices, int32_t batch, int32_t active_batch,
+                      int32_t T, int32_t nheads, int32_t ngroups, int32_t dim, int32_t dstate,
+                      int32_t *err_flags, ssu_stream_t stream);
+
+/*
  * pool_clear_slot -- zero one slot, or every slot when slot == -1.
  * Selective State Update page, invokeMambaStateClear; Recurrent State Manager page,
  * clearSlot / clear. slot_bytes is the slot stride in bytes; other slots are untouched.
@@ -169,6 +204,34 @@ int pool_clear_slot(void *pool, int64_t slot_bytes, int32_t P, int32_t slot,
 int pool_copy_slot(void *dst_pool, int32_t dst_P, int32_t dst_slot,
                    const void *src_pool, int32_t src_P, int32_t src_slot,
                    int64_t slot_bytes, ssu_stream_t stream);
+
+/*
+ * pool_clear_slot_layers -- pool_clear_slot over the recurrent and convolution states of
+ * num_layers layers in one launch. Selective State Update page, invokeMambaStateClear.
+ *   layers                device array [num_layers] of ssu_layer_states
+ *   recurrent_slot_bytes  slot stride of every recurrent pool, in bytes
+ *   conv_slot_bytes       slot stride of every convolution pool (0: none)
+ * Returns SSU_ERR_SHAPE for slot < -1 or slot >= P.
+ */
+int pool_clear_slot_layers(const ssu_layer_states *layers, int32_t num_layers, int32_t P,
+                           int32_t slot, int64_t recurrent_slot_bytes, int64_t conv_slot_bytes,
+                           ssu_stream_t stream);
+
+/*
+ * pool_gather / pool_scatter -- copy active rows between the pool and a dense batch.
+ * Selective State Update page, invokeMambaStateGather / invokeMambaStateScatter: for
+ * b < active_batch, dense[b] = pool[state_indices[b]] (gather) or
+ * pool[state_indices[b]] = dense[b] (scatter); rows are slot_bytes long, dense rows are
+ * contiguous ([batch, slot_bytes]), pool rows sit slot_bytes apart.
+ * A padding row (negative index): gather writes zeros to dense[b], scatter writes nothing.
+ * An index >= P: the row is skipped and SSU_FLAG_INDEX_RANGE is set.
+ */
+int pool_gather(const void *pool, int64_t slot_bytes, int32_t P, void *dense,
+                const int32_t *state_indices, int32_t batch, int32_t active_batch,
+                int32_t *err_flags, ssu_stream_t stream);
+int pool_scatter(const void *dense, void *pool, int64_t slot_bytes, int32_t P,
+                 const int32_t *state_indices, int32_t batch, int32_t active_batch,
+                 int32_t *err_flags, ssu_stream_t stream);
 
 /* A constant string naming an ssu_status value. */
 const char *ssu_status_string(int status);

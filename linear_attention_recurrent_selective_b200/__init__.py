@@ -11,8 +11,12 @@ from .ssu import (  # noqa: F401
     SSULibraryMissing,
     lib,
     pool_clear_slot,
+    pool_clear_slot_layers,
     pool_copy_slot,
+    pool_gather,
+    pool_scatter,
     ssu_decode,
     ssu_prefill,
     ssu_replay,
+    ssu_replay_layers,
 )

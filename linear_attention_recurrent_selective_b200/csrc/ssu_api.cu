@@ -176,6 +176,8 @@ int ssu_replay(void *state, int state_dtype, int64_t slot_stride, int32_t P,
     if (!aligned16(st_B))
         return SSU_ERR_ALIGN;
     ssu::ReplayArgs a;
+    a.layers = nullptr;
+    a.num_layers = 1;
     a.state = state;
     a.st_dA = st_dA;
     a.st_U = st_U;
@@ -194,6 +196,90 @@ int ssu_replay(void *state, int state_dtype, int64_t slot_stride, int32_t P,
     a.Dm = dim;
     a.N = dstate;
     return finish(ssu::launch_replay(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int ssu_replay_layers(const ssu_replay_layer *layers, int32_t num_layers, int state_dtype,
+                      int64_t slot_stride, int32_t P, const int32_t *accepted_lengths,
+                      const int32_t *state_indices, int32_t batch, int32_t active_batch,
+                      int32_t T, int32_t nheads, int32_t ngroups, int32_t dim, int32_t dstate,
+                      int32_t *err_flags, ssu_stream_t stream)
+{
+    if (T < 0 || num_layers < 0)
+        return SSU_ERR_SHAPE;
+    int rc = check_sizes(state_dtype, slot_stride, P, state_indices, batch, active_batch,
+                         nheads, ngroups, dim, dstate);
+    if (rc != SSU_OK || active_batch == 0 || T == 0 || num_layers == 0)
+        return rc;
+    if (!layers || !accepted_lengths)
+        return SSU_ERR_NULL;
+    if ((slot_stride * elem_bytes(state_dtype)) % 16 != 0)
+        return SSU_ERR_ALIGN;
+    ssu::ReplayArgs a;
+    a.layers = layers;                   // per-layer pointers are checked in-kernel
+    a.num_layers = num_layers;
+    a.state = nullptr;
+    a.st_dA = a.st_U = a.st_B = a.st_dt = nullptr;
+    a.acc = accepted_lengths;
+    a.idx = state_indices;
+    a.err = err_flags;
+    a.slot_stride = slot_stride;
+    a.P = P;
+    a.batch = batch;
+    a.active = active_batch;
+    a.T = T;
+    a.H = nheads;
+    a.G = ngroups;
+    a.Dm = dim;
+    a.N = dstate;
+    return finish(ssu::launch_replay(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int pool_clear_slot_layers(const ssu_layer_states *layers, int32_t num_layers, int32_t P,
+                           int32_t slot, int64_t recurrent_slot_bytes, int64_t conv_slot_bytes,
+                           ssu_stream_t stream)
+{
+    if (num_layers < 0 || P < 0 || slot < -1 || slot >= P || recurrent_slot_bytes < 0 ||
+        conv_slot_bytes < 0)
+        return SSU_ERR_SHAPE;
+    if (num_layers == 0)
+        return SSU_OK;
+    if (!layers)
+        return SSU_ERR_NULL;
+    return finish(ssu::launch_clear_layers(layers, num_layers, P, slot, recurrent_slot_bytes,
+                                           conv_slot_bytes,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static int gather_scatter(const void *pool, int64_t slot_bytes, int32_t P, void *dense,
+                          const int32_t *state_indices, int32_t batch, int32_t active_batch,
+                          int scatter, int32_t *err_flags, ssu_stream_t stream)
+{
+    if (slot_bytes < 0 || P < 0 || batch < 0 || active_batch < 0 || active_batch > batch)
+        return SSU_ERR_SHAPE;
+    if (!state_indices && active_batch > P)
+        return SSU_ERR_SHAPE;
+    if (active_batch == 0 || slot_bytes == 0)
+        return SSU_OK;
+    if (!pool || !dense)
+        return SSU_ERR_NULL;
+    return finish(ssu::launch_gather(pool, slot_bytes, P, dense, state_indices, active_batch,
+                                     scatter, err_flags, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int pool_gather(const void *pool, int64_t slot_bytes, int32_t P, void *dense,
+                const int32_t *state_indices, int32_t batch, int32_t active_batch,
+                int32_t *err_flags, ssu_stream_t stream)
+{
+    return gather_scatter(pool, slot_bytes, P, dense, state_indices, batch, active_batch, 0,
+                          err_flags, stream);
+}
+
+int pool_scatter(const void *dense, void *pool, int64_t slot_bytes, int32_t P,
+                 const int32_t *state_indices, int32_t batch, int32_t active_batch,
+                 int32_t *err_flags, ssu_stream_t stream)
+{
+    return gather_scatter(pool, slot_bytes, P, const_cast<void *>(dense), state_indices, batch,
+                          active_batch, 1, err_flags, stream);
 }
 
 int pool_clear_slot(void *pool, int64_t slot_bytes, int32_t P, int32_t slot,

@@ -43,6 +43,8 @@ struct PrefillArgs {
 };
 
 struct ReplayArgs {
+    const ssu_replay_layer *layers;   // device array [num_layers], or NULL: one layer below
+    int32_t num_layers;
     void *state;
     const float *st_dA, *st_U, *st_B, *st_dt;
     const int32_t *acc;
@@ -58,6 +60,11 @@ int launch_prefill(const PrefillArgs &a, int state_dtype, cudaStream_t s);
 int launch_replay(const ReplayArgs &a, int state_dtype, cudaStream_t s);
 int launch_clear(void *pool, int64_t bytes, cudaStream_t s);
 int launch_copy(void *dst, const void *src, int64_t bytes, cudaStream_t s);
+int launch_clear_layers(const ssu_layer_states *layers, int32_t num_layers, int32_t P,
+                        int32_t slot, int64_t rec_bytes, int64_t conv_bytes, cudaStream_t s);
+int launch_gather(const void *pool, int64_t slot_bytes, int32_t P, void *dense,
+                  const int32_t *idx, int32_t active, int scatter, int32_t *err,
+                  cudaStream_t s);
 
 // ---------------------------------------------------------------- scalar access
 

@@ -36,13 +36,17 @@ using namespace stream;
 constexpr int kUT = 8;
 
 struct DecodeRows {
+    const void *pool;
     const int32_t *idx;
     int32_t P;
-    __device__ __forceinline__ int2 resolve(int b) const
+    __device__ __forceinline__ UnitRes resolve(const LUnit &lu) const
     {
-        return make_int2(idx ? idx[b] : b, 0);
+        return UnitRes{static_cast<const char *>(pool), idx ? idx[lu.un.b] : lu.un.b, 0};
     }
-    __device__ __forceinline__ bool moves(int2 r) const { return r.x >= 0 && r.x < P; }
+    __device__ __forceinline__ bool moves(const UnitRes &r) const
+    {
+        return r.slot >= 0 && r.slot < P;
+    }
 };
 
 template <typename S, int N>
@@ -61,13 +65,13 @@ ssu_decode_kernel(const DecodeArgs a, const int cph, const int nunits)
     const int H = a.H, Dm = a.Dm, hpg = H / a.G;
     const int gw = blockIdx.x * kWarps + warp;
     const int nw = gridDim.x * kWarps;
-    const DecodeRows rows{a.idx, a.P};
+    const DecodeRows rows{a.state, a.idx, a.P};
     Producer<G, N, DecodeRows> prod;
     if (lane == 0) {
-        prod.start(rows, gw, nw, cph, nunits, H, Dm);
+        prod.start(rows, gw, nw, nunits, cph, nunits, H, Dm);
 #pragma unroll
         for (int s = 0; s < kStages; ++s)
-            prod.issue(rows, a.state, a.slot_stride, gw, nw, cph, nunits, H, Dm, w, s);
+            prod.issue(rows, a.slot_stride, gw, nw, nunits, cph, nunits, H, Dm, w, s);
     }
 
     const int ln = lane % G::LPR, sub = lane / G::LPR;
@@ -110,7 +114,7 @@ ssu_decode_kernel(const DecodeArgs a, const int cph, const int nunits)
                 return;
             const int s = c % kStages;
             slot = w.ctl->slot[s];
-            if (rows.moves(make_int2(slot, 0))) {
+            if (w.ctl->moves[s]) {
                 const int rt = min(G::RT, un.rows - j * G::RT);
                 const uint8_t *buf = w.ring + s * kTileBytes;
                 S *dst = static_cast<S *>(a.state) + (int64_t)slot * a.slot_stride +
@@ -153,7 +157,7 @@ ssu_decode_kernel(const DecodeArgs a, const int cph, const int nunits)
             }
             __syncwarp();                        // every lane is done with buffer s
             if (lane == 0)
-                prod.issue(rows, a.state, a.slot_stride, gw, nw, cph, nunits, H, Dm, w, s);
+                prod.issue(rows, a.slot_stride, gw, nw, nunits, cph, nunits, H, Dm, w, s);
         }
 
         // ---- the unit's outputs, one coalesced store per 32 rows

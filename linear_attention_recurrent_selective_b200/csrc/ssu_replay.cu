@@ -9,6 +9,10 @@
 // (dA = exp(A * dt_eff), dt = dt_eff, U = x), the same association the decode and
 // prefill kernels use, so fp32 results agree bit for bit with the decode steps.
 //
+// invokeMambaReplayReconstructBatched also takes a device array of per-layer pointers
+// (MambaReplayLayerInfo) and replays every layer in the same launch; units are numbered
+// layer-major, so consecutive warps stream through one layer's pool at a time.
+//
 // With a handful of tokens per row the work is one read and one write of every touched
 // state row, so the kernel runs on the per-warp bulk-copy pipeline of ssu_stream.cuh;
 // rows with nothing accepted are never copied. The stash values are read through L1
@@ -42,23 +46,57 @@ __device__ __forceinline__ void load_cols(const float *row, int ln, float *dst)
         }
 }
 
-struct ReplayRows {
-    const int32_t *idx;
-    const int32_t *acc;
-    int32_t P, T;
-    __device__ __forceinline__ int2 resolve(int b) const
-    {
-        return make_int2(idx ? idx[b] : b, acc[b]);
+__device__ __forceinline__ bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15) == 0;
+}
+
+// The pointers of one layer (from the layer array, or the single-layer arguments).
+struct LayerPtrs {
+    char *state;
+    const float *dA, *U, *B, *dt;
+    bool ok;
+};
+
+__device__ __forceinline__ LayerPtrs layer_ptrs(const ReplayArgs &a, int layer)
+{
+    LayerPtrs L;
+    if (a.layers) {
+        const ssu_replay_layer &l = a.layers[layer];
+        L.state = static_cast<char *>(l.state);
+        L.dA = l.st_dA;
+        L.U = l.st_U;
+        L.B = l.st_B;
+        L.dt = l.st_dt;
+    } else {
+        L.state = static_cast<char *>(a.state);
+        L.dA = a.st_dA;
+        L.U = a.st_U;
+        L.B = a.st_B;
+        L.dt = a.st_dt;
     }
-    __device__ __forceinline__ bool moves(int2 r) const
+    L.ok = L.state && L.dA && L.U && L.B && L.dt && aligned16(L.state) && aligned16(L.B);
+    return L;
+}
+
+struct ReplayRows {
+    const ReplayArgs *a;
+    __device__ __forceinline__ UnitRes resolve(const LUnit &lu) const
     {
-        return r.x >= 0 && r.x < P && min(r.y, T) > 0;
+        const LayerPtrs L = layer_ptrs(*a, lu.layer);
+        const int b = lu.un.b;
+        return UnitRes{L.ok ? L.state : nullptr, a->idx ? a->idx[b] : b, a->acc[b]};
+    }
+    __device__ __forceinline__ bool moves(const UnitRes &r) const
+    {
+        return r.pool != nullptr && r.slot >= 0 && r.slot < a->P && min(r.extra, a->T) > 0;
     }
 };
 
 template <typename S, int N>
 __global__ void __launch_bounds__(kWarps * 32)
-ssu_replay_kernel(const ReplayArgs a, const int cph, const int nunits)
+ssu_replay_kernel(const __grid_constant__ ReplayArgs a, const int cph, const int upl,
+                  const int nunits)
 {
     using G = Geo<S, N, kUT>;
     using V = Vec16<S>;
@@ -70,33 +108,35 @@ ssu_replay_kernel(const ReplayArgs a, const int cph, const int nunits)
     const int H = a.H, Dm = a.Dm, T = a.T, hpg = H / a.G;
     const int gw = blockIdx.x * kWarps + warp;
     const int nw = gridDim.x * kWarps;
-    const ReplayRows rows{a.idx, a.acc, a.P, T};
+    const ReplayRows rows{&a};
     Producer<G, N, ReplayRows> prod;
     if (lane == 0) {
-        prod.start(rows, gw, nw, cph, nunits, H, Dm);
+        prod.start(rows, gw, nw, upl, cph, nunits, H, Dm);
 #pragma unroll
         for (int s = 0; s < kStages; ++s)
-            prod.issue(rows, a.state, a.slot_stride, gw, nw, cph, nunits, H, Dm, w, s);
+            prod.issue(rows, a.slot_stride, gw, nw, upl, cph, nunits, H, Dm, w, s);
     }
 
     const int ln = lane % G::LPR, sub = lane / G::LPR;
     int c = 0;
     for (int u = gw; u < nunits; u += nw) {
-        const Unit un = unit_at(u, cph, G::CR, H, Dm);
+        const LUnit lu = lunit_at(u, upl, cph, G::CR, H, Dm);
+        const Unit &un = lu.un;
         const int tiles = (un.rows + G::RT - 1) / G::RT;
         const int g = un.h / hpg;
+        const LayerPtrs L = layer_ptrs(a, lu.layer);
 
         // ---- the unit's first kPre stashed tokens, loaded before its first tile is
         // waited for (addresses stay inside the stash whatever the accepted count is)
         float pdA[kPre], pdt[kPre], pB[kPre][G::E], pU[kPre][G::XR];
 #pragma unroll
         for (int t = 0; t < kPre; ++t) {
-            if (t < T) {
+            if (t < T && L.ok) {
                 const int64_t bt = (int64_t)un.b * T + t;
-                pdA[t] = a.st_dA[bt * H + un.h];
-                pdt[t] = a.st_dt[bt * H + un.h];
-                load_cols<G>(a.st_B + (bt * a.G + g) * N, ln, pB[t]);
-                const float *Ut = a.st_U + (bt * H + un.h) * Dm + un.row0;
+                pdA[t] = L.dA[bt * H + un.h];
+                pdt[t] = L.dt[bt * H + un.h];
+                load_cols<G>(L.B + (bt * a.G + g) * N, ln, pB[t]);
+                const float *Ut = L.U + (bt * H + un.h) * Dm + un.row0;
 #pragma unroll
                 for (int m = 0; m < G::XR; ++m)
                     pU[t][m] = lane + 32 * m < un.rows ? Ut[lane + 32 * m] : 0.f;
@@ -109,7 +149,7 @@ ssu_replay_kernel(const ReplayArgs a, const int cph, const int nunits)
                 return;
             const int s = c % kStages;
             r2 = make_int2(w.ctl->slot[s], w.ctl->extra[s]);
-            if (rows.moves(r2)) {
+            if (w.ctl->moves[s]) {
                 const int k = min(r2.y, T);
                 const int rt = min(G::RT, un.rows - j * G::RT);
                 const int r0 = un.row0 + j * G::RT;
@@ -150,11 +190,11 @@ ssu_replay_kernel(const ReplayArgs a, const int cph, const int nunits)
                 // longer acceptances: the remaining tokens straight from the stash
                 for (int t = kPre; t < k; ++t) {
                     const int64_t bt = (int64_t)un.b * T + t;
-                    const float dA = a.st_dA[bt * H + un.h];
-                    const float dte = a.st_dt[bt * H + un.h];
-                    const float *Ut = a.st_U + (bt * H + un.h) * Dm + r0;
+                    const float dA = L.dA[bt * H + un.h];
+                    const float dte = L.dt[bt * H + un.h];
+                    const float *Ut = L.U + (bt * H + un.h) * Dm + r0;
                     float Bn[G::E];
-                    load_cols<G>(a.st_B + (bt * a.G + g) * N, ln, Bn);
+                    load_cols<G>(L.B + (bt * a.G + g) * N, ln, Bn);
 #pragma unroll
                     for (int i = 0; i < G::RPT; ++i) {
                         const int r = i * G::RPW + sub;
@@ -164,7 +204,7 @@ ssu_replay_kernel(const ReplayArgs a, const int cph, const int nunits)
                             st[i][e] = fmaf(st[i][e], dA, Bn[e] * dtu);
                     }
                 }
-                S *dst = static_cast<S *>(a.state) + (int64_t)r2.x * a.slot_stride +
+                S *dst = reinterpret_cast<S *>(L.state) + (int64_t)r2.x * a.slot_stride +
                          ((int64_t)un.h * Dm + r0) * N;
 #pragma unroll
                 for (int i = 0; i < G::RPT; ++i) {
@@ -179,16 +219,20 @@ ssu_replay_kernel(const ReplayArgs a, const int cph, const int nunits)
             }
             __syncwarp();                        // every lane is done with buffer s
             if (lane == 0)
-                prod.issue(rows, a.state, a.slot_stride, gw, nw, cph, nunits, H, Dm, w, s);
+                prod.issue(rows, a.slot_stride, gw, nw, upl, cph, nunits, H, Dm, w, s);
         }
-        // ---- caller bugs, reported once per row (the row is clamped or skipped)
+        // ---- caller bugs, reported once per row (or layer): clamped or skipped
         if (lane == 0 && un.h == 0 && un.row0 == 0 && a.err) {
-            if (r2.x >= a.P)
-                atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
-            else if (r2.x >= 0 && r2.y > T)
-                atomicOr(a.err, SSU_FLAG_ACCEPTED_RANGE);
-            else if (r2.x >= 0 && r2.y < 0)
-                atomicOr(a.err, SSU_FLAG_NEGATIVE_LENGTH);
+            if (!L.ok && un.b == 0)
+                atomicOr(a.err, SSU_FLAG_LAYER);
+            if (lu.layer == 0) {
+                if (r2.x >= a.P)
+                    atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
+                else if (r2.x >= 0 && r2.y > T)
+                    atomicOr(a.err, SSU_FLAG_ACCEPTED_RANGE);
+                else if (r2.x >= 0 && r2.y < 0)
+                    atomicOr(a.err, SSU_FLAG_NEGATIVE_LENGTH);
+            }
         }
     }
 }
@@ -198,13 +242,15 @@ int launch_n(const ReplayArgs &a, cudaStream_t stream)
 {
     using G = Geo<S, N, kUT>;
     const int64_t cph = (a.Dm + G::CR - 1) / G::CR;
-    const int64_t nunits = (int64_t)a.active * a.H * cph;
+    const int64_t upl = (int64_t)a.active * a.H * cph;
+    const int64_t nunits = upl * a.num_layers;
     if (nunits == 0 || a.T == 0)
         return SSU_OK;
     if (nunits > 0x7fffffffLL)
         return SSU_ERR_SHAPE;
     const int grid = persistent_grid<ssu_replay_kernel<S, N>>(nunits);
-    ssu_replay_kernel<S, N><<<grid, kWarps * 32, kSmemBytes, stream>>>(a, (int)cph, (int)nunits);
+    ssu_replay_kernel<S, N><<<grid, kWarps * 32, kSmemBytes, stream>>>(a, (int)cph, (int)upl,
+                                                                       (int)nunits);
     return SSU_OK;
 }
 

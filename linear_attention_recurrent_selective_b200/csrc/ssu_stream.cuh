@@ -8,9 +8,9 @@
 // kTileBytes of contiguous state; every warp owns a ring of kStages shared-memory tile
 // buffers that the bulk-copy engine fills (cp.async.bulk, completion counted on a
 // per-buffer mbarrier), so kStages-1 tiles are in flight while the warp computes on one.
-// Lane 0 is the producer: it resolves the slot (and any per-row extra, such as an
-// accepted length) of the unit after the one it is copying one unit early, so the
-// index loads never stall the ring. Rows that touch no state (padding, out-of-range
+// Lane 0 is the producer: it resolves the pool, slot and any per-row extra (such as an
+// accepted length) of the unit after the one it is copying one unit early, so the index
+// loads never stall the ring. Multi-layer launches number units layer-major. Rows that touch no state (padding, out-of-range
 // index, nothing accepted) complete their buffer's barrier without a copy, which keeps
 // the consumer's phase bookkeeping uniform.
 #pragma once
@@ -56,6 +56,7 @@ struct Ring {
     uint64_t full[kStages];
     int slot[kStages];    // slot of the unit whose tile sits in each buffer
     int extra[kStages];   // per-row extra of that unit (e.g. the accepted length)
+    int moves[kStages];   // whether that tile was copied
 };
 static_assert(sizeof(Ring) <= 128, "per-warp control block");
 
@@ -80,6 +81,28 @@ __device__ __forceinline__ Unit unit_at(int u, int cph, int CR, int H, int Dm)
     return un;
 }
 
+// A unit of a multi-layer launch: units are numbered layer-major, upl units per layer.
+struct LUnit {
+    Unit un;
+    int layer;
+};
+
+__device__ __forceinline__ LUnit lunit_at(int u, int upl, int cph, int CR, int H, int Dm)
+{
+    LUnit lu;
+    lu.layer = u / upl;
+    lu.un = unit_at(u - lu.layer * upl, cph, CR, H, Dm);
+    return lu;
+}
+
+// What the producer needs to know about a unit: the base of its layer's pool, its slot and
+// a per-row extra (such as an accepted length).
+struct UnitRes {
+    const char *pool;
+    int slot;
+    int extra;
+};
+
 // Per-warp views of the dynamic shared memory.
 struct WarpViews {
     uint8_t *ring;     // kStages tile buffers
@@ -97,49 +120,51 @@ __device__ __forceinline__ WarpViews warp_views(uint8_t *smem, int warp)
     return w;
 }
 
-// Lane 0's side of a warp's pipeline. `Rows` maps a batch row to {slot, extra} and says
-// whether a unit of that row moves state:
-//   int2 resolve(int b) const;  bool moves(int2 r) const;
+// Lane 0's side of a warp's pipeline. `Rows` maps a unit to its pool, slot and extra and
+// says whether the unit moves state:
+//   UnitRes resolve(const LUnit &lu) const;  bool moves(const UnitRes &r) const;
 template <typename G, int N, typename Rows> struct Producer {
     int k;        // position in this warp's unit sequence
     int j;        // next tile within the unit
     int tiles;    // tiles of the current unit
-    int2 cur;     // {slot, extra} of the current unit
-    int2 nxt;     // the same for the next unit (loaded one unit early)
+    UnitRes cur;  // the current unit
+    UnitRes nxt;  // the next unit (resolved one unit early)
     int issued;   // tiles issued so far
 
-    __device__ void start(const Rows &rows, int gw, int nw, int cph, int nunits, int H, int Dm)
+    __device__ void start(const Rows &rows, int gw, int nw, int upl, int cph, int nunits, int H,
+                          int Dm)
     {
         k = 0;
         j = 0;
         issued = 0;
         tiles = 0;
-        cur = make_int2(-1, 0);
-        nxt = make_int2(-1, 0);
+        cur = UnitRes{nullptr, -1, 0};
+        nxt = UnitRes{nullptr, -1, 0};
         if (gw < nunits) {
-            const Unit un = unit_at(gw, cph, G::CR, H, Dm);
-            cur = rows.resolve(un.b);
-            tiles = (un.rows + G::RT - 1) / G::RT;
+            const LUnit lu = lunit_at(gw, upl, cph, G::CR, H, Dm);
+            cur = rows.resolve(lu);
+            tiles = (lu.un.rows + G::RT - 1) / G::RT;
             if (gw + nw < nunits)
-                nxt = rows.resolve(unit_at(gw + nw, cph, G::CR, H, Dm).b);
+                nxt = rows.resolve(lunit_at(gw + nw, upl, cph, G::CR, H, Dm));
         }
     }
 
-    __device__ void issue(const Rows &rows, const void *state, int64_t slot_stride, int gw,
-                          int nw, int cph, int nunits, int H, int Dm, const WarpViews &w, int s)
+    __device__ void issue(const Rows &rows, int64_t slot_stride, int gw, int nw, int upl, int cph,
+                          int nunits, int H, int Dm, const WarpViews &w, int s)
     {
         const int u = gw + k * nw;
         if (u >= nunits)
             return;
-        const Unit un = unit_at(u, cph, G::CR, H, Dm);
-        w.ctl->slot[s] = cur.x;
-        w.ctl->extra[s] = cur.y;
-        if (rows.moves(cur)) {
+        const Unit un = lunit_at(u, upl, cph, G::CR, H, Dm).un;
+        w.ctl->slot[s] = cur.slot;
+        w.ctl->extra[s] = cur.extra;
+        w.ctl->moves[s] = rows.moves(cur);
+        if (w.ctl->moves[s]) {
             const int nr = min(G::RT, un.rows - j * G::RT);
             const uint32_t bytes = (uint32_t)(nr * G::ROW_BYTES);
-            const char *src = static_cast<const char *>(state) +
-                              ((int64_t)cur.x * slot_stride +
-                               ((int64_t)un.h * Dm + un.row0 + j * G::RT) * N) * G::ELEM;
+            const char *src = cur.pool + ((int64_t)cur.slot * slot_stride +
+                                          ((int64_t)un.h * Dm + un.row0 + j * G::RT) * N) *
+                                             G::ELEM;
             mbar_arrive_expect_tx(&w.ctl->full[s], bytes);
             bulk_load(w.ring + s * kTileBytes, src, bytes, &w.ctl->full[s]);
         } else {
@@ -152,9 +177,9 @@ template <typename G, int N, typename Rows> struct Producer {
             const int u2 = gw + k * nw;
             if (u2 < nunits) {
                 cur = nxt;
-                tiles = (unit_at(u2, cph, G::CR, H, Dm).rows + G::RT - 1) / G::RT;
+                tiles = (lunit_at(u2, upl, cph, G::CR, H, Dm).un.rows + G::RT - 1) / G::RT;
                 if (u2 + nw < nunits)
-                    nxt = rows.resolve(unit_at(u2 + nw, cph, G::CR, H, Dm).b);
+                    nxt = rows.resolve(lunit_at(u2 + nw, upl, cph, G::CR, H, Dm));
             }
         }
     }

@@ -36,8 +36,14 @@ FLAG_NEGATIVE_LENGTH = 8
 FLAG_TIMEOUT = 16
 
 # Every C entry point declared in include/ssu.h, in declaration order.
-ENTRY_POINTS = ("ssu_decode", "ssu_prefill", "ssu_replay", "pool_clear_slot",
-                "pool_copy_slot", "ssu_status_string")
+ENTRY_POINTS = ("ssu_decode", "ssu_prefill", "ssu_replay", "ssu_replay_layers",
+                "pool_clear_slot", "pool_copy_slot", "pool_clear_slot_layers", "pool_gather",
+                "pool_scatter", "ssu_status_string")
+FLAG_LAYER = 32
+
+# Byte layouts of the per-layer pointer records of include/ssu.h (packed pointers).
+REPLAY_LAYER_FIELDS = 5     # state, st_dA, st_U, st_B, st_dt
+LAYER_STATES_FIELDS = 2     # recurrent_state, conv_state
 
 
 class SSULibraryMissing(RuntimeError):
@@ -75,8 +81,13 @@ def lib() -> ctypes.CDLL:
                               vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, ci, vp, vp]
     L.ssu_replay.argtypes = [vp, ci, i64, i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                              i32, i32, vp, vp]
+    L.ssu_replay_layers.argtypes = [vp, i32, ci, i64, i32, vp, vp, i32, i32, i32, i32, i32,
+                                    i32, i32, vp, vp]
     L.pool_clear_slot.argtypes = [vp, i64, i32, i32, vp]
     L.pool_copy_slot.argtypes = [vp, i32, i32, vp, i32, i32, i64, vp]
+    L.pool_clear_slot_layers.argtypes = [vp, i32, i32, i32, i64, i64, vp]
+    L.pool_gather.argtypes = [vp, i64, i32, vp, vp, i32, i32, vp, vp]
+    L.pool_scatter.argtypes = [vp, vp, i64, i32, vp, i32, i32, vp, vp]
     for f in ENTRY_POINTS[:-1]:
         getattr(L, f).restype = ci
     L.ssu_status_string.argtypes = [ci]
@@ -230,3 +241,86 @@ def pool_copy_slot(dst_pool, dst_slot, src_pool, src_slot, *, slot_bytes=None, d
                               ctypes.c_void_p(src_pool.data_ptr()), src_P, src_slot,
                               slot_bytes, _stream(stream))
     _check("pool_copy_slot", rc)
+
+
+def replay_layer_table(layers, device=None):
+    """Device array of ssu_replay_layer records for ``ssu_replay_layers``: ``layers`` is a
+    list of (state, (dA, U, B, dt)) CUDA tensors. Keep the returned tensor alive until
+    the launch that uses it has run."""
+    ptrs = []
+    for state, (sdA, sU, sB, sdt) in layers:
+        ptrs += [t.data_ptr() for t in (state, sdA, sU, sB, sdt)]
+    dev = device if device is not None else layers[0][0].device
+    return torch.tensor(ptrs, dtype=torch.int64, device=dev)
+
+
+def layer_states_table(layers, device=None):
+    """Device array of ssu_layer_states records for ``pool_clear_slot_layers``: ``layers``
+    is a list of (recurrent_state, conv_state or None) CUDA tensors."""
+    ptrs = []
+    for rec, conv in layers:
+        ptrs += [rec.data_ptr(), 0 if conv is None else conv.data_ptr()]
+    dev = device if device is not None else layers[0][0].device
+    return torch.tensor(ptrs, dtype=torch.int64, device=dev)
+
+
+def ssu_replay_layers(table, num_layers, like_state, like_stash, accepted_lengths, *,
+                      state_indices=None, active_batch=None, err_flags=None, slot_stride=None,
+                      P=None, stream=None):
+    """ssu_replay over ``num_layers`` layers in one launch. ``table`` comes from
+    ``replay_layer_table``; ``like_state`` / ``like_stash`` are any one layer's pool and
+    stash, which give the (shared) geometry and dtypes."""
+    sdA, sU, sB, sdt = like_stash
+    batch, T, H, Dm = sU.shape
+    G, N = sB.shape[2], sB.shape[3]
+    active = batch if active_batch is None else active_batch
+    stride, P = _pool_geometry(like_state, slot_stride, P, H * Dm * N)
+    rc = lib().ssu_replay_layers(
+        _ptr(table, "layer table", torch.int64), num_layers, _dt(like_state, "state"), stride,
+        P, _ptr(accepted_lengths, "accepted_lengths", torch.int32),
+        _ptr(state_indices, "state_indices", torch.int32), batch, active, T, H, G, Dm, N,
+        _ptr(err_flags, "err_flags", torch.int32), _stream(stream))
+    _check("ssu_replay_layers", rc)
+
+
+def pool_clear_slot_layers(table, num_layers, P, slot, recurrent_slot_bytes,
+                           conv_slot_bytes=0, *, stream=None):
+    """Zero one slot (or all, slot == -1) of every layer's recurrent and conv pools."""
+    rc = lib().pool_clear_slot_layers(_ptr(table, "layer table", torch.int64), num_layers, P,
+                                      slot, recurrent_slot_bytes, conv_slot_bytes,
+                                      _stream(stream))
+    _check("pool_clear_slot_layers", rc)
+
+
+def pool_gather(pool, dense, *, state_indices=None, active_batch=None, err_flags=None,
+                slot_bytes=None, P=None, stream=None):
+    """dense[b] = pool[state_indices[b]] for the active rows (padding rows get zeros)."""
+    batch = dense.shape[0]
+    active = batch if active_batch is None else active_batch
+    if slot_bytes is None:
+        slot_bytes = pool.stride(0) * pool.element_size()
+        P = pool.shape[0]
+    if not (pool.is_cuda and dense.is_cuda and dense.is_contiguous()):
+        raise ValueError("pool and dense must be CUDA tensors, dense contiguous")
+    rc = lib().pool_gather(ctypes.c_void_p(pool.data_ptr()), slot_bytes, P,
+                           ctypes.c_void_p(dense.data_ptr()),
+                           _ptr(state_indices, "state_indices", torch.int32), batch, active,
+                           _ptr(err_flags, "err_flags", torch.int32), _stream(stream))
+    _check("pool_gather", rc)
+
+
+def pool_scatter(dense, pool, *, state_indices=None, active_batch=None, err_flags=None,
+                 slot_bytes=None, P=None, stream=None):
+    """pool[state_indices[b]] = dense[b] for the active rows (padding rows are skipped)."""
+    batch = dense.shape[0]
+    active = batch if active_batch is None else active_batch
+    if slot_bytes is None:
+        slot_bytes = pool.stride(0) * pool.element_size()
+        P = pool.shape[0]
+    if not (pool.is_cuda and dense.is_cuda and dense.is_contiguous()):
+        raise ValueError("pool and dense must be CUDA tensors, dense contiguous")
+    rc = lib().pool_scatter(ctypes.c_void_p(dense.data_ptr()), ctypes.c_void_p(pool.data_ptr()),
+                            slot_bytes, P, _ptr(state_indices, "state_indices", torch.int32),
+                            batch, active, _ptr(err_flags, "err_flags", torch.int32),
+                            _stream(stream))
+    _check("pool_scatter", rc)

@@ -54,6 +54,10 @@ def lib():
         L.oracle_replay.argtypes = [vp, i, i64, i32, vp, vp, vp, vp, vp, vp,
                                     i32, i32, i32, i32, i32, i32, i32, vp]
         L.oracle_clear_slot.argtypes = [vp, i64, i32, i32]
+        L.oracle_replay_layers.argtypes = [vp, vp, vp, vp, vp, i32, i, i64, i32, vp, vp, i32,
+                                           i32, i32, i32, i32, i32, i32, vp]
+        L.oracle_clear_slot_layers.argtypes = [vp, vp, i32, i32, i32, i64, i64]
+        L.oracle_gather_scatter.argtypes = [vp, i64, i32, vp, vp, i32, i32, i, vp]
         L.oracle_copy_slot.argtypes = [vp, i32, i32, vp, i32, i32, i64]
         L.oracle_f16_to_double.argtypes = [ctypes.c_uint16]
         L.oracle_f16_to_double.restype = ctypes.c_double
@@ -64,7 +68,8 @@ def lib():
         L.oracle_double_to_bf16.argtypes = [ctypes.c_double]
         L.oracle_double_to_bf16.restype = ctypes.c_uint16
         for f in ("oracle_decode", "oracle_prefill", "oracle_replay",
-                  "oracle_clear_slot", "oracle_copy_slot"):
+                  "oracle_clear_slot", "oracle_copy_slot", "oracle_replay_layers",
+                  "oracle_clear_slot_layers", "oracle_gather_scatter"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -157,6 +162,57 @@ def clear_slot(pool, slot_bytes, P, slot):
 def copy_slot(dst_pool, dst_P, dst_slot, src_pool, src_P, src_slot, slot_bytes):
     _check(lib().oracle_copy_slot(_p(dst_pool), dst_P, dst_slot, _p(src_pool), src_P,
                                   src_slot, slot_bytes), "oracle_copy_slot")
+
+
+def _ptr_array(tensors):
+    arr = (ctypes.c_void_p * len(tensors))(*[None if t is None else t.data_ptr()
+                                             for t in tensors])
+    return arr
+
+
+def replay_layers(pools, stashes, accepted_lengths, *, state_indices=None, batch, active=None,
+                  T, H, G, Dm, N, slot_stride=None, P=None):
+    """Replay every layer l: pools[l] (in place) with stashes[l] = (DA, U, Bst, DT)."""
+    active = batch if active is None else active
+    slot_stride = H * Dm * N if slot_stride is None else slot_stride
+    P = pools[0].numel() // slot_stride if P is None else P
+    for t in list(pools) + [x for st in stashes for x in st]:
+        assert t.device.type == "cpu" and t.is_contiguous()
+    err = ctypes.c_int32(0)
+    rc = lib().oracle_replay_layers(
+        _ptr_array(pools), _ptr_array([s[0] for s in stashes]), _ptr_array([s[1] for s in stashes]),
+        _ptr_array([s[2] for s in stashes]), _ptr_array([s[3] for s in stashes]), len(pools),
+        _CODES[pools[0].dtype], slot_stride, P, _p(accepted_lengths), _p(state_indices), batch,
+        active, T, H, G, Dm, N, ctypes.byref(err))
+    _check(rc, "oracle_replay_layers")
+    return err.value
+
+
+def clear_slot_layers(recurrent, conv, P, slot, recurrent_slot_bytes, conv_slot_bytes):
+    """Zero slot ``slot`` (or all, -1) of every layer's recurrent and conv buffers."""
+    rc = lib().oracle_clear_slot_layers(_ptr_array(recurrent),
+                                        _ptr_array(conv) if conv is not None else None,
+                                        len(recurrent), P, slot, recurrent_slot_bytes,
+                                        conv_slot_bytes)
+    _check(rc, "oracle_clear_slot_layers")
+
+
+def gather(pool, dense, slot_bytes, P, *, state_indices=None, batch, active=None):
+    """dense[b] = pool[slot(b)] (zeros for padding rows). Returns err_flags."""
+    active = batch if active is None else active
+    err = ctypes.c_int32(0)
+    _check(lib().oracle_gather_scatter(_p(pool), slot_bytes, P, _p(dense), _p(state_indices),
+                                       batch, active, 0, ctypes.byref(err)), "oracle gather")
+    return err.value
+
+
+def scatter(dense, pool, slot_bytes, P, *, state_indices=None, batch, active=None):
+    """pool[slot(b)] = dense[b] (padding rows skipped). Returns err_flags."""
+    active = batch if active is None else active
+    err = ctypes.c_int32(0)
+    _check(lib().oracle_gather_scatter(_p(pool), slot_bytes, P, _p(dense), _p(state_indices),
+                                       batch, active, 1, ctypes.byref(err)), "oracle scatter")
+    return err.value
 
 
 # --- convenience wrappers over a workloads.SSUCase (inputs only; no arithmetic) ---

@@ -427,3 +427,79 @@ int oracle_copy_slot(void *dst_pool, int32_t dst_P, int32_t dst_slot,
             (const char *)src_pool + (int64_t)src_slot * slot_bytes, (size_t)slot_bytes);
     return 0;
 }
+
+/* ---------------- multi-layer launches and gather/scatter ----------------
+ * Selective State Update page: invokeMambaReplayReconstructBatched over an array of
+ * MambaReplayLayerInfo (every layer replays its own stash into its own pool, sharing
+ * acceptedLengths and stateIndices), invokeMambaStateClear over MambaStateLayerInfo
+ * (recurrent and convolution states of every layer), and invokeMambaStateGather /
+ * Scatter (copy active rows between the resident pool and a contiguous batch). */
+int oracle_replay_layers(void *const *pools, const float *const *st_DA,
+                         const float *const *st_U, const float *const *st_B,
+                         const float *const *st_DT, int32_t num_layers, int state_dt,
+                         int64_t slot_stride, int32_t P, const int32_t *accepted_lengths,
+                         const int32_t *state_indices, int32_t batch, int32_t active,
+                         int32_t T, int32_t H, int32_t G, int32_t Dm, int32_t N,
+                         int32_t *err_flags)
+{
+    for (int32_t l = 0; l < num_layers; ++l) {
+        int rc = oracle_replay(pools[l], state_dt, slot_stride, P, st_DA[l], st_U[l], st_B[l],
+                               st_DT[l], accepted_lengths, state_indices, batch, active, T, H,
+                               G, Dm, N, err_flags);
+        if (rc)
+            return rc;
+    }
+    return 0;
+}
+
+int oracle_clear_slot_layers(void *const *recurrent, void *const *conv, int32_t num_layers,
+                             int32_t P, int32_t slot, int64_t recurrent_slot_bytes,
+                             int64_t conv_slot_bytes)
+{
+    for (int32_t l = 0; l < num_layers; ++l) {
+        if (recurrent[l] && recurrent_slot_bytes) {
+            int rc = oracle_clear_slot(recurrent[l], recurrent_slot_bytes, P, slot);
+            if (rc)
+                return rc;
+        }
+        if (conv && conv[l] && conv_slot_bytes) {
+            int rc = oracle_clear_slot(conv[l], conv_slot_bytes, P, slot);
+            if (rc)
+                return rc;
+        }
+    }
+    return 0;
+}
+
+/* scatter == 0: dense[b] = pool[slot(b)], zeros for a padding row;
+ * scatter != 0: pool[slot(b)] = dense[b], nothing for a padding row;
+ * an index >= P skips the row and sets bit 1. */
+int oracle_gather_scatter(void *pool, int64_t slot_bytes, int32_t P, void *dense,
+                          const int32_t *state_indices, int32_t batch, int32_t active,
+                          int scatter, int32_t *err_flags)
+{
+    if (!pool || !dense || slot_bytes < 0 || active < 0 || active > batch)
+        return 2;
+    int32_t err = 0;
+    for (int32_t b = 0; b < active; ++b) {
+        int64_t s = state_indices ? state_indices[b] : b;
+        char *drow = (char *)dense + (int64_t)b * slot_bytes;
+        if (s >= P) {
+            err |= 1;
+            continue;
+        }
+        if (s < 0) {
+            if (!scatter)
+                memset(drow, 0, (size_t)slot_bytes);
+            continue;
+        }
+        char *prow = (char *)pool + s * slot_bytes;
+        if (scatter)
+            memcpy(prow, drow, (size_t)slot_bytes);
+        else
+            memcpy(drow, prow, (size_t)slot_bytes);
+    }
+    if (err_flags)
+        *err_flags |= err;
+    return 0;
+}

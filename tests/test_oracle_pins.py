@@ -439,3 +439,83 @@ def test_golden_tiny_decode_snapshot(orc):
     out, pool, _ = orc.decode_case(case)
     assert out.reshape(-1).tolist() == vals["out"]
     assert pool.view(4, -1)[[2, 0]].reshape(-1).tolist() == vals["state"]
+
+
+# ---------------------------------------------------------------- multi-layer, gather/scatter
+
+def test_replay_layers_is_every_layer_replayed(orc):
+    # Selective State Update page, invokeMambaReplayReconstructBatched: each layer replays
+    # its own stash into its own pool with the shared accepted lengths and indices.
+    base = make_case(seed=40, batch=4, P=7, T=3, H=2, G=1, Dm=4, N=8, lengths="accepted")
+    pools, stashes = [], []
+    for layer in range(3):
+        c = make_case(seed=41 + layer, batch=4, P=7, T=3, H=2, G=1, Dm=4, N=8)
+        c.state_indices = base.state_indices
+        _, _, st, _ = orc.prefill_case(c, stash=True)
+        pools.append(c.pool.clone())
+        stashes.append(st)
+    want = [p.clone() for p in pools]
+    for p, st in zip(want, stashes):
+        orc.replay(p, st, base.accepted_lengths, state_indices=base.state_indices, batch=4,
+                   T=3, H=2, G=1, Dm=4, N=8)
+    got = [p.clone() for p in pools]
+    orc.replay_layers(got, stashes, base.accepted_lengths, state_indices=base.state_indices,
+                      batch=4, T=3, H=2, G=1, Dm=4, N=8)
+    for g, w in zip(got, want):
+        assert same_bits(g, w)
+
+
+def test_gather_and_scatter_against_indexing(orc):
+    g = torch.Generator().manual_seed(42)
+    pool = torch.randn(9, 6, generator=g)
+    idx = torch.tensor([4, -1, 0, 8, 3], dtype=torch.int32)
+    dense = torch.full((5, 6), float("nan"))
+    err = orc.gather(pool, dense, 6 * 4, 9, state_indices=idx, batch=5, active=4)
+    assert err == 0
+    assert torch.equal(dense[0], pool[4]) and torch.equal(dense[2], pool[0])
+    assert torch.equal(dense[3], pool[8])
+    assert (dense[1] == 0).all()                    # padding row: zeros
+    assert torch.isnan(dense[4]).all()              # row >= active untouched
+    upd = torch.randn(5, 6, generator=g)
+    pool2 = pool.clone()
+    err = orc.scatter(upd, pool2, 6 * 4, 9, state_indices=idx, batch=5, active=4)
+    want = pool.clone()
+    for b in (0, 2, 3):
+        want[int(idx[b])] = upd[b]
+    assert err == 0 and torch.equal(pool2, want)
+    bad = torch.tensor([1, 9], dtype=torch.int32)
+    assert orc.gather(pool, torch.zeros(2, 6), 24, 9, state_indices=bad, batch=2) == 1
+
+
+def test_indexed_decode_equals_oracle_gather_run_scatter(orc):
+    case = make_case(seed=43, batch=5, P=9, H=4, G=2, Dm=4, N=8, z=True, active=4, n_pad=1)
+    out_idx, pool_idx, _ = orc.decode_case(case)
+    slot = case.slot_stride
+    dense = torch.zeros(case.batch, slot)
+    orc.gather(case.pool, dense, slot * 4, case.P, state_indices=case.state_indices,
+               batch=case.batch, active=case.active)
+    dense = dense.reshape(-1)
+    out_d, _ = orc.decode(case.x, case.A, case.B, case.C, case.dt, dense, dt_bias=case.dt_bias,
+                          D=case.D, z=case.z, batch=case.batch, active=case.active, H=4, G=2,
+                          Dm=4, N=8)
+    pool = case.pool.clone()
+    orc.scatter(dense, pool, slot * 4, case.P, state_indices=case.state_indices,
+                batch=case.batch, active=case.active)
+    assert same_bits(pool, pool_idx)
+    live = case.state_indices[: case.active] >= 0
+    assert same_bits(out_d[: case.active][live], out_idx[: case.active][live])
+
+
+def test_clear_slot_layers(orc):
+    g = torch.Generator().manual_seed(44)
+    rec = [torch.randn(5, 8, generator=g) + 3 for _ in range(3)]
+    conv = [torch.randn(5, 2, generator=g) + 3, None, torch.randn(5, 2, generator=g) + 3]
+    r2, c2 = [r.clone() for r in rec], [None if c is None else c.clone() for c in conv]
+    orc.clear_slot_layers(r2, c2, 5, 3, 8 * 4, 2 * 4)
+    for r, r0 in zip(r2, rec):
+        assert (r[3] == 0).all() and torch.equal(r[[0, 1, 2, 4]], r0[[0, 1, 2, 4]])
+    for c, c0 in zip(c2, conv):
+        if c is not None:
+            assert (c[3] == 0).all() and torch.equal(c[[0, 1, 2, 4]], c0[[0, 1, 2, 4]])
+    orc.clear_slot_layers(r2, c2, 5, -1, 8 * 4, 2 * 4)
+    assert all((r == 0).all() for r in r2) and all(c is None or (c == 0).all() for c in c2)
