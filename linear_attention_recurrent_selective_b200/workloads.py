@@ -1,9 +1,9 @@
-"""Seeded synthetic inputs for the selective state update (decode, prefill, replay).
+"""Seeded synthetic inputs for the selective state update (decode, prefill, replay, tree).
 
 This module only draws random numbers and lays them out in the shapes the
 Selective State Update page (TensorRT-Edge-LLM C++ API, ``invokeSelectiveStateUpdate``,
-``invokeSelectiveStateUpdatePrefill`` and ``MambaReplayLayerInfo``) gives for each
-argument. It holds no part of the recurrence: both the CUDA path and the CPU oracle
+``invokeSelectiveStateUpdatePrefill``, ``invokeSelectiveStateUpdateDDTree`` and
+``MambaReplayLayerInfo``) gives for each argument. It holds no part of the recurrence: both the CUDA path and the CPU oracle
 receive the same tensors from here and do all of the arithmetic themselves.
 
 Value laws (one set for every workload):
@@ -12,8 +12,15 @@ Value laws (one set for every workload):
   The "slow decay" variant draws A = -exp(U(-2, 0)) and sets dt_bias = -4, so that the
   state remembers many tokens.
 Every tensor is drawn in fp32 from one ``torch.Generator`` in a fixed order
-(pool, x, B, C, dt, z, A, dt_bias, D, stateIndices, padding positions, lengths) and then
-cast to its storage dtype, so both sides see the same (already rounded) values.
+(pool, x, B, C, dt, z, A, dt_bias, D, stateIndices, padding positions, lengths, tree)
+and then cast to its storage dtype, so both sides see the same (already rounded) values.
+
+Draft trees (tree verify): node 0 is a root; every later node i picks its parent
+uniformly among nodes 0..i-1 (a random recursive tree, expected depth about ln T), or
+i-1 ("chain"); "forest" turns each later node into another root with probability 1/8;
+"shuffled" relabels the nodes by a random permutation so that parents need not precede
+their children. An accepted path is the root-to-node path of a uniformly drawn node,
+with acceptedLengths ~ U{0..path length}.
 """
 
 from __future__ import annotations
@@ -36,6 +43,8 @@ class SSUCase:
       pool [P, H, Dm, N] (slot stride H*Dm*N elements unless ``slot_stride`` says more)
       A, dt_bias, D [H] fp32; state_indices [batch] int32 (None = row b uses slot b)
       context_lengths / accepted_lengths [batch] int32 (None = all T tokens)
+      tree verify: parent_ids, depths [batch, T] int32 (T = tree nodes);
+      accepted_node_ids [batch, T] int32 (an accepted root-to-node path, -1 beyond it)
     """
 
     name: str
@@ -61,6 +70,9 @@ class SSUCase:
     context_lengths: Optional[torch.Tensor] = None
     accepted_lengths: Optional[torch.Tensor] = None
     dt_softplus: bool = True
+    parent_ids: Optional[torch.Tensor] = None
+    depths: Optional[torch.Tensor] = None
+    accepted_node_ids: Optional[torch.Tensor] = None
 
     @property
     def x_dtype(self):
@@ -107,6 +119,7 @@ def make_case(
     lengths: Optional[str] = None,
     slot_pad: int = 0,
     slow_decay: bool = False,
+    tree: Optional[str] = None,
 ) -> SSUCase:
     """Draw one workload.
 
@@ -116,6 +129,8 @@ def make_case(
     lengths: None, "context" (contextLengths ~ U{1..T}) or "accepted"
       (acceptedLengths ~ U{0..T}).
     slot_pad: extra elements per pool slot beyond H*Dm*N (a padded slot stride).
+    tree: None, "random", "chain", "forest" or "shuffled" (draft trees of T nodes, with
+      an accepted path and acceptedLengths along it).
     """
     if P is None:
         P = batch
@@ -169,15 +184,77 @@ def make_case(
     elif lengths is not None:
         raise ValueError(f"unknown lengths mode {lengths!r}")
 
+    par = dep = nodes = None
+    if tree is not None:
+        par, dep = draw_trees(g, batch, T, tree)
+        nodes, acc = draw_accepted_paths(g, par, dep)
+
     return SSUCase(
         name=name, batch=batch, P=P, H=H, G=G, Dm=Dm, N=N, T=T, active=active,
         slot_stride=stride, x=x, B=B, C=C, dt=dt, A=A, pool=pool, z=zt,
         dt_bias=bias, D=Dv, state_indices=si, context_lengths=ctx,
-        accepted_lengths=acc, dt_softplus=dt_softplus,
+        accepted_lengths=acc, dt_softplus=dt_softplus, parent_ids=par, depths=dep,
+        accepted_node_ids=nodes,
     )
 
 
-# The five named workloads. Seeds: 0 for the tiny decode, then 1..4 in order.
+def tree_depths(parents: torch.Tensor) -> torch.Tensor:
+    """Number of tree ancestors of every node (parents [batch, T], -1 = root)."""
+    batch, T = parents.shape
+    dep = torch.zeros(batch, T, dtype=torch.int32)
+    for b in range(batch):
+        row = parents[b].tolist()
+        for i in range(T):
+            k, v = 0, row[i]
+            while v != -1:
+                k, v = k + 1, row[v]
+            dep[b, i] = k
+    return dep
+
+
+def draw_trees(g: torch.Generator, batch: int, T: int, mode: str):
+    """Parents and depths [batch, T] int32 of one draft tree per row (see module doc)."""
+    par = torch.full((batch, T), -1, dtype=torch.int32)
+    for i in range(1, T):
+        if mode == "chain":
+            par[:, i] = i - 1
+        else:
+            par[:, i] = torch.randint(0, i, (batch,), generator=g, dtype=torch.int32)
+    if mode == "forest":
+        roots = torch.rand(batch, T, generator=g) < 0.125
+        roots[:, 0] = True
+        par[roots] = -1
+    elif mode == "shuffled":
+        for b in range(batch):
+            perm = torch.randperm(T, generator=g)
+            new = torch.full((T,), -1, dtype=torch.int32)
+            for i in range(T):
+                p = int(par[b, i])
+                new[perm[i]] = -1 if p < 0 else int(perm[p])
+            par[b] = new
+    elif mode not in ("random", "chain"):
+        raise ValueError(f"unknown tree mode {mode!r}")
+    return par, tree_depths(par)
+
+
+def draw_accepted_paths(g: torch.Generator, par: torch.Tensor, dep: torch.Tensor):
+    """Accepted root-to-node paths [batch, T] (-1 beyond each path) and their lengths."""
+    batch, T = par.shape
+    nodes = torch.full((batch, T), -1, dtype=torch.int32)
+    acc = torch.zeros(batch, dtype=torch.int32)
+    for b in range(batch):
+        v = int(torch.randint(0, T, (1,), generator=g))
+        path = []
+        while v != -1:
+            path.append(v)
+            v = int(par[b, v])
+        path.reverse()
+        nodes[b, :len(path)] = torch.tensor(path, dtype=torch.int32)
+        acc[b] = int(torch.randint(0, len(path) + 1, (1,), generator=g))
+    return nodes, acc
+
+
+# The named workloads. Seeds: 0 for the tiny decode, then 1..5 in order.
 CONFIGS = {
     # batch 2, pool of 4 slots, H 4, Dm 16, N 16, fp32 everything, stateIndices [2, 0]
     "tiny_decode": dict(seed=0, batch=2, P=4, H=4, G=1, Dm=16, N=16,
@@ -198,6 +275,10 @@ CONFIGS = {
     "spec_replay_b64_t5": dict(seed=4, batch=64, P=128, T=5, H=80, G=1, Dm=64, N=128,
                                x_dtype=BF16, bc_dtype=BF16, state_dtype=F32, z=True,
                                lengths="accepted"),
+    # tree verify of one 128-node draft tree per row (the verify budget), no gate
+    "ddtree_b16_n128": dict(seed=5, batch=16, P=32, T=128, H=80, G=1, Dm=64, N=128,
+                            x_dtype=BF16, bc_dtype=BF16, state_dtype=F32, z=False,
+                            tree="random"),
 }
 
 

@@ -6,7 +6,8 @@ benchmark's CPU-baseline leg import this module. It never touches the CUDA libra
 The functions take CPU torch tensors (used here only as typed host buffers) and return
 float64 outputs. The pool is updated in place in its own storage type, exactly as the
 Selective State Update page (TensorRT-Edge-LLM C++ API) describes for
-``invokeSelectiveStateUpdate``, ``invokeSelectiveStateUpdatePrefill`` and the replay.
+``invokeSelectiveStateUpdate``, ``invokeSelectiveStateUpdatePrefill``, the tree verify
+``invokeSelectiveStateUpdateDDTree`` and the replay.
 """
 
 from __future__ import annotations
@@ -52,10 +53,13 @@ def lib():
                                      vp, vp, vp, vp, vp, vp, vp,
                                      i32, i32, i32, i32, i32, i32, i32, i, vp]
         L.oracle_replay.argtypes = [vp, i, i64, i32, vp, vp, vp, vp, vp, vp,
-                                    i32, i32, i32, i32, i32, i32, i32, vp]
+                                    i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
+        L.oracle_ddtree.argtypes = [vp, i, vp, vp, vp, i, vp, vp, vp, vp, i, i64, i32,
+                                    vp, vp, vp, vp, vp, vp, vp, vp,
+                                    i32, i32, i32, i32, i32, i32, i32, i, vp]
         L.oracle_clear_slot.argtypes = [vp, i64, i32, i32]
         L.oracle_replay_layers.argtypes = [vp, vp, vp, vp, vp, i32, i, i64, i32, vp, vp, i32,
-                                           i32, i32, i32, i32, i32, i32, vp]
+                                           i32, i32, i32, i32, i32, i32, vp, i32, vp]
         L.oracle_clear_slot_layers.argtypes = [vp, vp, i32, i32, i32, i64, i64]
         L.oracle_gather_scatter.argtypes = [vp, i64, i32, vp, vp, i32, i32, i, vp]
         L.oracle_copy_slot.argtypes = [vp, i32, i32, vp, i32, i32, i64]
@@ -69,7 +73,7 @@ def lib():
         L.oracle_double_to_bf16.restype = ctypes.c_uint16
         for f in ("oracle_decode", "oracle_prefill", "oracle_replay",
                   "oracle_clear_slot", "oracle_copy_slot", "oracle_replay_layers",
-                  "oracle_clear_slot_layers", "oracle_gather_scatter"):
+                  "oracle_clear_slot_layers", "oracle_gather_scatter", "oracle_ddtree"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -140,8 +144,10 @@ def new_stash(batch, T, H, G, Dm, N, fill=float("nan")):
 
 
 def replay(pool, stash, accepted_lengths, *, state_indices=None, batch, active=None, T,
-           H, G, Dm, N, slot_stride=None, P=None):
-    """Re-apply the first acceptedLengths[b] stashed tokens in place. Returns err_flags."""
+           H, G, Dm, N, slot_stride=None, P=None, node_ids=None):
+    """Re-apply the first acceptedLengths[b] stashed tokens in place; with ``node_ids``
+    ([batch, maxAcceptLen] int32) token t of row b is stash entry node_ids[b, t].
+    Returns err_flags."""
     active = batch if active is None else active
     slot_stride = H * Dm * N if slot_stride is None else slot_stride
     P = pool.numel() // slot_stride if P is None else P
@@ -150,9 +156,32 @@ def replay(pool, stash, accepted_lengths, *, state_indices=None, batch, active=N
     rc = lib().oracle_replay(
         _p(pool), _CODES[pool.dtype], slot_stride, P, _p(DA), _p(U), _p(Bst), _p(DT),
         _p(accepted_lengths), _p(state_indices), batch, active, T, H, G, Dm, N,
-        ctypes.byref(err))
+        _p(node_ids), 0 if node_ids is None else node_ids.shape[1], ctypes.byref(err))
     _check(rc, "oracle_replay")
     return err.value
+
+
+def ddtree(x, A, B, C, dt, pool, parent_ids, depths, *, dt_bias=None, D=None,
+           state_indices=None, batch, active=None, T, H, G, Dm, N, slot_stride=None,
+           P=None, dt_softplus=True, out=None, stash=None):
+    """Tree verify: every node's output from the committed state along its ancestor path
+    (the pool is only read). Returns (out float64 [batch,T,H,Dm], stash, err_flags)."""
+    active = batch if active is None else active
+    slot_stride = H * Dm * N if slot_stride is None else slot_stride
+    P = pool.numel() // slot_stride if P is None else P
+    if out is None:
+        out = torch.full((batch, T, H, Dm), float("nan"), dtype=torch.float64)
+    if stash is None:
+        stash = new_stash(batch, T, H, G, Dm, N)
+    DA, U, Bst, DT = stash
+    err = ctypes.c_int32(0)
+    rc = lib().oracle_ddtree(
+        _p(x), _CODES[x.dtype], _p(A), _p(B), _p(C), _CODES[B.dtype], _p(dt), _p(dt_bias),
+        _p(D), _p(pool), _CODES[pool.dtype], slot_stride, P, _p(out), _p(parent_ids),
+        _p(depths), _p(state_indices), _p(DA), _p(U), _p(Bst), _p(DT), batch, active, T, H,
+        G, Dm, N, int(dt_softplus), ctypes.byref(err))
+    _check(rc, "oracle_ddtree")
+    return out, stash, err.value
 
 
 def clear_slot(pool, slot_bytes, P, slot):
@@ -171,7 +200,7 @@ def _ptr_array(tensors):
 
 
 def replay_layers(pools, stashes, accepted_lengths, *, state_indices=None, batch, active=None,
-                  T, H, G, Dm, N, slot_stride=None, P=None):
+                  T, H, G, Dm, N, slot_stride=None, P=None, node_ids=None):
     """Replay every layer l: pools[l] (in place) with stashes[l] = (DA, U, Bst, DT)."""
     active = batch if active is None else active
     slot_stride = H * Dm * N if slot_stride is None else slot_stride
@@ -183,7 +212,8 @@ def replay_layers(pools, stashes, accepted_lengths, *, state_indices=None, batch
         _ptr_array(pools), _ptr_array([s[0] for s in stashes]), _ptr_array([s[1] for s in stashes]),
         _ptr_array([s[2] for s in stashes]), _ptr_array([s[3] for s in stashes]), len(pools),
         _CODES[pools[0].dtype], slot_stride, P, _p(accepted_lengths), _p(state_indices), batch,
-        active, T, H, G, Dm, N, ctypes.byref(err))
+        active, T, H, G, Dm, N, _p(node_ids), 0 if node_ids is None else node_ids.shape[1],
+        ctypes.byref(err))
     _check(rc, "oracle_replay_layers")
     return err.value
 
@@ -239,3 +269,12 @@ def prefill_case(case, pool=None, stash=False):
                        N=case.N, slot_stride=case.slot_stride, P=case.P,
                        dt_softplus=case.dt_softplus)
     return out, pool, st, err
+
+
+def ddtree_case(case):
+    """Run the oracle tree verify on a tree case; returns (out, stash, err)."""
+    return ddtree(case.x, case.A, case.B, case.C, case.dt, case.pool, case.parent_ids,
+                  case.depths, dt_bias=case.dt_bias, D=case.D,
+                  state_indices=case.state_indices, batch=case.batch, active=case.active,
+                  T=case.T, H=case.H, G=case.G, Dm=case.Dm, N=case.N,
+                  slot_stride=case.slot_stride, P=case.P, dt_softplus=case.dt_softplus)

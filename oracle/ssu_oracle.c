@@ -30,7 +30,8 @@
  *     (all T positions in prefill); the replay writes nothing for it;
  *   - an index >= P, a length > T or a negative length is undefined on the pages; here
  *     the row is skipped (index) or the length clamped, and a bit is set in err_flags:
- *     1 = index >= P, 2 = acceptedLengths > T, 4 = contextLengths > T, 8 = negative length.
+ *     1 = index >= P, 2 = acceptedLengths > T, 4 = contextLengths > T, 8 = negative length,
+ *     64 = malformed tree input (see the tree verify below).
  */
 #include <math.h>
 #include <stdint.h>
@@ -344,12 +345,18 @@ int oracle_prefill(const void *x, int x_dt, const float *A,
  * Selective State Update page, struct MambaReplayLayerInfo and
  * invokeMambaReplayReconstructBatched: re-run the recurrence over the first
  * acceptedLengths[b] stashed tokens, in place on the committed state; a count of 0
- * leaves the row untouched; rows b >= activeBatchSize are not visited. */
+ * leaves the row untouched; rows b >= activeBatchSize are not visited.
+ *
+ * With acceptedNodeIds ([activeBatch, maxAcceptLen], the tree-accept form of the same
+ * call) the t-th replayed token is stash entry acceptedNodeIds[b][t] instead of t, and
+ * the accepted count is bounded by maxAcceptLen. A node id outside [0, T) among the
+ * first acceptedLengths[b] leaves the whole row untouched and sets flag 64. */
 int oracle_replay(void *pool, int state_dt, int64_t slot_stride, int32_t P,
                   const float *st_DA, const float *st_U, const float *st_B,
                   const float *st_DT, const int32_t *accepted_lengths,
                   const int32_t *state_indices, int32_t batch, int32_t active, int32_t T,
-                  int32_t H, int32_t G, int32_t Dm, int32_t N, int32_t *err_flags)
+                  int32_t H, int32_t G, int32_t Dm, int32_t N,
+                  const int32_t *node_ids, int32_t max_accept_len, int32_t *err_flags)
 {
     if (!pool || !st_DA || !st_U || !st_B || !st_DT || !accepted_lengths)
         return 1;
@@ -357,6 +364,9 @@ int oracle_replay(void *pool, int state_dt, int64_t slot_stride, int32_t P,
         return 3;
     if (check_common(batch, active, H, G, Dm, N, slot_stride) || T < 0)
         return 2;
+    if (node_ids && max_accept_len < 0)
+        return 2;
+    const int32_t bound = node_ids ? max_accept_len : T;
     int32_t err = 0;
     int heads_per_group = H / G;
     double *S = malloc(sizeof(double) * (size_t)Dm * N);
@@ -365,13 +375,23 @@ int oracle_replay(void *pool, int state_dt, int64_t slot_stride, int32_t P,
         if (s < 0)
             continue;                        /* padding row or bad index: no state */
         int32_t k = accepted_lengths[b];
-        if (k > T) {
+        if (k > bound) {
             err |= 2;
-            k = T;
+            k = bound;
         }
         if (k < 0) {
             err |= 8;
             k = 0;
+        }
+        int ids_ok = 1;
+        for (int32_t t = 0; node_ids && t < k; ++t) {
+            int32_t id = node_ids[(int64_t)b * max_accept_len + t];
+            if (id < 0 || id >= T)
+                ids_ok = 0;
+        }
+        if (!ids_ok) {
+            err |= 64;
+            continue;
         }
         if (k == 0)
             continue;
@@ -380,7 +400,8 @@ int oracle_replay(void *pool, int state_dt, int64_t slot_stride, int32_t P,
             for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
                 S[i] = load(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i);
             for (int32_t t = 0; t < k; ++t) {
-                int64_t bt = (int64_t)b * T + t;
+                int32_t e = node_ids ? node_ids[(int64_t)b * max_accept_len + t] : t;
+                int64_t bt = (int64_t)b * T + e;
                 double decay = st_DA[bt * H + h];
                 double dte = st_DT[bt * H + h];
                 for (int d = 0; d < Dm; ++d) {
@@ -393,6 +414,120 @@ int oracle_replay(void *pool, int state_dt, int64_t slot_stride, int32_t P,
             }
             for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
                 store(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i, S[i]);
+        }
+    }
+    free(S);
+    if (err_flags)
+        *err_flags |= err;
+    return 0;
+}
+
+/* ---------------- tree verify (DDTree) ----------------
+ * Selective State Update page, mamba_ssm::invokeSelectiveStateUpdateDDTree: the committed
+ * state stays read-only; for every verify node i of row b the ancestors are found by
+ * following treeParentIds from i to the root, the recurrence is run from the committed
+ * state over that path in root-to-node order, node i's output is taken from the state
+ * reached at i, and node i's own (dA, x, B, dt) tuple is stored in the replay stash at
+ * position i. Paths stay within the verify budget of 128 nodes.
+ *
+ * x [batch,T,H,Dm], B/C [batch,T,G,N], dt [batch,T,H], out [batch,T,H,Dm] (no z gate in
+ * this call), treeParentIds/treeDepths [batch,T]. Readings: parent -1 attaches a node to
+ * the committed state; treeDepths[b][i] counts the tree ancestors of node i, so the walk
+ * from i takes exactly that many parent steps and must then reach parent -1. A node whose
+ * walk leaves [0, T), ends early or does not end there is malformed: its outputs are 0
+ * and flag 64 is set (its stash entry is written like any other). Padding rows output 0
+ * at every node and write no stash; an index >= P skips the row (flag 1). */
+int oracle_ddtree(const void *x, int x_dt, const float *A, const void *B, const void *C,
+                  int bc_dt, const float *dt, const float *dt_bias, const float *D,
+                  const void *pool, int state_dt, int64_t slot_stride, int32_t P,
+                  double *out, const int32_t *parent_ids, const int32_t *depths,
+                  const int32_t *state_indices, float *st_DA, float *st_U, float *st_B,
+                  float *st_DT, int32_t batch, int32_t active, int32_t T, int32_t H,
+                  int32_t G, int32_t Dm, int32_t N, int dt_softplus, int32_t *err_flags)
+{
+    if (!x || !A || !B || !C || !dt || !pool || !out || !parent_ids || !depths)
+        return 1;
+    if (!st_DA || !st_U || !st_B || !st_DT)
+        return 1;
+    if (!valid_dtype(x_dt) || !valid_dtype(bc_dt) || !valid_dtype(state_dt))
+        return 3;
+    if (check_common(batch, active, H, G, Dm, N, slot_stride) || T < 0 || T > 128)
+        return 2;
+    int32_t err = 0;
+    int heads_per_group = H / G;
+    double *S = malloc(sizeof(double) * (size_t)Dm * N);
+    int32_t path[128];
+    for (int32_t b = 0; b < active; ++b) {
+        int64_t s = resolve_slot(state_indices, b, P, &err);
+        if (s == -1) {                       /* padding row: every node outputs 0 */
+            for (int64_t i = 0; i < (int64_t)T * H * Dm; ++i)
+                out[(int64_t)b * T * H * Dm + i] = 0.0;
+            continue;
+        }
+        if (s < 0)
+            continue;
+        /* the stash: every node's own replay inputs */
+        for (int32_t i = 0; i < T; ++i) {
+            int64_t bi = (int64_t)b * T + i;
+            for (int h = 0; h < H; ++h) {
+                int g = h / heads_per_group;
+                double dte = effective_dt(dt[bi * H + h], dt_bias, h, dt_softplus);
+                st_DA[bi * H + h] = (float)exp((double)A[h] * dte);
+                st_DT[bi * H + h] = (float)dte;
+                for (int d = 0; d < Dm; ++d)
+                    st_U[(bi * H + h) * Dm + d] = (float)load(x, x_dt, (bi * H + h) * Dm + d);
+                for (int n = 0; n < N; ++n)
+                    st_B[(bi * G + g) * N + n] = (float)load(B, bc_dt, (bi * G + g) * N + n);
+            }
+        }
+        for (int32_t i = 0; i < T; ++i) {
+            int64_t bi = (int64_t)b * T + i;
+            /* walk from node i to the root: path[0] = i, path[k] = k-th ancestor */
+            int32_t depth = depths[bi];
+            int ok = depth >= 0 && depth < 128;
+            int32_t node = i;
+            for (int32_t k = 0; ok && k <= depth; ++k) {
+                path[k] = node;
+                int32_t par = parent_ids[(int64_t)b * T + node];
+                if (k < depth) {
+                    if (par < 0 || par >= T)
+                        ok = 0;
+                    node = par;
+                } else if (par != -1) {
+                    ok = 0;
+                }
+            }
+            if (!ok) {
+                err |= 64;
+                for (int64_t e = 0; e < (int64_t)H * Dm; ++e)
+                    out[bi * H * Dm + e] = 0.0;
+                continue;
+            }
+            for (int h = 0; h < H; ++h) {
+                int g = h / heads_per_group;
+                for (int64_t e = 0; e < (int64_t)Dm * N; ++e)
+                    S[e] = load(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + e);
+                for (int32_t k = depth; k >= 0; --k) {   /* root-to-node order */
+                    int64_t bj = (int64_t)b * T + path[k];
+                    double dte = effective_dt(dt[bj * H + h], dt_bias, h, dt_softplus);
+                    double decay = exp((double)A[h] * dte);
+                    for (int d = 0; d < Dm; ++d) {
+                        double xv = load(x, x_dt, (bj * H + h) * Dm + d);
+                        for (int n = 0; n < N; ++n) {
+                            double *sp = &S[(int64_t)d * N + n];
+                            *sp = *sp * decay + load(B, bc_dt, (bj * G + g) * N + n) * dte * xv;
+                        }
+                    }
+                }
+                for (int d = 0; d < Dm; ++d) {
+                    double y = 0.0;
+                    for (int n = 0; n < N; ++n)
+                        y += S[(int64_t)d * N + n] * load(C, bc_dt, (bi * G + g) * N + n);
+                    if (D)
+                        y += (double)D[h] * load(x, x_dt, (bi * H + h) * Dm + d);
+                    out[(bi * H + h) * Dm + d] = y;
+                }
+            }
         }
     }
     free(S);
@@ -440,12 +575,12 @@ int oracle_replay_layers(void *const *pools, const float *const *st_DA,
                          int64_t slot_stride, int32_t P, const int32_t *accepted_lengths,
                          const int32_t *state_indices, int32_t batch, int32_t active,
                          int32_t T, int32_t H, int32_t G, int32_t Dm, int32_t N,
-                         int32_t *err_flags)
+                         const int32_t *node_ids, int32_t max_accept_len, int32_t *err_flags)
 {
     for (int32_t l = 0; l < num_layers; ++l) {
         int rc = oracle_replay(pools[l], state_dt, slot_stride, P, st_DA[l], st_U[l], st_B[l],
                                st_DT[l], accepted_lengths, state_indices, batch, active, T, H,
-                               G, Dm, N, err_flags);
+                               G, Dm, N, node_ids, max_accept_len, err_flags);
         if (rc)
             return rc;
     }

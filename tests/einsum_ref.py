@@ -45,3 +45,42 @@ def prefill_dense(state, x, A, B, C, dt, dt_bias, D, z, G, softplus, lengths=Non
         s[live] = new[live]
         out[live, t] = y[live]
     return s, out
+
+
+def ancestor_path(parents, i):
+    """Root-to-node list of the nodes on node i's path (parents: list, -1 = root)."""
+    path = []
+    while i != -1:
+        path.append(i)
+        i = parents[i]
+    return path[::-1]
+
+
+def ddtree_dual(state, x, A, B, C, dt, dt_bias, D, G, softplus, parents):
+    """Tree verify in closed form, without any per-path state: for node i with path
+    j_0..j_k = i, unrolling the recurrence gives
+        s_i = W_i0 * s0 + sum_m W_im * B_jm * dt_jm * x_jm,  W_im = prod_{l>m} dA_jl,
+    with W_i0 the product over the whole path, and out_i = C_i . s_i + D * x_i.
+    state [b,H,Dm,N]; x [b,T,H,Dm]; B/C [b,T,G,N]; dt [b,T,H]; parents [b,T] (lists)."""
+    b, T, H, Dm = x.shape
+    grp = np.arange(H) // (H // G)
+    v = dt + (dt_bias[None, None, :] if dt_bias is not None else 0.0)
+    dte = np.logaddexp(0.0, v) if softplus else v
+    logdA = A[None, None, :] * dte                       # [b,T,H]
+    Bh, Ch = B[:, :, grp, :], C[:, :, grp, :]            # [b,T,H,N]
+    out = np.zeros(x.shape)
+    for r in range(b):
+        for i in range(T):
+            path = ancestor_path(parents[r], i)
+            total = sum(logdA[r, j] for j in path)       # [H]
+            a = np.einsum("hdn,hn->hd", state[r], Ch[r, i])
+            y = np.exp(total)[:, None] * a
+            after = np.zeros(H)                          # log of prod_{l>m} dA_jl
+            for j in reversed(path):
+                cb = np.einsum("hn,hn->h", Ch[r, i], Bh[r, j])
+                y = y + (np.exp(after) * dte[r, j] * cb)[:, None] * x[r, j]
+                after = after + logdA[r, j]
+            if D is not None:
+                y = y + D[:, None] * x[r, i]
+            out[r, i] = y
+    return out

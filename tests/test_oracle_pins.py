@@ -3,8 +3,9 @@
 Each test ties the oracle to a fact the pages or the mathematics fix: the decode
 formula of the Selective State Update page (TensorRT-Edge-LLM C++ API,
 invokeSelectiveStateUpdate), the prefill/stash and replay contracts on the same page,
-the padding contract of flashinfer.gdn_fused_decode_step (state_indices), closed forms,
-an independent vectorised formulation and the IEEE storage formats.
+the tree verify (invokeSelectiveStateUpdateDDTree) and the accepted-node replay on the
+same page, the padding contract of flashinfer.gdn_fused_decode_step (state_indices),
+closed forms, independent vectorised formulations and the IEEE storage formats.
 """
 
 import math
@@ -13,7 +14,7 @@ import numpy as np
 import pytest
 import torch
 
-from einsum_ref import decode_dense, f64, prefill_dense
+from einsum_ref import ancestor_path, ddtree_dual, decode_dense, f64, prefill_dense
 from linear_attention_recurrent_selective_b200.workloads import make_case, make_config
 
 F64 = torch.float64
@@ -519,3 +520,142 @@ def test_clear_slot_layers(orc):
             assert (c[3] == 0).all() and torch.equal(c[[0, 1, 2, 4]], c0[[0, 1, 2, 4]])
     orc.clear_slot_layers(r2, c2, 5, -1, 8 * 4, 2 * 4)
     assert all((r == 0).all() for r in r2) and all(c is None or (c == 0).all() for c in c2)
+
+
+# ---------------------------------------------------------------- tree verify (DDTree)
+
+def tree_case(seed, mode, **kw):
+    shape = dict(batch=3, P=6, T=9, H=4, G=2, Dm=3, N=8)
+    shape.update(kw)
+    return make_case(seed=seed, tree=mode, **shape)
+
+
+def test_ddtree_chain_equals_prefill_with_stash(orc):
+    """A chain tree's path to node i is tokens 0..i: the prefill over the same inputs."""
+    case = tree_case(40, "chain", x_dtype=torch.bfloat16, bc_dtype=torch.bfloat16)
+    out_t, st_t, err = orc.ddtree_case(case)
+    out_p, pool_p, st_p, _ = orc.prefill_case(case, stash=True)
+    assert err == 0
+    assert torch.equal(pool_p, case.pool)
+    for a, b in zip(st_t, st_p):
+        assert same_bits(a, b)
+    np.testing.assert_allclose(out_t.numpy(), out_p.numpy(), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", ["random", "forest", "shuffled"])
+def test_ddtree_matches_decodes_along_each_path(orc, mode):
+    case = tree_case(41, mode, state_dtype=F64)
+    out, _, err = orc.ddtree_case(case)
+    assert err == 0
+    idx = case.state_indices.long()
+    s0 = dense_state(case)[idx].numpy()
+    x, B, C, dt = f64(case.x), f64(case.B), f64(case.C), f64(case.dt)
+    for r in range(case.batch):
+        parents = case.parent_ids[r].tolist()
+        for i in range(case.T):
+            s = s0[r:r + 1].copy()
+            for j in ancestor_path(parents, i):
+                s, y = decode_dense(s, x[r:r + 1, j], f64(case.A), B[r:r + 1, j],
+                                    C[r:r + 1, j], dt[r:r + 1, j], f64(case.dt_bias),
+                                    f64(case.D), None, case.G, True)
+            np.testing.assert_allclose(out[r, i].numpy(), y[0], rtol=1e-12, atol=1e-12)
+
+
+def test_ddtree_matches_closed_form(orc):
+    case = tree_case(42, "shuffled", T=12, slow_decay=True, state_dtype=F64)
+    out, _, _ = orc.ddtree_case(case)
+    idx = case.state_indices.long()
+    want = ddtree_dual(dense_state(case)[idx].numpy(), f64(case.x), f64(case.A),
+                       f64(case.B), f64(case.C), f64(case.dt), f64(case.dt_bias),
+                       f64(case.D), case.G, True,
+                       [case.parent_ids[r].tolist() for r in range(case.batch)])
+    np.testing.assert_allclose(out.numpy(), want, rtol=1e-11, atol=1e-11)
+
+
+def test_ddtree_leaves_pool_and_handles_padding(orc):
+    case = tree_case(43, "random", batch=5, P=8, active=4, n_pad=1)
+    case.state_indices[3] = 8                         # out of range: skipped, flag 1
+    pool0 = case.pool.clone()
+    out, st, err = orc.ddtree_case(case)
+    assert err == 1
+    assert torch.equal(case.pool, pool0)
+    for b in range(case.batch):
+        si = int(case.state_indices[b])
+        if b >= case.active or si >= case.P:
+            assert torch.isnan(out[b]).all() and torch.isnan(st[1][b]).all()
+        elif si < 0:
+            assert (out[b] == 0).all() and torch.isnan(st[1][b]).all()
+        else:
+            assert not torch.isnan(out[b]).any()
+            assert torch.equal(st[1][b], case.x[b].float())
+            assert torch.equal(st[2][b], case.B[b].float())
+
+
+def test_ddtree_malformed_nodes_flagged_and_zeroed(orc):
+    case = tree_case(44, "random", batch=1, T=8, indices="none", P=1)
+    par = torch.tensor([[-1, 0, 1, 2, 1, 4, 5, 0]], dtype=torch.int32)
+    case.parent_ids = par.clone()
+    case.depths = torch.tensor([[0, 1, 2, 3, 2, 3, 4, 1]], dtype=torch.int32)
+    good, _, err = orc.ddtree_case(case)
+    assert err == 0
+    case.depths[0, 3] = 2                             # walk does not end at the root
+    case.parent_ids[0, 6] = 6                         # self-loop: 5 -> 6 -> 6 ...
+    case.depths[0, 6] = 9
+    case.parent_ids[0, 7] = 12                        # parent outside [0, T)
+    out, _, err = orc.ddtree_case(case)
+    assert err == 64
+    bad = [3, 6, 7]
+    assert (out[0, bad] == 0).all()
+    keep = [0, 1, 2, 4, 5]
+    assert same_bits(out[0, keep].contiguous(), good[0, keep].contiguous())
+
+
+@pytest.mark.parametrize("mode", ["random", "shuffled"])
+def test_replay_accepted_nodes_equals_decodes_along_path(orc, mode):
+    case = tree_case(45, mode, state_dtype=F64)
+    _, st, _ = orc.ddtree_case(case)
+    pool = case.pool.clone()
+    assert orc.replay(pool, st, case.accepted_lengths, state_indices=case.state_indices,
+                      batch=case.batch, T=case.T, H=4, G=2, Dm=3, N=8,
+                      node_ids=case.accepted_node_ids) == 0
+    idx = case.state_indices.long()
+    x, B, C, dt = f64(case.x), f64(case.B), f64(case.C), f64(case.dt)
+    for r in range(case.batch):
+        s = dense_state(case)[idx[r:r + 1]].numpy().copy()
+        k = int(case.accepted_lengths[r])
+        for j in case.accepted_node_ids[r, :k].tolist():
+            s, _ = decode_dense(s, x[r:r + 1, j], f64(case.A), B[r:r + 1, j], C[r:r + 1, j],
+                                dt[r:r + 1, j], f64(case.dt_bias), f64(case.D), None,
+                                case.G, True)
+        # the stash carries fp32 decay/dt factors
+        np.testing.assert_allclose(dense_state(case, pool)[idx[r]].numpy(), s[0],
+                                   rtol=1e-6, atol=1e-6)
+
+
+def test_replay_identity_node_ids_equal_plain_replay(orc):
+    case = make_case(seed=46, batch=4, P=6, T=5, H=2, G=1, Dm=4, N=8, lengths="accepted")
+    _, _, st, _ = orc.prefill_case(case, stash=True)
+    plain = case.pool.clone()
+    orc.replay(plain, st, case.accepted_lengths, state_indices=case.state_indices, batch=4,
+               T=5, H=2, G=1, Dm=4, N=8)
+    ids = torch.arange(5, dtype=torch.int32).repeat(4, 1)
+    by_ids = case.pool.clone()
+    orc.replay(by_ids, st, case.accepted_lengths, state_indices=case.state_indices, batch=4,
+               T=5, H=2, G=1, Dm=4, N=8, node_ids=ids)
+    assert same_bits(plain, by_ids)
+
+
+def test_replay_node_id_flags(orc):
+    case = tree_case(47, "random", batch=3, P=3, indices="none")
+    _, st, _ = orc.ddtree_case(case)
+    ids = case.accepted_node_ids[:, :4].contiguous()  # maxAcceptLen 4
+    ids[1] = torch.tensor([0, 3, 9, 2])               # 9 >= T
+    ids[2] = torch.tensor([0, 1, 2, 5])
+    acc = torch.tensor([2, 3, 7], dtype=torch.int32)  # 7 > maxAcceptLen: clamped to 4
+    ids[0] = torch.tensor([0, 1, 99, 99])             # beyond acc: never read
+    pool = case.pool.clone()
+    err = orc.replay(pool, st, acc, batch=3, T=9, H=4, G=2, Dm=3, N=8, node_ids=ids)
+    assert err == 2 | 64
+    assert torch.equal(dense_state(case, pool)[1], dense_state(case)[1])
+    assert not torch.equal(dense_state(case, pool)[0], dense_state(case)[0])
+    assert not torch.equal(dense_state(case, pool)[2], dense_state(case)[2])
