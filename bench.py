@@ -451,6 +451,64 @@ def form_layers(args, device, hbm_peak):
     return forms
 
 
+def form_ddtree(args, device, hbm_peak):
+    """Tree verify of one 128-node draft tree per row (batch 16, random recursive trees),
+    then the replay of each row's accepted root-to-node path through acceptedNodeIds.
+    The verify is FP32-issue bound (reported against the FP32 FMA peak), the replay HBM
+    bound."""
+    from linear_attention_recurrent_selective_b200 import ssu
+    from linear_attention_recurrent_selective_b200.workloads import make_config
+
+    steps, warm = max(3, min(args.steps, 50)), max(3, min(args.warmup, 5))
+    case = make_config("ddtree_b16_n128")
+    d = case.to(device)
+    f = dict(dtype=torch.float32, device=device)
+    b, T, H, G, Dm, N = case.batch, case.T, case.H, case.G, case.Dm, case.N
+    out = torch.empty_like(d.x)
+    st = (torch.empty(b, T, H, **f), torch.empty(b, T, H, Dm, **f),
+          torch.empty(b, T, G, N, **f), torch.empty(b, T, H, **f))
+
+    def verify():
+        ssu.ssu_ddtree(d.x, d.A, d.B, d.C, d.dt, d.pool, out, d.parent_ids, d.depths, st,
+                       dt_bias=d.dt_bias, D=d.D, state_indices=d.state_indices,
+                       slot_stride=case.slot_stride, P=case.P)
+
+    ms = time_launches(verify, steps, warm, device)
+    pairs = int((case.depths + 1).sum())          # (node, path node) pairs of all rows
+    # dense a_i = s0 . C_i per node, head and dim row; the path sums per (pair, head, dim
+    # row); C_i . B_j per (pair, group)
+    flop = 2 * b * H * T * Dm * N + 2 * pairs * H * Dm + 2 * pairs * G * N
+    xb = case.x.element_size()
+    vbytes = (b * H * Dm * N * 4 + 2 * b * T * H * Dm * xb + b * T * H * Dm * 4
+              + b * T * G * N * (2 * case.B.element_size() + 4) + b * T * H * 12 + 2 * b * T * 4)
+    sm = torch.cuda.get_device_properties(device).multi_processor_count
+    alu_peak = sm * 128 * 2 * 1.965e9 / 1e12
+    forms = {"ddtree": {
+        "workload": "ddtree_b16_n128", "batch": b, "nodes": b * T, "path_pairs": pairs,
+        "ms_per_launch": ms, "nodes_per_s": b * T / (ms / 1e3), "algorithmic_flop": flop,
+        "algorithmic_bytes": vbytes, "hbm_gbs": vbytes / (ms / 1e3) / 1e9,
+        "roofline": {"bound": "alu", "achieved": flop / (ms / 1e3) / 1e12, "peak": alu_peak,
+                     "unit": "TFLOP/s", "frac": flop / (ms / 1e3) / 1e12 / alu_peak,
+                     "traffic": None,
+                     "peak_source": "derived: SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz"}}}
+
+    pool = d.pool.clone()
+    acc, ids = d.accepted_lengths, d.accepted_node_ids
+    rms = time_launches(lambda: ssu.ssu_replay(pool, st, acc, state_indices=d.state_indices,
+                                               slot_stride=case.slot_stride, P=case.P,
+                                               accepted_node_ids=ids), steps, warm, device)
+    acc_h = case.accepted_lengths
+    rows, nacc = int((acc_h > 0).sum()), int(acc_h.sum())
+    rbytes = rows * H * Dm * N * 4 * 2 + nacc * (H * (4 + 4 + Dm * 4) + G * N * 4) + b * 4
+    forms["replay_nodes"] = {
+        "workload": "ddtree_b16_n128 accepted paths", "accepted_tokens": nacc,
+        "ms_per_launch": rms, "accepted_tokens_per_s": nacc / (rms / 1e3),
+        "roofline": {"bound": "hbm", "achieved": rbytes / (rms / 1e3) / 1e9, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": rbytes / (rms / 1e3) / 1e9 / hbm_peak,
+                     "traffic": None}}
+    return forms
+
+
 def cpu_baseline_decode(case, max_seconds=20.0):
     """The float64 oracle on whole decode steps of the same workload, timed on this host."""
     from oracle import oracle
@@ -488,11 +546,13 @@ def main_ours(args):
     device = torch.device("cuda", local if n_world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(device)
     hbm_peak, peak_src = measured_peaks()
-    if args.form in ("prefill", "replay", "layers"):   # one form alone, e.g. under ncu
+    if args.form in ("prefill", "replay", "layers", "ddtree"):   # one form alone
         if args.form == "prefill":
             forms = form_prefill(args, device, args.batch)
         elif args.form == "replay":
             forms = form_replay(args, device, hbm_peak, args.batch)
+        elif args.form == "ddtree":
+            forms = form_ddtree(args, device, hbm_peak)
         else:
             forms = form_layers(args, device, hbm_peak)
         if rank == 0:
@@ -526,7 +586,8 @@ def main_ours(args):
     }
     if n_world == 1 and not args.no_forms and args.form == "all":
         line["forms"] = {**form_prefill(args, device), **form_replay(args, device, hbm_peak),
-                         **form_layers(args, device, hbm_peak)}
+                         **form_layers(args, device, hbm_peak),
+                         **form_ddtree(args, device, hbm_peak)}
     if n_world == 1 and rank == 0 and not args.no_cpu_baseline and args.form == "all":
         line["cpu_baseline"] = cpu_baseline_decode(case)
     if rank == 0:
@@ -583,7 +644,7 @@ def parse(argv=None):
     ap.add_argument("--batch", type=int, default=0,
                     help="override the batch (pool = 2 x batch), e.g. for a small profile")
     ap.add_argument("--no-forms", action="store_true", help="skip the prefill/replay forms")
-    ap.add_argument("--form", choices=("all", "decode", "prefill", "replay", "layers"),
+    ap.add_argument("--form", choices=("all", "decode", "prefill", "replay", "layers", "ddtree"),
                     default="all",
                     help="run one kernel only (for profiling); its line carries that form")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -1,14 +1,16 @@
 /*
  * ssu.h -- C ABI of the B200 selective-state-update library (libssu.so).
  *
- * The Mamba selective state update over a paged recurrent-state pool, in its three
- * forms (single-token decode, multi-token prefill with an optional replay stash, and
- * the replay of accepted speculative tokens), plus slot clear and slot copy.
+ * The Mamba selective state update over a paged recurrent-state pool, in its forms
+ * (single-token decode, multi-token prefill with an optional replay stash, tree verify
+ * of a draft tree, and the replay of accepted speculative tokens or tree nodes), plus
+ * slot clear, slot copy and gather/scatter.
  *
  * Sources: the "Selective State Update" page of the TensorRT-Edge-LLM C++ API
  * (mamba_ssm::invokeSelectiveStateUpdate, invokeSelectiveStateUpdatePrefill,
- * struct MambaReplayLayerInfo, invokeMambaReplayReconstructBatched,
- * invokeMambaStateClear), the padding contract of the FlashInfer page
+ * invokeSelectiveStateUpdateDDTree, struct MambaReplayLayerInfo,
+ * invokeMambaReplayReconstructBatched, invokeMambaStateClear, invokeMambaStateGather,
+ * invokeMambaStateScatter), the padding contract of the FlashInfer page
  * "flashinfer.gdn_fused_decode_step" (parameters state_indices and ssm_state), and the
  * "Recurrent State Manager" page (clearSlot, clear, copySlotFrom).
  *
@@ -65,10 +67,12 @@ typedef enum {
     SSU_ERR_NULL = 1,         /* a required pointer is NULL, or the stash is partial */
     SSU_ERR_SHAPE = 2,        /* sizes inconsistent (H % G, active > batch, stride, ...) */
     SSU_ERR_DTYPE = 3,        /* dtype code not one of ssu_dtype */
-    SSU_ERR_UNSUPPORTED = 4,  /* dstate not in {8,16,32,64,128,256} */
+    SSU_ERR_UNSUPPORTED = 4,  /* dstate not in {8,16,32,64,128,256}, or (ssu_ddtree) a
+                                 tree whose tables exceed shared memory */
     SSU_ERR_CUDA = 5,         /* the kernel launch failed */
     SSU_ERR_ALIGN = 6         /* pool pointer or slot stride not 16-byte aligned, or (in
-                                 ssu_prefill / ssu_replay) B, C or the stash B not 16-byte
+                                 ssu_prefill / ssu_replay / ssu_ddtree) B, C or the stash B
+                                 not 16-byte
                                  aligned */
 } ssu_status;
 
@@ -79,8 +83,11 @@ enum {
     SSU_FLAG_NEGATIVE_LENGTH = 8, /* a negative length: treated as 0 */
     SSU_FLAG_TIMEOUT = 16,        /* an internal wait gave up after 2 s (never expected);
                                      the outputs of that launch are incomplete */
-    SSU_FLAG_LAYER = 32           /* a per-layer pointer was NULL or not 16-byte aligned:
+    SSU_FLAG_LAYER = 32,          /* a per-layer pointer was NULL or not 16-byte aligned:
                                      that layer was skipped */
+    SSU_FLAG_TREE = 64            /* ssu_ddtree: a node's parent walk was malformed (its
+                                     outputs are 0); replay: an accepted node id outside
+                                     [0, T) (the row was left untouched) */
 };
 
 /* Per-layer device pointers of a multi-layer replay: one entry per layer, in a device
@@ -160,14 +167,21 @@ int ssu_prefill(const void *x, int x_dtype, const float *A,
  * invokeMambaReplayReconstructBatched: for t < k_b = accepted_lengths[b],
  *     state = state * st_dA[b,t,h] + st_B[b,t,g,n] * st_dt[b,t,h] * st_U[b,t,h,d]
  * in place; the state is written once, and not at all when k_b == 0.
- *   stash buffers as written by ssu_prefill, with T their token extent;
- *   accepted_lengths [batch] int32 (required); no output.
+ *   stash buffers as written by ssu_prefill (or ssu_ddtree), with T their token (node)
+ *   extent; accepted_lengths [batch] int32 (required); no output.
+ *   accepted_node_ids [batch, max_accept_len] int32 (optional; the acceptedNodeIds and
+ *   maxAcceptLen arguments of invokeMambaReplayReconstructBatched): when given, the t-th
+ *   replayed token is stash entry accepted_node_ids[b][t] instead of t (the accepted
+ *   root-to-node path of a tree verify), and k_b is bounded by max_accept_len instead
+ *   of T. A row with an id outside [0, T) among its first k_b is left untouched and
+ *   flagged SSU_FLAG_TREE. When NULL, max_accept_len is ignored.
  */
 int ssu_replay(void *state, int state_dtype, int64_t slot_stride, int32_t P,
                const float *st_dA, const float *st_U, const float *st_B,
                const float *st_dt, const int32_t *accepted_lengths,
                const int32_t *state_indices, int32_t batch, int32_t active_batch,
                int32_t T, int32_t nheads, int32_t ngroups, int32_t dim, int32_t dstate,
+               const int32_t *accepted_node_ids, int32_t max_accept_len,
                int32_t *err_flags, ssu_stream_t stream);
 
 /*
@@ -183,7 +197,41 @@ int ssu_replay_layers(const ssu_replay_layer *layers, int32_t num_layers, int st
                       int64_t slot_stride, int32_t P, const int32_t *accepted_lengths,
                       const int32_t *state_indices, int32_t batch, int32_t active_batch,
                       int32_t T, int32_t nheads, int32_t ngroups, int32_t dim, int32_t dstate,
+                      const int32_t *accepted_node_ids, int32_t max_accept_len,
                       int32_t *err_flags, ssu_stream_t stream);
+
+/*
+ * ssu_ddtree -- tree verify: every node of one draft tree per row, each evaluated from the
+ * committed state along its own ancestor path.
+ * Selective State Update page, mamba_ssm::invokeSelectiveStateUpdateDDTree: the committed
+ * state is only read; for node i of row b the recurrence of ssu_decode runs from the
+ * committed state over the nodes on i's path (found by following tree_parent_ids from i
+ * to the root), in root-to-node order, and out[b,i] is node i's output there (no z gate);
+ * node i's own replay tuple goes to the stash at position i.
+ *
+ *   x, out [batch, T, H, Dm] x_dtype; B, C [batch, T, G, N] bc_dtype (B 16-byte
+ *   aligned); dt [batch, T, H] fp32; T = nodes per tree, 1..128 (the verify budget).
+ *   tree_parent_ids [batch, T] int32: parent node of each node, -1 for a node attached
+ *   directly to the committed state.
+ *   tree_depths [batch, T] int32: number of tree ancestors of each node (0 when its
+ *   parent is -1). A node whose walk does not take exactly that many steps inside
+ *   [0, T) and then reach -1 is malformed: its outputs are 0 and SSU_FLAG_TREE is set.
+ *   Stash (required, fp32, every node of every non-padding row): st_dA [batch, T, H],
+ *   st_U [batch, T, H, Dm], st_B [batch, T, G, N], st_dt [batch, T, H], as in
+ *   ssu_prefill; replay an accepted path with ssu_replay and accepted_node_ids.
+ *   A padding row writes zeros to out at every node and nothing else.
+ * Returns SSU_ERR_SHAPE for T > 128, SSU_ERR_UNSUPPORTED when the row's tables do not fit
+ * in shared memory (about T (dstate + 4) x 4 + 5 T (T + 1) + T x 64 x element bytes of x
+ * bytes must stay under 227 KB: every T up to 128 for dstate <= 128).
+ */
+int ssu_ddtree(const void *x, int x_dtype, const float *A, const void *B, const void *C,
+               int bc_dtype, const float *dt, const float *dt_bias, const float *D,
+               const void *state, int state_dtype, int64_t slot_stride, int32_t P, void *out,
+               const int32_t *tree_parent_ids, const int32_t *tree_depths,
+               const int32_t *state_indices, float *st_dA, float *st_U, float *st_B,
+               float *st_dt, int32_t batch, int32_t active_batch, int32_t T, int32_t nheads,
+               int32_t ngroups, int32_t dim, int32_t dstate, int dt_softplus,
+               int32_t *err_flags, ssu_stream_t stream);
 
 /*
  * pool_clear_slot -- zero one slot, or every slot when slot == -1.

@@ -4,8 +4,9 @@
 // (so it stays legal under CUDA-graph capture), returns an ssu_status error without
 // launching anything when a check fails, and otherwise enqueues exactly one kernel on
 // the caller's stream. Values that live on the device (stateIndices, contextLengths,
-// acceptedLengths) are checked in-kernel, as the padding contract of the FlashInfer page
-// flashinfer.gdn_fused_decode_step requires for graph replay.
+// acceptedLengths, tree parents and depths, accepted node ids) are checked in-kernel,
+// as the padding contract of the FlashInfer page flashinfer.gdn_fused_decode_step
+// requires for graph replay.
 #include "ssu_common.cuh"
 
 namespace {
@@ -160,10 +161,11 @@ int ssu_replay(void *state, int state_dtype, int64_t slot_stride, int32_t P,
                const float *st_dA, const float *st_U, const float *st_B, const float *st_dt,
                const int32_t *accepted_lengths, const int32_t *state_indices,
                int32_t batch, int32_t active_batch, int32_t T, int32_t nheads,
-               int32_t ngroups, int32_t dim, int32_t dstate, int32_t *err_flags,
+               int32_t ngroups, int32_t dim, int32_t dstate,
+               const int32_t *accepted_node_ids, int32_t max_accept_len, int32_t *err_flags,
                ssu_stream_t stream)
 {
-    if (T < 0)
+    if (T < 0 || (accepted_node_ids && max_accept_len < 0))
         return SSU_ERR_SHAPE;
     int rc = check_sizes(state_dtype, slot_stride, P, state_indices, batch, active_batch,
                          nheads, ngroups, dim, dstate);
@@ -185,6 +187,7 @@ int ssu_replay(void *state, int state_dtype, int64_t slot_stride, int32_t P,
     a.st_dt = st_dt;
     a.acc = accepted_lengths;
     a.idx = state_indices;
+    a.nodes = accepted_node_ids;
     a.err = err_flags;
     a.slot_stride = slot_stride;
     a.P = P;
@@ -195,6 +198,7 @@ int ssu_replay(void *state, int state_dtype, int64_t slot_stride, int32_t P,
     a.G = ngroups;
     a.Dm = dim;
     a.N = dstate;
+    a.max_accept = accepted_node_ids ? max_accept_len : T;
     return finish(ssu::launch_replay(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -202,9 +206,10 @@ int ssu_replay_layers(const ssu_replay_layer *layers, int32_t num_layers, int st
                       int64_t slot_stride, int32_t P, const int32_t *accepted_lengths,
                       const int32_t *state_indices, int32_t batch, int32_t active_batch,
                       int32_t T, int32_t nheads, int32_t ngroups, int32_t dim, int32_t dstate,
+                      const int32_t *accepted_node_ids, int32_t max_accept_len,
                       int32_t *err_flags, ssu_stream_t stream)
 {
-    if (T < 0 || num_layers < 0)
+    if (T < 0 || num_layers < 0 || (accepted_node_ids && max_accept_len < 0))
         return SSU_ERR_SHAPE;
     int rc = check_sizes(state_dtype, slot_stride, P, state_indices, batch, active_batch,
                          nheads, ngroups, dim, dstate);
@@ -221,6 +226,7 @@ int ssu_replay_layers(const ssu_replay_layer *layers, int32_t num_layers, int st
     a.st_dA = a.st_U = a.st_B = a.st_dt = nullptr;
     a.acc = accepted_lengths;
     a.idx = state_indices;
+    a.nodes = accepted_node_ids;
     a.err = err_flags;
     a.slot_stride = slot_stride;
     a.P = P;
@@ -231,7 +237,46 @@ int ssu_replay_layers(const ssu_replay_layer *layers, int32_t num_layers, int st
     a.G = ngroups;
     a.Dm = dim;
     a.N = dstate;
+    a.max_accept = accepted_node_ids ? max_accept_len : T;
     return finish(ssu::launch_replay(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int ssu_ddtree(const void *x, int x_dtype, const float *A, const void *B, const void *C,
+               int bc_dtype, const float *dt, const float *dt_bias, const float *D,
+               const void *state, int state_dtype, int64_t slot_stride, int32_t P, void *out,
+               const int32_t *tree_parent_ids, const int32_t *tree_depths,
+               const int32_t *state_indices, float *st_dA, float *st_U, float *st_B,
+               float *st_dt, int32_t batch, int32_t active_batch, int32_t T, int32_t nheads,
+               int32_t ngroups, int32_t dim, int32_t dstate, int dt_softplus,
+               int32_t *err_flags, ssu_stream_t stream)
+{
+    if (!valid_dtype(x_dtype) || !valid_dtype(bc_dtype))
+        return SSU_ERR_DTYPE;
+    if (T < 0 || T > 128)
+        return SSU_ERR_SHAPE;
+    int rc = check_sizes(state_dtype, slot_stride, P, state_indices, batch, active_batch,
+                         nheads, ngroups, dim, dstate);
+    if (rc != SSU_OK || active_batch == 0 || T == 0)
+        return rc;
+    if (!x || !A || !B || !C || !dt || !state || !out || !tree_parent_ids || !tree_depths ||
+        !st_dA || !st_U || !st_B || !st_dt)
+        return SSU_ERR_NULL;
+    if ((rc = check_pool_alignment(state, state_dtype, slot_stride)) != SSU_OK)
+        return rc;
+    if (!aligned16(B))
+        return SSU_ERR_ALIGN;
+    ssu::TreeArgs a;
+    a.d = pack_decode(x, x_dtype, A, B, C, bc_dtype, dt, dt_bias, D, nullptr,
+                      const_cast<void *>(state), slot_stride, P, out, state_indices, batch,
+                      active_batch, nheads, ngroups, dim, dstate, dt_softplus, err_flags);
+    a.parents = tree_parent_ids;
+    a.depths = tree_depths;
+    a.st_dA = st_dA;
+    a.st_U = st_U;
+    a.st_B = st_B;
+    a.st_dt = st_dt;
+    a.T = T;
+    return finish(ssu::launch_ddtree(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int pool_clear_slot_layers(const ssu_layer_states *layers, int32_t num_layers, int32_t P,
@@ -316,7 +361,9 @@ const char *ssu_status_string(int status)
     case SSU_ERR_NULL: return "SSU_ERR_NULL: a required pointer is NULL or the stash is partial";
     case SSU_ERR_SHAPE: return "SSU_ERR_SHAPE: inconsistent sizes";
     case SSU_ERR_DTYPE: return "SSU_ERR_DTYPE: unknown dtype code";
-    case SSU_ERR_UNSUPPORTED: return "SSU_ERR_UNSUPPORTED: dstate not in {8,16,32,64,128,256}";
+    case SSU_ERR_UNSUPPORTED:
+        return "SSU_ERR_UNSUPPORTED: dstate not in {8,16,32,64,128,256}, or a tree too large "
+               "for shared memory";
     case SSU_ERR_CUDA: return "SSU_ERR_CUDA: kernel launch failed";
     case SSU_ERR_ALIGN: return "SSU_ERR_ALIGN: pool or slot stride not 16-byte aligned";
     default: return "unknown ssu_status";

@@ -49,15 +49,25 @@ struct ReplayArgs {
     const float *st_dA, *st_U, *st_B, *st_dt;
     const int32_t *acc;
     const int32_t *idx;
+    const int32_t *nodes;     // acceptedNodeIds [batch, max_accept] or NULL (token t = t)
     int32_t *err;
     int64_t slot_stride;
-    int32_t P, batch, active, T, H, G, Dm, N;
+    int32_t P, batch, active, T, H, G, Dm, N, max_accept;
+};
+
+struct TreeArgs {
+    DecodeArgs d;             // x/B/C/dt/out carry a node axis [batch, T, ...]; z unused
+    const int32_t *parents;   // treeParentIds [batch, T]
+    const int32_t *depths;    // treeDepths [batch, T]
+    float *st_dA, *st_U, *st_B, *st_dt;
+    int32_t T;
 };
 
 // Host launchers, one per kernel family; each returns SSU_OK or SSU_ERR_UNSUPPORTED.
 int launch_decode(const DecodeArgs &a, int state_dtype, cudaStream_t s);
 int launch_prefill(const PrefillArgs &a, int state_dtype, cudaStream_t s);
 int launch_replay(const ReplayArgs &a, int state_dtype, cudaStream_t s);
+int launch_ddtree(const TreeArgs &a, int state_dtype, cudaStream_t s);
 int launch_clear(void *pool, int64_t bytes, cudaStream_t s);
 int launch_copy(void *dst, const void *src, int64_t bytes, cudaStream_t s);
 int launch_clear_layers(const ssu_layer_states *layers, int32_t num_layers, int32_t P,

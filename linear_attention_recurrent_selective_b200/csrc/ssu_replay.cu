@@ -9,6 +9,11 @@
 // (dA = exp(A * dt_eff), dt = dt_eff, U = x), the same association the decode and
 // prefill kernels use, so fp32 results agree bit for bit with the decode steps.
 //
+// With acceptedNodeIds ([batch, maxAcceptLen], the tree-accept form written for the tree
+// verify's stash), the t-th replayed token is stash entry acceptedNodeIds[b][t] and the
+// accepted count is bounded by maxAcceptLen; a row with an id outside [0, T) among its
+// accepted tokens is left untouched and flagged.
+//
 // invokeMambaReplayReconstructBatched also takes a device array of per-layer pointers
 // (MambaReplayLayerInfo) and replays every layer in the same launch; units are numbered
 // layer-major, so consecutive warps stream through one layer's pool at a time.
@@ -79,17 +84,44 @@ __device__ __forceinline__ LayerPtrs layer_ptrs(const ReplayArgs &a, int layer)
     return L;
 }
 
+// Accepted count of a row whose accepted node ids are not all inside [0, T): the row is
+// left untouched and SSU_FLAG_TREE reported.
+constexpr int kBadNodes = -0x40000000;
+
+// Stash entry of the t-th replayed token of row b: t itself, or acceptedNodeIds[b][t]
+// (the tree-accept form); ids outside [0, T) map to entry 0 so that a prefetch never
+// leaves the stash (such rows never use the values).
+__device__ __forceinline__ int entry_of(const ReplayArgs &a, int b, int t)
+{
+    if (!a.nodes)
+        return t;
+    const int e = a.nodes[(int64_t)b * a.max_accept + t];
+    return e >= 0 && e < a.T ? e : 0;
+}
+
 struct ReplayRows {
     const ReplayArgs *a;
     __device__ __forceinline__ UnitRes resolve(const LUnit &lu) const
     {
         const LayerPtrs L = layer_ptrs(*a, lu.layer);
         const int b = lu.un.b;
-        return UnitRes{L.ok ? L.state : nullptr, a->idx ? a->idx[b] : b, a->acc[b]};
+        int acc = a->acc[b];
+        if (a->nodes) {
+            const int k = min(acc, a->max_accept);
+            for (int t = 0; t < k; ++t) {
+                const int e = a->nodes[(int64_t)b * a->max_accept + t];
+                if (e < 0 || e >= a->T) {
+                    acc = kBadNodes;
+                    break;
+                }
+            }
+        }
+        return UnitRes{L.ok ? L.state : nullptr, a->idx ? a->idx[b] : b, acc};
     }
     __device__ __forceinline__ bool moves(const UnitRes &r) const
     {
-        return r.pool != nullptr && r.slot >= 0 && r.slot < a->P && min(r.extra, a->T) > 0;
+        return r.pool != nullptr && r.slot >= 0 && r.slot < a->P &&
+               min(r.extra, a->max_accept) > 0;
     }
 };
 
@@ -131,8 +163,8 @@ ssu_replay_kernel(const __grid_constant__ ReplayArgs a, const int cph, const int
         float pdA[kPre], pdt[kPre], pB[kPre][G::E], pU[kPre][G::XR];
 #pragma unroll
         for (int t = 0; t < kPre; ++t) {
-            if (t < T && L.ok) {
-                const int64_t bt = (int64_t)un.b * T + t;
+            if (t < a.max_accept && L.ok) {
+                const int64_t bt = (int64_t)un.b * T + entry_of(a, un.b, t);
                 pdA[t] = L.dA[bt * H + un.h];
                 pdt[t] = L.dt[bt * H + un.h];
                 load_cols<G>(L.B + (bt * a.G + g) * N, ln, pB[t]);
@@ -150,7 +182,7 @@ ssu_replay_kernel(const __grid_constant__ ReplayArgs a, const int cph, const int
             const int s = c % kStages;
             r2 = make_int2(w.ctl->slot[s], w.ctl->extra[s]);
             if (w.ctl->moves[s]) {
-                const int k = min(r2.y, T);
+                const int k = min(r2.y, a.max_accept);
                 const int rt = min(G::RT, un.rows - j * G::RT);
                 const int r0 = un.row0 + j * G::RT;
                 const uint8_t *buf = w.ring + s * kTileBytes;
@@ -189,7 +221,7 @@ ssu_replay_kernel(const __grid_constant__ ReplayArgs a, const int cph, const int
                 }
                 // longer acceptances: the remaining tokens straight from the stash
                 for (int t = kPre; t < k; ++t) {
-                    const int64_t bt = (int64_t)un.b * T + t;
+                    const int64_t bt = (int64_t)un.b * T + entry_of(a, un.b, t);
                     const float dA = L.dA[bt * H + un.h];
                     const float dte = L.dt[bt * H + un.h];
                     const float *Ut = L.U + (bt * H + un.h) * Dm + r0;
@@ -228,7 +260,9 @@ ssu_replay_kernel(const __grid_constant__ ReplayArgs a, const int cph, const int
             if (lu.layer == 0) {
                 if (r2.x >= a.P)
                     atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
-                else if (r2.x >= 0 && r2.y > T)
+                else if (r2.x >= 0 && r2.y == kBadNodes)
+                    atomicOr(a.err, SSU_FLAG_TREE);
+                else if (r2.x >= 0 && r2.y > a.max_accept)
                     atomicOr(a.err, SSU_FLAG_ACCEPTED_RANGE);
                 else if (r2.x >= 0 && r2.y < 0)
                     atomicOr(a.err, SSU_FLAG_NEGATIVE_LENGTH);

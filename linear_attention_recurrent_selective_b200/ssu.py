@@ -11,7 +11,10 @@ Semantics (Selective State Update page of the TensorRT-Edge-LLM C++ API):
                times silu(z) when z is given (invokeSelectiveStateUpdate)
   ssu_prefill  the same over [batch, T] tokens in one launch, optional replay stash
                (invokeSelectiveStateUpdatePrefill)
-  ssu_replay   re-apply the first acceptedLengths[b] stashed tokens (MambaReplayLayerInfo)
+  ssu_ddtree   tree verify: every node of a draft tree from the committed state along its
+               ancestor path, stash per node (invokeSelectiveStateUpdateDDTree)
+  ssu_replay   re-apply the first acceptedLengths[b] stashed tokens, or the accepted
+               tree nodes acceptedNodeIds[b][:acceptedLengths[b]] (MambaReplayLayerInfo)
   pool_clear_slot / pool_copy_slot  slot maintenance (invokeMambaStateClear;
                Recurrent State Manager clearSlot / copySlotFrom)
 """
@@ -34,12 +37,13 @@ FLAG_ACCEPTED_RANGE = 2
 FLAG_CONTEXT_RANGE = 4
 FLAG_NEGATIVE_LENGTH = 8
 FLAG_TIMEOUT = 16
+FLAG_LAYER = 32
+FLAG_TREE = 64
 
 # Every C entry point declared in include/ssu.h, in declaration order.
 ENTRY_POINTS = ("ssu_decode", "ssu_prefill", "ssu_replay", "ssu_replay_layers",
-                "pool_clear_slot", "pool_copy_slot", "pool_clear_slot_layers", "pool_gather",
-                "pool_scatter", "ssu_status_string")
-FLAG_LAYER = 32
+                "ssu_ddtree", "pool_clear_slot", "pool_copy_slot", "pool_clear_slot_layers",
+                "pool_gather", "pool_scatter", "ssu_status_string")
 
 # Byte layouts of the per-layer pointer records of include/ssu.h (packed pointers).
 REPLAY_LAYER_FIELDS = 5     # state, st_dA, st_U, st_B, st_dt
@@ -80,9 +84,11 @@ def lib() -> ctypes.CDLL:
     L.ssu_prefill.argtypes = [vp, ci, vp, vp, vp, ci, vp, vp, vp, vp, vp, ci, i64, i32, vp, vp,
                               vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, ci, vp, vp]
     L.ssu_replay.argtypes = [vp, ci, i64, i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
-                             i32, i32, vp, vp]
+                             i32, i32, vp, i32, vp, vp]
     L.ssu_replay_layers.argtypes = [vp, i32, ci, i64, i32, vp, vp, i32, i32, i32, i32, i32,
-                                    i32, i32, vp, vp]
+                                    i32, i32, vp, i32, vp, vp]
+    L.ssu_ddtree.argtypes = [vp, ci, vp, vp, vp, ci, vp, vp, vp, vp, ci, i64, i32, vp, vp, vp,
+                             vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, ci, vp, vp]
     L.pool_clear_slot.argtypes = [vp, i64, i32, i32, vp]
     L.pool_copy_slot.argtypes = [vp, i32, i32, vp, i32, i32, i64, vp]
     L.pool_clear_slot_layers.argtypes = [vp, i32, i32, i32, i64, i64, vp]
@@ -196,9 +202,19 @@ def ssu_prefill(x, A, B, C, dt, state, out, *, dt_bias=None, D=None, z=None,
     return out
 
 
+def _node_ids(accepted_node_ids):
+    if accepted_node_ids is None:
+        return None, 0
+    if accepted_node_ids.dim() != 2:
+        raise ValueError("accepted_node_ids must be [batch, maxAcceptLen]")
+    return _ptr(accepted_node_ids, "accepted_node_ids", torch.int32), accepted_node_ids.shape[1]
+
+
 def ssu_replay(state, stash, accepted_lengths, *, state_indices=None, active_batch=None,
-               err_flags=None, slot_stride=None, P=None, stream=None):
-    """Re-apply the first accepted_lengths[b] stashed tokens to the pool, in place."""
+               err_flags=None, slot_stride=None, P=None, accepted_node_ids=None, stream=None):
+    """Re-apply the first accepted_lengths[b] stashed tokens to the pool, in place; with
+    ``accepted_node_ids`` [batch, maxAcceptLen] token t of row b is stash entry
+    accepted_node_ids[b, t] (an accepted path of a tree verify)."""
     sdA, sU, sB, sdt = stash
     batch, T, H, Dm = sU.shape
     G, N = sB.shape[2], sB.shape[3]
@@ -210,8 +226,37 @@ def ssu_replay(state, stash, accepted_lengths, *, state_indices=None, active_bat
         _ptr(sdA, "stash dA", f32), _ptr(sU, "stash U", f32), _ptr(sB, "stash B", f32),
         _ptr(sdt, "stash dt", f32), _ptr(accepted_lengths, "accepted_lengths", torch.int32),
         _ptr(state_indices, "state_indices", torch.int32), batch, active, T, H, G, Dm, N,
-        _ptr(err_flags, "err_flags", torch.int32), _stream(stream))
+        *_node_ids(accepted_node_ids), _ptr(err_flags, "err_flags", torch.int32),
+        _stream(stream))
     _check("ssu_replay", rc)
+
+
+def ssu_ddtree(x, A, B, C, dt, state, out, parent_ids, depths, stash, *, dt_bias=None,
+               D=None, state_indices=None, active_batch=None, dt_softplus=True,
+               err_flags=None, slot_stride=None, P=None, stream=None):
+    """Tree verify of one draft tree of T <= 128 nodes per row. x/out [batch,T,H,Dm];
+    B/C [batch,T,G,N]; dt [batch,T,H]; parent_ids/depths [batch,T] int32; ``stash`` =
+    (dA [b,T,H], U [b,T,H,Dm], B [b,T,G,N], dt [b,T,H]) fp32, written for every node.
+    The pool is only read."""
+    batch, T, H, Dm = x.shape
+    G, N = B.shape[2], B.shape[3]
+    active = batch if active_batch is None else active_batch
+    stride, P = _pool_geometry(state, slot_stride, P, H * Dm * N)
+    if out.dtype != x.dtype or out.shape != x.shape:
+        raise ValueError("out must match x in shape and dtype")
+    f32, i32 = torch.float32, torch.int32
+    sdA, sU, sB, sdt = stash
+    rc = lib().ssu_ddtree(
+        _ptr(x, "x"), _dt(x, "x"), _ptr(A, "A", f32), _ptr(B, "B"), _ptr(C, "C", B.dtype),
+        _dt(B, "B"), _ptr(dt, "dt", f32), _ptr(dt_bias, "dt_bias", f32), _ptr(D, "D", f32),
+        ctypes.c_void_p(state.data_ptr()), _dt(state, "state"), stride, P, _ptr(out, "out"),
+        _ptr(parent_ids, "parent_ids", i32), _ptr(depths, "depths", i32),
+        _ptr(state_indices, "state_indices", i32), _ptr(sdA, "stash dA", f32),
+        _ptr(sU, "stash U", f32), _ptr(sB, "stash B", f32), _ptr(sdt, "stash dt", f32),
+        batch, active, T, H, G, Dm, N, int(bool(dt_softplus)),
+        _ptr(err_flags, "err_flags", i32), _stream(stream))
+    _check("ssu_ddtree", rc)
+    return out
 
 
 def pool_clear_slot(pool, slot, *, slot_bytes=None, P=None, stream=None):
@@ -266,7 +311,7 @@ def layer_states_table(layers, device=None):
 
 def ssu_replay_layers(table, num_layers, like_state, like_stash, accepted_lengths, *,
                       state_indices=None, active_batch=None, err_flags=None, slot_stride=None,
-                      P=None, stream=None):
+                      P=None, accepted_node_ids=None, stream=None):
     """ssu_replay over ``num_layers`` layers in one launch. ``table`` comes from
     ``replay_layer_table``; ``like_state`` / ``like_stash`` are any one layer's pool and
     stash, which give the (shared) geometry and dtypes."""
@@ -279,7 +324,8 @@ def ssu_replay_layers(table, num_layers, like_state, like_stash, accepted_length
         _ptr(table, "layer table", torch.int64), num_layers, _dt(like_state, "state"), stride,
         P, _ptr(accepted_lengths, "accepted_lengths", torch.int32),
         _ptr(state_indices, "state_indices", torch.int32), batch, active, T, H, G, Dm, N,
-        _ptr(err_flags, "err_flags", torch.int32), _stream(stream))
+        *_node_ids(accepted_node_ids), _ptr(err_flags, "err_flags", torch.int32),
+        _stream(stream))
     _check("ssu_replay_layers", rc)
 
 

@@ -48,13 +48,28 @@ def prefill(case, pool=None, stash=False, err=True):
     return out.cpu(), pool.cpu(), st_cpu, (int(e.item()) if err else None)
 
 
-def replay(case, stash, accepted, pool=None, err=True):
+def replay(case, stash, accepted, pool=None, err=True, node_ids=None):
     d = dev(case)
     pool = d.pool.clone() if pool is None else pool
     st = tuple(t.cuda() for t in stash)
     e = torch.zeros(1, dtype=torch.int32, device="cuda") if err else None
     ssu.ssu_replay(pool, st, accepted.cuda(), state_indices=d.state_indices,
                    active_batch=case.active, err_flags=e, slot_stride=case.slot_stride,
-                   P=case.P)
+                   P=case.P, accepted_node_ids=None if node_ids is None else node_ids.cuda())
     torch.cuda.synchronize()
     return pool.cpu(), (int(e.item()) if err else None)
+
+
+def ddtree(case, pool=None, err=True):
+    """Tree verify of a tree case; returns (out, pool after, stash, err) on the host."""
+    d = dev(case)
+    pool = d.pool.clone() if pool is None else pool
+    out = torch.full_like(d.x, NAN)
+    st = new_stash(case)
+    e = torch.zeros(1, dtype=torch.int32, device="cuda") if err else None
+    ssu.ssu_ddtree(d.x, d.A, d.B, d.C, d.dt, pool, out, d.parent_ids, d.depths, st,
+                   dt_bias=d.dt_bias, D=d.D, state_indices=d.state_indices,
+                   active_batch=case.active, dt_softplus=case.dt_softplus, err_flags=e,
+                   slot_stride=case.slot_stride, P=case.P)
+    torch.cuda.synchronize()
+    return out.cpu(), pool.cpu(), tuple(t.cpu() for t in st), (int(e.item()) if err else None)

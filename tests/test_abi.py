@@ -77,9 +77,14 @@ def test_prefill_rejects_partial_stash(L):
 
 def test_replay_and_pool_reject_bad_arguments(L):
     assert L.ssu_replay(P16, 0, 8192, 8, P16, P16, P16, P16, None, None, 4, 4, 5, 1, 1, 64,
-                        128, None, None) == 1
+                        128, None, 0, None, None) == 1
     assert L.ssu_replay(P16, 0, 8192, 8, P16, P16, ctypes.c_void_p(260), P16, P16, None, 4,
-                        4, 5, 1, 1, 64, 128, None, None) == 6
+                        4, 5, 1, 1, 64, 128, None, 0, None, None) == 6
+    # accepted node ids with a negative width
+    assert L.ssu_replay(P16, 0, 8192, 8, P16, P16, P16, P16, P16, None, 4, 4, 5, 1, 1, 64,
+                        128, P16, -1, None, None) == 2
+    assert L.ssu_replay_layers(P16, 2, 0, 8192, 8, P16, None, 4, 4, 5, 1, 1, 64, 128, P16,
+                               -3, None, None) == 2
     assert L.pool_clear_slot(P16, 1024, 4, 4, None) == 2
     assert L.pool_clear_slot(P16, 1024, 4, -2, None) == 2
     assert L.pool_clear_slot(None, 1024, 4, 0, None) == 1
@@ -92,3 +97,29 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ssu, "_lib", None)
     with pytest.raises(ssu.SSULibraryMissing):
         ssu.lib()
+
+
+def ddtree_args(**kw):
+    a = dict(x=P16, x_dt=2, A=P16, B=P16, C=P16, bc_dt=2, dt=P16, dt_bias=None, D=None,
+             state=P16, state_dt=0, stride=80 * 64 * 128, P=32, out=P16, par=P16, dep=P16,
+             idx=P16, sdA=P16, sU=P16, sB=P16, sdt=P16, batch=16, active=16, T=128, H=80,
+             G=1, Dm=64, N=128, sp=1, err=None, stream=None)
+    a.update(kw)
+    return list(a.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(par=None), 1), (dict(dep=None), 1), (dict(sU=None), 1), (dict(out=None), 1),
+    (dict(x_dt=5), 3), (dict(T=129), 2), (dict(T=-1), 2), (dict(G=3), 2),
+    (dict(N=24, stride=80 * 64 * 24), 4),
+    (dict(B=ctypes.c_void_p(258)), 6), (dict(state=ctypes.c_void_p(264)), 6),
+])
+def test_ddtree_rejects_bad_arguments(L, kw, status):
+    assert L.ssu_ddtree(*ddtree_args(**kw)) == status
+
+
+def test_ddtree_empty_calls_need_no_pointers(L):
+    nulls = dict(x=None, A=None, B=None, C=None, dt=None, state=None, out=None, par=None,
+                 dep=None, sdA=None, sU=None, sB=None, sdt=None)
+    assert L.ssu_ddtree(*ddtree_args(active=0, **nulls)) == 0
+    assert L.ssu_ddtree(*ddtree_args(T=0, **nulls)) == 0
