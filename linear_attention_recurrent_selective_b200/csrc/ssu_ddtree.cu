@@ -25,11 +25,17 @@
 //     parent -1; otherwise the node is malformed: outputs 0, SSU_FLAG_TREE);
 //   * C of every node widened to fp32 (rows padded against bank conflicts);
 //   * for every node i and every node j_m on its path: j_m and cb = C_i . B_jm.
-// Per item, the path coefficients w_im * dt_jm * cb and W_i are formed once per node;
-// a lane holds two dim rows of the committed state over one column group (64 columns at
-// dstate 128) in registers and accumulates a_i with packed FP32 FMAs against broadcast
-// shared loads of C_i; the column groups' partial sums meet in shared memory, and the
-// epilogue adds the path sums and writes the outputs.
+// The committed-state rows of the next item and its x tile are fetched by cp.async while
+// the current item computes: coalesced 16-byte copies into shared memory (the state rows
+// with an XOR swizzle of their 16-byte chunks, so that the row-per-lane reads below are
+// free of bank conflicts; the x tile double-buffered when it fits), and the next item's
+// dt is loaded into registers early. Per item, the path coefficients w_im * dt_jm * cb
+// and W_i are formed once per node; a lane holds two dim rows of the committed state
+// over one column group (64 columns at dstate 128) in registers and accumulates a_i with
+// packed FP32 FMAs against broadcast shared loads of C_i; the same warps add the path
+// sums, the column groups' partial sums meet in shared memory (two buffers, so one
+// barrier per chunk of nodes), and the epilogue adds D x and stores.
+#include "ssu_async.cuh"
 #include "ssu_common.cuh"
 
 namespace ssu {
@@ -38,32 +44,36 @@ namespace {
 constexpr int kThreads = 256;      // 8 warps, one CTA per SM
 constexpr int kTile = 64;          // dim rows per work item, two per lane
 constexpr int kMaxNodes = 128;     // the verify budget
-constexpr int kChunk = 16;         // nodes whose a_i are formed between two barriers
+constexpr int kSmemMax = 227 * 1024;
+constexpr int kBatch = 8;          // loads in flight per thread in the plain-load loops
 
 template <int N> struct TGeo {
-    static constexpr int CH = N > 64 ? N / 64 : 1;    // column groups
-    static constexpr int K = N / CH;                  // state columns per lane
-    static constexpr int NG = (kThreads / 32) / CH;   // node groups
-    static constexpr int NPG = kChunk / NG;           // nodes per group and chunk
+    static constexpr int KP = N < 128 ? N : 128;      // state columns per pass (per lane)
+    static constexpr int NP = N / KP;                 // passes over dstate
     static constexpr int CP = N + 4;                  // padded fp32 row of C (floats)
-    static_assert(K % 4 == 0 && NPG >= 1 && NG * NPG == kChunk, "tree geometry");
+    static_assert(KP % 8 == 0 || KP == 8, "tree geometry");
 };
 
+constexpr int kRowWarps = 2;                          // warps per 64-row dim tile
+constexpr int kNodeGroups = kThreads / 32 / kRowWarps;  // warp w takes nodes w/2 + 4k
+
 // Shared-memory layout (byte offsets, 16-byte aligned). E = T (T + 1) / 2 bounds the
-// number of (node, path node) pairs.
+// number of (node, path node) pairs; nxb x tiles (2: the next item's is prefetched).
 struct TLayout {
-    int cf, xs, cb, coef, pj, part, par, cnt, off, da, dtv, wt, total;
+    int cf, s0, xs, xbytes, cb, coef, pj, abuf, par, cnt, off, da, dtv, wt, total;
     __host__ __device__ static int up16(int v) { return (v + 15) & ~15; }
-    __host__ __device__ TLayout(int T, int N, int ch, int es_x)
+    __host__ __device__ TLayout(int T, int N, int np, int es_x, int es_s, int nxb)
     {
         const int E = T * (T + 1) / 2;
         cf = 0;
-        xs = cf + up16(T * (N + 4) * 4);
-        cb = xs + up16(T * kTile * es_x);
+        s0 = cf + up16(T * (N + 4) * 4);
+        xs = s0 + up16(kTile * N * es_s);
+        xbytes = up16(T * kTile * es_x);
+        cb = xs + nxb * xbytes;
         coef = cb + up16(E * 4);
         pj = coef + up16(E * 4);
-        part = pj + up16(E * 2);
-        par = part + ch * kChunk * kTile * 4;
+        abuf = pj + up16(E);
+        par = abuf + (np > 1 ? T * kTile * 4 : 0);    // partial a_i between dstate passes
         cnt = par + up16(T * 4);
         off = cnt + up16(T * 4);
         da = off + up16(T * 4);
@@ -72,6 +82,52 @@ struct TLayout {
         total = wt + up16(T * 4);
     }
 };
+
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)),
+                 "l"(src)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Byte offset of 16-byte chunk c of state row r in the staging buffer (cpr chunks per
+// row): chunks are XOR-swizzled by the row so that lanes reading the same chunk of
+// consecutive rows hit different banks.
+__device__ __forceinline__ int s0_off(int r, int c, int cpr)
+{
+    const int m = (cpr < 8 ? cpr : 8) - 1;
+    return (r * cpr + (c ^ (r & m))) * 16;
+}
+
+// One work item: row b, head h (group g), dim rows row0 .. row0 + rows, pool slot.
+struct Item {
+    int b, h, g, dtile, row0, rows, slot;
+    __device__ __forceinline__ bool valid(int P) const { return slot >= 0 && slot < P; }
+};
+
+__device__ __forceinline__ Item item_at(const TreeArgs &ta, int64_t it, int dtiles)
+{
+    const DecodeArgs &a = ta.d;
+    Item u;
+    u.dtile = (int)(it % dtiles);
+    u.h = (int)((it / dtiles) % a.H);
+    u.b = (int)(it / ((int64_t)dtiles * a.H));
+    u.g = u.h / (a.H / a.G);
+    u.row0 = u.dtile * kTile;
+    u.rows = min(kTile, a.Dm - u.row0);
+    u.slot = a.idx ? a.idx[u.b] : u.b;
+    return u;
+}
 
 // C_i . B_j over dstate: C_i from shared memory (fp32), B_j from global memory (16-byte
 // rows of the input type).
@@ -94,7 +150,7 @@ __device__ __forceinline__ float dot_cb(const float *ci, const void *B, int dtyp
     } else {
         const uint4 *bp =
             reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(B) + base);
-#pragma unroll 2
+#pragma unroll 4
         for (int q = 0; q < N / 8; ++q) {
             const uint4 raw = __ldg(bp + q);
             float f[8];
@@ -117,7 +173,7 @@ __device__ __forceinline__ float dot_cb(const float *ci, const void *B, int dtyp
     return s0 + s1;
 }
 
-// Element e of the x tile held in shared memory in its input type.
+// Element e of an x tile held in shared memory in its input type.
 __device__ __forceinline__ float xs_at(const uint8_t *xs, int x_dtype, int e)
 {
     if (x_dtype == SSU_F32)
@@ -125,7 +181,7 @@ __device__ __forceinline__ float xs_at(const uint8_t *xs, int x_dtype, int e)
     return bits_f32(reinterpret_cast<const uint16_t *>(xs)[e], x_dtype);
 }
 
-// Shared state of one (row, group): parents, path checks, C, path nodes and C . B.
+// Shared tables of one (row, group): parents, path checks, C, path nodes and C . B.
 template <int N>
 __device__ void stage_row(const TreeArgs &ta, const TLayout &lay, uint8_t *sm, int b, int g,
                           bool reporter)
@@ -135,16 +191,28 @@ __device__ void stage_row(const TreeArgs &ta, const TLayout &lay, uint8_t *sm, i
     const int T = ta.T, G = a.G, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float *Cf = reinterpret_cast<float *>(sm + lay.cf);
     float *cb = reinterpret_cast<float *>(sm + lay.cb);
-    uint16_t *pj = reinterpret_cast<uint16_t *>(sm + lay.pj);
+    uint8_t *pj = sm + lay.pj;
     int *par = reinterpret_cast<int *>(sm + lay.par);
     int *cnt = reinterpret_cast<int *>(sm + lay.cnt);
     int *off = reinterpret_cast<int *>(sm + lay.off);
 
     for (int i = tid; i < T; i += kThreads)
         par[i] = ta.parents[(int64_t)b * T + i];
-    for (int e = tid; e < T * N; e += kThreads) {
-        const int i = e / N, n = e % N;
-        Cf[i * Gm::CP + n] = ld_f32(a.C, a.bc_dtype, (((int64_t)b * T + i) * G + g) * N + n);
+    const int64_t cbase = (int64_t)b * T * G * N;
+    for (int e0 = tid; e0 < T * N; e0 += kThreads * kBatch) {
+        float v[kBatch];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {       // every load first, then the stores
+            const int e = e0 + q * kThreads;
+            v[q] = e < T * N ? ld_f32(a.C, a.bc_dtype, cbase + ((int64_t)(e / N) * G + g) * N + e % N)
+                             : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int e = e0 + q * kThreads;
+            if (e < T * N)
+                Cf[(e / N) * Gm::CP + e % N] = v[q];
+        }
     }
     __syncthreads();
     // every node's walk: exactly depth parent steps inside [0, T), then parent -1
@@ -186,7 +254,7 @@ __device__ void stage_row(const TreeArgs &ta, const TLayout &lay, uint8_t *sm, i
         int j = i;
         for (int k = 0; k < c; ++k) {
             if ((k & 1) == p) {
-                pj[o + k] = static_cast<uint16_t>(j);
+                pj[o + k] = static_cast<uint8_t>(j);
                 cb[o + k] = dot_cb<N>(Cf + i * Gm::CP, a.B, a.bc_dtype,
                                       (((int64_t)b * T + j) * G + g) * N);
             }
@@ -195,56 +263,86 @@ __device__ void stage_row(const TreeArgs &ta, const TLayout &lay, uint8_t *sm, i
     }
 }
 
-// Per-item values: dt_eff and dA of every node for head h (and their stash entries), the
-// x tile (and the U stash), the B stash once per (row, group).
-__device__ void stage_item(const TreeArgs &ta, const TLayout &lay, uint8_t *sm, int b, int h,
-                           int g, int row0, int rows, int dtile)
+// x tile of item u with plain loads (x rows not 16-byte aligned): rows >= u.rows are 0.
+__device__ void stage_x_plain(const TreeArgs &ta, uint8_t *xs, const Item &u)
 {
     const DecodeArgs &a = ta.d;
-    const int T = ta.T, H = a.H, G = a.G, Dm = a.Dm, N = a.N, tid = threadIdx.x;
-    const int es_x = a.x_dtype == SSU_F32 ? 4 : 2;
-    uint8_t *Xs = sm + lay.xs;
-    float *sdA = reinterpret_cast<float *>(sm + lay.da);
-    float *sdt = reinterpret_cast<float *>(sm + lay.dtv);
-    const float Ah = a.A[h];
-    for (int i = tid; i < T; i += kThreads) {
-        const int64_t bi = (int64_t)b * T + i;
-        const float dte = effective_dt(a.dt[bi * H + h], a.dt_bias, h, a.softplus);
-        const float dA = expf(Ah * dte);
-        sdA[i] = dA;
-        sdt[i] = dte;
-        if (dtile == 0) {
-            ta.st_dA[bi * H + h] = dA;
-            ta.st_dt[bi * H + h] = dte;
+    const int T = ta.T, H = a.H, Dm = a.Dm, tid = threadIdx.x;
+    for (int e0 = tid; e0 < T * kTile; e0 += kThreads * kBatch) {
+        uint32_t v[kBatch];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int e = e0 + q * kThreads, i = e / kTile, d = e % kTile;
+            v[q] = e < T * kTile && d < u.rows
+                       ? ld_bits(a.x, a.x_dtype, (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d)
+                       : 0u;
         }
-    }
-    for (int e = tid; e < T * kTile; e += kThreads) {
-        const int i = e / kTile, d = e % kTile;
-        uint32_t v = 0;
-        if (d < rows) {
-            const int64_t xi = (((int64_t)b * T + i) * H + h) * Dm + row0 + d;
-            v = ld_bits(a.x, a.x_dtype, xi);
-            ta.st_U[xi] = bits_f32(v, a.x_dtype);
-        }
-        if (es_x == 4)
-            reinterpret_cast<uint32_t *>(Xs)[e] = v;
-        else
-            reinterpret_cast<uint16_t *>(Xs)[e] = static_cast<uint16_t>(v);
-    }
-    if (dtile == 0 && h % (H / G) == 0) {
-        for (int e = tid; e < T * N; e += kThreads) {
-            const int64_t bi = ((int64_t)b * T + e / N) * G + g;
-            ta.st_B[bi * N + e % N] = ld_f32(a.B, a.bc_dtype, bi * N + e % N);
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int e = e0 + q * kThreads;
+            if (e < T * kTile) {
+                if (a.x_dtype == SSU_F32)
+                    reinterpret_cast<uint32_t *>(xs)[e] = v[q];
+                else
+                    reinterpret_cast<uint16_t *>(xs)[e] = static_cast<uint16_t>(v[q]);
+            }
         }
     }
 }
 
-// Path coefficients of head h: coef[o_i + m] = w_im * dt_jm * cb[o_i + m], W_i.
+// Per-item node values and stash: dt_eff and dA of every node for head h (from the
+// prefetched dt of node threadIdx.x), U from the x tile, B once per (row, group).
+__device__ void stage_nodes(const TreeArgs &ta, const TLayout &lay, uint8_t *sm, const Item &u,
+                            const uint8_t *xs, float dt_mine)
+{
+    const DecodeArgs &a = ta.d;
+    const int T = ta.T, H = a.H, G = a.G, Dm = a.Dm, N = a.N, tid = threadIdx.x;
+    float *sdA = reinterpret_cast<float *>(sm + lay.da);
+    float *sdt = reinterpret_cast<float *>(sm + lay.dtv);
+    if (tid < T) {
+        const int64_t bi = (int64_t)u.b * T + tid;
+        const float dte = effective_dt(dt_mine, a.dt_bias, u.h, a.softplus);
+        const float dA = expf(a.A[u.h] * dte);
+        sdA[tid] = dA;
+        sdt[tid] = dte;
+        if (u.dtile == 0) {
+            ta.st_dA[bi * H + u.h] = dA;
+            ta.st_dt[bi * H + u.h] = dte;
+        }
+    }
+    for (int e = tid; e < T * kTile; e += kThreads) {
+        const int i = e / kTile, d = e % kTile;
+        if (d < u.rows)
+            ta.st_U[(((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d] =
+                xs_at(xs, a.x_dtype, e);
+    }
+    if (u.dtile == 0 && u.h % (H / G) == 0) {
+        const int64_t rows = (int64_t)T * N;
+        for (int64_t e0 = tid; e0 < rows; e0 += kThreads * kBatch) {
+            float v[kBatch];
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int64_t e = e0 + q * kThreads;
+                v[q] = e < rows ? ld_f32(a.B, a.bc_dtype,
+                                         (((int64_t)u.b * T + e / N) * G + u.g) * N + e % N)
+                                : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int64_t e = e0 + q * kThreads;
+                if (e < rows)
+                    ta.st_B[(((int64_t)u.b * T + e / N) * G + u.g) * N + e % N] = v[q];
+            }
+        }
+    }
+}
+
+// Path coefficients of the item's head: coef[o_i + m] = w_im * dt_jm * cb[o_i + m], W_i.
 __device__ void path_coefs(const TLayout &lay, uint8_t *sm, int T)
 {
     const float *cb = reinterpret_cast<const float *>(sm + lay.cb);
     float *coef = reinterpret_cast<float *>(sm + lay.coef);
-    const uint16_t *pj = reinterpret_cast<const uint16_t *>(sm + lay.pj);
+    const uint8_t *pj = sm + lay.pj;
     const int *cnt = reinterpret_cast<const int *>(sm + lay.cnt);
     const int *off = reinterpret_cast<const int *>(sm + lay.off);
     const float *sdA = reinterpret_cast<const float *>(sm + lay.da);
@@ -262,140 +360,252 @@ __device__ void path_coefs(const TLayout &lay, uint8_t *sm, int T)
     }
 }
 
+// Four consecutive committed-state elements of row r (columns col .. col + 3) from the
+// swizzled staging buffer.
+template <typename S, int N>
+__device__ __forceinline__ float4 s0_quad(const uint8_t *buf, int r, int col)
+{
+    constexpr int cpr = N * (int)sizeof(S) / 16;
+    if constexpr (sizeof(S) == 4) {
+        return *reinterpret_cast<const float4 *>(buf + s0_off(r, col / 4, cpr));
+    } else {
+        const int c = col / 8, half = (col / 4) & 1;
+        return Quad<S>::load(reinterpret_cast<const S *>(buf + s0_off(r, c, cpr) + half * 8));
+    }
+}
+
+// Issue the cp.async copies of item u's committed-state rows into the staging buffer.
+template <typename S, int N>
+__device__ __forceinline__ void prefetch_s0(const TreeArgs &ta, const TLayout &lay, uint8_t *sm,
+                                            const Item &u)
+{
+    const DecodeArgs &a = ta.d;
+    constexpr int cpr = N * (int)sizeof(S) / 16;
+    const char *src = static_cast<const char *>(a.state) +
+                      ((int64_t)u.slot * a.slot_stride + ((int64_t)u.h * a.Dm + u.row0) * N) *
+                          (int64_t)sizeof(S);
+    for (int k = threadIdx.x; k < u.rows * cpr; k += kThreads)
+        cp_async16(sm + lay.s0 + s0_off(k / cpr, k % cpr, cpr), src + (int64_t)k * 16);
+}
+
+// Issue the cp.async copies of item u's x tile (rows 16-byte aligned) into buffer xbuf.
+__device__ __forceinline__ void prefetch_x(const TreeArgs &ta, const TLayout &lay, uint8_t *sm,
+                                           const Item &u, int xbuf)
+{
+    const DecodeArgs &a = ta.d;
+    const int T = ta.T, es_x = a.x_dtype == SSU_F32 ? 4 : 2;
+    const int cpn = u.rows * es_x / 16;              // 16-byte chunks per node row
+    uint8_t *dst = sm + lay.xs + xbuf * lay.xbytes;
+    const char *xg = static_cast<const char *>(a.x);
+    for (int k = threadIdx.x; k < T * cpn; k += kThreads) {
+        const int i = k / cpn, c = k % cpn;
+        cp_async16(dst + i * kTile * es_x + c * 16,
+                   xg + ((((int64_t)u.b * T + i) * a.H + u.h) * a.Dm + u.row0) * es_x + c * 16);
+    }
+}
+
+// dt of node threadIdx.x for item u (consumed when u is processed).
+__device__ __forceinline__ float dt_of(const TreeArgs &ta, const Item &u)
+{
+    const int T = ta.T;
+    return threadIdx.x < T ? ta.d.dt[((int64_t)u.b * T + threadIdx.x) * ta.d.H + u.h] : 0.f;
+}
+
+// Sum over node i's path of coef * x_j[d] for the lane's dim row d (four entries per step).
+__device__ __forceinline__ float path_sum(const float *coef, const uint8_t *pj,
+                                          const uint8_t *xs, int x_dtype, int o, int cn, int d)
+{
+    float p4[4] = {0.f, 0.f, 0.f, 0.f};
+    int k = 0;
+    for (; k + 4 <= cn; k += 4) {
+        float cf[4];
+        int j[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            cf[m] = coef[o + k + m];
+            j[m] = pj[o + k + m];
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            p4[m] = fmaf(cf[m], xs_at(xs, x_dtype, j[m] * kTile + d), p4[m]);
+    }
+    for (; k < cn; ++k)
+        p4[0] = fmaf(coef[o + k], xs_at(xs, x_dtype, pj[o + k] * kTile + d), p4[0]);
+    return (p4[0] + p4[1]) + (p4[2] + p4[3]);
+}
+
 template <typename S, int N>
 __global__ void __launch_bounds__(kThreads, 1)
-ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const int64_t nitems)
+ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const int64_t nitems,
+                  const int nxb, const int xasync)
 {
     using Gm = TGeo<N>;
     extern __shared__ __align__(16) uint8_t sm[];
     const DecodeArgs &a = ta.d;
-    const int T = ta.T, H = a.H, Dm = a.Dm, hpg = H / a.G;
+    const int T = ta.T, H = a.H, Dm = a.Dm;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int ch = warp % Gm::CH, ng = warp / Gm::CH;
+    const int ng = warp / kRowWarps;
+    const int d = (warp % kRowWarps) * 32 + lane;    // the lane's dim row within the tile
     const int es_x = a.x_dtype == SSU_F32 ? 4 : 2;
-    const TLayout lay(T, N, Gm::CH, es_x);
+    const TLayout lay(T, N, Gm::NP, es_x, (int)sizeof(S), nxb);
     const float *Cf = reinterpret_cast<const float *>(sm + lay.cf);
-    const uint8_t *Xs = sm + lay.xs;
     const float *coef = reinterpret_cast<const float *>(sm + lay.coef);
-    const uint16_t *pj = reinterpret_cast<const uint16_t *>(sm + lay.pj);
-    float *part = reinterpret_cast<float *>(sm + lay.part);
+    const uint8_t *pj = sm + lay.pj;
+    float *abuf = reinterpret_cast<float *>(sm + lay.abuf);
     const int *cnt = reinterpret_cast<const int *>(sm + lay.cnt);
     const int *off = reinterpret_cast<const int *>(sm + lay.off);
     const float *wt = reinterpret_cast<const float *>(sm + lay.wt);
 
+    // Copies for the next item start as early as their buffers allow: the state rows once
+    // every lane holds them in registers (after the last dstate pass when there are
+    // several), the x tile at once when it is double-buffered, else after the item.
+    const bool s0_mid = Gm::NP == 1, x_mid = xasync && nxb == 2;
     const int64_t first = nitems * blockIdx.x / gridDim.x;
     const int64_t last = nitems * (blockIdx.x + 1) / gridDim.x;
-    int cur_b = -1, cur_g = -1;
-    for (int64_t it = first; it < last; ++it) {
-        const int dtile = (int)(it % dtiles);
-        const int h = (int)((it / dtiles) % H);
-        const int b = (int)(it / ((int64_t)dtiles * H));
-        const int g = h / hpg;
-        const int row0 = dtile * kTile;
-        const int rows = min(kTile, Dm - row0);
-        const bool reporter = h == 0 && dtile == 0;
-        const int slot = a.idx ? a.idx[b] : b;
-        if (slot < 0) {                  // padding row: zero outputs at every node
-            for (int e = tid; e < T * rows; e += kThreads) {
-                const int i = e / rows, d = e % rows;
-                st_f32(a.out, a.x_dtype, (((int64_t)b * T + i) * H + h) * Dm + row0 + d, 0.f);
-            }
-            continue;
-        }
-        if (slot >= a.P) {
-            if (reporter && tid == 0 && a.err)
-                atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
-            continue;
-        }
-        __syncthreads();                 // shared memory of the previous item is free
-        if (b != cur_b || g != cur_g) {
-            stage_row<N>(ta, lay, sm, b, g, reporter);
-            cur_b = b;
-            cur_g = g;
-        }
-        stage_item(ta, lay, sm, b, h, g, row0, rows, dtile);
-
-        // the lane's two dim rows of the committed state, one column group
-        const S *base = static_cast<const S *>(a.state) + (int64_t)slot * a.slot_stride +
-                        (int64_t)h * Dm * N + ch * Gm::K;
-        float2 s[2][Gm::K / 2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int d = lane + 32 * r;
-#pragma unroll
-            for (int q = 0; q < Gm::K / 4; ++q) {
-                const float4 v = d < rows ? Quad<S>::load(base + (int64_t)(row0 + d) * N + 4 * q)
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-                s[r][2 * q] = make_float2(v.x, v.y);
-                s[r][2 * q + 1] = make_float2(v.z, v.w);
-            }
-        }
-        __syncthreads();                 // sdA, sdt, x tile (and the row's tables) ready
-        path_coefs(lay, sm, T);
-        const float Dh = a.D ? a.D[h] : 0.f;
-
-        const int nchunks = (T + kChunk - 1) / kChunk;
-        for (int c = 0; c < nchunks; ++c) {
-            // ---- a_i over this warp's column group for its NPG nodes of the chunk
-            const int n0 = c * kChunk + ng * Gm::NPG;
-            const float *crow[Gm::NPG];
-#pragma unroll
-            for (int nd = 0; nd < Gm::NPG; ++nd)
-                crow[nd] = Cf + (n0 + nd < T ? n0 + nd : 0) * Gm::CP + ch * Gm::K;
-            float2 acc[Gm::NPG][2];
-#pragma unroll
-            for (int nd = 0; nd < Gm::NPG; ++nd)
-                acc[nd][0] = acc[nd][1] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int q = 0; q < Gm::K / 4; ++q) {
-#pragma unroll
-                for (int nd = 0; nd < Gm::NPG; ++nd) {
-                    const float4 cv = *reinterpret_cast<const float4 *>(crow[nd] + 4 * q);
-                    const float2 lo = make_float2(cv.x, cv.y), hi = make_float2(cv.z, cv.w);
-#pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        acc[nd][r] = __ffma2_rn(s[r][2 * q], lo, acc[nd][r]);
-                        acc[nd][r] = __ffma2_rn(s[r][2 * q + 1], hi, acc[nd][r]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int nd = 0; nd < Gm::NPG; ++nd)
-#pragma unroll
-                for (int r = 0; r < 2; ++r)
-                    part[(ch * kChunk + ng * Gm::NPG + nd) * kTile + lane + 32 * r] =
-                        acc[nd][r].x + acc[nd][r].y;
-            __syncthreads();                 // partial sums (and path coefficients) ready
-
-            // ---- epilogue: out_i = W_i a_i + sum over the path + D x_i
-            for (int e = tid; e < kChunk * kTile; e += kThreads) {
-                const int n = e / kTile, d = e % kTile, i = c * kChunk + n;
-                if (i >= T || d >= rows)
-                    continue;
-                float av = 0.f;
-#pragma unroll
-                for (int q = 0; q < Gm::CH; ++q)
-                    av += part[(q * kChunk + n) * kTile + d];
-                float y = 0.f;
-                const int cn = cnt[i];
-                if (cn > 0) {
-                    const int o = off[i];
-                    float p0 = 0.f, p1 = 0.f;
-                    int k = 0;
-                    for (; k + 1 < cn; k += 2) {
-                        p0 = fmaf(coef[o + k], xs_at(Xs, a.x_dtype, pj[o + k] * kTile + d), p0);
-                        p1 = fmaf(coef[o + k + 1],
-                                  xs_at(Xs, a.x_dtype, pj[o + k + 1] * kTile + d), p1);
-                    }
-                    if (k < cn)
-                        p0 = fmaf(coef[o + k], xs_at(Xs, a.x_dtype, pj[o + k] * kTile + d), p0);
-                    y = fmaf(wt[i], av, p0 + p1) + Dh * xs_at(Xs, a.x_dtype, i * kTile + d);
-                }
-                st_f32(a.out, a.x_dtype, (((int64_t)b * T + i) * H + h) * Dm + row0 + d, y);
-            }
-            __syncthreads();                 // part is free for the next chunk
+    auto xbuf_of = [&](int64_t it) { return nxb == 2 ? (int)((it - first) & 1) : 0; };
+    float dt_next = 0.f;                 // dt of node tid for the next valid item
+    if (first < last) {
+        const Item u = item_at(ta, first, dtiles);
+        if (u.valid(a.P)) {
+            prefetch_s0<S, N>(ta, lay, sm, u);
+            if (xasync)
+                prefetch_x(ta, lay, sm, u, xbuf_of(first));
+            cp_async_commit();
+            dt_next = dt_of(ta, u);
         }
     }
+    int cur_b = -1, cur_g = -1;
+    for (int64_t it = first; it < last; ++it) {
+        const Item u = item_at(ta, it, dtiles);
+        const bool has_next = it + 1 < last;
+        const Item v = has_next ? item_at(ta, it + 1, dtiles) : u;
+        const bool next_valid = has_next && v.valid(a.P);
+        if (!u.valid(a.P)) {
+            if (u.slot < 0) {            // padding row: zero outputs at every node
+                for (int e = tid; e < T * kTile; e += kThreads) {
+                    const int i = e / kTile, dd = e % kTile;
+                    if (dd < u.rows)
+                        st_f32(a.out, a.x_dtype,
+                               (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + dd, 0.f);
+                }
+            } else if (u.h == 0 && u.dtile == 0 && tid == 0 && a.err) {
+                atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
+            }
+            if (next_valid) {            // this item used no buffer: start the next one
+                prefetch_s0<S, N>(ta, lay, sm, v);
+                if (xasync)
+                    prefetch_x(ta, lay, sm, v, xbuf_of(it + 1));
+                cp_async_commit();
+                dt_next = dt_of(ta, v);
+            }
+            continue;
+        }
+        uint8_t *xs = sm + lay.xs + xbuf_of(it) * lay.xbytes;
+        __syncthreads();                 // the previous item is done with shared memory
+        if (u.b != cur_b || u.g != cur_g) {
+            stage_row<N>(ta, lay, sm, u.b, u.g, u.h == 0 && u.dtile == 0);
+            cur_b = u.b;
+            cur_g = u.g;
+        }
+        if (!xasync)
+            stage_x_plain(ta, xs, u);
+        cp_async_wait_all();
+        __syncthreads();                 // state rows and x tile have landed
+        stage_nodes(ta, lay, sm, u, xs, dt_next);
+        __syncthreads();                 // dt_eff and dA of every node visible
+        path_coefs(lay, sm, T);
+
+        // the lane's dim row of the committed state, first dstate pass
+        float2 s[Gm::KP / 2];
+        auto load_pass = [&](int p) {
+#pragma unroll
+            for (int q = 0; q < Gm::KP / 4; ++q) {
+                const float4 f = d < u.rows ? s0_quad<S, N>(sm + lay.s0, d, p * Gm::KP + 4 * q)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                s[2 * q] = make_float2(f.x, f.y);
+                s[2 * q + 1] = make_float2(f.z, f.w);
+            }
+        };
+        load_pass(0);
+        __syncthreads();                 // path coefficients ready; staging buffer free
+        if (next_valid && (s0_mid || x_mid)) {
+            if (s0_mid)
+                prefetch_s0<S, N>(ta, lay, sm, v);
+            if (x_mid)
+                prefetch_x(ta, lay, sm, v, xbuf_of(it + 1));
+            cp_async_commit();
+        }
+        if (next_valid)
+            dt_next = dt_of(ta, v);
+        const float Dh = a.D ? a.D[u.h] : 0.f;
+
+        // y_i = W_i a_i + path sum + D x_i for this warp's nodes (every fourth, two at a
+        // time) and the lane's row; four partial-sum chains per node
+#pragma unroll 1
+        for (int p = 0; p < Gm::NP; ++p) {
+            if (p > 0)
+                load_pass(p);
+#pragma unroll 1
+            for (int i0 = ng; i0 < T; i0 += 2 * kNodeGroups) {
+                const int i1 = i0 + kNodeGroups;
+                const bool two = i1 < T;
+                const float *c0 = Cf + i0 * Gm::CP + p * Gm::KP;
+                const float *c1 = Cf + (two ? i1 : i0) * Gm::CP + p * Gm::KP;
+                float2 a0[4], a1[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    a0[m] = a1[m] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int q = 0; q < Gm::KP / 4; ++q) {
+                    const float4 u0 = *reinterpret_cast<const float4 *>(c0 + 4 * q);
+                    const float4 u1 = *reinterpret_cast<const float4 *>(c1 + 4 * q);
+                    const int m = 2 * (q & 1);
+                    a0[m] = __ffma2_rn(s[2 * q], make_float2(u0.x, u0.y), a0[m]);
+                    a1[m] = __ffma2_rn(s[2 * q], make_float2(u1.x, u1.y), a1[m]);
+                    a0[m + 1] = __ffma2_rn(s[2 * q + 1], make_float2(u0.z, u0.w), a0[m + 1]);
+                    a1[m + 1] = __ffma2_rn(s[2 * q + 1], make_float2(u1.z, u1.w), a1[m + 1]);
+                }
+                float r[2];
+                r[0] = ((a0[0].x + a0[0].y) + (a0[1].x + a0[1].y)) +
+                       ((a0[2].x + a0[2].y) + (a0[3].x + a0[3].y));
+                r[1] = ((a1[0].x + a1[0].y) + (a1[1].x + a1[1].y)) +
+                       ((a1[2].x + a1[2].y) + (a1[3].x + a1[3].y));
+#pragma unroll
+                for (int n = 0; n < 2; ++n) {
+                    const int i = n == 0 ? i0 : i1;
+                    if (n == 1 && !two)
+                        break;
+                    float av = r[n];
+                    if (Gm::NP > 1) {            // partial a_i between dstate passes
+                        if (p > 0)
+                            av += abuf[i * kTile + d];
+                        if (p + 1 < Gm::NP) {
+                            abuf[i * kTile + d] = av;
+                            continue;
+                        }
+                    }
+                    if (d >= u.rows)
+                        continue;
+                    const int cn = cnt[i];
+                    float y = 0.f;
+                    if (cn > 0)
+                        y = fmaf(wt[i], av, path_sum(coef, pj, xs, a.x_dtype, off[i], cn, d)) +
+                            Dh * xs_at(xs, a.x_dtype, i * kTile + d);
+                    st_f32(a.out, a.x_dtype, (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d,
+                           y);
+                }
+            }
+        }
+        __syncthreads();                 // every read of this item's buffers is done
+        if (next_valid && (!s0_mid || (xasync && !x_mid))) {
+            if (!s0_mid)
+                prefetch_s0<S, N>(ta, lay, sm, v);
+            if (xasync && !x_mid)
+                prefetch_x(ta, lay, sm, v, xbuf_of(it + 1));
+            cp_async_commit();
+        }
+    }
+    cp_async_wait_all();                 // no copy outlives the CTA
 }
 
 template <typename S, int N>
@@ -407,27 +617,34 @@ int launch_n(const TreeArgs &a, cudaStream_t stream)
     if (nitems == 0 || a.T == 0)
         return SSU_OK;
     const int es_x = a.d.x_dtype == SSU_F32 ? 4 : 2;
-    const TLayout lay(a.T, N, Gm::CH, es_x);
-    if (lay.total > 227 * 1024)
+    int nxb = 2;
+    TLayout lay(a.T, N, Gm::NP, es_x, (int)sizeof(S), nxb);
+    if (lay.total > kSmemMax) {
+        nxb = 1;
+        lay = TLayout(a.T, N, Gm::NP, es_x, (int)sizeof(S), nxb);
+    }
+    if (lay.total > kSmemMax)
         return SSU_ERR_UNSUPPORTED;
+    // x rows go through cp.async when every 16-byte chunk of a tile row is aligned
+    const int xasync = (reinterpret_cast<uintptr_t>(a.d.x) & 15) == 0 &&
+                       ((int64_t)a.d.Dm * es_x) % 16 == 0;
     static int configured[64], sms[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         dev = 0;
-    if (configured[dev] < lay.total) {
+    if (!configured[dev]) {
         if (cudaFuncSetAttribute(ssu_ddtree_kernel<S, N>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 227 * 1024) != cudaSuccess)
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) !=
+            cudaSuccess)
             return SSU_ERR_CUDA;
-        configured[dev] = 227 * 1024;
-    }
-    if (sms[dev] == 0) {
         int n = 0;
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
         sms[dev] = n > 0 ? n : 148;
+        configured[dev] = 1;
     }
     const int64_t grid = nitems < sms[dev] ? nitems : sms[dev];
-    ssu_ddtree_kernel<S, N><<<(unsigned)grid, kThreads, lay.total, stream>>>(a, dtiles, nitems);
+    ssu_ddtree_kernel<S, N><<<(unsigned)grid, kThreads, lay.total, stream>>>(a, dtiles, nitems,
+                                                                            nxb, xasync);
     return SSU_OK;
 }
 
