@@ -12,7 +12,8 @@ Value laws (one set for every workload):
   The "slow decay" variant draws A = -exp(U(-2, 0)) and sets dt_bias = -4, so that the
   state remembers many tokens.
 Every tensor is drawn in fp32 from one ``torch.Generator`` in a fixed order
-(pool, x, B, C, dt, z, A, dt_bias, D, stateIndices, padding positions, lengths, tree)
+(pool, x, B, C, dt, z, A, dt_bias, D, stateIndices, padding positions, lengths, tree,
+conv inputs)
 and then cast to its storage dtype, so both sides see the same (already rounded) values.
 
 Draft trees (tree verify): node 0 is a root; every later node i picks its parent
@@ -45,6 +46,9 @@ class SSUCase:
       context_lengths / accepted_lengths [batch] int32 (None = all T tokens)
       tree verify: parent_ids, depths [batch, T] int32 (T = tree nodes);
       accepted_node_ids [batch, T] int32 (an accepted root-to-node path, -1 beyond it)
+      fused conv1d decode: xbc [batch, conv_dim] raw channels (x, B, C order; conv_dim =
+      H*Dm + 2*G*N), conv_w [conv_dim, width], conv_b [conv_dim], conv_state flat pool
+      with element (s, c, k) at the conv_strides (slot, channel, tap) offsets
     """
 
     name: str
@@ -73,6 +77,13 @@ class SSUCase:
     parent_ids: Optional[torch.Tensor] = None
     depths: Optional[torch.Tensor] = None
     accepted_node_ids: Optional[torch.Tensor] = None
+    xbc: Optional[torch.Tensor] = None
+    conv_w: Optional[torch.Tensor] = None
+    conv_b: Optional[torch.Tensor] = None
+    conv_state: Optional[torch.Tensor] = None
+    conv_strides: Optional[tuple] = None
+    width: int = 0
+    conv_silu: bool = True
 
     @property
     def x_dtype(self):
@@ -120,6 +131,9 @@ def make_case(
     slot_pad: int = 0,
     slow_decay: bool = False,
     tree: Optional[str] = None,
+    conv: int = 0,
+    conv_layout: str = "ds",
+    conv_pad: int = 0,
 ) -> SSUCase:
     """Draw one workload.
 
@@ -131,6 +145,9 @@ def make_case(
     slot_pad: extra elements per pool slot beyond H*Dm*N (a padded slot stride).
     tree: None, "random", "chain", "forest" or "shuffled" (draft trees of T nodes, with
       an accepted path and acceptedLengths along it).
+    conv: conv1d width (0: no conv inputs); conv_layout "ds" (channel-major windows,
+      [P, conv_dim, width-1]) or "sd" (tap-major, [P, width-1, conv_dim]); conv_pad: extra
+      elements per conv slot.
     """
     if P is None:
         P = batch
@@ -189,12 +206,26 @@ def make_case(
         par, dep = draw_trees(g, batch, T, tree)
         nodes, acc = draw_accepted_paths(g, par, dep)
 
+    xbc = cw = cb = cst = strides = None
+    if conv:
+        cd = H * Dm + 2 * G * N
+        taps = conv - 1
+        cslot = cd * taps + conv_pad
+        xbc = randn(batch, cd).to(x_dtype)
+        cw = (randn(cd, conv) * 0.5).to(x_dtype)
+        cb = (randn(cd) * 0.1).to(x_dtype)
+        cst = randn(max(P * cslot, 1)).to(x_dtype)
+        strides = (cslot, taps, 1) if conv_layout == "ds" else (cslot, 1, cd)
+        if conv_layout not in ("ds", "sd"):
+            raise ValueError(f"unknown conv layout {conv_layout!r}")
+
     return SSUCase(
         name=name, batch=batch, P=P, H=H, G=G, Dm=Dm, N=N, T=T, active=active,
         slot_stride=stride, x=x, B=B, C=C, dt=dt, A=A, pool=pool, z=zt,
         dt_bias=bias, D=Dv, state_indices=si, context_lengths=ctx,
         accepted_lengths=acc, dt_softplus=dt_softplus, parent_ids=par, depths=dep,
-        accepted_node_ids=nodes,
+        accepted_node_ids=nodes, xbc=xbc, conv_w=cw, conv_b=cb, conv_state=cst,
+        conv_strides=strides, width=conv,
     )
 
 
@@ -254,7 +285,7 @@ def draw_accepted_paths(g: torch.Generator, par: torch.Tensor, dep: torch.Tensor
     return nodes, acc
 
 
-# The named workloads. Seeds: 0 for the tiny decode, then 1..5 in order.
+# The named workloads. Seeds: 0 for the tiny decode, then 1..6 in order.
 CONFIGS = {
     # batch 2, pool of 4 slots, H 4, Dm 16, N 16, fp32 everything, stateIndices [2, 0]
     "tiny_decode": dict(seed=0, batch=2, P=4, H=4, G=1, Dm=16, N=16,
@@ -275,6 +306,10 @@ CONFIGS = {
     "spec_replay_b64_t5": dict(seed=4, batch=64, P=128, T=5, H=80, G=1, Dm=64, N=128,
                                x_dtype=BF16, bc_dtype=BF16, state_dtype=F32, z=True,
                                lengths="accepted"),
+    # the batch-256 decode with the causal conv1d (width 4) of its xBC channels fused in
+    "mamba2_conv_decode_b256": dict(seed=6, batch=256, P=512, H=80, G=1, Dm=64, N=128,
+                                    x_dtype=BF16, bc_dtype=BF16, state_dtype=F32, z=True,
+                                    conv=4),
     # tree verify of one 128-node draft tree per row (the verify budget), no gate
     "ddtree_b16_n128": dict(seed=5, batch=16, P=32, T=128, H=80, G=1, Dm=64, N=128,
                             x_dtype=BF16, bc_dtype=BF16, state_dtype=F32, z=False,

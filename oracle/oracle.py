@@ -54,6 +54,9 @@ def lib():
                                      i32, i32, i32, i32, i32, i32, i32, i, vp]
         L.oracle_replay.argtypes = [vp, i, i64, i32, vp, vp, vp, vp, vp, vp,
                                     i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
+        L.oracle_conv_decode.argtypes = [vp, i, vp, vp, vp, i64, i64, i64, i32, i, vp, vp, vp,
+                                         vp, vp, vp, i, i64, i32, vp, vp, i32, i32, i32, i32,
+                                         i32, i32, i, vp]
         L.oracle_ddtree.argtypes = [vp, i, vp, vp, vp, i, vp, vp, vp, vp, i, i64, i32,
                                     vp, vp, vp, vp, vp, vp, vp, vp,
                                     i32, i32, i32, i32, i32, i32, i32, i, vp]
@@ -73,7 +76,8 @@ def lib():
         L.oracle_double_to_bf16.restype = ctypes.c_uint16
         for f in ("oracle_decode", "oracle_prefill", "oracle_replay",
                   "oracle_clear_slot", "oracle_copy_slot", "oracle_replay_layers",
-                  "oracle_clear_slot_layers", "oracle_gather_scatter", "oracle_ddtree"):
+                  "oracle_clear_slot_layers", "oracle_gather_scatter", "oracle_ddtree",
+                  "oracle_conv_decode"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -184,6 +188,28 @@ def ddtree(x, A, B, C, dt, pool, parent_ids, depths, *, dt_bias=None, D=None,
     return out, stash, err.value
 
 
+def conv_decode(xbc, conv_w, conv_b, conv_state, width, A, dt, pool, *, conv_strides,
+                dt_bias=None, D=None, z=None, state_indices=None, batch, active=None, H, G,
+                Dm, N, slot_stride=None, P=None, dt_softplus=True, conv_silu=True, out=None):
+    """Causal conv1d update of the raw xBC channels followed by one decode token; both
+    pools are updated in place. conv_strides = (slot, channel, tap) element strides of the
+    conv pool. Returns (out float64 [batch,H,Dm], err_flags)."""
+    active = batch if active is None else active
+    slot_stride = H * Dm * N if slot_stride is None else slot_stride
+    P = pool.numel() // slot_stride if P is None else P
+    if out is None:
+        out = torch.full((batch, H, Dm), float("nan"), dtype=torch.float64)
+    err = ctypes.c_int32(0)
+    cs, cc, ck = conv_strides
+    rc = lib().oracle_conv_decode(
+        _p(xbc), _CODES[xbc.dtype], _p(conv_w), _p(conv_b), _p(conv_state), cs, cc, ck, width,
+        int(conv_silu), _p(A), _p(dt), _p(dt_bias), _p(D), _p(z), _p(pool), _CODES[pool.dtype],
+        slot_stride, P, _p(out), _p(state_indices), batch, active, H, G, Dm, N,
+        int(dt_softplus), ctypes.byref(err))
+    _check(rc, "oracle_conv_decode")
+    return out, err.value
+
+
 def clear_slot(pool, slot_bytes, P, slot):
     _check(lib().oracle_clear_slot(_p(pool), slot_bytes, P, slot), "oracle_clear_slot")
 
@@ -278,3 +304,16 @@ def ddtree_case(case):
                   state_indices=case.state_indices, batch=case.batch, active=case.active,
                   T=case.T, H=case.H, G=case.G, Dm=case.Dm, N=case.N,
                   slot_stride=case.slot_stride, P=case.P, dt_softplus=case.dt_softplus)
+
+
+def conv_decode_case(case, pool=None, conv_state=None):
+    """Fused conv1d + decode on a conv case; returns (out, pool_after, conv_after, err)."""
+    pool = case.pool.clone() if pool is None else pool
+    conv = case.conv_state.clone() if conv_state is None else conv_state
+    out, err = conv_decode(case.xbc, case.conv_w, case.conv_b, conv, case.width, case.A,
+                           case.dt, pool, conv_strides=case.conv_strides, dt_bias=case.dt_bias,
+                           D=case.D, z=case.z, state_indices=case.state_indices,
+                           batch=case.batch, active=case.active, H=case.H, G=case.G,
+                           Dm=case.Dm, N=case.N, slot_stride=case.slot_stride, P=case.P,
+                           dt_softplus=case.dt_softplus, conv_silu=case.conv_silu)
+    return out, pool, conv, err

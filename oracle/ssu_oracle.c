@@ -536,6 +536,91 @@ int oracle_ddtree(const void *x, int x_dt, const float *A, const void *B, const 
     return 0;
 }
 
+/* ---------------- causal conv1d update fused with the decode ----------------
+ * The conv state of a slot holds the last width-1 raw inputs of every channel of the
+ * concatenated xBC input (conv_dim = H*Dm + 2*G*N channels, order x, B, C): Selective
+ * State Update page, struct MambaStateLayerInfo (convState beside recurrentState), and
+ * the causal conv1d update of the FlashInfer page flashinfer.gdn_fused_decode_step
+ * (conv_weight [dim, width], conv_bias [dim], conv_state [P, dim, width-1] of raw inputs,
+ * updated in place, both pools indexed by the same state index, padding rows skipped).
+ * Per channel c of an active row with slot s:
+ *     window  = (state[s,c,0], ..., state[s,c,width-2], xbc[b,c])     oldest first
+ *     v[c]    = sum_k weight[c,k] * window[k] + bias[c],  then v *= sigmoid(v) if conv_silu
+ *     state[s,c,:] = window[1..width-1]
+ * and the decode of oracle_decode runs with x = v[0 : H*Dm], B = v[H*Dm : H*Dm+G*N],
+ * C = v[H*Dm+G*N : conv_dim] (conv outputs kept in double, never rounded). Element (s,c,k)
+ * of the conv pool sits at s*conv_slot_stride + c*stride_c + k*stride_k. */
+int oracle_conv_decode(const void *xbc, int x_dt, const void *conv_w, const void *conv_b,
+                       void *conv_state, int64_t conv_slot_stride, int64_t stride_c,
+                       int64_t stride_k, int32_t width, int conv_silu, const float *A,
+                       const float *dt, const float *dt_bias, const float *D, const void *z,
+                       void *pool, int state_dt, int64_t slot_stride, int32_t P, double *out,
+                       const int32_t *state_indices, int32_t batch, int32_t active, int32_t H,
+                       int32_t G, int32_t Dm, int32_t N, int dt_softplus, int32_t *err_flags)
+{
+    if (!xbc || !conv_w || !A || !dt || !pool || !out || (width > 1 && !conv_state))
+        return 1;
+    if (!valid_dtype(x_dt) || !valid_dtype(state_dt))
+        return 3;
+    if (check_common(batch, active, H, G, Dm, N, slot_stride) || width < 1)
+        return 2;
+    const int64_t cd = (int64_t)H * Dm + 2 * (int64_t)G * N;
+    int32_t err = 0;
+    double *v = malloc(sizeof(double) * (size_t)cd);
+    double *win = malloc(sizeof(double) * (size_t)width);
+    int hpg = H / G;
+    for (int32_t b = 0; b < active; ++b) {
+        int64_t s = resolve_slot(state_indices, b, P, &err);
+        if (s == -1) {
+            for (int64_t i = 0; i < (int64_t)H * Dm; ++i)
+                out[(int64_t)b * H * Dm + i] = 0.0;
+            continue;
+        }
+        if (s < 0)
+            continue;
+        for (int64_t c = 0; c < cd; ++c) {
+            for (int k = 0; k + 1 < width; ++k)
+                win[k] = load(conv_state, x_dt, s * conv_slot_stride + c * stride_c + k * stride_k);
+            win[width - 1] = load(xbc, x_dt, (int64_t)b * cd + c);
+            double acc = conv_b ? load(conv_b, x_dt, c) : 0.0;
+            for (int k = 0; k < width; ++k)
+                acc += load(conv_w, x_dt, c * width + k) * win[k];
+            v[c] = conv_silu ? acc / (1.0 + exp(-acc)) : acc;
+            for (int k = 0; k + 1 < width; ++k)
+                store(conv_state, x_dt, s * conv_slot_stride + c * stride_c + k * stride_k,
+                      win[k + 1]);
+        }
+        for (int h = 0; h < H; ++h) {
+            int g = h / hpg;
+            double dte = effective_dt(dt[(int64_t)b * H + h], dt_bias, h, dt_softplus);
+            double decay = exp((double)A[h] * dte);
+            const double *Bv = v + (int64_t)H * Dm + (int64_t)g * N;
+            const double *Cv = v + (int64_t)H * Dm + (int64_t)G * N + (int64_t)g * N;
+            for (int d = 0; d < Dm; ++d) {
+                double xv = v[(int64_t)h * Dm + d];
+                double y = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    int64_t si = s * slot_stride + ((int64_t)h * Dm + d) * N + n;
+                    double sn = load(pool, state_dt, si) * decay + Bv[n] * dte * xv;
+                    store(pool, state_dt, si, sn);
+                    y += sn * Cv[n];
+                }
+                if (D)
+                    y += (double)D[h] * xv;
+                int64_t oi = ((int64_t)b * H + h) * Dm + d;
+                if (z)
+                    y *= silu(load(z, x_dt, oi));
+                out[oi] = y;
+            }
+        }
+    }
+    free(v);
+    free(win);
+    if (err_flags)
+        *err_flags |= err;
+    return 0;
+}
+
 /* ---------------- slot maintenance ----------------
  * Selective State Update page, invokeMambaStateClear (one slot, or all when slot is -1)
  * and Recurrent State Manager page, clearSlot / copySlotFrom. */

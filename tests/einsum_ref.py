@@ -84,3 +84,16 @@ def ddtree_dual(state, x, A, B, C, dt, dt_bias, D, G, softplus, parents):
                 y = y + D[:, None] * x[r, i]
             out[r, i] = y
     return out
+
+
+def causal_conv_step(state, xbc, w, bias, silu):
+    """One causal conv1d step per channel: window = (state taps oldest first, new input).
+    state [b, C, W-1], xbc [b, C], w [C, W], bias [C] or None (float64 numpy). Returns
+    (conv output [b, C], shifted state [b, C, W-1])."""
+    win = np.concatenate([state, xbc[:, :, None]], axis=2)
+    v = np.einsum("bck,ck->bc", win, w)
+    if bias is not None:
+        v = v + bias[None, :]
+    if silu:
+        v = v / (1.0 + np.exp(-v))
+    return v, win[:, :, 1:]

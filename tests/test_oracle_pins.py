@@ -4,7 +4,7 @@ Each test ties the oracle to a fact the pages or the mathematics fix: the decode
 formula of the Selective State Update page (TensorRT-Edge-LLM C++ API,
 invokeSelectiveStateUpdate), the prefill/stash and replay contracts on the same page,
 the tree verify (invokeSelectiveStateUpdateDDTree) and the accepted-node replay on the
-same page, the padding contract of flashinfer.gdn_fused_decode_step (state_indices),
+same page, the causal conv1d update of flashinfer.gdn_fused_decode_step, the padding contract of flashinfer.gdn_fused_decode_step (state_indices),
 closed forms, independent vectorised formulations and the IEEE storage formats.
 """
 
@@ -14,7 +14,8 @@ import numpy as np
 import pytest
 import torch
 
-from einsum_ref import ancestor_path, ddtree_dual, decode_dense, f64, prefill_dense
+from einsum_ref import (ancestor_path, causal_conv_step, ddtree_dual, decode_dense, f64,
+                        prefill_dense)
 from linear_attention_recurrent_selective_b200.workloads import make_case, make_config
 
 F64 = torch.float64
@@ -659,3 +660,130 @@ def test_replay_node_id_flags(orc):
     assert torch.equal(dense_state(case, pool)[1], dense_state(case)[1])
     assert not torch.equal(dense_state(case, pool)[0], dense_state(case)[0])
     assert not torch.equal(dense_state(case, pool)[2], dense_state(case)[2])
+
+
+# ---------------------------------------------------------------- fused conv1d + decode
+
+def conv_view(case, conv=None):
+    """The conv pool as [P, conv_dim, width-1] (a strided view for either layout)."""
+    conv = case.conv_state if conv is None else conv
+    cd = case.H * case.Dm + 2 * case.G * case.N
+    cs, cc, ck = case.conv_strides
+    return conv.as_strided((case.P, cd, case.width - 1), (cs, cc, ck))
+
+
+def split_xbc(case, v):
+    hd, gn = case.H * case.Dm, case.G * case.N
+    b = v.shape[0]
+    return (v[:, :hd].reshape(b, case.H, case.Dm), v[:, hd:hd + gn].reshape(b, case.G, case.N),
+            v[:, hd + gn:].reshape(b, case.G, case.N))
+
+
+def test_conv_width1_identity_is_plain_decode(orc):
+    case = make_case(seed=70, batch=3, P=5, H=4, G=2, Dm=3, N=8, z=True, conv=1,
+                     state_dtype=F64)
+    case.conv_w = torch.ones_like(case.conv_w)
+    case.conv_b = None
+    case.conv_silu = False
+    out_c, pool_c, _, err = orc.conv_decode_case(case)
+    x, B, C = split_xbc(case, case.xbc)
+    out_d, err_d = orc.decode(x.contiguous(), case.A, B.contiguous(), C.contiguous(), case.dt,
+                              pool_d := case.pool.clone(), dt_bias=case.dt_bias, D=case.D,
+                              z=case.z, state_indices=case.state_indices, batch=3, H=4, G=2,
+                              Dm=3, N=8)
+    assert err == err_d == 0
+    assert same_bits(out_c, out_d) and torch.equal(pool_c, pool_d)
+
+
+@pytest.mark.parametrize("layout", ["ds", "sd"])
+def test_conv_decode_matches_conv_then_einsum(orc, layout):
+    case = make_case(seed=71, batch=4, P=6, H=4, G=2, Dm=3, N=8, z=True, conv=4,
+                     conv_layout=layout, conv_pad=3, state_dtype=F64, n_pad=1)
+    out, pool, conv, err = orc.conv_decode_case(case)
+    assert err == 0
+    idx = case.state_indices.long()
+    live = idx >= 0
+    st0 = conv_view(case)[idx[live]].double().numpy()
+    v, shifted = causal_conv_step(st0, f64(case.xbc)[live.numpy()], f64(case.conv_w),
+                                  f64(case.conv_b), True)
+    x, B, C = split_xbc(case, torch.from_numpy(v))
+    s_new, y = decode_dense(dense_state(case)[idx[live]].numpy(), x.numpy(), f64(case.A),
+                            B.numpy(), C.numpy(), f64(case.dt)[live.numpy()], f64(case.dt_bias),
+                            f64(case.D), f64(case.z)[live.numpy()], case.G, True)
+    np.testing.assert_allclose(out[live].numpy(), y, rtol=1e-12, atol=1e-12)
+    assert (out[~live] == 0).all()
+    np.testing.assert_allclose(dense_state(case, pool)[idx[live]].numpy(), s_new, rtol=1e-12,
+                               atol=1e-12)
+    # the window shift is exact: new taps = old taps 1.. and the raw input
+    assert torch.equal(conv_view(case, conv)[idx[live]],
+                       torch.from_numpy(shifted).to(case.conv_state.dtype))
+    # padding rows and unindexed slots: both pools untouched, padding of the conv slots too
+    used = set(idx[live].tolist())
+    for s_ in range(case.P):
+        if s_ not in used:
+            assert torch.equal(dense_state(case, pool)[s_], dense_state(case)[s_])
+            assert torch.equal(conv_view(case, conv)[s_], conv_view(case)[s_])
+    cs = case.conv_strides[0]
+    pad = conv.view(case.P, cs)[:, cs - 3:]
+    assert torch.equal(pad, case.conv_state.view(case.P, cs)[:, cs - 3:])
+
+
+def test_conv_layouts_agree(orc):
+    a = make_case(seed=72, batch=3, P=4, H=2, G=1, Dm=4, N=8, conv=3, conv_layout="ds")
+    b = make_case(seed=72, batch=3, P=4, H=2, G=1, Dm=4, N=8, conv=3, conv_layout="sd")
+    cd = 2 * 4 + 2 * 8
+    b.conv_state = a.conv_state.view(4, cd, 2).transpose(1, 2).contiguous().view(-1)
+    out_a, pool_a, conv_a, _ = orc.conv_decode_case(a)
+    out_b, pool_b, conv_b, _ = orc.conv_decode_case(b)
+    assert same_bits(out_a, out_b) and same_bits(pool_a, pool_b)
+    assert torch.equal(conv_a.view(4, cd, 2), conv_b.view(4, 2, cd).transpose(1, 2))
+
+
+def test_T_conv_decodes_equal_sequence_conv_then_prefill(orc):
+    """T fused steps equal a causal conv over the whole raw sequence (from the initial
+    window) followed by one T-token prefill over the conv outputs."""
+    T = 5
+    case = make_case(seed=73, batch=2, P=3, H=2, G=1, Dm=4, N=8, z=True, conv=4,
+                     state_dtype=F64, slow_decay=True)
+    g = torch.Generator().manual_seed(74)
+    seq = torch.randn(2, T, case.xbc.shape[1], generator=g).to(case.xbc.dtype)
+    zs = torch.randn(2, T, 2, 4, generator=g)
+    dts = torch.randn(2, T, 2, generator=g)
+    pool, conv = case.pool.clone(), case.conv_state.clone()
+    outs = []
+    for t in range(T):
+        out, _ = orc.conv_decode(seq[:, t].contiguous(), case.conv_w, case.conv_b, conv,
+                                 case.width, case.A, dts[:, t].contiguous(), pool,
+                                 conv_strides=case.conv_strides, dt_bias=case.dt_bias,
+                                 D=case.D, z=zs[:, t].contiguous(),
+                                 state_indices=case.state_indices, batch=2, H=2, G=1, Dm=4,
+                                 N=8)
+        outs.append(out)
+    idx = case.state_indices.long()
+    st = conv_view(case)[idx].double().numpy()
+    full = np.concatenate([st, f64(seq).transpose(0, 2, 1)], axis=2)   # [b, C, W-1+T]
+    w = f64(case.conv_w)
+    v = np.stack([np.einsum("bck,ck->bc", full[:, :, t:t + 4], w) for t in range(T)], 1)
+    v = v + f64(case.conv_b)[None, None, :]
+    v = v / (1.0 + np.exp(-v))
+    hd, gn = 8, 8
+    x = torch.from_numpy(v[:, :, :hd].reshape(2, T, 2, 4).copy())
+    B = torch.from_numpy(v[:, :, hd:hd + gn].reshape(2, T, 1, 8).copy())
+    C = torch.from_numpy(v[:, :, hd + gn:].reshape(2, T, 1, 8).copy())
+    pool_p = case.pool.clone()
+    out_p, _ = orc.prefill(x, case.A, B, C, dts, pool_p, dt_bias=case.dt_bias, D=case.D,
+                           z=zs.double(), state_indices=case.state_indices, batch=2, T=T, H=2,
+                           G=1, Dm=4, N=8)
+    for t in range(T):
+        np.testing.assert_allclose(outs[t].numpy(), out_p[:, t].numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(pool.numpy(), pool_p.numpy(), rtol=1e-10, atol=1e-12)
+    # after T steps the window holds the last width-1 raw inputs
+    assert torch.equal(conv_view(case, conv)[idx], seq[:, T - 3:].transpose(1, 2))
+
+
+def test_conv_decode_index_flag(orc):
+    case = make_case(seed=75, batch=2, P=2, H=2, G=1, Dm=4, N=8, conv=2, indices=[1, 2])
+    out, pool, conv, err = orc.conv_decode_case(case)
+    assert err == 1
+    assert torch.isnan(out[1]).all()
+    assert torch.equal(conv_view(case, conv)[0], conv_view(case)[0])
