@@ -451,6 +451,40 @@ def form_layers(args, device, hbm_peak):
     return forms
 
 
+def form_conv(args, device, hbm_peak):
+    """The batch-256 decode with the causal conv1d (width 4) of its raw xBC channels fused
+    in (both launches of ssu_conv_decode); HBM bound."""
+    from linear_attention_recurrent_selective_b200 import ssu
+    from linear_attention_recurrent_selective_b200.workloads import make_config
+
+    steps, warm = max(3, min(args.steps, 50)), max(3, min(args.warmup, 5))
+    case = make_config("mamba2_conv_decode_b256")
+    d = case.to(device)
+    b, H, G, Dm, N, W = case.batch, case.H, case.G, case.Dm, case.N, case.width
+    out = torch.empty(b, H, Dm, dtype=case.xbc.dtype, device=device)
+
+    def step():
+        ssu.ssu_conv_decode(d.xbc, d.conv_w, d.conv_state, d.A, d.dt, d.pool, out, width=W,
+                            conv_strides=case.conv_strides, nheads=H, ngroups=G, dim=Dm,
+                            conv_bias=d.conv_b, dt_bias=d.dt_bias, D=d.D, z=d.z,
+                            state_indices=d.state_indices, slot_stride=case.slot_stride,
+                            P=case.P)
+
+    ms = time_launches(step, steps, warm, device)
+    xb = case.xbc.element_size()
+    cd = H * Dm + 2 * G * N
+    state_b = b * H * Dm * N * case.pool.element_size() * 2
+    cbytes = (state_b + 2 * b * H * Dm * xb + b * cd * xb + 2 * b * cd * (W - 1) * xb
+              + cd * (W + 1) * xb + b * H * 4)
+    return {"conv_decode": {
+        "workload": "mamba2_conv_decode_b256", "batch": b, "width": W, "ms_per_launch": ms,
+        "seq_head_updates_per_s": b * H / (ms / 1e3), "algorithmic_bytes": cbytes,
+        "launches": 2,
+        "roofline": {"bound": "hbm", "achieved": cbytes / (ms / 1e3) / 1e9, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": cbytes / (ms / 1e3) / 1e9 / hbm_peak,
+                     "traffic": None}}}
+
+
 def form_ddtree(args, device, hbm_peak):
     """Tree verify of one 128-node draft tree per row (batch 16, random recursive trees),
     then the replay of each row's accepted root-to-node path through acceptedNodeIds.
@@ -546,13 +580,15 @@ def main_ours(args):
     device = torch.device("cuda", local if n_world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(device)
     hbm_peak, peak_src = measured_peaks()
-    if args.form in ("prefill", "replay", "layers", "ddtree"):   # one form alone
+    if args.form in ("prefill", "replay", "layers", "ddtree", "conv"):   # one form alone
         if args.form == "prefill":
             forms = form_prefill(args, device, args.batch)
         elif args.form == "replay":
             forms = form_replay(args, device, hbm_peak, args.batch)
         elif args.form == "ddtree":
             forms = form_ddtree(args, device, hbm_peak)
+        elif args.form == "conv":
+            forms = form_conv(args, device, hbm_peak)
         else:
             forms = form_layers(args, device, hbm_peak)
         if rank == 0:
@@ -587,7 +623,7 @@ def main_ours(args):
     if n_world == 1 and not args.no_forms and args.form == "all":
         line["forms"] = {**form_prefill(args, device), **form_replay(args, device, hbm_peak),
                          **form_layers(args, device, hbm_peak),
-                         **form_ddtree(args, device, hbm_peak)}
+                         **form_ddtree(args, device, hbm_peak), **form_conv(args, device, hbm_peak)}
     if n_world == 1 and rank == 0 and not args.no_cpu_baseline and args.form == "all":
         line["cpu_baseline"] = cpu_baseline_decode(case)
     if rank == 0:
@@ -644,7 +680,8 @@ def parse(argv=None):
     ap.add_argument("--batch", type=int, default=0,
                     help="override the batch (pool = 2 x batch), e.g. for a small profile")
     ap.add_argument("--no-forms", action="store_true", help="skip the prefill/replay forms")
-    ap.add_argument("--form", choices=("all", "decode", "prefill", "replay", "layers", "ddtree"),
+    ap.add_argument("--form", choices=("all", "decode", "prefill", "replay", "layers", "ddtree",
+                                       "conv"),
                     default="all",
                     help="run one kernel only (for profiling); its line carries that form")
     ap.add_argument("--no-cpu-baseline", action="store_true")

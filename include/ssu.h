@@ -201,6 +201,39 @@ int ssu_replay_layers(const ssu_replay_layer *layers, int32_t num_layers, int st
                       int32_t *err_flags, ssu_stream_t stream);
 
 /*
+ * ssu_conv_decode -- the causal conv1d update of the raw xBC channels fused with one
+ * decode token, over the same slot of a conv pool and a recurrent pool.
+ * Selective State Update page (struct MambaStateLayerInfo: convState beside
+ * recurrentState; invokeSelectiveStateUpdate for the decode) and the causal conv1d update
+ * of the FlashInfer page flashinfer.gdn_fused_decode_step. For every channel c of a live
+ * row (conv_dim = H*Dm + 2*G*N channels in the order x, B, C):
+ *     window = (the slot's width-1 taps, oldest first, then xbc[b, c])
+ *     v[c]   = sum_k conv_weight[c, k] * window[k] + conv_bias[c], times sigmoid(v[c]) if
+ *              conv_silu;   the taps become window[1 ..]
+ * then ssu_decode runs with x = v[0 : H*Dm] as [H, Dm], B and C = the next two G*N
+ * blocks as [G, N] (kept in fp32, never stored).
+ *   xbc          [batch, conv_dim] x_dtype (raw, pre-conv channels)
+ *   conv_weight  [conv_dim, width] x_dtype;  conv_bias [conv_dim] x_dtype (optional)
+ *   conv_state   conv pool of x_dtype, tap k of channel c of slot s at element
+ *                s*conv_slot_stride + c*conv_stride_c + k*conv_stride_k (k < width-1):
+ *                channel-major windows [P, conv_dim, width-1] use (.., width-1, 1),
+ *                tap-major [P, width-1, conv_dim] use (.., 1, conv_dim); unused when
+ *                width == 1
+ *   width        1..16 taps;  other arguments as in ssu_decode (z, out [batch, H, Dm])
+ * Both pools are indexed by state_indices; a padding row touches neither and outputs 0.
+ * Two launches on `stream`: the fused conv + decode, which only reads the taps (B and C
+ * channels are shared by all heads of a group), then the shift of every live row's taps.
+ */
+int ssu_conv_decode(const void *xbc, int x_dtype, const void *conv_weight,
+                    const void *conv_bias, void *conv_state, int64_t conv_slot_stride,
+                    int64_t conv_stride_c, int64_t conv_stride_k, int32_t width, int conv_silu,
+                    const float *A, const float *dt, const float *dt_bias, const float *D,
+                    const void *z, void *state, int state_dtype, int64_t slot_stride,
+                    int32_t P, void *out, const int32_t *state_indices, int32_t batch,
+                    int32_t active_batch, int32_t nheads, int32_t ngroups, int32_t dim,
+                    int32_t dstate, int dt_softplus, int32_t *err_flags, ssu_stream_t stream);
+
+/*
  * ssu_ddtree -- tree verify: every node of one draft tree per row, each evaluated from the
  * committed state along its own ancestor path.
  * Selective State Update page, mamba_ssm::invokeSelectiveStateUpdateDDTree: the committed

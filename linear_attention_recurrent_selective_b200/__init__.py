@@ -15,6 +15,7 @@ from .ssu import (  # noqa: F401
     pool_copy_slot,
     pool_gather,
     pool_scatter,
+    ssu_conv_decode,
     ssu_ddtree,
     ssu_decode,
     ssu_prefill,

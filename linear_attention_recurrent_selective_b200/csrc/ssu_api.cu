@@ -2,8 +2,8 @@
 //
 // Every entry point validates its arguments on the host without touching device memory
 // (so it stays legal under CUDA-graph capture), returns an ssu_status error without
-// launching anything when a check fails, and otherwise enqueues exactly one kernel on
-// the caller's stream. Values that live on the device (stateIndices, contextLengths,
+// launching anything when a check fails, and otherwise enqueues its kernel on the
+// caller's stream (one launch; ssu_conv_decode enqueues two). Values that live on the device (stateIndices, contextLengths,
 // acceptedLengths, tree parents and depths, accepted node ids) are checked in-kernel,
 // as the padding contract of the FlashInfer page flashinfer.gdn_fused_decode_step
 // requires for graph replay.
@@ -239,6 +239,51 @@ int ssu_replay_layers(const ssu_replay_layer *layers, int32_t num_layers, int st
     a.N = dstate;
     a.max_accept = accepted_node_ids ? max_accept_len : T;
     return finish(ssu::launch_replay(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int ssu_conv_decode(const void *xbc, int x_dtype, const void *conv_weight,
+                    const void *conv_bias, void *conv_state, int64_t conv_slot_stride,
+                    int64_t conv_stride_c, int64_t conv_stride_k, int32_t width, int conv_silu,
+                    const float *A, const float *dt, const float *dt_bias, const float *D,
+                    const void *z, void *state, int state_dtype, int64_t slot_stride,
+                    int32_t P, void *out, const int32_t *state_indices, int32_t batch,
+                    int32_t active_batch, int32_t nheads, int32_t ngroups, int32_t dim,
+                    int32_t dstate, int dt_softplus, int32_t *err_flags, ssu_stream_t stream)
+{
+    if (!valid_dtype(x_dtype))
+        return SSU_ERR_DTYPE;
+    if (width < 1 || width > 16)
+        return SSU_ERR_SHAPE;
+    int rc = check_sizes(state_dtype, slot_stride, P, state_indices, batch, active_batch,
+                         nheads, ngroups, dim, dstate);
+    if (rc != SSU_OK || active_batch == 0)
+        return rc;
+    const int64_t cd = (int64_t)nheads * dim + 2 * (int64_t)ngroups * dstate;
+    if (width > 1) {
+        if (conv_slot_stride < 0 || conv_stride_c < 0 || conv_stride_k < 0)
+            return SSU_ERR_SHAPE;
+        // every (channel, tap) of a slot must lie inside the slot's extent
+        if ((cd - 1) * conv_stride_c + (int64_t)(width - 2) * conv_stride_k >= conv_slot_stride)
+            return SSU_ERR_SHAPE;
+    }
+    if (!xbc || !conv_weight || !A || !dt || !state || !out || (width > 1 && !conv_state))
+        return SSU_ERR_NULL;
+    if ((rc = check_pool_alignment(state, state_dtype, slot_stride)) != SSU_OK)
+        return rc;
+    ssu::ConvArgs a;
+    a.d = pack_decode(nullptr, x_dtype, A, nullptr, nullptr, x_dtype, dt, dt_bias, D, z, state,
+                      slot_stride, P, out, state_indices, batch, active_batch, nheads, ngroups,
+                      dim, dstate, dt_softplus, err_flags);
+    a.xbc = xbc;
+    a.w = conv_weight;
+    a.bias = conv_bias;
+    a.cstate = conv_state;
+    a.cslot = conv_slot_stride;
+    a.cc = conv_stride_c;
+    a.ck = conv_stride_k;
+    a.width = width;
+    a.silu = conv_silu ? 1 : 0;
+    return finish(ssu::launch_conv_decode(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int ssu_ddtree(const void *x, int x_dtype, const float *A, const void *B, const void *C,

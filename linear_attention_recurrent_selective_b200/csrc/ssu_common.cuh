@@ -55,6 +55,16 @@ struct ReplayArgs {
     int32_t P, batch, active, T, H, G, Dm, N, max_accept;
 };
 
+struct ConvArgs {
+    DecodeArgs d;             // x, B, C unused: the conv outputs take their place
+    const void *xbc;          // [batch, conv_dim] raw channels (x, B, C order), x dtype
+    const void *w;            // [conv_dim, width], x dtype
+    const void *bias;         // [conv_dim] or NULL, x dtype
+    void *cstate;             // conv pool, element (s, c, k) at s*cslot + c*cc + k*ck
+    int64_t cslot, cc, ck;
+    int32_t width, silu;
+};
+
 struct TreeArgs {
     DecodeArgs d;             // x/B/C/dt/out carry a node axis [batch, T, ...]; z unused
     const int32_t *parents;   // treeParentIds [batch, T]
@@ -68,6 +78,7 @@ int launch_decode(const DecodeArgs &a, int state_dtype, cudaStream_t s);
 int launch_prefill(const PrefillArgs &a, int state_dtype, cudaStream_t s);
 int launch_replay(const ReplayArgs &a, int state_dtype, cudaStream_t s);
 int launch_ddtree(const TreeArgs &a, int state_dtype, cudaStream_t s);
+int launch_conv_decode(const ConvArgs &a, int state_dtype, cudaStream_t s);
 int launch_clear(void *pool, int64_t bytes, cudaStream_t s);
 int launch_copy(void *dst, const void *src, int64_t bytes, cudaStream_t s);
 int launch_clear_layers(const ssu_layer_states *layers, int32_t num_layers, int32_t P,

@@ -1,0 +1,291 @@
+// ssu_conv.cu -- the causal conv1d update of the xBC channels fused with the decode.
+//
+// Selective State Update page (TensorRT-Edge-LLM C++ API): a slot carries a convolution
+// state beside the recurrent state (struct MambaStateLayerInfo, convState), and the
+// decode of invokeSelectiveStateUpdate consumes x, B and C. The causal conv1d update is
+// the one of the FlashInfer page flashinfer.gdn_fused_decode_step: depthwise weights
+// [conv_dim, width], bias [conv_dim], a conv pool of the last width-1 raw inputs of every
+// channel, updated in place and indexed by the same state index as the recurrent pool,
+// padding rows (negative index) touching neither pool. Per channel c of a live row:
+//     window = (taps of the slot, oldest first, then the new raw input xbc[b, c])
+//     v[c]   = sum_k w[c, k] window[k] + bias[c], then v * sigmoid(v)
+//     taps   = window[1 ..]
+// and x = v[0, H*Dm), B = v[H*Dm, +G*N), C = v[H*Dm+G*N, +G*N) feed the decode.
+//
+// The conv outputs are never stored: every unit of the decode pipeline (up to 128 dim
+// rows of one head, see ssu_stream.cuh) computes the conv outputs it needs -- its x rows
+// and its group's B and C columns -- in fp32 from the old taps, then streams its state
+// tiles as the decode kernel does. Each warp takes a contiguous range of units, so that
+// consecutive units share their batch row: the row's slot index and the lane's B and C
+// conv outputs are computed once per (row, group) and reused. B and C channels are shared by all heads of a group,
+// so no unit may shift their taps while another might still read them; the shift of
+// every tap therefore runs as a second, short launch on the same stream, after the first
+// has finished (a few tens of KB per row against MBs of recurrent state).
+#include "ssu_stream.cuh"
+
+namespace ssu {
+namespace {
+
+using namespace stream;
+
+constexpr int kUT = 8;   // units of up to 8 tiles, as in the decode
+
+struct ConvRows {
+    const void *pool;
+    const int32_t *idx;
+    int32_t P;
+    __device__ __forceinline__ UnitRes resolve(const LUnit &lu) const
+    {
+        return UnitRes{static_cast<const char *>(pool), idx ? idx[lu.un.b] : lu.un.b, 0};
+    }
+    __device__ __forceinline__ bool moves(const UnitRes &r) const
+    {
+        return r.slot >= 0 && r.slot < P;
+    }
+};
+
+// Conv output of channel ch of batch row b (slot's taps at tap0 = slot * cslot).
+__device__ __forceinline__ float conv_out(const ConvArgs &c, int dtype, int64_t xrow,
+                                          int64_t tap0, int64_t ch)
+{
+    float acc = c.bias ? ld_f32(c.bias, dtype, ch) : 0.f;
+    const int64_t w0 = ch * c.width;
+    const int64_t t0 = tap0 + ch * c.cc;
+#pragma unroll 4
+    for (int k = 0; k + 1 < c.width; ++k)
+        acc = fmaf(ld_f32(c.w, dtype, w0 + k), ld_f32(c.cstate, dtype, t0 + k * c.ck), acc);
+    acc = fmaf(ld_f32(c.w, dtype, w0 + c.width - 1), ld_f32(c.xbc, dtype, xrow + ch), acc);
+    return c.silu ? silu_f(acc) : acc;
+}
+
+template <typename S, int N>
+__global__ void __launch_bounds__(kWarps * 32)
+ssu_conv_decode_kernel(const __grid_constant__ ConvArgs ca, const int cph, const int nunits)
+{
+    using G = Geo<S, N, kUT>;
+    using V = Vec16<S>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const DecodeArgs &a = ca.d;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const WarpViews w = warp_views(smem, warp);
+    float *xs = w.f0;                           // unit x (conv outputs), [CR]
+    float *ys = w.f1;                           // unit row sums, [CR]
+    init_ring(w, lane);
+
+    const int H = a.H, Dm = a.Dm, hpg = H / a.G;
+    const int64_t cd = (int64_t)H * Dm + 2 * (int64_t)a.G * N;   // conv channels
+    // this warp's contiguous range of units [first, last): the producer walks it with a
+    // stride of 1 (its "unit count" is the range end)
+    const int gw = blockIdx.x * kWarps + warp;
+    const int nw = gridDim.x * kWarps;
+    const int first = (int)((int64_t)nunits * gw / nw);
+    const int last = (int)((int64_t)nunits * (gw + 1) / nw);
+    const ConvRows rows{a.state, a.idx, a.P};
+    Producer<G, N, ConvRows> prod;
+    if (lane == 0) {
+        prod.start(rows, first, 1, nunits, cph, last, H, Dm);
+#pragma unroll
+        for (int s = 0; s < kStages; ++s)
+            prod.issue(rows, a.slot_stride, first, 1, nunits, cph, last, H, Dm, w, s);
+    }
+
+    const int ln = lane % G::LPR, sub = lane / G::LPR;
+    int c = 0;                                  // tiles consumed by this warp
+    int cur_b = -1, cur_g = -1, slot0 = -1;
+    float Bn[G::E], Cn[G::E];
+    for (int u = first; u < last; ++u) {
+        const Unit un = unit_at(u, cph, G::CR, H, Dm);
+        const int tiles = (un.rows + G::RT - 1) / G::RT;
+        const int64_t orow = ((int64_t)un.b * H + un.h) * Dm + un.row0;
+        if (un.b != cur_b)
+            slot0 = a.idx ? a.idx[un.b] : un.b;
+        const bool live = slot0 >= 0 && slot0 < a.P;
+        const int64_t tap0 = (int64_t)(live ? slot0 : 0) * ca.cslot;
+        const int64_t xb = (int64_t)un.b * cd;
+
+        // ---- per-unit inputs: dt, the conv outputs of the unit's x rows and of the
+        // lane's B and C columns, z
+        const float dte = effective_dt(a.dt[(int64_t)un.b * H + un.h], a.dt_bias, un.h,
+                                       a.softplus);
+        const float dA = expf(a.A[un.h] * dte);
+        const float Dh = a.D ? a.D[un.h] : 0.f;
+        float xo[G::XR], zo[G::XR];
+        if (un.b != cur_b || un.h / hpg != cur_g) {     // B and C conv of a new (row, group)
+            cur_b = un.b;
+            cur_g = un.h / hpg;
+            const int64_t bch = (int64_t)H * Dm + (int64_t)(un.h / hpg) * N;
+            const int64_t cch = bch + (int64_t)a.G * N;
+#pragma unroll
+            for (int v = 0; v < G::NV; ++v)
+#pragma unroll
+                for (int e = 0; e < G::VEC; ++e) {
+                    const int n = G::col(v, ln, e);
+                    Bn[v * G::VEC + e] = live ? conv_out(ca, a.x_dtype, xb, tap0, bch + n) : 0.f;
+                    Cn[v * G::VEC + e] = live ? conv_out(ca, a.x_dtype, xb, tap0, cch + n) : 0.f;
+                }
+        }
+#pragma unroll
+        for (int m = 0; m < G::XR; ++m) {
+            const int r = lane + 32 * m;
+            const bool in = r < un.rows;
+            xo[m] = (in && live) ? conv_out(ca, a.x_dtype, xb, tap0,
+                                            (int64_t)un.h * Dm + un.row0 + r)
+                                 : 0.f;
+            zo[m] = (in && a.z) ? ld_f32(a.z, a.x_dtype, orow + r) : 0.f;
+            if (r < G::CR)
+                xs[r] = xo[m];
+        }
+        __syncwarp();
+
+        int slot = -1;
+        for (int j = 0; j < tiles; ++j, ++c) {
+            if (!wait_tile(w, c, lane == 0 ? prod.issued : 0, lane, a.err))
+                return;
+            const int s = c % kStages;
+            slot = w.ctl->slot[s];
+            if (w.ctl->moves[s]) {
+                const int rt = min(G::RT, un.rows - j * G::RT);
+                const uint8_t *buf = w.ring + s * kTileBytes;
+                S *dst = static_cast<S *>(a.state) + (int64_t)slot * a.slot_stride +
+                         ((int64_t)un.h * Dm + un.row0 + j * G::RT) * N;
+                uint4 raw[G::RPT][G::NV];
+#pragma unroll
+                for (int i = 0; i < G::RPT; ++i) {
+                    const int r = i * G::RPW + sub;
+#pragma unroll
+                    for (int v = 0; v < G::NV; ++v)
+                        raw[i][v] = r < rt ? *reinterpret_cast<const uint4 *>(
+                                                 buf + r * G::ROW_BYTES + (v * G::LPR + ln) * 16)
+                                           : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int i = 0; i < G::RPT; ++i) {
+                    const int r = i * G::RPW + sub;
+                    const float dtx = r < rt ? dte * xs[j * G::RT + r] : 0.f;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int v = 0; v < G::NV; ++v) {
+                        float f[G::VEC];
+                        V::unpack(raw[i][v], f);
+#pragma unroll
+                        for (int e = 0; e < G::VEC; ++e) {
+                            const float sn = fmaf(f[e], dA, Bn[v * G::VEC + e] * dtx);
+                            f[e] = sn;
+                            acc = fmaf(sn, Cn[v * G::VEC + e], acc);
+                        }
+                        if (r < rt)
+                            *reinterpret_cast<uint4 *>(dst + (int64_t)r * N + G::col(v, ln, 0)) =
+                                V::pack(f);
+                    }
+#pragma unroll
+                    for (int off = G::LPR / 2; off > 0; off >>= 1)
+                        acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                    if (ln == 0 && r < rt)
+                        ys[j * G::RT + r] = acc;
+                }
+            }
+            __syncwarp();                        // every lane is done with buffer s
+            if (lane == 0)
+                prod.issue(rows, a.slot_stride, first, 1, nunits, cph, last, H, Dm, w, s);
+        }
+
+        // ---- the unit's outputs, one coalesced store per 32 rows
+        if (slot >= a.P) {                       // caller bug: skip the row and report it
+            if (lane == 0 && un.h == 0 && un.row0 == 0 && a.err)
+                atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
+        } else {
+#pragma unroll
+            for (int m = 0; m < G::XR; ++m) {
+                const int r = lane + 32 * m;
+                if (r < un.rows) {
+                    float y = 0.f;               // padding row: zero
+                    if (slot >= 0) {
+                        y = ys[r] + Dh * xo[m];
+                        if (a.z)
+                            y *= silu_f(zo[m]);
+                    }
+                    st_f32(a.out, a.x_dtype, orow + r, y);
+                }
+            }
+        }
+        __syncwarp();                            // xs / ys are reused by the next unit
+    }
+}
+
+// Shift the conv window of every channel of every live row by one raw input (runs after
+// the fused decode has read the old windows).
+__global__ void __launch_bounds__(256)
+conv_shift_kernel(const __grid_constant__ ConvArgs ca, const int64_t cd, const int64_t total)
+{
+    const DecodeArgs &a = ca.d;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t b = e / cd, ch = e % cd;
+        const int slot = a.idx ? a.idx[b] : (int)b;
+        if (slot < 0 || slot >= a.P)
+            continue;
+        const int64_t t0 = (int64_t)slot * ca.cslot + ch * ca.cc;
+        uint32_t prev = ld_bits(ca.xbc, a.x_dtype, b * cd + ch);
+        for (int k = ca.width - 2; k >= 0; --k) {      // newest tap first
+            const uint32_t old = ld_bits(ca.cstate, a.x_dtype, t0 + k * ca.ck);
+            if (a.x_dtype == SSU_F32)
+                static_cast<uint32_t *>(ca.cstate)[t0 + k * ca.ck] = prev;
+            else
+                static_cast<uint16_t *>(ca.cstate)[t0 + k * ca.ck] = static_cast<uint16_t>(prev);
+            prev = old;
+        }
+    }
+}
+
+template <typename S, int N>
+int launch_n(const ConvArgs &ca, cudaStream_t stream)
+{
+    using G = Geo<S, N, kUT>;
+    const DecodeArgs &a = ca.d;
+    const int64_t cph = (a.Dm + G::CR - 1) / G::CR;
+    const int64_t nunits = (int64_t)a.active * a.H * cph;
+    if (nunits == 0)
+        return SSU_OK;
+    if (nunits > 0x7fffffffLL)
+        return SSU_ERR_SHAPE;
+    const int grid = persistent_grid<ssu_conv_decode_kernel<S, N>>(nunits);
+    ssu_conv_decode_kernel<S, N><<<grid, kWarps * 32, kSmemBytes, stream>>>(ca, (int)cph,
+                                                                            (int)nunits);
+    if (ca.width > 1) {
+        const int64_t cd = (int64_t)a.H * a.Dm + 2 * (int64_t)a.G * N;
+        const int64_t total = (int64_t)a.active * cd;
+        int64_t blocks = (total + 255) / 256;
+        if (blocks > 148 * 16)
+            blocks = 148 * 16;
+        conv_shift_kernel<<<(unsigned)blocks, 256, 0, stream>>>(ca, cd, total);
+    }
+    return SSU_OK;
+}
+
+template <typename S>
+int launch_s(const ConvArgs &a, cudaStream_t s)
+{
+    switch (a.d.N) {
+    case 8: return launch_n<S, 8>(a, s);
+    case 16: return launch_n<S, 16>(a, s);
+    case 32: return launch_n<S, 32>(a, s);
+    case 64: return launch_n<S, 64>(a, s);
+    case 128: return launch_n<S, 128>(a, s);
+    case 256: return launch_n<S, 256>(a, s);
+    default: return SSU_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace
+
+int launch_conv_decode(const ConvArgs &a, int state_dtype, cudaStream_t s)
+{
+    switch (state_dtype) {
+    case SSU_F32: return launch_s<float>(a, s);
+    case SSU_F16: return launch_s<__half>(a, s);
+    case SSU_BF16: return launch_s<__nv_bfloat16>(a, s);
+    default: return SSU_ERR_DTYPE;
+    }
+}
+
+}  // namespace ssu

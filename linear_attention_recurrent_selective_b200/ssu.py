@@ -11,6 +11,8 @@ Semantics (Selective State Update page of the TensorRT-Edge-LLM C++ API):
                times silu(z) when z is given (invokeSelectiveStateUpdate)
   ssu_prefill  the same over [batch, T] tokens in one launch, optional replay stash
                (invokeSelectiveStateUpdatePrefill)
+  ssu_conv_decode  causal conv1d update of the raw xBC channels fused with the decode
+               (convState beside the recurrent state; FlashInfer conv update)
   ssu_ddtree   tree verify: every node of a draft tree from the committed state along its
                ancestor path, stash per node (invokeSelectiveStateUpdateDDTree)
   ssu_replay   re-apply the first acceptedLengths[b] stashed tokens, or the accepted
@@ -42,7 +44,7 @@ FLAG_TREE = 64
 
 # Every C entry point declared in include/ssu.h, in declaration order.
 ENTRY_POINTS = ("ssu_decode", "ssu_prefill", "ssu_replay", "ssu_replay_layers",
-                "ssu_ddtree", "pool_clear_slot", "pool_copy_slot", "pool_clear_slot_layers",
+                "ssu_conv_decode", "ssu_ddtree", "pool_clear_slot", "pool_copy_slot", "pool_clear_slot_layers",
                 "pool_gather", "pool_scatter", "ssu_status_string")
 
 # Byte layouts of the per-layer pointer records of include/ssu.h (packed pointers).
@@ -87,6 +89,9 @@ def lib() -> ctypes.CDLL:
                              i32, i32, vp, i32, vp, vp]
     L.ssu_replay_layers.argtypes = [vp, i32, ci, i64, i32, vp, vp, i32, i32, i32, i32, i32,
                                     i32, i32, vp, i32, vp, vp]
+    L.ssu_conv_decode.argtypes = [vp, ci, vp, vp, vp, i64, i64, i64, i32, ci, vp, vp, vp, vp,
+                                  vp, vp, ci, i64, i32, vp, vp, i32, i32, i32, i32, i32, i32,
+                                  ci, vp, vp]
     L.ssu_ddtree.argtypes = [vp, ci, vp, vp, vp, ci, vp, vp, vp, vp, ci, i64, i32, vp, vp, vp,
                              vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, ci, vp, vp]
     L.pool_clear_slot.argtypes = [vp, i64, i32, i32, vp]
@@ -229,6 +234,40 @@ def ssu_replay(state, stash, accepted_lengths, *, state_indices=None, active_bat
         *_node_ids(accepted_node_ids), _ptr(err_flags, "err_flags", torch.int32),
         _stream(stream))
     _check("ssu_replay", rc)
+
+
+def ssu_conv_decode(xbc, conv_weight, conv_state, A, dt, state, out, *, width, conv_strides,
+                    nheads, ngroups, dim, conv_bias=None, conv_silu=True, dt_bias=None,
+                    D=None, z=None, state_indices=None, active_batch=None, dt_softplus=True,
+                    err_flags=None, slot_stride=None, P=None, stream=None):
+    """Causal conv1d update of the raw channels xbc [batch, H*Dm + 2*G*N] (x, B, C order)
+    fused with one decode token. conv_state: the conv pool (any layout), with
+    conv_strides = (slot, channel, tap) element strides; both pools updated in place."""
+    batch = xbc.shape[0]
+    H, G, Dm = nheads, ngroups, dim
+    N = (xbc.shape[1] - H * Dm) // (2 * G)
+    active = batch if active_batch is None else active_batch
+    stride, P = _pool_geometry(state, slot_stride, P, H * Dm * N)
+    if out.dtype != xbc.dtype or tuple(out.shape) != (batch, H, Dm):
+        raise ValueError("out must be [batch, H, Dm] in xbc's dtype")
+    for t, name in ((conv_weight, "conv_weight"), (conv_bias, "conv_bias"), (z, "z")):
+        if t is not None and t.dtype != xbc.dtype:
+            raise ValueError(f"{name} must have xbc's dtype")
+    if conv_state is not None and conv_state.dtype != xbc.dtype:
+        raise ValueError("conv_state must have xbc's dtype")
+    cs, cc, ck = conv_strides
+    f32 = torch.float32
+    rc = lib().ssu_conv_decode(
+        _ptr(xbc, "xbc"), _dt(xbc, "xbc"), _ptr(conv_weight, "conv_weight"),
+        _ptr(conv_bias, "conv_bias"),
+        None if conv_state is None else ctypes.c_void_p(conv_state.data_ptr()), cs, cc, ck,
+        width, int(bool(conv_silu)), _ptr(A, "A", f32), _ptr(dt, "dt", f32),
+        _ptr(dt_bias, "dt_bias", f32), _ptr(D, "D", f32), _ptr(z, "z"),
+        ctypes.c_void_p(state.data_ptr()), _dt(state, "state"), stride, P, _ptr(out, "out"),
+        _ptr(state_indices, "state_indices", torch.int32), batch, active, H, G, Dm, N,
+        int(bool(dt_softplus)), _ptr(err_flags, "err_flags", torch.int32), _stream(stream))
+    _check("ssu_conv_decode", rc)
+    return out
 
 
 def ssu_ddtree(x, A, B, C, dt, state, out, parent_ids, depths, stash, *, dt_bias=None,

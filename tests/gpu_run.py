@@ -73,3 +73,20 @@ def ddtree(case, pool=None, err=True):
                    slot_stride=case.slot_stride, P=case.P)
     torch.cuda.synchronize()
     return out.cpu(), pool.cpu(), tuple(t.cpu() for t in st), (int(e.item()) if err else None)
+
+
+def conv_decode(case, pool=None, conv=None, err=True, stream=None):
+    """Fused conv1d + decode of a conv case; returns (out, pool, conv pool, err) on the host."""
+    d = dev(case)
+    pool = d.pool.clone() if pool is None else pool
+    conv = d.conv_state.clone() if conv is None else conv
+    out = torch.full((case.batch, case.H, case.Dm), NAN, dtype=case.xbc.dtype, device="cuda")
+    e = torch.zeros(1, dtype=torch.int32, device="cuda") if err else None
+    ssu.ssu_conv_decode(d.xbc, d.conv_w, conv, d.A, d.dt, pool, out, width=case.width,
+                        conv_strides=case.conv_strides, nheads=case.H, ngroups=case.G,
+                        dim=case.Dm, conv_bias=d.conv_b, conv_silu=case.conv_silu,
+                        dt_bias=d.dt_bias, D=d.D, z=d.z, state_indices=d.state_indices,
+                        active_batch=case.active, dt_softplus=case.dt_softplus, err_flags=e,
+                        slot_stride=case.slot_stride, P=case.P, stream=stream)
+    torch.cuda.synchronize()
+    return out.cpu(), pool.cpu(), conv.cpu(), (int(e.item()) if err else None)
