@@ -322,3 +322,97 @@ def make_config(name: str, **overrides) -> SSUCase:
     kw = dict(CONFIGS[name])
     kw.update(overrides)
     return make_case(name, **kw)
+
+
+@dataclasses.dataclass
+class GDNCase:
+    """One seeded gated delta-rule decode workload (FlashInfer page
+    flashinfer.gdn_fused_decode_step, its recurrent core).
+
+    q, k [batch, HK, K]; v [batch, HV, V]; a (decay input), b (beta input) [batch, HV];
+    A_log, dt_bias [HV] fp32; pool: flat fp32 storage of P slots of slot_stride elements,
+    a slot being [HV, V, K] (V-major, K-last); state_indices [batch] int32 (None: slot b).
+    """
+
+    name: str
+    batch: int
+    P: int
+    HK: int
+    HV: int
+    K: int
+    V: int
+    active: int
+    slot_stride: int
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    a: torch.Tensor
+    b: torch.Tensor
+    A_log: torch.Tensor
+    dt_bias: Optional[torch.Tensor]
+    pool: torch.Tensor
+    state_indices: Optional[torch.Tensor]
+    scale: float = 0.0            # 0: the default 1/sqrt(K)
+    use_l2norm: bool = True
+
+    def to(self, device) -> "GDNCase":
+        fields = {}
+        for f in dataclasses.fields(self):
+            v = getattr(self, f.name)
+            fields[f.name] = v.to(device) if isinstance(v, torch.Tensor) else v
+        return GDNCase(**fields)
+
+
+def make_gdn_case(name: str = "gdn", *, seed: int, batch: int, P: Optional[int] = None,
+                  HK: int, HV: int, K: int, V: int, active: Optional[int] = None,
+                  x_dtype=BF16, indices: str | Sequence[int] = "perm", n_pad: int = 0,
+                  slot_pad: int = 0, dt_bias: bool = True) -> GDNCase:
+    """Draw a GDN decode workload. Laws: pool ~ N(0, 0.1^2); q, k, v, a, b ~ N(0, 1);
+    A_log = log(U(1, 16)); dt_bias ~ N(0, 0.5^2). Draw order: pool, q, k, v, a, b, A_log,
+    dt_bias, stateIndices, padding positions."""
+    P = batch if P is None else P
+    active = batch if active is None else active
+    g = torch.Generator().manual_seed(seed)
+    stride = HV * V * K + slot_pad
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, dtype=F32)
+
+    pool = randn(P * stride) * 0.1
+    q = randn(batch, HK, K).to(x_dtype)
+    k = randn(batch, HK, K).to(x_dtype)
+    v = randn(batch, HV, V).to(x_dtype)
+    a = randn(batch, HV).to(x_dtype)
+    b = randn(batch, HV).to(x_dtype)
+    A_log = torch.log(1.0 + 15.0 * torch.rand(HV, generator=g, dtype=F32))
+    bias = randn(HV) * 0.5 if dt_bias else None
+    if isinstance(indices, str):
+        if indices == "perm":
+            si = torch.randperm(P, generator=g)[:batch].to(torch.int32)
+        elif indices == "none":
+            si = None
+        else:
+            raise ValueError(f"unknown indices mode {indices!r}")
+    else:
+        si = torch.tensor(list(indices), dtype=torch.int32)
+    if n_pad:
+        rows = torch.randperm(active, generator=g)[:n_pad]
+        si = si.clone()
+        si[rows] = -1
+    return GDNCase(name=name, batch=batch, P=P, HK=HK, HV=HV, K=K, V=V, active=active,
+                   slot_stride=stride, q=q, k=k, v=v, a=a, b=b, A_log=A_log, dt_bias=bias,
+                   pool=pool, state_indices=si)
+
+
+# Gated delta-rule decode at a Qwen3-Next-like geometry: 16 key heads, 32 value heads,
+# 128 x 128 fp32 state per value head (2 MiB per slot), batch 256 over a 512-slot pool.
+GDN_CONFIGS = {
+    "gdn_decode_b256": dict(seed=7, batch=256, P=512, HK=16, HV=32, K=128, V=128,
+                            x_dtype=BF16),
+}
+
+
+def make_gdn_config(name: str, **overrides) -> GDNCase:
+    kw = dict(GDN_CONFIGS[name])
+    kw.update(overrides)
+    return make_gdn_case(name, **kw)

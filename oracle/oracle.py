@@ -57,6 +57,8 @@ def lib():
         L.oracle_conv_decode.argtypes = [vp, i, vp, vp, vp, i64, i64, i64, i32, i, vp, vp, vp,
                                          vp, vp, vp, i, i64, i32, vp, vp, i32, i32, i32, i32,
                                          i32, i32, i, vp]
+        L.oracle_gdn_decode.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, ctypes.c_double, i, vp,
+                                        i64, i32, vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.oracle_ddtree.argtypes = [vp, i, vp, vp, vp, i, vp, vp, vp, vp, i, i64, i32,
                                     vp, vp, vp, vp, vp, vp, vp, vp,
                                     i32, i32, i32, i32, i32, i32, i32, i, vp]
@@ -77,7 +79,7 @@ def lib():
         for f in ("oracle_decode", "oracle_prefill", "oracle_replay",
                   "oracle_clear_slot", "oracle_copy_slot", "oracle_replay_layers",
                   "oracle_clear_slot_layers", "oracle_gather_scatter", "oracle_ddtree",
-                  "oracle_conv_decode"):
+                  "oracle_conv_decode", "oracle_gdn_decode"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -210,6 +212,26 @@ def conv_decode(xbc, conv_w, conv_b, conv_state, width, A, dt, pool, *, conv_str
     return out, err.value
 
 
+def gdn_decode(q, k, v, a, b, A_log, pool, *, dt_bias=None, scale=None, use_l2norm=True,
+               state_indices=None, batch, active=None, HK, HV, K, V, slot_stride=None, P=None,
+               out=None):
+    """Gated delta-rule decode token; the fp32 pool [P, HV, V, K] is updated in place.
+    Returns (out float64 [batch, HV, V], err_flags)."""
+    active = batch if active is None else active
+    slot_stride = HV * V * K if slot_stride is None else slot_stride
+    P = pool.numel() // slot_stride if P is None else P
+    scale = K ** -0.5 if not scale else scale
+    if out is None:
+        out = torch.full((batch, HV, V), float("nan"), dtype=torch.float64)
+    err = ctypes.c_int32(0)
+    rc = lib().oracle_gdn_decode(
+        _p(q), _p(k), _p(v), _CODES[q.dtype], _p(a), _p(b), _p(A_log), _p(dt_bias), scale,
+        int(use_l2norm), _p(pool), slot_stride, P, _p(out), _p(state_indices), batch, active,
+        HK, HV, K, V, ctypes.byref(err))
+    _check(rc, "oracle_gdn_decode")
+    return out, err.value
+
+
 def clear_slot(pool, slot_bytes, P, slot):
     _check(lib().oracle_clear_slot(_p(pool), slot_bytes, P, slot), "oracle_clear_slot")
 
@@ -317,3 +339,14 @@ def conv_decode_case(case, pool=None, conv_state=None):
                            Dm=case.Dm, N=case.N, slot_stride=case.slot_stride, P=case.P,
                            dt_softplus=case.dt_softplus, conv_silu=case.conv_silu)
     return out, pool, conv, err
+
+
+def gdn_case(case, pool=None):
+    """Gated delta-rule decode of a workloads.GDNCase; returns (out, pool_after, err)."""
+    pool = case.pool.clone() if pool is None else pool
+    out, err = gdn_decode(case.q, case.k, case.v, case.a, case.b, case.A_log, pool,
+                          dt_bias=case.dt_bias, scale=case.scale, use_l2norm=case.use_l2norm,
+                          state_indices=case.state_indices, batch=case.batch,
+                          active=case.active, HK=case.HK, HV=case.HV, K=case.K, V=case.V,
+                          slot_stride=case.slot_stride, P=case.P)
+    return out, pool, err

@@ -621,6 +621,94 @@ int oracle_conv_decode(const void *xbc, int x_dt, const void *conv_w, const void
     return 0;
 }
 
+/* ---------------- gated delta-rule decode (GDN core) ----------------
+ * FlashInfer page flashinfer.gdn_fused_decode_step, its recurrent core: a paged fp32
+ * state pool [P, HV, V, K] (V-major, K-last, padded slot stride allowed), state_indices
+ * shared with the padding contract above (negative: no state access, output 0; >= P: row
+ * skipped, flag 1). Per active row b and value head hv (key head hk = hv / (HV / HK)):
+ *     q, k      the key head's query and key (K values); with use_l2norm each is divided
+ *               by sqrt(sum of squares + 1e-6); q is then multiplied by scale
+ *     g         = -exp(A_log[hv]) * softplus(a[b,hv] + dt_bias[hv]);  alpha = exp(g)
+ *     beta      = sigmoid(bgate[b,hv])
+ *     S         = alpha * S                         (decay of the whole head state)
+ *     for every row i < V:  u = sum_j S[i][j] k[j];  d = beta * (v[i] - u);
+ *                           S[i][j] += d * k[j];     out[i] = sum_j S[i][j] q[j]
+ * The state is stored back rounded to fp32; out is returned in double. */
+int oracle_gdn_decode(const void *q, const void *k, const void *v, int x_dt,
+                      const void *a_in, const void *b_in, const float *A_log,
+                      const float *dt_bias, double scale, int use_l2norm, float *pool,
+                      int64_t slot_stride, int32_t P, double *out,
+                      const int32_t *state_indices, int32_t batch, int32_t active, int32_t HK,
+                      int32_t HV, int32_t K, int32_t V, int32_t *err_flags)
+{
+    if (!q || !k || !v || !a_in || !b_in || !A_log || !pool || !out)
+        return 1;
+    if (!valid_dtype(x_dt))
+        return 3;
+    if (batch < 0 || active < 0 || active > batch || HK <= 0 || HV <= 0 || HV % HK != 0 ||
+        K <= 0 || V <= 0 || slot_stride < (int64_t)HV * V * K)
+        return 2;
+    int32_t err = 0;
+    double *S = malloc(sizeof(double) * (size_t)V * K);
+    double *qn = malloc(sizeof(double) * (size_t)K);
+    double *kn = malloc(sizeof(double) * (size_t)K);
+    int vpk = HV / HK;
+    for (int32_t b = 0; b < active; ++b) {
+        int64_t s = resolve_slot(state_indices, b, P, &err);
+        if (s == -1) {
+            for (int64_t i = 0; i < (int64_t)HV * V; ++i)
+                out[(int64_t)b * HV * V + i] = 0.0;
+            continue;
+        }
+        if (s < 0)
+            continue;
+        for (int hv = 0; hv < HV; ++hv) {
+            int hk = hv / vpk;
+            double nq = 0.0, nk = 0.0;
+            for (int j = 0; j < K; ++j) {
+                qn[j] = load(q, x_dt, ((int64_t)b * HK + hk) * K + j);
+                kn[j] = load(k, x_dt, ((int64_t)b * HK + hk) * K + j);
+                nq += qn[j] * qn[j];
+                nk += kn[j] * kn[j];
+            }
+            double fq = use_l2norm ? 1.0 / sqrt(nq + 1e-6) : 1.0;
+            double fk = use_l2norm ? 1.0 / sqrt(nk + 1e-6) : 1.0;
+            for (int j = 0; j < K; ++j) {
+                qn[j] *= fq * scale;
+                kn[j] *= fk;
+            }
+            double av = load(a_in, x_dt, (int64_t)b * HV + hv) + (dt_bias ? dt_bias[hv] : 0.0);
+            double g = -exp((double)A_log[hv]) * softplus(av);
+            double alpha = exp(g);
+            double beta = 1.0 / (1.0 + exp(-load(b_in, x_dt, (int64_t)b * HV + hv)));
+            int64_t base = s * slot_stride + (int64_t)hv * V * K;
+            for (int64_t e = 0; e < (int64_t)V * K; ++e)
+                S[e] = alpha * (double)pool[base + e];
+            for (int i = 0; i < V; ++i) {
+                double *row = S + (int64_t)i * K;
+                double u = 0.0;
+                for (int j = 0; j < K; ++j)
+                    u += row[j] * kn[j];
+                double d = beta * (load(v, x_dt, ((int64_t)b * HV + hv) * V + i) - u);
+                double o = 0.0;
+                for (int j = 0; j < K; ++j) {
+                    row[j] += d * kn[j];
+                    o += row[j] * qn[j];
+                }
+                out[((int64_t)b * HV + hv) * V + i] = o;
+            }
+            for (int64_t e = 0; e < (int64_t)V * K; ++e)
+                pool[base + e] = (float)S[e];
+        }
+    }
+    free(S);
+    free(qn);
+    free(kn);
+    if (err_flags)
+        *err_flags |= err;
+    return 0;
+}
+
 /* ---------------- slot maintenance ----------------
  * Selective State Update page, invokeMambaStateClear (one slot, or all when slot is -1)
  * and Recurrent State Manager page, clearSlot / copySlotFrom. */

@@ -97,3 +97,25 @@ def causal_conv_step(state, xbc, w, bias, silu):
     if silu:
         v = v / (1.0 + np.exp(-v))
     return v, win[:, :, 1:]
+
+
+def gdn_dense(S, q, k, v, a, b, A_log, dt_bias, scale, l2norm, HK):
+    """Gated delta-rule decode, vectorised over heads and rows (float64 numpy).
+    S [bt, HV, V, K]; q, k [bt, HK, K]; v [bt, HV, V]; a, b [bt, HV]. Returns (S', out)."""
+    HV = v.shape[1]
+    hk = np.arange(HV) // (HV // HK)
+    qh, kh = q[:, hk, :], k[:, hk, :]
+    if l2norm:
+        qh = qh / np.sqrt((qh * qh).sum(-1, keepdims=True) + 1e-6)
+        kh = kh / np.sqrt((kh * kh).sum(-1, keepdims=True) + 1e-6)
+    qh = qh * scale
+    e = a + (dt_bias[None, :] if dt_bias is not None else 0.0)
+    g = -np.exp(A_log)[None, :] * np.logaddexp(0.0, e)
+    alpha = np.exp(g)
+    beta = 1.0 / (1.0 + np.exp(-b))
+    Sd = S * alpha[:, :, None, None]
+    u = np.einsum("bhvk,bhk->bhv", Sd, kh)
+    d = beta[:, :, None] * (v - u)
+    Sn = Sd + np.einsum("bhv,bhk->bhvk", d, kh)
+    out = np.einsum("bhvk,bhk->bhv", Sn, qh)
+    return Sn, out

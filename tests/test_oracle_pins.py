@@ -4,7 +4,8 @@ Each test ties the oracle to a fact the pages or the mathematics fix: the decode
 formula of the Selective State Update page (TensorRT-Edge-LLM C++ API,
 invokeSelectiveStateUpdate), the prefill/stash and replay contracts on the same page,
 the tree verify (invokeSelectiveStateUpdateDDTree) and the accepted-node replay on the
-same page, the causal conv1d update of flashinfer.gdn_fused_decode_step, the padding contract of flashinfer.gdn_fused_decode_step (state_indices),
+same page, the causal conv1d update and the gated delta-rule core of flashinfer.gdn_fused_decode_step,
+the padding contract of flashinfer.gdn_fused_decode_step (state_indices),
 closed forms, independent vectorised formulations and the IEEE storage formats.
 """
 
@@ -15,8 +16,8 @@ import pytest
 import torch
 
 from einsum_ref import (ancestor_path, causal_conv_step, ddtree_dual, decode_dense, f64,
-                        prefill_dense)
-from linear_attention_recurrent_selective_b200.workloads import make_case, make_config
+                        gdn_dense, prefill_dense)
+from linear_attention_recurrent_selective_b200.workloads import make_case, make_config, make_gdn_case
 
 F64 = torch.float64
 
@@ -787,3 +788,97 @@ def test_conv_decode_index_flag(orc):
     assert err == 1
     assert torch.isnan(out[1]).all()
     assert torch.equal(conv_view(case, conv)[0], conv_view(case)[0])
+
+
+# ---------------------------------------------------------------- gated delta rule (GDN)
+
+def gdn_slots(case, pool=None):
+    pool = case.pool if pool is None else pool
+    return pool.view(case.P, case.slot_stride)[:, :case.HV * case.V * case.K].reshape(
+        case.P, case.HV, case.V, case.K)
+
+
+@pytest.mark.parametrize("l2norm", [True, False])
+def test_gdn_matches_einsum(orc, l2norm):
+    case = make_gdn_case(seed=80, batch=4, P=6, HK=2, HV=4, K=8, V=5, n_pad=1, slot_pad=3)
+    case.use_l2norm = l2norm
+    case.scale = 0.3 if not l2norm else 0.0
+    out, pool, err = orc.gdn_case(case)
+    assert err == 0
+    idx = case.state_indices.long()
+    live = idx >= 0
+    S0 = gdn_slots(case)[idx[live]].double().numpy()
+    Sn, y = gdn_dense(S0, f64(case.q)[live.numpy()], f64(case.k)[live.numpy()],
+                      f64(case.v)[live.numpy()], f64(case.a)[live.numpy()],
+                      f64(case.b)[live.numpy()], f64(case.A_log), f64(case.dt_bias),
+                      case.scale or case.K ** -0.5, l2norm, case.HK)
+    np.testing.assert_allclose(out[live].numpy(), y, rtol=1e-12, atol=1e-12)
+    assert (out[~live] == 0).all()
+    np.testing.assert_allclose(gdn_slots(case, pool)[idx[live]].double().numpy(), Sn,
+                               rtol=2e-7, atol=1e-12)      # one fp32 rounding of the state
+    untouched = set(range(case.P)) - set(idx[live].tolist())
+    for s_ in untouched:
+        assert torch.equal(gdn_slots(case, pool)[s_], gdn_slots(case)[s_])
+    pad = pool.view(case.P, case.slot_stride)[:, -3:]
+    assert torch.equal(pad, case.pool.view(case.P, case.slot_stride)[:, -3:])
+
+
+def test_gdn_delta_rule_stores_value_under_unit_key(orc):
+    """No decay (alpha = 1) and beta = 1 with a one-hot key e_j: the update writes v into
+    column j exactly (S k = v afterwards), leaves the other columns alone, and a query
+    e_j reads v back."""
+    case = make_gdn_case(seed=81, batch=2, P=2, HK=1, HV=2, K=8, V=6, indices="none",
+                         x_dtype=torch.float32, dt_bias=False)
+    case.use_l2norm = False
+    case.scale = 1.0
+    case.A_log = torch.full((2,), -100.0)
+    case.b = torch.full((2, 2), 40.0)
+    j = 3
+    case.k = torch.zeros(2, 1, 8)
+    case.k[:, :, j] = 1.0
+    case.q = case.k.clone()
+    out, pool, _ = orc.gdn_case(case)
+    np.testing.assert_allclose(out.numpy(), case.v.double().numpy(), rtol=0, atol=1e-15)
+    after, before = gdn_slots(case, pool), gdn_slots(case)
+    assert torch.equal(after[..., j], case.v.float())
+    others = [c for c in range(8) if c != j]
+    assert torch.equal(after[..., others], before[..., others])
+
+
+def test_gdn_beta_zero_is_pure_decay(orc):
+    case = make_gdn_case(seed=82, batch=3, P=3, HK=2, HV=2, K=16, V=4, indices="none")
+    case.b = torch.full((3, 2), -60.0).to(case.b.dtype)   # sigmoid(-60) ~ 9e-27
+    out, pool, _ = orc.gdn_case(case)
+    e = case.a.double() + case.dt_bias.double()
+    alpha = torch.exp(-torch.exp(case.A_log.double()) * torch.nn.functional.softplus(e))
+    S0 = gdn_slots(case).double()
+    np.testing.assert_allclose(gdn_slots(case, pool).double().numpy(),
+                               (S0 * alpha[:, :, None, None]).numpy(), rtol=1e-7, atol=1e-30)
+    kq = case.q.double()
+    qn = kq / torch.sqrt((kq * kq).sum(-1, keepdim=True) + 1e-6) * 16 ** -0.5
+    want = torch.einsum("bhvk,bhk->bhv", S0 * alpha[:, :, None, None], qn)
+    np.testing.assert_allclose(out.numpy(), want.numpy(), rtol=1e-6, atol=1e-12)
+
+
+def test_gdn_value_heads_share_their_key_head(orc):
+    """HV = 2 HK: value heads 2j and 2j+1 read key head j; giving them the same state,
+    value and gates gives them the same output."""
+    case = make_gdn_case(seed=83, batch=2, P=2, HK=2, HV=4, K=8, V=4, indices="none")
+    sl = gdn_slots(case)
+    sl[:, 1] = sl[:, 0]
+    sl[:, 3] = sl[:, 2]
+    for t in (case.v, case.a, case.b):
+        t[:, 1] = t[:, 0]
+        t[:, 3] = t[:, 2]
+    case.A_log[1], case.A_log[3] = case.A_log[0], case.A_log[2]
+    case.dt_bias[1], case.dt_bias[3] = case.dt_bias[0], case.dt_bias[2]
+    out, _, _ = orc.gdn_case(case)
+    assert torch.equal(out[:, 0], out[:, 1]) and torch.equal(out[:, 2], out[:, 3])
+    assert not torch.equal(out[:, 0], out[:, 2])
+
+
+def test_gdn_index_flag(orc):
+    case = make_gdn_case(seed=84, batch=2, P=2, HK=1, HV=1, K=8, V=4, indices=[1, 2])
+    out, pool, err = orc.gdn_case(case)
+    assert err == 1 and torch.isnan(out[1]).all()
+    assert torch.equal(gdn_slots(case, pool)[0], gdn_slots(case)[0])
