@@ -485,6 +485,34 @@ def form_conv(args, device, hbm_peak):
                      "traffic": None}}}
 
 
+def form_gdn(args, device, hbm_peak):
+    """Gated delta-rule decode (batch 256, 16 key / 32 value heads, 128 x 128 fp32 state per
+    value head); HBM bound."""
+    from linear_attention_recurrent_selective_b200 import ssu
+    from linear_attention_recurrent_selective_b200.workloads import make_gdn_config
+
+    steps, warm = max(3, min(args.steps, 50)), max(3, min(args.warmup, 5))
+    case = make_gdn_config("gdn_decode_b256")
+    d = case.to(device)
+    b, HK, HV, K, V = case.batch, case.HK, case.HV, case.K, case.V
+    out = torch.empty(b, HV, V, dtype=case.q.dtype, device=device)
+
+    def step():
+        ssu.gdn_decode(d.q, d.k, d.v, d.a, d.b, d.A_log, d.pool, out, dt_bias=d.dt_bias,
+                       state_indices=d.state_indices, slot_stride=case.slot_stride, P=case.P)
+
+    ms = time_launches(step, steps, warm, device)
+    xb = case.q.element_size()
+    gbytes = (b * HV * V * K * 4 * 2 + 2 * b * HK * K * xb + 2 * b * HV * V * xb
+              + 2 * b * HV * xb + b * 4)
+    return {"gdn_decode": {
+        "workload": "gdn_decode_b256", "batch": b, "ms_per_launch": ms,
+        "seq_head_updates_per_s": b * HV / (ms / 1e3), "algorithmic_bytes": gbytes,
+        "roofline": {"bound": "hbm", "achieved": gbytes / (ms / 1e3) / 1e9, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": gbytes / (ms / 1e3) / 1e9 / hbm_peak,
+                     "traffic": None}}}
+
+
 def form_ddtree(args, device, hbm_peak):
     """Tree verify of one 128-node draft tree per row (batch 16, random recursive trees),
     then the replay of each row's accepted root-to-node path through acceptedNodeIds.
@@ -580,7 +608,7 @@ def main_ours(args):
     device = torch.device("cuda", local if n_world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(device)
     hbm_peak, peak_src = measured_peaks()
-    if args.form in ("prefill", "replay", "layers", "ddtree", "conv"):   # one form alone
+    if args.form in ("prefill", "replay", "layers", "ddtree", "conv", "gdn"):   # one form
         if args.form == "prefill":
             forms = form_prefill(args, device, args.batch)
         elif args.form == "replay":
@@ -589,6 +617,8 @@ def main_ours(args):
             forms = form_ddtree(args, device, hbm_peak)
         elif args.form == "conv":
             forms = form_conv(args, device, hbm_peak)
+        elif args.form == "gdn":
+            forms = form_gdn(args, device, hbm_peak)
         else:
             forms = form_layers(args, device, hbm_peak)
         if rank == 0:
@@ -623,7 +653,8 @@ def main_ours(args):
     if n_world == 1 and not args.no_forms and args.form == "all":
         line["forms"] = {**form_prefill(args, device), **form_replay(args, device, hbm_peak),
                          **form_layers(args, device, hbm_peak),
-                         **form_ddtree(args, device, hbm_peak), **form_conv(args, device, hbm_peak)}
+                         **form_ddtree(args, device, hbm_peak), **form_conv(args, device, hbm_peak),
+                         **form_gdn(args, device, hbm_peak)}
     if n_world == 1 and rank == 0 and not args.no_cpu_baseline and args.form == "all":
         line["cpu_baseline"] = cpu_baseline_decode(case)
     if rank == 0:
@@ -681,7 +712,7 @@ def parse(argv=None):
                     help="override the batch (pool = 2 x batch), e.g. for a small profile")
     ap.add_argument("--no-forms", action="store_true", help="skip the prefill/replay forms")
     ap.add_argument("--form", choices=("all", "decode", "prefill", "replay", "layers", "ddtree",
-                                       "conv"),
+                                       "conv", "gdn"),
                     default="all",
                     help="run one kernel only (for profiling); its line carries that form")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -4,7 +4,8 @@
  * The Mamba selective state update over a paged recurrent-state pool, in its forms
  * (single-token decode, multi-token prefill with an optional replay stash, tree verify
  * of a draft tree, and the replay of accepted speculative tokens or tree nodes), plus
- * slot clear, slot copy and gather/scatter.
+ * slot clear, slot copy and gather/scatter; and the gated delta-rule decode core over a
+ * pool with the same conventions.
  *
  * Sources: the "Selective State Update" page of the TensorRT-Edge-LLM C++ API
  * (mamba_ssm::invokeSelectiveStateUpdate, invokeSelectiveStateUpdatePrefill,
@@ -232,6 +233,32 @@ int ssu_conv_decode(const void *xbc, int x_dtype, const void *conv_weight,
                     int32_t P, void *out, const int32_t *state_indices, int32_t batch,
                     int32_t active_batch, int32_t nheads, int32_t ngroups, int32_t dim,
                     int32_t dstate, int dt_softplus, int32_t *err_flags, ssu_stream_t stream);
+
+/*
+ * gdn_decode -- one gated delta-rule decode token over a paged fp32 state pool.
+ * The recurrent core of the FlashInfer page flashinfer.gdn_fused_decode_step (the b/a
+ * projection, the conv1d update and the q/k/v split that the page folds around it are
+ * not part of this call). Per active row b and value head hv, with key head
+ * hk = hv / (num_v_heads / num_k_heads):
+ *     q, k   [batch, num_k_heads, K] of head hk; with use_qk_l2norm each is divided by
+ *            sqrt(sum of squares + 1e-6); q is then multiplied by scale (0: 1/sqrt(K))
+ *     alpha  = exp(-exp(A_log[hv]) * softplus(a[b,hv] + dt_bias[hv]))
+ *     beta   = 1 / (1 + exp(-b[b,hv]))
+ *     every state row i < V (state [P, num_v_heads, V, K], K innermost, slot stride
+ *     slot_stride elements, fp32, updated in place):
+ *         d = beta * (v[b,hv,i] - alpha * (S_i . k));  S_i = alpha * S_i + d * k;
+ *         out[b,hv,i] = S_i . q
+ *   q, k [batch, num_k_heads, K]; v, out [batch, num_v_heads, V]; a, b
+ *   [batch, num_v_heads]: all x_dtype;
+ *   A_log, dt_bias (optional) [num_v_heads] fp32; K = head_k_dim in {8,...,256} (powers
+ *   of two), V = head_v_dim any. Padding and index rules as in ssu_decode.
+ */
+int gdn_decode(const void *q, const void *k, const void *v, int x_dtype, const void *a,
+               const void *b, const float *A_log, const float *dt_bias, float scale,
+               int use_qk_l2norm, float *state, int64_t slot_stride, int32_t P, void *out,
+               const int32_t *state_indices, int32_t batch, int32_t active_batch,
+               int32_t num_k_heads, int32_t num_v_heads, int32_t head_k_dim,
+               int32_t head_v_dim, int32_t *err_flags, ssu_stream_t stream);
 
 /*
  * ssu_ddtree -- tree verify: every node of one draft tree per row, each evaluated from the

@@ -9,6 +9,7 @@ from .ssu import (  # noqa: F401
     ENTRY_POINTS,
     SSUError,
     SSULibraryMissing,
+    gdn_decode,
     lib,
     pool_clear_slot,
     pool_clear_slot_layers,

@@ -286,6 +286,59 @@ int ssu_conv_decode(const void *xbc, int x_dtype, const void *conv_weight,
     return finish(ssu::launch_conv_decode(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int gdn_decode(const void *q, const void *k, const void *v, int x_dtype, const void *a,
+               const void *b, const float *A_log, const float *dt_bias, float scale,
+               int use_qk_l2norm, float *state, int64_t slot_stride, int32_t P, void *out,
+               const int32_t *state_indices, int32_t batch, int32_t active_batch,
+               int32_t num_k_heads, int32_t num_v_heads, int32_t head_k_dim,
+               int32_t head_v_dim, int32_t *err_flags, ssu_stream_t stream)
+{
+    if (!valid_dtype(x_dtype))
+        return SSU_ERR_DTYPE;
+    if (batch < 0 || active_batch < 0 || active_batch > batch || P < 0)
+        return SSU_ERR_SHAPE;
+    if (num_k_heads <= 0 || num_v_heads <= 0 || num_v_heads % num_k_heads != 0 ||
+        head_k_dim <= 0 || head_v_dim <= 0)
+        return SSU_ERR_SHAPE;
+    if (slot_stride < (int64_t)num_v_heads * head_v_dim * head_k_dim)
+        return SSU_ERR_SHAPE;
+    if (!state_indices && active_batch > P)
+        return SSU_ERR_SHAPE;
+    if (!supported_dstate(head_k_dim))
+        return SSU_ERR_UNSUPPORTED;
+    if (active_batch == 0)
+        return SSU_OK;
+    if (!q || !k || !v || !a || !b || !A_log || !state || !out)
+        return SSU_ERR_NULL;
+    int rc;
+    if ((rc = check_pool_alignment(state, SSU_F32, slot_stride)) != SSU_OK)
+        return rc;
+    ssu::GdnArgs g;
+    g.q = q;
+    g.k = k;
+    g.v = v;
+    g.a = a;
+    g.b = b;
+    g.A_log = A_log;
+    g.dt_bias = dt_bias;
+    g.state = state;
+    g.out = out;
+    g.idx = state_indices;
+    g.err = err_flags;
+    g.slot_stride = slot_stride;
+    g.scale = scale != 0.f ? scale : 1.f / sqrtf((float)head_k_dim);
+    g.P = P;
+    g.batch = batch;
+    g.active = active_batch;
+    g.HK = num_k_heads;
+    g.HV = num_v_heads;
+    g.K = head_k_dim;
+    g.V = head_v_dim;
+    g.x_dtype = x_dtype;
+    g.l2norm = use_qk_l2norm ? 1 : 0;
+    return finish(ssu::launch_gdn_decode(g, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int ssu_ddtree(const void *x, int x_dtype, const float *A, const void *B, const void *C,
                int bc_dtype, const float *dt, const float *dt_bias, const float *D,
                const void *state, int state_dtype, int64_t slot_stride, int32_t P, void *out,

@@ -65,6 +65,21 @@ struct ConvArgs {
     int32_t width, silu;
 };
 
+struct GdnArgs {
+    const void *q, *k;        // [batch, HK, K], x dtype
+    const void *v;            // [batch, HV, V], x dtype
+    const void *a, *b;        // decay and beta inputs [batch, HV], x dtype
+    const float *A_log;       // [HV]
+    const float *dt_bias;     // [HV] or NULL
+    float *state;             // fp32 pool [P, HV, V, K]
+    void *out;                // [batch, HV, V], x dtype
+    const int32_t *idx;
+    int32_t *err;
+    int64_t slot_stride;
+    float scale;
+    int32_t P, batch, active, HK, HV, K, V, x_dtype, l2norm;
+};
+
 struct TreeArgs {
     DecodeArgs d;             // x/B/C/dt/out carry a node axis [batch, T, ...]; z unused
     const int32_t *parents;   // treeParentIds [batch, T]
@@ -79,6 +94,7 @@ int launch_prefill(const PrefillArgs &a, int state_dtype, cudaStream_t s);
 int launch_replay(const ReplayArgs &a, int state_dtype, cudaStream_t s);
 int launch_ddtree(const TreeArgs &a, int state_dtype, cudaStream_t s);
 int launch_conv_decode(const ConvArgs &a, int state_dtype, cudaStream_t s);
+int launch_gdn_decode(const GdnArgs &a, cudaStream_t s);
 int launch_clear(void *pool, int64_t bytes, cudaStream_t s);
 int launch_copy(void *dst, const void *src, int64_t bytes, cudaStream_t s);
 int launch_clear_layers(const ssu_layer_states *layers, int32_t num_layers, int32_t P,

@@ -13,6 +13,7 @@ Semantics (Selective State Update page of the TensorRT-Edge-LLM C++ API):
                (invokeSelectiveStateUpdatePrefill)
   ssu_conv_decode  causal conv1d update of the raw xBC channels fused with the decode
                (convState beside the recurrent state; FlashInfer conv update)
+  gdn_decode   gated delta-rule decode core over a paged fp32 pool (FlashInfer GDN page)
   ssu_ddtree   tree verify: every node of a draft tree from the committed state along its
                ancestor path, stash per node (invokeSelectiveStateUpdateDDTree)
   ssu_replay   re-apply the first acceptedLengths[b] stashed tokens, or the accepted
@@ -44,7 +45,7 @@ FLAG_TREE = 64
 
 # Every C entry point declared in include/ssu.h, in declaration order.
 ENTRY_POINTS = ("ssu_decode", "ssu_prefill", "ssu_replay", "ssu_replay_layers",
-                "ssu_conv_decode", "ssu_ddtree", "pool_clear_slot", "pool_copy_slot", "pool_clear_slot_layers",
+                "ssu_conv_decode", "gdn_decode", "ssu_ddtree", "pool_clear_slot", "pool_copy_slot", "pool_clear_slot_layers",
                 "pool_gather", "pool_scatter", "ssu_status_string")
 
 # Byte layouts of the per-layer pointer records of include/ssu.h (packed pointers).
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
     L.ssu_conv_decode.argtypes = [vp, ci, vp, vp, vp, i64, i64, i64, i32, ci, vp, vp, vp, vp,
                                   vp, vp, ci, i64, i32, vp, vp, i32, i32, i32, i32, i32, i32,
                                   ci, vp, vp]
+    L.gdn_decode.argtypes = [vp, vp, vp, ci, vp, vp, vp, vp, ctypes.c_float, ci, vp, i64, i32,
+                             vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
     L.ssu_ddtree.argtypes = [vp, ci, vp, vp, vp, ci, vp, vp, vp, vp, ci, i64, i32, vp, vp, vp,
                              vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, ci, vp, vp]
     L.pool_clear_slot.argtypes = [vp, i64, i32, i32, vp]
@@ -267,6 +270,34 @@ def ssu_conv_decode(xbc, conv_weight, conv_state, A, dt, state, out, *, width, c
         _ptr(state_indices, "state_indices", torch.int32), batch, active, H, G, Dm, N,
         int(bool(dt_softplus)), _ptr(err_flags, "err_flags", torch.int32), _stream(stream))
     _check("ssu_conv_decode", rc)
+    return out
+
+
+def gdn_decode(q, k, v, a, b, A_log, state, out, *, dt_bias=None, scale=None,
+               use_qk_l2norm=True, state_indices=None, active_batch=None, err_flags=None,
+               slot_stride=None, P=None, stream=None):
+    """Gated delta-rule decode token. q, k [batch, HK, K]; v, out [batch, HV, V]; a, b
+    [batch, HV] (same dtype); A_log, dt_bias [HV] fp32; state: fp32 pool [P, HV, V, K]
+    (or flat with slot_stride), updated in place. scale None/0: 1/sqrt(K)."""
+    batch, HK, K = q.shape
+    HV, V = v.shape[1], v.shape[2]
+    active = batch if active_batch is None else active_batch
+    if state.dtype != torch.float32:
+        raise ValueError("the GDN state pool is fp32")
+    stride, P = _pool_geometry(state, slot_stride, P, HV * V * K)
+    for t, name in ((k, "k"), (v, "v"), (a, "a"), (b, "b"), (out, "out")):
+        if t.dtype != q.dtype:
+            raise ValueError(f"{name} must have q's dtype")
+    if tuple(out.shape) != (batch, HV, V):
+        raise ValueError("out must be [batch, HV, V]")
+    f32 = torch.float32
+    rc = lib().gdn_decode(
+        _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _dt(q, "q"), _ptr(a, "a"), _ptr(b, "b"),
+        _ptr(A_log, "A_log", f32), _ptr(dt_bias, "dt_bias", f32), float(scale or 0.0),
+        int(bool(use_qk_l2norm)), ctypes.c_void_p(state.data_ptr()), stride, P,
+        _ptr(out, "out"), _ptr(state_indices, "state_indices", torch.int32), batch, active,
+        HK, HV, K, V, _ptr(err_flags, "err_flags", torch.int32), _stream(stream))
+    _check("gdn_decode", rc)
     return out
 
 

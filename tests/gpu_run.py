@@ -90,3 +90,17 @@ def conv_decode(case, pool=None, conv=None, err=True, stream=None):
                         slot_stride=case.slot_stride, P=case.P, stream=stream)
     torch.cuda.synchronize()
     return out.cpu(), pool.cpu(), conv.cpu(), (int(e.item()) if err else None)
+
+
+def gdn(case, pool=None, err=True):
+    """Gated delta-rule decode of a GDNCase; returns (out, pool, err) on the host."""
+    d = case.to("cuda")
+    pool = d.pool.clone() if pool is None else pool
+    out = torch.full((case.batch, case.HV, case.V), NAN, dtype=case.q.dtype, device="cuda")
+    e = torch.zeros(1, dtype=torch.int32, device="cuda") if err else None
+    ssu.gdn_decode(d.q, d.k, d.v, d.a, d.b, d.A_log, pool, out, dt_bias=d.dt_bias,
+                   scale=case.scale, use_qk_l2norm=case.use_l2norm,
+                   state_indices=d.state_indices, active_batch=case.active, err_flags=e,
+                   slot_stride=case.slot_stride, P=case.P)
+    torch.cuda.synchronize()
+    return out.cpu(), pool.cpu(), (int(e.item()) if err else None)

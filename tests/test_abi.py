@@ -123,3 +123,39 @@ def test_ddtree_empty_calls_need_no_pointers(L):
                  dep=None, sdA=None, sU=None, sB=None, sdt=None)
     assert L.ssu_ddtree(*ddtree_args(active=0, **nulls)) == 0
     assert L.ssu_ddtree(*ddtree_args(T=0, **nulls)) == 0
+
+
+def test_conv_decode_rejects_bad_arguments(L):
+    cd = 80 * 64 + 2 * 128
+    good = dict(xbc=P16, x_dt=2, w=P16, b=None, cst=P16, cs=cd * 3, cc=3, ck=1, width=4, silu=1,
+                A=P16, dt=P16, dtb=None, D=None, z=None, state=P16, sdt=0,
+                stride=80 * 64 * 128, P=512, out=P16, idx=P16, batch=256, active=256, H=80,
+                G=1, Dm=64, N=128, sp=1, err=None, stream=None)
+
+    def call(**kw):
+        a = dict(good)
+        a.update(kw)
+        return L.ssu_conv_decode(*a.values())
+    assert call(xbc=None) == 1 and call(cst=None) == 1 and call(w=None) == 1
+    assert call(width=0) == 2 and call(width=17) == 2
+    assert call(cs=cd * 3 - 1) == 2                 # taps would leave the slot
+    assert call(x_dt=9) == 3 and call(N=24, stride=80 * 64 * 24) == 4
+    assert call(active=0, xbc=None, cst=None, w=None, A=None, dt=None, state=None,
+                out=None) == 0
+    assert call(width=1, cst=None, cs=0, xbc=None) == 1   # width 1 needs no conv pool
+
+
+def test_gdn_rejects_bad_arguments(L):
+    good = dict(q=P16, k=P16, v=P16, x_dt=2, a=P16, b=P16, A_log=P16, dtb=None, scale=0.0,
+                l2=1, state=P16, stride=32 * 128 * 128, P=512, out=P16, idx=P16, batch=256,
+                active=256, HK=16, HV=32, K=128, V=128, err=None, stream=None)
+
+    def call(**kw):
+        a = dict(good)
+        a.update(kw)
+        return L.gdn_decode(*a.values())
+    assert call(q=None) == 1 and call(state=None) == 1 and call(A_log=None) == 1
+    assert call(HV=24) == 2 and call(stride=100) == 2 and call(active=300) == 2
+    assert call(x_dt=7) == 3 and call(K=96, stride=32 * 128 * 96) == 4
+    assert call(state=ctypes.c_void_p(264)) == 6
+    assert call(active=0, q=None, k=None, v=None, state=None) == 0
