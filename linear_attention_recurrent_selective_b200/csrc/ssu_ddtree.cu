@@ -47,22 +47,34 @@ constexpr int kMaxNodes = 128;     // the verify budget
 constexpr int kSmemMax = 227 * 1024;
 constexpr int kBatch = 8;          // loads in flight per thread in the plain-load loops
 
+// Lane mapping of the dense products: the warp's lanes form QG column groups of LG lanes
+// (quarter warps at dstate >= 128); a lane holds R state rows over the K columns of its
+// group, interleaved in 16-byte groups (group q owns float4 column groups q, q + QG, ..).
+// All lanes of a group read the same C address and the groups read adjacent 16-byte
+// chunks, which costs the shared-memory pipe what a warp-wide broadcast costs (2.56 SM
+// cycles per warp-wide 16-byte load on B200, measured) while delivering QG times the
+// data, and every C value loaded serves R rows. RWT warps cover a 64-row tile; the
+// NG = 8 / RWT node groups take every NG-th node.
 template <int N> struct TGeo {
-    static constexpr int KP = N < 128 ? N : 128;      // state columns per pass (per lane)
-    static constexpr int NP = N / KP;                 // passes over dstate
-    static constexpr int CP = N + 4;                  // padded fp32 row of C (floats)
-    static_assert(KP % 8 == 0 || KP == 8, "tree geometry");
+    static constexpr int QG = N >= 128 ? 4 : (N == 64 ? 2 : 1);   // column groups
+    static constexpr int LG = 32 / QG;                  // lanes per column group
+    static constexpr int K = N / QG;                    // state columns per lane
+    static constexpr int R = N == 256 ? 2 : (N >= 64 ? 4 : 2);      // rows per lane
+    static constexpr int RW = LG * R;                   // rows per warp
+    static constexpr int RWT = kTile / RW;              // warps per 64-row tile
+    static constexpr int NG = kThreads / 32 / RWT;      // node groups
+    static constexpr int NOWN = QG == 4 ? 1 : (QG == 2 ? R / 2 : R);  // rows a lane finishes
+    static constexpr int CP = N + 4;                    // padded fp32 row of C (floats)
+    static_assert(RW * RWT == kTile && K % 4 == 0 && K * R <= 128 && NG >= 1,
+                  "tree geometry");
 };
-
-constexpr int kRowWarps = 2;                          // warps per 64-row dim tile
-constexpr int kNodeGroups = kThreads / 32 / kRowWarps;  // warp w takes nodes w/2 + 4k
 
 // Shared-memory layout (byte offsets, 16-byte aligned). E = T (T + 1) / 2 bounds the
 // number of (node, path node) pairs; nxb x tiles (2: the next item's is prefetched).
 struct TLayout {
-    int cf, s0, xs, xbytes, cb, coef, pj, abuf, par, cnt, off, da, dtv, wt, total;
+    int cf, s0, xs, xbytes, cb, coef, pj, par, cnt, off, da, dtv, wt, total;
     __host__ __device__ static int up16(int v) { return (v + 15) & ~15; }
-    __host__ __device__ TLayout(int T, int N, int np, int es_x, int es_s, int nxb)
+    __host__ __device__ TLayout(int T, int N, int es_x, int es_s, int nxb)
     {
         const int E = T * (T + 1) / 2;
         cf = 0;
@@ -72,8 +84,7 @@ struct TLayout {
         cb = xs + nxb * xbytes;
         coef = cb + up16(E * 4);
         pj = coef + up16(E * 4);
-        abuf = pj + up16(E);
-        par = abuf + (np > 1 ? T * kTile * 4 : 0);    // partial a_i between dstate passes
+        par = pj + up16(E);
         cnt = par + up16(T * 4);
         off = cnt + up16(T * 4);
         da = off + up16(T * 4);
@@ -444,22 +455,22 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
     const DecodeArgs &a = ta.d;
     const int T = ta.T, H = a.H, Dm = a.Dm;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int ng = warp / kRowWarps;
-    const int d = (warp % kRowWarps) * 32 + lane;    // the lane's dim row within the tile
+    const int ng = warp / Gm::RWT;                   // node group
+    const int cg = lane / Gm::LG;                    // column group
+    const int rb = (warp % Gm::RWT) * Gm::RW + lane % Gm::LG;   // row of the lane's i = 0
     const int es_x = a.x_dtype == SSU_F32 ? 4 : 2;
-    const TLayout lay(T, N, Gm::NP, es_x, (int)sizeof(S), nxb);
+    const TLayout lay(T, N, es_x, (int)sizeof(S), nxb);
     const float *Cf = reinterpret_cast<const float *>(sm + lay.cf);
     const float *coef = reinterpret_cast<const float *>(sm + lay.coef);
     const uint8_t *pj = sm + lay.pj;
-    float *abuf = reinterpret_cast<float *>(sm + lay.abuf);
     const int *cnt = reinterpret_cast<const int *>(sm + lay.cnt);
     const int *off = reinterpret_cast<const int *>(sm + lay.off);
     const float *wt = reinterpret_cast<const float *>(sm + lay.wt);
 
     // Copies for the next item start as early as their buffers allow: the state rows once
-    // every lane holds them in registers (after the last dstate pass when there are
-    // several), the x tile at once when it is double-buffered, else after the item.
-    const bool s0_mid = Gm::NP == 1, x_mid = xasync && nxb == 2;
+    // every lane holds them in registers, the x tile at once when it is double-buffered,
+    // else after the item.
+    const bool x_mid = xasync && nxb == 2;
     const int64_t first = nitems * blockIdx.x / gridDim.x;
     const int64_t last = nitems * (blockIdx.x + 1) / gridDim.x;
     auto xbuf_of = [&](int64_t it) { return nxb == 2 ? (int)((it - first) & 1) : 0; };
@@ -515,93 +526,122 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
         __syncthreads();                 // dt_eff and dA of every node visible
         path_coefs(lay, sm, T);
 
-        // the lane's dim row of the committed state, first dstate pass
-        float2 s[Gm::KP / 2];
-        auto load_pass = [&](int p) {
+        // the lane's R rows of the committed state over its column group
+        float2 st[Gm::R][Gm::K / 2];
 #pragma unroll
-            for (int q = 0; q < Gm::KP / 4; ++q) {
-                const float4 f = d < u.rows ? s0_quad<S, N>(sm + lay.s0, d, p * Gm::KP + 4 * q)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                s[2 * q] = make_float2(f.x, f.y);
-                s[2 * q + 1] = make_float2(f.z, f.w);
+        for (int i = 0; i < Gm::R; ++i) {
+            const int r = rb + i * Gm::LG;
+#pragma unroll
+            for (int j = 0; j < Gm::K / 4; ++j) {
+                const float4 f = r < u.rows
+                                     ? s0_quad<S, N>(sm + lay.s0, r, 4 * (j * Gm::QG + cg))
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                st[i][2 * j] = make_float2(f.x, f.y);
+                st[i][2 * j + 1] = make_float2(f.z, f.w);
             }
-        };
-        load_pass(0);
+        }
         __syncthreads();                 // path coefficients ready; staging buffer free
-        if (next_valid && (s0_mid || x_mid)) {
-            if (s0_mid)
-                prefetch_s0<S, N>(ta, lay, sm, v);
+        if (next_valid) {
+            prefetch_s0<S, N>(ta, lay, sm, v);
             if (x_mid)
                 prefetch_x(ta, lay, sm, v, xbuf_of(it + 1));
             cp_async_commit();
-        }
-        if (next_valid)
             dt_next = dt_of(ta, v);
+        }
         const float Dh = a.D ? a.D[u.h] : 0.f;
 
-        // y_i = W_i a_i + path sum + D x_i for this warp's nodes (every fourth, two at a
-        // time) and the lane's row; four partial-sum chains per node
+        // y_i = W_i a_i + path sum + D x_i for this warp's nodes, two at a time: partial
+        // dot products of the lane's R rows over its columns, then a transposing reduction
+        // across the column groups that leaves each lane with whole rows to finish
 #pragma unroll 1
-        for (int p = 0; p < Gm::NP; ++p) {
-            if (p > 0)
-                load_pass(p);
-#pragma unroll 1
-            for (int i0 = ng; i0 < T; i0 += 2 * kNodeGroups) {
-                const int i1 = i0 + kNodeGroups;
-                const bool two = i1 < T;
-                const float *c0 = Cf + i0 * Gm::CP + p * Gm::KP;
-                const float *c1 = Cf + (two ? i1 : i0) * Gm::CP + p * Gm::KP;
-                float2 a0[4], a1[4];
+        for (int i0 = ng; i0 < T; i0 += 2 * Gm::NG) {
+            const int i1 = i0 + Gm::NG;
+            const bool two = i1 < T;
+            const float *c0 = Cf + i0 * Gm::CP + 4 * cg;
+            const float *c1 = Cf + (two ? i1 : i0) * Gm::CP + 4 * cg;
+            float2 a0[Gm::R][2], a1[Gm::R][2];
 #pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    a0[m] = a1[m] = make_float2(0.f, 0.f);
+            for (int i = 0; i < Gm::R; ++i)
+                a0[i][0] = a0[i][1] = a1[i][0] = a1[i][1] = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int q = 0; q < Gm::KP / 4; ++q) {
-                    const float4 u0 = *reinterpret_cast<const float4 *>(c0 + 4 * q);
-                    const float4 u1 = *reinterpret_cast<const float4 *>(c1 + 4 * q);
-                    const int m = 2 * (q & 1);
-                    a0[m] = __ffma2_rn(s[2 * q], make_float2(u0.x, u0.y), a0[m]);
-                    a1[m] = __ffma2_rn(s[2 * q], make_float2(u1.x, u1.y), a1[m]);
-                    a0[m + 1] = __ffma2_rn(s[2 * q + 1], make_float2(u0.z, u0.w), a0[m + 1]);
-                    a1[m + 1] = __ffma2_rn(s[2 * q + 1], make_float2(u1.z, u1.w), a1[m + 1]);
+            for (int j = 0; j < Gm::K / 4; ++j) {
+                const float4 u0 = *reinterpret_cast<const float4 *>(c0 + 4 * Gm::QG * j);
+                const float4 u1 = *reinterpret_cast<const float4 *>(c1 + 4 * Gm::QG * j);
+#pragma unroll
+                for (int i = 0; i < Gm::R; ++i) {
+                    a0[i][0] = __ffma2_rn(st[i][2 * j], make_float2(u0.x, u0.y), a0[i][0]);
+                    a1[i][0] = __ffma2_rn(st[i][2 * j], make_float2(u1.x, u1.y), a1[i][0]);
+                    a0[i][1] = __ffma2_rn(st[i][2 * j + 1], make_float2(u0.z, u0.w), a0[i][1]);
+                    a1[i][1] = __ffma2_rn(st[i][2 * j + 1], make_float2(u1.z, u1.w), a1[i][1]);
                 }
-                float r[2];
-                r[0] = ((a0[0].x + a0[0].y) + (a0[1].x + a0[1].y)) +
-                       ((a0[2].x + a0[2].y) + (a0[3].x + a0[3].y));
-                r[1] = ((a1[0].x + a1[0].y) + (a1[1].x + a1[1].y)) +
-                       ((a1[2].x + a1[2].y) + (a1[3].x + a1[3].y));
+            }
 #pragma unroll
-                for (int n = 0; n < 2; ++n) {
-                    const int i = n == 0 ? i0 : i1;
-                    if (n == 1 && !two)
-                        break;
-                    float av = r[n];
-                    if (Gm::NP > 1) {            // partial a_i between dstate passes
-                        if (p > 0)
-                            av += abuf[i * kTile + d];
-                        if (p + 1 < Gm::NP) {
-                            abuf[i * kTile + d] = av;
-                            continue;
-                        }
+            for (int n = 0; n < 2; ++n) {
+                if (n == 1 && !two)
+                    break;
+                const int i = n == 0 ? i0 : i1;
+                float p[Gm::R];
+#pragma unroll
+                for (int r = 0; r < Gm::R; ++r) {
+                    const float2 *q2 = n == 0 ? a0[r] : a1[r];
+                    p[r] = (q2[0].x + q2[0].y) + (q2[1].x + q2[1].y);
+                }
+                float own[Gm::NOWN];
+                int oi[Gm::NOWN];                // which of the lane's rows each holds
+                bool ow = true;                  // whether this lane writes them
+                if constexpr (Gm::QG == 1) {
+#pragma unroll
+                    for (int r = 0; r < Gm::R; ++r) {
+                        own[r] = p[r];
+                        oi[r] = r;
                     }
-                    if (d >= u.rows)
+                } else {
+                    // groups cg and cg ^ 1 exchange halves of the rows (xor LG)
+                    const bool odd = cg & 1;
+                    float v[Gm::R / 2];
+#pragma unroll
+                    for (int k = 0; k < Gm::R / 2; ++k) {
+                        const float send = odd ? p[2 * k] : p[2 * k + 1];
+                        const float keep = odd ? p[2 * k + 1] : p[2 * k];
+                        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, Gm::LG);
+                    }
+                    if constexpr (Gm::QG == 2) {
+#pragma unroll
+                        for (int k = 0; k < Gm::R / 2; ++k) {
+                            own[k] = v[k];
+                            oi[k] = 2 * k + (cg & 1);
+                        }
+                    } else if constexpr (Gm::R == 4) {   // four groups: second exchange
+                        const bool hi = cg & 2;
+                        const float send = hi ? v[0] : v[1];
+                        const float keep = hi ? v[1] : v[0];
+                        own[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2 * Gm::LG);
+                        oi[0] = (cg & 1) + 2 * (hi ? 1 : 0);
+                    } else {                     // four groups, two rows
+                        own[0] = v[0] + __shfl_xor_sync(0xffffffffu, v[0], 2 * Gm::LG);
+                        oi[0] = cg & 1;
+                        ow = (cg & 2) == 0;
+                    }
+                }
+                const int cn = cnt[i];
+#pragma unroll
+                for (int k = 0; k < Gm::NOWN; ++k) {
+                    const int d = rb + oi[k] * Gm::LG;
+                    if (!ow || d >= u.rows)
                         continue;
-                    const int cn = cnt[i];
                     float y = 0.f;
                     if (cn > 0)
-                        y = fmaf(wt[i], av, path_sum(coef, pj, xs, a.x_dtype, off[i], cn, d)) +
+                        y = fmaf(wt[i], own[k],
+                                 path_sum(coef, pj, xs, a.x_dtype, off[i], cn, d)) +
                             Dh * xs_at(xs, a.x_dtype, i * kTile + d);
-                    st_f32(a.out, a.x_dtype, (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d,
-                           y);
+                    st_f32(a.out, a.x_dtype,
+                           (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d, y);
                 }
             }
         }
         __syncthreads();                 // every read of this item's buffers is done
-        if (next_valid && (!s0_mid || (xasync && !x_mid))) {
-            if (!s0_mid)
-                prefetch_s0<S, N>(ta, lay, sm, v);
-            if (xasync && !x_mid)
-                prefetch_x(ta, lay, sm, v, xbuf_of(it + 1));
+        if (next_valid && xasync && !x_mid) {
+            prefetch_x(ta, lay, sm, v, 0);
             cp_async_commit();
         }
     }
@@ -618,10 +658,10 @@ int launch_n(const TreeArgs &a, cudaStream_t stream)
         return SSU_OK;
     const int es_x = a.d.x_dtype == SSU_F32 ? 4 : 2;
     int nxb = 2;
-    TLayout lay(a.T, N, Gm::NP, es_x, (int)sizeof(S), nxb);
+    TLayout lay(a.T, N, es_x, (int)sizeof(S), nxb);
     if (lay.total > kSmemMax) {
         nxb = 1;
-        lay = TLayout(a.T, N, Gm::NP, es_x, (int)sizeof(S), nxb);
+        lay = TLayout(a.T, N, es_x, (int)sizeof(S), nxb);
     }
     if (lay.total > kSmemMax)
         return SSU_ERR_UNSUPPORTED;
