@@ -29,12 +29,11 @@
 // the current item computes: coalesced 16-byte copies into shared memory (the state rows
 // with an XOR swizzle of their 16-byte chunks, so that the row-per-lane reads below are
 // free of bank conflicts; the x tile double-buffered when it fits), and the next item's
-// dt is loaded into registers early. Per item, the path coefficients w_im * dt_jm * cb
-// and W_i are formed once per node; a lane holds two dim rows of the committed state
-// over one column group (64 columns at dstate 128) in registers and accumulates a_i with
-// packed FP32 FMAs against broadcast shared loads of C_i; the same warps add the path
-// sums, the column groups' partial sums meet in shared memory (two buffers, so one
-// barrier per chunk of nodes), and the epilogue adds D x and stores.
+// dt is loaded into registers early. Per item: the path coefficients w_im * dt_jm * cb
+// and W_i are formed once per node, then all path sums P[i][d] in one parallel pass (a
+// thread per node and half tile, 32 sums in registers); the dense products run with the
+// lane mapping described at TGeo, a transposing shuffle reduction leaves each lane with
+// whole rows, and out = W_i a_i + P[i][d] + D x is stored without further barriers.
 #include "ssu_async.cuh"
 #include "ssu_common.cuh"
 
@@ -42,10 +41,11 @@ namespace ssu {
 namespace {
 
 constexpr int kThreads = 256;      // 8 warps, one CTA per SM
-constexpr int kTile = 64;          // dim rows per work item, two per lane
+constexpr int kTile = 64;          // dim rows per work item
 constexpr int kMaxNodes = 128;     // the verify budget
 constexpr int kSmemMax = 227 * 1024;
 constexpr int kBatch = 8;          // loads in flight per thread in the plain-load loops
+constexpr int kXS = kTile + 8;     // x tile row stride (elements): rows start in different banks
 
 // Lane mapping of the dense products: the warp's lanes form QG column groups of LG lanes
 // (quarter warps at dstate >= 128); a lane holds R state rows over the K columns of its
@@ -80,10 +80,11 @@ struct TLayout {
         cf = 0;
         s0 = cf + up16(T * (N + 4) * 4);
         xs = s0 + up16(kTile * N * es_s);
-        xbytes = up16(T * kTile * es_x);
+        xbytes = up16(T * kXS * es_x);
         cb = xs + nxb * xbytes;
         coef = cb + up16(E * 4);
-        pj = coef + up16(E * 4);
+        // the coefficients of an item, then its path sums [T][kTile] in the same bytes
+        pj = coef + up16(E * 4 > T * kTile * 4 ? E * 4 : T * kTile * 4);
         par = pj + up16(E);
         cnt = par + up16(T * 4);
         off = cnt + up16(T * 4);
@@ -290,12 +291,12 @@ __device__ void stage_x_plain(const TreeArgs &ta, uint8_t *xs, const Item &u)
         }
 #pragma unroll
         for (int q = 0; q < kBatch; ++q) {
-            const int e = e0 + q * kThreads;
+            const int e = e0 + q * kThreads, xe = (e / kTile) * kXS + e % kTile;
             if (e < T * kTile) {
                 if (a.x_dtype == SSU_F32)
-                    reinterpret_cast<uint32_t *>(xs)[e] = v[q];
+                    reinterpret_cast<uint32_t *>(xs)[xe] = v[q];
                 else
-                    reinterpret_cast<uint16_t *>(xs)[e] = static_cast<uint16_t>(v[q]);
+                    reinterpret_cast<uint16_t *>(xs)[xe] = static_cast<uint16_t>(v[q]);
             }
         }
     }
@@ -325,7 +326,7 @@ __device__ void stage_nodes(const TreeArgs &ta, const TLayout &lay, uint8_t *sm,
         const int i = e / kTile, d = e % kTile;
         if (d < u.rows)
             ta.st_U[(((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d] =
-                xs_at(xs, a.x_dtype, e);
+                xs_at(xs, a.x_dtype, i * kXS + d);
     }
     if (u.dtile == 0 && u.h % (H / G) == 0) {
         const int64_t rows = (int64_t)T * N;
@@ -410,7 +411,7 @@ __device__ __forceinline__ void prefetch_x(const TreeArgs &ta, const TLayout &la
     const char *xg = static_cast<const char *>(a.x);
     for (int k = threadIdx.x; k < T * cpn; k += kThreads) {
         const int i = k / cpn, c = k % cpn;
-        cp_async16(dst + i * kTile * es_x + c * 16,
+        cp_async16(dst + i * kXS * es_x + c * 16,
                    xg + ((((int64_t)u.b * T + i) * a.H + u.h) * a.Dm + u.row0) * es_x + c * 16);
     }
 }
@@ -422,27 +423,58 @@ __device__ __forceinline__ float dt_of(const TreeArgs &ta, const Item &u)
     return threadIdx.x < T ? ta.d.dt[((int64_t)u.b * T + threadIdx.x) * ta.d.H + u.h] : 0.f;
 }
 
-// Sum over node i's path of coef * x_j[d] for the lane's dim row d (four entries per step).
-__device__ __forceinline__ float path_sum(const float *coef, const uint8_t *pj,
-                                          const uint8_t *xs, int x_dtype, int o, int cn, int d)
+// Path sums of the item: P[i][d] = sum over node i's path entries m of coef[o_i + m] *
+// x[j_m][d], for every node and dim row, written over the coefficients (which they no
+// longer need). Thread t takes node t / 2 and 32 consecutive rows (half t % 2), keeps the
+// 32 sums in registers and reads each path node's x row 16 bytes at a time.
+__device__ void path_sums(const TLayout &lay, uint8_t *sm, const uint8_t *xs, int x_dtype,
+                          int T)
 {
-    float p4[4] = {0.f, 0.f, 0.f, 0.f};
-    int k = 0;
-    for (; k + 4 <= cn; k += 4) {
-        float cf[4];
-        int j[4];
+    float *coef = reinterpret_cast<float *>(sm + lay.coef);
+    const uint8_t *pj = sm + lay.pj;
+    const int *cnt = reinterpret_cast<const int *>(sm + lay.cnt);
+    const int *off = reinterpret_cast<const int *>(sm + lay.off);
+    const int i = threadIdx.x >> 1, d0 = (threadIdx.x & 1) * 32;
+    float acc[32];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            cf[m] = coef[o + k + m];
-            j[m] = pj[o + k + m];
+    for (int e = 0; e < 32; ++e)
+        acc[e] = 0.f;
+    const int cn = i < T ? cnt[i] : 0, o = i < T ? off[i] : 0;
+    for (int k = 0; k < cn; ++k) {
+        const float cf = coef[o + k];
+        const int j = pj[o + k];
+        if (x_dtype == SSU_F32) {
+            const float4 *xr = reinterpret_cast<const float4 *>(xs + (j * kXS + d0) * 4);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 v = xr[q];
+                acc[4 * q] = fmaf(cf, v.x, acc[4 * q]);
+                acc[4 * q + 1] = fmaf(cf, v.y, acc[4 * q + 1]);
+                acc[4 * q + 2] = fmaf(cf, v.z, acc[4 * q + 2]);
+                acc[4 * q + 3] = fmaf(cf, v.w, acc[4 * q + 3]);
+            }
+        } else {
+            const uint4 *xr = reinterpret_cast<const uint4 *>(xs + (j * kXS + d0) * 2);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float f[8];
+                if (x_dtype == SSU_BF16)
+                    Vec16<__nv_bfloat16>::unpack(xr[q], f);
+                else
+                    Vec16<__half>::unpack(xr[q], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    acc[8 * q + e] = fmaf(cf, f[e], acc[8 * q + e]);
+            }
         }
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-            p4[m] = fmaf(cf[m], xs_at(xs, x_dtype, j[m] * kTile + d), p4[m]);
     }
-    for (; k < cn; ++k)
-        p4[0] = fmaf(coef[o + k], xs_at(xs, x_dtype, pj[o + k] * kTile + d), p4[0]);
-    return (p4[0] + p4[1]) + (p4[2] + p4[3]);
+    __syncthreads();                     // every coefficient has been read
+    if (i < T) {
+        float4 *pr = reinterpret_cast<float4 *>(coef + i * kTile + d0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            pr[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+    }
 }
 
 template <typename S, int N>
@@ -461,10 +493,8 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
     const int es_x = a.x_dtype == SSU_F32 ? 4 : 2;
     const TLayout lay(T, N, es_x, (int)sizeof(S), nxb);
     const float *Cf = reinterpret_cast<const float *>(sm + lay.cf);
-    const float *coef = reinterpret_cast<const float *>(sm + lay.coef);
-    const uint8_t *pj = sm + lay.pj;
+    const float *psum = reinterpret_cast<const float *>(sm + lay.coef);  // path sums [T][64]
     const int *cnt = reinterpret_cast<const int *>(sm + lay.cnt);
-    const int *off = reinterpret_cast<const int *>(sm + lay.off);
     const float *wt = reinterpret_cast<const float *>(sm + lay.wt);
 
     // Copies for the next item start as early as their buffers allow: the state rows once
@@ -525,6 +555,8 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
         stage_nodes(ta, lay, sm, u, xs, dt_next);
         __syncthreads();                 // dt_eff and dA of every node visible
         path_coefs(lay, sm, T);
+        __syncthreads();                 // path coefficients and W_i ready
+        path_sums(lay, sm, xs, a.x_dtype, T);
 
         // the lane's R rows of the committed state over its column group
         float2 st[Gm::R][Gm::K / 2];
@@ -540,7 +572,7 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
                 st[i][2 * j + 1] = make_float2(f.z, f.w);
             }
         }
-        __syncthreads();                 // path coefficients ready; staging buffer free
+        __syncthreads();                 // path sums ready; staging buffer free
         if (next_valid) {
             prefetch_s0<S, N>(ta, lay, sm, v);
             if (x_mid)
@@ -631,9 +663,8 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
                         continue;
                     float y = 0.f;
                     if (cn > 0)
-                        y = fmaf(wt[i], own[k],
-                                 path_sum(coef, pj, xs, a.x_dtype, off[i], cn, d)) +
-                            Dh * xs_at(xs, a.x_dtype, i * kTile + d);
+                        y = fmaf(wt[i], own[k], psum[i * kTile + d]) +
+                            Dh * xs_at(xs, a.x_dtype, i * kXS + d);
                     st_f32(a.out, a.x_dtype,
                            (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d, y);
                 }
