@@ -478,7 +478,8 @@ def form_conv(args, device, hbm_peak):
     from linear_attention_recurrent_selective_b200.workloads import make_config
 
     steps, warm = max(3, min(args.steps, 50)), max(3, min(args.warmup, 5))
-    case = make_config("mamba2_conv_decode_b256")
+    case = make_config("mamba2_conv_decode_b256",
+                       **(dict(batch=args.batch, P=2 * args.batch) if args.batch else {}))
     d = case.to(device)
     b, H, G, Dm, N, W = case.batch, case.H, case.G, case.Dm, case.N, case.width
     out = torch.empty(b, H, Dm, dtype=case.xbc.dtype, device=device)
@@ -512,7 +513,8 @@ def form_gdn(args, device, hbm_peak):
     from linear_attention_recurrent_selective_b200.workloads import make_gdn_config
 
     steps, warm = max(3, min(args.steps, 50)), max(3, min(args.warmup, 5))
-    case = make_gdn_config("gdn_decode_b256")
+    case = make_gdn_config("gdn_decode_b256",
+                           **(dict(batch=args.batch, P=2 * args.batch) if args.batch else {}))
     d = case.to(device)
     b, HK, HV, K, V = case.batch, case.HK, case.HV, case.K, case.V
     out = torch.empty(b, HV, V, dtype=case.q.dtype, device=device)
