@@ -222,8 +222,9 @@ int ssu_replay_layers(const ssu_replay_layer *layers, int32_t num_layers, int st
  *                width == 1
  *   width        1..16 taps;  other arguments as in ssu_decode (z, out [batch, H, Dm])
  * Both pools are indexed by state_indices; a padding row touches neither and outputs 0.
- * Two launches on `stream`: the fused conv + decode, which only reads the taps (B and C
- * channels are shared by all heads of a group), then the shift of every live row's taps.
+ * Two launches on `stream`: the fused conv + decode, which shifts the windows of the x
+ * channels (each owned by one unit of work) and only reads the B and C taps (shared by
+ * all heads of a group), then the shift of the B and C windows of every live row.
  */
 int ssu_conv_decode(const void *xbc, int x_dtype, const void *conv_weight,
                     const void *conv_bias, void *conv_state, int64_t conv_slot_stride,

@@ -17,10 +17,11 @@
 // and its group's B and C columns -- in fp32 from the old taps, then streams its state
 // tiles as the decode kernel does. Each warp takes a contiguous range of units, so that
 // consecutive units share their batch row: the row's slot index and the lane's B and C
-// conv outputs are computed once per (row, group) and reused. B and C channels are shared by all heads of a group,
-// so no unit may shift their taps while another might still read them; the shift of
-// every tap therefore runs as a second, short launch on the same stream, after the first
-// has finished (a few tens of KB per row against MBs of recurrent state).
+// conv outputs are computed once per (row, group) and reused. A unit owns its x channels
+// and advances their windows itself. B and C channels are shared by all heads of a group,
+// so no unit may shift their taps while another might still read them; their shift runs
+// as a second, short launch on the same stream after the first has finished (2*G*N
+// channels per row).
 #include "ssu_stream.cuh"
 
 namespace ssu {
@@ -44,9 +45,12 @@ struct ConvRows {
     }
 };
 
-// Conv output of channel ch of batch row b (slot's taps at tap0 = slot * cslot).
+// Conv output of channel ch of batch row b (slot's taps at tap0 = slot * cslot). With
+// `shift`, the caller owns the channel and its window is advanced here as well: in
+// ascending order tap k takes tap k+1 (read before it is overwritten), the last tap the
+// new input.
 __device__ __forceinline__ float conv_out(const ConvArgs &c, int dtype, int64_t xrow,
-                                          int64_t tap0, int64_t ch)
+                                          int64_t tap0, int64_t ch, bool shift = false)
 {
     float acc = c.bias ? ld_f32(c.bias, dtype, ch) : 0.f;
     const int64_t w0 = ch * c.width;
@@ -54,7 +58,18 @@ __device__ __forceinline__ float conv_out(const ConvArgs &c, int dtype, int64_t 
 #pragma unroll 4
     for (int k = 0; k + 1 < c.width; ++k)
         acc = fmaf(ld_f32(c.w, dtype, w0 + k), ld_f32(c.cstate, dtype, t0 + k * c.ck), acc);
-    acc = fmaf(ld_f32(c.w, dtype, w0 + c.width - 1), ld_f32(c.xbc, dtype, xrow + ch), acc);
+    const uint32_t xin = ld_bits(c.xbc, dtype, xrow + ch);
+    acc = fmaf(ld_f32(c.w, dtype, w0 + c.width - 1), bits_f32(xin, dtype), acc);
+    if (shift) {
+        for (int k = 0; k + 1 < c.width; ++k) {
+            const uint32_t v = k + 2 < c.width ? ld_bits(c.cstate, dtype, t0 + (k + 1) * c.ck)
+                                               : xin;
+            if (dtype == SSU_F32)
+                static_cast<uint32_t *>(c.cstate)[t0 + k * c.ck] = v;
+            else
+                static_cast<uint16_t *>(c.cstate)[t0 + k * c.ck] = static_cast<uint16_t>(v);
+        }
+    }
     return c.silu ? silu_f(acc) : acc;
 }
 
@@ -129,7 +144,7 @@ ssu_conv_decode_kernel(const __grid_constant__ ConvArgs ca, const int cph, const
             const int r = lane + 32 * m;
             const bool in = r < un.rows;
             xo[m] = (in && live) ? conv_out(ca, a.x_dtype, xb, tap0,
-                                            (int64_t)un.h * Dm + un.row0 + r)
+                                            (int64_t)un.h * Dm + un.row0 + r, true)
                                  : 0.f;
             zo[m] = (in && a.z) ? ld_f32(a.z, a.x_dtype, orow + r) : 0.f;
             if (r < G::CR)
@@ -212,15 +227,18 @@ ssu_conv_decode_kernel(const __grid_constant__ ConvArgs ca, const int cph, const
     }
 }
 
-// Shift the conv window of every channel of every live row by one raw input (runs after
-// the fused decode has read the old windows).
+// Shift the conv windows of the B and C channels of every live row by one raw input (runs
+// after the fused decode has read the old windows; the x channels were shifted there by
+// their owning units).
 __global__ void __launch_bounds__(256)
-conv_shift_kernel(const __grid_constant__ ConvArgs ca, const int64_t cd, const int64_t total)
+conv_shift_kernel(const __grid_constant__ ConvArgs ca, const int64_t cd, const int64_t ch0,
+                  const int64_t total)
 {
     const DecodeArgs &a = ca.d;
+    const int64_t nbc = cd - ch0;                // B and C channels per row
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t b = e / cd, ch = e % cd;
+        const int64_t b = e / nbc, ch = ch0 + e % nbc;
         const int slot = a.idx ? a.idx[b] : (int)b;
         if (slot < 0 || slot >= a.P)
             continue;
@@ -252,12 +270,13 @@ int launch_n(const ConvArgs &ca, cudaStream_t stream)
     ssu_conv_decode_kernel<S, N><<<grid, kWarps * 32, kSmemBytes, stream>>>(ca, (int)cph,
                                                                             (int)nunits);
     if (ca.width > 1) {
-        const int64_t cd = (int64_t)a.H * a.Dm + 2 * (int64_t)a.G * N;
-        const int64_t total = (int64_t)a.active * cd;
+        const int64_t ch0 = (int64_t)a.H * a.Dm;
+        const int64_t cd = ch0 + 2 * (int64_t)a.G * N;
+        const int64_t total = (int64_t)a.active * (cd - ch0);
         int64_t blocks = (total + 255) / 256;
         if (blocks > 148 * 16)
             blocks = 148 * 16;
-        conv_shift_kernel<<<(unsigned)blocks, 256, 0, stream>>>(ca, cd, total);
+        conv_shift_kernel<<<(unsigned)blocks, 256, 0, stream>>>(ca, cd, ch0, total);
     }
     return SSU_OK;
 }
