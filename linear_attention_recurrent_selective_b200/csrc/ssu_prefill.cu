@@ -66,7 +66,7 @@ template <int N> struct PGeo {
     static constexpr int R = N >= 128 ? 1 : ((128 / N) < 4 ? (128 / N) : 4);   // rows/lane
     static constexpr int RSTEP = 32 / LPR;                   // row stride inside a warp
     static constexpr int RW = RSTEP * R;                     // rows per warp
-    static constexpr int NA = SSU_PREFILL_NA;                // partial sums per row
+    static constexpr int NA = SSU_PREFILL_NA < K / 4 ? SSU_PREFILL_NA : K / 4;  // partial sums
     static_assert(K % 4 == 0 && (K / 4) % NA == 0, "prefill geometry");
 };
 
