@@ -173,11 +173,12 @@ ssu_conv_decode_kernel(const __grid_constant__ ConvArgs ca, const int cph, const
                                                  buf + r * G::ROW_BYTES + (v * G::LPR + ln) * 16)
                                            : make_uint4(0, 0, 0, 0);
                 }
+                float acc[G::RPT];
 #pragma unroll
                 for (int i = 0; i < G::RPT; ++i) {
                     const int r = i * G::RPW + sub;
                     const float dtx = r < rt ? dte * xs[j * G::RT + r] : 0.f;
-                    float acc = 0.f;
+                    acc[i] = 0.f;
 #pragma unroll
                     for (int v = 0; v < G::NV; ++v) {
                         float f[G::VEC];
@@ -186,17 +187,30 @@ ssu_conv_decode_kernel(const __grid_constant__ ConvArgs ca, const int cph, const
                         for (int e = 0; e < G::VEC; ++e) {
                             const float sn = fmaf(f[e], dA, Bn[v * G::VEC + e] * dtx);
                             f[e] = sn;
-                            acc = fmaf(sn, Cn[v * G::VEC + e], acc);
+                            acc[i] = fmaf(sn, Cn[v * G::VEC + e], acc[i]);
                         }
                         if (r < rt)
                             *reinterpret_cast<uint4 *>(dst + (int64_t)r * N + G::col(v, ln, 0)) =
                                 V::pack(f);
                     }
+                }
+                if constexpr (G::RPT <= G::LPR) {         // one transposing butterfly
+                    int i = 0;
+                    bool wr = false;
+                    const float y = row_sums<G::RPT, G::LPR>(acc, ln, i, wr);
+                    const int r = i * G::RPW + sub;
+                    if (wr && r < rt)
+                        ys[j * G::RT + r] = y;
+                } else {
 #pragma unroll
-                    for (int off = G::LPR / 2; off > 0; off >>= 1)
-                        acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                    if (ln == 0 && r < rt)
-                        ys[j * G::RT + r] = acc;
+                    for (int i0 = 0; i0 < G::RPT; ++i0) {
+                        int i = i0;
+                        bool wr = false;
+                        const float y = row_sums<G::RPT, G::LPR>(acc, ln, i, wr);
+                        const int r = i0 * G::RPW + sub;
+                        if (wr && r < rt)
+                            ys[j * G::RT + r] = y;
+                    }
                 }
             }
             __syncwarp();                        // every lane is done with buffer s

@@ -21,9 +21,11 @@
 //     instruction covers 512 contiguous bytes); the input term is formed as B * (dt * x),
 //     the association the prefill and replay kernels use too, so fp32 states agree bit
 //     for bit across the three forms;
-//   * the dstate reduction is a butterfly of warp shuffles inside each lane group; the
-//     per-row sums are collected in shared memory and the unit's outputs (skip term and
-//     gate applied) are written with one coalesced store per 32 rows.
+//   * the dstate reductions of a tile's rows share one transposing butterfly of warp
+//     shuffles inside each lane group (RPT - 1 + log2(LPR / RPT) shuffles for RPT rows
+//     instead of RPT log2(LPR)); the per-row sums are collected in shared memory and the
+//     unit's outputs (skip term and gate applied) are written with one coalesced store per
+//     32 rows.
 #include "ssu_stream.cuh"
 
 namespace ssu {
@@ -129,11 +131,12 @@ ssu_decode_kernel(const DecodeArgs a, const int cph, const int nunits)
                                                  buf + r * G::ROW_BYTES + (v * G::LPR + ln) * 16)
                                            : make_uint4(0, 0, 0, 0);
                 }
+                float acc[G::RPT];
 #pragma unroll
                 for (int i = 0; i < G::RPT; ++i) {
                     const int r = i * G::RPW + sub;
                     const float dtx = r < rt ? dte * xs[j * G::RT + r] : 0.f;
-                    float acc = 0.f;
+                    acc[i] = 0.f;
 #pragma unroll
                     for (int v = 0; v < G::NV; ++v) {
                         float f[G::VEC];
@@ -142,17 +145,31 @@ ssu_decode_kernel(const DecodeArgs a, const int cph, const int nunits)
                         for (int e = 0; e < G::VEC; ++e) {
                             const float sn = fmaf(f[e], dA, Bn[v * G::VEC + e] * dtx);
                             f[e] = sn;
-                            acc = fmaf(sn, Cn[v * G::VEC + e], acc);
+                            acc[i] = fmaf(sn, Cn[v * G::VEC + e], acc[i]);
                         }
                         if (r < rt)
                             *reinterpret_cast<uint4 *>(dst + (int64_t)r * N + G::col(v, ln, 0)) =
                                 V::pack(f);
                     }
+                }
+                // the rows' dstate sums: one transposing butterfly for the whole tile
+                if constexpr (G::RPT <= G::LPR) {
+                    int i = 0;
+                    bool wr = false;
+                    const float y = row_sums<G::RPT, G::LPR>(acc, ln, i, wr);
+                    const int r = i * G::RPW + sub;
+                    if (wr && r < rt)
+                        ys[j * G::RT + r] = y;
+                } else {
 #pragma unroll
-                    for (int off = G::LPR / 2; off > 0; off >>= 1)
-                        acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                    if (ln == 0 && r < rt)
-                        ys[j * G::RT + r] = acc;
+                    for (int i0 = 0; i0 < G::RPT; ++i0) {
+                        int i = i0;
+                        bool wr = false;
+                        const float y = row_sums<G::RPT, G::LPR>(acc, ln, i, wr);
+                        const int r = i0 * G::RPW + sub;
+                        if (wr && r < rt)
+                            ys[j * G::RT + r] = y;
+                    }
                 }
             }
             __syncwarp();                        // every lane is done with buffer s

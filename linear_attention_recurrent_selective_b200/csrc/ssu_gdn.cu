@@ -14,9 +14,11 @@
 // by HBM, so it runs on the per-warp bulk-copy pipeline of ssu_stream.cuh: units of up to
 // 64 rows of one value head, tiles of 4 KB streamed through a ring of shared-memory
 // buffers. Per unit the lane's columns of q and k are normalised with warp shuffles (every
-// lane group holds the same columns), k . q and the gates are formed once; per row the two
-// dot products S_i . k and S_i . q come from one pass over the row in registers and one
-// butterfly each, then the updated row is written straight back.
+// lane group holds the same columns), k . q and the gates are formed once; per tile the
+// dot products S_i . k and S_i . q of all rows come from one pass over the rows in
+// registers and one transposing butterfly each (ssu_stream.cuh, row_sums), the row's
+// owner lane forms d, every lane fetches d of its rows, and the updated rows are written
+// straight back.
 #include "ssu_stream.cuh"
 
 namespace ssu {
@@ -135,36 +137,65 @@ gdn_decode_kernel(const __grid_constant__ GdnArgs a, const int cph, const int nu
                 const uint8_t *buf = w.ring + s * kTileBytes;
                 float *dst = a.state + (int64_t)slot * a.slot_stride +
                              ((int64_t)un.h * Dm + un.row0 + j * G::RT) * K;
+                float f[G::RPT][G::E], pk[G::RPT], pq[G::RPT];
 #pragma unroll
                 for (int i = 0; i < G::RPT; ++i) {
                     const int r = i * G::RPW + sub;
-                    float f[G::E];
 #pragma unroll
                     for (int v = 0; v < G::NV; ++v) {
                         const uint4 q4 = r < rt ? *reinterpret_cast<const uint4 *>(
                                                       buf + r * G::ROW_BYTES + (v * G::LPR + ln) * 16)
                                                 : make_uint4(0, 0, 0, 0);
-                        Vec16<float>::unpack(q4, &f[v * G::VEC]);
+                        Vec16<float>::unpack(q4, &f[i][v * G::VEC]);
                     }
-                    float pk = 0.f, pq = 0.f;
+                    pk[i] = pq[i] = 0.f;
 #pragma unroll
                     for (int e = 0; e < G::E; ++e) {
-                        pk = fmaf(f[e], kn[e], pk);
-                        pq = fmaf(f[e], qn[e], pq);
+                        pk[i] = fmaf(f[i][e], kn[e], pk[i]);
+                        pq[i] = fmaf(f[i][e], qn[e], pq[i]);
                     }
-                    pk = group_sum<G::LPR>(pk);
-                    pq = group_sum<G::LPR>(pq);
-                    const float d = r < rt ? beta * (vs[j * G::RT + r] - alpha * pk) : 0.f;
+                }
+                // per-row d = beta (v - alpha S.k) and out = alpha S.q + d k.q
+                float d[G::RPT];
+                if constexpr (G::RPT <= G::LPR) {
+                    // transposing butterflies leave each lane one row's sums; its owner
+                    // forms d, and every lane of the row group fetches d of each row
+                    int i = 0, i2 = 0;
+                    bool wr = false, wr2 = false;
+                    const float tk = row_sums<G::RPT, G::LPR>(pk, ln, i, wr);
+                    const float tq = row_sums<G::RPT, G::LPR>(pq, ln, i2, wr2);
+                    const int r = i * G::RPW + sub;
+                    const float dm = r < rt ? beta * (vs[j * G::RT + r] - alpha * tk) : 0.f;
+                    if (wr && r < rt)
+                        ys[j * G::RT + r] = fmaf(alpha, tq, dm * kq);
+#pragma unroll
+                    for (int ii = 0; ii < G::RPT; ++ii)
+                        d[ii] = __shfl_sync(0xffffffffu, dm,
+                                            sub * G::LPR + ii * (G::LPR / G::RPT));
+                } else {
+#pragma unroll
+                    for (int ii = 0; ii < G::RPT; ++ii) {
+                        int i = ii;
+                        bool wr = false;
+                        const float tk = row_sums<G::RPT, G::LPR>(pk, ln, i, wr);
+                        const float tq = row_sums<G::RPT, G::LPR>(pq, ln, i, wr);
+                        const int r = ii * G::RPW + sub;
+                        d[ii] = r < rt ? beta * (vs[j * G::RT + r] - alpha * tk) : 0.f;
+                        if (wr && r < rt)
+                            ys[j * G::RT + r] = fmaf(alpha, tq, d[ii] * kq);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < G::RPT; ++i) {
+                    const int r = i * G::RPW + sub;
 #pragma unroll
                     for (int e = 0; e < G::E; ++e)
-                        f[e] = fmaf(alpha, f[e], d * kn[e]);
+                        f[i][e] = fmaf(alpha, f[i][e], d[i] * kn[e]);
                     if (r < rt) {
 #pragma unroll
                         for (int v = 0; v < G::NV; ++v)
                             *reinterpret_cast<uint4 *>(dst + (int64_t)r * K + G::col(v, ln, 0)) =
-                                Vec16<float>::pack(&f[v * G::VEC]);
-                        if (ln == 0)
-                            ys[j * G::RT + r] = fmaf(alpha, pq, d * kq);
+                                Vec16<float>::pack(&f[i][v * G::VEC]);
                     }
                 }
             }

@@ -185,6 +185,47 @@ template <typename G, int N, typename Rows> struct Producer {
     }
 };
 
+// Row sums of a tile. v[i] holds this lane's partial sum of its i-th row (RPT rows, each
+// spread over the LPR lanes ln = 0..LPR-1 of a row group). With RPT <= LPR the sums are
+// reduced by a transposing butterfly: at each of the first log2(RPT) steps a lane keeps
+// half of its values and sends the other half to its partner (RPT - 1 shuffles in all),
+// then plain butterfly steps finish the sum; otherwise every row takes its own butterfly.
+// Returns the full sum of row `row` of this lane; `writer` marks one lane per row.
+template <int RPT, int LPR>
+__device__ __forceinline__ float row_sums(float (&v)[RPT], int ln, int &row, bool &writer)
+{
+    if constexpr (RPT <= LPR && RPT > 1) {
+        int base = 0;
+#pragma unroll
+        for (int c = RPT, o = LPR / 2; c > 1; c >>= 1, o >>= 1) {
+            const bool hi = (ln & o) != 0;
+            const int half = c / 2;
+#pragma unroll
+            for (int k = 0; k < half; ++k) {
+                const float keep = hi ? v[k + half] : v[k];
+                const float send = hi ? v[k] : v[k + half];
+                v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+            base += hi ? half : 0;
+        }
+        float t = v[0];
+#pragma unroll
+        for (int o = LPR / RPT / 2; o > 0; o >>= 1)
+            t += __shfl_xor_sync(0xffffffffu, t, o);
+        row = base;
+        writer = (ln & (LPR / RPT - 1)) == 0;
+        return t;
+    } else {
+        // one butterfly per row; the caller asks for each row in turn through `row`
+        float t = v[row];
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1)
+            t += __shfl_xor_sync(0xffffffffu, t, o);
+        writer = ln == 0;
+        return t;
+    }
+}
+
 // Initialise the warp's ring barriers (lane 0) and make them visible to the copy engine.
 __device__ __forceinline__ void init_ring(const WarpViews &w, int lane)
 {
