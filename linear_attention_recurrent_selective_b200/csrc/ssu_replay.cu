@@ -30,10 +30,16 @@ namespace {
 using namespace stream;
 
 // Units of up to 2 tiles (8 KB): a replay touches few rows, and small units spread
-// them evenly over the warps of the grid.
-constexpr int kUT = 2;
-
-constexpr int kPre = 4;   // stashed tokens per unit held in registers
+// them evenly over the warps of the grid. Both counts can be overridden at build time
+// for tuning sweeps.
+#ifndef SSU_REPLAY_UT
+#define SSU_REPLAY_UT 2
+#endif
+#ifndef SSU_REPLAY_PRE
+#define SSU_REPLAY_PRE 4
+#endif
+constexpr int kUT = SSU_REPLAY_UT;
+constexpr int kPre = SSU_REPLAY_PRE;   // stashed tokens per unit held in registers
 
 // The lane's E columns of an fp32 [N] row, as 16-byte loads.
 template <typename G>
