@@ -322,27 +322,50 @@ __device__ void stage_nodes(const TreeArgs &ta, const TLayout &lay, uint8_t *sm,
             ta.st_dt[bi * H + u.h] = dte;
         }
     }
-    for (int e = tid; e < T * kTile; e += kThreads) {
-        const int i = e / kTile, d = e % kTile;
-        if (d < u.rows)
-            ta.st_U[(((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d] =
-                xs_at(xs, a.x_dtype, i * kXS + d);
+    if ((Dm & 3) == 0 && (reinterpret_cast<uintptr_t>(ta.st_U) & 15) == 0) {
+        // U: four rows per thread, 16-byte stores
+        for (int e = tid; e < T * (kTile / 4); e += kThreads) {
+            const int i = e / (kTile / 4), d = 4 * (e % (kTile / 4));
+            if (d < u.rows) {
+                float4 f;
+                if (a.x_dtype == SSU_F32) {
+                    f = *reinterpret_cast<const float4 *>(xs + (i * kXS + d) * 4);
+                } else {
+                    const uint2 w = *reinterpret_cast<const uint2 *>(xs + (i * kXS + d) * 2);
+                    f = make_float4(bits_f32(w.x & 0xffffu, a.x_dtype), bits_f32(w.x >> 16, a.x_dtype),
+                                    bits_f32(w.y & 0xffffu, a.x_dtype), bits_f32(w.y >> 16, a.x_dtype));
+                }
+                *reinterpret_cast<float4 *>(
+                    ta.st_U + (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d) = f;
+            }
+        }
+    } else {
+        for (int e = tid; e < T * kTile; e += kThreads) {
+            const int i = e / kTile, d = e % kTile;
+            if (d < u.rows)
+                ta.st_U[(((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d] =
+                    xs_at(xs, a.x_dtype, i * kXS + d);
+        }
     }
-    if (u.dtile == 0 && u.h % (H / G) == 0) {
-        const int64_t rows = (int64_t)T * N;
-        for (int64_t e0 = tid; e0 < rows; e0 += kThreads * kBatch) {
+    // B of the (row, group): every head of the group writes an equal share of it (the
+    // items of one row are spread over the CTAs, so no CTA carries the whole copy)
+    if (u.dtile == 0) {
+        const int hpg = H / G, hh = u.h % hpg;
+        const int64_t total = (int64_t)T * N;
+        const int64_t e0 = total * hh / hpg, e1 = total * (hh + 1) / hpg;
+        for (int64_t eb = e0 + tid; eb < e1; eb += kThreads * kBatch) {
             float v[kBatch];
 #pragma unroll
             for (int q = 0; q < kBatch; ++q) {
-                const int64_t e = e0 + q * kThreads;
-                v[q] = e < rows ? ld_f32(a.B, a.bc_dtype,
-                                         (((int64_t)u.b * T + e / N) * G + u.g) * N + e % N)
-                                : 0.f;
+                const int64_t e = eb + q * kThreads;
+                v[q] = e < e1 ? ld_f32(a.B, a.bc_dtype,
+                                       (((int64_t)u.b * T + e / N) * G + u.g) * N + e % N)
+                              : 0.f;
             }
 #pragma unroll
             for (int q = 0; q < kBatch; ++q) {
-                const int64_t e = e0 + q * kThreads;
-                if (e < rows)
+                const int64_t e = eb + q * kThreads;
+                if (e < e1)
                     ta.st_B[(((int64_t)u.b * T + e / N) * G + u.g) * N + e % N] = v[q];
             }
         }
