@@ -36,6 +36,7 @@
 // whole rows, and out = W_i a_i + P[i][d] + D x is stored without further barriers.
 #include "ssu_async.cuh"
 #include "ssu_common.cuh"
+#include "ssu_tc.cuh"
 
 namespace ssu {
 namespace {
@@ -304,13 +305,11 @@ __device__ void stage_x_plain(const TreeArgs &ta, uint8_t *xs, const Item &u)
 
 // Per-item node values and stash: dt_eff and dA of every node for head h (from the
 // prefetched dt of node threadIdx.x), U from the x tile, B once per (row, group).
-__device__ void stage_nodes(const TreeArgs &ta, const TLayout &lay, uint8_t *sm, const Item &u,
+__device__ void stage_nodes(const TreeArgs &ta, float *sdA, float *sdt, const Item &u,
                             const uint8_t *xs, float dt_mine)
 {
     const DecodeArgs &a = ta.d;
     const int T = ta.T, H = a.H, G = a.G, Dm = a.Dm, N = a.N, tid = threadIdx.x;
-    float *sdA = reinterpret_cast<float *>(sm + lay.da);
-    float *sdt = reinterpret_cast<float *>(sm + lay.dtv);
     if (tid < T) {
         const int64_t bi = (int64_t)u.b * T + tid;
         const float dte = effective_dt(dt_mine, a.dt_bias, u.h, a.softplus);
@@ -424,13 +423,14 @@ __device__ __forceinline__ void prefetch_s0(const TreeArgs &ta, const TLayout &l
 }
 
 // Issue the cp.async copies of item u's x tile (rows 16-byte aligned) into buffer xbuf.
-__device__ __forceinline__ void prefetch_x(const TreeArgs &ta, const TLayout &lay, uint8_t *sm,
+// xs_off, xbytes: the buffers' offset and size.
+__device__ __forceinline__ void prefetch_x(const TreeArgs &ta, int xs_off, int xbytes, uint8_t *sm,
                                            const Item &u, int xbuf)
 {
     const DecodeArgs &a = ta.d;
     const int T = ta.T, es_x = a.x_dtype == SSU_F32 ? 4 : 2;
     const int cpn = u.rows * es_x / 16;              // 16-byte chunks per node row
-    uint8_t *dst = sm + lay.xs + xbuf * lay.xbytes;
+    uint8_t *dst = sm + xs_off + xbuf * xbytes;
     const char *xg = static_cast<const char *>(a.x);
     for (int k = threadIdx.x; k < T * cpn; k += kThreads) {
         const int i = k / cpn, c = k % cpn;
@@ -533,7 +533,7 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
         if (u.valid(a.P)) {
             prefetch_s0<S, N>(ta, lay, sm, u);
             if (xasync)
-                prefetch_x(ta, lay, sm, u, xbuf_of(first));
+                prefetch_x(ta, lay.xs, lay.xbytes, sm, u, xbuf_of(first));
             cp_async_commit();
             dt_next = dt_of(ta, u);
         }
@@ -558,7 +558,7 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
             if (next_valid) {            // this item used no buffer: start the next one
                 prefetch_s0<S, N>(ta, lay, sm, v);
                 if (xasync)
-                    prefetch_x(ta, lay, sm, v, xbuf_of(it + 1));
+                    prefetch_x(ta, lay.xs, lay.xbytes, sm, v, xbuf_of(it + 1));
                 cp_async_commit();
                 dt_next = dt_of(ta, v);
             }
@@ -575,7 +575,8 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
             stage_x_plain(ta, xs, u);
         cp_async_wait_all();
         __syncthreads();                 // state rows and x tile have landed
-        stage_nodes(ta, lay, sm, u, xs, dt_next);
+        stage_nodes(ta, reinterpret_cast<float *>(sm + lay.da),
+                    reinterpret_cast<float *>(sm + lay.dtv), u, xs, dt_next);
         __syncthreads();                 // dt_eff and dA of every node visible
         path_coefs(lay, sm, T);
         __syncthreads();                 // path coefficients and W_i ready
@@ -599,7 +600,7 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
         if (next_valid) {
             prefetch_s0<S, N>(ta, lay, sm, v);
             if (x_mid)
-                prefetch_x(ta, lay, sm, v, xbuf_of(it + 1));
+                prefetch_x(ta, lay.xs, lay.xbytes, sm, v, xbuf_of(it + 1));
             cp_async_commit();
             dt_next = dt_of(ta, v);
         }
@@ -695,11 +696,483 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
         }
         __syncthreads();                 // every read of this item's buffers is done
         if (next_valid && xasync && !x_mid) {
-            prefetch_x(ta, lay, sm, v, 0);
+            prefetch_x(ta, lay.xs, lay.xbytes, sm, v, 0);
             cp_async_commit();
         }
     }
     cp_async_wait_all();                 // no copy outlives the CTA
+}
+
+// ---------------------------------------------------------------- tensor-core form
+//
+// With bf16 B and C and dstate 64 or 128, the dense products run on the tensor cores.
+// For item (b, h, dim tile) they form one matrix product: D[i][d] = sum_n C_i[n] s0[d][n]
+// for the 128 node slots i (rows T .. 127 of C are zero) and the tile's 64 dim rows d.
+// C is bf16, so it enters the MMA exactly; the committed state is split into bf16
+// pieces s0 = p1 + p2 + p3 (p1 = bf16(s0), p2 = bf16(s0 - p1), p3 = bf16(s0 - p1 - p2);
+// each difference is exact in fp32, and the three pieces carry 24 significant bits, the
+// fp32 significand), every product of two bf16 values is exact in the fp32 accumulator,
+// and D = C p3^T + C p2^T + C p1^T accumulates in fp32. An fp16 state needs two pieces
+// (11 significant bits), a bf16 state one. D lives in tensor memory: 128 lanes (node
+// slots) x 64 fp32 columns (dim rows).
+//
+// Per item, in order: the state rows (prefetched by cp.async during the previous item)
+// are split into the pieces in the 128-byte-swizzled operand layout; one thread issues
+// the MMAs (pieces x dstate / 16 of them) and commits them to an mbarrier; the next
+// item's copies start; meanwhile every thread forms the path sums of one node over 32
+// dim rows (thread t: node 32 (warp % 4) + lane, rows 32 (warp / 4) ..), with the path
+// coefficients w_im dt_jm (C_i . B_jm) built on the way; then each thread reads its
+// node's 32 accumulator columns from tensor memory (a warp's lanes are the TMEM lanes of
+// its quarter) and stores out = W_i D + P + D_h x. Per (row, group), C goes into the
+// operand layout by cp.async and the C_i . B_j of every path pair are computed a thread
+// per pair (C from shared memory, B from global memory, all 16-byte loads in flight).
+
+// Shared-memory layout of the tensor-core form (byte offsets from a 1024-byte aligned
+// base). npc state pieces; E bounds the path pairs as in TLayout.
+struct TcLayout {
+    int ca, sp, raw, xs, xbytes, cb, pj, pi, par, cnt, off, da, dtv, bar, tptr, total;
+    __host__ __device__ static int up16(int v) { return (v + 15) & ~15; }
+    __host__ __device__ TcLayout(int T, int N, int es_x, int es_s, int npc, int nxb)
+    {
+        const int E = T * (T + 1) / 2;
+        ca = 0;                               // C operand: N / 64 blocks of 128 x 128 B
+        sp = ca + 128 * N * 2;                // pieces: npc x N / 64 blocks of 64 x 128 B
+        raw = sp + npc * kTile * N * 2;       // state rows as stored, row-major
+        xs = raw + up16(kTile * N * es_s);
+        xbytes = up16(T * kXS * es_x);
+        cb = xs + nxb * xbytes;
+        pj = cb + up16(E * 4);
+        pi = pj + up16(E);
+        par = pi + up16(E);
+        cnt = par + up16(T * 4);
+        off = cnt + up16(T * 4);
+        da = off + up16((T + 1) * 4);
+        dtv = da + up16(T * 4);
+        bar = dtv + up16(T * 4);
+        tptr = bar + 16;
+        total = tptr + 16 + 1024;             // slack for aligning the base
+    }
+};
+
+constexpr uint32_t kTcCols = 64;              // TMEM columns: the 64 dim rows of a tile
+
+// Byte offset of 16-byte chunk c (columns 8c .. 8c + 7) of row r in a K-major operand
+// with 128-byte swizzle and `block` bytes per 64-column block.
+__device__ __forceinline__ int sw128_off(int r, int c, int block)
+{
+    return (c >> 3) * block + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+
+// Per-(row, group) tables of the tensor-core form: parents, path checks, C in the
+// operand layout, path pairs (pj: path node, pi: node) and C_i . B_j of every pair.
+template <int N>
+__device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm, int b, int g,
+                             bool reporter)
+{
+    constexpr int CPR = N / 8;                // 16-byte chunks per bf16 row
+    const DecodeArgs &a = ta.d;
+    const int T = ta.T, G = a.G, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float *cb = reinterpret_cast<float *>(sm + lay.cb);
+    uint8_t *pj = sm + lay.pj;
+    uint8_t *pi = sm + lay.pi;
+    int *par = reinterpret_cast<int *>(sm + lay.par);
+    int *cnt = reinterpret_cast<int *>(sm + lay.cnt);
+    int *off = reinterpret_cast<int *>(sm + lay.off);
+    const uint16_t *Cg = static_cast<const uint16_t *>(a.C);
+    const uint16_t *Bg = static_cast<const uint16_t *>(a.B);
+
+    for (int k = tid; k < 128 * CPR; k += kThreads) {
+        const int i = k / CPR, c = k % CPR;
+        uint8_t *dst = sm + lay.ca + sw128_off(i, c, 128 * 128);
+        if (i < T)
+            cp_async16(dst, Cg + (((int64_t)b * T + i) * G + g) * N + c * 8);
+        else
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_commit();
+    for (int i = tid; i < T; i += kThreads)
+        par[i] = ta.parents[(int64_t)b * T + i];
+    __syncthreads();
+    // every node's walk: exactly depth parent steps inside [0, T), then parent -1
+    for (int i = tid; i < T; i += kThreads) {
+        const int depth = ta.depths[(int64_t)b * T + i];
+        bool ok = depth >= 0 && depth < kMaxNodes;
+        int j = i;
+        for (int k = 0; ok && k < depth; ++k) {
+            j = par[j];
+            ok = j >= 0 && j < T;
+        }
+        ok = ok && par[j] == -1;
+        cnt[i] = ok ? depth + 1 : 0;
+        if (!ok && reporter && a.err)
+            atomicOr(a.err, SSU_FLAG_TREE);
+    }
+    __syncthreads();
+    if (warp == 0) {                          // exclusive prefix sum; off[T] = all pairs
+        int carry = 0;
+        for (int base = 0; base < T; base += 32) {
+            const int i = base + lane;
+            const int v = i < T ? cnt[i] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o)
+                    incl += t;
+            }
+            if (i < T)
+                off[i] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0)
+            off[T] = carry;
+    }
+    __syncthreads();
+    for (int i = tid; i < T; i += kThreads) {
+        const int c = cnt[i], o = off[i];
+        int j = i;
+        for (int k = 0; k < c; ++k) {
+            pj[o + k] = static_cast<uint8_t>(j);
+            pi[o + k] = static_cast<uint8_t>(i);
+            j = par[j];
+        }
+    }
+    cp_async_wait_all();                      // C rows (and the item's prefetches) landed
+    __syncthreads();
+    const int total = off[T];
+    for (int p = tid; p < total; p += kThreads) {
+        const int i = pi[p], j = pj[p];
+        const uint4 *bp = reinterpret_cast<const uint4 *>(Bg + (((int64_t)b * T + j) * G + g) * N);
+        uint4 bv[CPR];
+#pragma unroll
+        for (int c = 0; c < CPR; ++c)
+            bv[c] = __ldg(bp + c);
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < CPR; ++c) {
+            const uint4 cv = *reinterpret_cast<const uint4 *>(sm + lay.ca + sw128_off(i, c, 128 * 128));
+            float fc[8], fb[8];
+            Vec16<__nv_bfloat16>::unpack(cv, fc);
+            Vec16<__nv_bfloat16>::unpack(bv[c], fb);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                s[e & 3] = fmaf(fc[e], fb[e], s[e & 3]);
+        }
+        cb[p] = (s[0] + s[1]) + (s[2] + s[3]);
+    }
+}
+
+// Number of bf16 pieces that carry a state element exactly (fp32: to within 2^-24 of it).
+template <typename S> struct Pieces { static constexpr int n = 3; };
+template <> struct Pieces<__half> { static constexpr int n = 2; };
+template <> struct Pieces<__nv_bfloat16> { static constexpr int n = 1; };
+
+// The item's state rows (raw staging, row-major) split into bf16 pieces in the operand
+// layout; rows >= rows are zero.
+template <typename S, int N>
+__device__ void split_state(const TcLayout &lay, uint8_t *sm, int rows)
+{
+    constexpr int CPR = N / 8, NPC = Pieces<S>::n;
+    for (int e = threadIdx.x; e < kTile * CPR; e += kThreads) {
+        const int r = e / CPR, c = e % CPR;
+        float f[8];
+        if (r < rows) {
+            const uint8_t *src = sm + lay.raw + ((int64_t)r * N + c * 8) * (int)sizeof(S);
+            if constexpr (sizeof(S) == 4) {
+                Vec16<float>::unpack(*reinterpret_cast<const uint4 *>(src), f);
+                Vec16<float>::unpack(*reinterpret_cast<const uint4 *>(src + 16), f + 4);
+            } else {
+                Vec16<S>::unpack(*reinterpret_cast<const uint4 *>(src), f);
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                f[q] = 0.f;
+        }
+        const int o = sw128_off(r, c, kTile * 128);
+#pragma unroll
+        for (int p = 0; p < NPC; ++p) {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * q], f[2 * q + 1]);
+                const float2 back = __bfloat1622float2(h);
+                f[2 * q] -= back.x;            // exact: the piece is within 2^-8 of f
+                f[2 * q + 1] -= back.y;
+                memcpy(&w[q], &h, 4);
+            }
+            *reinterpret_cast<uint4 *>(sm + lay.sp + p * (kTile * N * 2) + o) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
+// Issue the cp.async copies of item u's state rows (one contiguous block) into the raw
+// staging buffer.
+template <typename S, int N>
+__device__ __forceinline__ void prefetch_raw(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm,
+                                             const Item &u)
+{
+    const DecodeArgs &a = ta.d;
+    const char *src = static_cast<const char *>(a.state) +
+                      ((int64_t)u.slot * a.slot_stride + ((int64_t)u.h * a.Dm + u.row0) * N) *
+                          (int64_t)sizeof(S);
+    const int chunks = u.rows * N * (int)sizeof(S) / 16;
+    for (int k = threadIdx.x; k < chunks; k += kThreads)
+        cp_async16(sm + lay.raw + k * 16, src + (int64_t)k * 16);
+}
+
+// 32 outputs of node i from dim row d0 of item u (fewer at the tile's ragged end).
+__device__ __forceinline__ void store_out32(const DecodeArgs &a, int64_t base, int n,
+                                            const float (&y)[32])
+{
+    if (n == 32 && a.x_dtype != SSU_F32 && (reinterpret_cast<uintptr_t>(a.out) & 15) == 0 &&
+        (base & 7) == 0) {
+        uint4 *op = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.out) + base);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            op[q] = a.x_dtype == SSU_BF16 ? Vec16<__nv_bfloat16>::pack(y + 8 * q)
+                                          : Vec16<__half>::pack(y + 8 * q);
+    } else if (n == 32 && a.x_dtype == SSU_F32 && (reinterpret_cast<uintptr_t>(a.out) & 15) == 0 &&
+               (base & 3) == 0) {
+        float4 *op = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + base);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            op[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            if (e < n)
+                st_f32(a.out, a.x_dtype, base + e, y[e]);
+    }
+}
+
+template <typename S, int N>
+__global__ void __launch_bounds__(kThreads, 1)
+ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const int64_t nitems,
+                     const int nxb, const int xasync)
+{
+    constexpr int NPC = Pieces<S>::n;
+    constexpr uint32_t kIdesc = idesc_bf16_f32(128, kTile);
+    extern __shared__ __align__(16) uint8_t sm_dyn[];
+    uint8_t *sm = sm_dyn + ((1024 - (smem_u32(sm_dyn) & 1023)) & 1023);
+    const DecodeArgs &a = ta.d;
+    const int T = ta.T, H = a.H, Dm = a.Dm;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int es_x = a.x_dtype == SSU_F32 ? 4 : 2;
+    const TcLayout lay(T, N, es_x, (int)sizeof(S), NPC, nxb);
+    const float *cb = reinterpret_cast<const float *>(sm + lay.cb);
+    const uint8_t *pj = sm + lay.pj;
+    const int *cnt = reinterpret_cast<const int *>(sm + lay.cnt);
+    const int *off = reinterpret_cast<const int *>(sm + lay.off);
+    float *sdA = reinterpret_cast<float *>(sm + lay.da);
+    float *sdt = reinterpret_cast<float *>(sm + lay.dtv);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + lay.bar);
+    uint32_t *tptr = reinterpret_cast<uint32_t *>(sm + lay.tptr);
+
+    if (warp == 0)
+        tmem_alloc(tptr, kTcCols);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tptr;
+    // this thread's node (TMEM lane) and its 32 dim rows (TMEM columns)
+    const int ni = 32 * (warp & 3) + lane, d0 = 32 * (warp >> 2);
+    const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)d0;
+    uint32_t phase = 0;
+
+    const bool x_mid = xasync && nxb == 2;
+    const int64_t first = nitems * blockIdx.x / gridDim.x;
+    const int64_t last = nitems * (blockIdx.x + 1) / gridDim.x;
+    auto xbuf_of = [&](int64_t it) { return nxb == 2 ? (int)((it - first) & 1) : 0; };
+    float dt_next = 0.f;
+    if (first < last) {
+        const Item u = item_at(ta, first, dtiles);
+        if (u.valid(a.P)) {
+            prefetch_raw<S, N>(ta, lay, sm, u);
+            if (xasync)
+                prefetch_x(ta, lay.xs, lay.xbytes, sm, u, xbuf_of(first));
+            cp_async_commit();
+            dt_next = dt_of(ta, u);
+        }
+    }
+    int cur_b = -1, cur_g = -1;
+    for (int64_t it = first; it < last; ++it) {
+        const Item u = item_at(ta, it, dtiles);
+        const bool has_next = it + 1 < last;
+        const Item v = has_next ? item_at(ta, it + 1, dtiles) : u;
+        const bool next_valid = has_next && v.valid(a.P);
+        if (!u.valid(a.P)) {
+            if (u.slot < 0) {            // padding row: zero outputs at every node
+                for (int e = tid; e < T * kTile; e += kThreads) {
+                    const int i = e / kTile, dd = e % kTile;
+                    if (dd < u.rows)
+                        st_f32(a.out, a.x_dtype,
+                               (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + dd, 0.f);
+                }
+            } else if (u.h == 0 && u.dtile == 0 && tid == 0 && a.err) {
+                atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
+            }
+            if (next_valid) {
+                prefetch_raw<S, N>(ta, lay, sm, v);
+                if (xasync)
+                    prefetch_x(ta, lay.xs, lay.xbytes, sm, v, xbuf_of(it + 1));
+                cp_async_commit();
+                dt_next = dt_of(ta, v);
+            }
+            continue;
+        }
+        uint8_t *xs = sm + lay.xs + xbuf_of(it) * lay.xbytes;
+        __syncthreads();                 // the previous item is done with shared memory
+        if (u.b != cur_b || u.g != cur_g) {
+            stage_row_tc<N>(ta, lay, sm, u.b, u.g, u.h == 0 && u.dtile == 0);
+            cur_b = u.b;
+            cur_g = u.g;
+        }
+        if (!xasync)
+            stage_x_plain(ta, xs, u);
+        cp_async_wait_all();
+        __syncthreads();                 // state rows and x tile have landed
+        split_state<S, N>(lay, sm, u.rows);
+        stage_nodes(ta, sdA, sdt, u, xs, dt_next);
+        fence_async_smem();              // operands visible to the tensor cores
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t base = smem_u32(sm);
+            uint32_t acc = 0;
+#pragma unroll 1
+            for (int p = NPC - 1; p >= 0; --p)        // smallest piece first
+                for (int kb = 0; kb < N / 64; ++kb)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = desc_k_sw128(base + lay.ca + kb * 16384 + kk * 32);
+                        const uint64_t bd = desc_k_sw128(base + lay.sp + p * (kTile * N * 2) +
+                                                         kb * (kTile * 128) + kk * 32);
+                        tc_mma_bf16(tmem, ad, bd, kIdesc, acc);
+                        acc = 1;
+                    }
+            tc_commit(bar);
+        }
+        if (next_valid) {                // raw staging consumed by the split
+            prefetch_raw<S, N>(ta, lay, sm, v);
+            if (x_mid)
+                prefetch_x(ta, lay.xs, lay.xbytes, sm, v, xbuf_of(it + 1));
+            cp_async_commit();
+            dt_next = dt_of(ta, v);
+        }
+
+        // path sums of node ni over rows d0 .. d0 + 31 while the MMAs run
+        float ps[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            ps[e] = 0.f;
+        float wi = 1.f;
+        const int cn = ni < T ? cnt[ni] : 0, o = ni < T ? off[ni] : 0;
+        for (int k = 0; k < cn; ++k) {
+            const int j = pj[o + k];
+            const float cf = wi * sdt[j] * cb[o + k];
+            wi *= sdA[j];
+            if (a.x_dtype == SSU_F32) {
+                const float4 *xr = reinterpret_cast<const float4 *>(xs + (j * kXS + d0) * 4);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 xv = xr[q];
+                    ps[4 * q] = fmaf(cf, xv.x, ps[4 * q]);
+                    ps[4 * q + 1] = fmaf(cf, xv.y, ps[4 * q + 1]);
+                    ps[4 * q + 2] = fmaf(cf, xv.z, ps[4 * q + 2]);
+                    ps[4 * q + 3] = fmaf(cf, xv.w, ps[4 * q + 3]);
+                }
+            } else {
+                const uint4 *xr = reinterpret_cast<const uint4 *>(xs + (j * kXS + d0) * 2);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float f[8];
+                    if (a.x_dtype == SSU_BF16)
+                        Vec16<__nv_bfloat16>::unpack(xr[q], f);
+                    else
+                        Vec16<__half>::unpack(xr[q], f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        ps[8 * q + e] = fmaf(cf, f[e], ps[8 * q + e]);
+                }
+            }
+        }
+        const bool ok = mbar_wait(bar, phase);
+        phase ^= 1u;
+        if (__syncthreads_or(!ok)) {     // the MMAs never completed: give up on the launch
+            if (tid == 0 && a.err)
+                atomicOr(a.err, SSU_FLAG_TIMEOUT);
+            break;
+        }
+        tc_fence_after();
+        float dv[32];
+        tmem_ld32(taddr, dv);
+        if (ni < T && d0 < u.rows) {
+            const float Dh = a.D ? a.D[u.h] : 0.f;
+            float y[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                y[e] = cn > 0 ? fmaf(wi, dv[e], ps[e]) +
+                                    Dh * xs_at(xs, a.x_dtype, ni * kXS + d0 + e)
+                              : 0.f;
+            store_out32(a, (((int64_t)u.b * T + ni) * H + u.h) * Dm + u.row0 + d0,
+                        min(32, u.rows - d0), y);
+        }
+        tc_fence_before();
+        __syncthreads();                 // every read of this item's buffers is done
+        if (next_valid && xasync && !x_mid) {
+            prefetch_x(ta, lay.xs, lay.xbytes, sm, v, 0);
+            cp_async_commit();
+        }
+    }
+    cp_async_wait_all();                 // no copy outlives the CTA
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0)
+        tmem_dealloc(tmem, kTcCols);
+}
+
+// The tensor-core form when it applies (bf16 B and C with 16-byte aligned C, dstate 64 or
+// 128, layout within the shared-memory limit); -1 otherwise.
+template <typename S, int N>
+int launch_tc(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles, int xasync,
+              int sms)
+{
+    if constexpr (N != 64 && N != 128) {
+        return -1;
+    } else {
+        if (a.d.bc_dtype != SSU_BF16 || (reinterpret_cast<uintptr_t>(a.d.C) & 15) != 0)
+            return -1;
+        const int es_x = a.d.x_dtype == SSU_F32 ? 4 : 2;
+        int nxb = 2;
+        TcLayout lay(a.T, N, es_x, (int)sizeof(S), Pieces<S>::n, nxb);
+        if (lay.total > kSmemMax) {
+            nxb = 1;
+            lay = TcLayout(a.T, N, es_x, (int)sizeof(S), Pieces<S>::n, nxb);
+        }
+        if (lay.total > kSmemMax)
+            return -1;
+        static int configured[64];
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+            dev = 0;
+        if (!configured[dev]) {
+            if (cudaFuncSetAttribute(ssu_ddtree_tc_kernel<S, N>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) !=
+                cudaSuccess)
+                return SSU_ERR_CUDA;
+            configured[dev] = 1;
+        }
+        const int64_t grid = nitems < sms ? nitems : sms;
+        ssu_ddtree_tc_kernel<S, N><<<(unsigned)grid, kThreads, lay.total, stream>>>(
+            a, dtiles, nitems, nxb, xasync);
+        return SSU_OK;
+    }
 }
 
 template <typename S, int N>
@@ -711,6 +1184,21 @@ int launch_n(const TreeArgs &a, cudaStream_t stream)
     if (nitems == 0 || a.T == 0)
         return SSU_OK;
     const int es_x = a.d.x_dtype == SSU_F32 ? 4 : 2;
+    // x rows go through cp.async when every 16-byte chunk of a tile row is aligned
+    const int xasync = (reinterpret_cast<uintptr_t>(a.d.x) & 15) == 0 &&
+                       ((int64_t)a.d.Dm * es_x) % 16 == 0;
+    static int configured[64], sms[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        dev = 0;
+    if (!sms[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        sms[dev] = n > 0 ? n : 148;
+    }
+    const int tc = launch_tc<S, N>(a, stream, nitems, dtiles, xasync, sms[dev]);
+    if (tc >= 0)
+        return tc;
     int nxb = 2;
     TLayout lay(a.T, N, es_x, (int)sizeof(S), nxb);
     if (lay.total > kSmemMax) {
@@ -719,21 +1207,11 @@ int launch_n(const TreeArgs &a, cudaStream_t stream)
     }
     if (lay.total > kSmemMax)
         return SSU_ERR_UNSUPPORTED;
-    // x rows go through cp.async when every 16-byte chunk of a tile row is aligned
-    const int xasync = (reinterpret_cast<uintptr_t>(a.d.x) & 15) == 0 &&
-                       ((int64_t)a.d.Dm * es_x) % 16 == 0;
-    static int configured[64], sms[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        dev = 0;
     if (!configured[dev]) {
         if (cudaFuncSetAttribute(ssu_ddtree_kernel<S, N>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) !=
             cudaSuccess)
             return SSU_ERR_CUDA;
-        int n = 0;
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        sms[dev] = n > 0 ? n : 148;
         configured[dev] = 1;
     }
     const int64_t grid = nitems < sms[dev] ? nitems : sms[dev];

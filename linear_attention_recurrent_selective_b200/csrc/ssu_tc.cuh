@@ -1,0 +1,126 @@
+// ssu_tc.cuh -- fifth-generation tensor cores (tcgen05) for sm_100a, inline PTX.
+//
+// What the tree verify needs of them: a tensor-memory (TMEM) accumulator allocated per
+// CTA, bf16 x bf16 -> fp32 MMAs issued by one thread from operands in shared memory,
+// completion signalled on a shared-memory mbarrier (tcgen05.commit), and the accumulator
+// read back into registers (tcgen05.ld). No cluster or multicast form is used.
+//
+// Operand layout in shared memory ("K-major, 128-byte swizzle"): a matrix of R rows and
+// K bf16 columns is stored as K/64 column blocks; in a block, row r takes 128 bytes at
+// (r / 8) * 1024 + (r % 8) * 128, and its 16-byte chunk c (columns 8c .. 8c + 7 of the
+// block) sits at chunk position c ^ (r % 8). Blocks start on 1024-byte boundaries. One
+// MMA consumes 16 columns (32 bytes of every row); the next 16 columns of a block are
+// addressed by moving the descriptor's start 32 bytes on, since the swizzle is applied
+// to the final address bits.
+#pragma once
+
+#include <stdint.h>
+
+#include "ssu_async.cuh"
+
+namespace ssu {
+
+// Shared-memory matrix descriptor of a K-major, 128-byte-swizzled bf16 operand starting
+// at shared address saddr: start address (16-byte units) in bits 0..13, leading byte
+// offset 16 (unused by swizzled K-major layouts), stride byte offset 1024 between 8-row
+// groups in bits 32..45, descriptor version 1 in bits 46..47, swizzle mode 2 (128 bytes)
+// in bits 61..63.
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr)
+{
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B (both K-major), fp32 D, shape
+// M x N: D format in bits 4..5 (1 = f32), A and B formats in bits 7..9 and 10..12
+// (1 = bf16), N / 8 in bits 17..22, M / 16 in bits 24..28.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+// D (+)= A * B^T for one K step, issued by a single thread.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every MMA this thread issued before has completed.
+__device__ __forceinline__ void tc_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Allocate ncols (a power of two >= 32) TMEM columns; the whole warp calls it and the
+// base address lands in *dst.
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(dst)), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr),
+                 "r"(ncols)
+                 : "memory");
+}
+
+// Ordering of tcgen05 operations across a thread barrier.
+__device__ __forceinline__ void tc_fence_before()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Make this thread's shared-memory writes visible to the tensor cores' operand reads.
+__device__ __forceinline__ void fence_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes
+// 32 (w % 4) .. + 31; taddr carries the lane base in bits 16..31 and the column in
+// bits 0..15). Waits for the load before returning.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+        "[%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+          "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+          "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]),
+          "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
+}  // namespace ssu
