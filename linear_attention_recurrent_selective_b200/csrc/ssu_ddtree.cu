@@ -142,6 +142,26 @@ __device__ __forceinline__ Item item_at(const TreeArgs &ta, int64_t it, int dtil
     return u;
 }
 
+// The item after u in row-major order; the slot index is loaded again only when the row
+// changes.
+__device__ __forceinline__ Item item_after(const TreeArgs &ta, const Item &u, int dtiles)
+{
+    const DecodeArgs &a = ta.d;
+    Item v = u;
+    if (++v.dtile == dtiles) {
+        v.dtile = 0;
+        if (++v.h == a.H) {
+            v.h = 0;
+            ++v.b;
+            v.slot = a.idx ? a.idx[v.b] : v.b;
+        }
+        v.g = v.h / (a.H / a.G);
+    }
+    v.row0 = v.dtile * kTile;
+    v.rows = min(kTile, a.Dm - v.row0);
+    return v;
+}
+
 // C_i . B_j over dstate: C_i from shared memory (fp32), B_j from global memory (16-byte
 // rows of the input type).
 template <int N>
@@ -277,22 +297,23 @@ __device__ void stage_row(const TreeArgs &ta, const TLayout &lay, uint8_t *sm, i
 }
 
 // x tile of item u with plain loads (x rows not 16-byte aligned): rows >= u.rows are 0.
+template <int NT>
 __device__ void stage_x_plain(const TreeArgs &ta, uint8_t *xs, const Item &u)
 {
     const DecodeArgs &a = ta.d;
     const int T = ta.T, H = a.H, Dm = a.Dm, tid = threadIdx.x;
-    for (int e0 = tid; e0 < T * kTile; e0 += kThreads * kBatch) {
+    for (int e0 = tid; e0 < T * kTile; e0 += NT * kBatch) {
         uint32_t v[kBatch];
 #pragma unroll
         for (int q = 0; q < kBatch; ++q) {
-            const int e = e0 + q * kThreads, i = e / kTile, d = e % kTile;
+            const int e = e0 + q * NT, i = e / kTile, d = e % kTile;
             v[q] = e < T * kTile && d < u.rows
                        ? ld_bits(a.x, a.x_dtype, (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d)
                        : 0u;
         }
 #pragma unroll
         for (int q = 0; q < kBatch; ++q) {
-            const int e = e0 + q * kThreads, xe = (e / kTile) * kXS + e % kTile;
+            const int e = e0 + q * NT, xe = (e / kTile) * kXS + e % kTile;
             if (e < T * kTile) {
                 if (a.x_dtype == SSU_F32)
                     reinterpret_cast<uint32_t *>(xs)[xe] = v[q];
@@ -303,27 +324,77 @@ __device__ void stage_x_plain(const TreeArgs &ta, uint8_t *xs, const Item &u)
     }
 }
 
-// Per-item node values and stash: dt_eff and dA of every node for head h (from the
-// prefetched dt of node threadIdx.x), U from the x tile, B once per (row, group).
-__device__ void stage_nodes(const TreeArgs &ta, float *sdA, float *sdt, const Item &u,
-                            const uint8_t *xs, float dt_mine)
+// Per-head scalars of an item, loaded ahead of their use.
+struct HeadVals {
+    float A, bias, D;
+};
+
+__device__ __forceinline__ HeadVals head_vals(const DecodeArgs &a, int h)
+{
+    return {a.A[h], a.dt_bias ? a.dt_bias[h] : 0.f, a.D ? a.D[h] : 0.f};
+}
+
+// dt_eff and dA of every node for the item's head (node threadIdx.x, from its prefetched
+// dt) into shared memory, and into the stash once per (row, head).
+__device__ __forceinline__ void node_values(const TreeArgs &ta, float *sdA, float *sdt,
+                                            const Item &u, float dt_mine, const HeadVals &hv)
 {
     const DecodeArgs &a = ta.d;
-    const int T = ta.T, H = a.H, G = a.G, Dm = a.Dm, N = a.N, tid = threadIdx.x;
+    const int T = ta.T, tid = threadIdx.x;
     if (tid < T) {
         const int64_t bi = (int64_t)u.b * T + tid;
-        const float dte = effective_dt(dt_mine, a.dt_bias, u.h, a.softplus);
-        const float dA = expf(a.A[u.h] * dte);
+        const float v = dt_mine + hv.bias;
+        const float dte = a.softplus ? softplus_f(v) : v;
+        const float dA = expf(hv.A * dte);
         sdA[tid] = dA;
         sdt[tid] = dte;
         if (u.dtile == 0) {
-            ta.st_dA[bi * H + u.h] = dA;
-            ta.st_dt[bi * H + u.h] = dte;
+            ta.st_dA[bi * a.H + u.h] = dA;
+            ta.st_dt[bi * a.H + u.h] = dte;
         }
     }
+}
+
+// B of the (row, group) in equal shares by the group's heads (the items of one row are
+// spread over the CTAs, so no CTA carries the whole copy).
+template <int NT>
+__device__ void stash_b(const TreeArgs &ta, const Item &u)
+{
+    const DecodeArgs &a = ta.d;
+    const int T = ta.T, H = a.H, G = a.G, N = a.N, tid = threadIdx.x;
+    if (u.dtile == 0 && tid < NT) {
+        // flat element e of the row's [T][N] block: node e / N, column e % N (32-bit
+        // arithmetic: T N <= 2^15)
+        const int hpg = H / G, hh = u.h % hpg, total = T * N;
+        const int e0 = total * hh / hpg, e1 = total * (hh + 1) / hpg;
+        const int64_t rbase = ((int64_t)u.b * T * G + u.g) * N;   // node 0 of the row
+        const int64_t rstride = (int64_t)G * N;                    // node to node
+        for (int eb = e0 + tid; eb < e1; eb += NT * kBatch) {
+            float v[kBatch];
+            int64_t at[kBatch];
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int e = eb + q * NT, i = e / N;
+                at[q] = rbase + i * rstride + (e - i * N);
+                v[q] = e < e1 ? ld_f32(a.B, a.bc_dtype, at[q]) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q)
+                if (eb + q * NT < e1)
+                    ta.st_B[at[q]] = v[q];
+        }
+    }
+}
+
+// Stash of the item: U from the x tile, then its share of B.
+template <int NT>
+__device__ void stash_ub(const TreeArgs &ta, const Item &u, const uint8_t *xs)
+{
+    const DecodeArgs &a = ta.d;
+    const int T = ta.T, H = a.H, Dm = a.Dm, tid = threadIdx.x;
     if ((Dm & 3) == 0 && (reinterpret_cast<uintptr_t>(ta.st_U) & 15) == 0) {
         // U: four rows per thread, 16-byte stores
-        for (int e = tid; e < T * (kTile / 4); e += kThreads) {
+        for (int e = tid; e < T * (kTile / 4); e += NT) {
             const int i = e / (kTile / 4), d = 4 * (e % (kTile / 4));
             if (d < u.rows) {
                 float4 f;
@@ -339,36 +410,22 @@ __device__ void stage_nodes(const TreeArgs &ta, float *sdA, float *sdt, const It
             }
         }
     } else {
-        for (int e = tid; e < T * kTile; e += kThreads) {
+        for (int e = tid; e < T * kTile; e += NT) {
             const int i = e / kTile, d = e % kTile;
             if (d < u.rows)
                 ta.st_U[(((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d] =
                     xs_at(xs, a.x_dtype, i * kXS + d);
         }
     }
-    // B of the (row, group): every head of the group writes an equal share of it (the
-    // items of one row are spread over the CTAs, so no CTA carries the whole copy)
-    if (u.dtile == 0) {
-        const int hpg = H / G, hh = u.h % hpg;
-        const int64_t total = (int64_t)T * N;
-        const int64_t e0 = total * hh / hpg, e1 = total * (hh + 1) / hpg;
-        for (int64_t eb = e0 + tid; eb < e1; eb += kThreads * kBatch) {
-            float v[kBatch];
-#pragma unroll
-            for (int q = 0; q < kBatch; ++q) {
-                const int64_t e = eb + q * kThreads;
-                v[q] = e < e1 ? ld_f32(a.B, a.bc_dtype,
-                                       (((int64_t)u.b * T + e / N) * G + u.g) * N + e % N)
-                              : 0.f;
-            }
-#pragma unroll
-            for (int q = 0; q < kBatch; ++q) {
-                const int64_t e = eb + q * kThreads;
-                if (e < e1)
-                    ta.st_B[(((int64_t)u.b * T + e / N) * G + u.g) * N + e % N] = v[q];
-            }
-        }
-    }
+    stash_b<NT>(ta, u);
+}
+
+// Node values and stash of an item (dt of node threadIdx.x prefetched).
+__device__ void stage_nodes(const TreeArgs &ta, float *sdA, float *sdt, const Item &u,
+                            const uint8_t *xs, float dt_mine)
+{
+    node_values(ta, sdA, sdt, u, dt_mine, head_vals(ta.d, u.h));
+    stash_ub<kThreads>(ta, u, xs);
 }
 
 // Path coefficients of the item's head: coef[o_i + m] = w_im * dt_jm * cb[o_i + m], W_i.
@@ -572,7 +629,7 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
             cur_g = u.g;
         }
         if (!xasync)
-            stage_x_plain(ta, xs, u);
+            stage_x_plain<kThreads>(ta, xs, u);
         cp_async_wait_all();
         __syncthreads();                 // state rows and x tile have landed
         stage_nodes(ta, reinterpret_cast<float *>(sm + lay.da),
@@ -716,16 +773,23 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
 // (11 significant bits), a bf16 state one. D lives in tensor memory: 128 lanes (node
 // slots) x 64 fp32 columns (dim rows).
 //
-// Per item, in order: the state rows (prefetched by cp.async during the previous item)
-// are split into the pieces in the 128-byte-swizzled operand layout; one thread issues
-// the MMAs (pieces x dstate / 16 of them) and commits them to an mbarrier; the next
-// item's copies start; meanwhile every thread forms the path sums of one node over 32
-// dim rows (thread t: node 32 (warp % 4) + lane, rows 32 (warp / 4) ..), with the path
-// coefficients w_im dt_jm (C_i . B_jm) built on the way; then each thread reads its
-// node's 32 accumulator columns from tensor memory (a warp's lanes are the TMEM lanes of
-// its quarter) and stores out = W_i D + P + D_h x. Per (row, group), C goes into the
+// A CTA of 16 warps takes a contiguous range of items. Per item, in order: the state
+// rows and the x tile (bulk copies issued during the previous item, each buffer on its
+// own mbarrier) are waited for; the state rows are split into the pieces in the
+// 128-byte-swizzled operand layout and the nodes' dt_eff and dA formed; thread 0 issues
+// the MMAs (pieces x dstate / 16 of them) and commits them to an mbarrier, while the
+// other threads start the next item's copies (the x rows one per thread), write the
+// stash and form the path sums, a thread per node and 16 dim rows (thread t: node
+// 32 (warp % 4) + lane, rows 16 (warp / 4) ..), with the path coefficients
+// w_im dt_jm (C_i . B_jm) built on the way; then each thread reads its node's 16
+// accumulator columns from tensor memory (a warp's lanes are the TMEM lanes of its
+// quarter), forms out = W_i D + P + D_h x and writes it over its x values in the tile,
+// which then goes out as whole 16-byte-aligned rows. Per (row, group), C goes into the
 // operand layout by cp.async and the C_i . B_j of every path pair are computed a thread
 // per pair (C from shared memory, B from global memory, all 16-byte loads in flight).
+
+constexpr int kTcThreads = 512;       // 16 warps, one CTA per SM
+constexpr uint32_t kTcCols = 64;      // TMEM columns: the 64 dim rows of a tile
 
 // Shared-memory layout of the tensor-core form (byte offsets from a 1024-byte aligned
 // base). npc state pieces; E bounds the path pairs as in TLayout.
@@ -748,13 +812,11 @@ struct TcLayout {
         off = cnt + up16(T * 4);
         da = off + up16((T + 1) * 4);
         dtv = da + up16(T * 4);
-        bar = dtv + up16(T * 4);
-        tptr = bar + 16;
+        bar = dtv + up16(T * 4);              // mbarriers: MMA, state rows, x tiles 0 / 1
+        tptr = bar + 32;
         total = tptr + 16 + 1024;             // slack for aligning the base
     }
 };
-
-constexpr uint32_t kTcCols = 64;              // TMEM columns: the 64 dim rows of a tile
 
 // Byte offset of 16-byte chunk c (columns 8c .. 8c + 7) of row r in a K-major operand
 // with 128-byte swizzle and `block` bytes per 64-column block.
@@ -781,7 +843,7 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
     const uint16_t *Cg = static_cast<const uint16_t *>(a.C);
     const uint16_t *Bg = static_cast<const uint16_t *>(a.B);
 
-    for (int k = tid; k < 128 * CPR; k += kThreads) {
+    for (int k = tid; k < 128 * CPR; k += kTcThreads) {
         const int i = k / CPR, c = k % CPR;
         uint8_t *dst = sm + lay.ca + sw128_off(i, c, 128 * 128);
         if (i < T)
@@ -790,11 +852,11 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
             *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
     cp_async_commit();
-    for (int i = tid; i < T; i += kThreads)
+    for (int i = tid; i < T; i += kTcThreads)
         par[i] = ta.parents[(int64_t)b * T + i];
     __syncthreads();
     // every node's walk: exactly depth parent steps inside [0, T), then parent -1
-    for (int i = tid; i < T; i += kThreads) {
+    for (int i = tid; i < T; i += kTcThreads) {
         const int depth = ta.depths[(int64_t)b * T + i];
         bool ok = depth >= 0 && depth < kMaxNodes;
         int j = i;
@@ -828,7 +890,7 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
             off[T] = carry;
     }
     __syncthreads();
-    for (int i = tid; i < T; i += kThreads) {
+    for (int i = tid; i < T; i += kTcThreads) {
         const int c = cnt[i], o = off[i];
         int j = i;
         for (int k = 0; k < c; ++k) {
@@ -837,10 +899,10 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
             j = par[j];
         }
     }
-    cp_async_wait_all();                      // C rows (and the item's prefetches) landed
+    cp_async_wait_all();                      // C rows landed
     __syncthreads();
     const int total = off[T];
-    for (int p = tid; p < total; p += kThreads) {
+    for (int p = tid; p < total; p += kTcThreads) {
         const int i = pi[p], j = pj[p];
         const uint4 *bp = reinterpret_cast<const uint4 *>(Bg + (((int64_t)b * T + j) * G + g) * N);
         uint4 bv[CPR];
@@ -873,11 +935,11 @@ template <typename S, int N>
 __device__ void split_state(const TcLayout &lay, uint8_t *sm, int rows)
 {
     constexpr int CPR = N / 8, NPC = Pieces<S>::n;
-    for (int e = threadIdx.x; e < kTile * CPR; e += kThreads) {
+    for (int e = threadIdx.x; e < kTile * CPR; e += kTcThreads) {
         const int r = e / CPR, c = e % CPR;
         float f[8];
         if (r < rows) {
-            const uint8_t *src = sm + lay.raw + ((int64_t)r * N + c * 8) * (int)sizeof(S);
+            const uint8_t *src = sm + lay.raw + (r * N + c * 8) * (int)sizeof(S);
             if constexpr (sizeof(S) == 4) {
                 Vec16<float>::unpack(*reinterpret_cast<const uint4 *>(src), f);
                 Vec16<float>::unpack(*reinterpret_cast<const uint4 *>(src + 16), f + 4);
@@ -907,59 +969,113 @@ __device__ void split_state(const TcLayout &lay, uint8_t *sm, int rows)
     }
 }
 
-// Issue the cp.async copies of item u's state rows (one contiguous block) into the raw
-// staging buffer.
+// Bulk (TMA) copies of an item's inputs; each buffer completes on its own mbarrier, armed
+// by one thread with the whole byte count. The state rows are one contiguous block (at most
+// four copies by the leader).
 template <typename S, int N>
-__device__ __forceinline__ void prefetch_raw(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm,
-                                             const Item &u)
+__device__ __forceinline__ void bulk_raw(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm,
+                                         const Item &u, uint64_t *bar, bool leader)
 {
+    if (!leader)
+        return;
     const DecodeArgs &a = ta.d;
     const char *src = static_cast<const char *>(a.state) +
                       ((int64_t)u.slot * a.slot_stride + ((int64_t)u.h * a.Dm + u.row0) * N) *
                           (int64_t)sizeof(S);
-    const int chunks = u.rows * N * (int)sizeof(S) / 16;
-    for (int k = threadIdx.x; k < chunks; k += kThreads)
-        cp_async16(sm + lay.raw + k * 16, src + (int64_t)k * 16);
+    const uint32_t bytes = (uint32_t)(u.rows * N * (int)sizeof(S));
+    const uint32_t part = ((bytes + 3) / 4 + 15) & ~15u;
+    mbar_arrive_expect_tx(bar, bytes);
+    for (uint32_t o = 0; o < bytes; o += part)
+        bulk_load(sm + lay.raw + o, src + o, bytes - o < part ? bytes - o : part, bar);
 }
 
-// 32 outputs of node i from dim row d0 of item u (fewer at the tile's ragged end).
-__device__ __forceinline__ void store_out32(const DecodeArgs &a, int64_t base, int n,
-                                            const float (&y)[32])
+// The x tile: one copy per node row (rows 16-byte aligned), spread over nt issuing
+// threads (this one is t; t = 0 arms the barrier).
+template <typename X>
+__device__ __forceinline__ void bulk_x(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm,
+                                       const Item &u, int xbuf, uint64_t *bar, int t, int nt)
 {
-    if (n == 32 && a.x_dtype != SSU_F32 && (reinterpret_cast<uintptr_t>(a.out) & 15) == 0 &&
-        (base & 7) == 0) {
-        uint4 *op = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.out) + base);
+    const DecodeArgs &a = ta.d;
+    const int T = ta.T;
+    constexpr int es = (int)sizeof(X);
+    const uint32_t rb = (uint32_t)(u.rows * es);
+    if (t == 0)
+        mbar_arrive_expect_tx(bar, rb * (uint32_t)T);
+    for (int i = t; i < T; i += nt)
+        bulk_load(sm + lay.xs + xbuf * lay.xbytes + i * kXS * es,
+                  static_cast<const X *>(a.x) + (((int64_t)u.b * T + i) * a.H + u.h) * a.Dm +
+                      u.row0,
+                  rb, bar);
+}
+
+// 16 consecutive x values of node i from dim row d0 of an x tile, and the same positions
+// overwritten (rounded to X).
+template <typename X>
+__device__ __forceinline__ void x_seg16(const uint8_t *xs, int i, int d0, float (&f)[16])
+{
+    constexpr int per = 16 / (int)sizeof(X);
+    const uint4 *p = reinterpret_cast<const uint4 *>(xs + (i * kXS + d0) * (int)sizeof(X));
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            op[q] = a.x_dtype == SSU_BF16 ? Vec16<__nv_bfloat16>::pack(y + 8 * q)
-                                          : Vec16<__half>::pack(y + 8 * q);
-    } else if (n == 32 && a.x_dtype == SSU_F32 && (reinterpret_cast<uintptr_t>(a.out) & 15) == 0 &&
-               (base & 3) == 0) {
-        float4 *op = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + base);
+    for (int q = 0; q < 16 / per; ++q)
+        Vec16<X>::unpack(p[q], f + per * q);
+}
+
+template <typename X>
+__device__ __forceinline__ void put_seg16(uint8_t *xs, int i, int d0, const float (&y)[16])
+{
+    constexpr int per = 16 / (int)sizeof(X);
+    uint4 *p = reinterpret_cast<uint4 *>(xs + (i * kXS + d0) * (int)sizeof(X));
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-            op[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+    for (int q = 0; q < 16 / per; ++q)
+        p[q] = Vec16<X>::pack(y + per * q);
+}
+
+// U of the item (x widened to fp32): 16 bytes of the tile per task, 16-byte stores.
+template <typename X>
+__device__ void stash_u_tc(const TreeArgs &ta, const Item &u, const uint8_t *xs)
+{
+    const DecodeArgs &a = ta.d;
+    const int T = ta.T, H = a.H, Dm = a.Dm;
+    constexpr int per = 16 / (int)sizeof(X);              // x values per task
+    if ((Dm & 3) == 0 && (reinterpret_cast<uintptr_t>(ta.st_U) & 15) == 0) {
+        for (int e = threadIdx.x; e < T * (kTile / per); e += kTcThreads) {
+            const int i = e / (kTile / per), d = per * (e % (kTile / per));
+            if (d < u.rows) {
+                float f[per];
+                Vec16<X>::unpack(*reinterpret_cast<const uint4 *>(xs + (i * kXS + d) * (int)sizeof(X)), f);
+                float *dst = ta.st_U + (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d;
+#pragma unroll
+                for (int q = 0; q < per / 4; ++q)
+                    if (d + 4 * q < u.rows)
+                        *reinterpret_cast<float4 *>(dst + 4 * q) =
+                            make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
+            }
+        }
     } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-            if (e < n)
-                st_f32(a.out, a.x_dtype, base + e, y[e]);
+        for (int e = threadIdx.x; e < T * kTile; e += kTcThreads) {
+            const int i = e / kTile, d = e % kTile;
+            if (d < u.rows)
+                ta.st_U[(((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d] =
+                    xs_at(xs, a.x_dtype, i * kXS + d);
+        }
     }
 }
 
-template <typename S, int N>
-__global__ void __launch_bounds__(kThreads, 1)
+// ocopy: out rows are 16-byte aligned, so the outputs go out through the x tile as whole
+// rows (each node's dim rows are contiguous in out); otherwise each thread stores its own.
+template <typename S, typename X, int N>
+__global__ void __launch_bounds__(kTcThreads, 1)
 ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const int64_t nitems,
-                     const int nxb, const int xasync)
+                     const int nxb, const int xasync, const int ocopy)
 {
     constexpr int NPC = Pieces<S>::n;
+    constexpr int es_x = (int)sizeof(X);
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, kTile);
     extern __shared__ __align__(16) uint8_t sm_dyn[];
     uint8_t *sm = sm_dyn + ((1024 - (smem_u32(sm_dyn) & 1023)) & 1023);
     const DecodeArgs &a = ta.d;
     const int T = ta.T, H = a.H, Dm = a.Dm;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int es_x = a.x_dtype == SSU_F32 ? 4 : 2;
     const TcLayout lay(T, N, es_x, (int)sizeof(S), NPC, nxb);
     const float *cb = reinterpret_cast<const float *>(sm + lay.cb);
     const uint8_t *pj = sm + lay.pj;
@@ -967,48 +1083,62 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
     const int *off = reinterpret_cast<const int *>(sm + lay.off);
     float *sdA = reinterpret_cast<float *>(sm + lay.da);
     float *sdt = reinterpret_cast<float *>(sm + lay.dtv);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + lay.bar);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + lay.bar);     // MMA completion
+    uint64_t *sbar = bar + 1;                                         // state rows landed
+    uint64_t *xbar = bar + 2;                                         // x tile 0 / 1 landed
     uint32_t *tptr = reinterpret_cast<uint32_t *>(sm + lay.tptr);
 
     if (warp == 0)
         tmem_alloc(tptr, kTcCols);
     if (tid == 0) {
-        mbar_init(bar, 1);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            mbar_init(bar + k, 1);
         fence_mbar_init();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tptr;
-    // this thread's node (TMEM lane) and its 32 dim rows (TMEM columns)
-    const int ni = 32 * (warp & 3) + lane, d0 = 32 * (warp >> 2);
+    // this thread's node (TMEM lane) and its 16 dim rows (TMEM columns)
+    const int ni = 32 * (warp & 3) + lane, d0 = 16 * (warp >> 2);
     const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)d0;
-    uint32_t phase = 0;
+    uint32_t phase = 0;                  // parity of the MMA barrier's next phase
+    // copies in flight (uniform): state rows, x tiles by buffer bit; parities likewise
+    uint32_t s_out = 0, x_out = 0, sph = 0, xph = 0;
 
     const bool x_mid = xasync && nxb == 2;
     const int64_t first = nitems * blockIdx.x / gridDim.x;
     const int64_t last = nitems * (blockIdx.x + 1) / gridDim.x;
     auto xbuf_of = [&](int64_t it) { return nxb == 2 ? (int)((it - first) & 1) : 0; };
-    float dt_next = 0.f;
-    if (first < last) {
-        const Item u = item_at(ta, first, dtiles);
-        if (u.valid(a.P)) {
-            prefetch_raw<S, N>(ta, lay, sm, u);
-            if (xasync)
-                prefetch_x(ta, lay.xs, lay.xbytes, sm, u, xbuf_of(first));
-            cp_async_commit();
-            dt_next = dt_of(ta, u);
-        }
+    // copies of item w: the state block by thread 0, the x rows one per thread
+    auto issue = [&](const Item &w, int64_t wit, bool with_x) {
+        const int xb = xbuf_of(wit);
+        bulk_raw<S, N>(ta, lay, sm, w, sbar, tid == 0);
+        if (with_x)
+            bulk_x<X>(ta, lay, sm, w, xb, xbar + xb, tid, kTcThreads);
+        s_out = 1;
+        if (with_x)
+            x_out |= 1u << xb;
+    };
+    Item u = item_at(ta, first < last ? first : 0, dtiles);
+    float dt_next = 0.f;                 // node tid's dt and the head's scalars, next item
+    HeadVals hv_next = {0.f, 0.f, 0.f};
+    if (first < last && u.valid(a.P)) {
+        issue(u, first, xasync);
+        dt_next = dt_of(ta, u);
+        hv_next = head_vals(a, u.h);
     }
     int cur_b = -1, cur_g = -1;
-    for (int64_t it = first; it < last; ++it) {
-        const Item u = item_at(ta, it, dtiles);
+    Item v = u;
+    for (int64_t it = first; it < last; ++it, u = v) {
         const bool has_next = it + 1 < last;
-        const Item v = has_next ? item_at(ta, it + 1, dtiles) : u;
+        if (has_next)
+            v = item_after(ta, u, dtiles);
         const bool next_valid = has_next && v.valid(a.P);
         if (!u.valid(a.P)) {
             if (u.slot < 0) {            // padding row: zero outputs at every node
-                for (int e = tid; e < T * kTile; e += kThreads) {
+                for (int e = tid; e < T * kTile; e += kTcThreads) {
                     const int i = e / kTile, dd = e % kTile;
                     if (dd < u.rows)
                         st_f32(a.out, a.x_dtype,
@@ -1017,36 +1147,51 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
             } else if (u.h == 0 && u.dtile == 0 && tid == 0 && a.err) {
                 atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
             }
-            if (next_valid) {
-                prefetch_raw<S, N>(ta, lay, sm, v);
-                if (xasync)
-                    prefetch_x(ta, lay.xs, lay.xbytes, sm, v, xbuf_of(it + 1));
-                cp_async_commit();
+            if (next_valid) {            // this item used no buffer: start the next one
+                issue(v, it + 1, xasync);
                 dt_next = dt_of(ta, v);
+                hv_next = head_vals(a, v.h);
             }
             continue;
         }
+        // (every thread passed the previous item's closing barrier)
         uint8_t *xs = sm + lay.xs + xbuf_of(it) * lay.xbytes;
-        __syncthreads();                 // the previous item is done with shared memory
         if (u.b != cur_b || u.g != cur_g) {
             stage_row_tc<N>(ta, lay, sm, u.b, u.g, u.h == 0 && u.dtile == 0);
             cur_b = u.b;
             cur_g = u.g;
         }
         if (!xasync)
-            stage_x_plain(ta, xs, u);
-        cp_async_wait_all();
-        __syncthreads();                 // state rows and x tile have landed
+            stage_x_plain<kTcThreads>(ta, xs, u);
+        bool landed = true;
+        if (s_out) {
+            landed = mbar_wait(sbar, sph);
+            sph ^= 1u;
+            s_out = 0;
+        }
+        const int xb = xbuf_of(it);
+        if ((x_out >> xb) & 1u) {
+            landed = mbar_wait(xbar + xb, (xph >> xb) & 1u) && landed;
+            xph ^= 1u << xb;
+            x_out &= ~(1u << xb);
+        }
+        if (__syncthreads_or(!landed)) { // state rows and x tile have landed
+            if (tid == 0 && a.err)
+                atomicOr(a.err, SSU_FLAG_TIMEOUT);
+            break;
+        }
+        const HeadVals hv = hv_next;
         split_state<S, N>(lay, sm, u.rows);
-        stage_nodes(ta, sdA, sdt, u, xs, dt_next);
         fence_async_smem();              // operands visible to the tensor cores
+        node_values(ta, sdA, sdt, u, dt_next, hv);
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
             const uint32_t base = smem_u32(sm);
             uint32_t acc = 0;
-#pragma unroll 1
+#pragma unroll
             for (int p = NPC - 1; p >= 0; --p)        // smallest piece first
+#pragma unroll
                 for (int kb = 0; kb < N / 64; ++kb)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
@@ -1059,17 +1204,17 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
             tc_commit(bar);
         }
         if (next_valid) {                // raw staging consumed by the split
-            prefetch_raw<S, N>(ta, lay, sm, v);
-            if (x_mid)
-                prefetch_x(ta, lay.xs, lay.xbytes, sm, v, xbuf_of(it + 1));
-            cp_async_commit();
+            issue(v, it + 1, x_mid);
             dt_next = dt_of(ta, v);
+            hv_next = head_vals(a, v.h);
         }
+        stash_u_tc<X>(ta, u, xs);
+        stash_b<kTcThreads>(ta, u);
 
-        // path sums of node ni over rows d0 .. d0 + 31 while the MMAs run
-        float ps[32];
+        // path sums of node ni over rows d0 .. d0 + 15 while the MMAs run
+        float ps[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
+        for (int e = 0; e < 16; ++e)
             ps[e] = 0.f;
         float wi = 1.f;
         const int cn = ni < T ? cnt[ni] : 0, o = ni < T ? off[ni] : 0;
@@ -1077,30 +1222,11 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
             const int j = pj[o + k];
             const float cf = wi * sdt[j] * cb[o + k];
             wi *= sdA[j];
-            if (a.x_dtype == SSU_F32) {
-                const float4 *xr = reinterpret_cast<const float4 *>(xs + (j * kXS + d0) * 4);
+            float xv[16];
+            x_seg16<X>(xs, j, d0, xv);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 xv = xr[q];
-                    ps[4 * q] = fmaf(cf, xv.x, ps[4 * q]);
-                    ps[4 * q + 1] = fmaf(cf, xv.y, ps[4 * q + 1]);
-                    ps[4 * q + 2] = fmaf(cf, xv.z, ps[4 * q + 2]);
-                    ps[4 * q + 3] = fmaf(cf, xv.w, ps[4 * q + 3]);
-                }
-            } else {
-                const uint4 *xr = reinterpret_cast<const uint4 *>(xs + (j * kXS + d0) * 2);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float f[8];
-                    if (a.x_dtype == SSU_BF16)
-                        Vec16<__nv_bfloat16>::unpack(xr[q], f);
-                    else
-                        Vec16<__half>::unpack(xr[q], f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        ps[8 * q + e] = fmaf(cf, f[e], ps[8 * q + e]);
-                }
-            }
+            for (int e = 0; e < 16; ++e)
+                ps[e] = fmaf(cf, xv[e], ps[e]);
         }
         const bool ok = mbar_wait(bar, phase);
         phase ^= 1u;
@@ -1110,27 +1236,51 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
             break;
         }
         tc_fence_after();
-        float dv[32];
-        tmem_ld32(taddr, dv);
-        if (ni < T && d0 < u.rows) {
-            const float Dh = a.D ? a.D[u.h] : 0.f;
-            float y[32];
+        float dv[16];
+        tmem_ld16(taddr, dv);
+        const bool mine = ni < T && d0 < u.rows;
+        float y[16];
+        if (mine) {
+            float xv[16];
+            x_seg16<X>(xs, ni, d0, xv);
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                y[e] = cn > 0 ? fmaf(wi, dv[e], ps[e]) +
-                                    Dh * xs_at(xs, a.x_dtype, ni * kXS + d0 + e)
-                              : 0.f;
-            store_out32(a, (((int64_t)u.b * T + ni) * H + u.h) * Dm + u.row0 + d0,
-                        min(32, u.rows - d0), y);
+            for (int e = 0; e < 16; ++e)
+                y[e] = cn > 0 ? fmaf(wi, dv[e], ps[e]) + hv.D * xv[e] : 0.f;
         }
         tc_fence_before();
+        if (ocopy) {
+            if (mine)
+                put_seg16<X>(xs, ni, d0, y);
+            fence_async_smem();          // these writes before any copy refills the tile
+            __syncthreads();             // the tile holds every output of the item
+            const int cpr = u.rows * es_x / 16;
+            X *og = static_cast<X *>(a.out);
+            for (int k = tid; k < T * cpr; k += kTcThreads) {
+                const int i = k / cpr, c = k % cpr;
+                *reinterpret_cast<uint4 *>(og + (((int64_t)u.b * T + i) * H + u.h) * Dm +
+                                           u.row0 + c * (16 / es_x)) =
+                    *reinterpret_cast<const uint4 *>(xs + i * kXS * es_x + c * 16);
+            }
+        } else if (mine) {
+            const int64_t base = (((int64_t)u.b * T + ni) * H + u.h) * Dm + u.row0 + d0;
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                if (d0 + e < u.rows)
+                    st_f32(a.out, a.x_dtype, base + e, y[e]);
+        }
         __syncthreads();                 // every read of this item's buffers is done
         if (next_valid && xasync && !x_mid) {
-            prefetch_x(ta, lay.xs, lay.xbytes, sm, v, 0);
-            cp_async_commit();
+            bulk_x<X>(ta, lay, sm, v, 0, xbar, tid, kTcThreads);
+            x_out |= 1u;
         }
     }
-    cp_async_wait_all();                 // no copy outlives the CTA
+    // no copy outlives the CTA (only a launch that gave up leaves some in flight)
+    if (s_out)
+        mbar_wait(sbar, sph);
+    for (int k = 0; k < 2; ++k)
+        if ((x_out >> k) & 1u)
+            mbar_wait(xbar + k, (xph >> k) & 1u);
+    cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0)
@@ -1139,6 +1289,38 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
 
 // The tensor-core form when it applies (bf16 B and C with 16-byte aligned C, dstate 64 or
 // 128, layout within the shared-memory limit); -1 otherwise.
+template <typename S, typename X, int N>
+int launch_tc_x(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles, int xasync,
+                int sms)
+{
+    constexpr int es_x = (int)sizeof(X);
+    int nxb = 2;
+    TcLayout lay(a.T, N, es_x, (int)sizeof(S), Pieces<S>::n, nxb);
+    if (lay.total > kSmemMax) {
+        nxb = 1;
+        lay = TcLayout(a.T, N, es_x, (int)sizeof(S), Pieces<S>::n, nxb);
+    }
+    if (lay.total > kSmemMax)
+        return -1;
+    static int configured[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        dev = 0;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(ssu_ddtree_tc_kernel<S, X, N>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) !=
+            cudaSuccess)
+            return SSU_ERR_CUDA;
+        configured[dev] = 1;
+    }
+    const int ocopy = (reinterpret_cast<uintptr_t>(a.d.out) & 15) == 0 &&
+                      ((int64_t)a.d.Dm * es_x) % 16 == 0;
+    const int64_t grid = nitems < sms ? nitems : sms;
+    ssu_ddtree_tc_kernel<S, X, N><<<(unsigned)grid, kTcThreads, lay.total, stream>>>(
+        a, dtiles, nitems, nxb, xasync, ocopy);
+    return SSU_OK;
+}
+
 template <typename S, int N>
 int launch_tc(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles, int xasync,
               int sms)
@@ -1148,30 +1330,11 @@ int launch_tc(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles
     } else {
         if (a.d.bc_dtype != SSU_BF16 || (reinterpret_cast<uintptr_t>(a.d.C) & 15) != 0)
             return -1;
-        const int es_x = a.d.x_dtype == SSU_F32 ? 4 : 2;
-        int nxb = 2;
-        TcLayout lay(a.T, N, es_x, (int)sizeof(S), Pieces<S>::n, nxb);
-        if (lay.total > kSmemMax) {
-            nxb = 1;
-            lay = TcLayout(a.T, N, es_x, (int)sizeof(S), Pieces<S>::n, nxb);
+        switch (a.d.x_dtype) {
+        case SSU_F32: return launch_tc_x<S, float, N>(a, stream, nitems, dtiles, xasync, sms);
+        case SSU_F16: return launch_tc_x<S, __half, N>(a, stream, nitems, dtiles, xasync, sms);
+        default: return launch_tc_x<S, __nv_bfloat16, N>(a, stream, nitems, dtiles, xasync, sms);
         }
-        if (lay.total > kSmemMax)
-            return -1;
-        static int configured[64];
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-            dev = 0;
-        if (!configured[dev]) {
-            if (cudaFuncSetAttribute(ssu_ddtree_tc_kernel<S, N>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) !=
-                cudaSuccess)
-                return SSU_ERR_CUDA;
-            configured[dev] = 1;
-        }
-        const int64_t grid = nitems < sms ? nitems : sms;
-        ssu_ddtree_tc_kernel<S, N><<<(unsigned)grid, kThreads, lay.total, stream>>>(
-            a, dtiles, nitems, nxb, xasync);
-        return SSU_OK;
     }
 }
 
