@@ -43,6 +43,7 @@ METRIC = "decode state-update HBM GB/s (% of B200 peak); seq-head updates/s at b
 UNIT = "seq-head updates/s"
 WORKLOAD = "mamba2_decode_b256"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 REASON_BITS = {
     0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -53,6 +54,15 @@ REASON_BITS = {
 
 
 # ----------------------------------------------------------------------------- helpers
+
+def measured_bf16_tflops():
+    """The burst bf16 GEMM rate of MEASURED_PEAKS.json (TFLOP/s), else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
 
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -538,8 +548,10 @@ def form_gdn(args, device, hbm_peak):
 def form_ddtree(args, device, hbm_peak):
     """Tree verify of one 128-node draft tree per row (batch 16, random recursive trees),
     then the replay of each row's accepted root-to-node path through acceptedNodeIds.
-    The verify is FP32-issue bound (reported against the FP32 FMA peak), the replay HBM
-    bound."""
+    With bf16 B and C the verify's dense products run on the tensor cores (three bf16
+    pieces of the fp32 state per product), so its binding roofline is HBM: the algorithmic
+    bytes take longer at the measured copy bandwidth than the tensor work at the measured
+    bf16 GEMM rate (reported beside it as "compute"). The replay is HBM bound."""
     from linear_attention_recurrent_selective_b200 import ssu
     from linear_attention_recurrent_selective_b200.workloads import make_config
 
@@ -565,16 +577,21 @@ def form_ddtree(args, device, hbm_peak):
     xb = case.x.element_size()
     vbytes = (b * H * Dm * N * 4 + 2 * b * T * H * Dm * xb + b * T * H * Dm * 4
               + b * T * G * N * (2 * case.B.element_size() + 4) + b * T * H * 12 + 2 * b * T * 4)
-    sm = torch.cuda.get_device_properties(device).multi_processor_count
-    alu_peak = sm * 128 * 2 * 1.965e9 / 1e12
+    tc_peak, tc_src = measured_bf16_tflops()
+    pieces = {torch.float32: 3, torch.float16: 2, torch.bfloat16: 1}[case.pool.dtype]
+    tc_flop = 2 * b * H * 128 * Dm * N * pieces        # the MMAs as issued (128 node slots)
+    gbs = vbytes / (ms / 1e3) / 1e9
     forms = {"ddtree": {
         "workload": "ddtree_b16_n128", "batch": b, "nodes": b * T, "path_pairs": pairs,
         "ms_per_launch": ms, "nodes_per_s": b * T / (ms / 1e3), "algorithmic_flop": flop,
-        "algorithmic_bytes": vbytes, "hbm_gbs": vbytes / (ms / 1e3) / 1e9,
-        "roofline": {"bound": "alu", "achieved": flop / (ms / 1e3) / 1e12, "peak": alu_peak,
-                     "unit": "TFLOP/s", "frac": flop / (ms / 1e3) / 1e12 / alu_peak,
-                     "traffic": None,
-                     "peak_source": "derived: SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz"}}}
+        "algorithmic_bytes": vbytes,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": gbs / hbm_peak, "traffic": None},
+        "compute": {"unit": "TFLOP/s", "algorithmic": flop / (ms / 1e3) / 1e12,
+                    "tensor_issued": tc_flop / (ms / 1e3) / 1e12, "bf16_peak": tc_peak,
+                    "bf16_peak_source": tc_src,
+                    "tensor_floor_ms": tc_flop / (tc_peak * 1e12) * 1e3,
+                    "hbm_floor_ms": vbytes / (hbm_peak * 1e9) * 1e3}}}
 
     pool = d.pool.clone()
     acc, ids = d.accepted_lengths, d.accepted_node_ids
