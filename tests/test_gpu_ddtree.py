@@ -55,6 +55,28 @@ def test_ddtree_shapes(orc, N, sdt, Dm, H, G, T, xdt, tree):
     compare_ddtree(orc, case)
 
 
+# bf16 B/C with dstate 64 or 128 take the tensor-core form (the state split into bf16
+# pieces: three for fp32, two for fp16, one for bf16); every state and x type of it, with
+# ragged dim tiles and rows whose x/out are not 16-byte aligned (Dm 33 in 16-bit types)
+TC_SHAPES = [
+    # (N, state dtype, Dm, H, G, T, x dtype, tree)
+    (128, F32, 64, 4, 1, 57, F32, "random"),
+    (64, F16, 40, 4, 2, 23, F16, "forest"),
+    (128, BF16, 70, 2, 1, 128, BF16, "random"),
+    (64, F32, 130, 2, 2, 128, F16, "shuffled"),
+    (128, F32, 33, 3, 1, 19, BF16, "chain"),
+    (64, BF16, 8, 2, 1, 9, F32, "random"),
+]
+
+
+@pytest.mark.parametrize("N,sdt,Dm,H,G,T,xdt,tree", TC_SHAPES)
+def test_ddtree_tensor_core_types(orc, N, sdt, Dm, H, G, T, xdt, tree):
+    case = make_case(seed=650 + N + T + Dm, batch=4, P=7, T=T, H=H, G=G, Dm=Dm, N=N,
+                     x_dtype=xdt, bc_dtype=BF16, state_dtype=sdt, active=3, n_pad=1,
+                     slot_pad=4 if sdt == F32 else 8, tree=tree)
+    compare_ddtree(orc, case)
+
+
 @pytest.mark.parametrize("T", [1, 2, 31, 128])
 def test_ddtree_node_counts(orc, T):
     case = make_case(seed=610 + T, batch=3, P=4, T=T, H=2, G=1, Dm=64, N=128,
