@@ -801,7 +801,8 @@ struct TcLayout {
         const int E = T * (T + 1) / 2;
         ca = 0;                               // C operand: N / 64 blocks of 128 x 128 B
         sp = ca + 128 * N * 2;                // pieces: npc x N / 64 blocks of 64 x 128 B
-        raw = sp + npc * kTile * N * 2;       // state rows as stored, row-major
+        // (between items the same bytes stage the row's B rows: 128 x N bf16)
+        raw = sp + (npc * kTile > 128 ? npc * kTile : 128) * N * 2;   // state rows as stored
         xs = raw + up16(kTile * N * es_s);
         xbytes = up16(T * kXS * es_x);
         cb = xs + nxb * xbytes;
@@ -826,7 +827,11 @@ __device__ __forceinline__ int sw128_off(int r, int c, int block)
 }
 
 // Per-(row, group) tables of the tensor-core form: parents, path checks, C in the
-// operand layout, path pairs (pj: path node, pi: node) and C_i . B_j of every pair.
+// operand layout, path pairs (pj: path node, pi: node) and C_i . B_j of every pair. All
+// of the row's loads are issued at once: C rows into the operand layout and B rows into
+// the piece buffer (free between items; 16-byte chunks XOR-swizzled by the row) by
+// cp.async, parents and depths into registers; the C . B products then read shared
+// memory only.
 template <int N>
 __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm, int b, int g,
                              bool reporter)
@@ -837,6 +842,7 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
     float *cb = reinterpret_cast<float *>(sm + lay.cb);
     uint8_t *pj = sm + lay.pj;
     uint8_t *pi = sm + lay.pi;
+    uint8_t *bst = sm + lay.sp;               // B rows of the row's nodes
     int *par = reinterpret_cast<int *>(sm + lay.par);
     int *cnt = reinterpret_cast<int *>(sm + lay.cnt);
     int *off = reinterpret_cast<int *>(sm + lay.off);
@@ -851,21 +857,28 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
         else
             *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
+    for (int k = tid; k < T * CPR; k += kTcThreads) {
+        const int j = k / CPR, c = k % CPR;
+        cp_async16(bst + j * (N * 2) + ((c ^ (j & 7)) << 4),
+                   Bg + (((int64_t)b * T + j) * G + g) * N + c * 8);
+    }
     cp_async_commit();
-    for (int i = tid; i < T; i += kTcThreads)
-        par[i] = ta.parents[(int64_t)b * T + i];
+    int depth = 0;                            // node tid's depth (T <= 128 < threads)
+    if (tid < T) {
+        par[tid] = ta.parents[(int64_t)b * T + tid];
+        depth = ta.depths[(int64_t)b * T + tid];
+    }
     __syncthreads();
     // every node's walk: exactly depth parent steps inside [0, T), then parent -1
-    for (int i = tid; i < T; i += kTcThreads) {
-        const int depth = ta.depths[(int64_t)b * T + i];
+    if (tid < T) {
         bool ok = depth >= 0 && depth < kMaxNodes;
-        int j = i;
+        int j = tid;
         for (int k = 0; ok && k < depth; ++k) {
             j = par[j];
             ok = j >= 0 && j < T;
         }
         ok = ok && par[j] == -1;
-        cnt[i] = ok ? depth + 1 : 0;
+        cnt[tid] = ok ? depth + 1 : 0;
         if (!ok && reporter && a.err)
             atomicOr(a.err, SSU_FLAG_TREE);
     }
@@ -890,32 +903,29 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
             off[T] = carry;
     }
     __syncthreads();
-    for (int i = tid; i < T; i += kTcThreads) {
-        const int c = cnt[i], o = off[i];
-        int j = i;
+    if (tid < T) {
+        const int c = cnt[tid], o = off[tid];
+        int j = tid;
         for (int k = 0; k < c; ++k) {
             pj[o + k] = static_cast<uint8_t>(j);
-            pi[o + k] = static_cast<uint8_t>(i);
+            pi[o + k] = static_cast<uint8_t>(tid);
             j = par[j];
         }
     }
-    cp_async_wait_all();                      // C rows landed
+    cp_async_wait_all();                      // C and B rows landed
     __syncthreads();
     const int total = off[T];
     for (int p = tid; p < total; p += kTcThreads) {
         const int i = pi[p], j = pj[p];
-        const uint4 *bp = reinterpret_cast<const uint4 *>(Bg + (((int64_t)b * T + j) * G + g) * N);
-        uint4 bv[CPR];
-#pragma unroll
-        for (int c = 0; c < CPR; ++c)
-            bv[c] = __ldg(bp + c);
+        const uint8_t *brow = bst + j * (N * 2);
         float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < CPR; ++c) {
             const uint4 cv = *reinterpret_cast<const uint4 *>(sm + lay.ca + sw128_off(i, c, 128 * 128));
+            const uint4 bv = *reinterpret_cast<const uint4 *>(brow + ((c ^ (j & 7)) << 4));
             float fc[8], fb[8];
             Vec16<__nv_bfloat16>::unpack(cv, fc);
-            Vec16<__nv_bfloat16>::unpack(bv[c], fb);
+            Vec16<__nv_bfloat16>::unpack(bv, fb);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
                 s[e & 3] = fmaf(fc[e], fb[e], s[e & 3]);
