@@ -1071,6 +1071,23 @@ __device__ void stash_u_tc(const TreeArgs &ta, const Item &u, const uint8_t *xs)
     }
 }
 
+// Items of this CTA. With at least as many CTAs as rows, every CTA takes a share of one
+// row's items (each CTA then builds one row's tables); otherwise contiguous ranges.
+__device__ __forceinline__ void cta_range(int64_t nitems, int64_t per_row, int rows,
+                                          int64_t &first, int64_t &last)
+{
+    const int64_t c = blockIdx.x, grid = gridDim.x;
+    if (grid >= rows && rows > 0) {
+        const int64_t r = c * rows / grid;
+        const int64_t c0 = (r * grid + rows - 1) / rows, c1 = ((r + 1) * grid + rows - 1) / rows;
+        first = r * per_row + per_row * (c - c0) / (c1 - c0);
+        last = r * per_row + per_row * (c - c0 + 1) / (c1 - c0);
+    } else {
+        first = nitems * c / grid;
+        last = nitems * (c + 1) / grid;
+    }
+}
+
 // ocopy: out rows are 16-byte aligned, so the outputs go out through the x tile as whole
 // rows (each node's dim rows are contiguous in out); otherwise each thread stores its own.
 template <typename S, typename X, int N>
@@ -1118,8 +1135,8 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
     uint32_t s_out = 0, x_out = 0, sph = 0, xph = 0;
 
     const bool x_mid = xasync && nxb == 2;
-    const int64_t first = nitems * blockIdx.x / gridDim.x;
-    const int64_t last = nitems * (blockIdx.x + 1) / gridDim.x;
+    int64_t first, last;
+    cta_range(nitems, nitems / a.active, a.active, first, last);
     auto xbuf_of = [&](int64_t it) { return nxb == 2 ? (int)((it - first) & 1) : 0; };
     // copies of item w: the state block by thread 0, the x rows one per thread
     auto issue = [&](const Item &w, int64_t wit, bool with_x) {
