@@ -831,10 +831,12 @@ __device__ __forceinline__ int sw128_off(int r, int c, int block)
 // of the row's loads are issued at once: C rows into the operand layout and B rows into
 // the piece buffer (free between items; 16-byte chunks XOR-swizzled by the row) by
 // cp.async, parents and depths into registers; the C . B products then read shared
-// memory only.
+// memory only. The staged B rows also give the stash its B: the shares of heads hh0 ..
+// hh1 (indices within the group) of this CTA's items, each head's share being elements
+// [T N hh / hpg, T N (hh + 1) / hpg) of the row's [T][N] block.
 template <int N>
 __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm, int b, int g,
-                             bool reporter)
+                             bool reporter, int hh0, int hh1)
 {
     constexpr int CPR = N / 8;                // 16-byte chunks per bf16 row
     const DecodeArgs &a = ta.d;
@@ -931,6 +933,17 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
                 s[e & 3] = fmaf(fc[e], fb[e], s[e & 3]);
         }
         cb[p] = (s[0] + s[1]) + (s[2] + s[3]);
+    }
+    if (hh0 <= hh1) {                         // stash B: this CTA's heads' shares
+        const int hpg = a.H / G, total = T * N;
+        const int e0 = total * hh0 / hpg, e1 = total * (hh1 + 1) / hpg;
+        const int64_t rbase = ((int64_t)b * T * G + g) * N;     // node 0 of the row
+        for (int e = e0 + tid; e < e1; e += kTcThreads) {
+            const int j = e / N, n = e - j * N;
+            const uint16_t bits = *reinterpret_cast<const uint16_t *>(
+                bst + j * (N * 2) + (((n >> 3) ^ (j & 7)) << 4) + (n & 7) * 2);
+            ta.st_B[rbase + (int64_t)j * G * N + n] = __uint_as_float((uint32_t)bits << 16);
+        }
     }
 }
 
@@ -1184,7 +1197,15 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
         // (every thread passed the previous item's closing barrier)
         uint8_t *xs = sm + lay.xs + xbuf_of(it) * lay.xbytes;
         if (u.b != cur_b || u.g != cur_g) {
-            stage_row_tc<N>(ta, lay, sm, u.b, u.g, u.h == 0 && u.dtile == 0);
+            // heads of (u.b, u.g) whose dim tile 0 lies in this CTA's range: their B stash
+            const int hpg = H / a.G;
+            const int64_t rs = (int64_t)u.b * H * dtiles;              // the row's item 0
+            const int64_t i0 = (first > rs ? first : rs) - rs;
+            const int64_t i1 = (last < rs + (int64_t)H * dtiles ? last : rs + (int64_t)H * dtiles) - rs;
+            const int hlo = max((int)((i0 + dtiles - 1) / dtiles), u.g * hpg);
+            const int hhi = min((int)((i1 - 1) / dtiles), (u.g + 1) * hpg - 1);
+            stage_row_tc<N>(ta, lay, sm, u.b, u.g, u.h == 0 && u.dtile == 0, hlo - u.g * hpg,
+                            hhi - u.g * hpg);
             cur_b = u.b;
             cur_g = u.g;
         }
@@ -1236,7 +1257,6 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
             hv_next = head_vals(a, v.h);
         }
         stash_u_tc<X>(ta, u, xs);
-        stash_b<kTcThreads>(ta, u);
 
         // path sums of node ni over rows d0 .. d0 + 15 while the MMAs run
         float ps[16];
