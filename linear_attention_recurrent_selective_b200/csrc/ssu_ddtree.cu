@@ -1151,12 +1151,15 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
     int64_t first, last;
     cta_range(nitems, nitems / a.active, a.active, first, last);
     auto xbuf_of = [&](int64_t it) { return nxb == 2 ? (int)((it - first) & 1) : 0; };
-    // copies of item w: the state block by thread 0, the x rows one per thread
+    // copies of item w: the state block by thread 0, the x rows one per thread from the
+    // top thread down (measured: issuing them from warps 0-3, which also issue the MMAs
+    // and hold the shallowest nodes, makes the launch 7 % slower)
+    const int xt = kTcThreads - 1 - tid;
     auto issue = [&](const Item &w, int64_t wit, bool with_x) {
         const int xb = xbuf_of(wit);
         bulk_raw<S, N>(ta, lay, sm, w, sbar, tid == 0);
         if (with_x)
-            bulk_x<X>(ta, lay, sm, w, xb, xbar + xb, tid, kTcThreads);
+            bulk_x<X>(ta, lay, sm, w, xb, xbar + xb, xt, kTcThreads);
         s_out = 1;
         if (with_x)
             x_out |= 1u << xb;
@@ -1317,7 +1320,7 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
         }
         __syncthreads();                 // every read of this item's buffers is done
         if (next_valid && xasync && !x_mid) {
-            bulk_x<X>(ta, lay, sm, v, 0, xbar, tid, kTcThreads);
+            bulk_x<X>(ta, lay, sm, v, 0, xbar, xt, kTcThreads);
             x_out |= 1u;
         }
     }
