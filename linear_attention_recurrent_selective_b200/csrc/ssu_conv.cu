@@ -30,6 +30,7 @@ namespace {
 using namespace stream;
 
 constexpr int kUT = 8;   // units of up to 8 tiles, as in the decode
+constexpr int kMaxConvWidth = 16;   // the widest window ssu_conv_decode accepts
 
 struct ConvRows {
     const void *pool;
@@ -245,26 +246,32 @@ ssu_conv_decode_kernel(const __grid_constant__ ConvArgs ca, const int cph, const
 // after the fused decode has read the old windows; the x channels were shifted there by
 // their owning units).
 __global__ void __launch_bounds__(256)
-conv_shift_kernel(const __grid_constant__ ConvArgs ca, const int64_t cd, const int64_t ch0,
-                  const int64_t total)
+conv_shift_kernel(const __grid_constant__ ConvArgs ca, const int64_t cd, const int64_t ch0)
 {
+    // block (x, y): row y, B/C channels ch0 + 256 x + threadIdx.x
     const DecodeArgs &a = ca.d;
-    const int64_t nbc = cd - ch0;                // B and C channels per row
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-         e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t b = e / nbc, ch = ch0 + e % nbc;
-        const int slot = a.idx ? a.idx[b] : (int)b;
-        if (slot < 0 || slot >= a.P)
-            continue;
-        const int64_t t0 = (int64_t)slot * ca.cslot + ch * ca.cc;
-        uint32_t prev = ld_bits(ca.xbc, a.x_dtype, b * cd + ch);
-        for (int k = ca.width - 2; k >= 0; --k) {      // newest tap first
-            const uint32_t old = ld_bits(ca.cstate, a.x_dtype, t0 + k * ca.ck);
-            if (a.x_dtype == SSU_F32)
-                static_cast<uint32_t *>(ca.cstate)[t0 + k * ca.ck] = prev;
+    const int64_t b = blockIdx.y;
+    const int64_t ch = ch0 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int slot = a.idx ? a.idx[b] : (int)b;
+    if (ch >= cd || slot < 0 || slot >= a.P)
+        return;
+    const int64_t t0 = (int64_t)slot * ca.cslot + ch * ca.cc;
+    const int W = ca.width, dty = a.x_dtype;
+    // every old tap first (registers: the loops are unrolled to the widest window), then
+    // every store: tap k takes tap k+1, the last tap the new input
+    uint32_t tap[kMaxConvWidth - 1];
+#pragma unroll
+    for (int k = 0; k < kMaxConvWidth - 1; ++k)
+        tap[k] = k + 1 < W ? ld_bits(ca.cstate, dty, t0 + k * ca.ck) : 0u;
+    const uint32_t xin = ld_bits(ca.xbc, dty, b * cd + ch);
+#pragma unroll
+    for (int k = 0; k < kMaxConvWidth - 1; ++k) {
+        if (k + 1 < W) {
+            const uint32_t v = k + 2 < W ? tap[k + 1 < kMaxConvWidth - 1 ? k + 1 : 0] : xin;
+            if (dty == SSU_F32)
+                static_cast<uint32_t *>(ca.cstate)[t0 + k * ca.ck] = v;
             else
-                static_cast<uint16_t *>(ca.cstate)[t0 + k * ca.ck] = static_cast<uint16_t>(prev);
-            prev = old;
+                static_cast<uint16_t *>(ca.cstate)[t0 + k * ca.ck] = static_cast<uint16_t>(v);
         }
     }
 }
@@ -286,11 +293,8 @@ int launch_n(const ConvArgs &ca, cudaStream_t stream)
     if (ca.width > 1) {
         const int64_t ch0 = (int64_t)a.H * a.Dm;
         const int64_t cd = ch0 + 2 * (int64_t)a.G * N;
-        const int64_t total = (int64_t)a.active * (cd - ch0);
-        int64_t blocks = (total + 255) / 256;
-        if (blocks > 148 * 16)
-            blocks = 148 * 16;
-        conv_shift_kernel<<<(unsigned)blocks, 256, 0, stream>>>(ca, cd, ch0, total);
+        const dim3 blocks((unsigned)((cd - ch0 + 255) / 256), (unsigned)a.active);
+        conv_shift_kernel<<<blocks, 256, 0, stream>>>(ca, cd, ch0);
     }
     return SSU_OK;
 }

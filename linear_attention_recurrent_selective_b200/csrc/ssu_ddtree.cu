@@ -1053,15 +1053,16 @@ __device__ __forceinline__ void put_seg16(uint8_t *xs, int i, int d0, const floa
         p[q] = Vec16<X>::pack(y + per * q);
 }
 
-// U of the item (x widened to fp32): 16 bytes of the tile per task, 16-byte stores.
+// U of the item (x widened to fp32): 16 bytes of the tile per task, 16-byte stores; thread
+// t of the nt taking part.
 template <typename X>
-__device__ void stash_u_tc(const TreeArgs &ta, const Item &u, const uint8_t *xs)
+__device__ void stash_u_tc(const TreeArgs &ta, const Item &u, const uint8_t *xs, int t, int nt)
 {
     const DecodeArgs &a = ta.d;
     const int T = ta.T, H = a.H, Dm = a.Dm;
     constexpr int per = 16 / (int)sizeof(X);              // x values per task
     if ((Dm & 3) == 0 && (reinterpret_cast<uintptr_t>(ta.st_U) & 15) == 0) {
-        for (int e = threadIdx.x; e < T * (kTile / per); e += kTcThreads) {
+        for (int e = t; e < T * (kTile / per); e += nt) {
             const int i = e / (kTile / per), d = per * (e % (kTile / per));
             if (d < u.rows) {
                 float f[per];
@@ -1075,7 +1076,7 @@ __device__ void stash_u_tc(const TreeArgs &ta, const Item &u, const uint8_t *xs)
             }
         }
     } else {
-        for (int e = threadIdx.x; e < T * kTile; e += kTcThreads) {
+        for (int e = t; e < T * kTile; e += nt) {
             const int i = e / kTile, d = e % kTile;
             if (d < u.rows)
                 ta.st_U[(((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d] =
@@ -1259,7 +1260,7 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
             dt_next = dt_of(ta, v);
             hv_next = head_vals(a, v.h);
         }
-        stash_u_tc<X>(ta, u, xs);
+        stash_u_tc<X>(ta, u, xs, tid, kTcThreads);
 
         // path sums of node ni over rows d0 .. d0 + 15 while the MMAs run
         float ps[16];
