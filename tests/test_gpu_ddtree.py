@@ -77,6 +77,15 @@ def test_ddtree_tensor_core_types(orc, N, sdt, Dm, H, G, T, xdt, tree):
     compare_ddtree(orc, case)
 
 
+def test_ddtree_more_rows_than_ctas(orc):
+    """160 rows over at most 148 CTAs: contiguous item ranges that cross rows, so a CTA
+    builds several rows' tables and a row's heads (and their B stash shares) are split
+    between CTAs; some rows are padding or out of range."""
+    case = make_case(seed=660, batch=160, P=170, T=6, H=2, G=1, Dm=16, N=64,
+                     x_dtype=BF16, bc_dtype=BF16, tree="random", n_pad=3)
+    compare_ddtree(orc, case)
+
+
 @pytest.mark.parametrize("T", [1, 2, 31, 128])
 def test_ddtree_node_counts(orc, T):
     case = make_case(seed=610 + T, batch=3, P=4, T=T, H=2, G=1, Dm=64, N=128,
