@@ -281,6 +281,10 @@ int gdn_decode(const void *q, const void *k, const void *v, int x_dtype, const v
  *   st_U [batch, T, H, Dm], st_B [batch, T, G, N], st_dt [batch, T, H], as in
  *   ssu_prefill; replay an accepted path with ssu_replay and accepted_node_ids.
  *   A padding row writes zeros to out at every node and nothing else.
+ *   With bf16 B and C (C 16-byte aligned) and dstate 64 or 128 the dense part, the dot
+ *   products of the committed state with every node's C, runs on the tensor cores with
+ *   the state split into bf16 pieces that sum to it exactly (fp32 state: to within 2^-24
+ *   of each element), so either way the outputs carry fp32 accuracy.
  * Returns SSU_ERR_SHAPE for T > 128, SSU_ERR_UNSUPPORTED when the row's tables do not fit
  * in shared memory (about T (dstate + 4) x 4 + 5 T (T + 1) + T x 64 x element bytes of x
  * bytes must stay under 227 KB: every T up to 128 for dstate <= 128).
