@@ -40,7 +40,7 @@ def test_mamba2_decode_b256(orc):
 
 
 def test_mamba2_decode_b256_fp32_output(orc):
-    # x and z widened exactly to fp32 (same values), so the output is fp32 and is judged
+    # x and z widened exactly to fp32 (same values), so the output is fp32 and is checked
     # at the fp32 tolerance; B and C stay bf16.
     case = make_config("mamba2_decode_b256", batch=64, P=128)
     case.x, case.z = case.x.float(), case.z.float()
