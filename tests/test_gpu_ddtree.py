@@ -77,11 +77,12 @@ def test_ddtree_tensor_core_types(orc, N, sdt, Dm, H, G, T, xdt, tree):
     compare_ddtree(orc, case)
 
 
-def test_ddtree_more_rows_than_ctas(orc):
+@pytest.mark.parametrize("H,G,Dm", [(2, 1, 16), (4, 2, 80), (3, 3, 64)])
+def test_ddtree_more_rows_than_ctas(orc, H, G, Dm):
     """160 rows over at most 148 CTAs: contiguous item ranges that cross rows, so a CTA
-    builds several rows' tables and a row's heads (and their B stash shares) are split
-    between CTAs; some rows are padding or out of range."""
-    case = make_case(seed=660, batch=160, P=170, T=6, H=2, G=1, Dm=16, N=64,
+    builds several rows' tables and a row's heads (and their B stash shares, by group and
+    over several dim tiles) are split between CTAs; some rows are padding."""
+    case = make_case(seed=660 + H + Dm, batch=160, P=170, T=6, H=H, G=G, Dm=Dm, N=64,
                      x_dtype=BF16, bc_dtype=BF16, tree="random", n_pad=3)
     compare_ddtree(orc, case)
 
