@@ -39,6 +39,8 @@ SHAPES = [
     (128, F32, 64, 4, 1, BF16, 4, "ds"),
     (128, F16, 40, 4, 2, F16, 1, "ds"),
     (256, F32, 36, 2, 1, F32, 4, "sd"),
+    (64, F32, 32, 2, 1, BF16, 16, "sd"),     # the widest window the ABI takes
+    (128, BF16, 64, 2, 2, F32, 8, "ds"),
 ]
 
 
