@@ -113,8 +113,10 @@ def test_ddtree_chain_matches_prefill_with_stash():
     check_fp32(out_t, out_p.double(), tol=2e-5)
 
 
-def test_ddtree_malformed_nodes_and_bad_index(orc):
-    case = make_case(seed=640, batch=4, P=6, T=10, H=2, G=1, Dm=16, N=64, tree="random")
+@pytest.mark.parametrize("bcdt", [F32, BF16])     # the CUDA-core and tensor-core forms
+def test_ddtree_malformed_nodes_and_bad_index(orc, bcdt):
+    case = make_case(seed=640, batch=4, P=6, T=10, H=2, G=1, Dm=16, N=64, tree="random",
+                     x_dtype=bcdt, bc_dtype=bcdt)
     case.depths[0, 3] += 1                           # walk runs past the root
     case.parent_ids[1, 5] = 10                       # parent outside [0, T)
     case.parent_ids[1, 7] = 7                        # self loop
