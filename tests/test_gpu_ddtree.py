@@ -94,9 +94,11 @@ def test_ddtree_node_counts(orc, T):
     compare_ddtree(orc, case)
 
 
-def test_ddtree_options_off(orc):
-    case = make_case(seed=620, batch=3, P=5, T=12, H=2, G=2, Dm=24, N=32, dt_bias=False,
-                     D=False, dt_softplus=False, tree="random", indices="none")
+@pytest.mark.parametrize("bcdt,N", [(F32, 32), (BF16, 64)])   # CUDA-core and tensor-core forms
+def test_ddtree_options_off(orc, bcdt, N):
+    case = make_case(seed=620, batch=3, P=5, T=12, H=2, G=2, Dm=24, N=N, dt_bias=False,
+                     D=False, dt_softplus=False, tree="random", indices="none",
+                     x_dtype=bcdt, bc_dtype=bcdt)
     case.dt = case.dt.abs()                          # softplus off: keep dt_eff >= 0
     compare_ddtree(orc, case)
 
