@@ -103,10 +103,12 @@ def test_ddtree_options_off(orc, bcdt, N):
     compare_ddtree(orc, case)
 
 
-def test_ddtree_chain_matches_prefill_with_stash():
+@pytest.mark.parametrize("bcdt", [F32, BF16])     # bf16 B/C: the tensor-core form, fp32 out
+def test_ddtree_chain_matches_prefill_with_stash(bcdt):
     """A chain tree evaluates the prefill's token sequence: same stash bits, outputs
     within the fp32 output tolerance of each other (different summation orders)."""
-    case = make_case(seed=630, batch=4, P=6, T=24, H=4, G=1, Dm=64, N=128, tree="chain")
+    case = make_case(seed=630, batch=4, P=6, T=24, H=4, G=1, Dm=64, N=128, tree="chain",
+                     bc_dtype=bcdt)
     out_t, _, st_t, err = gpu_run.ddtree(case)
     out_p, _, st_p, _ = gpu_run.prefill(case, stash=True)
     assert err == 0
