@@ -773,20 +773,22 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
 // (11 significant bits), a bf16 state one. D lives in tensor memory: 128 lanes (node
 // slots) x 64 fp32 columns (dim rows).
 //
-// A CTA of 16 warps takes a contiguous range of items. Per item, in order: the state
-// rows and the x tile (bulk copies issued during the previous item, each buffer on its
-// own mbarrier) are waited for; the state rows are split into the pieces in the
+// A CTA of 16 warps takes a share of one row's items when there are at least as many
+// CTAs as rows, else a contiguous range of items. Per item, in order: the state rows and
+// the x tile (bulk copies issued during the previous item, each buffer on its own
+// mbarrier) are waited for; the state rows are split into the pieces in the
 // 128-byte-swizzled operand layout and the nodes' dt_eff and dA formed; thread 0 issues
 // the MMAs (pieces x dstate / 16 of them) and commits them to an mbarrier, while the
 // other threads start the next item's copies (the x rows one per thread), write the
-// stash and form the path sums, a thread per node and 16 dim rows (thread t: node
+// stash's U and form the path sums, a thread per node and 16 dim rows (thread t: node
 // 32 (warp % 4) + lane, rows 16 (warp / 4) ..), with the path coefficients
 // w_im dt_jm (C_i . B_jm) built on the way; then each thread reads its node's 16
 // accumulator columns from tensor memory (a warp's lanes are the TMEM lanes of its
 // quarter), forms out = W_i D + P + D_h x and writes it over its x values in the tile,
-// which then goes out as whole 16-byte-aligned rows. Per (row, group), C goes into the
-// operand layout by cp.async and the C_i . B_j of every path pair are computed a thread
-// per pair (C from shared memory, B from global memory, all 16-byte loads in flight).
+// which then goes out as whole 16-byte-aligned rows. Per (row, group) the row's tables
+// are built once in the CTA (see stage_row_tc): C in the operand layout, the path pairs
+// and their C_i . B_j from the row's B rows staged in shared memory, which also give
+// the stash its B.
 
 constexpr int kTcThreads = 512;       // 16 warps, one CTA per SM
 constexpr uint32_t kTcCols = 64;      // TMEM columns: the 64 dim rows of a tile
