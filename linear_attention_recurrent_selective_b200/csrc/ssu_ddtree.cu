@@ -18,6 +18,10 @@
 // step without its state write); the path sums cost (path length) x (dim + dstate). No
 // node's state is ever formed and nothing is written to the pool.
 //
+// Two forms share the tables and the stash: with bf16 B and C and dstate 64 or 128 the
+// dense products run on the tcgen05 tensor cores (the tensor-core form further down);
+// for every other type the CUDA-core form described here runs.
+//
 // Work items are (row, head, 64-row dim tile), row-major. A persistent CTA of 8 warps
 // takes a contiguous range of items, so consecutive items share their row's tree and its
 // C . B products, built once per (row, group) in shared memory:
