@@ -18,7 +18,7 @@
 // step without its state write); the path sums cost (path length) x (dim + dstate). No
 // node's state is ever formed and nothing is written to the pool.
 //
-// Two forms share the tables and the stash: with bf16 B and C and dstate 64 or 128 the
+// Two forms compute the same outputs and stash: with bf16 B and C and dstate 64 or 128 the
 // dense products run on the tcgen05 tensor cores (the tensor-core form further down);
 // for every other type the CUDA-core form described here runs.
 //
