@@ -1325,7 +1325,12 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
                 if (d0 + e < u.rows)
                     st_f32(a.out, a.x_dtype, base + e, y[e]);
         }
-        __syncthreads();                 // every read of this item's buffers is done
+        // Every read of this item's buffers done. Not needed when the x tile is double-
+        // buffered and the next item is valid: until the next item's first barrier a
+        // thread writes only buffers the output copy-out does not read (the row's tables,
+        // the piece buffer), and this item's x tile is refilled only after that barrier.
+        if (!(x_mid && next_valid))
+            __syncthreads();
         if (next_valid && xasync && !x_mid) {
             bulk_x<X>(ta, lay, sm, v, 0, xbar, xt, kTcThreads);
             x_out |= 1u;
