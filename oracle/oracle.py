@@ -30,7 +30,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
         tmp = LIB + ".tmp"
         subprocess.run(
-            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-Wall", "-Wextra",
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-Wall", "-Wextra", "-fopenmp",
              "-fno-fast-math", "-ffp-contract=off", "-o", tmp, SRC, "-lm"],
             check=True,
         )
@@ -76,6 +76,10 @@ def lib():
         L.oracle_double_to_f16.restype = ctypes.c_uint16
         L.oracle_double_to_bf16.argtypes = [ctypes.c_double]
         L.oracle_double_to_bf16.restype = ctypes.c_uint16
+        L.oracle_set_threads.argtypes = [i]
+        L.oracle_set_threads.restype = None
+        L.oracle_max_threads.restype = ctypes.c_int
+        L.oracle_host_cores.restype = ctypes.c_int
         for f in ("oracle_decode", "oracle_prefill", "oracle_replay",
                   "oracle_clear_slot", "oracle_copy_slot", "oracle_replay_layers",
                   "oracle_clear_slot_layers", "oracle_gather_scatter", "oracle_ddtree",
@@ -83,6 +87,21 @@ def lib():
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
+
+
+def set_threads(n: int) -> int:
+    """Run the oracle's independent (row, head) units on n OpenMP threads (n <= 0: every
+    host core). Results do not depend on n. Returns the thread count now in effect."""
+    lib().oracle_set_threads(int(n))
+    return lib().oracle_max_threads()
+
+
+def threads() -> int:
+    return lib().oracle_max_threads()
+
+
+def host_cores() -> int:
+    return lib().oracle_host_cores()
 
 
 def _p(t):

@@ -18,6 +18,9 @@
  * Everything is computed in double. Inputs are decoded exactly from their storage type;
  * the pool is read in its storage type and the final state is rounded once (to nearest,
  * ties to even) when it is stored back. Outputs are returned unrounded, in double.
+ * The (row, head) units of a call are independent (each owns its state block, outputs
+ * and stash entries), so they run in parallel on OpenMP threads; the arithmetic of one
+ * unit is the same sequential loop whatever the thread count.
  *
  * Readings taken where the pages leave a point open:
  *   - head h uses group g = h / (H / G) (contiguous blocks of heads per group);
@@ -34,6 +37,7 @@
  *     64 = malformed tree input (see the tree verify below).
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -203,44 +207,47 @@ int oracle_decode(const void *x, int x_dt, const float *A,
     if (check_common(batch, active, H, G, Dm, N, slot_stride))
         return 2;
     int32_t err = 0;
-    int heads_per_group = H / G;
-    double *snew = malloc(sizeof(double) * (size_t)N);
-    for (int32_t b = 0; b < active; ++b) {
+    const int heads_per_group = H / G;
+    const int64_t units = (int64_t)active * H;
+    /* every (row, head) unit owns its state block and its output rows */
+#pragma omp parallel for schedule(dynamic, 1) reduction(|:err)
+    for (int64_t u = 0; u < units; ++u) {
+        const int32_t b = (int32_t)(u / H);
+        const int h = (int)(u % H);
         int64_t s = resolve_slot(state_indices, b, P, &err);
         if (s == -1) {                       /* padding row: output zero, no state */
-            for (int64_t i = 0; i < (int64_t)H * Dm; ++i)
-                out[(int64_t)b * H * Dm + i] = 0.0;
+            for (int d = 0; d < Dm; ++d)
+                out[((int64_t)b * H + h) * Dm + d] = 0.0;
             continue;
         }
         if (s < 0)
             continue;
-        for (int h = 0; h < H; ++h) {
-            int g = h / heads_per_group;
-            double dte = effective_dt(dt[(int64_t)b * H + h], dt_bias, h, dt_softplus);
-            double decay = exp((double)A[h] * dte);
-            for (int d = 0; d < Dm; ++d) {
-                int64_t xi = ((int64_t)b * H + h) * Dm + d;
-                double xv = load(x, x_dt, xi);
-                double y = 0.0;
-                for (int n = 0; n < N; ++n) {
-                    int64_t si = s * slot_stride + ((int64_t)h * Dm + d) * N + n;
-                    int64_t bi = ((int64_t)b * G + g) * N + n;
-                    snew[n] = load(pool, state_dt, si) * decay
-                              + load(B, bc_dt, bi) * dte * xv;
-                    y += snew[n] * load(C, bc_dt, bi);
-                }
-                for (int n = 0; n < N; ++n)
-                    store(pool, state_dt, s * slot_stride + ((int64_t)h * Dm + d) * N + n,
-                          snew[n]);
-                if (D)
-                    y += (double)D[h] * xv;
-                if (z)
-                    y *= silu(load(z, x_dt, xi));
-                out[xi] = y;
+        double *snew = malloc(sizeof(double) * (size_t)N);
+        int g = h / heads_per_group;
+        double dte = effective_dt(dt[(int64_t)b * H + h], dt_bias, h, dt_softplus);
+        double decay = exp((double)A[h] * dte);
+        for (int d = 0; d < Dm; ++d) {
+            int64_t xi = ((int64_t)b * H + h) * Dm + d;
+            double xv = load(x, x_dt, xi);
+            double y = 0.0;
+            for (int n = 0; n < N; ++n) {
+                int64_t si = s * slot_stride + ((int64_t)h * Dm + d) * N + n;
+                int64_t bi = ((int64_t)b * G + g) * N + n;
+                snew[n] = load(pool, state_dt, si) * decay
+                          + load(B, bc_dt, bi) * dte * xv;
+                y += snew[n] * load(C, bc_dt, bi);
             }
+            for (int n = 0; n < N; ++n)
+                store(pool, state_dt, s * slot_stride + ((int64_t)h * Dm + d) * N + n,
+                      snew[n]);
+            if (D)
+                y += (double)D[h] * xv;
+            if (z)
+                y *= silu(load(z, x_dt, xi));
+            out[xi] = y;
         }
+        free(snew);
     }
-    free(snew);
     if (err_flags)
         *err_flags |= err;
     return 0;
@@ -275,13 +282,19 @@ int oracle_prefill(const void *x, int x_dt, const float *A,
         return 1;
     int stash = given == 4;
     int32_t err = 0;
-    int heads_per_group = H / G;
-    double *S = malloc(sizeof(double) * (size_t)Dm * N);
-    for (int32_t b = 0; b < active; ++b) {
+    const int heads_per_group = H / G;
+    const int64_t units = (int64_t)active * H;
+    /* every (row, head) unit owns its state block, output rows and stash entries (the
+     * stash's B of a group is written by the group's first head) */
+#pragma omp parallel for schedule(dynamic, 1) reduction(|:err)
+    for (int64_t u = 0; u < units; ++u) {
+        const int32_t b = (int32_t)(u / H);
+        const int h = (int)(u % H);
         int64_t s = resolve_slot(state_indices, b, P, &err);
         if (s == -1) {                       /* padding row: every position outputs 0 */
-            for (int64_t i = 0; i < (int64_t)T * H * Dm; ++i)
-                out[(int64_t)b * T * H * Dm + i] = 0.0;
+            for (int32_t t = 0; t < T; ++t)
+                for (int d = 0; d < Dm; ++d)
+                    out[(((int64_t)b * T + t) * H + h) * Dm + d] = 0.0;
             continue;
         }
         if (s < 0)
@@ -297,45 +310,45 @@ int oracle_prefill(const void *x, int x_dt, const float *A,
         }
         if (L == 0)
             continue;
-        for (int h = 0; h < H; ++h) {
-            int g = h / heads_per_group;
-            for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
-                S[i] = load(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i);
-            for (int32_t t = 0; t < L; ++t) {
-                int64_t bt = (int64_t)b * T + t;
-                double dte = effective_dt(dt[bt * H + h], dt_bias, h, dt_softplus);
-                double decay = exp((double)A[h] * dte);
-                if (stash) {
-                    st_DA[bt * H + h] = (float)decay;
-                    st_DT[bt * H + h] = (float)dte;
+        int g = h / heads_per_group;
+        double *S = malloc(sizeof(double) * (size_t)Dm * N);
+        for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
+            S[i] = load(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i);
+        for (int32_t t = 0; t < L; ++t) {
+            int64_t bt = (int64_t)b * T + t;
+            double dte = effective_dt(dt[bt * H + h], dt_bias, h, dt_softplus);
+            double decay = exp((double)A[h] * dte);
+            if (stash) {
+                st_DA[bt * H + h] = (float)decay;
+                st_DT[bt * H + h] = (float)dte;
+                if (h % heads_per_group == 0)
                     for (int n = 0; n < N; ++n)
                         st_B[(bt * G + g) * N + n] = (float)load(B, bc_dt, (bt * G + g) * N + n);
-                }
-                for (int d = 0; d < Dm; ++d) {
-                    int64_t xi = (bt * H + h) * Dm + d;
-                    double xv = load(x, x_dt, xi);
-                    if (stash)
-                        st_U[xi] = (float)xv;
-                    double y = 0.0;
-                    for (int n = 0; n < N; ++n) {
-                        int64_t bi = (bt * G + g) * N + n;
-                        double *sp = &S[(int64_t)d * N + n];
-                        *sp = *sp * decay + load(B, bc_dt, bi) * dte * xv;
-                        y += *sp * load(C, bc_dt, bi);
-                    }
-                    if (D)
-                        y += (double)D[h] * xv;
-                    if (z)
-                        y *= silu(load(z, x_dt, xi));
-                    out[xi] = y;
-                }
             }
-            if (!stash)
-                for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
-                    store(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i, S[i]);
+            for (int d = 0; d < Dm; ++d) {
+                int64_t xi = (bt * H + h) * Dm + d;
+                double xv = load(x, x_dt, xi);
+                if (stash)
+                    st_U[xi] = (float)xv;
+                double y = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    int64_t bi = (bt * G + g) * N + n;
+                    double *sp = &S[(int64_t)d * N + n];
+                    *sp = *sp * decay + load(B, bc_dt, bi) * dte * xv;
+                    y += *sp * load(C, bc_dt, bi);
+                }
+                if (D)
+                    y += (double)D[h] * xv;
+                if (z)
+                    y *= silu(load(z, x_dt, xi));
+                out[xi] = y;
+            }
         }
+        if (!stash)
+            for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
+                store(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i, S[i]);
+        free(S);
     }
-    free(S);
     if (err_flags)
         *err_flags |= err;
     return 0;
@@ -368,9 +381,13 @@ int oracle_replay(void *pool, int state_dt, int64_t slot_stride, int32_t P,
         return 2;
     const int32_t bound = node_ids ? max_accept_len : T;
     int32_t err = 0;
-    int heads_per_group = H / G;
-    double *S = malloc(sizeof(double) * (size_t)Dm * N);
-    for (int32_t b = 0; b < active; ++b) {
+    const int heads_per_group = H / G;
+    const int64_t units = (int64_t)active * H;
+    /* every (row, head) unit owns its state block */
+#pragma omp parallel for schedule(dynamic, 1) reduction(|:err)
+    for (int64_t u = 0; u < units; ++u) {
+        const int32_t b = (int32_t)(u / H);
+        const int h = (int)(u % H);
         int64_t s = resolve_slot(state_indices, b, P, &err);
         if (s < 0)
             continue;                        /* padding row or bad index: no state */
@@ -395,28 +412,27 @@ int oracle_replay(void *pool, int state_dt, int64_t slot_stride, int32_t P,
         }
         if (k == 0)
             continue;
-        for (int h = 0; h < H; ++h) {
-            int g = h / heads_per_group;
-            for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
-                S[i] = load(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i);
-            for (int32_t t = 0; t < k; ++t) {
-                int32_t e = node_ids ? node_ids[(int64_t)b * max_accept_len + t] : t;
-                int64_t bt = (int64_t)b * T + e;
-                double decay = st_DA[bt * H + h];
-                double dte = st_DT[bt * H + h];
-                for (int d = 0; d < Dm; ++d) {
-                    double u = st_U[(bt * H + h) * Dm + d];
-                    for (int n = 0; n < N; ++n) {
-                        double *sp = &S[(int64_t)d * N + n];
-                        *sp = *sp * decay + (double)st_B[(bt * G + g) * N + n] * dte * u;
-                    }
+        int g = h / heads_per_group;
+        double *S = malloc(sizeof(double) * (size_t)Dm * N);
+        for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
+            S[i] = load(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i);
+        for (int32_t t = 0; t < k; ++t) {
+            int32_t e = node_ids ? node_ids[(int64_t)b * max_accept_len + t] : t;
+            int64_t bt = (int64_t)b * T + e;
+            double decay = st_DA[bt * H + h];
+            double dte = st_DT[bt * H + h];
+            for (int d = 0; d < Dm; ++d) {
+                double uv = st_U[(bt * H + h) * Dm + d];
+                for (int n = 0; n < N; ++n) {
+                    double *sp = &S[(int64_t)d * N + n];
+                    *sp = *sp * decay + (double)st_B[(bt * G + g) * N + n] * dte * uv;
                 }
             }
-            for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
-                store(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i, S[i]);
         }
+        for (int64_t i = 0; i < (int64_t)Dm * N; ++i)
+            store(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + i, S[i]);
+        free(S);
     }
-    free(S);
     if (err_flags)
         *err_flags |= err;
     return 0;
@@ -454,32 +470,38 @@ int oracle_ddtree(const void *x, int x_dt, const float *A, const void *B, const 
     if (check_common(batch, active, H, G, Dm, N, slot_stride) || T < 0 || T > 128)
         return 2;
     int32_t err = 0;
-    int heads_per_group = H / G;
-    double *S = malloc(sizeof(double) * (size_t)Dm * N);
-    int32_t path[128];
-    for (int32_t b = 0; b < active; ++b) {
+    const int heads_per_group = H / G;
+    const int64_t units = (int64_t)active * H;
+    /* every (row, head) unit owns its output rows and stash entries (the stash's B of a
+     * group is written by the group's first head); the pool is only read */
+#pragma omp parallel for schedule(dynamic, 1) reduction(|:err)
+    for (int64_t u = 0; u < units; ++u) {
+        const int32_t b = (int32_t)(u / H);
+        const int h = (int)(u % H);
         int64_t s = resolve_slot(state_indices, b, P, &err);
         if (s == -1) {                       /* padding row: every node outputs 0 */
-            for (int64_t i = 0; i < (int64_t)T * H * Dm; ++i)
-                out[(int64_t)b * T * H * Dm + i] = 0.0;
+            for (int32_t i = 0; i < T; ++i)
+                for (int d = 0; d < Dm; ++d)
+                    out[(((int64_t)b * T + i) * H + h) * Dm + d] = 0.0;
             continue;
         }
         if (s < 0)
             continue;
+        int g = h / heads_per_group;
         /* the stash: every node's own replay inputs */
         for (int32_t i = 0; i < T; ++i) {
             int64_t bi = (int64_t)b * T + i;
-            for (int h = 0; h < H; ++h) {
-                int g = h / heads_per_group;
-                double dte = effective_dt(dt[bi * H + h], dt_bias, h, dt_softplus);
-                st_DA[bi * H + h] = (float)exp((double)A[h] * dte);
-                st_DT[bi * H + h] = (float)dte;
-                for (int d = 0; d < Dm; ++d)
-                    st_U[(bi * H + h) * Dm + d] = (float)load(x, x_dt, (bi * H + h) * Dm + d);
+            double dte = effective_dt(dt[bi * H + h], dt_bias, h, dt_softplus);
+            st_DA[bi * H + h] = (float)exp((double)A[h] * dte);
+            st_DT[bi * H + h] = (float)dte;
+            for (int d = 0; d < Dm; ++d)
+                st_U[(bi * H + h) * Dm + d] = (float)load(x, x_dt, (bi * H + h) * Dm + d);
+            if (h % heads_per_group == 0)
                 for (int n = 0; n < N; ++n)
                     st_B[(bi * G + g) * N + n] = (float)load(B, bc_dt, (bi * G + g) * N + n);
-            }
         }
+        double *S = malloc(sizeof(double) * (size_t)Dm * N);
+        int32_t path[128];
         for (int32_t i = 0; i < T; ++i) {
             int64_t bi = (int64_t)b * T + i;
             /* walk from node i to the root: path[0] = i, path[k] = k-th ancestor */
@@ -499,38 +521,35 @@ int oracle_ddtree(const void *x, int x_dt, const float *A, const void *B, const 
             }
             if (!ok) {
                 err |= 64;
-                for (int64_t e = 0; e < (int64_t)H * Dm; ++e)
-                    out[bi * H * Dm + e] = 0.0;
+                for (int d = 0; d < Dm; ++d)
+                    out[(bi * H + h) * Dm + d] = 0.0;
                 continue;
             }
-            for (int h = 0; h < H; ++h) {
-                int g = h / heads_per_group;
-                for (int64_t e = 0; e < (int64_t)Dm * N; ++e)
-                    S[e] = load(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + e);
-                for (int32_t k = depth; k >= 0; --k) {   /* root-to-node order */
-                    int64_t bj = (int64_t)b * T + path[k];
-                    double dte = effective_dt(dt[bj * H + h], dt_bias, h, dt_softplus);
-                    double decay = exp((double)A[h] * dte);
-                    for (int d = 0; d < Dm; ++d) {
-                        double xv = load(x, x_dt, (bj * H + h) * Dm + d);
-                        for (int n = 0; n < N; ++n) {
-                            double *sp = &S[(int64_t)d * N + n];
-                            *sp = *sp * decay + load(B, bc_dt, (bj * G + g) * N + n) * dte * xv;
-                        }
+            for (int64_t e = 0; e < (int64_t)Dm * N; ++e)
+                S[e] = load(pool, state_dt, s * slot_stride + (int64_t)h * Dm * N + e);
+            for (int32_t k = depth; k >= 0; --k) {   /* root-to-node order */
+                int64_t bj = (int64_t)b * T + path[k];
+                double dte = effective_dt(dt[bj * H + h], dt_bias, h, dt_softplus);
+                double decay = exp((double)A[h] * dte);
+                for (int d = 0; d < Dm; ++d) {
+                    double xv = load(x, x_dt, (bj * H + h) * Dm + d);
+                    for (int n = 0; n < N; ++n) {
+                        double *sp = &S[(int64_t)d * N + n];
+                        *sp = *sp * decay + load(B, bc_dt, (bj * G + g) * N + n) * dte * xv;
                     }
                 }
-                for (int d = 0; d < Dm; ++d) {
-                    double y = 0.0;
-                    for (int n = 0; n < N; ++n)
-                        y += S[(int64_t)d * N + n] * load(C, bc_dt, (bi * G + g) * N + n);
-                    if (D)
-                        y += (double)D[h] * load(x, x_dt, (bi * H + h) * Dm + d);
-                    out[(bi * H + h) * Dm + d] = y;
-                }
+            }
+            for (int d = 0; d < Dm; ++d) {
+                double y = 0.0;
+                for (int n = 0; n < N; ++n)
+                    y += S[(int64_t)d * N + n] * load(C, bc_dt, (bi * G + g) * N + n);
+                if (D)
+                    y += (double)D[h] * load(x, x_dt, (bi * H + h) * Dm + d);
+                out[(bi * H + h) * Dm + d] = y;
             }
         }
+        free(S);
     }
-    free(S);
     if (err_flags)
         *err_flags |= err;
     return 0;
@@ -566,9 +585,10 @@ int oracle_conv_decode(const void *xbc, int x_dt, const void *conv_w, const void
         return 2;
     const int64_t cd = (int64_t)H * Dm + 2 * (int64_t)G * N;
     int32_t err = 0;
-    double *v = malloc(sizeof(double) * (size_t)cd);
-    double *win = malloc(sizeof(double) * (size_t)width);
-    int hpg = H / G;
+    const int hpg = H / G;
+    /* every row owns its slot of both pools and its output rows (the B and C channels of
+     * a row are shared by its heads, so the unit of parallel work is the row) */
+#pragma omp parallel for schedule(dynamic, 1) reduction(|:err)
     for (int32_t b = 0; b < active; ++b) {
         int64_t s = resolve_slot(state_indices, b, P, &err);
         if (s == -1) {
@@ -578,6 +598,8 @@ int oracle_conv_decode(const void *xbc, int x_dt, const void *conv_w, const void
         }
         if (s < 0)
             continue;
+        double *v = malloc(sizeof(double) * (size_t)cd);
+        double *win = malloc(sizeof(double) * (size_t)width);
         for (int64_t c = 0; c < cd; ++c) {
             for (int k = 0; k + 1 < width; ++k)
                 win[k] = load(conv_state, x_dt, s * conv_slot_stride + c * stride_c + k * stride_k);
@@ -613,9 +635,9 @@ int oracle_conv_decode(const void *xbc, int x_dt, const void *conv_w, const void
                 out[oi] = y;
             }
         }
+        free(v);
+        free(win);
     }
-    free(v);
-    free(win);
     if (err_flags)
         *err_flags |= err;
     return 0;
@@ -649,65 +671,78 @@ int oracle_gdn_decode(const void *q, const void *k, const void *v, int x_dt,
         K <= 0 || V <= 0 || slot_stride < (int64_t)HV * V * K)
         return 2;
     int32_t err = 0;
-    double *S = malloc(sizeof(double) * (size_t)V * K);
-    double *qn = malloc(sizeof(double) * (size_t)K);
-    double *kn = malloc(sizeof(double) * (size_t)K);
-    int vpk = HV / HK;
-    for (int32_t b = 0; b < active; ++b) {
+    const int vpk = HV / HK;
+    const int64_t units = (int64_t)active * HV;
+    /* every (row, value head) unit owns its state block and output row */
+#pragma omp parallel for schedule(dynamic, 1) reduction(|:err)
+    for (int64_t u = 0; u < units; ++u) {
+        const int32_t b = (int32_t)(u / HV);
+        const int hv = (int)(u % HV);
         int64_t s = resolve_slot(state_indices, b, P, &err);
         if (s == -1) {
-            for (int64_t i = 0; i < (int64_t)HV * V; ++i)
-                out[(int64_t)b * HV * V + i] = 0.0;
+            for (int i = 0; i < V; ++i)
+                out[((int64_t)b * HV + hv) * V + i] = 0.0;
             continue;
         }
         if (s < 0)
             continue;
-        for (int hv = 0; hv < HV; ++hv) {
-            int hk = hv / vpk;
-            double nq = 0.0, nk = 0.0;
-            for (int j = 0; j < K; ++j) {
-                qn[j] = load(q, x_dt, ((int64_t)b * HK + hk) * K + j);
-                kn[j] = load(k, x_dt, ((int64_t)b * HK + hk) * K + j);
-                nq += qn[j] * qn[j];
-                nk += kn[j] * kn[j];
-            }
-            double fq = use_l2norm ? 1.0 / sqrt(nq + 1e-6) : 1.0;
-            double fk = use_l2norm ? 1.0 / sqrt(nk + 1e-6) : 1.0;
-            for (int j = 0; j < K; ++j) {
-                qn[j] *= fq * scale;
-                kn[j] *= fk;
-            }
-            double av = load(a_in, x_dt, (int64_t)b * HV + hv) + (dt_bias ? dt_bias[hv] : 0.0);
-            double g = -exp((double)A_log[hv]) * softplus(av);
-            double alpha = exp(g);
-            double beta = 1.0 / (1.0 + exp(-load(b_in, x_dt, (int64_t)b * HV + hv)));
-            int64_t base = s * slot_stride + (int64_t)hv * V * K;
-            for (int64_t e = 0; e < (int64_t)V * K; ++e)
-                S[e] = alpha * (double)pool[base + e];
-            for (int i = 0; i < V; ++i) {
-                double *row = S + (int64_t)i * K;
-                double u = 0.0;
-                for (int j = 0; j < K; ++j)
-                    u += row[j] * kn[j];
-                double d = beta * (load(v, x_dt, ((int64_t)b * HV + hv) * V + i) - u);
-                double o = 0.0;
-                for (int j = 0; j < K; ++j) {
-                    row[j] += d * kn[j];
-                    o += row[j] * qn[j];
-                }
-                out[((int64_t)b * HV + hv) * V + i] = o;
-            }
-            for (int64_t e = 0; e < (int64_t)V * K; ++e)
-                pool[base + e] = (float)S[e];
+        double *S = malloc(sizeof(double) * (size_t)V * K);
+        double *qn = malloc(sizeof(double) * (size_t)K);
+        double *kn = malloc(sizeof(double) * (size_t)K);
+        int hk = hv / vpk;
+        double nq = 0.0, nk = 0.0;
+        for (int j = 0; j < K; ++j) {
+            qn[j] = load(q, x_dt, ((int64_t)b * HK + hk) * K + j);
+            kn[j] = load(k, x_dt, ((int64_t)b * HK + hk) * K + j);
+            nq += qn[j] * qn[j];
+            nk += kn[j] * kn[j];
         }
+        double fq = use_l2norm ? 1.0 / sqrt(nq + 1e-6) : 1.0;
+        double fk = use_l2norm ? 1.0 / sqrt(nk + 1e-6) : 1.0;
+        for (int j = 0; j < K; ++j) {
+            qn[j] *= fq * scale;
+            kn[j] *= fk;
+        }
+        double av = load(a_in, x_dt, (int64_t)b * HV + hv) + (dt_bias ? dt_bias[hv] : 0.0);
+        double g = -exp((double)A_log[hv]) * softplus(av);
+        double alpha = exp(g);
+        double beta = 1.0 / (1.0 + exp(-load(b_in, x_dt, (int64_t)b * HV + hv)));
+        int64_t base = s * slot_stride + (int64_t)hv * V * K;
+        for (int64_t e = 0; e < (int64_t)V * K; ++e)
+            S[e] = alpha * (double)pool[base + e];
+        for (int i = 0; i < V; ++i) {
+            double *row = S + (int64_t)i * K;
+            double uk = 0.0;
+            for (int j = 0; j < K; ++j)
+                uk += row[j] * kn[j];
+            double d = beta * (load(v, x_dt, ((int64_t)b * HV + hv) * V + i) - uk);
+            double o = 0.0;
+            for (int j = 0; j < K; ++j) {
+                row[j] += d * kn[j];
+                o += row[j] * qn[j];
+            }
+            out[((int64_t)b * HV + hv) * V + i] = o;
+        }
+        for (int64_t e = 0; e < (int64_t)V * K; ++e)
+            pool[base + e] = (float)S[e];
+        free(S);
+        free(qn);
+        free(kn);
     }
-    free(S);
-    free(qn);
-    free(kn);
     if (err_flags)
         *err_flags |= err;
     return 0;
 }
+
+/* ---------------- thread count ----------------
+ * The loops above run their independent units (a row and head, or a row) on the
+ * OpenMP threads; each unit's arithmetic is sequential and in the same order for any
+ * thread count, so results do not depend on it. n <= 0 selects every host core. */
+void oracle_set_threads(int n) { omp_set_num_threads(n > 0 ? n : omp_get_num_procs()); }
+
+int oracle_max_threads(void) { return omp_get_max_threads(); }
+
+int oracle_host_cores(void) { return omp_get_num_procs(); }
 
 /* ---------------- slot maintenance ----------------
  * Selective State Update page, invokeMambaStateClear (one slot, or all when slot is -1)

@@ -882,3 +882,60 @@ def test_gdn_index_flag(orc):
     out, pool, err = orc.gdn_case(case)
     assert err == 1 and torch.isnan(out[1]).all()
     assert torch.equal(gdn_slots(case, pool)[0], gdn_slots(case)[0])
+
+
+# ---------------------------------------------------------------- thread count
+
+def _run_all_forms(orc):
+    """Every parallel oracle routine on a small case with padding, lengths, a padded slot
+    stride, several groups, trees and out-of-range lengths; returns everything written."""
+    outs = []
+    c = make_case(seed=901, batch=6, P=9, T=5, H=4, G=2, Dm=12, N=16, z=True, active=5,
+                  n_pad=1, lengths="context", slot_pad=4)
+    c.context_lengths[1] = 9                      # clamped, flagged
+    outs += list(orc.decode_case(dataclass_t0(c)))
+    o, p, st, e = orc.prefill_case(c, stash=True)
+    outs += [o, p, *st, e]
+    o, p, _, e = orc.prefill_case(c, stash=False)
+    outs += [o, p, e]
+    acc = torch.tensor([3, 0, 5, 7, 1, 2], dtype=torch.int32)
+    pool = c.pool.clone()
+    outs += [orc.replay(pool, st, acc, state_indices=c.state_indices, batch=c.batch,
+                        active=c.active, T=c.T, H=c.H, G=c.G, Dm=c.Dm, N=c.N,
+                        slot_stride=c.slot_stride, P=c.P), pool]
+    t = make_case(seed=902, batch=4, P=6, T=9, H=4, G=2, Dm=8, N=16, tree="forest", active=4,
+                  n_pad=1)
+    t.parent_ids[2, 3] = 7                        # one malformed walk
+    o, st, e = orc.ddtree_case(t)
+    outs += [o, *st, e]
+    k = make_case(seed=903, batch=5, P=7, H=4, G=2, Dm=8, N=16, z=True, conv=4, n_pad=1)
+    outs += list(orc.conv_decode_case(k))
+    gd = make_gdn_case(seed=904, batch=5, P=7, HK=2, HV=4, K=16, V=8, n_pad=1)
+    outs += list(orc.gdn_case(gd))
+    return outs
+
+
+def dataclass_t0(case):
+    """Token 0 of a prefill case as a decode case (x/B/C/dt/z without the token axis)."""
+    import dataclasses
+    one = {f: getattr(case, f)[:, 0].contiguous() for f in ("x", "B", "C", "dt", "z")}
+    return dataclasses.replace(case, T=1, **one)
+
+
+def test_results_do_not_depend_on_thread_count(orc):
+    """The (row, head) units run on OpenMP threads; each unit's arithmetic is sequential,
+    so one thread and every host core give the same bytes."""
+    before = orc.threads()
+    try:
+        orc.set_threads(1)
+        one = _run_all_forms(orc)
+        orc.set_threads(max(4, orc.host_cores()))
+        many = _run_all_forms(orc)
+    finally:
+        orc.set_threads(before)
+    assert len(one) == len(many)
+    for a, b in zip(one, many):
+        if isinstance(a, torch.Tensor):
+            assert same_bits(a, b)
+        else:
+            assert a == b
