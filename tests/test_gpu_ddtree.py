@@ -13,7 +13,7 @@ import torch
 import gpu_run
 from linear_attention_recurrent_selective_b200 import ssu
 from linear_attention_recurrent_selective_b200.workloads import make_case, make_config
-from parity import check_fp32, check_out, check_state, same_bits
+from parity import changed_slots, check_fp32, check_out, check_state, same_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -134,22 +134,29 @@ def test_ddtree_malformed_nodes_and_bad_index(orc, bcdt):
     assert (out_g[0, 3] == 0).all() and (out_g[1, 5] == 0).all()
 
 
-def test_ddtree_headline_workload_sampled_rows(orc):
-    """The 16 x 128-node workload in its own launch shape; the oracle recomputes two rows
-    (same pool, same row inputs) and those rows must match."""
+def test_ddtree_headline_workload_every_row(orc):
+    """The 16 x 128-node workload in its benchmarked launch, every row compared with the
+    oracle: every node's outputs and the whole stash; the pool is only read. Then the
+    accepted root-to-node paths replayed from each side's stash."""
     case = make_config("ddtree_b16_n128")
     out_g, pool_g, st_g, err_g = gpu_run.ddtree(case)
-    assert err_g == 0
+    out_o, st_o, err_o = orc.ddtree_case(case)
+    assert err_g == err_o == 0
     assert same_bits(pool_g, case.pool)
-    for r in (0, 11):
-        sub = dataclasses.replace(
-            case, batch=1, active=1, x=case.x[r:r + 1].clone(), B=case.B[r:r + 1].clone(),
-            C=case.C[r:r + 1].clone(), dt=case.dt[r:r + 1].clone(),
-            state_indices=case.state_indices[r:r + 1].clone(),
-            parent_ids=case.parent_ids[r:r + 1].clone(), depths=case.depths[r:r + 1].clone())
-        out_o, st_o, _ = orc.ddtree_case(sub)
-        check_out(out_g[r:r + 1], out_o, case.x_dtype)
-        assert same_bits(st_g[1][r:r + 1], st_o[1]) and same_bits(st_g[2][r:r + 1], st_o[2])
+    check_out(out_g, out_o, case.x_dtype)
+    assert same_bits(st_g[1], st_o[1]) and same_bits(st_g[2], st_o[2])   # U, B widened
+    check_fp32(st_g[0], st_o[0])
+    check_fp32(st_g[3], st_o[3])
+    want = case.pool.clone()
+    err_o = orc.replay(want, st_o, case.accepted_lengths, state_indices=case.state_indices,
+                       batch=case.batch, active=case.active, T=case.T, H=case.H, G=case.G,
+                       Dm=case.Dm, N=case.N, slot_stride=case.slot_stride, P=case.P,
+                       node_ids=case.accepted_node_ids)
+    pool_r, err_r = gpu_run.replay(case, st_g, case.accepted_lengths,
+                                   node_ids=case.accepted_node_ids)
+    assert err_r == err_o == 0
+    check_state(pool_r, want, case.state_dtype)
+    assert changed_slots(case.pool, pool_r, case) == changed_slots(case.pool, want, case)
 
 
 # ---------------------------------------------------------------- accepted-node replay

@@ -3,8 +3,6 @@
 Selective State Update page (TensorRT-Edge-LLM C++ API),
 invokeSelectiveStateUpdatePrefill."""
 
-import dataclasses
-
 import pytest
 import torch
 
@@ -76,28 +74,16 @@ def test_prefill_length_edge_cases(orc):
     assert torch.isnan(out_g[0].float()).all() and torch.isnan(out_g[3].float()).all()
 
 
-def test_prefill_b16_t512_sampled_rows(orc):
-    """Full-size multi-token prefill on the GPU (the benchmarked launch); the oracle
-    recomputes three rows (the longest, the shortest and one more) one by one."""
+def test_prefill_b16_t512_every_row(orc):
+    """The full multi-token prefill workload in the benchmarked launch, every row compared
+    with the oracle element by element: with the replay stash the outputs, the whole
+    stash and the untouched committed state; without it the outputs and every pool slot
+    (the live rows' final states, all other slots byte-identical)."""
     case = make_config("prefill_b16_t512")
-    out_g, pool_g, st_g, _ = gpu_run.prefill(case, stash=True)
-    out_n, pool_n, _, _ = gpu_run.prefill(case, stash=False)
-    assert same_bits(out_g, out_n)                  # stash changes nothing in the outputs
-    assert same_bits(pool_g, case.pool)
-    L = case.context_lengths
-    rows = sorted({int(L.argmax()), int(L.argmin()), 5})
-    for b in rows:
-        rows_of = {f: getattr(case, f)[b: b + 1].contiguous()
-                   for f in ("x", "B", "C", "dt", "z", "state_indices", "context_lengths")}
-        sub = dataclasses.replace(case, batch=1, active=1, **rows_of)
-        out_o, pool_o, st_o, _ = orc.prefill_case(sub, stash=True)
-        check_out(out_g[b: b + 1], out_o, case.x_dtype)
-        assert same_bits(st_g[1][b: b + 1], st_o[1]) and same_bits(st_g[2][b: b + 1], st_o[2])
-        check_fp32(st_g[0][b: b + 1], st_o[0])
-        _, pool_o, _, _ = orc.prefill_case(sub, stash=False)
-        s = int(case.state_indices[b])
-        sl = slice(s * case.slot_stride, (s + 1) * case.slot_stride)
-        check_state(pool_n[sl], pool_o[sl], case.state_dtype)
+    assert int(case.context_lengths.min()) < case.T    # ragged lengths
+    out_s, _, _ = compare_prefill(orc, case, stash=True)
+    out_n, pool_n, _ = compare_prefill(orc, case, stash=False)
+    assert same_bits(out_s, out_n)                  # the stash changes nothing in the outputs
     touched = {int(case.state_indices[b]) for b in range(case.batch)}
     assert changed_slots(case.pool, pool_n, case) == touched
 
