@@ -15,7 +15,8 @@ steps do not hit in L2 and no flush is needed (checked at run time).
              from pinned host memory and the output copied back inside the timed region
   forms      (one GPU only) the prefill scan and the speculative replay on their own
              workloads, same timing method
-  cpu_baseline  the float64 CPU oracle on a bounded sample, rank 0, one GPU only
+  cpu_baseline  the float64 CPU oracle on a bounded sample, rank 0, one GPU only: on
+             every host core (value, cores) and on one thread, with the CPU model
 
 Multi-GPU (torchrun): replicas only -- every rank runs its own pool and batch, no data
 collective; the barrier and the max-over-ranks reduction are measurement plumbing.
@@ -75,7 +76,7 @@ def measured_peaks():
 
 
 DECODE_SOURCES = ("ssu_decode.cu", "ssu_stream.cuh", "ssu_async.cuh", "ssu_common.cuh")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ssu_decode_kernel.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ssu_decode_traffic.json")
 
 
 def decode_source_hash() -> str:
@@ -90,24 +91,19 @@ def decode_source_hash() -> str:
 
 
 def recorded_traffic(batch: int):
-    """DRAM bytes per decode launch recorded from ncu in the decode profile summary, or
-    None when the summary is missing, is for another batch, or was taken on sources
-    other than the ones built now."""
+    """DRAM bytes per decode launch measured by ncu (profiles/ssu_decode_traffic.json), or
+    None when the record is missing, is for another batch, or was taken on sources other
+    than the ones built now."""
     try:
-        text = open(TRAFFIC_FILE).read()
-    except OSError:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
-    rec = {}
-    for line in text.splitlines():
-        if line.startswith("traffic_record:"):
-            for kv in line.split(":", 1)[1].split():
-                k, _, v = kv.partition("=")
-                rec[k] = v
-    if rec.get("source_sha256") != decode_source_hash() or rec.get("batch") != str(batch):
+    if rec.get("source_sha256") != decode_source_hash() or rec.get("batch") != batch:
         return None
     try:
         return int(rec["bytes_per_launch"])
-    except (KeyError, ValueError):
+    except (KeyError, TypeError, ValueError):
         return None
 
 
@@ -153,7 +149,7 @@ def barrier(device):
 class ClockSampler:
     """Polls SM clock and clock-event reasons via NVML while the timed region runs."""
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples = []      # (t, sm_mhz, reasons_mask)
         self.max_mhz = None
         self._stop = threading.Event()
@@ -265,6 +261,27 @@ def run_decode(args, device):
     kern_ms = statistics.fmean(s.elapsed_time(e) for s, e in zip(starts, ends))
     res = dict(case=case, units=units, total_ms=total_ms, kern_ms=kern_ms, state_b=state_b,
                alg_b=alg_b, clocks=clocks.summary(wall0, wall1), flush=flush, l2=l2)
+
+    # ---- clock record over a longer window (not part of the reported value): the same
+    # step back to back for at least 0.5 s, NVML sampled every 5 ms, so that the clock the
+    # kernel ran at rests on many samples even when the timed region above is short
+    n_sus = max(10, int(0.6 / max(kern_ms / 1e3, 1e-6)))
+    sus = ClockSampler(device.index, period_s=0.005).start()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    w0 = time.perf_counter()
+    s0.record(stream)
+    for _ in range(n_sus):
+        if flush:
+            flush_buf.zero_()
+        step()
+    s1.record(stream)
+    torch.cuda.synchronize(device)
+    w1 = time.perf_counter()
+    sus.stop()
+    sus_ms = s0.elapsed_time(s1) / n_sus
+    res["clocks_sustained"] = {**sus.summary(w0, w1), "steps": n_sus,
+                               "seconds": round(w1 - w0, 3), "ms_per_step": sus_ms}
 
     # ---- end to end through the binding: pinned host inputs in, output back out.
     # Every step copies its inputs from pinned host memory and reads its output back; the
@@ -610,21 +627,53 @@ def form_ddtree(args, device, hbm_peak):
     return forms
 
 
-def cpu_baseline_decode(case, max_seconds=20.0):
-    """The float64 oracle on whole decode steps of the same workload, timed on this host."""
+def cpu_model() -> str:
+    """The host CPU's model name from /proc/cpuinfo (empty when unavailable)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return ""
+
+
+def _time_oracle_steps(oracle, case, threads, budget_s, max_steps):
+    """Whole decode steps of the oracle on `threads` threads until budget_s has passed
+    (at least one step). Returns (steps, seconds, threads used)."""
+    used = oracle.set_threads(threads)
+    pool = case.pool.clone()             # updated in place step after step, like the GPU's
+    runs, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode_case(case, pool=pool)
+        runs += 1
+        el = time.perf_counter() - t0
+        if el > budget_s or runs >= max_steps:
+            return runs, el, used
+
+
+def cpu_baseline_decode(case, budget_s=8.0):
+    """The float64 oracle on whole decode steps of the same workload, timed on this host:
+    on every host core (the reported value; the oracle's (row, head) units run on OpenMP
+    threads) and on one thread, each for about budget_s seconds."""
     from oracle import oracle
     oracle.build()
     units = case.batch * case.H
-    runs, t0 = 0, time.perf_counter()
-    while True:
-        oracle.decode_case(case)
-        runs += 1
-        el = time.perf_counter() - t0
-        if el > max_seconds / 2 or runs >= 2:
-            break
-    return {"value": units * runs / el, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{runs} full decode step(s) of the batch-{case.batch} workload "
-                      f"({units} seq-head updates each), single thread, {el:.1f} s"}
+    before = oracle.threads()
+    try:
+        runs_n, el_n, cores = _time_oracle_steps(oracle, case, 0, budget_s, 1000)
+        runs_1, el_1, _ = _time_oracle_steps(oracle, case, 1, budget_s, 1000)
+    finally:
+        oracle.set_threads(before)
+    model = cpu_model()
+    return {"value": units * runs_n / el_n, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{runs_n} full decode step(s) of the batch-{case.batch} workload "
+                      f"({units} seq-head updates each) on {cores} threads, {el_n:.1f} s",
+            "host_cores": oracle.host_cores(), "cpu_model": model,
+            "single_thread": {"value": units * runs_1 / el_1, "unit": UNIT, "cores": 1,
+                              "sample": f"{runs_1} full decode step(s), one thread, "
+                                        f"{el_1:.1f} s"}}
 
 
 def config_block(case, res=None):
@@ -690,7 +739,7 @@ def main_ours(args):
                           "streams, double-buffered so they overlap the neighbouring steps' "
                           "compute"},
         "gpu_launches": args.steps,
-        "clocks": res["clocks"],
+        "clocks": {**res["clocks"], "sustained": res["clocks_sustained"]},
     }
     if n_world == 1 and not args.no_forms and args.form == "all":
         line["forms"] = {**form_prefill(args, device), **form_replay(args, device, hbm_peak),
@@ -709,26 +758,36 @@ def main_ours(args):
 # ----------------------------------------------------------------------------- reference arm
 
 def main_reference(args):
-    """The float64 CPU oracle as the reference arm: rank 0 only, bounded per-step samples."""
+    """The float64 CPU oracle as the reference arm: rank 0 only, on every host core, each
+    step the whole decode workload or, on a small host, a bounded row sample of it."""
     n_world, rank, _ = world()
     if rank != 0:
         return
+    import dataclasses
     from linear_attention_recurrent_selective_b200.workloads import make_config
     from oracle import oracle
     oracle.build()
+    cores = oracle.set_threads(0)
     case = make_config(WORKLOAD)
-    # one head-row of work is ~20 ms in the oracle: keep the whole run near a minute
-    rows = max(1, min(case.batch, int(60.0 / max(1, args.steps + args.warmup) / 0.02)))
-    sub = case
-    import dataclasses
-    pick = {f: getattr(case, f)[:rows].contiguous()
+    # one probe step on a 16-row sample sets the row count: the whole run near a minute
+    probe = 16
+    pick = {f: getattr(case, f)[:probe].contiguous()
             for f in ("x", "z", "B", "C", "dt", "state_indices")}
-    sub = dataclasses.replace(case, batch=rows, active=rows, **pick)
+    pool = case.pool.clone()             # updated in place step after step, like the GPU's
+    t0 = time.perf_counter()
+    oracle.decode_case(dataclasses.replace(case, batch=probe, active=probe, **pick), pool=pool)
+    per_row = (time.perf_counter() - t0) / probe
+    rows = max(1, min(case.batch, int(60.0 / max(1, args.steps + args.warmup) / per_row)))
+    sub = case
+    if rows < case.batch:
+        pick = {f: getattr(case, f)[:rows].contiguous()
+                for f in ("x", "z", "B", "C", "dt", "state_indices")}
+        sub = dataclasses.replace(case, batch=rows, active=rows, **pick)
     for _ in range(args.warmup):
-        oracle.decode_case(sub)
+        oracle.decode_case(sub, pool=pool)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.decode_case(sub)
+        oracle.decode_case(sub, pool=pool)
     el = time.perf_counter() - t0
     units = rows * case.H * args.steps
     value = units / el
@@ -737,8 +796,9 @@ def main_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_block(case), "impl": "reference",
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{rows} of {case.batch} rows x {case.H} heads per step"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} of {case.batch} rows x {case.H} heads per step",
+                         "host_cores": oracle.host_cores(), "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
