@@ -18,9 +18,12 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Device pointers unless stated otherwise. The caller owns every buffer; the library
- *    allocates nothing, keeps no state between calls and never synchronises the host.
- *    All work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
- *    stream), so every entry point may be recorded into a CUDA graph.
+ *    allocates nothing and never synchronises the host. The only state it keeps is a
+ *    per-device cache of facts about the device and each kernel (SM count, occupancy,
+ *    the kernel's shared-memory limit), filled once under std::call_once, so first calls
+ *    from several host threads are safe; it never affects results. All work is enqueued
+ *    on `stream` (a cudaStream_t; NULL is the legacy default stream), so every entry
+ *    point may be recorded into a CUDA graph.
  *  - Optional inputs are NULL when absent.
  *  - Layouts are dense, row-major and batch-major as written beside each argument.
  *    Names: batch rows b, tokens t, heads h < nheads (H), groups g < ngroups (G),
@@ -33,7 +36,8 @@
  *  - state_indices [batch] int32 maps row b to its pool slot (NULL: row b uses slot b).
  *    A negative index marks a padding row: its state is neither read nor written and
  *    its output rows are written as zero. Indices of the active rows that are >= 0 must
- *    be distinct (two rows updating one slot would race).
+ *    be distinct (two rows updating one slot would race); the kernels do not check this,
+ *    ssu_check_state_indices does (for debugging).
  *  - Only rows b < active_batch are visited; rows beyond it are left untouched, so a
  *    graph captured at the maximum batch can run a smaller live batch.
  *  - An index >= P, or a length outside [0, T], is a caller bug that the pages leave
@@ -43,7 +47,9 @@
  *    SSU_FLAG_NEGATIVE_LENGTH. Kernels that wait on their own asynchronous copies bound
  *    every wait and report SSU_FLAG_TIMEOUT instead of hanging.
  *  - Return value: SSU_OK, or an ssu_status error, in which case nothing was launched
- *    (SSU_ERR_CUDA: the launch itself failed). Sizes and dtype codes are checked first;
+ *    (SSU_ERR_CUDA: the launch itself failed, as cudaLaunchKernelEx reported it for this
+ *    launch; an error left by unrelated earlier work in the calling thread is neither
+ *    reported nor cleared). Sizes and dtype codes are checked first;
  *    a call with nothing to do (active_batch == 0, or T == 0) then returns SSU_OK without
  *    looking at any pointer, since empty tensors may carry NULL data pointers.
  *  - Arithmetic is fp32; fp16/bf16 values are widened exactly and results are rounded
@@ -70,11 +76,11 @@ typedef enum {
     SSU_ERR_DTYPE = 3,        /* dtype code not one of ssu_dtype */
     SSU_ERR_UNSUPPORTED = 4,  /* dstate not in {8,16,32,64,128,256}, or (ssu_ddtree) a
                                  tree whose tables exceed shared memory */
-    SSU_ERR_CUDA = 5,         /* the kernel launch failed */
+    SSU_ERR_CUDA = 5,         /* the kernel launch failed (or the device could not be
+                                 queried before it) */
     SSU_ERR_ALIGN = 6         /* pool pointer or slot stride not 16-byte aligned, or (in
                                  ssu_prefill / ssu_replay / ssu_ddtree) B, C or the stash B
-                                 not 16-byte
-                                 aligned */
+                                 not 16-byte aligned */
 } ssu_status;
 
 enum {
@@ -86,9 +92,11 @@ enum {
                                      the outputs of that launch are incomplete */
     SSU_FLAG_LAYER = 32,          /* a per-layer pointer was NULL or not 16-byte aligned:
                                      that layer was skipped */
-    SSU_FLAG_TREE = 64            /* ssu_ddtree: a node's parent walk was malformed (its
+    SSU_FLAG_TREE = 64,           /* ssu_ddtree: a node's parent walk was malformed (its
                                      outputs are 0); replay: an accepted node id outside
                                      [0, T) (the row was left untouched) */
+    SSU_FLAG_DUPLICATE_INDEX = 128 /* ssu_check_state_indices only: two active rows name
+                                     the same slot */
 };
 
 /* Per-layer device pointers of a multi-layer replay: one entry per layer, in a device
@@ -345,6 +353,24 @@ int pool_gather(const void *pool, int64_t slot_bytes, int32_t P, void *dense,
 int pool_scatter(const void *dense, void *pool, int64_t slot_bytes, int32_t P,
                  const int32_t *state_indices, int32_t batch, int32_t active_batch,
                  int32_t *err_flags, ssu_stream_t stream);
+
+/*
+ * ssu_check_state_indices -- debug check of a row-to-slot map before it is used.
+ * The padding contract of the FlashInfer page flashinfer.gdn_fused_decode_step
+ * (state_indices): every batch row reads and writes its own slot, so the active rows'
+ * non-negative indices must be distinct (the other entry points take that as a
+ * precondition and do not check it). One launch on `stream` that ORs into the device
+ * int32 *err_flags (required): SSU_FLAG_DUPLICATE_INDEX when two rows b < active_batch
+ * hold the same index >= 0, SSU_FLAG_INDEX_RANGE when one holds an index >= P. Negative
+ * indices (padding) may repeat. O(active_batch^2) comparisons: meant for debugging and
+ * tests, not for every step. Like every entry point it allocates nothing and does not
+ * synchronise; the caller reads the flags when it chooses.
+ * Returns SSU_ERR_NULL for a NULL state_indices or err_flags (when active_batch > 0),
+ * SSU_ERR_SHAPE for active_batch outside [0, batch] or P < 0.
+ */
+int ssu_check_state_indices(const int32_t *state_indices, int32_t batch,
+                            int32_t active_batch, int32_t P, int32_t *err_flags,
+                            ssu_stream_t stream);
 
 /* A constant string naming an ssu_status value. */
 const char *ssu_status_string(int status);

@@ -3,11 +3,21 @@
 // Every entry point validates its arguments on the host without touching device memory
 // (so it stays legal under CUDA-graph capture), returns an ssu_status error without
 // launching anything when a check fails, and otherwise enqueues its kernel on the
-// caller's stream (one launch; ssu_conv_decode enqueues two). Values that live on the device (stateIndices, contextLengths,
+// caller's stream (one launch; ssu_conv_decode enqueues two). Kernels are launched with
+// cudaLaunchKernelEx and the call returns that launch's own status: an error left by
+// unrelated earlier work in the caller's thread is neither reported nor cleared. Values that live on the device (stateIndices, contextLengths,
 // acceptedLengths, tree parents and depths, accepted node ids) are checked in-kernel,
 // as the padding contract of the FlashInfer page flashinfer.gdn_fused_decode_step
 // requires for graph replay.
 #include "ssu_common.cuh"
+#ifdef SSU_WAIT_TEST
+#include "ssu_async.cuh"
+#include "ssu_wait_test.h"
+static_assert(SSU_WAIT_STREAM == ssu::kFaultStream && SSU_WAIT_PREFILL == ssu::kFaultPrefill &&
+                  SSU_WAIT_TREE_STATE == ssu::kFaultTreeState &&
+                  SSU_WAIT_TREE_X == ssu::kFaultTreeX && SSU_WAIT_TREE_MMA == ssu::kFaultTreeMma,
+              "wait sites of the test header and the kernels agree");
+#endif
 
 namespace {
 
@@ -47,13 +57,6 @@ int check_pool_alignment(const void *state, int state_dtype, int64_t slot_stride
     if (!aligned16(state) || (slot_stride * elem_bytes(state_dtype)) % 16 != 0)
         return SSU_ERR_ALIGN;
     return SSU_OK;
-}
-
-int finish(int rc)
-{
-    if (rc != SSU_OK)
-        return rc;
-    return cudaGetLastError() == cudaSuccess ? SSU_OK : SSU_ERR_CUDA;
 }
 
 ssu::DecodeArgs pack_decode(const void *x, int x_dtype, const float *A, const void *B,
@@ -114,7 +117,7 @@ int ssu_decode(const void *x, int x_dtype, const float *A, const void *B, const 
     ssu::DecodeArgs a = pack_decode(x, x_dtype, A, B, C, bc_dtype, dt, dt_bias, D, z, state,
                                     slot_stride, P, out, state_indices, batch, active_batch,
                                     nheads, ngroups, dim, dstate, dt_softplus, err_flags);
-    return finish(ssu::launch_decode(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+    return ssu::launch_decode(a, state_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int ssu_prefill(const void *x, int x_dtype, const float *A, const void *B, const void *C,
@@ -154,7 +157,7 @@ int ssu_prefill(const void *x, int x_dtype, const float *A, const void *B, const
     a.st_B = st_B;
     a.st_dt = st_dt;
     a.T = T;
-    return finish(ssu::launch_prefill(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+    return ssu::launch_prefill(a, state_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int ssu_replay(void *state, int state_dtype, int64_t slot_stride, int32_t P,
@@ -199,7 +202,7 @@ int ssu_replay(void *state, int state_dtype, int64_t slot_stride, int32_t P,
     a.Dm = dim;
     a.N = dstate;
     a.max_accept = accepted_node_ids ? max_accept_len : T;
-    return finish(ssu::launch_replay(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+    return ssu::launch_replay(a, state_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int ssu_replay_layers(const ssu_replay_layer *layers, int32_t num_layers, int state_dtype,
@@ -238,7 +241,7 @@ int ssu_replay_layers(const ssu_replay_layer *layers, int32_t num_layers, int st
     a.Dm = dim;
     a.N = dstate;
     a.max_accept = accepted_node_ids ? max_accept_len : T;
-    return finish(ssu::launch_replay(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+    return ssu::launch_replay(a, state_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int ssu_conv_decode(const void *xbc, int x_dtype, const void *conv_weight,
@@ -283,7 +286,7 @@ int ssu_conv_decode(const void *xbc, int x_dtype, const void *conv_weight,
     a.ck = conv_stride_k;
     a.width = width;
     a.silu = conv_silu ? 1 : 0;
-    return finish(ssu::launch_conv_decode(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+    return ssu::launch_conv_decode(a, state_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int gdn_decode(const void *q, const void *k, const void *v, int x_dtype, const void *a,
@@ -336,7 +339,7 @@ int gdn_decode(const void *q, const void *k, const void *v, int x_dtype, const v
     g.V = head_v_dim;
     g.x_dtype = x_dtype;
     g.l2norm = use_qk_l2norm ? 1 : 0;
-    return finish(ssu::launch_gdn_decode(g, reinterpret_cast<cudaStream_t>(stream)));
+    return ssu::launch_gdn_decode(g, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int ssu_ddtree(const void *x, int x_dtype, const float *A, const void *B, const void *C,
@@ -374,7 +377,7 @@ int ssu_ddtree(const void *x, int x_dtype, const float *A, const void *B, const 
     a.st_B = st_B;
     a.st_dt = st_dt;
     a.T = T;
-    return finish(ssu::launch_ddtree(a, state_dtype, reinterpret_cast<cudaStream_t>(stream)));
+    return ssu::launch_ddtree(a, state_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int pool_clear_slot_layers(const ssu_layer_states *layers, int32_t num_layers, int32_t P,
@@ -388,9 +391,9 @@ int pool_clear_slot_layers(const ssu_layer_states *layers, int32_t num_layers, i
         return SSU_OK;
     if (!layers)
         return SSU_ERR_NULL;
-    return finish(ssu::launch_clear_layers(layers, num_layers, P, slot, recurrent_slot_bytes,
+    return ssu::launch_clear_layers(layers, num_layers, P, slot, recurrent_slot_bytes,
                                            conv_slot_bytes,
-                                           reinterpret_cast<cudaStream_t>(stream)));
+                                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 static int gather_scatter(const void *pool, int64_t slot_bytes, int32_t P, void *dense,
@@ -405,8 +408,8 @@ static int gather_scatter(const void *pool, int64_t slot_bytes, int32_t P, void 
         return SSU_OK;
     if (!pool || !dense)
         return SSU_ERR_NULL;
-    return finish(ssu::launch_gather(pool, slot_bytes, P, dense, state_indices, active_batch,
-                                     scatter, err_flags, reinterpret_cast<cudaStream_t>(stream)));
+    return ssu::launch_gather(pool, slot_bytes, P, dense, state_indices, active_batch,
+                                     scatter, err_flags, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int pool_gather(const void *pool, int64_t slot_bytes, int32_t P, void *dense,
@@ -434,9 +437,9 @@ int pool_clear_slot(void *pool, int64_t slot_bytes, int32_t P, int32_t slot,
         return SSU_ERR_SHAPE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (slot == -1)
-        return finish(ssu::launch_clear(pool, slot_bytes * P, s));
-    return finish(ssu::launch_clear(static_cast<uint8_t *>(pool) + slot * slot_bytes,
-                                    slot_bytes, s));
+        return ssu::launch_clear(pool, slot_bytes * P, s);
+    return ssu::launch_clear(static_cast<uint8_t *>(pool) + slot * slot_bytes,
+                                    slot_bytes, s);
 }
 
 int pool_copy_slot(void *dst_pool, int32_t dst_P, int32_t dst_slot, const void *src_pool,
@@ -447,10 +450,38 @@ int pool_copy_slot(void *dst_pool, int32_t dst_P, int32_t dst_slot, const void *
     if (slot_bytes < 0 || dst_slot < 0 || dst_slot >= dst_P || src_slot < 0 ||
         src_slot >= src_P)
         return SSU_ERR_SHAPE;
-    return finish(ssu::launch_copy(static_cast<uint8_t *>(dst_pool) + dst_slot * slot_bytes,
+    return ssu::launch_copy(static_cast<uint8_t *>(dst_pool) + dst_slot * slot_bytes,
                                    static_cast<const uint8_t *>(src_pool) + src_slot * slot_bytes,
-                                   slot_bytes, reinterpret_cast<cudaStream_t>(stream)));
+                                   slot_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
+
+int ssu_check_state_indices(const int32_t *state_indices, int32_t batch,
+                            int32_t active_batch, int32_t P, int32_t *err_flags,
+                            ssu_stream_t stream)
+{
+    if (batch < 0 || active_batch < 0 || active_batch > batch || P < 0)
+        return SSU_ERR_SHAPE;
+    if (active_batch == 0)
+        return SSU_OK;
+    if (!state_indices || !err_flags)
+        return SSU_ERR_NULL;
+    return ssu::launch_check_indices(state_indices, active_batch, P, err_flags,
+                                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+#ifdef SSU_WAIT_TEST
+// Test build only (libssu_waittest.so; declared in include/ssu_wait_test.h).
+int ssu_test_wait_fault(int site, int block, int warp, int index, unsigned long long limit_ns)
+{
+    if (limit_ns == 0)
+        return SSU_ERR_SHAPE;
+    const ssu::WaitFault f{limit_ns, site, block, warp, index};
+    const int bad = ssu::wait_fault_set_decode(f) | ssu::wait_fault_set_replay(f) |
+                    ssu::wait_fault_set_conv(f) | ssu::wait_fault_set_gdn(f) |
+                    ssu::wait_fault_set_prefill(f) | ssu::wait_fault_set_ddtree(f);
+    return bad ? SSU_ERR_CUDA : SSU_OK;
+}
+#endif
 
 const char *ssu_status_string(int status)
 {

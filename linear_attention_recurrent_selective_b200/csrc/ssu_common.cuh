@@ -11,9 +11,99 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <utility>
+
 #include "ssu.h"
 
 namespace ssu {
+
+// ---------------------------------------------------------------- launching
+
+constexpr int kMaxDevices = 64;
+
+// The calling thread's current device, or -1 when it cannot be had or lies beyond the
+// per-device caches below.
+inline int current_device()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return -1;
+    return dev;
+}
+
+// Launch `kernel` on `stream` and return the status of this launch alone: an error left
+// behind by unrelated earlier work in the calling thread is neither reported here nor
+// cleared.
+template <typename... KArgs, typename... Args>
+int launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                  cudaStream_t stream, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess
+               ? SSU_OK
+               : SSU_ERR_CUDA;
+}
+
+// What a launch needs to know about the device, found once per process, kernel and
+// device under std::call_once (so concurrent first calls from several host threads are
+// safe): the SM count, the kernel's dynamic shared-memory limit raised to `smem` bytes,
+// and how many CTAs of `threads` threads with `smem` bytes fit on one SM. This cache of
+// device facts is the only host state the library keeps; it never affects results.
+struct KernelFacts {
+    int sms = 0;
+    int blocks_per_sm = 0;
+    int status = SSU_ERR_CUDA;
+};
+
+template <auto kernel>
+const KernelFacts *kernel_facts(int threads, int smem)
+{
+    static std::once_flag once[kMaxDevices];
+    static KernelFacts facts[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0)
+        return nullptr;
+    std::call_once(once[dev], [&] {
+        KernelFacts f;
+        int n = 0, occ = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
+                cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, smem) ==
+                cudaSuccess &&
+            n > 0 && occ > 0) {
+            f.sms = n;
+            f.blocks_per_sm = occ;
+            f.status = SSU_OK;
+        }
+        facts[dev] = f;
+    });
+    return &facts[dev];
+}
+
+#ifdef SSU_WAIT_TEST
+// Test build only (libssu_waittest.so): which bounded wait is made to run out, and the
+// limit of every wait. site 0 injects nothing; warp < 0 matches every warp of the CTA;
+// index counts the wait's instances within that CTA (or warp).
+struct WaitFault {
+    unsigned long long limit_ns;
+    int site, block, warp, index;
+};
+// one per translation unit that holds bounded waits
+int wait_fault_set_decode(const WaitFault &f);
+int wait_fault_set_replay(const WaitFault &f);
+int wait_fault_set_conv(const WaitFault &f);
+int wait_fault_set_gdn(const WaitFault &f);
+int wait_fault_set_prefill(const WaitFault &f);
+int wait_fault_set_ddtree(const WaitFault &f);
+#endif
 
 // ---------------------------------------------------------------- launch descriptors
 
@@ -102,6 +192,8 @@ int launch_clear_layers(const ssu_layer_states *layers, int32_t num_layers, int3
 int launch_gather(const void *pool, int64_t slot_bytes, int32_t P, void *dense,
                   const int32_t *idx, int32_t active, int scatter, int32_t *err,
                   cudaStream_t s);
+int launch_check_indices(const int32_t *idx, int32_t active, int32_t P, int32_t *err,
+                         cudaStream_t s);
 
 // ---------------------------------------------------------------- scalar access
 

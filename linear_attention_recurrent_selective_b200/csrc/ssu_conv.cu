@@ -288,15 +288,17 @@ int launch_n(const ConvArgs &ca, cudaStream_t stream)
     if (nunits > 0x7fffffffLL)
         return SSU_ERR_SHAPE;
     const int grid = persistent_grid<ssu_conv_decode_kernel<S, N>>(nunits);
-    ssu_conv_decode_kernel<S, N><<<grid, kWarps * 32, kSmemBytes, stream>>>(ca, (int)cph,
-                                                                            (int)nunits);
-    if (ca.width > 1) {
+    if (grid < 0)
+        return SSU_ERR_CUDA;
+    int rc = launch_kernel(ssu_conv_decode_kernel<S, N>, grid, kWarps * 32, kSmemBytes, stream,
+                           ca, (int)cph, (int)nunits);
+    if (rc == SSU_OK && ca.width > 1) {
         const int64_t ch0 = (int64_t)a.H * a.Dm;
         const int64_t cd = ch0 + 2 * (int64_t)a.G * N;
         const dim3 blocks((unsigned)((cd - ch0 + 255) / 256), (unsigned)a.active);
-        conv_shift_kernel<<<blocks, 256, 0, stream>>>(ca, cd, ch0);
+        rc = launch_kernel(conv_shift_kernel, blocks, 256, 0, stream, ca, cd, ch0);
     }
-    return SSU_OK;
+    return rc;
 }
 
 template <typename S>
@@ -314,6 +316,10 @@ int launch_s(const ConvArgs &a, cudaStream_t s)
 }
 
 }  // namespace
+
+#ifdef SSU_WAIT_TEST
+SSU_WAIT_FAULT_SETTER(wait_fault_set_conv)
+#endif
 
 int launch_conv_decode(const ConvArgs &a, int state_dtype, cudaStream_t s)
 {

@@ -840,6 +840,12 @@ __device__ __forceinline__ int sw128_off(int r, int c, int block)
 // memory only. The staged B rows also give the stash its B: the shares of heads hh0 ..
 // hh1 (indices within the group) of this CTA's items, each head's share being elements
 // [T N hh / hpg, T N (hh + 1) / hpg) of the row's [T][N] block.
+//
+// Invariant the kernel relies on when it skips an item's closing barrier: before its
+// first __syncthreads this function writes only par (plain stores) and, by cp.async, the
+// C operand and the piece buffer, which the finished item's MMAs no longer read. It must
+// not touch an x tile, cb, pj, cnt, off, sdA or sdt before that barrier, because slower
+// threads may still be writing the previous item's outputs out of its x tile.
 template <int N>
 __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm, int b, int g,
                              bool reporter, int hh0, int hh1)
@@ -1003,7 +1009,8 @@ __device__ void split_state(const TcLayout &lay, uint8_t *sm, int rows)
 // four copies by the leader).
 template <typename S, int N>
 __device__ __forceinline__ void bulk_raw(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm,
-                                         const Item &u, uint64_t *bar, bool leader)
+                                         const Item &u, uint64_t *bar, bool leader,
+                                         uint32_t extra)
 {
     if (!leader)
         return;
@@ -1013,7 +1020,7 @@ __device__ __forceinline__ void bulk_raw(const TreeArgs &ta, const TcLayout &lay
                           (int64_t)sizeof(S);
     const uint32_t bytes = (uint32_t)(u.rows * N * (int)sizeof(S));
     const uint32_t part = ((bytes + 3) / 4 + 15) & ~15u;
-    mbar_arrive_expect_tx(bar, bytes);
+    mbar_arrive_expect_tx(bar, bytes + extra);
     for (uint32_t o = 0; o < bytes; o += part)
         bulk_load(sm + lay.raw + o, src + o, bytes - o < part ? bytes - o : part, bar);
 }
@@ -1022,14 +1029,15 @@ __device__ __forceinline__ void bulk_raw(const TreeArgs &ta, const TcLayout &lay
 // threads (this one is t; t = 0 arms the barrier).
 template <typename X>
 __device__ __forceinline__ void bulk_x(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm,
-                                       const Item &u, int xbuf, uint64_t *bar, int t, int nt)
+                                       const Item &u, int xbuf, uint64_t *bar, int t, int nt,
+                                       uint32_t extra)
 {
     const DecodeArgs &a = ta.d;
     const int T = ta.T;
     constexpr int es = (int)sizeof(X);
     const uint32_t rb = (uint32_t)(u.rows * es);
     if (t == 0)
-        mbar_arrive_expect_tx(bar, rb * (uint32_t)T);
+        mbar_arrive_expect_tx(bar, rb * (uint32_t)T + extra);
     for (int i = t; i < T; i += nt)
         bulk_load(sm + lay.xs + xbuf * lay.xbytes + i * kXS * es,
                   static_cast<const X *>(a.x) + (((int64_t)u.b * T + i) * a.H + u.h) * a.Dm +
@@ -1151,6 +1159,7 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
     const int ni = 32 * (warp & 3) + lane, d0 = 16 * (warp >> 2);
     const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)d0;
     uint32_t phase = 0;                  // parity of the MMA barrier's next phase
+    bool mma_out = false;                // an MMA wait gave up (its phase is still awaited)
     // copies in flight (uniform): state rows, x tiles by buffer bit; parities likewise
     uint32_t s_out = 0, x_out = 0, sph = 0, xph = 0;
 
@@ -1164,9 +1173,11 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
     const int xt = kTcThreads - 1 - tid;
     auto issue = [&](const Item &w, int64_t wit, bool with_x) {
         const int xb = xbuf_of(wit);
-        bulk_raw<S, N>(ta, lay, sm, w, sbar, tid == 0);
+        bulk_raw<S, N>(ta, lay, sm, w, sbar, tid == 0,
+                       fault_tx(kFaultTreeState, -1, (int)(wit - first)));
         if (with_x)
-            bulk_x<X>(ta, lay, sm, w, xb, xbar + xb, xt, kTcThreads);
+            bulk_x<X>(ta, lay, sm, w, xb, xbar + xb, xt, kTcThreads,
+                      fault_tx(kFaultTreeX, -1, (int)(wit - first)));
         s_out = 1;
         if (with_x)
             x_out |= 1u << xb;
@@ -1221,17 +1232,25 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
         }
         if (!xasync)
             stage_x_plain<kTcThreads>(ta, xs, u);
+        // a copy counts as landed (its in-flight bit cleared) only once its wait succeeded,
+        // so that after a give-up the final drain waits for it again
         bool landed = true;
         if (s_out) {
-            landed = mbar_wait(sbar, sph);
-            sph ^= 1u;
-            s_out = 0;
+            if (mbar_wait(sbar, sph)) {
+                sph ^= 1u;
+                s_out = 0;
+            } else {
+                landed = false;
+            }
         }
         const int xb = xbuf_of(it);
         if ((x_out >> xb) & 1u) {
-            landed = mbar_wait(xbar + xb, (xph >> xb) & 1u) && landed;
-            xph ^= 1u << xb;
-            x_out &= ~(1u << xb);
+            if (mbar_wait(xbar + xb, (xph >> xb) & 1u)) {
+                xph ^= 1u << xb;
+                x_out &= ~(1u << xb);
+            } else {
+                landed = false;
+            }
         }
         if (__syncthreads_or(!landed)) { // state rows and x tile have landed
             if (tid == 0 && a.err)
@@ -1243,7 +1262,7 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
         fence_async_smem();              // operands visible to the tensor cores
         node_values(ta, sdA, sdt, u, dt_next, hv);
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0 && !fault_tx(kFaultTreeMma, -1, (int)(it - first))) {
             tc_fence_after();
             const uint32_t base = smem_u32(sm);
             uint32_t acc = 0;
@@ -1286,12 +1305,13 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
                 ps[e] = fmaf(cf, xv[e], ps[e]);
         }
         const bool ok = mbar_wait(bar, phase);
-        phase ^= 1u;
         if (__syncthreads_or(!ok)) {     // the MMAs never completed: give up on the launch
             if (tid == 0 && a.err)
                 atomicOr(a.err, SSU_FLAG_TIMEOUT);
+            mma_out = true;
             break;
         }
+        phase ^= 1u;
         tc_fence_after();
         float dv[16];
         tmem_ld16(taddr, dv);
@@ -1327,21 +1347,30 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
         }
         // Every read of this item's buffers done. Not needed when the x tile is double-
         // buffered and the next item is valid: until the next item's first barrier a
-        // thread writes only buffers the output copy-out does not read (the row's tables,
-        // the piece buffer), and this item's x tile is refilled only after that barrier.
+        // thread writes only buffers the output copy-out does not read (par, and by
+        // cp.async the C operand and the piece buffer: the invariant stated at
+        // stage_row_tc), and this item's x tile is refilled only after that barrier.
+        // The parity cases with several items per CTA crossing a (row, group) change
+        // (tests/test_gpu_ddtree.py, many rows over groups and dim tiles) run this path.
         if (!(x_mid && next_valid))
             __syncthreads();
         if (next_valid && xasync && !x_mid) {
-            bulk_x<X>(ta, lay, sm, v, 0, xbar, xt, kTcThreads);
+            bulk_x<X>(ta, lay, sm, v, 0, xbar, xt, kTcThreads,
+                      fault_tx(kFaultTreeX, -1, (int)(it + 1 - first)));
             x_out |= 1u;
         }
     }
-    // no copy outlives the CTA (only a launch that gave up leaves some in flight)
+    // No copy outlives the CTA and no MMA outlives its TMEM: after a give-up every copy
+    // still marked in flight and the awaited MMA phase are waited for once more (bounded).
+    // Should one of these waits run out as well (never expected), its copy may still
+    // write this CTA's shared memory, or its MMAs the released TMEM, after the CTA ends.
     if (s_out)
         mbar_wait(sbar, sph);
     for (int k = 0; k < 2; ++k)
         if ((x_out >> k) & 1u)
             mbar_wait(xbar + k, (xph >> k) & 1u);
+    if (mma_out)
+        mbar_wait(bar, phase);
     cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
@@ -1352,8 +1381,7 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
 // The tensor-core form when it applies (bf16 B and C with 16-byte aligned C, dstate 64 or
 // 128, layout within the shared-memory limit); -1 otherwise.
 template <typename S, typename X, int N>
-int launch_tc_x(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles, int xasync,
-                int sms)
+int launch_tc_x(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles, int xasync)
 {
     constexpr int es_x = (int)sizeof(X);
     int nxb = 2;
@@ -1364,28 +1392,18 @@ int launch_tc_x(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtil
     }
     if (lay.total > kSmemMax)
         return -1;
-    static int configured[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        dev = 0;
-    if (!configured[dev]) {
-        if (cudaFuncSetAttribute(ssu_ddtree_tc_kernel<S, X, N>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) !=
-            cudaSuccess)
-            return SSU_ERR_CUDA;
-        configured[dev] = 1;
-    }
+    const KernelFacts *f = kernel_facts<ssu_ddtree_tc_kernel<S, X, N>>(kTcThreads, kSmemMax);
+    if (!f || f->status != SSU_OK)
+        return SSU_ERR_CUDA;
     const int ocopy = (reinterpret_cast<uintptr_t>(a.d.out) & 15) == 0 &&
                       ((int64_t)a.d.Dm * es_x) % 16 == 0;
-    const int64_t grid = nitems < sms ? nitems : sms;
-    ssu_ddtree_tc_kernel<S, X, N><<<(unsigned)grid, kTcThreads, lay.total, stream>>>(
-        a, dtiles, nitems, nxb, xasync, ocopy);
-    return SSU_OK;
+    const int64_t grid = nitems < f->sms ? nitems : f->sms;
+    return launch_kernel(ssu_ddtree_tc_kernel<S, X, N>, (unsigned)grid, kTcThreads, lay.total,
+                         stream, a, dtiles, nitems, nxb, xasync, ocopy);
 }
 
 template <typename S, int N>
-int launch_tc(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles, int xasync,
-              int sms)
+int launch_tc(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles, int xasync)
 {
     if constexpr (N != 64 && N != 128) {
         return -1;
@@ -1393,9 +1411,9 @@ int launch_tc(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles
         if (a.d.bc_dtype != SSU_BF16 || (reinterpret_cast<uintptr_t>(a.d.C) & 15) != 0)
             return -1;
         switch (a.d.x_dtype) {
-        case SSU_F32: return launch_tc_x<S, float, N>(a, stream, nitems, dtiles, xasync, sms);
-        case SSU_F16: return launch_tc_x<S, __half, N>(a, stream, nitems, dtiles, xasync, sms);
-        default: return launch_tc_x<S, __nv_bfloat16, N>(a, stream, nitems, dtiles, xasync, sms);
+        case SSU_F32: return launch_tc_x<S, float, N>(a, stream, nitems, dtiles, xasync);
+        case SSU_F16: return launch_tc_x<S, __half, N>(a, stream, nitems, dtiles, xasync);
+        default: return launch_tc_x<S, __nv_bfloat16, N>(a, stream, nitems, dtiles, xasync);
         }
     }
 }
@@ -1412,16 +1430,7 @@ int launch_n(const TreeArgs &a, cudaStream_t stream)
     // x rows go through cp.async when every 16-byte chunk of a tile row is aligned
     const int xasync = (reinterpret_cast<uintptr_t>(a.d.x) & 15) == 0 &&
                        ((int64_t)a.d.Dm * es_x) % 16 == 0;
-    static int configured[64], sms[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        dev = 0;
-    if (!sms[dev]) {
-        int n = 0;
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        sms[dev] = n > 0 ? n : 148;
-    }
-    const int tc = launch_tc<S, N>(a, stream, nitems, dtiles, xasync, sms[dev]);
+    const int tc = launch_tc<S, N>(a, stream, nitems, dtiles, xasync);
     if (tc >= 0)
         return tc;
     int nxb = 2;
@@ -1432,17 +1441,12 @@ int launch_n(const TreeArgs &a, cudaStream_t stream)
     }
     if (lay.total > kSmemMax)
         return SSU_ERR_UNSUPPORTED;
-    if (!configured[dev]) {
-        if (cudaFuncSetAttribute(ssu_ddtree_kernel<S, N>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) !=
-            cudaSuccess)
-            return SSU_ERR_CUDA;
-        configured[dev] = 1;
-    }
-    const int64_t grid = nitems < sms[dev] ? nitems : sms[dev];
-    ssu_ddtree_kernel<S, N><<<(unsigned)grid, kThreads, lay.total, stream>>>(a, dtiles, nitems,
-                                                                            nxb, xasync);
-    return SSU_OK;
+    const KernelFacts *f = kernel_facts<ssu_ddtree_kernel<S, N>>(kThreads, kSmemMax);
+    if (!f || f->status != SSU_OK)
+        return SSU_ERR_CUDA;
+    const int64_t grid = nitems < f->sms ? nitems : f->sms;
+    return launch_kernel(ssu_ddtree_kernel<S, N>, (unsigned)grid, kThreads, lay.total, stream, a,
+                         dtiles, nitems, nxb, xasync);
 }
 
 template <typename S>
@@ -1460,6 +1464,10 @@ int launch_s(const TreeArgs &a, cudaStream_t s)
 }
 
 }  // namespace
+
+#ifdef SSU_WAIT_TEST
+SSU_WAIT_FAULT_SETTER(wait_fault_set_ddtree)
+#endif
 
 int launch_ddtree(const TreeArgs &a, int state_dtype, cudaStream_t s)
 {

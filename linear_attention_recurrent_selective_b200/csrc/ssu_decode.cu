@@ -211,8 +211,10 @@ int launch_n(const DecodeArgs &a, cudaStream_t stream)
     if (nunits > 0x7fffffffLL)
         return SSU_ERR_SHAPE;
     const int grid = persistent_grid<ssu_decode_kernel<S, N>>(nunits);
-    ssu_decode_kernel<S, N><<<grid, kWarps * 32, kSmemBytes, stream>>>(a, (int)cph, (int)nunits);
-    return SSU_OK;
+    if (grid < 0)
+        return SSU_ERR_CUDA;
+    return launch_kernel(ssu_decode_kernel<S, N>, grid, kWarps * 32, kSmemBytes, stream, a,
+                         (int)cph, (int)nunits);
 }
 
 template <typename S>
@@ -230,6 +232,10 @@ int launch_s(const DecodeArgs &a, cudaStream_t s)
 }
 
 }  // namespace
+
+#ifdef SSU_WAIT_TEST
+SSU_WAIT_FAULT_SETTER(wait_fault_set_decode)
+#endif
 
 int launch_decode(const DecodeArgs &a, int state_dtype, cudaStream_t s)
 {

@@ -231,11 +231,17 @@ int launch_k(const GdnArgs &a, cudaStream_t stream)
     if (nunits > 0x7fffffffLL)
         return SSU_ERR_SHAPE;
     const int grid = persistent_grid<gdn_decode_kernel<K>>(nunits);
-    gdn_decode_kernel<K><<<grid, kWarps * 32, kSmemBytes, stream>>>(a, (int)cph, (int)nunits);
-    return SSU_OK;
+    if (grid < 0)
+        return SSU_ERR_CUDA;
+    return launch_kernel(gdn_decode_kernel<K>, grid, kWarps * 32, kSmemBytes, stream, a,
+                         (int)cph, (int)nunits);
 }
 
 }  // namespace
+
+#ifdef SSU_WAIT_TEST
+SSU_WAIT_FAULT_SETTER(wait_fault_set_gdn)
+#endif
 
 int launch_gdn_decode(const GdnArgs &a, cudaStream_t s)
 {

@@ -126,8 +126,8 @@ int launch_clear(void *pool, int64_t bytes, cudaStream_t s)
 {
     if (bytes <= 0)
         return SSU_OK;
-    clear_kernel<<<grid_for(bytes), kPoolThreads, 0, s>>>(static_cast<uint8_t *>(pool), bytes);
-    return SSU_OK;
+    return launch_kernel(clear_kernel, grid_for(bytes), kPoolThreads, 0, s,
+                         static_cast<uint8_t *>(pool), bytes);
 }
 
 int launch_clear_layers(const ssu_layer_states *layers, int32_t num_layers, int32_t P,
@@ -141,9 +141,8 @@ int launch_clear_layers(const ssu_layer_states *layers, int32_t num_layers, int3
         return SSU_ERR_SHAPE;
     const int64_t want = (per / 16 + kPoolThreads - 1) / kPoolThreads;
     const unsigned gx = (unsigned)(want < 1 ? 1 : (want < 64 ? want : 64));
-    clear_layers_kernel<<<dim3(gx, 2 * num_layers), kPoolThreads, 0, s>>>(layers, slot, P,
-                                                                           rec_bytes, conv_bytes);
-    return SSU_OK;
+    return launch_kernel(clear_layers_kernel, dim3(gx, 2 * num_layers), kPoolThreads, 0, s,
+                         layers, slot, P, rec_bytes, conv_bytes);
 }
 
 int launch_gather(const void *pool, int64_t slot_bytes, int32_t P, void *dense,
@@ -153,20 +152,17 @@ int launch_gather(const void *pool, int64_t slot_bytes, int32_t P, void *dense,
         return SSU_ERR_SHAPE;
     const int64_t want = (slot_bytes / 16 + kPoolThreads - 1) / kPoolThreads;
     const unsigned gx = (unsigned)(want < 1 ? 1 : (want < 32 ? want : 32));
-    gather_kernel<<<dim3(gx, active), kPoolThreads, 0, s>>>(
-        static_cast<const uint8_t *>(pool), slot_bytes, P, static_cast<uint8_t *>(dense), idx,
-        scatter, err);
-    return SSU_OK;
+    return launch_kernel(gather_kernel, dim3(gx, active), kPoolThreads, 0, s,
+                         static_cast<const uint8_t *>(pool), slot_bytes, P,
+                         static_cast<uint8_t *>(dense), idx, scatter, err);
 }
 
 int launch_copy(void *dst, const void *src, int64_t bytes, cudaStream_t s)
 {
     if (bytes <= 0 || dst == src)
         return SSU_OK;
-    copy_kernel<<<grid_for(bytes), kPoolThreads, 0, s>>>(static_cast<uint8_t *>(dst),
-                                                          static_cast<const uint8_t *>(src),
-                                                          bytes);
-    return SSU_OK;
+    return launch_kernel(copy_kernel, grid_for(bytes), kPoolThreads, 0, s,
+                         static_cast<uint8_t *>(dst), static_cast<const uint8_t *>(src), bytes);
 }
 
 }  // namespace ssu

@@ -196,7 +196,8 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles, const int rtc, const 
             if (tid == 0) {
                 uint64_t *bar = &full[c & 1];
                 const uint32_t nb = (uint32_t)(N * es_bc), nx = (uint32_t)(rows_c * es_x);
-                mbar_arrive_expect_tx(bar, 2u * nt * nb + (a.z ? 2u : 1u) * nt * nx);
+                mbar_arrive_expect_tx(bar, 2u * nt * nb + (a.z ? 2u : 1u) * nt * nx +
+                                               fault_tx(kFaultPrefill, -1, c));
                 if (G == 1) {
                     bulk_load(raw + lay.raw_b, Bg + bt0 * nb, nt * nb, bar);
                     bulk_load(raw + lay.raw_c, Cg + bt0 * nb, nt * nb, bar);
@@ -271,13 +272,13 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles, const int rtc, const 
         const uint8_t *raw = sm + (c & 1) * lay.raw_bytes;
         if (bulk) {
             if (!__syncthreads_and(mbar_wait(&full[c & 1], (uint32_t)(c >> 1) & 1u))) {
-                // Never expected: report, let the copies already started land, stop.
+                // Never expected: report, wait (bounded) for both chunks in flight so
+                // that their copies land before the CTA ends, stop.
                 if (tid == 0) {
                     if (a.err)
                         atomicOr(a.err, SSU_FLAG_TIMEOUT);
                     for (int cc = c; cc < min(c + 2, nchunks); ++cc)
-                        if (!mbar_wait(&full[cc & 1], (uint32_t)(cc >> 1) & 1u))
-                            break;
+                        mbar_wait(&full[cc & 1], (uint32_t)(cc >> 1) & 1u);
                 }
                 return;
             }
@@ -407,6 +408,13 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles, const int rtc, const 
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Shared memory of the largest prefill layout at dstate N (fp32 B/C, x and z).
+template <int N>
+int smem_limit()
+{
+    return PLayout(N, kWarpsPerCta * PGeo<N>::RW, 4, 4).total;
+}
+
 template <typename S, int N>
 int launch_n(const PrefillArgs &a, cudaStream_t s)
 {
@@ -428,18 +436,12 @@ int launch_n(const PrefillArgs &a, cudaStream_t s)
     const int bulk = aligned16(a.d.x) && (!a.d.z || aligned16(a.d.z)) &&
                      (Dm * es_x) % 16 == 0 && (rtc * es_x) % 16 == 0;
     const PLayout lay(N, rtc, es_bc, es_x);
-    static int configured[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        dev = 0;
-    if (configured[dev] < lay.total) {
-        cudaFuncSetAttribute(ssu_prefill_kernel<S, N>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
-        configured[dev] = lay.total;
-    }
-    ssu_prefill_kernel<S, N><<<(unsigned)grid, warps * 32, lay.total, s>>>(a, (int)dtiles, rtc,
-                                                                          bulk);
-    return SSU_OK;
+    // the limit is raised once to the largest layout any dtype combination needs
+    const KernelFacts *f = kernel_facts<ssu_prefill_kernel<S, N>>(warps * 32, smem_limit<N>());
+    if (!f || f->status != SSU_OK || lay.total > smem_limit<N>())
+        return SSU_ERR_CUDA;
+    return launch_kernel(ssu_prefill_kernel<S, N>, (unsigned)grid, warps * 32, lay.total, s, a,
+                         (int)dtiles, rtc, bulk);
 }
 
 template <typename S>
@@ -457,6 +459,10 @@ int launch_s(const PrefillArgs &a, cudaStream_t s)
 }
 
 }  // namespace
+
+#ifdef SSU_WAIT_TEST
+SSU_WAIT_FAULT_SETTER(wait_fault_set_prefill)
+#endif
 
 int launch_prefill(const PrefillArgs &a, int state_dtype, cudaStream_t s)
 {

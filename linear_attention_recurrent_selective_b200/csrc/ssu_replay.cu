@@ -289,9 +289,10 @@ int launch_n(const ReplayArgs &a, cudaStream_t stream)
     if (nunits > 0x7fffffffLL)
         return SSU_ERR_SHAPE;
     const int grid = persistent_grid<ssu_replay_kernel<S, N>>(nunits);
-    ssu_replay_kernel<S, N><<<grid, kWarps * 32, kSmemBytes, stream>>>(a, (int)cph, (int)upl,
-                                                                       (int)nunits);
-    return SSU_OK;
+    if (grid < 0)
+        return SSU_ERR_CUDA;
+    return launch_kernel(ssu_replay_kernel<S, N>, grid, kWarps * 32, kSmemBytes, stream, a,
+                         (int)cph, (int)upl, (int)nunits);
 }
 
 template <typename S>
@@ -309,6 +310,10 @@ int launch_s(const ReplayArgs &a, cudaStream_t s)
 }
 
 }  // namespace
+
+#ifdef SSU_WAIT_TEST
+SSU_WAIT_FAULT_SETTER(wait_fault_set_replay)
+#endif
 
 int launch_replay(const ReplayArgs &a, int state_dtype, cudaStream_t s)
 {

@@ -159,14 +159,17 @@ template <typename G, int N, typename Rows> struct Producer {
         w.ctl->slot[s] = cur.slot;
         w.ctl->extra[s] = cur.extra;
         w.ctl->moves[s] = rows.moves(cur);
+        const uint32_t extra = fault_tx(kFaultStream, (int)(threadIdx.x >> 5), issued);
         if (w.ctl->moves[s]) {
             const int nr = min(G::RT, un.rows - j * G::RT);
             const uint32_t bytes = (uint32_t)(nr * G::ROW_BYTES);
             const char *src = cur.pool + ((int64_t)cur.slot * slot_stride +
                                           ((int64_t)un.h * Dm + un.row0 + j * G::RT) * N) *
                                              G::ELEM;
-            mbar_arrive_expect_tx(&w.ctl->full[s], bytes);
+            mbar_arrive_expect_tx(&w.ctl->full[s], bytes + extra);
             bulk_load(w.ring + s * kTileBytes, src, bytes, &w.ctl->full[s]);
+        } else if (extra) {
+            mbar_arrive_expect_tx(&w.ctl->full[s], extra);
         } else {
             mbar_arrive(&w.ctl->full[s]);
         }
@@ -238,8 +241,10 @@ __device__ __forceinline__ void init_ring(const WarpViews &w, int lane)
     __syncwarp();
 }
 
-// Wait for consumed-tile number c; on a (never expected) timeout, report it, let the
-// copies this warp started land and return false. The verdict is warp-uniform.
+// Wait for consumed-tile number c; on a (never expected) timeout, report it, wait (each
+// wait bounded again) for every tile this warp still has in flight, so that no copy
+// outlives the warp unless its barrier also gives up, and return false. The verdict is
+// warp-uniform.
 __device__ __forceinline__ bool wait_tile(const WarpViews &w, int c, int issued_lane0,
                                           int lane, int32_t *err)
 {
@@ -250,31 +255,20 @@ __device__ __forceinline__ bool wait_tile(const WarpViews &w, int c, int issued_
         atomicOr(err, SSU_FLAG_TIMEOUT);
     const int issued = __shfl_sync(0xffffffffu, issued_lane0, 0);
     for (int cc = c; cc < issued; ++cc)
-        if (!mbar_wait(&w.ctl->full[cc % kStages], (uint32_t)(cc / kStages) & 1u))
-            break;
+        mbar_wait(&w.ctl->full[cc % kStages], (uint32_t)(cc / kStages) & 1u);
     return false;
 }
 
-// Grid size for a persistent launch: as many CTAs as fit, no more than the work needs.
-// One instantiation (and one cache of the occupancy query) per kernel.
+// Grid size for a persistent launch: as many CTAs as fit, no more than the work needs;
+// -1 when the device could not be queried (the launcher then reports SSU_ERR_CUDA).
 template <auto kernel>
 int persistent_grid(int64_t nunits)
 {
-    static int blocks_per_sm[64];
-    static int sms[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        dev = 0;
-    if (blocks_per_sm[dev] == 0) {
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        int occ = 0, n = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kWarps * 32, kSmemBytes);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        sms[dev] = n > 0 ? n : 148;
-        blocks_per_sm[dev] = occ > 0 ? occ : 1;
-    }
+    const KernelFacts *f = kernel_facts<kernel>(kWarps * 32, kSmemBytes);
+    if (!f || f->status != SSU_OK)
+        return -1;
     const int64_t want = (nunits + kWarps - 1) / kWarps;
-    const int64_t cap = (int64_t)sms[dev] * blocks_per_sm[dev];
+    const int64_t cap = (int64_t)f->sms * f->blocks_per_sm;
     return (int)(want < cap ? want : cap);
 }
 

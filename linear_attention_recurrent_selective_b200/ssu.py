@@ -42,11 +42,13 @@ FLAG_NEGATIVE_LENGTH = 8
 FLAG_TIMEOUT = 16
 FLAG_LAYER = 32
 FLAG_TREE = 64
+FLAG_DUPLICATE_INDEX = 128
 
 # Every C entry point declared in include/ssu.h, in declaration order.
 ENTRY_POINTS = ("ssu_decode", "ssu_prefill", "ssu_replay", "ssu_replay_layers",
-                "ssu_conv_decode", "gdn_decode", "ssu_ddtree", "pool_clear_slot", "pool_copy_slot", "pool_clear_slot_layers",
-                "pool_gather", "pool_scatter", "ssu_status_string")
+                "ssu_conv_decode", "gdn_decode", "ssu_ddtree", "pool_clear_slot",
+                "pool_copy_slot", "pool_clear_slot_layers", "pool_gather", "pool_scatter",
+                "ssu_check_state_indices", "ssu_status_string")
 
 # Byte layouts of the per-layer pointer records of include/ssu.h (packed pointers).
 REPLAY_LAYER_FIELDS = 5     # state, st_dA, st_U, st_B, st_dt
@@ -71,16 +73,22 @@ _lib = None
 def lib() -> ctypes.CDLL:
     """The loaded library with argument types declared (loads it on first use)."""
     global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
+    if _lib is None:
+        _lib = load(LIB_PATH)
+    return _lib
+
+
+def load(path: str) -> ctypes.CDLL:
+    """Load a build of the library (libssu.so, or the test suite's libssu_waittest.so,
+    which exports the same entry points) and declare the entry points' argument types."""
+    if not os.path.exists(path):
         raise SSULibraryMissing(
-            f"{LIB_PATH} is missing: build it with "
+            f"{path} is missing: build it with "
             "`python -m linear_attention_recurrent_selective_b200.build`")
     try:
-        L = ctypes.CDLL(LIB_PATH)
+        L = ctypes.CDLL(path)
     except OSError as e:
-        raise SSULibraryMissing(f"cannot load {LIB_PATH}: {e}") from e
+        raise SSULibraryMissing(f"cannot load {path}: {e}") from e
     vp, i32, i64, ci = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int
     L.ssu_decode.argtypes = [vp, ci, vp, vp, vp, ci, vp, vp, vp, vp, vp, ci, i64, i32, vp, vp,
                              i32, i32, i32, i32, i32, i32, ci, vp, vp]
@@ -102,12 +110,25 @@ def lib() -> ctypes.CDLL:
     L.pool_clear_slot_layers.argtypes = [vp, i32, i32, i32, i64, i64, vp]
     L.pool_gather.argtypes = [vp, i64, i32, vp, vp, i32, i32, vp, vp]
     L.pool_scatter.argtypes = [vp, vp, i64, i32, vp, i32, i32, vp, vp]
+    L.ssu_check_state_indices.argtypes = [vp, i32, i32, i32, vp, vp]
     for f in ENTRY_POINTS[:-1]:
         getattr(L, f).restype = ci
     L.ssu_status_string.argtypes = [ci]
     L.ssu_status_string.restype = ctypes.c_char_p
-    _lib = L
     return L
+
+
+# Debug mode: when on, every call that takes state_indices first checks them with
+# check_state_indices (which synchronises, so it cannot run under CUDA-graph capture).
+_debug_checks = os.environ.get("SSU_DEBUG_CHECKS", "") not in ("", "0")
+
+
+def set_debug_checks(enabled: bool) -> bool:
+    """Turn the debug check of state_indices before every call on or off (also set by the
+    environment variable SSU_DEBUG_CHECKS=1). Returns the previous setting."""
+    global _debug_checks
+    before, _debug_checks = _debug_checks, bool(enabled)
+    return before
 
 
 def _check(fn: str, status: int) -> None:
@@ -157,6 +178,43 @@ def _dt(t: torch.Tensor, name: str) -> int:
         raise ValueError(f"{name} dtype {t.dtype} is not fp32, fp16 or bf16") from None
 
 
+def ssu_check_state_indices(state_indices, P, err_flags, *, active_batch=None, stream=None):
+    """Enqueue the library's check of a row-to-slot map: ORs FLAG_DUPLICATE_INDEX into
+    err_flags when two active rows name the same slot (>= 0), FLAG_INDEX_RANGE when one
+    names a slot >= P. Asynchronous, like every entry point."""
+    batch = state_indices.shape[0]
+    active = batch if active_batch is None else active_batch
+    rc = lib().ssu_check_state_indices(
+        _ptr(state_indices, "state_indices", torch.int32), batch, active, P,
+        _ptr(err_flags, "err_flags", torch.int32), _stream(stream))
+    _check("ssu_check_state_indices", rc)
+
+
+def check_state_indices(state_indices, P, *, active_batch=None, stream=None) -> None:
+    """Debug helper: run the library's check on ``stream``, wait for it and raise
+    ValueError when the active rows' indices repeat a slot or leave the pool. It
+    synchronises the stream, so it is not for use under CUDA-graph capture."""
+    if state_indices is None:
+        return
+    flags = torch.zeros(1, dtype=torch.int32, device=state_indices.device)
+    ssu_check_state_indices(state_indices, P, flags, active_batch=active_batch, stream=stream)
+    s = torch.cuda.current_stream(state_indices.device) if stream is None else stream
+    s.synchronize()
+    f = int(flags.item())
+    problems = []
+    if f & FLAG_DUPLICATE_INDEX:
+        problems.append("two active rows share a pool slot")
+    if f & FLAG_INDEX_RANGE:
+        problems.append(f"an active row's slot is >= P ({P})")
+    if problems:
+        raise ValueError("state_indices: " + "; ".join(problems))
+
+
+def _debug_indices(state_indices, P, active, stream):
+    if _debug_checks and state_indices is not None:
+        check_state_indices(state_indices, P, active_batch=active, stream=stream)
+
+
 def ssu_decode(x, A, B, C, dt, state, out, *, dt_bias=None, D=None, z=None,
                state_indices=None, active_batch=None, dt_softplus=True, err_flags=None,
                slot_stride=None, P=None, stream=None):
@@ -170,6 +228,7 @@ def ssu_decode(x, A, B, C, dt, state, out, *, dt_bias=None, D=None, z=None,
         raise ValueError("z must have x's dtype")
     if out.dtype != x.dtype or out.shape != x.shape:
         raise ValueError("out must match x in shape and dtype")
+    _debug_indices(state_indices, P, active, stream)
     rc = lib().ssu_decode(
         _ptr(x, "x"), _dt(x, "x"), _ptr(A, "A", torch.float32), _ptr(B, "B"), _ptr(C, "C", B.dtype),
         _dt(B, "B"), _ptr(dt, "dt", torch.float32), _ptr(dt_bias, "dt_bias", torch.float32),
@@ -197,6 +256,7 @@ def ssu_prefill(x, A, B, C, dt, state, out, *, dt_bias=None, D=None, z=None,
         raise ValueError("out must match x in shape and dtype")
     f32 = torch.float32
     sdA, sU, sB, sdt = stash if stash is not None else (None, None, None, None)
+    _debug_indices(state_indices, P, active, stream)
     rc = lib().ssu_prefill(
         _ptr(x, "x"), _dt(x, "x"), _ptr(A, "A", f32), _ptr(B, "B"), _ptr(C, "C", B.dtype),
         _dt(B, "B"), _ptr(dt, "dt", f32), _ptr(dt_bias, "dt_bias", f32), _ptr(D, "D", f32),
@@ -229,6 +289,7 @@ def ssu_replay(state, stash, accepted_lengths, *, state_indices=None, active_bat
     active = batch if active_batch is None else active_batch
     stride, P = _pool_geometry(state, slot_stride, P, H * Dm * N)
     f32 = torch.float32
+    _debug_indices(state_indices, P, active, stream)
     rc = lib().ssu_replay(
         ctypes.c_void_p(state.data_ptr()), _dt(state, "state"), stride, P,
         _ptr(sdA, "stash dA", f32), _ptr(sU, "stash U", f32), _ptr(sB, "stash B", f32),
@@ -260,6 +321,7 @@ def ssu_conv_decode(xbc, conv_weight, conv_state, A, dt, state, out, *, width, c
         raise ValueError("conv_state must have xbc's dtype")
     cs, cc, ck = conv_strides
     f32 = torch.float32
+    _debug_indices(state_indices, P, active, stream)
     rc = lib().ssu_conv_decode(
         _ptr(xbc, "xbc"), _dt(xbc, "xbc"), _ptr(conv_weight, "conv_weight"),
         _ptr(conv_bias, "conv_bias"),
@@ -291,6 +353,7 @@ def gdn_decode(q, k, v, a, b, A_log, state, out, *, dt_bias=None, scale=None,
     if tuple(out.shape) != (batch, HV, V):
         raise ValueError("out must be [batch, HV, V]")
     f32 = torch.float32
+    _debug_indices(state_indices, P, active, stream)
     rc = lib().gdn_decode(
         _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _dt(q, "q"), _ptr(a, "a"), _ptr(b, "b"),
         _ptr(A_log, "A_log", f32), _ptr(dt_bias, "dt_bias", f32), float(scale or 0.0),
@@ -316,6 +379,7 @@ def ssu_ddtree(x, A, B, C, dt, state, out, parent_ids, depths, stash, *, dt_bias
         raise ValueError("out must match x in shape and dtype")
     f32, i32 = torch.float32, torch.int32
     sdA, sU, sB, sdt = stash
+    _debug_indices(state_indices, P, active, stream)
     rc = lib().ssu_ddtree(
         _ptr(x, "x"), _dt(x, "x"), _ptr(A, "A", f32), _ptr(B, "B"), _ptr(C, "C", B.dtype),
         _dt(B, "B"), _ptr(dt, "dt", f32), _ptr(dt_bias, "dt_bias", f32), _ptr(D, "D", f32),
@@ -390,6 +454,7 @@ def ssu_replay_layers(table, num_layers, like_state, like_stash, accepted_length
     G, N = sB.shape[2], sB.shape[3]
     active = batch if active_batch is None else active_batch
     stride, P = _pool_geometry(like_state, slot_stride, P, H * Dm * N)
+    _debug_indices(state_indices, P, active, stream)
     rc = lib().ssu_replay_layers(
         _ptr(table, "layer table", torch.int64), num_layers, _dt(like_state, "state"), stride,
         P, _ptr(accepted_lengths, "accepted_lengths", torch.int32),
@@ -418,6 +483,7 @@ def pool_gather(pool, dense, *, state_indices=None, active_batch=None, err_flags
         P = pool.shape[0]
     if not (pool.is_cuda and dense.is_cuda and dense.is_contiguous()):
         raise ValueError("pool and dense must be CUDA tensors, dense contiguous")
+    _debug_indices(state_indices, P, active, stream)
     rc = lib().pool_gather(ctypes.c_void_p(pool.data_ptr()), slot_bytes, P,
                            ctypes.c_void_p(dense.data_ptr()),
                            _ptr(state_indices, "state_indices", torch.int32), batch, active,
@@ -435,6 +501,7 @@ def pool_scatter(dense, pool, *, state_indices=None, active_batch=None, err_flag
         P = pool.shape[0]
     if not (pool.is_cuda and dense.is_cuda and dense.is_contiguous()):
         raise ValueError("pool and dense must be CUDA tensors, dense contiguous")
+    _debug_indices(state_indices, P, active, stream)
     rc = lib().pool_scatter(ctypes.c_void_p(dense.data_ptr()), ctypes.c_void_p(pool.data_ptr()),
                             slot_bytes, P, _ptr(state_indices, "state_indices", torch.int32),
                             batch, active, _ptr(err_flags, "err_flags", torch.int32),

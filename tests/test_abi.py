@@ -13,8 +13,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "ssu.h")
 
 
-def declared_functions():
-    text = open(HEADER).read()
+def declared_functions(header=HEADER):
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
 
@@ -33,6 +33,24 @@ def test_header_declares_the_entry_points():
 def test_library_exports_every_declared_symbol(L):
     for name in declared_functions():
         assert hasattr(L, name), name
+
+
+WAIT_TEST_HEADER = os.path.join(ROOT, "include", "ssu_wait_test.h")
+
+
+def test_product_library_has_no_test_hooks(L):
+    assert declared_functions(WAIT_TEST_HEADER) == ["ssu_test_wait_fault"]
+    for name in declared_functions(WAIT_TEST_HEADER):
+        assert not hasattr(L, name), name
+
+
+def test_wait_test_library_exports_both_headers():
+    """The test library (same sources, SSU_WAIT_TEST) exports every product entry point and
+    the test hook of include/ssu_wait_test.h."""
+    from linear_attention_recurrent_selective_b200 import build
+    T = ssu.load(build.build(waittest=True))
+    for name in declared_functions() + declared_functions(WAIT_TEST_HEADER):
+        assert hasattr(T, name), name
 
 
 def test_status_strings(L):
@@ -159,3 +177,11 @@ def test_gdn_rejects_bad_arguments(L):
     assert call(x_dt=7) == 3 and call(K=96, stride=32 * 128 * 96) == 4
     assert call(state=ctypes.c_void_p(264)) == 6
     assert call(active=0, q=None, k=None, v=None, state=None) == 0
+
+
+@pytest.mark.parametrize("idx,batch,active,P,err,status", [
+    (None, 4, 4, 8, P16, 1), (P16, 4, 4, 8, None, 1), (P16, 4, 5, 8, P16, 2),
+    (P16, 4, -1, 8, P16, 2), (P16, 4, 4, -1, P16, 2), (None, 4, 0, 8, None, 0),
+])
+def test_check_state_indices_host_validation(L, idx, batch, active, P, err, status):
+    assert L.ssu_check_state_indices(idx, batch, active, P, err, None) == status
