@@ -265,7 +265,7 @@ def run_decode(args, device):
     # ---- clock record over a longer window (not part of the reported value): the same
     # step back to back for at least 0.5 s, NVML sampled every 5 ms, so that the clock the
     # kernel ran at rests on many samples even when the timed region above is short
-    n_sus = max(10, int(0.6 / max(kern_ms / 1e3, 1e-6)))
+    n_sus = 0 if args.no_clock_window else max(10, int(0.6 / max(kern_ms / 1e3, 1e-6)))
     sus = ClockSampler(device.index, period_s=0.005).start()
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(device)
@@ -279,7 +279,7 @@ def run_decode(args, device):
     torch.cuda.synchronize(device)
     w1 = time.perf_counter()
     sus.stop()
-    sus_ms = s0.elapsed_time(s1) / n_sus
+    sus_ms = s0.elapsed_time(s1) / max(n_sus, 1)
     res["clocks_sustained"] = {**sus.summary(w0, w1), "steps": n_sus,
                                "seconds": round(w1 - w0, 3), "ms_per_step": sus_ms}
 
@@ -818,6 +818,9 @@ def parse(argv=None):
                     default="all",
                     help="run one kernel only (for profiling); its line carries that form")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clock-window", action="store_true",
+                    help="skip the >= 0.5 s clock-sampling window after the timed region "
+                         "(for profiler runs)")
     a = ap.parse_args(argv)
     if a.warmup < 3 and a.impl == "ours":
         ap.error("--warmup must be at least 3")
