@@ -262,27 +262,6 @@ def run_decode(args, device):
     res = dict(case=case, units=units, total_ms=total_ms, kern_ms=kern_ms, state_b=state_b,
                alg_b=alg_b, clocks=clocks.summary(wall0, wall1), flush=flush, l2=l2)
 
-    # ---- clock record over a longer window (not part of the reported value): the same
-    # step back to back for at least 0.5 s, NVML sampled every 5 ms, so that the clock the
-    # kernel ran at rests on many samples even when the timed region above is short
-    n_sus = 0 if args.no_clock_window else max(10, int(0.6 / max(kern_ms / 1e3, 1e-6)))
-    sus = ClockSampler(device.index, period_s=0.005).start()
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize(device)
-    w0 = time.perf_counter()
-    s0.record(stream)
-    for _ in range(n_sus):
-        if flush:
-            flush_buf.zero_()
-        step()
-    s1.record(stream)
-    torch.cuda.synchronize(device)
-    w1 = time.perf_counter()
-    sus.stop()
-    sus_ms = s0.elapsed_time(s1) / max(n_sus, 1)
-    res["clocks_sustained"] = {**sus.summary(w0, w1), "steps": n_sus,
-                               "seconds": round(w1 - w0, 3), "ms_per_step": sus_ms}
-
     # ---- end to end through the binding: pinned host inputs in, output back out.
     # Every step copies its inputs from pinned host memory and reads its output back; the
     # copies run on their own streams, double-buffered, so that step k+1's inputs arrive
@@ -332,6 +311,27 @@ def run_decode(args, device):
     res["e2e_ms"] = e0.elapsed_time(e1)
     res["h2d"] = sum(v.numel() * v.element_size() for v in host.values())
     res["d2h"] = outs_h[0].numel() * outs_h[0].element_size()
+
+    # ---- clock record over a longer window (not part of the reported value): the same
+    # step back to back for at least 0.5 s, NVML sampled every 5 ms, so that the clock the
+    # kernel ran at rests on many samples even when the timed region above is short
+    n_sus = 0 if args.no_clock_window else max(10, int(0.6 / max(kern_ms / 1e3, 1e-6)))
+    sus = ClockSampler(device.index, period_s=0.005).start()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    w0 = time.perf_counter()
+    s0.record(stream)
+    for _ in range(n_sus):
+        if flush:
+            flush_buf.zero_()
+        step()
+    s1.record(stream)
+    torch.cuda.synchronize(device)
+    w1 = time.perf_counter()
+    sus.stop()
+    sus_ms = s0.elapsed_time(s1) / max(n_sus, 1)
+    res["clocks_sustained"] = {**sus.summary(w0, w1), "steps": n_sus,
+                               "seconds": round(w1 - w0, 3), "ms_per_step": sus_ms}
     return res
 
 
