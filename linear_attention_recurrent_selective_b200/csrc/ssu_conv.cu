@@ -32,7 +32,7 @@ using namespace stream;
 constexpr int kUT = 8;   // units of up to 8 tiles, as in the decode
 constexpr int kMaxConvWidth = 16;   // the widest window ssu_conv_decode accepts
 
-struct ConvRows {
+struct ConvRows : UnitsInOrder {
     const void *pool;
     const int32_t *idx;
     int32_t P;
@@ -96,7 +96,7 @@ ssu_conv_decode_kernel(const __grid_constant__ ConvArgs ca, const int cph, const
     const int nw = gridDim.x * kWarps;
     const int first = (int)((int64_t)nunits * gw / nw);
     const int last = (int)((int64_t)nunits * (gw + 1) / nw);
-    const ConvRows rows{a.state, a.idx, a.P};
+    const ConvRows rows{{}, a.state, a.idx, a.P};
     Producer<G, N, ConvRows> prod;
     if (lane == 0) {
         prod.start(rows, first, 1, nunits, cph, last, H, Dm);

@@ -37,7 +37,7 @@ using namespace stream;
 // so its metadata is loaded once per 64 KB of traffic.
 constexpr int kUT = 8;
 
-struct DecodeRows {
+struct DecodeRows : UnitsInOrder {
     const void *pool;
     const int32_t *idx;
     int32_t P;
@@ -67,7 +67,7 @@ ssu_decode_kernel(const DecodeArgs a, const int cph, const int nunits)
     const int H = a.H, Dm = a.Dm, hpg = H / a.G;
     const int gw = blockIdx.x * kWarps + warp;
     const int nw = gridDim.x * kWarps;
-    const DecodeRows rows{a.state, a.idx, a.P};
+    const DecodeRows rows{{}, a.state, a.idx, a.P};
     Producer<G, N, DecodeRows> prod;
     if (lane == 0) {
         prod.start(rows, gw, nw, nunits, cph, nunits, H, Dm);

@@ -28,7 +28,7 @@ using namespace stream;
 
 constexpr int kUT = 8;
 
-struct GdnRows {
+struct GdnRows : UnitsInOrder {
     const void *pool;
     const int32_t *idx;
     int32_t P;
@@ -67,7 +67,7 @@ gdn_decode_kernel(const __grid_constant__ GdnArgs a, const int cph, const int nu
     const int H = a.HV, Dm = a.V, vpk = a.HV / a.HK;
     const int gw = blockIdx.x * kWarps + warp;
     const int nw = gridDim.x * kWarps;
-    const GdnRows rows{a.state, a.idx, a.P};
+    const GdnRows rows{{}, a.state, a.idx, a.P};
     Producer<G, K, GdnRows> prod;
     if (lane == 0) {
         prod.start(rows, gw, nw, nunits, cph, nunits, H, Dm);

@@ -18,7 +18,7 @@
 //   * the update and the output sums use the packed two-wide FP32 instructions of sm_100
 //     (__fmul2_rn / __ffma2_rn, element-wise round-to-nearest, so every element is
 //     computed exactly as fmaf(s, dA, B * (dt * x)) and the state matches the decode
-//     kernel bit for bit), with two partial sums per row to shorten dependency chains;
+//     kernel bit for bit), with four partial sums per row to shorten dependency chains;
 //   * inputs arrive per chunk of kTC tokens: B, C, x and z are fetched by the bulk-copy
 //     engine (cp.async.bulk, completion on an mbarrier, bounded waits) into a
 //     double-buffered raw stage one chunk ahead; B and C are widened to fp32 once per
@@ -49,7 +49,7 @@ constexpr int kRankMax = 32;    // batches up to this size are scheduled longest
 #define SSU_PREFILL_MIN_CTAS 4
 #endif
 #ifndef SSU_PREFILL_NA
-#define SSU_PREFILL_NA 2
+#define SSU_PREFILL_NA 4
 #endif
 #ifndef SSU_PREFILL_UNROLL_T
 #define SSU_PREFILL_UNROLL_T 1

@@ -21,7 +21,12 @@
 // With a handful of tokens per row the work is one read and one write of every touched
 // state row, so the kernel runs on the per-warp bulk-copy pipeline of ssu_stream.cuh;
 // rows with nothing accepted are never copied. The stash values are read through L1
-// (B and dA/dt are shared by all tiles of a unit).
+// (B and dA/dt are shared by all tiles of a unit). Units are numbered over the live rows
+// only (a valid slot, something accepted, node ids inside the stash): every CTA lists
+// them in shared memory from the device lengths at launch, so each warp gets the same
+// number of units that move state (within one) instead of a share of the batch in which
+// rows with nothing accepted leave holes; batches of more than kLiveMax rows are
+// numbered over all rows.
 #include "ssu_stream.cuh"
 
 namespace ssu {
@@ -29,17 +34,20 @@ namespace {
 
 using namespace stream;
 
-// Units of up to 2 tiles (8 KB): a replay touches few rows, and small units spread
-// them evenly over the warps of the grid. Both counts can be overridden at build time
-// for tuning sweeps.
+// Units of up to 4 tiles (16 KB). With units numbered over the live rows every warp
+// gets an even share anyway, so the unit only has to be long enough to hide the loads
+// of its first stashed tokens (measured on the batch-64 replay: 1 tile 0.072 ms, 2 tiles
+// 0.064 ms, 4 tiles 0.061 ms, 8 tiles 0.073 ms). Both counts can be overridden at build
+// time for tuning sweeps.
 #ifndef SSU_REPLAY_UT
-#define SSU_REPLAY_UT 2
+#define SSU_REPLAY_UT 4
 #endif
 #ifndef SSU_REPLAY_PRE
 #define SSU_REPLAY_PRE 4
 #endif
 constexpr int kUT = SSU_REPLAY_UT;
 constexpr int kPre = SSU_REPLAY_PRE;   // stashed tokens per unit held in registers
+constexpr int kLiveMax = 1024;         // batches up to this size number units over live rows
 
 // The lane's E columns of an fp32 [N] row, as 16-byte loads.
 template <typename G>
@@ -107,6 +115,14 @@ __device__ __forceinline__ int entry_of(const ReplayArgs &a, int b, int t)
 
 struct ReplayRows {
     const ReplayArgs *a;
+    const int *live;     // live rows (shared memory), or NULL: units over all active rows
+    __device__ __forceinline__ LUnit unit(int u, int upl, int cph, int CR, int H, int Dm) const
+    {
+        LUnit lu = lunit_at(u, upl, cph, CR, H, Dm);
+        if (live)
+            lu.un.b = live[lu.un.b];
+        return lu;
+    }
     __device__ __forceinline__ UnitRes resolve(const LUnit &lu) const
     {
         const LayerPtrs L = layer_ptrs(*a, lu.layer);
@@ -131,14 +147,70 @@ struct ReplayRows {
     }
 };
 
+// The rows whose state moves, in row order, into list[]; returns their count. All
+// threads of the CTA take part. CTA 0 also reports every row's caller bugs (index >= P,
+// node id outside the stash, accepted length out of range) and every layer whose pointers
+// are unusable, since units of rows that do not move are never visited.
+__device__ int list_live_rows(const ReplayArgs &a, int *list, int *wcount)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool reporter = blockIdx.x == 0 && a.err;
+    if (reporter)
+        for (int l = tid; l < a.num_layers; l += kWarps * 32)
+            if (!layer_ptrs(a, l).ok)
+                atomicOr(a.err, SSU_FLAG_LAYER);
+    int total = 0;
+    for (int b0 = 0; b0 < a.active; b0 += kWarps * 32) {
+        const int b = b0 + tid;
+        bool live = false;
+        if (b < a.active) {
+            const int slot = a.idx ? a.idx[b] : b;
+            const int acc = a.acc[b];
+            const int k = min(acc, a.max_accept);
+            bool bad = false;
+            if (a.nodes && slot >= 0 && slot < a.P)
+                for (int t = 0; t < k && !bad; ++t) {
+                    const int e = a.nodes[(int64_t)b * a.max_accept + t];
+                    bad = e < 0 || e >= a.T;
+                }
+            live = slot >= 0 && slot < a.P && k > 0 && !bad;
+            if (reporter) {
+                if (slot >= a.P)
+                    atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
+                else if (slot >= 0 && bad)
+                    atomicOr(a.err, SSU_FLAG_TREE);
+                else if (slot >= 0 && acc > a.max_accept)
+                    atomicOr(a.err, SSU_FLAG_ACCEPTED_RANGE);
+                else if (slot >= 0 && acc < 0)
+                    atomicOr(a.err, SSU_FLAG_NEGATIVE_LENGTH);
+            }
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, live);
+        if (lane == 0)
+            wcount[warp] = __popc(m);
+        __syncthreads();
+        int before = total;
+        for (int v = 0; v < kWarps; ++v) {
+            if (v < warp)
+                before += wcount[v];
+            total += wcount[v];
+        }
+        if (live)
+            list[before + __popc(m & ((1u << lane) - 1u))] = b;
+        __syncthreads();                 // wcount is reused by the next chunk of rows
+    }
+    return total;
+}
+
 template <typename S, int N>
 __global__ void __launch_bounds__(kWarps * 32)
-ssu_replay_kernel(const __grid_constant__ ReplayArgs a, const int cph, const int upl,
-                  const int nunits)
+ssu_replay_kernel(const __grid_constant__ ReplayArgs a, const int cph)
 {
     using G = Geo<S, N, kUT>;
     using V = Vec16<S>;
     extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_live[kLiveMax];
+    __shared__ int s_wcount[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const WarpViews w = warp_views(smem, warp);
     init_ring(w, lane);
@@ -146,7 +218,11 @@ ssu_replay_kernel(const __grid_constant__ ReplayArgs a, const int cph, const int
     const int H = a.H, Dm = a.Dm, T = a.T, hpg = H / a.G;
     const int gw = blockIdx.x * kWarps + warp;
     const int nw = gridDim.x * kWarps;
-    const ReplayRows rows{&a};
+    const bool listed = a.active <= kLiveMax;
+    const int nrows = listed ? list_live_rows(a, s_live, s_wcount) : a.active;
+    const int upl = nrows * H * cph;     // units per layer (the host checked the full count)
+    const int nunits = upl * a.num_layers;
+    const ReplayRows rows{&a, listed ? s_live : nullptr};
     Producer<G, N, ReplayRows> prod;
     if (lane == 0) {
         prod.start(rows, gw, nw, upl, cph, nunits, H, Dm);
@@ -158,7 +234,7 @@ ssu_replay_kernel(const __grid_constant__ ReplayArgs a, const int cph, const int
     const int ln = lane % G::LPR, sub = lane / G::LPR;
     int c = 0;
     for (int u = gw; u < nunits; u += nw) {
-        const LUnit lu = lunit_at(u, upl, cph, G::CR, H, Dm);
+        const LUnit lu = rows.unit(u, upl, cph, G::CR, H, Dm);
         const Unit &un = lu.un;
         const int tiles = (un.rows + G::RT - 1) / G::RT;
         const int g = un.h / hpg;
@@ -259,8 +335,9 @@ ssu_replay_kernel(const __grid_constant__ ReplayArgs a, const int cph, const int
             if (lane == 0)
                 prod.issue(rows, a.slot_stride, gw, nw, upl, cph, nunits, H, Dm, w, s);
         }
-        // ---- caller bugs, reported once per row (or layer): clamped or skipped
-        if (lane == 0 && un.h == 0 && un.row0 == 0 && a.err) {
+        // ---- caller bugs, reported once per row (or layer): clamped or skipped (listed
+        // launches reported them while listing the rows)
+        if (!listed && lane == 0 && un.h == 0 && un.row0 == 0 && a.err) {
             if (!L.ok && un.b == 0)
                 atomicOr(a.err, SSU_FLAG_LAYER);
             if (lu.layer == 0) {
@@ -288,11 +365,12 @@ int launch_n(const ReplayArgs &a, cudaStream_t stream)
         return SSU_OK;
     if (nunits > 0x7fffffffLL)
         return SSU_ERR_SHAPE;
+    // sized for every active row; a listed launch may have fewer units that move
     const int grid = persistent_grid<ssu_replay_kernel<S, N>>(nunits);
     if (grid < 0)
         return SSU_ERR_CUDA;
     return launch_kernel(ssu_replay_kernel<S, N>, grid, kWarps * 32, kSmemBytes, stream, a,
-                         (int)cph, (int)upl, (int)nunits);
+                         (int)cph);
 }
 
 template <typename S>

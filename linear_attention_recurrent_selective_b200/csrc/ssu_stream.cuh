@@ -95,6 +95,14 @@ __device__ __forceinline__ LUnit lunit_at(int u, int upl, int cph, int CR, int H
     return lu;
 }
 
+// Units numbered in order: layer-major, then row, head and dim chunk.
+struct UnitsInOrder {
+    __device__ __forceinline__ LUnit unit(int u, int upl, int cph, int CR, int H, int Dm) const
+    {
+        return lunit_at(u, upl, cph, CR, H, Dm);
+    }
+};
+
 // What the producer needs to know about a unit: the base of its layer's pool, its slot and
 // a per-row extra (such as an accepted length).
 struct UnitRes {
@@ -120,8 +128,9 @@ __device__ __forceinline__ WarpViews warp_views(uint8_t *smem, int warp)
     return w;
 }
 
-// Lane 0's side of a warp's pipeline. `Rows` maps a unit to its pool, slot and extra and
-// says whether the unit moves state:
+// Lane 0's side of a warp's pipeline. `Rows` numbers the units, maps a unit to its pool,
+// slot and extra, and says whether the unit moves state:
+//   LUnit unit(int u, int upl, int cph, int CR, int H, int Dm) const;
 //   UnitRes resolve(const LUnit &lu) const;  bool moves(const UnitRes &r) const;
 template <typename G, int N, typename Rows> struct Producer {
     int k;        // position in this warp's unit sequence
@@ -141,11 +150,11 @@ template <typename G, int N, typename Rows> struct Producer {
         cur = UnitRes{nullptr, -1, 0};
         nxt = UnitRes{nullptr, -1, 0};
         if (gw < nunits) {
-            const LUnit lu = lunit_at(gw, upl, cph, G::CR, H, Dm);
+            const LUnit lu = rows.unit(gw, upl, cph, G::CR, H, Dm);
             cur = rows.resolve(lu);
             tiles = (lu.un.rows + G::RT - 1) / G::RT;
             if (gw + nw < nunits)
-                nxt = rows.resolve(lunit_at(gw + nw, upl, cph, G::CR, H, Dm));
+                nxt = rows.resolve(rows.unit(gw + nw, upl, cph, G::CR, H, Dm));
         }
     }
 
@@ -155,7 +164,7 @@ template <typename G, int N, typename Rows> struct Producer {
         const int u = gw + k * nw;
         if (u >= nunits)
             return;
-        const Unit un = lunit_at(u, upl, cph, G::CR, H, Dm).un;
+        const Unit un = rows.unit(u, upl, cph, G::CR, H, Dm).un;
         w.ctl->slot[s] = cur.slot;
         w.ctl->extra[s] = cur.extra;
         w.ctl->moves[s] = rows.moves(cur);
@@ -180,9 +189,9 @@ template <typename G, int N, typename Rows> struct Producer {
             const int u2 = gw + k * nw;
             if (u2 < nunits) {
                 cur = nxt;
-                tiles = (lunit_at(u2, upl, cph, G::CR, H, Dm).un.rows + G::RT - 1) / G::RT;
+                tiles = (rows.unit(u2, upl, cph, G::CR, H, Dm).un.rows + G::RT - 1) / G::RT;
                 if (u2 + nw < nunits)
-                    nxt = rows.resolve(lunit_at(u2 + nw, upl, cph, G::CR, H, Dm));
+                    nxt = rows.resolve(rows.unit(u2 + nw, upl, cph, G::CR, H, Dm));
             }
         }
     }
