@@ -22,7 +22,9 @@ enum {
     SSU_WAIT_STREAM = 1,      /* a state tile of the per-warp streaming pipeline (decode,
                                  replay, fused conv decode, GDN decode); index = the tile's
                                  number in the chosen warp's sequence */
-    SSU_WAIT_PREFILL = 2,     /* a chunk of the prefill's staged inputs; index = chunk */
+    SSU_WAIT_PREFILL = 2,     /* prefill chunk `index`: in the CUDA-core form its staged
+                                 inputs, in the chunked tensor-core form its first MMAs
+                                 (then not issued at all) */
     SSU_WAIT_TREE_STATE = 3,  /* the committed-state rows of a tree-verify item (tensor-core
                                  form); index = the item's position in its CTA's range */
     SSU_WAIT_TREE_X = 4,      /* the x tile of such an item */

@@ -478,7 +478,8 @@ int ssu_test_wait_fault(int site, int block, int warp, int index, unsigned long 
     const ssu::WaitFault f{limit_ns, site, block, warp, index};
     const int bad = ssu::wait_fault_set_decode(f) | ssu::wait_fault_set_replay(f) |
                     ssu::wait_fault_set_conv(f) | ssu::wait_fault_set_gdn(f) |
-                    ssu::wait_fault_set_prefill(f) | ssu::wait_fault_set_ddtree(f);
+                    ssu::wait_fault_set_prefill(f) | ssu::wait_fault_set_prefill_tc(f) |
+                    ssu::wait_fault_set_ddtree(f);
     return bad ? SSU_ERR_CUDA : SSU_OK;
 }
 #endif

@@ -24,7 +24,8 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 // The bounded waits a test build can make run out.
 enum {
     kFaultStream = 1,      // a tile of the per-warp streaming pipeline (decode, replay, ...)
-    kFaultPrefill = 2,     // a chunk of the prefill's input staging
+    kFaultPrefill = 2,     // a prefill chunk: its input staging, or (tensor-core form)
+                           // its first MMAs, which are then not issued
     kFaultTreeState = 3,   // the tree verify's committed-state rows (tensor-core form)
     kFaultTreeX = 4,       // the tree verify's x tile (tensor-core form)
     kFaultTreeMma = 5      // the tree verify's MMA completion (its MMAs are not issued)

@@ -102,6 +102,7 @@ int wait_fault_set_replay(const WaitFault &f);
 int wait_fault_set_conv(const WaitFault &f);
 int wait_fault_set_gdn(const WaitFault &f);
 int wait_fault_set_prefill(const WaitFault &f);
+int wait_fault_set_prefill_tc(const WaitFault &f);
 int wait_fault_set_ddtree(const WaitFault &f);
 #endif
 
@@ -181,6 +182,7 @@ struct TreeArgs {
 // Host launchers, one per kernel family; each returns SSU_OK or SSU_ERR_UNSUPPORTED.
 int launch_decode(const DecodeArgs &a, int state_dtype, cudaStream_t s);
 int launch_prefill(const PrefillArgs &a, int state_dtype, cudaStream_t s);
+int launch_prefill_tc(const PrefillArgs &a, int state_dtype, cudaStream_t s);  // -1: n/a
 int launch_replay(const ReplayArgs &a, int state_dtype, cudaStream_t s);
 int launch_ddtree(const TreeArgs &a, int state_dtype, cudaStream_t s);
 int launch_conv_decode(const ConvArgs &a, int state_dtype, cudaStream_t s);
@@ -247,6 +249,46 @@ __device__ __forceinline__ float effective_dt(float dt, const float *bias, int h
 {
     float v = dt + (bias ? bias[h] : 0.f);
     return sp ? softplus_f(v) : v;
+}
+
+// ---------------------------------------------------------------- prefill scheduling
+
+constexpr int kRankMax = 32;    // prefill batches up to this size run longest rows first
+
+// Length used for scheduling a prefill row: padding and out-of-range rows do (almost) no
+// work.
+__device__ __forceinline__ int prefill_sched_len(const PrefillArgs &pa, int b)
+{
+    const int slot = pa.d.idx ? pa.d.idx[b] : b;
+    if (slot < 0 || slot >= pa.d.P)
+        return 0;
+    const int L = pa.ctx ? pa.ctx[b] : pa.T;
+    return L < 0 ? 0 : (L > pa.T ? pa.T : L);
+}
+
+// The row a prefill CTA of rank `rank` takes: with at most kRankMax active rows, rows are
+// ranked by decreasing length from the device lengths (ties by index) so that the longest
+// scans start first; otherwise row `rank`. Every thread of the CTA calls it (s_len
+// [kRankMax] and s_row in shared memory).
+__device__ __forceinline__ int prefill_ranked_row(const PrefillArgs &pa, int rank, int *s_len,
+                                                  int *s_row)
+{
+    const int tid = threadIdx.x, active = pa.d.active;
+    if (active > kRankMax)
+        return rank;
+    if (tid < active)
+        s_len[tid] = prefill_sched_len(pa, tid);
+    __syncthreads();
+    if (tid < active) {
+        const int mine = s_len[tid];
+        int r = 0;
+        for (int o = 0; o < active; ++o)
+            r += (s_len[o] > mine) || (s_len[o] == mine && o < tid);
+        if (r == rank)
+            *s_row = tid;
+    }
+    __syncthreads();
+    return *s_row;
 }
 
 // ---------------------------------------------------------------- 16-byte state vectors

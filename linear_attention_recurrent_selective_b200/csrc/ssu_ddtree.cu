@@ -100,23 +100,6 @@ struct TLayout {
     }
 };
 
-__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)),
-                 "l"(src)
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit()
-{
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all()
-{
-    asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
 // Byte offset of 16-byte chunk c of state row r in the staging buffer (cpr chunks per
 // row): chunks are XOR-swizzled by the row so that lanes reading the same chunk of
 // consecutive rows hit different banks.
@@ -824,13 +807,6 @@ struct TcLayout {
         total = tptr + 16 + 1024;             // slack for aligning the base
     }
 };
-
-// Byte offset of 16-byte chunk c (columns 8c .. 8c + 7) of row r in a K-major operand
-// with 128-byte swizzle and `block` bytes per 64-column block.
-__device__ __forceinline__ int sw128_off(int r, int c, int block)
-{
-    return (c >> 3) * block + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4);
-}
 
 // Per-(row, group) tables of the tensor-core form: parents, path checks, C in the
 // operand layout, path pairs (pj: path node, pi: node) and C_i . B_j of every pair. All

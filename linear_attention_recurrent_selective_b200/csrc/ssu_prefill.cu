@@ -37,8 +37,6 @@
 namespace ssu {
 namespace {
 
-constexpr int kRankMax = 32;    // batches up to this size are scheduled longest-first
-
 // Tokens per staged chunk and the register budget (CTAs of kWarpsPerCta warps that must
 // fit kMinCtas per SM); the defaults are the measured best on B200, overridable at build
 // time for tuning sweeps.
@@ -92,16 +90,6 @@ struct PLayout {
     }
 };
 
-// Length used for scheduling: padding and out-of-range rows do (almost) no work.
-__device__ __forceinline__ int sched_len(const PrefillArgs &pa, int b)
-{
-    const int slot = pa.d.idx ? pa.d.idx[b] : b;
-    if (slot < 0 || slot >= pa.d.P)
-        return 0;
-    const int L = pa.ctx ? pa.ctx[b] : pa.T;
-    return L < 0 ? 0 : (L > pa.T ? pa.T : L);
-}
-
 template <typename S, int N>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, kMinCtas)
 ssu_prefill_kernel(const PrefillArgs pa, const int dtiles, const int rtc, const int bulk)
@@ -129,22 +117,7 @@ ssu_prefill_kernel(const PrefillArgs pa, const int dtiles, const int rtc, const 
     const int rank = blockIdx.x / per_row;
     const int rem = blockIdx.x % per_row;
     const int h = rem / dtiles, dtile = rem % dtiles;
-    int b = rank;
-    if (a.active <= kRankMax) {
-        if (tid < a.active)
-            s_len[tid] = sched_len(pa, tid);
-        __syncthreads();
-        if (tid < a.active) {
-            const int mine = s_len[tid];
-            int r = 0;
-            for (int o = 0; o < a.active; ++o)
-                r += (s_len[o] > mine) || (s_len[o] == mine && o < tid);
-            if (r == rank)
-                s_row = tid;
-        }
-        __syncthreads();
-        b = s_row;
-    }
+    const int b = prefill_ranked_row(pa, rank, s_len, &s_row);
 
     const int row0 = dtile * rtc;
     const int rows_c = min(rtc, Dm - row0);
@@ -466,6 +439,9 @@ SSU_WAIT_FAULT_SETTER(wait_fault_set_prefill)
 
 int launch_prefill(const PrefillArgs &a, int state_dtype, cudaStream_t s)
 {
+    const int tc = launch_prefill_tc(a, state_dtype, s);   // the chunked tensor-core form
+    if (tc >= 0)
+        return tc;
     switch (state_dtype) {
     case SSU_F32: return launch_s<float>(a, s);
     case SSU_F16: return launch_s<__half>(a, s);

@@ -20,6 +20,32 @@
 
 namespace ssu {
 
+// Byte offset of 16-byte chunk c (columns 8c .. 8c + 7) of row r in a K-major operand
+// with 128-byte swizzle and `block` bytes (rows x 128) per 64-column block.
+__host__ __device__ __forceinline__ int sw128_off(int r, int c, int block)
+{
+    return (c >> 3) * block + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+
+// 16-byte asynchronous global -> shared copies (cp.async, L2 only), grouped and waited
+// for as a whole.
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)),
+                 "l"(src)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor of a K-major, 128-byte-swizzled bf16 operand starting
 // at shared address saddr: start address (16-byte units) in bits 0..13, leading byte
 // offset 16 (unused by swizzled K-major layouts), stride byte offset 1024 between 8-row

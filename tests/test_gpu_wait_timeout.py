@@ -102,8 +102,9 @@ def test_decode_tile_wait_runs_out(orc, waitlib):
 
 
 def test_replay_tile_wait_runs_out(orc, waitlib):
-    # replay units are 2 tiles (16 rows): 2 rows x 2 heads x 4 units = 16 units on 2 CTAs;
-    # warp 1 of CTA 0 (unit 1: row 0, head 0, rows 16 .. 31) loses its first tile
+    # replay units are 4 tiles (32 rows): 2 rows x 2 heads x 2 units = 8 units (both rows
+    # live) on one CTA of 8 warps; warp 1 (unit 1: row 0, head 0, rows 32 .. 63) loses its
+    # first tile
     case = make_case(seed=991, batch=2, P=4, T=3, H=2, G=1, Dm=64, N=128, x_dtype=BF16,
                      bc_dtype=BF16, lengths="accepted")
     case.accepted_lengths = torch.tensor([3, 2], dtype=torch.int32)
@@ -116,19 +117,19 @@ def test_replay_tile_wait_runs_out(orc, waitlib):
                T=3, H=2, G=1, Dm=64, N=128)
     s0 = int(case.state_indices[0])
     g, o, before = (head_rows(p, case, s0, 0) for p in (pool_g, want, case.pool))
-    assert same_bits(g[16:32], before[16:32])             # the unit that gave up
-    check_state(g[:16], o[:16], F32)
-    check_state(g[32:], o[32:], F32)
+    assert same_bits(g[32:], before[32:])                 # the unit that gave up
+    check_state(g[:32], o[:32], F32)
     check_state(without_head(pool_g, case, s0, 0), without_head(want, case, s0, 0), F32)
     ssu._lib = None
     product_still_runs(orc)
 
 
 def test_prefill_chunk_wait_runs_out(orc, waitlib):
-    # 2 rows x 2 heads, one CTA each (rows ranked by length: equal lengths keep index
-    # order, so CTA 1 is row 0, head 1); its second 16-token chunk never completes
+    # the CUDA-core form (fp32 B and C): 2 rows x 2 heads, one CTA each (rows ranked by
+    # length: equal lengths keep index order, so CTA 1 is row 0, head 1); its second
+    # 16-token chunk of staged inputs never completes
     case = make_case(seed=992, batch=2, P=4, T=40, H=2, G=1, Dm=64, N=128, x_dtype=BF16,
-                     bc_dtype=BF16, z=True)
+                     bc_dtype=F32, z=True)
     assert case.context_lengths is None
     arm(waitlib, PREFILL, 1, -1, 1)
     out_g, pool_g, _, err = gpu_run.prefill(case)
@@ -141,6 +142,30 @@ def test_prefill_chunk_wait_runs_out(orc, waitlib):
     keep[0, :, 1] = False
     check_out(out_g[keep], out_o[keep], BF16)
     # its final state is never stored; every other head's is
+    assert same_bits(head_rows(pool_g, case, s0, 1), head_rows(case.pool, case, s0, 1))
+    check_state(without_head(pool_g, case, s0, 1), without_head(pool_o, case, s0, 1), F32)
+    ssu._lib = None
+    product_still_runs(orc)
+
+
+def test_prefill_tensor_core_mma_wait_runs_out(orc, waitlib):
+    # the chunked tensor-core form (bf16 x, B, C): 2 rows x 2 heads, one CTA each; CTA 1
+    # (row 0, head 1) does not issue the first products of its second 128-token chunk,
+    # so that chunk's wait runs out: its first chunk's outputs are written, the rest not,
+    # and its final state is never stored
+    case = make_case(seed=996, batch=2, P=4, T=200, H=2, G=1, Dm=64, N=128, x_dtype=BF16,
+                     bc_dtype=BF16, z=True)
+    assert case.context_lengths is None
+    arm(waitlib, PREFILL, 1, -1, 1)
+    out_g, pool_g, _, err = gpu_run.prefill(case)
+    assert err == ssu.FLAG_TIMEOUT
+    out_o, pool_o, _, _ = orc.prefill_case(case)
+    s0 = int(case.state_indices[0])
+    check_out(out_g[0, :128, 1], out_o[0, :128, 1], BF16)
+    assert torch.isnan(out_g[0, 128:, 1].float()).all()
+    keep = torch.ones(2, 200, 2, dtype=torch.bool)
+    keep[0, :, 1] = False
+    check_out(out_g[keep], out_o[keep], BF16)
     assert same_bits(head_rows(pool_g, case, s0, 1), head_rows(case.pool, case, s0, 1))
     check_state(without_head(pool_g, case, s0, 1), without_head(pool_o, case, s0, 1), F32)
     ssu._lib = None
