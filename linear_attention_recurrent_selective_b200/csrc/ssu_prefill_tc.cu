@@ -66,7 +66,7 @@ constexpr int kPieceN = 2 * kBlkN;
 constexpr int kOffBT = kOffS + 3 * kPieceN;       // B^T [n][m]
 constexpr int kOffXT = kOffBT + 2 * kBlkM;        // X^T [d][m]
 constexpr int kOffX = kOffXT + kPieceN;           // x rows as loaded [t][d], 128 B a row
-constexpr int kOffLam = kOffX + kL * kDT * 2;     // Lambda_t, double
+constexpr int kOffLam = kOffX + kL * kDT * 2;     // Lambda_t in units of log2, double
 constexpr int kOffDt = kOffLam + kL * 8;          // dt_eff of each token
 constexpr int kOffPt = kOffDt + kL * 4;           // e^{Lambda_t}
 constexpr int kOffWl = kOffPt + kL * 4;           // w(last, m) dt_m
@@ -74,6 +74,7 @@ constexpr int kOffTot = kOffWl + kL * 4;          // per-warp Lambda totals (4 d
 constexpr int kOffBar = kOffTot + 32;             // two mbarriers: D1 and D2, D3 and D4
 constexpr int kOffTptr = kOffBar + 16;
 constexpr int kSmem = kOffTptr + 16 + 1024;       // + slack for aligning the base
+constexpr double kLog2e = 1.4426950408889634;
 static_assert(kOffS % 1024 == 0 && kOffBT % 1024 == 0 && kOffXT % 1024 == 0,
               "operands start on 1024-byte boundaries");
 static_assert(kSmem <= 227 * 1024, "shared memory of the chunked prefill");
@@ -223,10 +224,11 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
     const uint32_t tmem = *tptr;
     const uint32_t tl = tmem + ((uint32_t)(32 * quarter) << 16);   // this warp's lanes
 
-    // ---- the chunk's C, B and x rows into shared memory; rows past the chunk are zero
+    // ---- the chunk's C and B rows, then its x rows, into shared memory (two commit
+    // groups, waited for together); rows past the chunk are zero
     const int nchunks = (L + kL - 1) / kL;
     const int xch = rows / 8;                 // 16-byte chunks of a token's x row
-    auto load_chunk = [&](int c) {
+    auto load_cb = [&](int c) {
         const int t0 = c * kL, nt = min(kL, L - t0);
         for (int k = tid; k < kL * 16; k += kThr) {
             const int t = k >> 4, ch = k & 15;
@@ -241,6 +243,10 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
                 zero16(db);
             }
         }
+        cp_async_commit();
+    };
+    auto load_x = [&](int c) {
+        const int t0 = c * kL, nt = min(kL, L - t0);
         for (int k = tid; k < kL * 8; k += kThr) {
             const int t = k >> 3, ch = k & 7;
             uint8_t *dx = sm + kOffX + t * 128 + ch * 16;
@@ -275,7 +281,8 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
         }
     };
     put_state();
-    load_chunk(0);
+    load_cb(0);
+    load_x(0);
 
     constexpr uint32_t kI64 = idesc_bf16_f32(kL, 64);
     constexpr uint32_t kI128 = idesc_bf16_f32(kL, 128);
@@ -297,7 +304,7 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
                     pa.st_dA[bth] = expf(Ah * dte);
                     pa.st_dt[bth] = dte;
                 }
-                l = (double)Ah * (double)dte;
+                l = (double)Ah * (double)dte * kLog2e;
             }
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -348,8 +355,12 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
                 }
             tc_commit(bar);
         }
-        {   // B^T: one 8 x 8 block per thread (m-block tid / 16, n-block tid % 16)
-            const int mb = tid >> 4, nb = tid & 15;
+        {   // B^T: one 8 x 8 block per thread. Within each group of 8 lanes the blocks run
+            // along a diagonal (n-blocks a, m-blocks a + s), so that both the reads (rows
+            // 8 mb + i, chunk nb) and the writes (rows 8 nb + j, chunk mb) of the 8 lanes
+            // fall on 8 different 16-byte bank groups of the swizzled layouts
+            const int a8 = tid & 7, s8 = (tid >> 3) & 7, mh = (tid >> 6) & 1, nh = tid >> 7;
+            const int nb = 8 * nh + a8, mb = 8 * mh + ((a8 + s8) & 7);
             uint4 in[8], out[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -359,12 +370,13 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
             for (int j = 0; j < 8; ++j)
                 *reinterpret_cast<uint4 *>(sm + kOffBT + sw128_off(8 * nb + j, mb, kBlkM)) = out[j];
         }
-        if (tid < 128) {   // X^T: 16 token blocks x 8 dim blocks
-            const int tb = tid >> 3, db = tid & 7;
+        if (tid < 128) {   // X^T: 16 token blocks x 8 dim blocks, on diagonals as above
+            const int db = tid & 7, tb = 8 * (tid >> 6) + ((db + (tid >> 3)) & 7);
             uint4 in[8], out[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                in[i] = *reinterpret_cast<const uint4 *>(sm + kOffX + (8 * tb + i) * 128 + db * 16);
+                in[i] = *reinterpret_cast<const uint4 *>(sm + kOffX +
+                                                         (8 * tb + i) * 128 + db * 16);
             transpose8(in, out);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -372,8 +384,8 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
         } else {           // e^{Lambda_t} and w(last, m) dt_m of every token
             const int t = tid - 128;
             const double last = lam[nt - 1];
-            spt[t] = t < nt ? expf((float)lam[t]) : 0.f;
-            swl[t] = t < nt ? expf((float)(last - lam[t])) * sdt[t] : 0.f;
+            spt[t] = t < nt ? exp2f((float)lam[t]) : 0.f;
+            swl[t] = t < nt ? exp2f((float)(last - lam[t])) * sdt[t] : 0.f;
         }
         if (write_group) {   // the stash's B: the chunk's B rows widened
             for (int k = tid; k < nt * 16; k += kThr) {
@@ -400,29 +412,41 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
         tc_fence_after();
 
         // ---- phase 2: G from D2 (over C and B) and (w dt X)^T (over the state pieces)
-        {   // thread (t = r, half): columns m = 64 half .. + 63 of row t
-            float cbv[2][32];
-            tmem_ld32(tl + kD2 + 64 * half, cbv[0]);
-            tmem_ld32(tl + kD2 + 64 * half + 32, cbv[1]);
+        {   // thread (t = r, half): columns m = 64 half .. + 63 of row t. A warp whose 32
+            // rows all lie above those columns (or past the chunk) only writes zeros.
             const int t = r;
-            const double lt = lam[t];
+            const bool zero = 32 * quarter + 31 < 64 * half || 32 * quarter >= nt;
+            if (zero) {
 #pragma unroll
-            for (int jc = 0; jc < 8; ++jc) {
-                float gv[8];
+                for (int jc = 0; jc < 8; ++jc) {
+                    const int o = sw128_off(t, 8 * half + jc, kBlkM);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int m = 64 * half + 8 * jc + e;
-                    gv[e] = (m <= t && t < nt)
-                                ? cbv[jc >> 2][8 * (jc & 3) + e] *
-                                      (expf((float)(lt - lam[m])) * sdt[m])
-                                : 0.f;
+                    for (int k = 0; k < 3; ++k)
+                        zero16(sm + kOffG + k * kPieceG + o);
                 }
-                uint4 p[3];
-                split8(gv, p);
-                const int o = sw128_off(t, 8 * half + jc, kBlkM);
+            } else {
+                float cbv[2][32];
+                tmem_ld32(tl + kD2 + 64 * half, cbv[0]);
+                tmem_ld32(tl + kD2 + 64 * half + 32, cbv[1]);
+                const double lt = lam[t];
 #pragma unroll
-                for (int k = 0; k < 3; ++k)
-                    *reinterpret_cast<uint4 *>(sm + kOffG + k * kPieceG + o) = p[k];
+                for (int jc = 0; jc < 8; ++jc) {
+                    float gv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int m = 64 * half + 8 * jc + e;
+                        gv[e] = (m <= t && t < nt)
+                                    ? cbv[jc >> 2][8 * (jc & 3) + e] *
+                                          (exp2f((float)(lt - lam[m])) * sdt[m])
+                                    : 0.f;
+                    }
+                    uint4 p[3];
+                    split8(gv, p);
+                    const int o = sw128_off(t, 8 * half + jc, kBlkM);
+#pragma unroll
+                    for (int k = 0; k < 3; ++k)
+                        *reinterpret_cast<uint4 *>(sm + kOffG + k * kPieceG + o) = p[k];
+                }
             }
         }
         for (int k = tid; k < kDT * 16; k += kThr) {   // (d, 8 tokens) per task
@@ -472,6 +496,16 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
                     }
             tc_commit(bar + 1);
         }
+        // this thread's z values (token r, dims 32 half .. + 31) while the products run
+        uint4 zr[4];
+        {
+            const int64_t xi = (((int64_t)b * T + t0 + r) * H + h) * Dm + row0 + 32 * half;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                zr[q] = (Zg && r < nt && 32 * half + 8 * q < rows)
+                            ? *reinterpret_cast<const uint4 *>(Zg + xi + 8 * q)
+                            : make_uint4(0u, 0u, 0u, 0u);
+        }
         {
             const bool ok = mbar_wait(bar + 1, ph1);
             if (__syncthreads_or(!ok)) {      // D3 and D4 never completed: give up
@@ -484,8 +518,8 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
             ph1 ^= 1u;
         }
         tc_fence_after();
-        if (c + 1 < nchunks)                  // C, B, G and the x rows are free
-            load_chunk(c + 1);
+        if (c + 1 < nchunks)                  // C, B and G are free
+            load_cb(c + 1);
 
         // ---- phase 4: outputs of token t = r, dims 32 half .. + 31
         {
@@ -497,21 +531,21 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
                 const int64_t xi = (((int64_t)b * T + t0 + t) * H + h) * Dm + row0 + 32 * half;
                 const float pt = spt[t];
                 float xv[32], y[32];
+                const uint8_t *xrow = sm + kOffX + t * 128 + 64 * half;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int d = 32 * half + j;
-                    xv[j] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                        sm + kOffXT + sw128_off(d, t >> 3, kBlkN) + (t & 7) * 2));
+                for (int q = 0; q < 4; ++q)
+                    Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4 *>(xrow + 16 * q),
+                                                 xv + 8 * q);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
                     y[j] = fmaf(pt, d1[j], d3[j]) + Dh * xv[j];
-                }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     if (32 * half + 8 * q >= rows)
                         break;
                     if (Zg) {
                         float zf[8];
-                        Vec16<__nv_bfloat16>::unpack(
-                            *reinterpret_cast<const uint4 *>(Zg + xi + 8 * q), zf);
+                        Vec16<__nv_bfloat16>::unpack(zr[q], zf);
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
                             y[8 * q + e] *= __fdividef(zf[e], 1.f + __expf(-zf[e]));
@@ -544,7 +578,9 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
         }
         tc_fence_before();
         fence_async_smem();
-        __syncthreads();
+        __syncthreads();                      // this chunk's x rows and accumulators are read
+        if (c + 1 < nchunks)
+            load_x(c + 1);
     }
 
     // ---- the final state, once (the stash mode leaves the committed state read-only)
