@@ -24,7 +24,10 @@
 // to within 2^-24 of each element (p1 = bf16(v), p2 = bf16(v - p1), p3 = bf16(v - p1 - p2),
 // each difference exact in fp32); bf16 inputs enter exactly; products of two bf16 values
 // are exact in the fp32 accumulator. The results therefore carry fp32 accuracy: the same
-// values as the sequential form up to the order of the fp32 sums.
+// values as the sequential form up to the order of the fp32 sums. (Two pieces, 2^-17, were
+// measured not to be enough even for the bf16 outputs: the error is relative to the terms
+// summed, and where terms of order 10 cancel to an output near zero it exceeds the 1e-5
+// absolute part of the tolerance.)
 //
 // Work: one CTA of 8 warps per (row, head, dim tile), rows ranked longest first; the
 // state lives in registers (thread (n, half) holds s[d][n] for 32 dim rows d) and in
@@ -52,25 +55,32 @@ constexpr int kThr = 256;               // 8 warps; warp w reads TMEM lanes 32 (
 constexpr uint32_t kCols = 512;         // tensor-memory columns, the whole SM's
 constexpr uint32_t kD1 = 0, kD2 = 64, kD3 = 192, kD4 = 256;   // accumulator columns
 
+// bf16 pieces per operand (G, the state's copy in D1, (w dt X)^T)
+constexpr int kPG = 3, kPS = 3, kPW = 3;
+
 // Shared memory, byte offsets from a 1024-byte aligned base. A K-block (64 columns) of a
 // 128-row bf16 operand is kBlkM bytes, of a 64-row one kBlkN.
 constexpr int kBlkM = kL * 128;
 constexpr int kBlkN = kDT * 128;
 constexpr int kOffC = 0;                          // C chunk [t][n]            (phase 1)
 constexpr int kOffB = kOffC + 2 * kBlkM;          // B chunk [m][n]            (phase 1)
-constexpr int kOffG = 0;                          // G pieces [t][m] x 3       (phase 2)
+constexpr int kOffG = 0;                          // G pieces [t][m]           (phase 2)
 constexpr int kPieceG = 2 * kBlkM;
-constexpr int kOffS = kOffG + 3 * kPieceG;        // state pieces [d][n] x 3   (phase 1)
-constexpr int kOffW = kOffS;                      // (w dt X)^T pieces [d][m] x 3 (phase 2)
+constexpr int kOffS = kOffG + kPG * kPieceG;      // state pieces [d][n]       (phase 1)
+constexpr int kOffW = kOffS;                      // (w dt X)^T pieces [d][m]  (phase 2)
 constexpr int kPieceN = 2 * kBlkN;
-constexpr int kOffBT = kOffS + 3 * kPieceN;       // B^T [n][m]
+constexpr int kOffBT = kOffS + kPW * kPieceN;     // B^T [n][m]
 constexpr int kOffXT = kOffBT + 2 * kBlkM;        // X^T [d][m]
-constexpr int kOffX = kOffXT + kPieceN;           // x rows as loaded [t][d], 128 B a row
-constexpr int kOffLam = kOffX + kL * kDT * 2;     // Lambda_t in units of log2, double
+constexpr int kOffX = kOffXT + kPieceN;           // x rows [t][d], 128 B a row (epilogue)
+constexpr int kOffXL = kOffG + 2 * kPieceG;       // where the next chunk's x rows land: in
+                                                  // the third G piece, free from the last
+                                                  // products' completion to phase 2
+constexpr int kOffLam = kOffX + kL * kDT * 2;     // Lambda_t (log2 units) as a float pair
 constexpr int kOffDt = kOffLam + kL * 8;          // dt_eff of each token
 constexpr int kOffPt = kOffDt + kL * 4;           // e^{Lambda_t}
 constexpr int kOffWl = kOffPt + kL * 4;           // w(last, m) dt_m
 constexpr int kOffTot = kOffWl + kL * 4;          // per-warp Lambda totals (4 doubles)
+static_assert(kPG * kPieceG >= kOffB + 2 * kBlkM && kPS <= kPW, "G over C and B");
 constexpr int kOffBar = kOffTot + 32;             // two mbarriers: D1 and D2, D3 and D4
 constexpr int kOffTptr = kOffBar + 16;
 constexpr int kSmem = kOffTptr + 16 + 1024;       // + slack for aligning the base
@@ -106,15 +116,16 @@ __device__ __forceinline__ void transpose8(const uint4 (&in)[8], uint4 (&out)[8]
     }
 }
 
-// Three bf16 pieces of eight fp32 values, packed 16 bytes each.
-__device__ __forceinline__ void split8(const float (&v)[8], uint4 (&p)[3])
+// NP bf16 pieces of eight fp32 values, packed 16 bytes each.
+template <int NP>
+__device__ __forceinline__ void split8(const float (&v)[8], uint4 (&p)[NP])
 {
     float r[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e)
         r[e] = v[e];
 #pragma unroll
-    for (int k = 0; k < 3; ++k) {
+    for (int k = 0; k < NP; ++k) {
         uint32_t w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -128,16 +139,26 @@ __device__ __forceinline__ void split8(const float (&v)[8], uint4 (&p)[3])
     }
 }
 
+// 2^v by the special-function unit (ex2.approx.ftz: about 2^-22 relative error, results
+// below 2^-126 flushed to zero, which is what a decay that small contributes anyway).
+__device__ __forceinline__ float pow2(float v)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+
 // The ssu_dtype code of a state storage type.
 template <typename S> struct StateCode { static constexpr int v = SSU_F32; };
 template <> struct StateCode<__half> { static constexpr int v = SSU_F16; };
 template <> struct StateCode<__nv_bfloat16> { static constexpr int v = SSU_BF16; };
 
-// Three bf16 pieces of one fp32 value.
-__device__ __forceinline__ void split1(float v, __nv_bfloat16 (&p)[3])
+// NP bf16 pieces of one fp32 value.
+template <int NP>
+__device__ __forceinline__ void split1(float v, __nv_bfloat16 (&p)[NP])
 {
 #pragma unroll
-    for (int k = 0; k < 3; ++k) {
+    for (int k = 0; k < NP; ++k) {
         p[k] = __float2bfloat16_rn(v);
         v -= __bfloat162float(p[k]);
     }
@@ -203,7 +224,8 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
     const __nv_bfloat16 *Xg = static_cast<const __nv_bfloat16 *>(a.x);
     const __nv_bfloat16 *Zg = static_cast<const __nv_bfloat16 *>(a.z);
     __nv_bfloat16 *Og = static_cast<__nv_bfloat16 *>(a.out);
-    double *lam = reinterpret_cast<double *>(sm + kOffLam);
+    double *lam = reinterpret_cast<double *>(sm + kOffLam);   // first double, then (hi, lo)
+    float2 *lam2 = reinterpret_cast<float2 *>(sm + kOffLam);
     float *sdt = reinterpret_cast<float *>(sm + kOffDt);
     float *spt = reinterpret_cast<float *>(sm + kOffPt);
     float *swl = reinterpret_cast<float *>(sm + kOffWl);
@@ -249,7 +271,7 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
         const int t0 = c * kL, nt = min(kL, L - t0);
         for (int k = tid; k < kL * 8; k += kThr) {
             const int t = k >> 3, ch = k & 7;
-            uint8_t *dx = sm + kOffX + t * 128 + ch * 16;
+            uint8_t *dx = sm + kOffXL + t * 128 + ch * 16;
             if (t < nt && ch < xch)
                 cp_async16(dx, Xg + (((int64_t)b * T + t0 + t) * H + h) * Dm + row0 + ch * 8);
             else
@@ -272,11 +294,11 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             const int d = 32 * half + j;
-            __nv_bfloat16 p[3];
-            split1(st[j], p);
+            __nv_bfloat16 p[kPS];
+            split1<kPS>(st[j], p);
             uint8_t *dst = sm + kOffS + sw128_off(d, r >> 3, kBlkN) + (r & 7) * 2;
 #pragma unroll
-            for (int k = 0; k < 3; ++k)
+            for (int k = 0; k < kPS; ++k)
                 *reinterpret_cast<__nv_bfloat16 *>(dst + k * kPieceN) = p[k];
         }
     };
@@ -320,21 +342,28 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
         cp_async_wait_all();                  // this chunk's C, B and x rows
         fence_async_smem();                   // ... and the state pieces, for the MMAs
         __syncthreads();
+        double lfull = 0.0;
         if (tid < kL) {
             double off = 0.0;
             for (int w = 0; w < warp; ++w)
                 off += stot[w];
-            lam[tid] += off;
+            lfull = lam[tid] + off;
+        }
+        __syncthreads();                      // every warp total read
+        if (tid < kL) {                       // Lambda_t as hi + lo, hi = fp32(Lambda_t)
+            const float hi = (float)lfull;
+            lam2[tid] = make_float2(hi, (float)(lfull - (double)hi));
         }
         __syncthreads();                      // Lambda complete
 
-        // ---- phase 1: D1 = C s^T, D2 = C B^T (one thread), while the others build B^T,
-        // X^T, the per-token factors and the stash's B
+        // ---- phase 1: D1 = C s^T, D2 = C B^T (one thread), while the others copy the x
+        // rows out of their landing buffer and build B^T, X^T, the per-token factors and
+        // the stash's B
         if (tid == 0 && !fault_tx(kFaultPrefill, -1, c)) {
             tc_fence_after();
             uint32_t acc = 0;
 #pragma unroll
-            for (int p = 2; p >= 0; --p)                     // smallest piece first
+            for (int p = kPS - 1; p >= 0; --p)               // smallest piece first
 #pragma unroll
                 for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
@@ -354,6 +383,13 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
                     acc = 1;
                 }
             tc_commit(bar);
+        }
+        {   // the x rows from their landing buffer to the epilogue's buffer
+            const uint4 *src = reinterpret_cast<const uint4 *>(sm + kOffXL);
+            uint4 *dst = reinterpret_cast<uint4 *>(sm + kOffX);
+#pragma unroll
+            for (int k = 0; k < kL * 8 / kThr; ++k)
+                dst[tid + kThr * k] = src[tid + kThr * k];
         }
         {   // B^T: one 8 x 8 block per thread. Within each group of 8 lanes the blocks run
             // along a diagonal (n-blocks a, m-blocks a + s), so that both the reads (rows
@@ -375,17 +411,17 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
             uint4 in[8], out[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                in[i] = *reinterpret_cast<const uint4 *>(sm + kOffX +
-                                                         (8 * tb + i) * 128 + db * 16);
+                in[i] = *reinterpret_cast<const uint4 *>(sm + kOffXL + (8 * tb + i) * 128 +
+                                                         db * 16);
             transpose8(in, out);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 *reinterpret_cast<uint4 *>(sm + kOffXT + sw128_off(8 * db + j, tb, kBlkN)) = out[j];
         } else {           // e^{Lambda_t} and w(last, m) dt_m of every token
             const int t = tid - 128;
-            const double last = lam[nt - 1];
-            spt[t] = t < nt ? exp2f((float)lam[t]) : 0.f;
-            swl[t] = t < nt ? exp2f((float)(last - lam[t])) * sdt[t] : 0.f;
+            const float2 lt = lam2[t], ll = lam2[nt - 1];
+            spt[t] = t < nt ? pow2(lt.x + lt.y) : 0.f;
+            swl[t] = t < nt ? pow2((ll.x - lt.x) + (ll.y - lt.y)) * sdt[t] : 0.f;
         }
         if (write_group) {   // the stash's B: the chunk's B rows widened
             for (int k = tid; k < nt * 16; k += kThr) {
@@ -421,30 +457,31 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
                 for (int jc = 0; jc < 8; ++jc) {
                     const int o = sw128_off(t, 8 * half + jc, kBlkM);
 #pragma unroll
-                    for (int k = 0; k < 3; ++k)
+                    for (int k = 0; k < kPG; ++k)
                         zero16(sm + kOffG + k * kPieceG + o);
                 }
             } else {
                 float cbv[2][32];
                 tmem_ld32(tl + kD2 + 64 * half, cbv[0]);
                 tmem_ld32(tl + kD2 + 64 * half + 32, cbv[1]);
-                const double lt = lam[t];
+                const float2 lt = lam2[t];
 #pragma unroll
                 for (int jc = 0; jc < 8; ++jc) {
                     float gv[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int m = 64 * half + 8 * jc + e;
+                        const float2 lm = lam2[m];
                         gv[e] = (m <= t && t < nt)
                                     ? cbv[jc >> 2][8 * (jc & 3) + e] *
-                                          (exp2f((float)(lt - lam[m])) * sdt[m])
+                                          (pow2((lt.x - lm.x) + (lt.y - lm.y)) * sdt[m])
                                     : 0.f;
                     }
-                    uint4 p[3];
-                    split8(gv, p);
+                    uint4 p[kPG];
+                    split8<kPG>(gv, p);
                     const int o = sw128_off(t, 8 * half + jc, kBlkM);
 #pragma unroll
-                    for (int k = 0; k < 3; ++k)
+                    for (int k = 0; k < kPG; ++k)
                         *reinterpret_cast<uint4 *>(sm + kOffG + k * kPieceG + o) = p[k];
                 }
             }
@@ -457,10 +494,10 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
 #pragma unroll
             for (int e = 0; e < 8; ++e)
                 v[e] = swl[8 * ch + e] * xv[e];
-            uint4 p[3];
-            split8(v, p);
+            uint4 p[kPW];
+            split8<kPW>(v, p);
 #pragma unroll
-            for (int q = 0; q < 3; ++q)
+            for (int q = 0; q < kPW; ++q)
                 *reinterpret_cast<uint4 *>(sm + kOffW + q * kPieceN + o) = p[q];
         }
         fence_async_smem();
@@ -472,7 +509,7 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
             tc_fence_after();
             uint32_t acc = 0;
 #pragma unroll
-            for (int p = 2; p >= 0; --p)
+            for (int p = kPG - 1; p >= 0; --p)
 #pragma unroll
                 for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
@@ -484,7 +521,7 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
                     }
             acc = 0;
 #pragma unroll
-            for (int p = 2; p >= 0; --p)
+            for (int p = kPW - 1; p >= 0; --p)
 #pragma unroll
                 for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
@@ -518,8 +555,10 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
             ph1 ^= 1u;
         }
         tc_fence_after();
-        if (c + 1 < nchunks)                  // C, B and G are free
+        if (c + 1 < nchunks) {                // C, B and G (the x landing buffer) are free
             load_cb(c + 1);
+            load_x(c + 1);
+        }
 
         // ---- phase 4: outputs of token t = r, dims 32 half .. + 31
         {
@@ -579,8 +618,6 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
         tc_fence_before();
         fence_async_smem();
         __syncthreads();                      // this chunk's x rows and accumulators are read
-        if (c + 1 < nchunks)
-            load_x(c + 1);
     }
 
     // ---- the final state, once (the stash mode leaves the committed state read-only)
