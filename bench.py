@@ -352,7 +352,11 @@ def time_launches(fn, steps, warmup, device):
 
 def form_prefill(args, device, batch=0):
     """Multi-token prefill (batch 16, T 512, contextLengths ~ U{1..512}), without and with
-    the replay stash; FP32-issue bound, reported against the FP32 FMA peak."""
+    the replay stash. Reported against the FP32 peak at the sequential form's FLOP count
+    (5 per state element and token), the measure the scope table fixes; with bf16 inputs
+    the library evaluates the recurrence in chunks of 128 tokens on the tensor cores, so
+    the MMA work as issued (against the measured bf16 GEMM rate) and the algorithmic
+    bytes (against the measured HBM copy rate) are reported beside it."""
     from linear_attention_recurrent_selective_b200 import ssu
     from linear_attention_recurrent_selective_b200.workloads import make_config
 
@@ -375,16 +379,41 @@ def form_prefill(args, device, batch=0):
     flop = tokens * H * Dm * N * 5       # per state element: mul + FMA update, FMA output
     sm = torch.cuda.get_device_properties(device).multi_processor_count
     alu_peak = sm * 128 * 2 * 1.965e9 / 1e12   # fp32 FMA lanes x 2 FLOP x max SM clock
+    tc = (case.x.dtype == torch.bfloat16 and case.B.dtype == torch.bfloat16 and N == 128
+          and Dm % 8 == 0)
+    # chunked tensor-core form: per (row, head, 64-row dim tile) and chunk of 128 tokens,
+    # C s^T and G X (3 pieces x 8 K-steps of M128 N64 K16 each), C B^T (8 of M128 N128 K16)
+    # and B^T (w dt X) (3 x 8 of M128 N64 K16)
+    chunks = int(sum(-(-int(L) // 128) for L in case.context_lengths.tolist()))
+    mma_flop = chunks * H * -(-Dm // 64) * (72 * 2 * 128 * 64 * 16 + 8 * 2 * 128 * 128 * 16)
+    tc_peak, tc_src = measured_bf16_tflops()
     forms = {}
     for name, st in (("prefill", None), ("prefill_stash", stash)):
         ms = time_launches(lambda: prefill(st), steps, warm, device)
+        # algorithmic bytes: x, z and out (and with the stash U, dA and dt) per valid
+        # token-head, B and C per token (and the stash's B), the state read (and written)
+        xb = case.x.element_size()
+        io = tokens * H * Dm * xb * 3 + tokens * H * 4 + tokens * G * N * xb * 2
+        if st is not None:
+            io += tokens * H * Dm * 4 + tokens * H * 8 + tokens * G * N * 4
+        state = b * H * Dm * N * 4 * (1 if st is not None else 2)
         forms[name] = {
             "workload": "prefill_b16_t512", "batch": b, "tokens": tokens, "ms_per_launch": ms,
             "tokens_per_s": tokens / (ms / 1e3),
+            "form": "chunked tensor-core" if tc else "sequential CUDA-core",
             "roofline": {"bound": "alu", "achieved": flop / (ms / 1e3) / 1e12,
                          "peak": alu_peak, "unit": "TFLOP/s",
                          "frac": flop / (ms / 1e3) / 1e12 / alu_peak, "traffic": None,
-                         "peak_source": "derived: SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz"}}
+                         "peak_source": "derived: SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz",
+                         "flop_count": "5 per state element and token (sequential form)"},
+            "hbm": {"algorithmic_bytes": io + state,
+                    "achieved_gbs": (io + state) / (ms / 1e3) / 1e9,
+                    "frac_of_measured": (io + state) / (ms / 1e3) / 1e9 / measured_peaks()[0]}}
+        if tc:
+            forms[name]["tensor"] = {"mma_flop_issued": mma_flop,
+                                     "achieved_tflops": mma_flop / (ms / 1e3) / 1e12,
+                                     "bf16_peak": tc_peak, "bf16_peak_source": tc_src,
+                                     "frac": mma_flop / (ms / 1e3) / 1e12 / tc_peak}
     return forms
 
 
