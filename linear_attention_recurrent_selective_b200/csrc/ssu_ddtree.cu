@@ -38,9 +38,12 @@
 // thread per node and half tile, 32 sums in registers); the dense products run with the
 // lane mapping described at TGeo, a transposing shuffle reduction leaves each lane with
 // whole rows, and out = W_i a_i + P[i][d] + D x is stored without further barriers.
+#include <type_traits>
+
 #include "ssu_async.cuh"
 #include "ssu_common.cuh"
 #include "ssu_tc.cuh"
+#include "ssu_tmap.cuh"
 
 namespace ssu {
 namespace {
@@ -141,6 +144,36 @@ __device__ __forceinline__ Item item_after(const TreeArgs &ta, const Item &u, in
             v.h = 0;
             ++v.b;
             v.slot = a.idx ? a.idx[v.b] : v.b;
+        }
+        v.g = v.h / (a.H / a.G);
+    }
+    v.row0 = v.dtile * kTile;
+    v.rows = min(kTile, a.Dm - v.row0);
+    return v;
+}
+
+// The pool slot of row b (-1 past the active rows).
+__device__ __forceinline__ int row_slot(const TreeArgs &ta, int b)
+{
+    const DecodeArgs &a = ta.d;
+    return b < a.active ? (a.idx ? a.idx[b] : b) : -1;
+}
+
+// item_after with the slot of the next row prefetched in nslot: at a row change the row
+// takes it, and the slot of the row after is loaded, a whole row ahead of its use (a load
+// consumed at once would hold up every item by its latency).
+__device__ __forceinline__ Item item_after_pf(const TreeArgs &ta, const Item &u, int dtiles,
+                                              int &nslot)
+{
+    const DecodeArgs &a = ta.d;
+    Item v = u;
+    if (++v.dtile == dtiles) {
+        v.dtile = 0;
+        if (++v.h == a.H) {
+            v.h = 0;
+            ++v.b;
+            v.slot = nslot;
+            nslot = row_slot(ta, v.b + 1);
         }
         v.g = v.h / (a.H / a.G);
     }
@@ -751,87 +784,101 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
 //
 // With bf16 B and C and dstate 64 or 128, the dense products run on the tensor cores.
 // For item (b, h, dim tile) they form one matrix product: D[i][d] = sum_n C_i[n] s0[d][n]
-// for the 128 node slots i (rows T .. 127 of C are zero) and the tile's 64 dim rows d.
+// for the 128 node slots i (slots T .. 127 hold zero C rows) and the tile's 64 dim rows d.
 // C is bf16, so it enters the MMA exactly; the committed state is split into bf16
 // pieces s0 = p1 + p2 + p3 (p1 = bf16(s0), p2 = bf16(s0 - p1), p3 = bf16(s0 - p1 - p2);
 // each difference is exact in fp32, and the three pieces carry 24 significant bits, the
-// fp32 significand), every product of two bf16 values is exact in the fp32 accumulator,
-// and D = C p3^T + C p2^T + C p1^T accumulates in fp32. An fp16 state needs two pieces
-// (11 significant bits), a bf16 state one. D lives in tensor memory: 128 lanes (node
-// slots) x 64 fp32 columns (dim rows).
+// fp32 significand), and every product of two bf16 values is exact in the fp32
+// accumulator. The pieces are stacked as the rows of one B operand (64 rows each), so a
+// single chain of dstate / 16 MMAs of N = 64 x pieces reads C once and leaves C p1^T,
+// C p2^T and C p3^T side by side in tensor memory (128 lanes = slots, 64 fp32 columns
+// per piece), summed smallest first in the epilogue. An fp16 state needs two pieces
+// (11 significant bits), a bf16 state one.
 //
 // A CTA of 16 warps takes a share of one row's items when there are at least as many
-// CTAs as rows, else a contiguous range of items. Per item, in order: the state rows and
-// the x tile (bulk copies issued during the previous item, each buffer on its own
-// mbarrier) are waited for; the state rows are split into the pieces in the
-// 128-byte-swizzled operand layout and the nodes' dt_eff and dA formed; thread 0 issues
-// the MMAs (pieces x dstate / 16 of them) and commits them to an mbarrier, while the
-// other threads start the next item's copies (the x rows one per thread), write the
-// stash's U and form the path sums, a thread per node and 16 dim rows (thread t: node
-// 32 (warp % 4) + lane, rows 16 (warp / 4) ..), with the path coefficients
-// w_im dt_jm (C_i . B_jm) built on the way; then each thread reads its node's 16
-// accumulator columns from tensor memory (a warp's lanes are the TMEM lanes of its
-// quarter), forms out = W_i D + P + D_h x and writes it over its x values in the tile,
-// which then goes out as whole 16-byte-aligned rows. Per (row, group) the row's tables
-// are built once in the CTA (see stage_row_tc): C in the operand layout, the path pairs
-// and their C_i . B_j from the row's B rows staged in shared memory, which also give
-// the stash its B.
+// CTAs as rows, else a contiguous range of items. Per (row, group) the row's tables are
+// built once (stage_row_tc): the path pairs and their C_i . B_j, and the nodes ranked by
+// path length, node i's C row going to operand row (slot) rank(i). Per item, in order:
+// the state rows (one bulk copy) and the x tile (one tensor copy, 128-byte swizzled),
+// issued during the previous item, are waited for; the state rows are split into the
+// pieces and the nodes' dt_eff and dA formed; thread 0 issues the MMAs and commits them
+// to an mbarrier, while the producer thread starts the next item's copies and every
+// thread forms its path sums: warp w takes slots 8w .. 8w + 7 with four lanes each and
+// 16 dim rows per lane, so a warp's paths are about equally long, with the coefficients
+// w_im dt_jm (C_i . B_jm) built on the way; then the stash's U is written. Once the MMAs
+// are done, the path sums and each slot's W go through shared memory (over the pieces)
+// to the epilogue thread of the slot (a warp's lanes are the TMEM lanes of its quarter),
+// which forms out = W_i D + P + D_h x and writes it over its x values in the tile; one
+// tensor store per tile sends it out.
 
 constexpr int kTcThreads = 512;       // 16 warps, one CTA per SM
-constexpr uint32_t kTcCols = 64;      // TMEM columns: the 64 dim rows of a tile
+constexpr uint32_t kTcCols = 256;     // TMEM columns: 64 dim rows per state piece (<= 3)
 
 // Shared-memory layout of the tensor-core form (byte offsets from a 1024-byte aligned
 // base). npc state pieces; E bounds the path pairs as in TLayout.
 struct TcLayout {
-    int ca, sp, raw, xs, xbytes, cb, pj, pi, par, cnt, off, da, dtv, bar, tptr, total;
+    int ca, sp, raw, xs, tp, xbytes, cb, pj, pi, par, cnt, off, sn, ns, wsl, da, dtv, bar, tptr,
+        total;
     __host__ __device__ static int up16(int v) { return (v + 15) & ~15; }
     __host__ __device__ TcLayout(int T, int N, int es_x, int es_s, int npc, int nxb)
     {
         const int E = T * (T + 1) / 2;
         ca = 0;                               // C operand: N / 64 blocks of 128 x 128 B
         sp = ca + 128 * N * 2;                // pieces: npc x N / 64 blocks of 64 x 128 B
-        // (between items the same bytes stage the row's B rows: 128 x N bf16)
-        raw = sp + (npc * kTile > 128 ? npc * kTile : 128) * N * 2;   // state rows as stored
-        xs = raw + up16(kTile * N * es_s);
-        xbytes = up16(T * kXS * es_x);
+        // (the same bytes stage the row's B rows between items, 128 x N bf16, and hand the
+        // path sums to the epilogue once an item's products are done, 32 KB)
+        int spb = (npc * kTile > 128 ? npc * kTile : 128) * N * 2;
+        spb = spb > 32768 ? spb : 32768;
+        raw = sp + spb;                       // state rows as stored
+        // x tiles: kTile * es_x / 128 blocks of tp 128-byte rows (see xt_off), each block
+        // 1024-byte aligned
+        xs = (raw + kTile * N * es_s + 1023) & ~1023;
+        tp = (T + 7) & ~7;
+        xbytes = (kTile * es_x / 128) * tp * 128;
         cb = xs + nxb * xbytes;
         pj = cb + up16(E * 4);
         pi = pj + up16(E);
         par = pi + up16(E);
         cnt = par + up16(T * 4);
         off = cnt + up16(T * 4);
-        da = off + up16((T + 1) * 4);
-        dtv = da + up16(T * 4);
-        bar = dtv + up16(T * 4);              // mbarriers: MMA, state rows, x tiles 0 / 1
+        sn = off + up16((T + 1) * 4);        // node of each operand row (slot)
+        ns = sn + up16(T);                    // slot of each node
+        wsl = ns + up16(T);                   // W of each slot's node (128 floats)
+        da = wsl + 128 * 4;                   // {dt_eff, dA} of each node (float2)
+        dtv = da;
+        bar = da + up16(T * 8);               // mbarriers: MMA, state rows, x tiles 0 / 1
         tptr = bar + 32;
         total = tptr + 16 + 1024;             // slack for aligning the base
     }
 };
 
 // Per-(row, group) tables of the tensor-core form: parents, path checks, C in the
-// operand layout, path pairs (pj: path node, pi: node) and C_i . B_j of every pair. All
-// of the row's loads are issued at once: C rows into the operand layout and B rows into
-// the piece buffer (free between items; 16-byte chunks XOR-swizzled by the row) by
-// cp.async, parents and depths into registers; the C . B products then read shared
-// memory only. The staged B rows also give the stash its B: the shares of heads hh0 ..
-// hh1 (indices within the group) of this CTA's items, each head's share being elements
-// [T N hh / hpg, T N (hh + 1) / hpg) of the row's [T][N] block.
+// operand layout, path pairs (pj: path node, pi: node) and C_i . B_j of every pair. The
+// row's B rows are fetched into the piece buffer (free between items; 16-byte chunks
+// XOR-swizzled by the row) by cp.async and its C rows into registers, all at once, while
+// parents and depths load and every node's path is walked. The nodes are then ranked by
+// path length, and node i's C row goes to operand row (slot) ns[i] = its rank (sn[] maps
+// back): the accumulator lane of a slot is its node's, and the threads that take a
+// warp's 32 slots in the per-item path sums then have paths of about equal length, so
+// that no warp runs many more path steps than its lanes need. The C . B products then
+// read shared memory only. The staged B rows also give the stash its B: the shares of
+// heads hh0 .. hh1 (indices within the group) of this CTA's items, each head's share
+// being elements [T N hh / hpg, T N (hh + 1) / hpg) of the row's [T][N] block.
 //
-// Invariant the kernel relies on when it skips an item's closing barrier: before its
-// first __syncthreads this function writes only par (plain stores) and, by cp.async, the
-// C operand and the piece buffer, which the finished item's MMAs no longer read. It must
-// not touch an x tile, cb, pj, cnt, off, sdA or sdt before that barrier, because slower
-// threads may still be writing the previous item's outputs out of its x tile.
+// The kernel calls it behind a barrier, so every buffer of the previous item is free.
 template <int N>
 __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm, int b, int g,
                              bool reporter, int hh0, int hh1)
 {
     constexpr int CPR = N / 8;                // 16-byte chunks per bf16 row
+    constexpr int CQ = 128 * CPR / kTcThreads;    // C chunks per thread (128 operand rows)
     const DecodeArgs &a = ta.d;
     const int T = ta.T, G = a.G, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float *cb = reinterpret_cast<float *>(sm + lay.cb);
     uint8_t *pj = sm + lay.pj;
     uint8_t *pi = sm + lay.pi;
+    uint8_t *sn = sm + lay.sn;
+    uint8_t *ns = sm + lay.ns;
     uint8_t *bst = sm + lay.sp;               // B rows of the row's nodes
     int *par = reinterpret_cast<int *>(sm + lay.par);
     int *cnt = reinterpret_cast<int *>(sm + lay.cnt);
@@ -839,13 +886,12 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
     const uint16_t *Cg = static_cast<const uint16_t *>(a.C);
     const uint16_t *Bg = static_cast<const uint16_t *>(a.B);
 
-    for (int k = tid; k < 128 * CPR; k += kTcThreads) {
-        const int i = k / CPR, c = k % CPR;
-        uint8_t *dst = sm + lay.ca + sw128_off(i, c, 128 * 128);
-        if (i < T)
-            cp_async16(dst, Cg + (((int64_t)b * T + i) * G + g) * N + c * 8);
-        else
-            *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    uint4 creg[CQ];                           // chunk tid + q * threads: row k / CPR
+#pragma unroll
+    for (int q = 0; q < CQ; ++q) {
+        const int k = tid + q * kTcThreads, i = k / CPR, c = k % CPR;
+        creg[q] = i < T ? *reinterpret_cast<const uint4 *>(Cg + (((int64_t)b * T + i) * G + g) * N + c * 8)
+                        : make_uint4(0u, 0u, 0u, 0u);
     }
     for (int k = tid; k < T * CPR; k += kTcThreads) {
         const int j = k / CPR, c = k % CPR;
@@ -891,8 +937,24 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
         }
         if (lane == 0)
             off[T] = carry;
+    } else if (tid >= 128 && tid < 128 + T) { // rank by path length, ties by node index
+        const int i = tid - 128, ci = cnt[i];
+        int r = 0;
+        for (int k = 0; k < T; ++k) {
+            const int ck = cnt[k];
+            r += ck < ci || (ck == ci && k < i);
+        }
+        ns[i] = static_cast<uint8_t>(r);
+        sn[r] = static_cast<uint8_t>(i);
     }
     __syncthreads();
+    // C rows into their slots; the slots past T (no node) are zero
+#pragma unroll
+    for (int q = 0; q < CQ; ++q) {
+        const int k = tid + q * kTcThreads, i = k / CPR, c = k % CPR;
+        *reinterpret_cast<uint4 *>(sm + lay.ca + sw128_off(i < T ? ns[i] : i, c, 128 * 128)) =
+            creg[q];
+    }
     if (tid < T) {
         const int c = cnt[tid], o = off[tid];
         int j = tid;
@@ -902,16 +964,16 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
             j = par[j];
         }
     }
-    cp_async_wait_all();                      // C and B rows landed
+    cp_async_wait_all();                      // B rows landed
     __syncthreads();
     const int total = off[T];
     for (int p = tid; p < total; p += kTcThreads) {
-        const int i = pi[p], j = pj[p];
+        const int i = pi[p], j = pj[p], si = ns[i];
         const uint8_t *brow = bst + j * (N * 2);
         float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < CPR; ++c) {
-            const uint4 cv = *reinterpret_cast<const uint4 *>(sm + lay.ca + sw128_off(i, c, 128 * 128));
+            const uint4 cv = *reinterpret_cast<const uint4 *>(sm + lay.ca + sw128_off(si, c, 128 * 128));
             const uint4 bv = *reinterpret_cast<const uint4 *>(brow + ((c ^ (j & 7)) << 4));
             float fc[8], fb[8];
             Vec16<__nv_bfloat16>::unpack(cv, fc);
@@ -962,7 +1024,6 @@ __device__ void split_state(const TcLayout &lay, uint8_t *sm, int rows)
             for (int q = 0; q < 8; ++q)
                 f[q] = 0.f;
         }
-        const int o = sw128_off(r, c, kTile * 128);
 #pragma unroll
         for (int p = 0; p < NPC; ++p) {
             uint32_t w[4];
@@ -974,7 +1035,7 @@ __device__ void split_state(const TcLayout &lay, uint8_t *sm, int rows)
                 f[2 * q + 1] -= back.y;
                 memcpy(&w[q], &h, 4);
             }
-            *reinterpret_cast<uint4 *>(sm + lay.sp + p * (kTile * N * 2) + o) =
+            *reinterpret_cast<uint4 *>(sm + lay.sp + sw128_off(p * kTile + r, c, NPC * kTile * 128)) =
                 make_uint4(w[0], w[1], w[2], w[3]);
         }
     }
@@ -1001,52 +1062,122 @@ __device__ __forceinline__ void bulk_raw(const TreeArgs &ta, const TcLayout &lay
         bulk_load(sm + lay.raw + o, src + o, bytes - o < part ? bytes - o : part, bar);
 }
 
-// The x tile: one copy per node row (rows 16-byte aligned), spread over nt issuing
-// threads (this one is t; t = 0 arms the barrier).
+// Byte offset in an x tile of the 16-byte chunk holding dims d .. d + 16 / es - 1 of node
+// i (d a multiple of 16 / es). The tile is kTile * es / 128 blocks of tp rows of 128 bytes
+// (64 / es dims), and the chunks of row i are XOR-swizzled by i % 8: the layout the tensor
+// copies' 128-byte swizzle gives a 1024-byte aligned box. Lanes reading the same chunk of
+// different rows (the path sums) or their own rows (the epilogue) thereby spread over the
+// banks.
 template <typename X>
-__device__ __forceinline__ void bulk_x(const TreeArgs &ta, const TcLayout &lay, uint8_t *sm,
-                                       const Item &u, int xbuf, uint64_t *bar, int t, int nt,
-                                       uint32_t extra)
+__device__ __forceinline__ int xt_off(int i, int d, int tp)
+{
+    constexpr int es = (int)sizeof(X), per = 128 / es;
+    const int c = (d % per) * es / 16;
+    return (d / per) * (tp * 128) + i * 128 + ((c ^ (i & 7)) << 4);
+}
+
+// Element d of node i of an x tile, widened.
+template <typename X>
+__device__ __forceinline__ float xt_at(const uint8_t *xs, int i, int d, int tp)
+{
+    constexpr int es = (int)sizeof(X), per16 = 16 / es;
+    const uint8_t *p = xs + xt_off<X>(i, d - d % per16, tp) + (d % per16) * es;
+    if constexpr (es == 4)
+        return *reinterpret_cast<const float *>(p);
+    else
+        return bits_f32(*reinterpret_cast<const uint16_t *>(p),
+                        std::is_same<X, __half>::value ? SSU_F16 : SSU_BF16);
+}
+
+// The x tile of item u by one tensor copy per 128-byte block (thread `issuer` arms the
+// barrier and issues them): rows 0 .. T - 1 of the tile, dims past Dm read as zero.
+template <typename X>
+__device__ __forceinline__ void tma_x(const TreeArgs &ta, const CUtensorMap *xmap, uint8_t *xs,
+                                      const Item &u, uint64_t *bar, uint32_t extra, int tp)
+{
+    constexpr int nblk = kTile * (int)sizeof(X) / 128, per = 128 / (int)sizeof(X);
+    mbar_arrive_expect_tx(bar, (uint32_t)(nblk * ta.T * 128) + extra);
+#pragma unroll
+    for (int q = 0; q < nblk; ++q)
+        tma_load_rows(xs + q * tp * 128, xmap, u.row0 + q * per, u.h, u.b * ta.T, bar);
+}
+
+// The x tile of item u with plain loads, in the same layout (x rows not 16-byte aligned,
+// or too short for a tensor copy): dims >= u.rows are 0.
+template <typename X>
+__device__ void stage_x_tc(const TreeArgs &ta, uint8_t *xs, const Item &u, int tp)
 {
     const DecodeArgs &a = ta.d;
-    const int T = ta.T;
-    constexpr int es = (int)sizeof(X);
-    const uint32_t rb = (uint32_t)(u.rows * es);
-    if (t == 0)
-        mbar_arrive_expect_tx(bar, rb * (uint32_t)T + extra);
-    for (int i = t; i < T; i += nt)
-        bulk_load(sm + lay.xs + xbuf * lay.xbytes + i * kXS * es,
-                  static_cast<const X *>(a.x) + (((int64_t)u.b * T + i) * a.H + u.h) * a.Dm +
-                      u.row0,
-                  rb, bar);
+    const int T = ta.T, H = a.H, Dm = a.Dm;
+    constexpr int per16 = 16 / (int)sizeof(X);            // dims per 16-byte chunk
+    for (int e = threadIdx.x; e < T * (kTile / per16); e += kTcThreads) {
+        const int i = e / (kTile / per16), d = per16 * (e % (kTile / per16));
+        const int64_t src = (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d;
+        float f[per16];
+#pragma unroll
+        for (int q = 0; q < per16; ++q)
+            f[q] = d + q < u.rows ? ld_f32(a.x, a.x_dtype, src + q) : 0.f;
+        *reinterpret_cast<uint4 *>(xs + xt_off<X>(i, d, tp)) = Vec16<X>::pack(f);
+    }
 }
 
-// 16 consecutive x values of node i from dim row d0 of an x tile, and the same positions
-// overwritten (rounded to X).
+// 16 consecutive x values of node i from dim row d0 (a multiple of 16) of an x tile, and
+// the same positions overwritten (rounded to X).
 template <typename X>
-__device__ __forceinline__ void x_seg16(const uint8_t *xs, int i, int d0, float (&f)[16])
+__device__ __forceinline__ void x_seg16(const uint8_t *xs, int i, int d0, int tp, float (&f)[16])
 {
     constexpr int per = 16 / (int)sizeof(X);
-    const uint4 *p = reinterpret_cast<const uint4 *>(xs + (i * kXS + d0) * (int)sizeof(X));
 #pragma unroll
     for (int q = 0; q < 16 / per; ++q)
-        Vec16<X>::unpack(p[q], f + per * q);
+        Vec16<X>::unpack(*reinterpret_cast<const uint4 *>(xs + xt_off<X>(i, d0 + per * q, tp)),
+                         f + per * q);
+}
+
+// The same 16 values as 8 pairs (dims d0 + 2q, d0 + 2q + 1), for packed arithmetic.
+template <typename X>
+__device__ __forceinline__ void x_pairs16(const uint8_t *xs, int i, int d0, int tp, float2 (&f)[8])
+{
+    if constexpr (sizeof(X) == 4) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = *reinterpret_cast<const float4 *>(xs + xt_off<X>(i, d0 + 4 * q, tp));
+            f[2 * q] = make_float2(v.x, v.y);
+            f[2 * q + 1] = make_float2(v.z, v.w);
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(xs + xt_off<X>(i, d0 + 8 * q, tp));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if constexpr (std::is_same<X, __nv_bfloat16>::value) {
+                    f[4 * q + k] = make_float2(__uint_as_float(w[k] << 16),
+                                               __uint_as_float(w[k] & 0xFFFF0000u));
+                } else {
+                    __half2 h;
+                    memcpy(&h, &w[k], 4);
+                    f[4 * q + k] = __half22float2(h);
+                }
+            }
+        }
+    }
 }
 
 template <typename X>
-__device__ __forceinline__ void put_seg16(uint8_t *xs, int i, int d0, const float (&y)[16])
+__device__ __forceinline__ void put_seg16(uint8_t *xs, int i, int d0, int tp, const float (&y)[16])
 {
     constexpr int per = 16 / (int)sizeof(X);
-    uint4 *p = reinterpret_cast<uint4 *>(xs + (i * kXS + d0) * (int)sizeof(X));
 #pragma unroll
     for (int q = 0; q < 16 / per; ++q)
-        p[q] = Vec16<X>::pack(y + per * q);
+        *reinterpret_cast<uint4 *>(xs + xt_off<X>(i, d0 + per * q, tp)) = Vec16<X>::pack(y + per * q);
 }
 
 // U of the item (x widened to fp32): 16 bytes of the tile per task, 16-byte stores; thread
 // t of the nt taking part.
 template <typename X>
-__device__ void stash_u_tc(const TreeArgs &ta, const Item &u, const uint8_t *xs, int t, int nt)
+__device__ void stash_u_tc(const TreeArgs &ta, const Item &u, const uint8_t *xs, int tp, int t,
+                           int nt)
 {
     const DecodeArgs &a = ta.d;
     const int T = ta.T, H = a.H, Dm = a.Dm;
@@ -1056,7 +1187,7 @@ __device__ void stash_u_tc(const TreeArgs &ta, const Item &u, const uint8_t *xs,
             const int i = e / (kTile / per), d = per * (e % (kTile / per));
             if (d < u.rows) {
                 float f[per];
-                Vec16<X>::unpack(*reinterpret_cast<const uint4 *>(xs + (i * kXS + d) * (int)sizeof(X)), f);
+                Vec16<X>::unpack(*reinterpret_cast<const uint4 *>(xs + xt_off<X>(i, d, tp)), f);
                 float *dst = ta.st_U + (((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d;
 #pragma unroll
                 for (int q = 0; q < per / 4; ++q)
@@ -1070,7 +1201,27 @@ __device__ void stash_u_tc(const TreeArgs &ta, const Item &u, const uint8_t *xs,
             const int i = e / kTile, d = e % kTile;
             if (d < u.rows)
                 ta.st_U[(((int64_t)u.b * T + i) * H + u.h) * Dm + u.row0 + d] =
-                    xs_at(xs, a.x_dtype, i * kXS + d);
+                    xt_at<X>(xs, i, d, tp);
+        }
+    }
+}
+
+// dt_eff and dA of every node for the item's head (node threadIdx.x, from its prefetched
+// dt) into shared memory as {dt_eff, dA} pairs, and into the stash once per (row, head).
+__device__ __forceinline__ void node_values_tc(const TreeArgs &ta, float2 *sdtA, const Item &u,
+                                               float dt_mine, const HeadVals &hv)
+{
+    const DecodeArgs &a = ta.d;
+    const int T = ta.T, tid = threadIdx.x;
+    if (tid < T) {
+        const int64_t bi = (int64_t)u.b * T + tid;
+        const float v = dt_mine + hv.bias;
+        const float dte = a.softplus ? softplus_f(v) : v;
+        const float dA = expf(hv.A * dte);
+        sdtA[tid] = make_float2(dte, dA);
+        if (u.dtile == 0) {
+            ta.st_dA[bi * a.H + u.h] = dA;
+            ta.st_dt[bi * a.H + u.h] = dte;
         }
     }
 }
@@ -1092,28 +1243,37 @@ __device__ __forceinline__ void cta_range(int64_t nitems, int64_t per_row, int r
     }
 }
 
-// ocopy: out rows are 16-byte aligned, so the outputs go out through the x tile as whole
-// rows (each node's dim rows are contiguous in out); otherwise each thread stores its own.
+// xtma / otma: the x tiles come in and the outputs go out by tensor copies (tensor maps
+// xmap / omap over x and out); otherwise the x tiles are staged with plain loads and each
+// thread stores its own outputs.
 template <typename S, typename X, int N>
 __global__ void __launch_bounds__(kTcThreads, 1)
-ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const int64_t nitems,
-                     const int nxb, const int xasync, const int ocopy)
+ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const __grid_constant__ CUtensorMap xmap,
+                     const __grid_constant__ CUtensorMap omap, const int dtiles,
+                     const int64_t nitems, const int nxb, const int xtma, const int otma)
 {
     constexpr int NPC = Pieces<S>::n;
     constexpr int es_x = (int)sizeof(X);
-    constexpr uint32_t kIdesc = idesc_bf16_f32(128, kTile);
+    constexpr int nblk = kTile * es_x / 128, per_blk = 128 / es_x;   // x tile blocks, dims each
+    constexpr uint32_t kIdesc = idesc_bf16_f32(128, NPC * kTile);
+    // the thread that issues every copy of the items' inputs and every output store: lane 0
+    // of warp 1, whose path-sum slots have short paths (as have warp 0's: thread 0 issues
+    // the MMAs)
+    constexpr int kProducer = 32;
     extern __shared__ __align__(16) uint8_t sm_dyn[];
     uint8_t *sm = sm_dyn + ((1024 - (smem_u32(sm_dyn) & 1023)) & 1023);
     const DecodeArgs &a = ta.d;
     const int T = ta.T, H = a.H, Dm = a.Dm;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool producer = tid == kProducer;
     const TcLayout lay(T, N, es_x, (int)sizeof(S), NPC, nxb);
+    const int tp = lay.tp;
     const float *cb = reinterpret_cast<const float *>(sm + lay.cb);
     const uint8_t *pj = sm + lay.pj;
     const int *cnt = reinterpret_cast<const int *>(sm + lay.cnt);
     const int *off = reinterpret_cast<const int *>(sm + lay.off);
-    float *sdA = reinterpret_cast<float *>(sm + lay.da);
-    float *sdt = reinterpret_cast<float *>(sm + lay.dtv);
+    const uint8_t *sn = sm + lay.sn;
+    float2 *sdtA = reinterpret_cast<float2 *>(sm + lay.da);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + lay.bar);     // MMA completion
     uint64_t *sbar = bar + 1;                                         // state rows landed
     uint64_t *xbar = bar + 2;                                         // x tile 0 / 1 landed
@@ -1131,38 +1291,50 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tptr;
-    // this thread's node (TMEM lane) and its 16 dim rows (TMEM columns)
+    // this thread's slot (TMEM lane; its node is sn[ni]) and its 16 dim rows (TMEM columns)
     const int ni = 32 * (warp & 3) + lane, d0 = 16 * (warp >> 2);
+    // Its path sums: slot pslot (of warp w's 8 slots 8w .. 8w + 7, four lanes each) over
+    // dim rows pd0 .. pd0 + 15. The slots are ranked by path length, so the paths of a
+    // warp's slots are about equally long, and the four warps of a scheduler (w, w + 4,
+    // w + 8, w + 12) take slot groups from every quarter of the ranking. The sums reach the
+    // slot's epilogue thread through shared memory.
+    const int pslot = 8 * warp + (lane >> 2), pd0 = 16 * (lane & 3);
     const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)d0;
     uint32_t phase = 0;                  // parity of the MMA barrier's next phase
     bool mma_out = false;                // an MMA wait gave up (its phase is still awaited)
     // copies in flight (uniform): state rows, x tiles by buffer bit; parities likewise
     uint32_t s_out = 0, x_out = 0, sph = 0, xph = 0;
 
-    const bool x_mid = xasync && nxb == 2;
+    // with two x buffers the next item's tile is fetched while this one computes
+    const bool x_mid = xtma && nxb == 2;
     int64_t first, last;
     cta_range(nitems, nitems / a.active, a.active, first, last);
     auto xbuf_of = [&](int64_t it) { return nxb == 2 ? (int)((it - first) & 1) : 0; };
-    // copies of item w: the state block by thread 0, the x rows one per thread from the
-    // top thread down (measured: issuing them from warps 0-3, which also issue the MMAs
-    // and hold the shallowest nodes, makes the launch 7 % slower)
-    const int xt = kTcThreads - 1 - tid;
-    auto issue = [&](const Item &w, int64_t wit, bool with_x) {
-        const int xb = xbuf_of(wit);
-        bulk_raw<S, N>(ta, lay, sm, w, sbar, tid == 0,
+    // the state block of item w (the raw staging must be free)
+    auto issue_s = [&](const Item &w, int64_t wit) {
+        bulk_raw<S, N>(ta, lay, sm, w, sbar, producer,
                        fault_tx(kFaultTreeState, -1, (int)(wit - first)));
-        if (with_x)
-            bulk_x<X>(ta, lay, sm, w, xb, xbar + xb, xt, kTcThreads,
-                      fault_tx(kFaultTreeX, -1, (int)(wit - first)));
         s_out = 1;
-        if (with_x)
-            x_out |= 1u << xb;
+    };
+    // the x tile of item w into its buffer (no thread may still read that buffer; the
+    // producer first waits for its own output stores to have read it)
+    auto issue_x = [&](const Item &w, int64_t wit) {
+        const int xb = xbuf_of(wit);
+        if (producer) {
+            bulk_wait_read_all();
+            tma_x<X>(ta, &xmap, sm + lay.xs + xb * lay.xbytes, w, xbar + xb,
+                     fault_tx(kFaultTreeX, -1, (int)(wit - first)), tp);
+        }
+        x_out |= 1u << xb;
     };
     Item u = item_at(ta, first < last ? first : 0, dtiles);
+    int nslot = row_slot(ta, u.b + 1);   // slot of the row after u's
     float dt_next = 0.f;                 // node tid's dt and the head's scalars, next item
     HeadVals hv_next = {0.f, 0.f, 0.f};
     if (first < last && u.valid(a.P)) {
-        issue(u, first, xasync);
+        issue_s(u, first);
+        if (xtma)
+            issue_x(u, first);
         dt_next = dt_of(ta, u);
         hv_next = head_vals(a, u.h);
     }
@@ -1171,7 +1343,7 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
     for (int64_t it = first; it < last; ++it, u = v) {
         const bool has_next = it + 1 < last;
         if (has_next)
-            v = item_after(ta, u, dtiles);
+            v = item_after_pf(ta, u, dtiles, nslot);
         const bool next_valid = has_next && v.valid(a.P);
         if (!u.valid(a.P)) {
             if (u.slot < 0) {            // padding row: zero outputs at every node
@@ -1185,13 +1357,16 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
                 atomicOr(a.err, SSU_FLAG_INDEX_RANGE);
             }
             if (next_valid) {            // this item used no buffer: start the next one
-                issue(v, it + 1, xasync);
+                issue_s(v, it + 1);
+                if (xtma)
+                    issue_x(v, it + 1);
                 dt_next = dt_of(ta, v);
                 hv_next = head_vals(a, v.h);
             }
             continue;
         }
-        // (every thread passed the previous item's closing barrier)
+        // (every thread passed the previous item's closing barrier, or its epilogue barrier
+        // and the next one below)
         uint8_t *xs = sm + lay.xs + xbuf_of(it) * lay.xbytes;
         if (u.b != cur_b || u.g != cur_g) {
             // heads of (u.b, u.g) whose dim tile 0 lies in this CTA's range: their B stash
@@ -1201,13 +1376,18 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
             const int64_t i1 = (last < rs + (int64_t)H * dtiles ? last : rs + (int64_t)H * dtiles) - rs;
             const int hlo = max((int)((i0 + dtiles - 1) / dtiles), u.g * hpg);
             const int hhi = min((int)((i1 - 1) / dtiles), (u.g + 1) * hpg - 1);
+            __syncthreads();             // the previous item's epilogue is done with its buffers
             stage_row_tc<N>(ta, lay, sm, u.b, u.g, u.h == 0 && u.dtile == 0, hlo - u.g * hpg,
                             hhi - u.g * hpg);
             cur_b = u.b;
             cur_g = u.g;
         }
-        if (!xasync)
-            stage_x_plain<kTcThreads>(ta, xs, u);
+        if (!xtma) {
+            if (producer)
+                bulk_wait_read_all();    // an earlier output store has read this buffer
+            __syncthreads();
+            stage_x_tc<X>(ta, xs, u, tp);
+        }
         // a copy counts as landed (its in-flight bit cleared) only once its wait succeeded,
         // so that after a give-up the final drain waits for it again
         bool landed = true;
@@ -1236,50 +1416,58 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
         const HeadVals hv = hv_next;
         split_state<S, N>(lay, sm, u.rows);
         fence_async_smem();              // operands visible to the tensor cores
-        node_values(ta, sdA, sdt, u, dt_next, hv);
+        node_values_tc(ta, sdtA, u, dt_next, hv);
         __syncthreads();
         if (tid == 0 && !fault_tx(kFaultTreeMma, -1, (int)(it - first))) {
             tc_fence_after();
             const uint32_t base = smem_u32(sm);
             uint32_t acc = 0;
 #pragma unroll
-            for (int p = NPC - 1; p >= 0; --p)        // smallest piece first
+            for (int kb = 0; kb < N / 64; ++kb)
 #pragma unroll
-                for (int kb = 0; kb < N / 64; ++kb)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t ad = desc_k_sw128(base + lay.ca + kb * 16384 + kk * 32);
-                        const uint64_t bd = desc_k_sw128(base + lay.sp + p * (kTile * N * 2) +
-                                                         kb * (kTile * 128) + kk * 32);
-                        tc_mma_bf16(tmem, ad, bd, kIdesc, acc);
-                        acc = 1;
-                    }
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = desc_k_sw128(base + lay.ca + kb * 16384 + kk * 32);
+                    const uint64_t bd = desc_k_sw128(base + lay.sp + kb * (NPC * kTile * 128) +
+                                                     kk * 32);
+                    tc_mma_bf16(tmem, ad, bd, kIdesc, acc);
+                    acc = 1;
+                }
             tc_commit(bar);
         }
-        if (next_valid) {                // raw staging consumed by the split
-            issue(v, it + 1, x_mid);
+        if (next_valid) {
+            issue_s(v, it + 1);          // the raw staging was consumed by the split
+            // Every thread has finished the previous item, so the other x buffer (the
+            // previous item's) is free once the producer's store of its outputs has read
+            // it: one tensor copy brings the next item's tile there while this one computes.
+            if (x_mid)
+                issue_x(v, it + 1);
             dt_next = dt_of(ta, v);
             hv_next = head_vals(a, v.h);
         }
-        stash_u_tc<X>(ta, u, xs, tid, kTcThreads);
 
-        // path sums of node ni over rows d0 .. d0 + 15 while the MMAs run
-        float ps[16];
+        // path sums of slot pslot's node over rows pd0 .. pd0 + 15 while the MMAs run
+        float2 ps[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-            ps[e] = 0.f;
+        for (int e = 0; e < 8; ++e)
+            ps[e] = make_float2(0.f, 0.f);
         float wi = 1.f;
-        const int cn = ni < T ? cnt[ni] : 0, o = ni < T ? off[ni] : 0;
-        for (int k = 0; k < cn; ++k) {
-            const int j = pj[o + k];
-            const float cf = wi * sdt[j] * cb[o + k];
-            wi *= sdA[j];
-            float xv[16];
-            x_seg16<X>(xs, j, d0, xv);
+        {
+            const int pnode = pslot < T ? sn[pslot] : 0;
+            const int cn = pslot < T ? cnt[pnode] : 0, o = off[pnode];
+            for (int k = 0; k < cn; ++k) {
+                const int j = pj[o + k];
+                const float2 tA = sdtA[j];                // {dt_eff, dA}
+                const float cf = wi * tA.x * cb[o + k];
+                wi *= tA.y;
+                float2 xv[8];
+                x_pairs16<X>(xs, j, pd0, tp, xv);
+                const float2 c2 = make_float2(cf, cf);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                ps[e] = fmaf(cf, xv[e], ps[e]);
+                for (int e = 0; e < 8; ++e)
+                    ps[e] = __ffma2_rn(c2, xv[e], ps[e]);
+            }
         }
+        stash_u_tc<X>(ta, u, xs, tp, tid, kTcThreads);
         const bool ok = mbar_wait(bar, phase);
         if (__syncthreads_or(!ok)) {     // the MMAs never completed: give up on the launch
             if (tid == 0 && a.err)
@@ -1289,52 +1477,82 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
         }
         phase ^= 1u;
         tc_fence_after();
-        float dv[16];
-        tmem_ld16(taddr, dv);
+        // hand over the path sums (the piece buffer is free: the products are done): slot s
+        // takes 256 bytes, its 16-byte chunk c (dims 4c .. 4c + 3) at position c ^ (s % 16),
+        // so that the epilogue's lanes (consecutive slots, the same chunks) spread over the
+        // banks; and W of every slot's node
+        uint8_t *pex = sm + lay.sp;
+        float *wsl = reinterpret_cast<float *>(sm + lay.wsl);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<float4 *>(pex + pslot * 256 + (((pd0 / 4 + c) ^ (pslot & 15)) << 4)) =
+                make_float4(ps[2 * c].x, ps[2 * c].y, ps[2 * c + 1].x, ps[2 * c + 1].y);
+        if ((lane & 3) == 0)
+            wsl[pslot] = wi;
+        __syncthreads();
+        float pv[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float4 v4 =
+                *reinterpret_cast<const float4 *>(pex + ni * 256 + (((d0 / 4 + c) ^ (ni & 15)) << 4));
+            pv[4 * c] = v4.x;
+            pv[4 * c + 1] = v4.y;
+            pv[4 * c + 2] = v4.z;
+            pv[4 * c + 3] = v4.w;
+        }
+        const float wn = wsl[ni];
+        const int node = ni < T ? sn[ni] : 0;
+        float dv[16];                    // the pieces' products, smallest first
+        tmem_ld16(taddr + (uint32_t)((NPC - 1) * kTile), dv);
+#pragma unroll
+        for (int p = NPC - 2; p >= 0; --p) {
+            float dp[16];
+            tmem_ld16(taddr + (uint32_t)(p * kTile), dp);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                dv[e] += dp[e];
+        }
         const bool mine = ni < T && d0 < u.rows;
         float y[16];
         if (mine) {
             float xv[16];
-            x_seg16<X>(xs, ni, d0, xv);
+            x_seg16<X>(xs, node, d0, tp, xv);
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-                y[e] = cn > 0 ? fmaf(wi, dv[e], ps[e]) + hv.D * xv[e] : 0.f;
+                y[e] = cnt[node] > 0 ? fmaf(wn, dv[e], pv[e]) + hv.D * xv[e] : 0.f;
         }
         tc_fence_before();
-        if (ocopy) {
+        if (otma) {
+            // the outputs over the x values in the tile, then one tensor store per block
+            // (dims past Dm are not written)
             if (mine)
-                put_seg16<X>(xs, ni, d0, y);
-            fence_async_smem();          // these writes before any copy refills the tile
+                put_seg16<X>(xs, node, d0, tp, y);
+            fence_async_smem();          // these writes visible to the store
             __syncthreads();             // the tile holds every output of the item
-            const int cpr = u.rows * es_x / 16;
-            X *og = static_cast<X *>(a.out);
-            for (int k = tid; k < T * cpr; k += kTcThreads) {
-                const int i = k / cpr, c = k % cpr;
-                *reinterpret_cast<uint4 *>(og + (((int64_t)u.b * T + i) * H + u.h) * Dm +
-                                           u.row0 + c * (16 / es_x)) =
-                    *reinterpret_cast<const uint4 *>(xs + i * kXS * es_x + c * 16);
+            if (producer) {
+#pragma unroll
+                for (int q = 0; q < nblk; ++q)
+                    tma_store_rows(&omap, xs + q * tp * 128, u.row0 + q * per_blk, u.h, u.b * T);
+                bulk_commit_group();
             }
         } else if (mine) {
-            const int64_t base = (((int64_t)u.b * T + ni) * H + u.h) * Dm + u.row0 + d0;
+            const int64_t base = (((int64_t)u.b * T + node) * H + u.h) * Dm + u.row0 + d0;
 #pragma unroll
             for (int e = 0; e < 16; ++e)
                 if (d0 + e < u.rows)
                     st_f32(a.out, a.x_dtype, base + e, y[e]);
         }
         // Every read of this item's buffers done. Not needed when the x tile is double-
-        // buffered and the next item is valid: until the next item's first barrier a
-        // thread writes only buffers the output copy-out does not read (par, and by
-        // cp.async the C operand and the piece buffer: the invariant stated at
-        // stage_row_tc), and this item's x tile is refilled only after that barrier.
-        // The parity cases with several items per CTA crossing a (row, group) change
-        // (tests/test_gpu_ddtree.py, many rows over groups and dim tiles) run this path.
+        // buffered and the next item is valid: until the next item's first barrier (its
+        // row staging starts with one) a thread writes nothing this item still reads, and
+        // this item's x tile is refilled only after that barrier (by the producer, once its
+        // store has read the tile). The parity cases with several items per CTA crossing a
+        // (row, group) change (tests/test_gpu_ddtree.py, many rows over groups and dim
+        // tiles) run this path.
         if (!(x_mid && next_valid))
             __syncthreads();
-        if (next_valid && xasync && !x_mid) {
-            bulk_x<X>(ta, lay, sm, v, 0, xbar, xt, kTcThreads,
-                      fault_tx(kFaultTreeX, -1, (int)(it + 1 - first)));
-            x_out |= 1u;
-        }
+        if (next_valid && xtma && !x_mid)
+            issue_x(v, it + 1);
     }
     // No copy outlives the CTA and no MMA outlives its TMEM: after a give-up every copy
     // still marked in flight and the awaited MMA phase are waited for once more (bounded).
@@ -1347,6 +1565,8 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
             mbar_wait(xbar + k, (xph >> k) & 1u);
     if (mma_out)
         mbar_wait(bar, phase);
+    if (producer)
+        bulk_wait_all();                 // the output stores are complete
     cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
@@ -1355,9 +1575,10 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, cons
 }
 
 // The tensor-core form when it applies (bf16 B and C with 16-byte aligned C, dstate 64 or
-// 128, layout within the shared-memory limit); -1 otherwise.
+// 128, layout within the shared-memory limit); -1 otherwise. x and out take tensor copies
+// when their rows allow (16-byte aligned, at least 128 bytes of dims).
 template <typename S, typename X, int N>
-int launch_tc_x(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles, int xasync)
+int launch_tc_x(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles)
 {
     constexpr int es_x = (int)sizeof(X);
     int nxb = 2;
@@ -1371,15 +1592,19 @@ int launch_tc_x(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtil
     const KernelFacts *f = kernel_facts<ssu_ddtree_tc_kernel<S, X, N>>(kTcThreads, kSmemMax);
     if (!f || f->status != SSU_OK)
         return SSU_ERR_CUDA;
-    const int ocopy = (reinterpret_cast<uintptr_t>(a.d.out) & 15) == 0 &&
-                      ((int64_t)a.d.Dm * es_x) % 16 == 0;
+    CUtensorMap xmap, omap;
+    memset(&xmap, 0, sizeof xmap);
+    memset(&omap, 0, sizeof omap);
+    const int64_t rows = (int64_t)a.d.active * a.T;    // the rows the items touch
+    const int xtma = encode_rows_map(&xmap, a.d.x, a.d.x_dtype, a.d.Dm, a.d.H, rows, a.T);
+    const int otma = encode_rows_map(&omap, a.d.out, a.d.x_dtype, a.d.Dm, a.d.H, rows, a.T);
     const int64_t grid = nitems < f->sms ? nitems : f->sms;
     return launch_kernel(ssu_ddtree_tc_kernel<S, X, N>, (unsigned)grid, kTcThreads, lay.total,
-                         stream, a, dtiles, nitems, nxb, xasync, ocopy);
+                         stream, a, xmap, omap, dtiles, nitems, nxb, xtma, otma);
 }
 
 template <typename S, int N>
-int launch_tc(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles, int xasync)
+int launch_tc(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles)
 {
     if constexpr (N != 64 && N != 128) {
         return -1;
@@ -1387,9 +1612,9 @@ int launch_tc(const TreeArgs &a, cudaStream_t stream, int64_t nitems, int dtiles
         if (a.d.bc_dtype != SSU_BF16 || (reinterpret_cast<uintptr_t>(a.d.C) & 15) != 0)
             return -1;
         switch (a.d.x_dtype) {
-        case SSU_F32: return launch_tc_x<S, float, N>(a, stream, nitems, dtiles, xasync);
-        case SSU_F16: return launch_tc_x<S, __half, N>(a, stream, nitems, dtiles, xasync);
-        default: return launch_tc_x<S, __nv_bfloat16, N>(a, stream, nitems, dtiles, xasync);
+        case SSU_F32: return launch_tc_x<S, float, N>(a, stream, nitems, dtiles);
+        case SSU_F16: return launch_tc_x<S, __half, N>(a, stream, nitems, dtiles);
+        default: return launch_tc_x<S, __nv_bfloat16, N>(a, stream, nitems, dtiles);
         }
     }
 }
@@ -1406,7 +1631,7 @@ int launch_n(const TreeArgs &a, cudaStream_t stream)
     // x rows go through cp.async when every 16-byte chunk of a tile row is aligned
     const int xasync = (reinterpret_cast<uintptr_t>(a.d.x) & 15) == 0 &&
                        ((int64_t)a.d.Dm * es_x) % 16 == 0;
-    const int tc = launch_tc<S, N>(a, stream, nitems, dtiles, xasync);
+    const int tc = launch_tc<S, N>(a, stream, nitems, dtiles);
     if (tc >= 0)
         return tc;
     int nxb = 2;
