@@ -77,6 +77,50 @@ def test_ddtree_tensor_core_types(orc, N, sdt, Dm, H, G, T, xdt, tree):
     compare_ddtree(orc, case)
 
 
+def _shifted(t):
+    """A copy of t whose data starts one element past a 16-byte boundary."""
+    buf = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+    v = buf[1:].view(t.shape)
+    v.copy_(t)
+    return v
+
+
+# The tensor-core form moves the x tiles in and the outputs out by tensor copies when
+# their rows allow it (16-byte aligned, 128 bytes of dims or more), and by plain loads and
+# stores otherwise; each side decides for itself. Here one side is shifted off the
+# 16-byte boundary, so the launch mixes the two ways.
+@pytest.mark.parametrize("shift_x,shift_out", [(True, False), (False, True)])
+def test_ddtree_tensor_core_mixed_copy_paths(orc, shift_x, shift_out):
+    case = make_case(seed=656, batch=3, P=5, T=40, H=4, G=1, Dm=64, N=128, x_dtype=BF16,
+                     bc_dtype=BF16, tree="random")
+    out_o, st_o, err_o = orc.ddtree_case(case)
+    d = gpu_run.dev(case)
+    x = _shifted(d.x) if shift_x else d.x
+    out = torch.full_like(d.x, float("nan"))
+    if shift_out:
+        out = _shifted(out)
+    st = gpu_run.new_stash(case)
+    e = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pool = d.pool.clone()
+    ssu.ssu_ddtree(x, d.A, d.B, d.C, d.dt, pool, out, d.parent_ids, d.depths, st,
+                   dt_bias=d.dt_bias, D=d.D, state_indices=d.state_indices,
+                   active_batch=case.active, dt_softplus=case.dt_softplus, err_flags=e,
+                   slot_stride=case.slot_stride, P=case.P)
+    torch.cuda.synchronize()
+    assert int(e.item()) == err_o
+    check_out(out.cpu(), out_o, BF16)
+    assert same_bits(pool.cpu(), case.pool)
+    assert same_bits(st[1].cpu(), st_o[1]) and same_bits(st[2].cpu(), st_o[2])
+
+
+def test_ddtree_tensor_core_single_x_buffer(orc):
+    # fp32 x at 128 nodes leaves room for one x tile only: the next item's tile is then
+    # fetched after the item's closing barrier, behind its output store
+    case = make_case(seed=657, batch=3, P=5, T=128, H=3, G=1, Dm=64, N=128, x_dtype=F32,
+                     bc_dtype=BF16, tree="random")
+    compare_ddtree(orc, case)
+
+
 @pytest.mark.parametrize("H,G,Dm", [(2, 1, 16), (4, 2, 80), (3, 3, 64)])
 def test_ddtree_more_rows_than_ctas(orc, H, G, Dm):
     """160 rows over at most 148 CTAs: contiguous item ranges that cross rows, so a CTA
