@@ -71,7 +71,8 @@ constexpr int kOffW = kOffS;                      // (w dt X)^T pieces [d][m]  (
 constexpr int kPieceN = 2 * kBlkN;
 constexpr int kOffBT = kOffS + kPW * kPieceN;     // B^T [n][m]
 constexpr int kOffXT = kOffBT + 2 * kBlkM;        // X^T [d][m]
-constexpr int kOffX = kOffXT + kPieceN;           // x rows [t][d], 128 B a row (epilogue)
+constexpr int kOffX = kOffXT + kPieceN;           // x rows [t][d], 128 B a row (epilogue;
+                                                   // chunks swizzled by t % 8)
 constexpr int kOffXL = kOffG + 2 * kPieceG;       // where the next chunk's x rows land: in
                                                   // the third G piece, free from the last
                                                   // products' completion to phase 2
@@ -384,12 +385,16 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
                 }
             tc_commit(bar);
         }
-        {   // the x rows from their landing buffer to the epilogue's buffer
+        {   // the x rows from their landing buffer to the epilogue's buffer, the 16-byte
+            // chunks of row t XOR-swizzled by t % 8: the epilogue's lanes read the same
+            // chunk of consecutive rows, which then fall on different bank groups
             const uint4 *src = reinterpret_cast<const uint4 *>(sm + kOffXL);
             uint4 *dst = reinterpret_cast<uint4 *>(sm + kOffX);
 #pragma unroll
-            for (int k = 0; k < kL * 8 / kThr; ++k)
-                dst[tid + kThr * k] = src[tid + kThr * k];
+            for (int k = 0; k < kL * 8 / kThr; ++k) {
+                const int e = tid + kThr * k, t = e >> 3;
+                dst[t * 8 + ((e & 7) ^ (t & 7))] = src[e];
+            }
         }
         {   // B^T: one 8 x 8 block per thread. Within each group of 8 lanes the blocks run
             // along a diagonal (n-blocks a, m-blocks a + s), so that both the reads (rows
@@ -570,11 +575,12 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
                 const int64_t xi = (((int64_t)b * T + t0 + t) * H + h) * Dm + row0 + 32 * half;
                 const float pt = spt[t];
                 float xv[32], y[32];
-                const uint8_t *xrow = sm + kOffX + t * 128 + 64 * half;
+                const uint8_t *xrow = sm + kOffX + t * 128;
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4 *>(xrow + 16 * q),
-                                                 xv + 8 * q);
+                    Vec16<__nv_bfloat16>::unpack(
+                        *reinterpret_cast<const uint4 *>(xrow + (((4 * half + q) ^ (t & 7)) << 4)),
+                        xv + 8 * q);
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
                     y[j] = fmaf(pt, d1[j], d3[j]) + Dh * xv[j];
