@@ -51,6 +51,42 @@ int launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                : SSU_ERR_CUDA;
 }
 
+// The same, as a programmatic dependent launch: the kernel may start while the previous
+// kernel on the stream still runs (once that kernel's CTAs have all signalled
+// griddepcontrol.launch_dependents, or exited), and must execute griddepcontrol.wait
+// before it touches anything the previous kernel writes or still reads.
+template <typename... KArgs, typename... Args>
+int launch_kernel_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t stream, Args &&...args)
+{
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess
+               ? SSU_OK
+               : SSU_ERR_CUDA;
+}
+
+// griddepcontrol: let the dependent kernel launch (primary side), and wait until every
+// prerequisite kernel has completed and its memory is visible (dependent side; returns at
+// once for a kernel launched without a programmatic dependency).
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // What a launch needs to know about the device, found once per process, kernel and
 // device under std::call_once (so concurrent first calls from several host threads are
 // safe): the SM count, the kernel's dynamic shared-memory limit raised to `smem` bytes,

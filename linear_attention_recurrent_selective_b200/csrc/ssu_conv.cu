@@ -87,6 +87,7 @@ ssu_conv_decode_kernel(const __grid_constant__ ConvArgs ca, const int cph, const
     float *xs = w.f0;                           // unit x (conv outputs), [CR]
     float *ys = w.f1;                           // unit row sums, [CR]
     init_ring(w, lane);
+    grid_launch_dependents();                   // the B/C window shift may start loading
 
     const int H = a.H, Dm = a.Dm, hpg = H / a.G;
     const int64_t cd = (int64_t)H * Dm + 2 * (int64_t)a.G * N;   // conv channels
@@ -242,9 +243,11 @@ ssu_conv_decode_kernel(const __grid_constant__ ConvArgs ca, const int cph, const
     }
 }
 
-// Shift the conv windows of the B and C channels of every live row by one raw input (runs
-// after the fused decode has read the old windows; the x channels were shifted there by
-// their owning units).
+// Shift the conv windows of the B and C channels of every live row by one raw input (the
+// x channels were shifted by their owning units in the fused decode). Launched as a
+// programmatic dependent of the fused decode, which never writes these taps: the old taps
+// and the new input are loaded while the decode runs, and the stores wait until it has
+// completed, so that no unit can still be reading a tap.
 __global__ void __launch_bounds__(256)
 conv_shift_kernel(const __grid_constant__ ConvArgs ca, const int64_t cd, const int64_t ch0)
 {
@@ -264,6 +267,7 @@ conv_shift_kernel(const __grid_constant__ ConvArgs ca, const int64_t cd, const i
     for (int k = 0; k < kMaxConvWidth - 1; ++k)
         tap[k] = k + 1 < W ? ld_bits(ca.cstate, dty, t0 + k * ca.ck) : 0u;
     const uint32_t xin = ld_bits(ca.xbc, dty, b * cd + ch);
+    grid_dependency_wait();
 #pragma unroll
     for (int k = 0; k < kMaxConvWidth - 1; ++k) {
         if (k + 1 < W) {
@@ -296,7 +300,7 @@ int launch_n(const ConvArgs &ca, cudaStream_t stream)
         const int64_t ch0 = (int64_t)a.H * a.Dm;
         const int64_t cd = ch0 + 2 * (int64_t)a.G * N;
         const dim3 blocks((unsigned)((cd - ch0 + 255) / 256), (unsigned)a.active);
-        rc = launch_kernel(conv_shift_kernel, blocks, 256, 0, stream, ca, cd, ch0);
+        rc = launch_kernel_dependent(conv_shift_kernel, blocks, 256, 0, stream, ca, cd, ch0);
     }
     return rc;
 }
