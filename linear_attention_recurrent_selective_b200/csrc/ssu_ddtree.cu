@@ -132,26 +132,6 @@ __device__ __forceinline__ Item item_at(const TreeArgs &ta, int64_t it, int dtil
     return u;
 }
 
-// The item after u in row-major order; the slot index is loaded again only when the row
-// changes.
-__device__ __forceinline__ Item item_after(const TreeArgs &ta, const Item &u, int dtiles)
-{
-    const DecodeArgs &a = ta.d;
-    Item v = u;
-    if (++v.dtile == dtiles) {
-        v.dtile = 0;
-        if (++v.h == a.H) {
-            v.h = 0;
-            ++v.b;
-            v.slot = a.idx ? a.idx[v.b] : v.b;
-        }
-        v.g = v.h / (a.H / a.G);
-    }
-    v.row0 = v.dtile * kTile;
-    v.rows = min(kTile, a.Dm - v.row0);
-    return v;
-}
-
 // The pool slot of row b (-1 past the active rows).
 __device__ __forceinline__ int row_slot(const TreeArgs &ta, int b)
 {
@@ -159,9 +139,9 @@ __device__ __forceinline__ int row_slot(const TreeArgs &ta, int b)
     return b < a.active ? (a.idx ? a.idx[b] : b) : -1;
 }
 
-// item_after with the slot of the next row prefetched in nslot: at a row change the row
-// takes it, and the slot of the row after is loaded, a whole row ahead of its use (a load
-// consumed at once would hold up every item by its latency).
+// The item after u in row-major order, with the slot of the next row prefetched in nslot:
+// at a row change the row takes it, and the slot of the row after is loaded, a whole row
+// ahead of its use.
 __device__ __forceinline__ Item item_after_pf(const TreeArgs &ta, const Item &u, int dtiles,
                                               int &nslot)
 {
