@@ -766,10 +766,10 @@ ssu_ddtree_kernel(const __grid_constant__ TreeArgs ta, const int dtiles, const i
 // For item (b, h, dim tile) they form one matrix product: D[i][d] = sum_n C_i[n] s0[d][n]
 // for the 128 node slots i (slots T .. 127 hold zero C rows) and the tile's 64 dim rows d.
 // C is bf16, so it enters the MMA exactly; the committed state is split into bf16
-// pieces s0 = p1 + p2 + p3 (p1 = bf16(s0), p2 = bf16(s0 - p1), p3 = bf16(s0 - p1 - p2);
-// each difference is exact in fp32, and the three pieces carry 24 significant bits, the
-// fp32 significand), and every product of two bf16 values is exact in the fp32
-// accumulator. The pieces are stacked as the rows of one B operand (64 rows each), so a
+// pieces s0 = p1 + p2 + p3 by truncation (p1 = s0 with its low 16 bits cleared, p2 the
+// same of s0 - p1, p3 = s0 - p1 - p2: each difference is exact in fp32, and p3 keeps at
+// most the 8 significant bits a bf16 holds, so the pieces sum to s0 exactly), and every
+// product of two bf16 values is exact in the fp32 accumulator. The pieces are stacked as the rows of one B operand (64 rows each), so a
 // single chain of dstate / 16 MMAs of N = 64 x pieces reads C once and leaves C p1^T,
 // C p2^T and C p3^T side by side in tensor memory (128 lanes = slots, 64 fp32 columns
 // per piece), summed smallest first in the epilogue. An fp16 state needs two pieces
@@ -1009,11 +1009,14 @@ __device__ void split_state(const TcLayout &lay, uint8_t *sm, int rows)
             uint32_t w[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * q], f[2 * q + 1]);
-                const float2 back = __bfloat1622float2(h);
-                f[2 * q] -= back.x;            // exact: the piece is within 2^-8 of f
-                f[2 * q + 1] -= back.y;
-                memcpy(&w[q], &h, 4);
+                // the piece is the value with the low 16 bits cleared (bf16 truncation); two
+                // pieces' high halves pack into one word by a byte permute
+                const uint32_t u0 = __float_as_uint(f[2 * q]), u1 = __float_as_uint(f[2 * q + 1]);
+                w[q] = __byte_perm(u0, u1, 0x7632);
+                if (p + 1 < NPC) {             // the rest, exact: it is f's low mantissa bits
+                    f[2 * q] -= __uint_as_float(u0 & 0xFFFF0000u);
+                    f[2 * q + 1] -= __uint_as_float(u1 & 0xFFFF0000u);
+                }
             }
             *reinterpret_cast<uint4 *>(sm + lay.sp + sw128_off(p * kTile + r, c, NPC * kTile * 128)) =
                 make_uint4(w[0], w[1], w[2], w[3]);
