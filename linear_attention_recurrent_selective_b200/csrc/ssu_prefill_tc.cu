@@ -21,8 +21,9 @@
 //     D4[n][d] = sum_m B[m][n] w(last, m) dt_m X[m][d]   A = B^T, B = (w dt X)^T in pieces
 // after which y = e^{Lambda_t} D1 + D3 + D x (gated) and s_end = e^{Lambda_last} s + D4^T.
 // Every fp32 operand (the state, G, w dt X) is split into three bf16 pieces that sum to it
-// to within 2^-24 of each element (p1 = bf16(v), p2 = bf16(v - p1), p3 = bf16(v - p1 - p2),
-// each difference exact in fp32); bf16 inputs enter exactly; products of two bf16 values
+// exactly (p1 = v with its low 16 bits cleared, p2 the same of v - p1, p3 = v - p1 - p2:
+// each difference exact in fp32, p3 within the 8 significant bits of a bf16); bf16 inputs
+// enter exactly; products of two bf16 values
 // are exact in the fp32 accumulator. The results therefore carry fp32 accuracy: the same
 // values as the sequential form up to the order of the fp32 sums. (Two pieces, 2^-17, were
 // measured not to be enough even for the bf16 outputs: the error is relative to the terms
@@ -117,7 +118,9 @@ __device__ __forceinline__ void transpose8(const uint4 (&in)[8], uint4 (&out)[8]
     }
 }
 
-// NP bf16 pieces of eight fp32 values, packed 16 bytes each.
+// NP bf16 pieces of eight fp32 values, packed 16 bytes each. Each piece is the rest so
+// far with its low 16 bits cleared (bf16 truncation), and the rest after it is exact (the
+// cleared bits); three pieces hold an fp32 value exactly.
 template <int NP>
 __device__ __forceinline__ void split8(const float (&v)[8], uint4 (&p)[NP])
 {
@@ -130,11 +133,12 @@ __device__ __forceinline__ void split8(const float (&v)[8], uint4 (&p)[NP])
         uint32_t w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(r[2 * q], r[2 * q + 1]);
-            const float2 back = __bfloat1622float2(h);
-            r[2 * q] -= back.x;                      // exact: the piece is within 2^-8 of r
-            r[2 * q + 1] -= back.y;
-            memcpy(&w[q], &h, 4);
+            const uint32_t u0 = __float_as_uint(r[2 * q]), u1 = __float_as_uint(r[2 * q + 1]);
+            w[q] = __byte_perm(u0, u1, 0x7632);      // the two high halves
+            if (k + 1 < NP) {
+                r[2 * q] -= __uint_as_float(u0 & 0xFFFF0000u);
+                r[2 * q + 1] -= __uint_as_float(u1 & 0xFFFF0000u);
+            }
         }
         p[k] = make_uint4(w[0], w[1], w[2], w[3]);
     }
@@ -154,14 +158,15 @@ template <typename S> struct StateCode { static constexpr int v = SSU_F32; };
 template <> struct StateCode<__half> { static constexpr int v = SSU_F16; };
 template <> struct StateCode<__nv_bfloat16> { static constexpr int v = SSU_BF16; };
 
-// NP bf16 pieces of one fp32 value.
+// NP bf16 pieces of one fp32 value (truncation, as split8).
 template <int NP>
 __device__ __forceinline__ void split1(float v, __nv_bfloat16 (&p)[NP])
 {
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
-        p[k] = __float2bfloat16_rn(v);
-        v -= __bfloat162float(p[k]);
+        const uint32_t u = __float_as_uint(v);
+        p[k] = __ushort_as_bfloat16(static_cast<unsigned short>(u >> 16));
+        v -= __uint_as_float(u & 0xFFFF0000u);
     }
 }
 
