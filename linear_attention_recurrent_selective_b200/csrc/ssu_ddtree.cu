@@ -897,6 +897,8 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
         cnt[tid] = ok ? depth + 1 : 0;
         if (!ok && reporter && a.err)
             atomicOr(a.err, SSU_FLAG_TREE);
+    } else if (tid < ((T + 3) & ~3)) {
+        cnt[tid] = 0x7fffffff;               // padding to a whole int4, ranked after all
     }
     __syncthreads();
     if (warp == 0) {                          // exclusive prefix sum; off[T] = all pairs
@@ -920,9 +922,10 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
     } else if (tid >= 128 && tid < 128 + T) { // rank by path length, ties by node index
         const int i = tid - 128, ci = cnt[i];
         int r = 0;
-        for (int k = 0; k < T; ++k) {
-            const int ck = cnt[k];
-            r += ck < ci || (ck == ci && k < i);
+        for (int k = 0; k < T; k += 4) {
+            const int4 c4 = *reinterpret_cast<const int4 *>(cnt + k);
+            r += (c4.x < ci || (c4.x == ci && k < i)) + (c4.y < ci || (c4.y == ci && k + 1 < i)) +
+                 (c4.z < ci || (c4.z == ci && k + 2 < i)) + (c4.w < ci || (c4.w == ci && k + 3 < i));
         }
         ns[i] = static_cast<uint8_t>(r);
         sn[r] = static_cast<uint8_t>(i);
@@ -950,19 +953,20 @@ __device__ void stage_row_tc(const TreeArgs &ta, const TcLayout &lay, uint8_t *s
     for (int p = tid; p < total; p += kTcThreads) {
         const int i = pi[p], j = pj[p], si = ns[i];
         const uint8_t *brow = bst + j * (N * 2);
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < CPR; ++c) {
             const uint4 cv = *reinterpret_cast<const uint4 *>(sm + lay.ca + sw128_off(si, c, 128 * 128));
             const uint4 bv = *reinterpret_cast<const uint4 *>(brow + ((c ^ (j & 7)) << 4));
-            float fc[8], fb[8];
-            Vec16<__nv_bfloat16>::unpack(cv, fc);
-            Vec16<__nv_bfloat16>::unpack(bv, fb);
+            const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                s[e & 3] = fmaf(fc[e], fb[e], s[e & 3]);
+            for (int q = 0; q < 4; ++q)       // a bf16 pair widens to floats by shift and mask
+                s2[q & 1] = __ffma2_rn(
+                    make_float2(__uint_as_float(cw[q] << 16), __uint_as_float(cw[q] & 0xFFFF0000u)),
+                    make_float2(__uint_as_float(bw[q] << 16), __uint_as_float(bw[q] & 0xFFFF0000u)),
+                    s2[q & 1]);
         }
-        cb[p] = (s[0] + s[1]) + (s[2] + s[3]);
+        cb[p] = (s2[0].x + s2[0].y) + (s2[1].x + s2[1].y);
     }
     if (hh0 <= hh1) {                         // stash B: this CTA's heads' shares
         const int hpg = a.H / G, total = T * N;
@@ -1492,17 +1496,26 @@ ssu_ddtree_tc_kernel(const __grid_constant__ TreeArgs ta, const __grid_constant_
             float dp[16];
             tmem_ld16(taddr + (uint32_t)(p * kTile), dp);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                dv[e] += dp[e];
+            for (int e = 0; e < 16; e += 2) {
+                const float2 t2 = __fadd2_rn(make_float2(dv[e], dv[e + 1]), make_float2(dp[e], dp[e + 1]));
+                dv[e] = t2.x;
+                dv[e + 1] = t2.y;
+            }
         }
         const bool mine = ni < T && d0 < u.rows;
         float y[16];
         if (mine) {
-            float xv[16];
-            x_seg16<X>(xs, node, d0, tp, xv);
+            float2 xv[8];
+            x_pairs16<X>(xs, node, d0, tp, xv);
+            const bool live = cnt[node] > 0;
+            const float2 w2 = make_float2(wn, wn), D2 = make_float2(hv.D, hv.D);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                y[e] = cnt[node] > 0 ? fmaf(wn, dv[e], pv[e]) + hv.D * xv[e] : 0.f;
+            for (int e = 0; e < 8; ++e) {
+                const float2 y2 = __ffma2_rn(D2, xv[e], __ffma2_rn(w2, make_float2(dv[2 * e], dv[2 * e + 1]),
+                                                                  make_float2(pv[2 * e], pv[2 * e + 1])));
+                y[2 * e] = live ? y2.x : 0.f;
+                y[2 * e + 1] = live ? y2.y : 0.f;
+            }
         }
         tc_fence_before();
         if (otma) {
