@@ -54,7 +54,11 @@ constexpr int kDT = 64;                 // dim rows per CTA: N of D1, D3, D4
 constexpr int kNS = 128;                // dstate
 constexpr int kThr = 256;               // 8 warps; warp w reads TMEM lanes 32 (w % 4) ..
 constexpr uint32_t kCols = 512;         // tensor-memory columns, the whole SM's
-constexpr uint32_t kD1 = 0, kD2 = 64, kD3 = 192, kD4 = 256;   // accumulator columns
+// Accumulator columns. D1 and D4 take the three pieces of their B operand stacked as one
+// operand of 192 rows (64 per piece), so each is one MMA chain of N = 192 whose three
+// 64-column blocks are summed in the epilogue; D4 reuses D2's columns, which phase 2 has
+// read before phase 3 issues it.
+constexpr uint32_t kD1 = 0, kD3 = 192, kD2 = 256, kD4 = 256;
 
 // bf16 pieces per operand (G, the state's copy in D1, (w dt X)^T)
 constexpr int kPG = 3, kPS = 3, kPW = 3;
@@ -302,10 +306,11 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
             const int d = 32 * half + j;
             __nv_bfloat16 p[kPS];
             split1<kPS>(st[j], p);
-            uint8_t *dst = sm + kOffS + sw128_off(d, r >> 3, kBlkN) + (r & 7) * 2;
+            uint8_t *dst = sm + kOffS + (r & 7) * 2;
 #pragma unroll
             for (int k = 0; k < kPS; ++k)
-                *reinterpret_cast<__nv_bfloat16 *>(dst + k * kPieceN) = p[k];
+                *reinterpret_cast<__nv_bfloat16 *>(dst + sw128_off(k * kDT + d, r >> 3, kPS * kBlkN)) =
+                    p[k];
         }
     };
     put_state();
@@ -313,6 +318,7 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
     load_x(0);
 
     constexpr uint32_t kI64 = idesc_bf16_f32(kL, 64);
+    constexpr uint32_t kI192 = idesc_bf16_f32(kL, 3 * kDT);
     constexpr uint32_t kI128 = idesc_bf16_f32(kL, 128);
     const uint32_t base = smem_u32(sm);
     uint32_t ph0 = 0, ph1 = 0;
@@ -369,16 +375,14 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
             tc_fence_after();
             uint32_t acc = 0;
 #pragma unroll
-            for (int p = kPS - 1; p >= 0; --p)               // smallest piece first
+            for (int kb = 0; kb < 2; ++kb)                   // the pieces stacked
 #pragma unroll
-                for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        tc_mma_bf16(tmem + kD1, desc_k_sw128(base + kOffC + kb * kBlkM + kk * 32),
-                                    desc_k_sw128(base + kOffS + p * kPieceN + kb * kBlkN + kk * 32),
-                                    kI64, acc);
-                        acc = 1;
-                    }
+                for (int kk = 0; kk < 4; ++kk) {
+                    tc_mma_bf16(tmem + kD1, desc_k_sw128(base + kOffC + kb * kBlkM + kk * 32),
+                                desc_k_sw128(base + kOffS + kb * (kPS * kBlkN) + kk * 32), kI192,
+                                acc);
+                    acc = 1;
+                }
             acc = 0;
 #pragma unroll
             for (int kb = 0; kb < 2; ++kb)
@@ -508,7 +512,7 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
             split8<kPW>(v, p);
 #pragma unroll
             for (int q = 0; q < kPW; ++q)
-                *reinterpret_cast<uint4 *>(sm + kOffW + q * kPieceN + o) = p[q];
+                *reinterpret_cast<uint4 *>(sm + kOffW + sw128_off(q * kDT + d, ch, kPW * kBlkN)) = p[q];
         }
         fence_async_smem();
         tc_fence_before();
@@ -531,16 +535,14 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
                     }
             acc = 0;
 #pragma unroll
-            for (int p = kPW - 1; p >= 0; --p)
+            for (int kb = 0; kb < 2; ++kb)                   // the pieces stacked
 #pragma unroll
-                for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        tc_mma_bf16(tmem + kD4, desc_k_sw128(base + kOffBT + kb * kBlkM + kk * 32),
-                                    desc_k_sw128(base + kOffW + p * kPieceN + kb * kBlkN + kk * 32),
-                                    kI64, acc);
-                        acc = 1;
-                    }
+                for (int kk = 0; kk < 4; ++kk) {
+                    tc_mma_bf16(tmem + kD4, desc_k_sw128(base + kOffBT + kb * kBlkM + kk * 32),
+                                desc_k_sw128(base + kOffW + kb * (kPW * kBlkN) + kk * 32), kI192,
+                                acc);
+                    acc = 1;
+                }
             tc_commit(bar + 1);
         }
         // this thread's z values (token r, dims 32 half .. + 31) while the products run
@@ -573,7 +575,15 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
         // ---- phase 4: outputs of token t = r, dims 32 half .. + 31
         {
             float d1[32], d3[32];
-            tmem_ld32(tl + kD1 + 32 * half, d1);
+            tmem_ld32(tl + kD1 + 2 * kDT + 32 * half, d1);          // pieces, smallest first
+#pragma unroll
+            for (int p = kPS - 2; p >= 0; --p) {
+                float dp[32];
+                tmem_ld32(tl + kD1 + p * kDT + 32 * half, dp);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    d1[j] += dp[j];
+            }
             tmem_ld32(tl + kD3 + 32 * half, d3);
             const int t = r;
             if (t < nt) {
@@ -618,7 +628,15 @@ ssu_prefill_tc_kernel(const __grid_constant__ PrefillArgs pa, const int dtiles)
         // ---- the state: s[d][n] = e^{Lambda_last} s[d][n] + D4[n][d], then its pieces
         {
             float d4[32];
-            tmem_ld32(tl + kD4 + 32 * half, d4);
+            tmem_ld32(tl + kD4 + 2 * kDT + 32 * half, d4);          // pieces, smallest first
+#pragma unroll
+            for (int p = kPW - 2; p >= 0; --p) {
+                float dp[32];
+                tmem_ld32(tl + kD4 + p * kDT + 32 * half, dp);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    d4[j] += dp[j];
+            }
             const float pl = spt[nt - 1];
 #pragma unroll
             for (int j = 0; j < 32; ++j)
