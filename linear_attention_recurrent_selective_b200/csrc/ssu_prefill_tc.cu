@@ -23,8 +23,10 @@
 // Every fp32 operand (the state, G, w dt X) is split into three bf16 pieces that sum to it
 // exactly (p1 = v with its low 16 bits cleared, p2 the same of v - p1, p3 = v - p1 - p2:
 // each difference exact in fp32, p3 within the 8 significant bits of a bf16); bf16 inputs
-// enter exactly; products of two bf16 values
-// are exact in the fp32 accumulator. The results therefore carry fp32 accuracy: the same
+// enter exactly; products of two bf16 values are exact in the fp32 accumulator. Where the
+// pieces are the B operand (D1, D4) they are stacked as one operand of 192 rows, so one
+// chain of N = 192 gives the three partial products side by side; G's pieces, the A
+// operand of D3, take a chain each. The results therefore carry fp32 accuracy: the same
 // values as the sequential form up to the order of the fp32 sums. (Two pieces, 2^-17, were
 // measured not to be enough even for the bf16 outputs: the error is relative to the terms
 // summed, and where terms of order 10 cancel to an output near zero it exceeds the 1e-5
