@@ -53,6 +53,40 @@ struct ConvRows : UnitsInOrder {
 __device__ __forceinline__ float conv_out(const ConvArgs &c, int dtype, int64_t xrow,
                                           int64_t tap0, int64_t ch, bool shift = false)
 {
+    if (c.width <= 4) {
+        // windows of up to 4 (the common case): every input loaded at once into registers
+        // (one round trip instead of one per dependent step), the taps reused by the shift
+        const int W = c.width;
+        const int64_t w0 = ch * W, t0 = tap0 + ch * c.cc;
+        uint32_t tap[3], wt[4];
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+            tap[k] = k + 1 < W ? ld_bits(c.cstate, dtype, t0 + k * c.ck) : 0u;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            wt[k] = k < W ? ld_bits(c.w, dtype, w0 + k) : 0u;
+        const uint32_t xin = ld_bits(c.xbc, dtype, xrow + ch);
+        float acc = c.bias ? ld_f32(c.bias, dtype, ch) : 0.f;
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+            if (k + 1 < W)
+                acc = fmaf(bits_f32(wt[k], dtype), bits_f32(tap[k], dtype), acc);
+        const uint32_t wl = W == 4 ? wt[3] : W == 3 ? wt[2] : W == 2 ? wt[1] : wt[0];
+        acc = fmaf(bits_f32(wl, dtype), bits_f32(xin, dtype), acc);
+        if (shift) {
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+                if (k + 1 < W) {
+                    const uint32_t v = k + 2 < W ? tap[k + 1 < 3 ? k + 1 : 2] : xin;
+                    if (dtype == SSU_F32)
+                        static_cast<uint32_t *>(c.cstate)[t0 + k * c.ck] = v;
+                    else
+                        static_cast<uint16_t *>(c.cstate)[t0 + k * c.ck] = static_cast<uint16_t>(v);
+                }
+            }
+        }
+        return c.silu ? silu_f(acc) : acc;
+    }
     float acc = c.bias ? ld_f32(c.bias, dtype, ch) : 0.f;
     const int64_t w0 = ch * c.width;
     const int64_t t0 = tap0 + ch * c.cc;
