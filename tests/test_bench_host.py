@@ -88,3 +88,20 @@ def test_reference_arm_prints_one_line():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["unit"] == bench.UNIT and rec["value"] > 0
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_traffic_record_is_tied_to_the_decode_sources(tmp_path, monkeypatch):
+    """roofline.traffic comes from the ncu record only when it was taken on the decode
+    sources built now and at the workload's batch; otherwise it is null."""
+    rec = {"batch": 256, "bytes_per_launch": 1234, "source_sha256": bench.decode_source_hash()}
+    path = tmp_path / "traffic.json"
+    path.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(path))
+    assert bench.recorded_traffic(256) == 1234
+    assert bench.recorded_traffic(128) is None                # another batch
+    path.write_text(json.dumps(dict(rec, source_sha256="0" * 64)))
+    assert bench.recorded_traffic(256) is None                # other sources
+    path.write_text("not json")
+    assert bench.recorded_traffic(256) is None
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
+    assert bench.recorded_traffic(256) is None
